@@ -1,0 +1,444 @@
+"""Benchmark: BitLinear decode over the 125M-shape decode workload.
+
+One step = the decode hot path for every projection of all 12 layers
+(q,o 768x768; k,v 256x768; gate,up 2048x768; down 768x2048 -- 84 problems)
+at M = 1, 4 and 8 tokens: per M, one grouped activation-quant launch and one
+grouped ternary GEMV launch.  The ternary weights (29/42/29 split) are
+packed once at load time.  Weight bytes per step would fit in L2, so the
+packed weights are replicated and every step reads a different replica
+(the replicas total more than 3x the L2 size).
+
+Metric: decode GB/s = (packed weight bytes + x_q bytes) per step / time,
+whole job, N GPUs = N independent replicas of the workload (weak scaling).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from ternary_quantized_linear_bitlinear_b200 import workloads  # noqa: E402
+
+METRIC = "BitLinear decode weight GB/s & prefill int8 TOPS, as % of roofline"
+UNIT = "GB/s"
+MS = (1, 4, 8)
+SPAD = {M: (M + 3) // 4 * 4 for M in MS}
+WORKLOAD = "decode125m: 12 layers x {q,o 768x768; k,v 256x768; gate,up 2048x768; down 768x2048}, M in {1,4,8}"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -- workload ----------------------------------------------------------------
+
+def step_bytes():
+    """Algorithmic bytes of one step: packed weights + x_q, per M."""
+    shapes = workloads.decode125m_layer_shapes()
+    L = workloads.DECODE125M["layers"]
+    wbytes = L * sum(N * K // 4 for _, N, K, _ in shapes)
+    xbytes = {M: L * sum(M * K for _, N, K, _ in shapes) for M in MS}
+    return wbytes, xbytes
+
+
+class Clocks:
+    """nvidia-smi sampling during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = str(index)
+        try:
+            uuid = torch.cuda.get_device_properties(index).uuid
+            self.index = f"GPU-{uuid}"
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            if vis:
+                self.index = vis.split(",")[index]
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+
+    def __enter__(self):
+        os.makedirs(os.path.dirname(self.path), exist_ok=True)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", self.index, f"--query-gpu={q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        rows = []
+        for ln in open(self.path):
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def native(args, rank, world, local):
+    from ternary_quantized_linear_bitlinear_b200 import api
+
+    dev = torch.device("cuda", torch.cuda.current_device())
+    props = torch.cuda.get_device_properties(dev)
+    l2 = getattr(props, "L2_cache_size", 126 * 2 ** 20)
+    wbytes, xbytes = step_bytes()
+    R = max(2, (3 * l2) // wbytes + 1)  # weight replicas totalling > 3x L2
+
+    # ---- load: pack the ternary weights once per replica (not timed) -------
+    items = workloads.decode125m(seed=1 + rank, M=max(MS))
+    shapes = [(W.shape[0], W.shape[1]) for _, W, _ in items]
+    packed0, gammas = [], []
+    for _, W, _ in items:
+        p, g = api.bl_quant_weights(W.to(dev))
+        packed0.append(p)
+        gammas.append(g)
+    flat0 = torch.cat([p.view(-1) for p in packed0])
+    offs = []
+    o = 0
+    for p in packed0:
+        offs.append(o)
+        o += p.numel()
+    replicas = [flat0] + [flat0.clone() for _ in range(R - 1)]
+
+    # activations: one contiguous bf16 buffer per M (inputs of all 84 problems)
+    xin, xq, sc, Y = {}, {}, {}, {}
+    xin_host, y_host = {}, {}
+    for M in MS:
+        Xs = [X[:M].contiguous() for _, _, X in items]
+        xin_host[M] = torch.cat([x.view(-1) for x in Xs]).pin_memory()
+        xin[M] = xin_host[M].to(dev)
+        xq[M] = torch.empty(xin[M].numel(), dtype=torch.int8, device=dev)
+        sc[M] = torch.empty(len(items) * SPAD[M], dtype=torch.float32, device=dev)  # 16-byte aligned per problem
+        ytot = sum(M * N for N, _ in shapes)
+        Y[M] = torch.empty(ytot + 4 * len(items), dtype=torch.float32, device=dev)
+        y_host[M] = torch.empty_like(Y[M], device="cpu").pin_memory()
+
+    def views(M):
+        """Per-problem device views into the contiguous buffers (16-byte aligned)."""
+        act, fwd = [], []
+        xo = yo = 0
+        for i, (N, K) in enumerate(shapes):
+            xv = xin[M][xo:xo + M * K].view(M, K)
+            qv = xq[M][xo:xo + M * K].view(M, K)
+            sv = sc[M][i * SPAD[M]:i * SPAD[M] + M]
+            yv = Y[M][yo:yo + M * N].view(M, N)
+            act.append((xv, None, qv, sv))
+            fwd.append((qv, sv, yv, N, K))
+            xo += M * K
+            yo += (M * N + 3) // 4 * 4
+        return act, fwd
+
+    def act_problems(act):
+        arr = (api.ActProblem * len(act))()
+        for i, (X, g, q, s) in enumerate(act):
+            arr[i] = api.ActProblem(X.data_ptr(), None, q.data_ptr(), s.data_ptr(), X.shape[1])
+        return arr
+
+    def fwd_problems(fwd, rep):
+        arr = (api.Problem * len(fwd))()
+        base = replicas[rep].data_ptr()
+        for i, (q, s, y, N, K) in enumerate(fwd):
+            arr[i] = api.Problem(base + offs[i], gammas[i].data_ptr(), q.data_ptr(), s.data_ptr(), y.data_ptr(),
+                                 None, N, K)
+        return arr
+
+    L = api.lib()
+    acts = {M: act_problems(views(M)[0]) for M in MS}
+    fwds = {(M, r): fwd_problems(views(M)[1], r) for M in MS for r in range(R)}
+    count = len(items)
+
+    def launch_step(stream_ptr, rep, decode_only=False):
+        for M in MS:
+            if not decode_only:
+                rc = L.bl_quant_act_grouped(acts[M], count, api.BL_BF16, M, 1e-6, stream_ptr)
+                if rc:
+                    raise api.BitLinearError(rc, "bl_quant_act_grouped")
+            rc = L.bl_forward_grouped(fwds[(M, rep)], count, M, stream_ptr)
+            if rc:
+                raise api.BitLinearError(rc, "bl_forward_grouped")
+
+    # ---- capture one cycle (R steps, one per replica) as a CUDA graph ------
+    stream = torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        for r in range(R):  # eager warm-up: also runs the one-time device set-up
+            launch_step(sp, r)
+    torch.cuda.synchronize()
+
+    def capture(decode_only):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for r in range(R):
+                launch_step(stream.cuda_stream, r, decode_only)
+        return g
+
+    g_step = capture(False)
+    g_dec = capture(True)
+    torch.cuda.synchronize()
+
+    K, Wm = args.steps, max(3, args.warmup)
+    cycles = max(1, (K + R - 1) // R)
+    steps_timed = cycles * R
+    for _ in range(max(1, (Wm + R - 1) // R)):
+        g_step.replay()
+    torch.cuda.synchronize()
+
+    # ---- timed region: whole steps ----------------------------------------
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    with Clocks(local) as clk:
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(cycles):
+                g_step.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
+    ms_per_step = ms_total / steps_timed
+    bytes_step = sum(wbytes + xbytes[M] for M in MS)
+    value = world * bytes_step * steps_timed / (ms_total * 1e-3) / 1e9
+
+    # ---- dominant kernel alone: the grouped GEMV launches ------------------
+    with torch.cuda.stream(stream):
+        d0 = torch.cuda.Event(enable_timing=True)
+        d1 = torch.cuda.Event(enable_timing=True)
+        g_dec.replay()
+        d0.record(stream)
+        dec_cycles = max(1, cycles // 2)
+        for _ in range(dec_cycles):
+            g_dec.replay()
+        d1.record(stream)
+    torch.cuda.synchronize()
+    dec_launches = dec_cycles * R * len(MS)
+    dec_us = d0.elapsed_time(d1) * 1e3 / dec_launches
+    dec_bytes = sum(wbytes + xbytes[M] for M in MS) / len(MS)  # per launch, averaged over M
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    peak = float(peaks.get("hbm_gbs", 6650.0))
+    achieved = dec_bytes / (dec_us * 1e-6) / 1e9
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    if os.path.exists(tpath):
+        try:
+            traffic = json.load(open(tpath)).get("dram_bytes_per_launch")
+        except (OSError, ValueError):
+            traffic = None
+    roofline = {"bound": "hbm", "kernel": "k_decode (grouped GEMV, 84 problems)", "achieved": round(achieved, 1),
+                "peak": peak, "peak_source": "measured" if "hbm_gbs" in peaks else "fallback",
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                "avg_launch_us": round(dec_us, 3)}
+    # ---- end to end through the C ABI with host buffers --------------------
+    e2e = None
+    if not args.no_e2e:
+        act_v = {M: views(M) for M in MS}
+        h2d = sum(xin_host[M].numel() * 2 for M in MS)
+        d2h = sum(y_host[M].numel() * 4 for M in MS)
+        n_e2e = max(3, min(steps_timed, 300))
+        with torch.cuda.stream(stream):
+            for it in range(n_e2e + 3):
+                if it == 3:
+                    torch.cuda.synchronize()
+                    t0 = time.perf_counter()
+                for M in MS:
+                    xin[M].copy_(xin_host[M], non_blocking=True)
+                launch_step(sp, it % R)
+                for M in MS:
+                    y_host[M].copy_(Y[M], non_blocking=True)
+            stream.synchronize()
+        e2e_s = max_over_ranks(time.perf_counter() - t0, world)
+        e2e = {"value": round(world * bytes_step * n_e2e / e2e_s / 1e9, 2), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+        del act_v
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": steps_timed,
+        "warmup": Wm, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens_per_step": sum(MS), "projections": count,
+                   "weight_bytes_per_m": wbytes, "weight_replicas": R,
+                   "l2": f"{R} rotating packed-weight replicas ({R * wbytes / 2**20:.0f} MiB > 3x L2)",
+                   "parallelism": f"replicas x{world}", "launch": "CUDA graph of whole steps"},
+        "roofline": roofline, "e2e": e2e,
+        "gpu_launches": steps_timed * 2 * len(MS),
+    }
+    out["clocks"] = clk.summary()
+    return out
+
+
+def cpu_oracle_step(items_q, wbytes, xbytes):
+    """One step of the decode workload on the CPU oracle; returns seconds."""
+    import oracle
+    t0 = time.perf_counter()
+    for M in MS:
+        for (wq, g, X) in items_q:
+            xq, s = oracle.quant_act(X[:M])
+            acc = oracle.contract(xq, wq)
+            oracle.rescale(acc, g, s[:, None])
+    return time.perf_counter() - t0
+
+
+def oracle_items(seed=1):
+    import numpy as np
+    import oracle
+    out = []
+    for _, W, X in workloads.decode125m(seed=seed, M=max(MS)):
+        packed, g, wq = oracle.quant_weights(W.numpy())
+        out.append((wq, g, X.float().numpy().astype(np.float32)))
+    return out
+
+
+def cpu_baseline():
+    import oracle
+    wbytes, xbytes = step_bytes()
+    items = oracle_items()
+    secs = cpu_oracle_step(items, wbytes, xbytes)
+    bytes_step = sum(wbytes + xbytes[M] for M in MS)
+    return {"value": round(bytes_step / secs / 1e9, 4), "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "one whole step (84 projections at M = 1, 4, 8: act quant, int64 contraction, rescale); "
+                      "OpenMP over token rows"}
+
+
+def reference(args, rank, world):
+    """The CPU oracle as the reference arm, on the same metric and workload;
+    each step is one projection (cycling through the 84 and M = 1, 4, 8),
+    rows of W subsampled so the run stays within a few minutes."""
+    if rank != 0:
+        return None
+    import numpy as np
+    import oracle
+    items = oracle_items()
+    jobs = [(M, i) for M in MS for i in range(len(items))]
+    total_steps = args.steps + max(3, args.warmup)
+    budget_s = 90.0 / max(1, total_steps)
+    # calibrate the oracle's rows-per-second on one projection (not timed)
+    wq, g, X = items[4]
+    t0 = time.perf_counter()
+    xq, s = oracle.quant_act(X[:8])
+    oracle.rescale(oracle.contract(xq, wq[:256]), g, s[:, None])
+    per_row = (time.perf_counter() - t0) / 256
+    rows = int(max(16, min(4096, budget_s / max(per_row, 1e-9))))
+    done_bytes = 0
+    t_start = None
+    for it in range(total_steps):
+        if it == max(3, args.warmup):
+            t_start = time.perf_counter()
+            done_bytes = 0
+        M, i = jobs[it % len(jobs)]
+        wq, g, X = items[i]
+        n = min(rows, wq.shape[0])
+        xq, s = oracle.quant_act(X[:M])
+        oracle.rescale(oracle.contract(xq, wq[:n]), g, s[:, None])
+        done_bytes += n * wq.shape[1] // 4 + M * wq.shape[1]
+    secs = time.perf_counter() - t_start
+    value = done_bytes / secs / 1e9
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(secs * 1e3 / args.steps, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64",
+            "data": "synthetic", "config": {"workload": WORKLOAD},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"per step one projection (cycling 84 x M in 1,4,8), first {rows} rows of W"},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            out = reference(args, rank, world)
+        else:
+            out = native(args, rank, world, local)
+            if rank == 0 and world == 1 and not args.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline()
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,205 @@
+/*
+ * bitlinear.h -- C ABI of libbitlinear.so: the BitNet b1.58 BitLinear forward
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The forward has four steps; each entry point below names the passage that
+ * defines what it computes:
+ *   1. absmean weight quantization + 2-bit packing      bl_quant_weights
+ *   2. per-token absmax INT8 activation quantization    bl_quant_act
+ *      (optionally after a SubLN RMSNorm)
+ *   3. exact ternary x INT8 contraction (int32)          bl_forward
+ *   4. rescale Y = acc * gamma / s                       bl_forward
+ *   all four in one call                                 bl_linear
+ *
+ * Conventions shared by every entry point
+ *   - Shapes: W is [N, K] row-major (out_features x in_features, as a torch
+ *     Linear weight), X is [M, K] row-major, Y is [M, N] row-major float32:
+ *     Y = X * W^T.
+ *   - Every data pointer is a DEVICE pointer on the current CUDA device,
+ *     allocated and owned by the caller; the library never allocates, frees
+ *     or keeps a pointer after the call returns.  Pointers must be 16-byte
+ *     aligned; rows are contiguous (no strides).
+ *   - Work is enqueued asynchronously on `stream` (NULL = legacy default
+ *     stream); a returned BL_OK means "validated and launched".  Outputs are
+ *     ready when the stream has reached that point.
+ *   - No exception crosses the ABI; errors are returned as bl_status.  Bad
+ *     arguments are detected on the host before anything is launched, and
+ *     nothing is written then.  Device-side bounded waits that give up set a
+ *     sticky device error word, read (and cleared) by bl_check_device_error.
+ *   - Inputs must be finite; NaN or Inf input gives unspecified (but memory-
+ *     safe) outputs.
+ *   - Limits: 1 <= M <= 2^31-1, 1 <= N <= 2^31-1, 64 <= K <= 32768 with
+ *     K % 64 == 0; N*K < 2^31 for the weight quantizer.  With |x_q| <= 127
+ *     and K <= 32768, |acc| <= 2^22, so acc converts to float exactly.
+ *
+ * Packed weight format (the pages give no layout; they state ~1.58 bits per
+ * weight, "bitone" README, "How 1.58-bit Works", and a memory table at
+ * ~1.6 bits): 2 bits per weight, N * K / 4 bytes.  Row n occupies K/4
+ * contiguous bytes = K/16 little-endian 32-bit words.  Weight k = 16*w + 4*j
+ * + i (0 <= i, j < 4) has its code in word w at bits [8*i + 2*j,
+ * 8*i + 2*j + 1].  Codes: 00 = 0, 01 = +1, 11 = -1 (2-bit two's complement);
+ * 10 is never written.  So byte i of a word holds the codes of k = i, i+4,
+ * i+8, i+12 of its 16-weight group.
+ */
+#ifndef BITLINEAR_H
+#define BITLINEAR_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t; the header needs no CUDA include. */
+typedef struct CUstream_st *bl_stream_t;
+
+typedef enum {
+    BL_OK = 0,
+    BL_ERR_NULL = 1,      /* a required pointer is NULL */
+    BL_ERR_SHAPE = 2,     /* M, N, K (or a group count) outside the limits above */
+    BL_ERR_ALIGN = 3,     /* a pointer is not 16-byte aligned */
+    BL_ERR_DTYPE = 4,     /* unknown bl_dtype code */
+    BL_ERR_CUDA = 5,      /* a CUDA runtime call or kernel launch failed */
+    BL_ERR_TIMEOUT = 6,   /* a bounded device-side wait gave up (see bl_check_device_error) */
+    BL_ERR_WORKSPACE = 7, /* workspace NULL or smaller than the *_workspace_bytes query */
+    BL_ERR_DEVICE = 8     /* the current device is not a compute capability 10.x GPU */
+} bl_status;
+
+typedef enum {
+    BL_F32 = 0,  /* IEEE float32 */
+    BL_BF16 = 1  /* bfloat16 (upcast to float32 exactly) */
+} bl_dtype;
+
+/* Human-readable name of a status code; never NULL. */
+const char *bl_status_string(bl_status s);
+
+/* Library ABI version (major * 100 + minor). */
+int bl_version(void);
+
+/* Reads and clears the device error word set by bounded device-side waits.
+ * Synchronizes `stream` first.  Returns BL_OK, BL_ERR_TIMEOUT or
+ * BL_ERR_CUDA. */
+bl_status bl_check_device_error(bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Step 1: absmean ternary weight quantization + 2-bit packing.              */
+/*                                                                           */
+/* Defined by: "Distillix" README, "Key Innovations / 1. BitNet b1.58 Core"  */
+/* (W_q = round(clip(W / mean|W|, -1, 1))); "bitone" README, Triton-fused   */
+/* QAT BitLinear "Forward pass" (gamma = mean(|W|) from one reduction over   */
+/* W, then W_q per tile); "SLM750-Edge" model card, section 3.1 "Ternary     */
+/* Weight Quantization" (round_clip: 0 when |W/gamma| <= 0.5).               */
+/*                                                                           */
+/*   gamma = float(double(S) / double(N*K)) + 1e-5f, S = sum |W| exactly     */
+/*           (order-independent; rounded once to double)                     */
+/*   W_q   = clamp(round_half_even(float(W / gamma)), -1, 1)                 */
+/*                                                                           */
+/* W        [N, K] of dtype wdt (BL_F32 or BL_BF16), device                  */
+/* packed   [N, K/4] bytes out, format above, device                         */
+/* gamma    1 float out, device                                              */
+/* workspace device scratch of at least bl_quant_weights_workspace_bytes();  */
+/*          contents on entry are ignored, clobbered on exit                 */
+/* Errors: NULL pointer, misalignment, K % 64, N*K >= 2^31, small workspace. */
+/* ------------------------------------------------------------------------ */
+size_t bl_quant_weights_workspace_bytes(int64_t N, int64_t K);
+bl_status bl_quant_weights(const void *W, bl_dtype wdt, int64_t N, int64_t K,
+                           uint8_t *packed, float *gamma,
+                           void *workspace, size_t workspace_bytes, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Step 2: per-token absmax INT8 activation quantization, optionally fused  */
+/* with a preceding SubLN RMSNorm.                                           */
+/*                                                                           */
+/* Defined by: "BitDistill" article, "Evaluation and results" (activations   */
+/* quantized to INT8); SubLN placement: "BitDistill", "Stage 1 --            */
+/* Architectural refinement with SubLN" (before the attention output and    */
+/* FFN output projections); "SLM750-Edge" section 2.1 (SubLN = pre-RMSNorm + */
+/* activation quantization) and "Key Architectural Features" (RMSNorm eps    */
+/* 1e-6).                                                                    */
+/*                                                                           */
+/*   y   = x                                   if subln_gain == NULL         */
+/*   y_k = float(float(x_k / r) * g_k)         otherwise, with               */
+/*         r = sqrtf(float(double(sum_k x_k^2) / K) + eps), the sum exact    */
+/*   s   = float(127 / max(max_k |y_k|, 1e-5f))                              */
+/*   x_q = clamp(round_half_even(float(y * s)), -128, 127)                   */
+/*                                                                           */
+/* X [M, K] of dtype xdt; subln_gain [K] float or NULL; x_q [M, K] int8 out;  */
+/* s [M] float out.  All device.                                             */
+/* ------------------------------------------------------------------------ */
+bl_status bl_quant_act(const void *X, bl_dtype xdt, int64_t M, int64_t K,
+                       const float *subln_gain, float subln_eps,
+                       int8_t *x_q, float *s, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Steps 3 + 4: exact ternary x INT8 contraction and rescale.                */
+/*                                                                           */
+/* Defined by: "bitone" README, "How 1.58-bit Works" (each weight adds,      */
+/* subtracts or skips an input: no multiplication needed) and "Forward      */
+/* pass" (Y = X @ W_q^T * gamma), with the INT8 scale s of step 2:           */
+/*                                                                           */
+/*   acc[m, n] = sum_k x_q[m, k] * W_q[n, k]          (exact, int32)         */
+/*   Y[m, n]   = float(float(acc) * float(gamma / s[m]))                     */
+/*               (two float roundings: |Y - acc*gamma/s| <= 2^-23 |Y|)       */
+/*                                                                           */
+/* Engine: M <= 16 and M*K <= 96 KiB -> bandwidth-bound decode GEMV;         */
+/* otherwise the tcgen05 prefill GEMM.  Both give identical acc.             */
+/* packed [N, K/4] (format above); gamma [1]; x_q [M, K]; s [M]; Y [M, N]    */
+/* out; acc_out [M, N] int32 out or NULL.  All device.                       */
+/* ------------------------------------------------------------------------ */
+bl_status bl_forward(const uint8_t *packed, const float *gamma, const int8_t *x_q,
+                     const float *s, int64_t M, int64_t N, int64_t K, float *Y,
+                     int32_t *acc_out, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* All four steps in one call: bl_quant_weights, bl_quant_act, bl_forward.   */
+/* workspace >= bl_linear_workspace_bytes(M, N, K) holds packed W, gamma,    */
+/* x_q and s between the steps.                                              */
+/* ------------------------------------------------------------------------ */
+size_t bl_linear_workspace_bytes(int64_t M, int64_t N, int64_t K);
+bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt,
+                    int64_t M, int64_t N, int64_t K,
+                    const float *subln_gain, float subln_eps,
+                    void *workspace, size_t workspace_bytes, float *Y, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Grouped decode: up to BL_MAX_GROUP independent steps-3+4 problems that    */
+/* share M, in ONE kernel launch (e.g. every projection of a decode step).   */
+/* Same arithmetic as bl_forward; requires M <= 16 and M*K <= 96 KiB for    */
+/* each problem.  `problems` is a HOST array, read during the call only.     */
+/* ------------------------------------------------------------------------ */
+#define BL_MAX_GROUP 128
+
+typedef struct {
+    const uint8_t *packed;  /* [N, K/4] */
+    const float *gamma;     /* [1] */
+    const int8_t *x_q;      /* [M, K] */
+    const float *s;         /* [M] */
+    float *Y;               /* [M, N] out */
+    int32_t *acc_out;       /* [M, N] out or NULL */
+    int64_t N;
+    int64_t K;
+} bl_problem;
+
+bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M,
+                             bl_stream_t stream);
+
+/* Grouped step 2: up to BL_MAX_GROUP activation inputs sharing M and dtype,
+ * one launch.  Same arithmetic as bl_quant_act.  `problems` is a HOST
+ * array. */
+typedef struct {
+    const void *X;           /* [M, K] of the call's dtype */
+    const float *subln_gain; /* [K] or NULL */
+    int8_t *x_q;             /* [M, K] out */
+    float *s;                /* [M] out */
+    int64_t K;
+} bl_act_problem;
+
+bl_status bl_quant_act_grouped(const bl_act_problem *problems, int count, bl_dtype xdt,
+                               int64_t M, float subln_eps, bl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BITLINEAR_H */

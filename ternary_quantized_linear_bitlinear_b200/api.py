@@ -1,0 +1,218 @@
+"""Python binding of libbitlinear.so (include/bitlinear.h).
+
+Argument marshalling only: every function here checks that torch tensors are
+CUDA, contiguous and of the right dtype, allocates outputs with torch when
+the caller passes none, and calls the C entry point of the same name with
+raw device pointers and the current torch stream.  All arithmetic runs in
+the library's kernels; if the library is missing, loading fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_LIB = None
+
+BL_F32, BL_BF16 = 0, 1
+BL_MAX_GROUP = 128
+_DTYPES = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}
+
+_i64 = ctypes.c_int64
+_p = ctypes.c_void_p
+_sz = ctypes.c_size_t
+_f32 = ctypes.c_float
+_int = ctypes.c_int
+
+
+class BitLinearError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+class Problem(ctypes.Structure):
+    """bl_problem: one (packed, gamma, x_q, s, Y) problem of a grouped forward."""
+    _fields_ = [("packed", _p), ("gamma", _p), ("x_q", _p), ("s", _p), ("Y", _p),
+                ("acc_out", _p), ("N", _i64), ("K", _i64)]
+
+
+class ActProblem(ctypes.Structure):
+    """bl_act_problem: one activation input of a grouped act quant."""
+    _fields_ = [("X", _p), ("subln_gain", _p), ("x_q", _p), ("s", _p), ("K", _i64)]
+
+
+_SIGS = {
+    "bl_status_string": (ctypes.c_char_p, [_int]),
+    "bl_version": (_int, []),
+    "bl_check_device_error": (_int, [_p]),
+    "bl_quant_weights_workspace_bytes": (_sz, [_i64, _i64]),
+    "bl_quant_weights": (_int, [_p, _int, _i64, _i64, _p, _p, _p, _sz, _p]),
+    "bl_quant_act": (_int, [_p, _int, _i64, _i64, _p, _f32, _p, _p, _p]),
+    "bl_forward": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
+    "bl_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "bl_linear": (_int, [_p, _int, _p, _int, _i64, _i64, _i64, _p, _f32, _p, _sz, _p, _p]),
+    "bl_forward_grouped": (_int, [ctypes.POINTER(Problem), _int, _i64, _p]),
+    "bl_quant_act_grouped": (_int, [ctypes.POINTER(ActProblem), _int, _int, _i64, _f32, _p]),
+}
+
+EXPORTED = tuple(_SIGS)
+
+
+def lib_path() -> str:
+    return _build.LIB
+
+
+def lib():
+    """Load libbitlinear.so (raises if it has not been built)."""
+    global _LIB
+    if _LIB is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with "
+                               "`python -m ternary_quantized_linear_bitlinear_b200.build`")
+        L = ctypes.CDLL(path)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+def status_string(status: int) -> str:
+    return lib().bl_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise BitLinearError(status, where)
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+# -- workspace queries ---------------------------------------------------------
+
+def quant_weights_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().bl_quant_weights_workspace_bytes(N, K))
+
+
+def linear_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().bl_linear_workspace_bytes(M, N, K))
+
+
+# -- step 1 --------------------------------------------------------------------
+
+def bl_quant_weights(W: torch.Tensor, packed=None, gamma=None, workspace=None, stream=None):
+    """-> (packed uint8 [N, K/4], gamma float32 [1])."""
+    _dev(W, "W")
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty(N, K // 4, dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(4, dtype=torch.float32, device=W.device)[:1]
+    if workspace is None:
+        workspace = torch.empty(quant_weights_workspace_bytes(N, K), dtype=torch.uint8, device=W.device)
+    rc = lib().bl_quant_weights(W.data_ptr(), _DTYPES.get(W.dtype, -1), N, K, packed.data_ptr(), gamma.data_ptr(),
+                                workspace.data_ptr(), workspace.numel(), _stream(stream))
+    _check(rc, "bl_quant_weights")
+    return packed, gamma
+
+
+# -- step 2 --------------------------------------------------------------------
+
+def bl_quant_act(X: torch.Tensor, subln_gain=None, subln_eps: float = 1e-6, x_q=None, s=None, stream=None):
+    """-> (x_q int8 [M, K], s float32 [M])."""
+    _dev(X, "X")
+    M, K = X.shape
+    if x_q is None:
+        x_q = torch.empty(M, K, dtype=torch.int8, device=X.device)
+    if s is None:
+        s = torch.empty(M, dtype=torch.float32, device=X.device)
+    if subln_gain is not None:
+        _dev(subln_gain, "subln_gain", torch.float32)
+    rc = lib().bl_quant_act(X.data_ptr(), _DTYPES.get(X.dtype, -1), M, K, _ptr(subln_gain), subln_eps,
+                            x_q.data_ptr(), s.data_ptr(), _stream(stream))
+    _check(rc, "bl_quant_act")
+    return x_q, s
+
+
+def bl_quant_act_grouped(items, dtype=torch.bfloat16, subln_eps: float = 1e-6, stream=None):
+    """items: list of (X [M, K], gain or None, x_q [M, K], s [M]), same M and dtype."""
+    arr = (ActProblem * len(items))()
+    M = items[0][0].shape[0]
+    for i, (X, gain, xq, s) in enumerate(items):
+        arr[i] = ActProblem(X.data_ptr(), _ptr(gain), xq.data_ptr(), s.data_ptr(), X.shape[1])
+    rc = lib().bl_quant_act_grouped(arr, len(items), _DTYPES.get(dtype, -1), M, subln_eps, _stream(stream))
+    _check(rc, "bl_quant_act_grouped")
+
+
+# -- steps 3 + 4 ---------------------------------------------------------------
+
+def bl_forward(packed, gamma, x_q, s, N: int, Y=None, acc_out=None, stream=None):
+    """-> Y float32 [M, N] (acc_out int32 [M, N] filled when given)."""
+    M, K = x_q.shape
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float32, device=x_q.device)
+    rc = lib().bl_forward(packed.data_ptr(), gamma.data_ptr(), x_q.data_ptr(), s.data_ptr(), M, N, K, Y.data_ptr(),
+                          _ptr(acc_out), _stream(stream))
+    _check(rc, "bl_forward")
+    return Y
+
+
+def make_problems(items):
+    """items: list of (packed, gamma, x_q, s, Y, acc_out or None, N, K) -> ctypes array."""
+    arr = (Problem * len(items))()
+    for i, (packed, gamma, xq, s, Y, acc, N, K) in enumerate(items):
+        arr[i] = Problem(packed.data_ptr(), gamma.data_ptr(), xq.data_ptr(), s.data_ptr(), Y.data_ptr(),
+                         _ptr(acc), N, K)
+    return arr
+
+
+def bl_forward_grouped(problems, count: int, M: int, stream=None):
+    """problems: ctypes array from make_problems (built once, launched many times)."""
+    rc = lib().bl_forward_grouped(problems, count, M, _stream(stream))
+    _check(rc, "bl_forward_grouped")
+
+
+# -- all four steps ------------------------------------------------------------
+
+def bl_linear(W, X, subln_gain=None, subln_eps: float = 1e-6, Y=None, workspace=None, stream=None):
+    """-> Y float32 [M, N] = BitLinear(X) with weights W quantized in the call."""
+    _dev(W, "W")
+    _dev(X, "X")
+    N, K = W.shape
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
+    if workspace is None:
+        workspace = torch.empty(linear_workspace_bytes(M, N, K), dtype=torch.uint8, device=X.device)
+    rc = lib().bl_linear(W.data_ptr(), _DTYPES.get(W.dtype, -1), X.data_ptr(), _DTYPES.get(X.dtype, -1), M, N, K,
+                         _ptr(subln_gain), subln_eps, workspace.data_ptr(), workspace.numel(), Y.data_ptr(),
+                         _stream(stream))
+    _check(rc, "bl_linear")
+    return Y
+
+
+def bl_check_device_error(stream=None):
+    _check(lib().bl_check_device_error(_stream(stream)), "bl_check_device_error")

@@ -1,0 +1,349 @@
+// libbitlinear.so: the C ABI declared in include/bitlinear.h.
+//
+// Host side only validates, picks an engine and enqueues kernels on the
+// caller's stream; it never allocates device memory and never synchronizes
+// (except bl_check_device_error, which is documented to).
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "bitlinear.h"
+#include "bl_common.cuh"
+#include "k_act_quant.cuh"
+#include "k_decode.cuh"
+#include "k_prefill.cuh"
+#include "k_weight_quant.cuh"
+
+using namespace bl;
+
+namespace {
+
+constexpr int BL_VERSION = 100;
+constexpr int64_t K_MAX = 32768;
+constexpr int MAX_DEVICES = 64;
+
+struct DeviceInfo {
+    bool init = false;
+    bool ok = false;
+    int sms = 0;
+};
+DeviceInfo g_dev[MAX_DEVICES];
+std::mutex g_dev_mu;
+
+bl_status device_info(DeviceInfo **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return BL_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    DeviceInfo &d = g_dev[dev];
+    if (!d.init) {
+        int major = 0, sms = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return BL_ERR_CUDA;
+        d.ok = (major == 10);
+        d.sms = sms;
+        if (d.ok) {
+            // opt in to large dynamic shared memory once per device
+            bool fail = false;
+            fail |= cudaFuncSetAttribute(k_decode<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         DEC_MAX_XQ_SMEM) != cudaSuccess;
+            fail |= cudaFuncSetAttribute(k_decode<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         DEC_MAX_XQ_SMEM) != cudaSuccess;
+            fail |= prefill_setup() != cudaSuccess;
+            if (fail) return BL_ERR_CUDA;
+        }
+        d.init = true;
+    }
+    if (!d.ok) return BL_ERR_DEVICE;
+    *out = &d;
+    return BL_OK;
+}
+
+inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+inline bl_status launch_status() {
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+bl_status check_k(int64_t K) {
+    if (K < 64 || K > K_MAX || (K % 64) != 0) return BL_ERR_SHAPE;
+    return BL_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Step 1
+
+bl_status quant_weights_impl(const DeviceInfo &d, const void *W, bl_dtype wdt, int64_t N, int64_t K,
+                             uint8_t *packed, float *gamma, void *ws, cudaStream_t st) {
+    const long long n = (long long)N * K;
+    const bool bf16 = wdt == BL_BF16;
+    const int epv = bf16 ? 8 : 4;
+    const long long nvec = n / epv;
+    long long grid = 2LL * d.sms;
+    long long need = (nvec + WQ_THREADS - 1) / WQ_THREADS;
+    if (grid > need) grid = need;
+    if (grid < 1) grid = 1;
+    // at most 2^14 terms per thread keeps each 64-bit window accumulator exact
+    while (grid < WQ_MAX_BLOCKS && ((nvec + grid * WQ_THREADS - 1) / (grid * WQ_THREADS)) * epv > 16384) grid *= 2;
+    if (grid > WQ_MAX_BLOCKS) grid = WQ_MAX_BLOCKS;
+
+    u64 *partials = reinterpret_cast<u64 *>(ws);
+    u32 *thresh = reinterpret_cast<u32 *>(reinterpret_cast<uint8_t *>(ws) + WQ_WS_PARTIALS);
+    const uint4 *Wv = reinterpret_cast<const uint4 *>(W);
+    if (bf16)
+        k_absmean_partial<true><<<(unsigned)grid, WQ_THREADS, 0, st>>>(Wv, nvec, partials);
+    else
+        k_absmean_partial<false><<<(unsigned)grid, WQ_THREADS, 0, st>>>(Wv, nvec, partials);
+    k_gamma_finalize<<<1, 32, 0, st>>>(partials, (int)grid, n, gamma, thresh);
+    const long long nwords = n / 16;
+    long long pgrid = (nwords + 255) / 256;
+    long long pcap = 8LL * d.sms;
+    if (pgrid > pcap) pgrid = pcap;
+    if (bf16)
+        k_ternary_pack<true><<<(unsigned)pgrid, 256, 0, st>>>(Wv, nwords, thresh, reinterpret_cast<u32 *>(packed));
+    else
+        k_ternary_pack<false><<<(unsigned)pgrid, 256, 0, st>>>(Wv, nwords, thresh, reinterpret_cast<u32 *>(packed));
+    return launch_status();
+}
+
+// ---------------------------------------------------------------------------
+// Step 2
+
+bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStream_t st) {
+    const bool bf16 = xdt == BL_BF16;
+    const int epv = bf16 ? 8 : 4;
+    const long long nvec = Kmax / epv;
+    int vec = 1;
+    while ((nvec + vec - 1) / vec > 1024) vec *= 2;
+    int T = (int)(((nvec + vec - 1) / vec + 31) / 32 * 32);
+    const unsigned grid = (unsigned)(P.count * P.M);
+#define BL_AQ_CASE(B, V)                                                        \
+    if (bf16 == B && vec == V) {                                                \
+        k_act_quant<B, V><<<grid, T, 0, st>>>(P);                               \
+        return launch_status();                                                 \
+    }
+    // at most 32 values per thread (bf16: 4 vectors, f32: 8 vectors)
+    BL_AQ_CASE(true, 1)
+    BL_AQ_CASE(true, 2)
+    BL_AQ_CASE(true, 4)
+    BL_AQ_CASE(false, 1)
+    BL_AQ_CASE(false, 2)
+    BL_AQ_CASE(false, 4)
+    BL_AQ_CASE(false, 8)
+    return BL_ERR_SHAPE;
+#undef BL_AQ_CASE
+}
+
+// ---------------------------------------------------------------------------
+// Steps 3 + 4
+
+int decode_glog(int64_t K) {
+    int steps = (int)((K + 255) / 256);
+    if (steps <= 3) return 0;
+    if (steps <= 6) return 1;
+    if (steps <= 12) return 2;
+    return 3;
+}
+
+bool decode_eligible(int64_t M, int64_t K) { return M <= 16 && M * dec_row_stride((int)K) <= DEC_MAX_XQ_SMEM; }
+
+bl_status decode_launch(DecodeParams &P, cudaStream_t st) {
+    int total = 0;
+    int rs_max = 0;
+    for (int i = 0; i < P.count; ++i) {
+        DecodeProblem &q = P.p[i];
+        q.g_log2 = decode_glog(q.K);
+        int tiles = (q.N + 15) / 16;
+        int per = DEC_WARPS >> q.g_log2;
+        q.cta_begin = total;
+        total += (tiles + per - 1) / per;
+        int rs = dec_row_stride(q.K);
+        rs_max = rs > rs_max ? rs : rs_max;
+    }
+    size_t smem = (size_t)P.M * rs_max;
+    if (P.M <= 8)
+        k_decode<1><<<total, DEC_THREADS, smem, st>>>(P);
+    else
+        k_decode<2><<<total, DEC_THREADS, smem, st>>>(P);
+    return launch_status();
+}
+
+bl_status forward_impl(const uint8_t *packed, const float *gamma, const int8_t *x_q, const float *s,
+                       int64_t M, int64_t N, int64_t K, float *Y, int32_t *acc_out, cudaStream_t st) {
+    if (decode_eligible(M, K)) {
+        DecodeParams P;
+        P.count = 1;
+        P.M = (int)M;
+        P.p[0] = DecodeProblem{packed, gamma, x_q, s, Y, acc_out, (int)N, (int)K, 0, 0};
+        return decode_launch(P, st);
+    }
+    return prefill_launch(packed, gamma, x_q, s, M, N, K, Y, acc_out, st);
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+
+extern "C" {
+
+const char *bl_status_string(bl_status s) {
+    switch (s) {
+        case BL_OK: return "BL_OK";
+        case BL_ERR_NULL: return "BL_ERR_NULL: a required pointer is NULL";
+        case BL_ERR_SHAPE: return "BL_ERR_SHAPE: M, N, K or count outside the supported range";
+        case BL_ERR_ALIGN: return "BL_ERR_ALIGN: a pointer is not 16-byte aligned";
+        case BL_ERR_DTYPE: return "BL_ERR_DTYPE: unknown dtype code";
+        case BL_ERR_CUDA: return "BL_ERR_CUDA: a CUDA runtime call or launch failed";
+        case BL_ERR_TIMEOUT: return "BL_ERR_TIMEOUT: a bounded device-side wait gave up";
+        case BL_ERR_WORKSPACE: return "BL_ERR_WORKSPACE: workspace missing or too small";
+        case BL_ERR_DEVICE: return "BL_ERR_DEVICE: current device is not compute capability 10.x";
+    }
+    return "BL_ERR_UNKNOWN";
+}
+
+int bl_version(void) { return BL_VERSION; }
+
+bl_status bl_check_device_error(bl_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return BL_ERR_CUDA;
+    u32 v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return BL_ERR_CUDA;
+    if (v != 0 && cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return BL_ERR_CUDA;
+    return v ? BL_ERR_TIMEOUT : BL_OK;
+}
+
+size_t bl_quant_weights_workspace_bytes(int64_t N, int64_t K) {
+    (void)N;
+    (void)K;
+    return align256(WQ_WS_BYTES);
+}
+
+bl_status bl_quant_weights(const void *W, bl_dtype wdt, int64_t N, int64_t K, uint8_t *packed, float *gamma,
+                           void *workspace, size_t workspace_bytes, bl_stream_t stream) {
+    if (!W || !packed || !gamma) return BL_ERR_NULL;
+    if (wdt != BL_F32 && wdt != BL_BF16) return BL_ERR_DTYPE;
+    if (N < 1 || check_k(K) != BL_OK || N * K >= (1LL << 31)) return BL_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(packed) || !aligned16(gamma)) return BL_ERR_ALIGN;
+    if (!workspace || workspace_bytes < bl_quant_weights_workspace_bytes(N, K)) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGN;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return quant_weights_impl(*d, W, wdt, N, K, packed, gamma, workspace, (cudaStream_t)stream);
+}
+
+bl_status bl_quant_act_grouped(const bl_act_problem *problems, int count, bl_dtype xdt, int64_t M, float subln_eps,
+                               bl_stream_t stream) {
+    if (!problems) return BL_ERR_NULL;
+    if (count < 1 || count > BL_MAX_GROUP || M < 1 || M * (int64_t)count > 0x7fffffffLL) return BL_ERR_SHAPE;
+    if (xdt != BL_F32 && xdt != BL_BF16) return BL_ERR_DTYPE;
+    ActParams P;
+    P.count = count;
+    P.M = (int)M;
+    P.eps = subln_eps;
+    int64_t kmax = 0;
+    for (int i = 0; i < count; ++i) {
+        const bl_act_problem &q = problems[i];
+        if (!q.X || !q.x_q || !q.s) return BL_ERR_NULL;
+        if (check_k(q.K) != BL_OK) return BL_ERR_SHAPE;
+        if (!aligned16(q.X) || !aligned16(q.x_q) || !aligned16(q.s) || (q.subln_gain && !aligned16(q.subln_gain)))
+            return BL_ERR_ALIGN;
+        P.p[i] = ActProblem{q.X, q.subln_gain, q.x_q, q.s, (int)q.K, 0};
+        kmax = q.K > kmax ? q.K : kmax;
+    }
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return quant_act_impl(P, xdt, kmax, (cudaStream_t)stream);
+}
+
+bl_status bl_quant_act(const void *X, bl_dtype xdt, int64_t M, int64_t K, const float *subln_gain, float subln_eps,
+                       int8_t *x_q, float *s, bl_stream_t stream) {
+    bl_act_problem q{X, subln_gain, x_q, s, K};
+    return bl_quant_act_grouped(&q, 1, xdt, M, subln_eps, stream);
+}
+
+bl_status bl_forward(const uint8_t *packed, const float *gamma, const int8_t *x_q, const float *s, int64_t M,
+                     int64_t N, int64_t K, float *Y, int32_t *acc_out, bl_stream_t stream) {
+    if (!packed || !gamma || !x_q || !s || !Y) return BL_ERR_NULL;
+    if (M < 1 || N < 1 || M > 0x7fffffffLL || N > 0x7fffffffLL || check_k(K) != BL_OK) return BL_ERR_SHAPE;
+    if (!aligned16(packed) || !aligned16(gamma) || !aligned16(x_q) || !aligned16(s) || !aligned16(Y) ||
+        (acc_out && !aligned16(acc_out)))
+        return BL_ERR_ALIGN;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return forward_impl(packed, gamma, x_q, s, M, N, K, Y, acc_out, (cudaStream_t)stream);
+}
+
+bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, bl_stream_t stream) {
+    if (!problems) return BL_ERR_NULL;
+    if (count < 1 || count > BL_MAX_GROUP || M < 1 || M > 16) return BL_ERR_SHAPE;
+    DecodeParams P;
+    P.count = count;
+    P.M = (int)M;
+    long long ctas = 0;
+    for (int i = 0; i < count; ++i) {
+        const bl_problem &q = problems[i];
+        if (!q.packed || !q.gamma || !q.x_q || !q.s || !q.Y) return BL_ERR_NULL;
+        if (q.N < 1 || q.N > 0x7fffffffLL || check_k(q.K) != BL_OK || !decode_eligible(M, q.K)) return BL_ERR_SHAPE;
+        if (!aligned16(q.packed) || !aligned16(q.gamma) || !aligned16(q.x_q) || !aligned16(q.s) || !aligned16(q.Y) ||
+            (q.acc_out && !aligned16(q.acc_out)))
+            return BL_ERR_ALIGN;
+        P.p[i] = DecodeProblem{q.packed, q.gamma, q.x_q, q.s, q.Y, q.acc_out, (int)q.N, (int)q.K, 0, 0};
+        ctas += (q.N + 15) / 16;
+    }
+    if (ctas > 0x7fffffffLL) return BL_ERR_SHAPE;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return decode_launch(P, (cudaStream_t)stream);
+}
+
+size_t bl_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M < 1 || N < 1 || K < 1) return 0;
+    return align256(WQ_WS_BYTES) + align256((size_t)N * (size_t)K / 4) + 256 + align256((size_t)M * (size_t)K) +
+           align256((size_t)M * 4);
+}
+
+bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt, int64_t M, int64_t N, int64_t K,
+                    const float *subln_gain, float subln_eps, void *workspace, size_t workspace_bytes, float *Y,
+                    bl_stream_t stream) {
+    if (!W || !X || !Y) return BL_ERR_NULL;
+    if (wdt != BL_F32 && wdt != BL_BF16) return BL_ERR_DTYPE;
+    if (xdt != BL_F32 && xdt != BL_BF16) return BL_ERR_DTYPE;
+    if (M < 1 || N < 1 || M > 0x7fffffffLL || check_k(K) != BL_OK || N * K >= (1LL << 31)) return BL_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(X) || !aligned16(Y) || (subln_gain && !aligned16(subln_gain)))
+        return BL_ERR_ALIGN;
+    if (!workspace || workspace_bytes < bl_linear_workspace_bytes(M, N, K)) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGN;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    uint8_t *p = reinterpret_cast<uint8_t *>(workspace);
+    void *wq_ws = p;
+    p += align256(WQ_WS_BYTES);
+    uint8_t *packed = p;
+    p += align256((size_t)N * (size_t)K / 4);
+    float *gamma = reinterpret_cast<float *>(p);
+    p += 256;
+    int8_t *x_q = reinterpret_cast<int8_t *>(p);
+    p += align256((size_t)M * (size_t)K);
+    float *s = reinterpret_cast<float *>(p);
+    cudaStream_t st = (cudaStream_t)stream;
+    rc = quant_weights_impl(*d, W, wdt, N, K, packed, gamma, wq_ws, st);
+    if (rc) return rc;
+    ActParams P;
+    P.count = 1;
+    P.M = (int)M;
+    P.eps = subln_eps;
+    P.p[0] = ActProblem{X, subln_gain, x_q, s, (int)K, 0};
+    rc = quant_act_impl(P, xdt, K, st);
+    if (rc) return rc;
+    return forward_impl(packed, gamma, x_q, s, M, N, K, Y, nullptr, st);
+}
+
+}  // extern "C"

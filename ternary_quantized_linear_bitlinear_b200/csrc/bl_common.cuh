@@ -1,0 +1,157 @@
+// Shared device helpers for libbitlinear (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "bitlinear.h"
+
+namespace bl {
+
+typedef unsigned long long u64;
+typedef unsigned int u32;
+
+// Sticky device error word: bounded waits that give up OR a code in here and
+// return; the host reads it with bl_check_device_error.
+enum : u32 {
+    DEVERR_NONE = 0,
+    DEVERR_TIMEOUT_PRODUCER = 1u << 0,
+    DEVERR_TIMEOUT_MMA = 1u << 1,
+    DEVERR_TIMEOUT_EXPAND = 1u << 2,
+    DEVERR_TIMEOUT_EPILOGUE = 1u << 3,
+    DEVERR_TMEM_ALLOC = 1u << 4,
+};
+
+__device__ u32 g_device_error;
+
+__device__ __forceinline__ void raise_device_error(u32 code) { atomicOr(&g_device_error, code); }
+
+// Float bits of element i of a 16-byte vector of the given dtype.
+__device__ __forceinline__ u32 bf16_bits_to_f32_bits(uint16_t h) { return (u32)h << 16; }
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Streamed once: do not keep in L1.
+__device__ __forceinline__ uint4 ldg_stream_v4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ u64 mad_wide_u32(u32 a, u32 b, u64 c) {
+    u64 d;
+    asm("mad.wide.u32 %0, %1, %2, %3;" : "=l"(d) : "r"(a), "r"(b), "l"(c));
+    return d;
+}
+
+// ---------------------------------------------------------------------------
+// Exact multi-limb fixed point (little-endian u64 limbs).
+
+// L += (hi:lo) << sh, 0 <= sh; bits shifted past the last limb are dropped
+// (callers size L so that never happens).
+template <int NL>
+__device__ __forceinline__ void limbs_add_u128_shl(u64 (&L)[NL], u64 lo, u64 hi, int sh) {
+    int w = sh >> 6, b = sh & 63;
+    u64 p0 = lo << b;
+    u64 p1 = b ? ((hi << b) | (lo >> (64 - b))) : hi;
+    u64 p2 = b ? (hi >> (64 - b)) : 0ull;
+    u64 carry = 0;
+#pragma unroll
+    for (int i = 0; i < NL; ++i) {
+        u64 add = (i == w) ? p0 : (i == w + 1) ? p1 : (i == w + 2) ? p2 : 0ull;
+        if (i < w) continue;
+        u64 s = L[i] + add;
+        u64 c1 = s < add;
+        u64 s2 = s + carry;
+        u64 c2 = s2 < carry;
+        L[i] = s2;
+        carry = c1 | c2;
+    }
+}
+
+template <int NL>
+__device__ __forceinline__ void limbs_add(u64 (&L)[NL], const u64 (&R)[NL]) {
+    u64 carry = 0;
+#pragma unroll
+    for (int i = 0; i < NL; ++i) {
+        u64 s = L[i] + R[i];
+        u64 c1 = s < R[i];
+        u64 s2 = s + carry;
+        u64 c2 = s2 < carry;
+        L[i] = s2;
+        carry = c1 | c2;
+    }
+}
+
+// 2^e as a double, -1022 <= e <= 1023.
+__device__ __forceinline__ double pow2_double(int e) {
+    return __longlong_as_double((long long)(e + 1023) << 52);
+}
+
+// Round the non-negative integer in L to the nearest double (ties to even)
+// and scale by 2^scale_exp.
+template <int NL>
+__device__ double limbs_to_double_rn(const u64 (&L)[NL], int scale_exp) {
+    int top = -1;
+#pragma unroll
+    for (int i = NL - 1; i >= 0; --i) {
+        if (top < 0 && L[i] != 0ull) top = i * 64 + 63 - __clzll((long long)L[i]);
+    }
+    if (top < 0) return 0.0;
+    int lo = top - 63;  // bit index of window bit 0
+    u64 w;
+    bool sticky = false;
+    if (lo >= 0) {
+        int wi = lo >> 6, s = lo & 63;
+        u64 cur = 0, nxt = 0;
+#pragma unroll
+        for (int i = 0; i < NL; ++i) {
+            if (i == wi) cur = L[i];
+            if (i == wi + 1) nxt = L[i];
+            if (i < wi && L[i] != 0ull) sticky = true;
+        }
+        w = s ? ((cur >> s) | (nxt << (64 - s))) : cur;
+        if (s && (cur & ((1ull << s) - 1ull))) sticky = true;
+    } else {
+        w = L[0] << (-lo);
+    }
+    u64 mant = w >> 11;
+    bool rb = (w >> 10) & 1ull;
+    if (w & 0x3ffull) sticky = true;
+    int e = lo + 11 + scale_exp;
+    if (rb && (sticky || (mant & 1ull))) {
+        mant += 1ull;
+        if (mant == (1ull << 53)) {
+            mant >>= 1;
+            e += 1;
+        }
+    }
+    return __ll2double_rn((long long)mant) * pow2_double(e);
+}
+
+// ---------------------------------------------------------------------------
+// Block-wide reductions (blockDim.x multiple of 32, <= 1024).
+
+__device__ __forceinline__ u32 warp_max_u32(u32 v) { return __reduce_max_sync(0xffffffffu, v); }
+
+__device__ __forceinline__ void warp_sum_u128(u64 &lo, u64 &hi) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        u64 olo = __shfl_down_sync(0xffffffffu, lo, off);
+        u64 ohi = __shfl_down_sync(0xffffffffu, hi, off);
+        u64 s = lo + olo;
+        hi += ohi + (s < lo ? 1ull : 0ull);
+        lo = s;
+    }
+}
+
+}  // namespace bl

@@ -1,0 +1,199 @@
+// Step 1 of the BitLinear forward: absmean ternary weight quantization and
+// 2-bit packing ("Distillix" README, 1. BitNet b1.58 Core; "bitone" README,
+// Forward pass; "SLM750-Edge" section 3.1).
+//
+// Three launches, all on the caller's stream:
+//   k_absmean_partial  one pass over W: exact per-block sum of |w| as a
+//                      384-bit fixed-point integer in units of 2^-149
+//   k_gamma_finalize   one warp: sums the block partials, rounds once to
+//                      double, gamma = float(S / n) + 1e-5f, and the float
+//                      threshold T with  |w| >= T  <=>  float(|w|/gamma) > 0.5
+//   k_ternary_pack     second pass over W: code = sign(w) * (|w| >= T), four
+//                      codes per byte in the packed word layout
+//
+// Exactness: every finite float is an integer multiple of 2^-149, so sum|w|
+// is an integer in those units.  Each thread accumulates m << (e - base) in a
+// 64-bit register for exponents inside a 26-binade window chosen per block
+// from a sample of its data (term < 2^49, at most 2^14 terms per thread).
+// Anything outside the window (tiny, huge or subnormal values) is added
+// exactly into per-block shared-memory bins indexed by exponent.  The result
+// does not depend on the window, the grid or the order of the additions.
+#pragma once
+
+#include "bl_common.cuh"
+
+namespace bl {
+
+constexpr int WQ_THREADS = 512;
+constexpr int WQ_WINDOW = 25;       // fast path: base <= e <= base + 25
+constexpr int WQ_PART_LIMBS = 6;    // per-block partial, 384 bits
+constexpr int WQ_MAX_BLOCKS = 1024;
+constexpr size_t WQ_WS_PARTIALS = (size_t)WQ_MAX_BLOCKS * WQ_PART_LIMBS * 8;
+constexpr size_t WQ_WS_BYTES = WQ_WS_PARTIALS + 256;  // + threshold scratch
+
+// Float bits of the j-th element of a 16-byte vector.
+template <bool BF16>
+__device__ __forceinline__ u32 vec_elem_bits(const uint4 &v, int j) {
+    const u32 w[4] = {v.x, v.y, v.z, v.w};
+    if (BF16) {
+        u32 word = w[j >> 1];
+        return (j & 1) ? (word & 0xffff0000u) : (word << 16);
+    } else {
+        return w[j];
+    }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const uint4 *__restrict__ W, long long nvec,
+                                                                 u64 *__restrict__ partials) {
+    constexpr int EPV = BF16 ? 8 : 4;  // elements per 16-byte vector
+    __shared__ u64 s_bins[256];
+    __shared__ u32 s_emax;
+    __shared__ u64 s_wlo[WQ_THREADS / 32], s_whi[WQ_THREADS / 32];
+
+    const int tid = threadIdx.x;
+    for (int i = tid; i < 256; i += WQ_THREADS) s_bins[i] = 0ull;
+    if (tid == 0) s_emax = 0;
+
+    const long long stride = (long long)gridDim.x * WQ_THREADS;
+    const long long first = (long long)blockIdx.x * WQ_THREADS + tid;
+
+    // Window from a sample: the block's first vector per thread.
+    u32 emax = 0;
+    uint4 v0 = make_uint4(0, 0, 0, 0);
+    if (first < nvec) {
+        v0 = ldg_stream_v4(W + first);
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) {
+            u32 e = (vec_elem_bits<BF16>(v0, j) & 0x7fffffffu) >> 23;
+            emax = e > emax ? e : emax;
+        }
+    }
+    emax = warp_max_u32(emax);
+    __syncthreads();
+    if ((tid & 31) == 0) atomicMax(&s_emax, emax);
+    __syncthreads();
+    int top = (int)s_emax + 2;
+    if (top > 254) top = 254;
+    int base = top - WQ_WINDOW;
+    if (base < 1) base = 1;
+
+    u64 acc = 0ull;
+    auto add_vec = [&](const uint4 &v) {
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) {
+            u32 u = vec_elem_bits<BF16>(v, j) & 0x7fffffffu;
+            u32 e = u >> 23;
+            u32 m = (u & 0x7fffffu) | 0x800000u;
+            u32 d = e - (u32)base;
+            if (d <= (u32)WQ_WINDOW) {
+                acc = mad_wide_u32(m, 1u << d, acc);
+            } else if (u != 0u) {
+                atomicAdd(&s_bins[e], (u64)(e ? m : (u & 0x7fffffu)));
+            }
+        }
+    };
+    if (first < nvec) add_vec(v0);
+    long long i = first + stride;
+    // two vectors in flight per iteration
+    for (; i + stride < nvec; i += 2 * stride) {
+        uint4 a = ldg_stream_v4(W + i);
+        uint4 b = ldg_stream_v4(W + i + stride);
+        add_vec(a);
+        add_vec(b);
+    }
+    if (i < nvec) add_vec(ldg_stream_v4(W + i));
+
+    // Block sum of the 64-bit window accumulators as 128 bits.
+    u64 lo = acc, hi = 0ull;
+    warp_sum_u128(lo, hi);
+    if ((tid & 31) == 0) {
+        s_wlo[tid >> 5] = lo;
+        s_whi[tid >> 5] = hi;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        u64 L[WQ_PART_LIMBS] = {0, 0, 0, 0, 0, 0};
+        u64 blo = 0, bhi = 0;
+        for (int w = 0; w < WQ_THREADS / 32; ++w) {
+            u64 s = blo + s_wlo[w];
+            bhi += s_whi[w] + (s < blo ? 1ull : 0ull);
+            blo = s;
+        }
+        // term m << (e - base) stands for m * 2^(e - 150) = term * 2^(base - 1) units
+        limbs_add_u128_shl(L, blo, bhi, base - 1);
+        for (int e = 0; e < 256; ++e) {
+            u64 b = s_bins[e];
+            if (b) limbs_add_u128_shl(L, b, 0ull, e > 0 ? e - 1 : 0);
+        }
+#pragma unroll
+        for (int k = 0; k < WQ_PART_LIMBS; ++k) partials[(size_t)blockIdx.x * WQ_PART_LIMBS + k] = L[k];
+    }
+}
+
+// One warp.  Writes gamma and the threshold bits (as u32) into ws_thresh.
+__global__ void __launch_bounds__(32) k_gamma_finalize(const u64 *__restrict__ partials, int nblocks,
+                                                         long long n, float *__restrict__ gamma_out,
+                                                         u32 *__restrict__ ws_thresh) {
+    constexpr int NL = WQ_PART_LIMBS + 1;
+    __shared__ u64 s_L[32][NL];
+    const int lane = threadIdx.x;
+    u64 L[NL];
+#pragma unroll
+    for (int k = 0; k < NL; ++k) L[k] = 0ull;
+    for (int b = lane; b < nblocks; b += 32) {
+        u64 R[NL];
+#pragma unroll
+        for (int k = 0; k < WQ_PART_LIMBS; ++k) R[k] = partials[(size_t)b * WQ_PART_LIMBS + k];
+        R[NL - 1] = 0ull;
+        limbs_add(L, R);
+    }
+#pragma unroll
+    for (int k = 0; k < NL; ++k) s_L[lane][k] = L[k];
+    __syncwarp();
+    if (lane == 0) {
+        for (int l = 1; l < 32; ++l) {
+            u64 R[NL];
+#pragma unroll
+            for (int k = 0; k < NL; ++k) R[k] = s_L[l][k];
+            limbs_add(L, R);
+        }
+        double S = limbs_to_double_rn(L, -149);
+        float mean = __double2float_rn(__ddiv_rn(S, (double)n));
+        float g = __fadd_rn(mean, 1e-5f);
+        // smallest t with float(t / g) > 0.5: start at g/2 (exact, quotient 0.5)
+        float t = __fmul_rn(0.5f, g);
+        for (int it = 0; it < 64 && !(__fdiv_rn(t, g) > 0.5f); ++it)
+            t = __uint_as_float(__float_as_uint(t) + 1u);
+        gamma_out[0] = g;
+        ws_thresh[0] = __float_as_uint(t);
+    }
+}
+
+// Each thread packs 16 consecutive weights into one 32-bit word per step.
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_ternary_pack(const uint4 *__restrict__ W, long long nwords,
+                                                        const u32 *__restrict__ ws_thresh,
+                                                        u32 *__restrict__ packed) {
+    constexpr int VPW = BF16 ? 2 : 4;  // 16-byte vectors per 16 weights
+    const u32 T = ws_thresh[0];
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long wi = (long long)blockIdx.x * blockDim.x + threadIdx.x; wi < nwords; wi += stride) {
+        uint4 v[VPW];
+#pragma unroll
+        for (int q = 0; q < VPW; ++q) v[q] = ldg_stream_v4(W + wi * VPW + q);
+        u32 word = 0;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            constexpr int EPV = BF16 ? 8 : 4;
+            u32 bits = vec_elem_bits<BF16>(v[k / EPV], k % EPV);
+            u32 nz = (bits & 0x7fffffffu) >= T ? 1u : 0u;
+            u32 code = nz | ((bits >> 30) & 2u & (nz << 1));  // 01 = +1, 11 = -1
+            int i = k & 3, j = k >> 2;
+            word |= code << (8 * i + 2 * j);
+        }
+        packed[wi] = word;
+    }
+}
+
+}  // namespace bl

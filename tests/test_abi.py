@@ -1,0 +1,139 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/bitlinear.h declares, and rejects bad arguments on the host before
+touching the device (validation pattern: "bitone" README, Security --
+ndim / dtype / contiguity / bounds / null checks at the binding boundary)."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from ternary_quantized_linear_bitlinear_b200 import api, build
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "bitlinear.h")
+
+OK, NULL, SHAPE, ALIGN, DTYPE, CUDA, TIMEOUT, WORKSPACE, DEVICE = range(9)
+A = 1 << 20  # a fake, 16-byte aligned "device address" (never dereferenced)
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return api.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bl_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(api.EXPORTED)
+
+
+def test_status_strings_and_version(L):
+    for s in range(9):
+        assert api.status_string(s).startswith("BL_")
+    assert api.status_string(99) == "BL_ERR_UNKNOWN"
+    assert L.bl_version() == 100
+
+
+def test_workspace_queries(L):
+    assert L.bl_quant_weights_workspace_bytes(2048, 768) >= 49152
+    M, N, K = 16, 2048, 768
+    ws = L.bl_linear_workspace_bytes(M, N, K)
+    assert ws >= L.bl_quant_weights_workspace_bytes(N, K) + N * K // 4 + M * K + 4 * M
+    assert L.bl_linear_workspace_bytes(0, N, K) == 0
+
+
+def qw(L, W=A, wdt=0, N=64, K=128, packed=A, gamma=A, ws=A, wsb=1 << 20):
+    return L.bl_quant_weights(W, wdt, N, K, packed, gamma, ws, wsb, None)
+
+
+def test_quant_weights_validation(L):
+    assert qw(L, W=None) == NULL
+    assert qw(L, packed=None) == NULL
+    assert qw(L, gamma=None) == NULL
+    assert qw(L, wdt=7) == DTYPE
+    assert qw(L, K=100) == SHAPE
+    assert qw(L, K=0) == SHAPE
+    assert qw(L, K=32768 + 64) == SHAPE
+    assert qw(L, N=0) == SHAPE
+    assert qw(L, N=1 << 17, K=1 << 14) == SHAPE  # N*K = 2^31
+    assert qw(L, W=A + 8) == ALIGN
+    assert qw(L, packed=A + 4) == ALIGN
+    assert qw(L, ws=None) == WORKSPACE
+    assert qw(L, wsb=16) == WORKSPACE
+    # valid arguments reach the device query, which fails without a GPU
+    assert qw(L) in (CUDA, DEVICE)
+
+
+def test_quant_act_validation(L):
+    f = L.bl_quant_act
+    assert f(None, 0, 4, 128, None, 1e-6, A, A, None) == NULL
+    assert f(A, 0, 4, 128, None, 1e-6, None, A, None) == NULL
+    assert f(A, 2, 4, 128, None, 1e-6, A, A, None) == DTYPE
+    assert f(A, 0, 0, 128, None, 1e-6, A, A, None) == SHAPE
+    assert f(A, 0, 4, 96, None, 1e-6, A, A, None) == SHAPE
+    assert f(A, 0, 4, 128, A + 4, 1e-6, A, A, None) == ALIGN
+    assert f(A, 1, 4, 128, None, 1e-6, A, A, None) in (CUDA, DEVICE)
+
+
+def test_forward_validation(L):
+    f = L.bl_forward
+    assert f(None, A, A, A, 1, 64, 128, A, None, None) == NULL
+    assert f(A, A, A, A, 1, 64, 128, None, None, None) == NULL
+    assert f(A, A, A, A, 0, 64, 128, A, None, None) == SHAPE
+    assert f(A, A, A, A, 1, 0, 128, A, None, None) == SHAPE
+    assert f(A, A, A, A, 1, 64, 130, A, None, None) == SHAPE
+    assert f(A, A, A, A, 1, 64, 128, A + 1, None, None) == ALIGN
+    assert f(A, A, A, A, 1, 64, 128, A, A + 2, None) == ALIGN
+    assert f(A, A, A, A, 1, 64, 128, A, None, None) in (CUDA, DEVICE)
+
+
+def test_linear_validation(L):
+    f = L.bl_linear
+    wsb = L.bl_linear_workspace_bytes(8, 64, 128)
+    assert f(None, 0, A, 0, 8, 64, 128, None, 1e-6, A, wsb, A, None) == NULL
+    assert f(A, 3, A, 0, 8, 64, 128, None, 1e-6, A, wsb, A, None) == DTYPE
+    assert f(A, 0, A, 3, 8, 64, 128, None, 1e-6, A, wsb, A, None) == DTYPE
+    assert f(A, 0, A, 0, 8, 64, 127, None, 1e-6, A, wsb, A, None) == SHAPE
+    assert f(A, 0, A, 0, 8, 64, 128, None, 1e-6, A, wsb - 1, A, None) == WORKSPACE
+    assert f(A, 0, A, 0, 8, 64, 128, None, 1e-6, A + 8, wsb, A, None) == ALIGN
+    assert f(A, 0, A, 0, 8, 64, 128, None, 1e-6, A, wsb, A, None) in (CUDA, DEVICE)
+
+
+def test_grouped_validation(L):
+    P = (api.Problem * 2)()
+    for i in range(2):
+        P[i] = api.Problem(A, A, A, A, A, None, 64, 128)
+    g = L.bl_forward_grouped
+    assert g(None, 1, 1, None) == NULL
+    assert g(P, 0, 1, None) == SHAPE
+    assert g(P, api.BL_MAX_GROUP + 1, 1, None) == SHAPE
+    assert g(P, 2, 17, None) == SHAPE  # grouped decode is for M <= 16
+    P[1].K = 100
+    assert g(P, 2, 1, None) == SHAPE
+    P[1].K = 128
+    P[1].Y = None
+    assert g(P, 2, 1, None) == NULL
+    P[1].Y = A
+    assert g(P, 2, 1, None) in (CUDA, DEVICE)
+    Q = (api.ActProblem * 1)()
+    Q[0] = api.ActProblem(A, None, A, A, 128)
+    assert L.bl_quant_act_grouped(Q, 1, 5, 1, 1e-6, None) == DTYPE
+    assert L.bl_quant_act_grouped(Q, 1, 1, 1, 1e-6, None) in (CUDA, DEVICE)
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(api, "_LIB", None)
+    monkeypatch.setattr(build, "LIB", str(tmp_path / "libbitlinear.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        api.lib()

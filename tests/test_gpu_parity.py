@@ -1,0 +1,193 @@
+"""GPU path vs CPU oracle, element by element, through the C ABI.
+
+Bit-exact: packed weights, gamma, x_q, s, acc.  Y: |Y - Y_ref| <= 1e-6 |Y_ref|.
+Small cases cover several tiles plus ragged tails; the full-size cases run
+the workloads' shapes in the launch configuration the benchmark times and
+compare sampled outputs (all outputs where the oracle is fast enough).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from ternary_quantized_linear_bitlinear_b200 import api, workloads
+from _parity import check_act, check_forward_full, check_forward_sampled, check_weights, gpu_quant_weights, np32
+
+pytestmark = pytest.mark.gpu
+
+
+def chain(W_cpu, X_cpu, gain_cpu=None, eps=1e-6, want_acc=True):
+    """GPU: quant weights, quant act, forward.  Returns device tensors."""
+    W = W_cpu.cuda()
+    X = X_cpu.cuda()
+    packed, gamma = api.bl_quant_weights(W)
+    x_q, s = api.bl_quant_act(X, None if gain_cpu is None else gain_cpu.cuda(), eps)
+    M, N = X.shape[0], W.shape[0]
+    acc = torch.empty(M, N, dtype=torch.int32, device="cuda") if want_acc else None
+    Y = api.bl_forward(packed, gamma, x_q, s, N, acc_out=acc)
+    api.bl_check_device_error()
+    return packed, gamma, x_q, s, Y, acc
+
+
+# -- step 1 --------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,K,dtype,kind", [
+    (2048, 768, torch.float32, "normal"),
+    (37, 192, torch.float32, "normal"),
+    (37, 192, torch.bfloat16, "normal"),
+    (1, 64, torch.float32, "normal"),
+    (300, 4096, torch.bfloat16, "normal"),
+    (64, 1024, torch.float32, "wide"),
+    (48, 512, torch.float32, "zeros"),
+    (33, 320, torch.bfloat16, "ternary"),
+    (9728, 2560, torch.bfloat16, "normal"),
+])
+def test_quant_weights(N, K, dtype, kind):
+    if kind == "normal":
+        W = workloads.normal((N, K), 0.02, 100 + N, dtype)
+    elif kind == "wide":
+        # exponents spread over ~230 binades, subnormals and zeros: every
+        # exact-sum path (window, bins, subnormal) is exercised
+        g = torch.Generator().manual_seed(5)
+        mant = torch.randn(N, K, generator=g, dtype=torch.float64)
+        ex = torch.randint(-150, 80, (N, K), generator=g).double()
+        W = (mant * torch.pow(2.0, ex)).float()
+        W[0, :17] = 0.0
+        W[1, :5] = torch.tensor([1e-45, -3e-44, 1e-39, 3e38, -2e38])
+        W = W.to(dtype)
+    elif kind == "zeros":
+        W = torch.zeros(N, K, dtype=dtype)
+    else:
+        W = workloads.ternary_weights(N, K, seed=3, dtype=dtype)
+    packed, gamma = gpu_quant_weights(W)
+    check_weights(W, packed, gamma)
+    if kind == "zeros":
+        assert gamma.item() == np.float32(1e-5)
+        assert int(packed.sum()) == 0
+
+
+# -- step 2 --------------------------------------------------------------------
+
+def _wide_rows(M, K, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn(M, K, generator=g, dtype=torch.float64)
+    x = x * torch.pow(2.0, torch.randint(-90, 20, (M, K), generator=g).double())
+    return x.float()
+
+
+@pytest.mark.parametrize("M,K,dtype,subln,kind", [
+    (16, 768, torch.float32, False, "outlier"),
+    (5, 3200, torch.bfloat16, False, "outlier"),
+    (3, 64, torch.float32, False, "normal"),
+    (2, 32768, torch.float32, False, "normal"),
+    (2, 32768, torch.bfloat16, True, "normal"),
+    (4, 128, torch.float32, False, "tiny"),
+    (33, 2560, torch.bfloat16, True, "normal"),
+    (4, 9728, torch.float32, True, "normal"),
+    (6, 1024, torch.float32, True, "wide"),
+    (7, 9728, torch.bfloat16, True, "student"),
+])
+def test_quant_act(M, K, dtype, subln, kind):
+    if kind == "outlier":
+        X = workloads.with_outlier_channels(workloads.normal((M, K), 1.0, 7, dtype), max(1, K // 100), 30.0, 8)
+    elif kind == "normal":
+        X = workloads.normal((M, K), 1.0, 9, dtype)
+    elif kind == "student":
+        X = workloads.student_t((M, K), 3, 0.5, 10, dtype)
+    elif kind == "wide":
+        X = _wide_rows(M, K, 11).to(dtype)
+    else:  # rows below the 1e-5 floor, and an all-zero row
+        X = (workloads.normal((M, K), 1.0, 12) * 1e-7).to(dtype)
+        X[1] = 0
+    gain = workloads.uniform((K,), 0.9, 1.1, 13) if subln else None
+    x_q, s = api.bl_quant_act(X.cuda(), None if gain is None else gain.cuda(), 1e-6)
+    torch.cuda.synchronize()
+    check_act(X, x_q, s, gain)
+
+
+# -- steps 3 + 4 -------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K", [
+    (1, 2048, 768), (3, 37, 192), (8, 2048, 768), (16, 300, 3200), (1, 8640, 3200),
+    (4, 3200, 8640), (1, 17, 64), (16, 64, 6144), (2, 33, 32768),
+    (17, 300, 1536), (100, 37, 4096), (257, 130, 768), (64, 256, 64),
+])
+def test_forward(M, N, K):
+    W = workloads.normal((N, K), 0.02, 200 + K)
+    X = workloads.with_outlier_channels(workloads.normal((M, K), 1.0, 300 + M, torch.bfloat16), 2, 20.0, 4)
+    packed, gamma, x_q, s, Y, acc = chain(W, X)
+    wq_ref, g_ref = check_weights(W, packed, gamma)
+    xq_ref, s_ref = check_act(X, x_q, s)
+    check_forward_full(xq_ref, s_ref, wq_ref, g_ref, Y, acc)
+
+
+def test_forward_without_acc_and_zero_rows():
+    M, N, K = 9, 50, 256
+    W = workloads.normal((N, K), 0.02, 1)
+    X = workloads.normal((M, K), 1.0, 2)
+    X[3] = 0
+    packed, gamma, x_q, s, Y, acc = chain(W, X)
+    wq_ref, g_ref = check_weights(W, packed, gamma)
+    xq_ref, s_ref = check_act(X, x_q, s)
+    check_forward_full(xq_ref, s_ref, wq_ref, g_ref, Y, acc)
+    Y2 = api.bl_forward(packed, gamma, x_q, s, N)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
+    assert torch.all(Y[3] == 0)
+
+
+# -- grouped decode: every projection of the 125M decode workload -----------
+
+@pytest.mark.parametrize("M", [1, 4, 8])
+def test_grouped_decode_125m(M):
+    items = workloads.decode125m(M=M)
+    dev, probs, refs = [], [], []
+    for name, W, X in items:
+        packed, gamma = gpu_quant_weights(W)
+        x_q, s = api.bl_quant_act(X.cuda())
+        N, K = W.shape
+        Y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+        acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
+        dev.append((packed, gamma, x_q, s, Y, acc, N, K))
+        refs.append((W, X))
+    arr = api.make_problems(dev)
+    api.bl_forward_grouped(arr, len(dev), M)
+    api.bl_check_device_error()
+    for (packed, gamma, x_q, s, Y, acc, N, K), (W, X) in zip(dev, refs):
+        wq_ref, g_ref = check_weights(W, packed, gamma)
+        xq_ref, s_ref = check_act(X, x_q, s)
+        check_forward_full(xq_ref, s_ref, wq_ref, g_ref, Y, acc)
+
+
+def test_grouped_act_quant_matches_single():
+    items = workloads.decode125m(M=4, layers=1)
+    dev = []
+    for name, W, X in items:
+        Xd = X.cuda()
+        dev.append((Xd, None, torch.empty_like(Xd, dtype=torch.int8), torch.empty(4, device="cuda")))
+    api.bl_quant_act_grouped(dev, torch.bfloat16)
+    torch.cuda.synchronize()
+    for (Xd, _, xq, s), (name, W, X) in zip(dev, items):
+        check_act(X, xq, s)
+
+
+# -- fused bl_linear -----------------------------------------------------------
+
+def test_linear_single_workload():
+    W, X = workloads.single()
+    Y = api.bl_linear(W.cuda(), X.cuda())
+    torch.cuda.synchronize()
+    ref = oracle.linear(np32(W), np32(X))
+    err = np.abs(Y.cpu().numpy().astype(np.float64) - ref["Y"])
+    assert np.all(err <= 1e-6 * np.abs(ref["Y"]))
+
+
+def test_linear_subln_qat4b_oproj_small():
+    name, W, X, gain = workloads.qat4b(M=96, which=("o",))[0]
+    Y = api.bl_linear(W.cuda(), X.cuda(), gain.cuda(), workloads.SUBLN_EPS)
+    torch.cuda.synchronize()
+    ref = oracle.linear(np32(W), np32(X), np32(gain), workloads.SUBLN_EPS)
+    err = np.abs(Y.cpu().numpy().astype(np.float64) - ref["Y"])
+    assert np.all(err <= 1e-6 * np.abs(ref["Y"]))
