@@ -107,6 +107,29 @@ bl_status bl_quant_weights(const void *W, bl_dtype wdt, int64_t N, int64_t K,
                            uint8_t *packed, float *gamma,
                            void *workspace, size_t workspace_bytes, bl_stream_t stream);
 
+/* Same computation and outputs as bl_quant_weights, for callers that cannot
+ * allocate device memory: a plain C host or a runtime that only hands out
+ * pointers to tensors it owns, or a program whose device-memory budget is
+ * fixed at start-up.  The scratch the reduction needs lives in a static
+ * device array inside the library (BL_NOALLOC_SCRATCH_BYTES bytes on every
+ * GPU that loads the library, held until process exit); this call never
+ * calls cudaMalloc or cudaFree.  No source page has a counterpart: this is
+ * an interface convenience of this library.
+ *   - Limits: those of bl_quant_weights (N*K < 2^31, K % 64 == 0,
+ *     64 <= K <= 32768); the fixed scratch covers every such size.  Other
+ *     sizes return BL_ERR_SHAPE.
+ *   - The first call on each device looks up the device address of the
+ *     static scratch (cudaGetSymbolAddress) with that device current; make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one scratch array and it keeps the
+ *     previous call's contents (the kernels overwrite every word they read,
+ *     so nothing needs clearing).  Calls whose kernels overlap on the GPU --
+ *     different streams, or different host threads -- race on it: serialize
+ *     them (one stream, or events). */
+#define BL_NOALLOC_SCRATCH_BYTES 49408
+bl_status bl_quant_weights_noalloc(const void *W, bl_dtype wdt, int64_t N, int64_t K,
+                                   uint8_t *packed, float *gamma, bl_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Step 2: per-token absmax INT8 activation quantization, optionally fused  */
 /* with a preceding SubLN RMSNorm.                                           */

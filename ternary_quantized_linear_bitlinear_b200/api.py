@@ -51,6 +51,7 @@ _SIGS = {
     "bl_check_device_error": (_int, [_p]),
     "bl_quant_weights_workspace_bytes": (_sz, [_i64, _i64]),
     "bl_quant_weights": (_int, [_p, _int, _i64, _i64, _p, _p, _p, _sz, _p]),
+    "bl_quant_weights_noalloc": (_int, [_p, _int, _i64, _i64, _p, _p, _p]),
     "bl_quant_act": (_int, [_p, _int, _i64, _i64, _p, _f32, _p, _p, _p]),
     "bl_forward": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
     "bl_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
@@ -136,6 +137,23 @@ def bl_quant_weights(W: torch.Tensor, packed=None, gamma=None, workspace=None, s
     rc = lib().bl_quant_weights(W.data_ptr(), _DTYPES.get(W.dtype, -1), N, K, packed.data_ptr(), gamma.data_ptr(),
                                 workspace.data_ptr(), workspace.numel(), _stream(stream))
     _check(rc, "bl_quant_weights")
+    return packed, gamma
+
+
+def bl_quant_weights_noalloc(W: torch.Tensor, packed=None, gamma=None, stream=None):
+    """bl_quant_weights without a workspace argument: the library's static
+    device scratch is used instead (for callers that cannot allocate device
+    memory; see include/bitlinear.h).  Outputs are allocated here only when
+    the caller passes none."""
+    _dev(W, "W")
+    N, K = W.shape
+    if packed is None:
+        packed = torch.empty(N, K // 4, dtype=torch.uint8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(4, dtype=torch.float32, device=W.device)[:1]
+    rc = lib().bl_quant_weights_noalloc(W.data_ptr(), _DTYPES.get(W.dtype, -1), N, K, packed.data_ptr(),
+                                        gamma.data_ptr(), _stream(stream))
+    _check(rc, "bl_quant_weights_noalloc")
     return packed, gamma
 
 

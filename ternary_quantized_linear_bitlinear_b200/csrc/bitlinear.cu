@@ -347,3 +347,51 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt, in
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Weight quantization without caller-provided scratch (see the header): the
+// reduction's per-block partials and the threshold word live in this static
+// array.  Host code must not hand the symbol itself to a kernel -- in host
+// code it names a host-side stand-in -- so the device address is looked up
+// once per device with cudaGetSymbolAddress.
+
+namespace {
+
+static_assert(WQ_WS_BYTES <= BL_NOALLOC_SCRATCH_BYTES, "static weight-quant scratch too small");
+static __device__ __align__(256) unsigned char g_noalloc_scratch[BL_NOALLOC_SCRATCH_BYTES];
+
+void *g_noalloc_ptr[MAX_DEVICES];
+std::mutex g_noalloc_mu;
+
+// Device address of g_noalloc_scratch on the current device (set up on the
+// first call per device, with that device current).
+bl_status noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return BL_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return BL_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return BL_OK;
+}
+
+}  // namespace
+
+extern "C" bl_status bl_quant_weights_noalloc(const void *W, bl_dtype wdt, int64_t N, int64_t K, uint8_t *packed,
+                                              float *gamma, bl_stream_t stream) {
+    if (!W || !packed || !gamma) return BL_ERR_NULL;
+    if (wdt != BL_F32 && wdt != BL_BF16) return BL_ERR_DTYPE;
+    if (N < 1 || check_k(K) != BL_OK || N * K >= (1LL << 31)) return BL_ERR_SHAPE;
+    if (!aligned16(W) || !aligned16(packed) || !aligned16(gamma)) return BL_ERR_ALIGN;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    void *scratch = nullptr;
+    rc = noalloc_scratch(&scratch);
+    if (rc) return rc;
+    return quant_weights_impl(*d, W, wdt, N, K, packed, gamma, scratch, (cudaStream_t)stream);
+}
+
