@@ -46,6 +46,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--mode", default="all", choices=["all", "decode", "prefill"],
+                    help="decode: the headline decode workload only; prefill: only the prefill measurement")
     return ap.parse_args()
 
 
@@ -228,7 +230,7 @@ def native(args, rank, world, local):
                 rc = L.bl_quant_act_grouped(acts[M], count, api.BL_BF16, M, 1e-6, stream_ptr)
                 if rc:
                     raise api.BitLinearError(rc, "bl_quant_act_grouped")
-            rc = L.bl_forward_grouped(fwds[(M, rep)], count, M, stream_ptr)
+            rc = L.bl_forward_grouped(fwds[(M, rep)], count, M, api.BL_FWD_WEIGHTS_READY, stream_ptr)
             if rc:
                 raise api.BitLinearError(rc, "bl_forward_grouped")
 
@@ -346,6 +348,78 @@ def native(args, rank, world, local):
     return out
 
 
+def prefill(args, dev):
+    """Prefill engine on the 1.4B-shape layer (7 projections, M = 8192 tokens):
+    int8 TOPS of the contraction (2*M*N*K per projection) for the engine alone
+    (bl_forward on pre-quantized inputs) and for the whole per-call path
+    (bl_linear: weight quant + act quant + GEMM + rescale)."""
+    from ternary_quantized_linear_bitlinear_b200 import api
+
+    items = workloads.prefill1b4()
+    M = workloads.PREFILL1B4["tokens"]
+    ops = sum(2 * M * W.shape[0] * W.shape[1] for _, W, _ in items)
+    dev_items = []
+    for name, W, X in items:
+        Wd, Xd = W.to(dev), X.to(dev)
+        packed, gamma = api.bl_quant_weights(Wd)
+        x_q, s = api.bl_quant_act(Xd)
+        N, K = W.shape
+        Y = torch.empty(M, N, dtype=torch.float32, device=dev)
+        ws = torch.empty(api.linear_workspace_bytes(M, N, K), dtype=torch.uint8, device=dev)
+        dev_items.append((Wd, Xd, packed, gamma, x_q, s, Y, ws))
+    L = api.lib()
+    stream = torch.cuda.Stream(device=dev)
+    sp = stream.cuda_stream
+
+    def engine():
+        for (Wd, Xd, packed, gamma, x_q, s, Y, ws) in dev_items:
+            rc = L.bl_forward(packed.data_ptr(), gamma.data_ptr(), x_q.data_ptr(), s.data_ptr(), x_q.shape[0],
+                              Y.shape[1], x_q.shape[1], Y.data_ptr(), None, sp)
+            if rc:
+                raise api.BitLinearError(rc, "bl_forward")
+
+    def whole():
+        for (Wd, Xd, packed, gamma, x_q, s, Y, ws) in dev_items:
+            rc = L.bl_linear(Wd.data_ptr(), api.BL_BF16, Xd.data_ptr(), api.BL_BF16, Xd.shape[0], Wd.shape[0],
+                             Wd.shape[1], None, 1e-6, ws.data_ptr(), ws.numel(), Y.data_ptr(), sp)
+            if rc:
+                raise api.BitLinearError(rc, "bl_linear")
+
+    out = {}
+    reps = max(3, min(args.steps, 20))
+    for label, fn in (("engine", engine), ("per_call_quant", whole)):
+        with torch.cuda.stream(stream):
+            for _ in range(max(3, args.warmup if args.warmup < 10 else 3)):
+                fn()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                fn()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        out[label] = {"ms_per_layer": round(ms, 4), "tops": round(ops / (ms * 1e-3) / 1e12, 1)}
+    api.bl_check_device_error(stream)
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+    except (OSError, ValueError):
+        pass
+    # int8 dense peak = measured bf16 dense peak x the nominal int8:bf16 ratio (4.5 : 2.25)
+    bf16 = float(peaks.get("bf16_tflops", 1590.0))
+    peak = 2.0 * bf16
+    return {"workload": "prefill1b4: hidden 1536, FFN 4096, q,o 1536^2, k,v 512x1536, gate,up 4096x1536, "
+                        "down 1536x4096, M = 8192", "ops_per_layer": ops,
+            "engine": out["engine"], "per_call_quant": out["per_call_quant"],
+            "roofline": {"bound": "tensor", "kernel": "k_prefill_tc", "achieved": out["engine"]["tops"],
+                         "peak": round(peak, 1), "unit": "TOPS",
+                         "peak_source": ("measured bf16 x 2 (nominal int8:bf16)" if "bf16_tflops" in peaks
+                                         else "fallback bf16 x 2"),
+                         "frac": round(out["engine"]["tops"] / peak, 4)},
+            "reps": reps, "l2": "inputs and outputs of the layer total > 700 MB"}
+
+
 def cpu_oracle_step(items_q, wbytes, xbytes):
     """One step of the decode workload on the CPU oracle; returns seconds."""
     import oracle
@@ -428,8 +502,13 @@ def main():
     try:
         if args.impl == "reference":
             out = reference(args, rank, world)
+        elif args.mode == "prefill":
+            dev = torch.device("cuda", torch.cuda.current_device())
+            out = {"mode": "prefill", "prefill": prefill(args, dev)}
         else:
             out = native(args, rank, world, local)
+            if args.mode == "all" and rank == 0:
+                out["prefill"] = prefill(args, torch.device("cuda", torch.cuda.current_device()))
             if rank == 0 and world == 1 and not args.no_cpu_baseline:
                 out["cpu_baseline"] = cpu_baseline()
         if rank == 0 and out is not None:

@@ -165,7 +165,8 @@ bl_status bl_quant_act(const void *X, bl_dtype xdt, int64_t M, int64_t K,
 /*   Y[m, n]   = float(float(acc) * float(gamma / s[m]))                     */
 /*               (two float roundings: |Y - acc*gamma/s| <= 2^-23 |Y|)       */
 /*                                                                           */
-/* Engine: M <= 16 and M*K <= 96 KiB -> bandwidth-bound decode GEMV;         */
+/* Engine: the bandwidth-bound decode GEMV when M <= 16 and its shared-     */
+/* memory staging fits (every M <= 16 for K <= 9728; M <= 2 at K = 32768),   */
 /* otherwise the tcgen05 prefill GEMM.  Both give identical acc.             */
 /* packed [N, K/4] (format above); gamma [1]; x_q [M, K]; s [M]; Y [M, N]    */
 /* out; acc_out [M, N] int32 out or NULL.  All device.                       */
@@ -188,10 +189,17 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt,
 /* ------------------------------------------------------------------------ */
 /* Grouped decode: up to BL_MAX_GROUP independent steps-3+4 problems that    */
 /* share M, in ONE kernel launch (e.g. every projection of a decode step).   */
-/* Same arithmetic as bl_forward; requires M <= 16 and M*K <= 96 KiB for    */
-/* each problem.  `problems` is a HOST array, read during the call only.     */
+/* Same arithmetic as bl_forward; every problem must be decode-eligible      */
+/* (M <= 16 and the staging fits, see bl_forward), else BL_ERR_SHAPE.        */
+/* `problems` is a HOST array, read during the call only.                    */
+/* flags: 0, or BL_FWD_WEIGHTS_READY -- the caller promises that every       */
+/* problem's packed weights and gamma were complete before the kernel        */
+/* enqueued just before this call began; the engine may then be launched as */
+/* a programmatic dependent launch that streams weights while that kernel    */
+/* finishes (it still waits for it before reading x_q and s).                */
 /* ------------------------------------------------------------------------ */
 #define BL_MAX_GROUP 128
+#define BL_FWD_WEIGHTS_READY 1u
 
 typedef struct {
     const uint8_t *packed;  /* [N, K/4] */
@@ -204,7 +212,7 @@ typedef struct {
     int64_t K;
 } bl_problem;
 
-bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M,
+bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, unsigned flags,
                              bl_stream_t stream);
 
 /* Grouped step 2: up to BL_MAX_GROUP activation inputs sharing M and dtype,

@@ -19,6 +19,7 @@ _LIB = None
 
 BL_F32, BL_BF16 = 0, 1
 BL_MAX_GROUP = 128
+BL_FWD_WEIGHTS_READY = 1
 _DTYPES = {torch.float32: BL_F32, torch.bfloat16: BL_BF16}
 
 _i64 = ctypes.c_int64
@@ -56,7 +57,9 @@ _SIGS = {
     "bl_forward": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
     "bl_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_linear": (_int, [_p, _int, _p, _int, _i64, _i64, _i64, _p, _f32, _p, _sz, _p, _p]),
-    "bl_forward_grouped": (_int, [ctypes.POINTER(Problem), _int, _i64, _p]),
+    "bl_forward_grouped": (_int, [ctypes.POINTER(Problem), _int, _i64, ctypes.c_uint, _p]),
+    "bl_debug_forward_prefill": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, ctypes.c_longlong,
+                                        ctypes.c_uint32, _p]),
     "bl_quant_act_grouped": (_int, [ctypes.POINTER(ActProblem), _int, _int, _i64, _f32, _p]),
 }
 
@@ -207,9 +210,9 @@ def make_problems(items):
     return arr
 
 
-def bl_forward_grouped(problems, count: int, M: int, stream=None):
+def bl_forward_grouped(problems, count: int, M: int, flags: int = 0, stream=None):
     """problems: ctypes array from make_problems (built once, launched many times)."""
-    rc = lib().bl_forward_grouped(problems, count, M, _stream(stream))
+    rc = lib().bl_forward_grouped(problems, count, M, flags, _stream(stream))
     _check(rc, "bl_forward_grouped")
 
 
@@ -229,6 +232,20 @@ def bl_linear(W, X, subln_gain=None, subln_eps: float = 1e-6, Y=None, workspace=
                          _ptr(subln_gain), subln_eps, workspace.data_ptr(), workspace.numel(), Y.data_ptr(),
                          _stream(stream))
     _check(rc, "bl_linear")
+    return Y
+
+
+def bl_debug_forward_prefill(packed, gamma, x_q, s, N: int, Y=None, acc_out=None, skip_iter: int = -1,
+                             timeout_us: int = 2_000_000, stream=None):
+    """Test hook (include/bitlinear_debug.h): bl_forward forced through the
+    tcgen05 prefill engine, with bounded waits of timeout_us and an optional
+    stalled k-iteration."""
+    M, K = x_q.shape
+    if Y is None:
+        Y = torch.empty(M, N, dtype=torch.float32, device=x_q.device)
+    rc = lib().bl_debug_forward_prefill(packed.data_ptr(), gamma.data_ptr(), x_q.data_ptr(), s.data_ptr(), M, N, K,
+                                        Y.data_ptr(), _ptr(acc_out), skip_iter, timeout_us, _stream(stream))
+    _check(rc, "bl_debug_forward_prefill")
     return Y
 
 

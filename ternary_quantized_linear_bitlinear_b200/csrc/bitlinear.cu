@@ -8,10 +8,11 @@
 #include <mutex>
 
 #include "bitlinear.h"
+#include "bitlinear_debug.h"
 #include "bl_common.cuh"
 #include "k_act_quant.cuh"
 #include "k_decode.cuh"
-#include "k_prefill.cuh"
+#include "k_prefill_tc.cuh"
 #include "k_weight_quant.cuh"
 
 using namespace bl;
@@ -46,9 +47,9 @@ bl_status device_info(DeviceInfo **out) {
             // opt in to large dynamic shared memory once per device
             bool fail = false;
             fail |= cudaFuncSetAttribute(k_decode<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         DEC_MAX_XQ_SMEM) != cudaSuccess;
+                                         DEC_SMEM_LIMIT) != cudaSuccess;
             fail |= cudaFuncSetAttribute(k_decode<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         DEC_MAX_XQ_SMEM) != cudaSuccess;
+                                         DEC_SMEM_LIMIT) != cudaSuccess;
             fail |= prefill_setup() != cudaSuccess;
             if (fail) return BL_ERR_CUDA;
         }
@@ -114,6 +115,29 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
     const bool bf16 = xdt == BL_BF16;
     const int epv = bf16 ? 8 : 4;
     const long long nvec = Kmax / epv;
+    bool subln = false;
+    for (int i = 0; i < P.count; ++i) subln |= P.p[i].gain != nullptr;
+    if (!subln && nvec <= 8 * 32) {
+        // short rows: one warp per row
+        int vpl = 1;
+        while (vpl * 32 < nvec) vpl *= 2;
+        const long long rows = (long long)P.count * P.M;
+        const unsigned grid = (unsigned)((rows + AQW_WARPS - 1) / AQW_WARPS);
+#define BL_AQW_CASE(B, V)                                                         \
+        if (bf16 == B && vpl == V) {                                              \
+            k_act_quant_warp<B, V><<<grid, AQW_WARPS * 32, 0, st>>>(P);           \
+            return launch_status();                                               \
+        }
+        BL_AQW_CASE(true, 1)
+        BL_AQW_CASE(true, 2)
+        BL_AQW_CASE(true, 4)
+        BL_AQW_CASE(true, 8)
+        BL_AQW_CASE(false, 1)
+        BL_AQW_CASE(false, 2)
+        BL_AQW_CASE(false, 4)
+        BL_AQW_CASE(false, 8)
+#undef BL_AQW_CASE
+    }
     int vec = 1;
     while ((nvec + vec - 1) / vec > 1024) vec *= 2;
     int T = (int)(((nvec + vec - 1) / vec + 31) / 32 * 32);
@@ -138,47 +162,54 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
 // ---------------------------------------------------------------------------
 // Steps 3 + 4
 
-int decode_glog(int64_t K) {
-    int steps = (int)((K + 255) / 256);
-    if (steps <= 3) return 0;
-    if (steps <= 6) return 1;
-    if (steps <= 12) return 2;
-    return 3;
+int dec_xq_off(int64_t K) { return (dec_w_bytes((int)K) + 127) & ~127; }
+
+bool decode_eligible(int64_t M, int64_t K) {
+    return M <= 16 && dec_xq_off(K) + M * dec_row_stride((int)K) <= DEC_SMEM_LIMIT;
 }
 
-bool decode_eligible(int64_t M, int64_t K) { return M <= 16 && M * dec_row_stride((int)K) <= DEC_MAX_XQ_SMEM; }
-
-bl_status decode_launch(DecodeParams &P, cudaStream_t st) {
+bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st) {
     int total = 0;
-    int rs_max = 0;
+    int rs_max = 0, xq_off = 0;
     for (int i = 0; i < P.count; ++i) {
         DecodeProblem &q = P.p[i];
-        q.g_log2 = decode_glog(q.K);
+        q.g_log2 = dec_glog(q.K);
         int tiles = (q.N + 15) / 16;
         int per = DEC_WARPS >> q.g_log2;
         q.cta_begin = total;
         total += (tiles + per - 1) / per;
         int rs = dec_row_stride(q.K);
         rs_max = rs > rs_max ? rs : rs_max;
+        int xo = dec_xq_off(q.K);
+        xq_off = xo > xq_off ? xo : xq_off;
     }
-    size_t smem = (size_t)P.M * rs_max;
-    if (P.M <= 8)
-        k_decode<1><<<total, DEC_THREADS, smem, st>>>(P);
-    else
-        k_decode<2><<<total, DEC_THREADS, smem, st>>>(P);
-    return launch_status();
+    P.xq_off = xq_off;
+    const size_t smem = (size_t)xq_off + (size_t)P.M * rs_max;
+    if (smem > DEC_SMEM_LIMIT) return BL_ERR_SHAPE;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)total);
+    cfg.blockDim = dim3(DEC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t e = P.M <= 8 ? cudaLaunchKernelEx(&cfg, k_decode<1>, P) : cudaLaunchKernelEx(&cfg, k_decode<2>, P);
+    return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 
-bl_status forward_impl(const uint8_t *packed, const float *gamma, const int8_t *x_q, const float *s,
-                       int64_t M, int64_t N, int64_t K, float *Y, int32_t *acc_out, cudaStream_t st) {
+bl_status forward_impl(const DeviceInfo &d, const uint8_t *packed, const float *gamma, const int8_t *x_q,
+                       const float *s, int64_t M, int64_t N, int64_t K, float *Y, int32_t *acc_out, cudaStream_t st) {
     if (decode_eligible(M, K)) {
         DecodeParams P;
         P.count = 1;
         P.M = (int)M;
         P.p[0] = DecodeProblem{packed, gamma, x_q, s, Y, acc_out, (int)N, (int)K, 0, 0};
-        return decode_launch(P, st);
+        return decode_launch(P, false, st);
     }
-    return prefill_launch(packed, gamma, x_q, s, M, N, K, Y, acc_out, st);
+    return prefill_launch(d.sms, packed, gamma, x_q, s, M, N, K, Y, acc_out, st);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -276,10 +307,11 @@ bl_status bl_forward(const uint8_t *packed, const float *gamma, const int8_t *x_
     DeviceInfo *d;
     bl_status rc = device_info(&d);
     if (rc) return rc;
-    return forward_impl(packed, gamma, x_q, s, M, N, K, Y, acc_out, (cudaStream_t)stream);
+    return forward_impl(*d, packed, gamma, x_q, s, M, N, K, Y, acc_out, (cudaStream_t)stream);
 }
 
-bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, bl_stream_t stream) {
+bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, unsigned flags,
+                             bl_stream_t stream) {
     if (!problems) return BL_ERR_NULL;
     if (count < 1 || count > BL_MAX_GROUP || M < 1 || M > 16) return BL_ERR_SHAPE;
     DecodeParams P;
@@ -300,7 +332,7 @@ bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, b
     DeviceInfo *d;
     bl_status rc = device_info(&d);
     if (rc) return rc;
-    return decode_launch(P, (cudaStream_t)stream);
+    return decode_launch(P, (flags & BL_FWD_WEIGHTS_READY) != 0, (cudaStream_t)stream);
 }
 
 size_t bl_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -343,7 +375,7 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt, in
     P.p[0] = ActProblem{X, subln_gain, x_q, s, (int)K, 0};
     rc = quant_act_impl(P, xdt, K, st);
     if (rc) return rc;
-    return forward_impl(packed, gamma, x_q, s, M, N, K, Y, nullptr, st);
+    return forward_impl(*d, packed, gamma, x_q, s, M, N, K, Y, nullptr, st);
 }
 
 }  // extern "C"
@@ -395,3 +427,19 @@ extern "C" bl_status bl_quant_weights_noalloc(const void *W, bl_dtype wdt, int64
     return quant_weights_impl(*d, W, wdt, N, K, packed, gamma, scratch, (cudaStream_t)stream);
 }
 
+extern "C" bl_status bl_debug_forward_prefill(const uint8_t *packed, const float *gamma, const int8_t *x_q,
+                                              const float *s, int64_t M, int64_t N, int64_t K, float *Y,
+                                              int32_t *acc_out, long long skip_iter, uint32_t timeout_us,
+                                              bl_stream_t stream) {
+    if (!packed || !gamma || !x_q || !s || !Y) return BL_ERR_NULL;
+    if (M < 1 || N < 1 || M > 0x7fffffffLL || N > 0x7fffffffLL || check_k(K) != BL_OK || timeout_us == 0)
+        return BL_ERR_SHAPE;
+    if (!aligned16(packed) || !aligned16(gamma) || !aligned16(x_q) || !aligned16(s) || !aligned16(Y) ||
+        (acc_out && !aligned16(acc_out)))
+        return BL_ERR_ALIGN;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return prefill_launch(d->sms, packed, gamma, x_q, s, M, N, K, Y, acc_out, (cudaStream_t)stream,
+                          (unsigned long long)timeout_us * 1000ull, skip_iter < 0 ? -1 : skip_iter);
+}

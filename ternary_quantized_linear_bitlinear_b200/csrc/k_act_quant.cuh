@@ -61,6 +61,9 @@ __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ A
     __shared__ u64 s_lo[32], s_hi[32];
     __shared__ float s_r;
 
+    // let a programmatically dependent launch (the GEMV) start streaming its
+    // weights; it waits for this grid to finish before it reads x_q
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int pi = blockIdx.x / P.M;
     const int m = blockIdx.x - pi * P.M;
     const ActProblem &pr = P.p[pi];
@@ -167,6 +170,64 @@ __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ A
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 int qi = __float2int_rn(__fmul_rn(x[v * EPV + q * 4 + j], s));
+                qi = max(-128, min(127, qi));
+                word |= ((u32)qi & 0xffu) << (8 * j);
+            }
+            out[q] = word;
+        }
+        if (BF16) {
+            *reinterpret_cast<uint2 *>(qr + (size_t)vi * 8) = make_uint2(out[0], out[EPV / 4 - 1]);
+        } else {
+            *reinterpret_cast<u32 *>(qr + (size_t)vi * 4) = out[0];
+        }
+    }
+}
+
+// One warp per row, no SubLN (short rows): VPL 16-byte vectors per lane, the
+// row in registers, absmax by a warp reduction -- no block barrier at all.
+constexpr int AQW_WARPS = 8;
+
+template <bool BF16, int VPL>
+__global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_constant__ ActParams P) {
+    constexpr int EPV = BF16 ? 8 : 4;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int gw = blockIdx.x * AQW_WARPS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (gw >= P.count * P.M) return;
+    const int pi = gw / P.M, m = gw - pi * P.M;
+    const ActProblem &pr = P.p[pi];
+    const int K = pr.K, nvec = K / EPV;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(pr.X) + (size_t)m * nvec;
+    uint4 raw[VPL];
+    u32 amax = 0;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        const int vi = lane + v * 32;
+        raw[v] = vi < nvec ? ldg_stream_v4(xr + vi) : make_uint4(0, 0, 0, 0);
+        const u32 w4[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) {
+            u32 bits = BF16 ? ((j & 1) ? (w4[j >> 1] & 0xffff0000u) : (w4[j >> 1] << 16)) : w4[j];
+            amax = max(amax, bits & 0x7fffffffu);
+        }
+    }
+    amax = warp_max_u32(amax);
+    const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(amax), 1e-5f));
+    if (lane == 0) pr.s[m] = s;
+    int8_t *qr = pr.xq + (size_t)m * K;
+#pragma unroll
+    for (int v = 0; v < VPL; ++v) {
+        const int vi = lane + v * 32;
+        if (vi >= nvec) continue;
+        const u32 w4[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
+        u32 out[EPV / 4];
+#pragma unroll
+        for (int q = 0; q < EPV / 4; ++q) {
+            u32 word = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int e = q * 4 + j;
+                u32 bits = BF16 ? ((e & 1) ? (w4[e >> 1] & 0xffff0000u) : (w4[e >> 1] << 16)) : w4[e];
+                int qi = __float2int_rn(__fmul_rn(__uint_as_float(bits), s));
                 qi = max(-128, min(127, qi));
                 word |= ((u32)qi & 0xffu) << (8 * j);
             }

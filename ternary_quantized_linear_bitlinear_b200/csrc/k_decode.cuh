@@ -5,11 +5,13 @@
 //
 // The work is bound by streaming the packed weights from HBM (2 bits per
 // weight).  Design:
-//   - A warp owns a 16-row tile of W; a CTA (8 warps) owns 8/G tiles, with G
-//     warps splitting each tile's K range (G picked per problem from K).
-//   - Each thread streams 16 bytes of row g and 16 bytes of row g+8 per
-//     256-k step with 128-bit non-caching loads; lanes of a quad read one
-//     contiguous 64-byte run of a row.
+//   - A CTA (8 warps) owns T = 8/G consecutive 16-row tiles of one problem;
+//     their packed rows are one contiguous byte range, which one thread
+//     requests with cp.async.bulk copies into shared memory (completion on an
+//     mbarrier, bounded wait), so the memory system sees a few large requests
+//     per CTA and the warps issue no global loads for weights.
+//   - A warp owns a 16-row tile; G warps split its K range (G picked per
+//     problem from K so that each warp has at most 4 steps of 256 k).
 //   - Unpacking costs 1-2 ALU ops per 4 weights: with the packed layout, word
 //     (w << (6 - 2j)) & 0xC0C0C0C0 puts the codes of k = 16w' + 4j .. 4j+3 in
 //     the top two bits of four bytes, i.e. the int8 values 64 * W_q.
@@ -32,7 +34,9 @@ namespace bl {
 
 constexpr int DEC_THREADS = 256;
 constexpr int DEC_WARPS = DEC_THREADS / 32;
-constexpr int DEC_MAX_XQ_SMEM = 96 * 1024;
+constexpr int DEC_SMEM_LIMIT = 200 * 1024;  // weight tiles + staged x_q, per CTA
+constexpr int DEC_PF = 4;                   // target 256-k steps per warp (G is chosen from it)
+constexpr unsigned long long DEC_TIMEOUT_NS = 2000000000ull;
 
 struct DecodeProblem {
     const uint8_t *packed;
@@ -51,14 +55,20 @@ struct DecodeParams {
     DecodeProblem p[BL_MAX_GROUP];
     int count;
     int M;
+    int xq_off;  // shared-memory offset of the staged x_q (after the weight tiles)
 };
 
 __host__ __device__ inline int dec_row_stride(int K) { return (K + 255) & ~255; }
 
-__device__ __forceinline__ int dec_swz_chunk(int L, int row) {
-    int x = (((L >> 3) & 1) << 1) | (row & 1);
-    return (L & ~7) | ((L ^ x) & 7);
+__host__ __device__ inline int dec_glog(int K) {
+    // smallest G = 2^glog <= 8 with ceil(steps / G) <= DEC_PF
+    int steps = (K + 255) >> 8, g = 0;
+    while (g < 3 && ((steps + (1 << g) - 1) >> g) > DEC_PF) ++g;
+    return g;
 }
+
+// bytes of packed weights one CTA stages
+__host__ __device__ inline int dec_w_bytes(int K) { return (DEC_WARPS >> dec_glog(K)) * 16 * (K >> 2); }
 
 __device__ __forceinline__ u32 dec_unpack(u32 w, int j) {
     // codes of k = 4j .. 4j+3 of this 16-weight word -> int8 lanes holding 64 * W_q
@@ -76,41 +86,65 @@ __device__ __forceinline__ void mma_s8_16832(int (&c)[4], u32 a0, u32 a1, u32 a2
 // NT: 8-token column tiles (1: M <= 8, 2: M <= 16).
 template <int NT>
 __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ DecodeParams P) {
-    extern __shared__ __align__(16) uint8_t s_xq[];
+    extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_red[DEC_WARPS][NT][4][32];
+    __shared__ __align__(8) u64 s_bar;
 
+    // problem of this CTA: binary search over the CTA prefix
     const int b = blockIdx.x;
-    int pi = 0;
-    while (pi + 1 < P.count && P.p[pi + 1].cta_begin <= b) ++pi;
-    const DecodeProblem &pr = P.p[pi];
+    int lo = 0, hi = P.count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.p[mid].cta_begin <= b) lo = mid; else hi = mid - 1;
+    }
+    const DecodeProblem &pr = P.p[lo];
     const int M = P.M, N = pr.N, K = pr.K;
     const int glog = pr.g_log2, G = 1 << glog;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles_per_cta = DEC_WARPS >> glog;
-    const int tile = (b - pr.cta_begin) * tiles_per_cta + (warp >> glog);
-    const int kslot = warp & (G - 1);
-    const int row0 = tile * 16;
-    const int RS = dec_row_stride(K);
+    const int T = DEC_WARPS >> glog;
     const int Kw = K >> 2;         // packed bytes per row
-    const int nchunk64 = K >> 6;   // 64-k chunks (16 packed bytes each)
-    const int steps = (K + 255) >> 8;
+    const int row_base = (b - pr.cta_begin) * T * 16;
+    const int rows = min(T * 16, N - row_base);
+    const u32 bar = smem_u32(&s_bar);
+
+    // One thread requests the CTA's weight rows (contiguous bytes).
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        const u32 bytes = (u32)rows * (u32)Kw;
+        mbar_arrive_expect_tx(bar, bytes);
+        const uint8_t *src = pr.packed + (size_t)row_base * Kw;
+        const u32 dst = smem_u32(smem);
+        for (u32 off = 0; off < bytes; off += 32768u) {
+            const u32 n = bytes - off < 32768u ? bytes - off : 32768u;
+            bulk_g2s(dst + off, src + off, n, bar);
+        }
+    }
+
+    // x_q may be produced by the kernel launched just before this one.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 
     // Stage x_q rows [0, M) into shared memory, swizzled, zero-padded to RS.
+    const int RS = dec_row_stride(K);
+    uint8_t *s_xq = smem + P.xq_off;
     {
         const int chunks = RS >> 4;
-        for (int idx = threadIdx.x; idx < M * chunks; idx += DEC_THREADS) {
-            int r = idx / chunks, L = idx - r * chunks;
-            uint4 v = make_uint4(0, 0, 0, 0);
-            if (L * 16 < K) v = *reinterpret_cast<const uint4 *>(pr.xq + (size_t)r * K + L * 16);
-            *reinterpret_cast<uint4 *>(s_xq + r * RS + dec_swz_chunk(L, r) * 16) = v;
+        for (int r = 0; r < M; ++r) {
+            for (int L = threadIdx.x; L < chunks; L += DEC_THREADS) {
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (L * 16 < K) v = *reinterpret_cast<const uint4 *>(pr.xq + (size_t)r * K + L * 16);
+                const int x = (((L >> 3) & 1) << 1) | (r & 1);
+                *reinterpret_cast<uint4 *>(s_xq + r * RS + (((L & ~7) | ((L ^ x) & 7)) << 4)) = v;
+            }
         }
     }
     __syncthreads();
 
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const bool rowA = row0 + g < N, rowB = row0 + g + 8 < N;
-    const uint8_t *wA = pr.packed + (size_t)(row0 + g) * Kw;
-    const uint8_t *wB = pr.packed + (size_t)(row0 + g + 8) * Kw;
+    const int wt = warp >> glog, kslot = warp & (G - 1);
+    const int row0 = wt * 16;  // within the CTA
+    const int steps = (K + 255) >> 8;
+    const int nchunk64 = K >> 6;
 
     int acc[NT][4];
 #pragma unroll
@@ -118,41 +152,40 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
 #pragma unroll
         for (int i = 0; i < 4; ++i) acc[nt][i] = 0;
 
-    // token rows of the B fragments this lane reads
-    const int tr0 = g, tr1 = g + 8;
-    const bool tv0 = tr0 < M, tv1 = NT > 1 && tr1 < M;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0, DEC_TIMEOUT_NS, nullptr));
+    if (!ok && lane == 0) raise_device_error(DEVERR_TIMEOUT_PRODUCER);
 
-    for (int st = kslot; st < steps; st += 2 * G) {
-        // two steps in flight: st and st + G
-        uint4 a[2], bb[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            int s2 = st + u * G;
-            bool kv = s2 < steps && (s2 * 4 + t) < nchunk64;
-            a[u] = (rowA && kv) ? ldg_stream_v4(wA + s2 * 64 + t * 16) : make_uint4(0, 0, 0, 0);
-            bb[u] = (rowB && kv) ? ldg_stream_v4(wB + s2 * 64 + t * 16) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            int s2 = st + u * G;
-            if (s2 >= steps) break;
-            const u32 wa[4] = {a[u].x, a[u].y, a[u].z, a[u].w};
-            const u32 wb[4] = {bb[u].x, bb[u].y, bb[u].z, bb[u].w};
+    if (ok && row0 < rows) {
+        const uint8_t *wA = smem + (row0 + g) * Kw + t * 16;
+        const uint8_t *wB = smem + (row0 + g + 8) * Kw + t * 16;
+        // B fragments: token rows g (and g + 8); chunk c of a step sits at
+        // 16 * (4t + (c ^ xb)) within the step's 256 bytes (the swizzle)
+        const bool tv0 = g < M, tv1 = NT > 1 && g + 8 < M;
+        const int xb0 = ((t >> 1) << 1) | (g & 1);
+        const int xb1 = ((t >> 1) << 1) | ((g + 8) & 1);
+        const uint8_t *xr0 = s_xq + g * RS + t * 64;
+        const uint8_t *xr1 = s_xq + (g + 8) * RS + t * 64;
+#pragma unroll 4
+        for (int s2 = kslot; s2 < steps; s2 += G) {
+            const bool kv = (s2 * 4 + t) < nchunk64;
+            const uint4 va = kv ? *reinterpret_cast<const uint4 *>(wA + s2 * 64) : make_uint4(0, 0, 0, 0);
+            const uint4 vb = kv ? *reinterpret_cast<const uint4 *>(wB + s2 * 64) : make_uint4(0, 0, 0, 0);
+            const u32 wa[4] = {va.x, va.y, va.z, va.w};
+            const u32 wb[4] = {vb.x, vb.y, vb.z, vb.w};
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const int L = s2 * 16 + t * 4 + c;  // 16-byte chunk of x_q
-                uint4 x0 = tv0 ? *reinterpret_cast<const uint4 *>(s_xq + tr0 * RS + dec_swz_chunk(L, tr0) * 16)
-                               : make_uint4(0, 0, 0, 0);
+                const uint4 x0 = tv0 ? *reinterpret_cast<const uint4 *>(xr0 + s2 * 256 + ((c ^ xb0) << 4))
+                                     : make_uint4(0, 0, 0, 0);
                 uint4 x1 = make_uint4(0, 0, 0, 0);
-                if (NT > 1 && tv1) x1 = *reinterpret_cast<const uint4 *>(s_xq + tr1 * RS + dec_swz_chunk(L, tr1) * 16);
-                const u32 xb0[4] = {x0.x, x0.y, x0.z, x0.w};
-                const u32 xb1[4] = {x1.x, x1.y, x1.z, x1.w};
+                if (NT > 1 && tv1) x1 = *reinterpret_cast<const uint4 *>(xr1 + s2 * 256 + ((c ^ xb1) << 4));
+                const u32 xq0[4] = {x0.x, x0.y, x0.z, x0.w};
+                const u32 xq1[4] = {x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    u32 a0 = dec_unpack(wa[c], 2 * h), a2 = dec_unpack(wa[c], 2 * h + 1);
-                    u32 a1 = dec_unpack(wb[c], 2 * h), a3 = dec_unpack(wb[c], 2 * h + 1);
-                    mma_s8_16832(acc[0], a0, a1, a2, a3, xb0[2 * h], xb0[2 * h + 1]);
-                    if (NT > 1) mma_s8_16832(acc[NT - 1], a0, a1, a2, a3, xb1[2 * h], xb1[2 * h + 1]);
+                    const u32 a0 = dec_unpack(wa[c], 2 * h), a2 = dec_unpack(wa[c], 2 * h + 1);
+                    const u32 a1 = dec_unpack(wb[c], 2 * h), a3 = dec_unpack(wb[c], 2 * h + 1);
+                    mma_s8_16832(acc[0], a0, a1, a2, a3, xq0[2 * h], xq0[2 * h + 1]);
+                    if (NT > 1) mma_s8_16832(acc[NT - 1], a0, a1, a2, a3, xq1[2 * h], xq1[2 * h + 1]);
                 }
             }
         }
@@ -173,20 +206,24 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
                     for (int i = 0; i < 4; ++i) acc[nt][i] += s_red[warp + q][nt][i][lane];
         }
     }
-    if (kslot != 0) return;
+    if (kslot != 0 || !ok || row0 >= rows) return;
 
     const float gamma = *pr.gamma;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int m = nt * 8 + 2 * t + (i & 1);
-            const int n = row0 + g + 8 * (i >> 1);
-            if (m < M && n < N) {
-                const int a = acc[nt][i] >> 6;  // exact: the sum is a multiple of 64
-                const float f = __fdiv_rn(gamma, pr.s[m]);
-                pr.Y[(size_t)m * N + n] = __fmul_rn(__int2float_rn(a), f);
-                if (pr.acc) pr.acc[(size_t)m * N + n] = a;
+        for (int e = 0; e < 2; ++e) {
+            const int m = nt * 8 + 2 * t + e;
+            if (m >= M) continue;
+            const float f = __fdiv_rn(gamma, pr.s[m]);
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int n = row_base + row0 + g + 8 * hh;
+                if (n < N) {
+                    const int a_ = acc[nt][2 * hh + e] >> 6;  // exact: the sum is a multiple of 64
+                    pr.Y[(size_t)m * N + n] = __fmul_rn(__int2float_rn(a_), f);
+                    if (pr.acc) pr.acc[(size_t)m * N + n] = a_;
+                }
             }
         }
     }

@@ -1,0 +1,462 @@
+// Steps 3 + 4 for large M: the tcgen05 prefill engine (sm_100a).
+//
+// What it computes ("bitone" README, How 1.58-bit Works and Forward pass):
+//   acc[m, n] = sum_k x_q[m, k] * W_q[n, k];  Y[m, n] = acc * (gamma / s[m])
+//
+// One output tile = 128 weight rows (n) x 128 tokens (m), computed as
+// Y^T_tile = W_tile * x_q_tile^T on the 5th-generation tensor cores:
+//   A (M = 128, K = 32 per MMA) = 64 * W_q as int8, in TENSOR MEMORY: the
+//     packed 2-bit rows arrive by TMA, four expander warps unpack them
+//     ((word << (6 - 2j)) & 0xC0C0C0C0 gives four int8 lanes) and write them
+//     with tcgen05.st, so expanded weights never touch shared memory;
+//   B (N = 128 tokens, K = 32) = x_q, by TMA with 128-byte swizzle, K-major,
+//     read by the MMA from shared memory;
+//   D = int32 accumulators in TMEM, two buffers so the epilogue of one tile
+//     overlaps the MMAs of the next.
+// The exact sum is 64 * acc (no overflow: |64 acc| <= 2^28), shifted back
+// by 6 in the epilogue, which also applies float(gamma / s[m]).
+//
+// Warp roles (persistent: one CTA per SM loops over tiles):
+//   warp 0       TMA producer (one thread)
+//   warp 1       TMEM allocator + MMA issuer (one thread)
+//   warps 2..5   expanders: TMEM lanes 32*(w % 4) .. +31 = weight rows
+//   warps 6..9   epilogue:  same lane quarters
+// Every mbarrier wait is bounded (globaltimer); a wait that gives up raises
+// the device error word, sets a CTA abort flag and the CTA drains its
+// in-flight copies and MMAs (again with bounded waits) before it frees TMEM
+// and exits.  No wait is unbounded and nothing traps.
+#pragma once
+
+#include <cuda.h>
+
+#include "bl_common.cuh"
+
+namespace bl {
+
+constexpr int PF_BM = 128;        // weight rows per tile (MMA M, TMEM lanes)
+constexpr int PF_BN = 128;        // tokens per tile (MMA N)
+constexpr int PF_BK = 128;        // k per pipeline stage (4 MMAs of K = 32)
+constexpr int PF_STAGES = 6;
+constexpr int PF_THREADS = 320;
+constexpr int PF_B_BYTES = PF_BN * PF_BK;          // x_q stage: 16 KiB
+constexpr int PF_P_BYTES = PF_BM * PF_BK / 4;      // packed stage: 4 KiB
+constexpr int PF_TMEM_COLS = 512;
+constexpr int PF_ACC_COL = 0;                      // 2 x 128 columns
+constexpr int PF_A_COL = 2 * PF_BN;                // PF_STAGES x 32 columns
+static_assert(PF_A_COL + PF_STAGES * (PF_BK / 4) <= PF_TMEM_COLS, "TMEM budget");
+
+// shared memory carve-up (offsets from a 1024-byte aligned base)
+constexpr int PF_OFF_B = 0;
+constexpr int PF_OFF_P = PF_OFF_B + PF_STAGES * PF_B_BYTES;
+constexpr int PF_OFF_F = PF_OFF_P + PF_STAGES * PF_P_BYTES;           // [4 warps][2][128] float
+constexpr int PF_OFF_BAR = PF_OFF_F + 4 * 2 * PF_BN * 4;
+constexpr int PF_NBAR = 3 * PF_STAGES + 4;                            // full, empty, aready, accfull x2, accempty x2
+constexpr int PF_OFF_MISC = PF_OFF_BAR + PF_NBAR * 8;
+constexpr int PF_SMEM_USED = PF_OFF_MISC + 16;
+constexpr int PF_SMEM_BYTES = PF_SMEM_USED + 1024;                     // + alignment slack
+static_assert(PF_SMEM_BYTES > 116 * 1024, "keeps one CTA per SM, so the TMEM allocation never waits");
+
+struct PrefillParams {
+    const float *gamma;
+    const float *s;
+    float *Y;
+    int32_t *acc;
+    int M, N, K;
+    int n_tiles, m_tiles, k_stages;
+    unsigned long long timeout_ns;
+    long long dbg_skip_iter;  // >= 0: the producer never issues this k-iteration (bounded-wait test)
+};
+
+// ---------------------------------------------------------------------------
+// PTX wrappers
+
+__device__ __forceinline__ void tma_load_2d(u32 dst, const CUtensorMap *map, int x, int y, u32 bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[tmem] * B[smem desc], kind::i8, cta_group::1
+__device__ __forceinline__ void tc_mma_i8_ts(u32 d_tmem, u32 a_tmem, unsigned long long b_desc, u32 idesc,
+                                             u32 accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit(u32 bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_st_32x32b_x32(u32 taddr, const u32 (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_ld_32x32b_x32(u32 taddr, u32 (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (SBO), version 1 (sm_100), base offset 0 (stage bases are
+// 1024-byte aligned).
+__device__ __forceinline__ unsigned long long smem_desc_k_sw128(u32 saddr) {
+    unsigned long long d = 0;
+    d |= (unsigned long long)((saddr >> 4) & 0x3FFFu);
+    d |= (unsigned long long)1u << 16;          // leading byte offset (unused for swizzled K-major) = 16 B
+    d |= (unsigned long long)(1024u >> 4) << 32;  // stride byte offset
+    d |= (unsigned long long)1u << 46;          // descriptor version
+    d |= (unsigned long long)2u << 61;          // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::i8: D s32, A s8, B s8, both K-major, N = PF_BN, M = 128.
+constexpr u32 pf_idesc() {
+    return (2u << 4)                 // D format: s32
+           | (1u << 7)               // A format: signed 8-bit
+           | (1u << 10)              // B format: signed 8-bit
+           | ((u32)(PF_BN >> 3) << 17)  // N >> 3
+           | ((u32)(PF_BM >> 4) << 24);  // M >> 4
+}
+
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_constant__ CUtensorMap tm_x,
+                                                               const __grid_constant__ CUtensorMap tm_w,
+                                                               const __grid_constant__ PrefillParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    const u32 sbase = smem_u32(sm);
+    const u32 bar0 = sbase + PF_OFF_BAR;
+    auto BAR_FULL = [&](int s) { return bar0 + 8u * s; };
+    auto BAR_EMPTY = [&](int s) { return bar0 + 8u * (PF_STAGES + s); };
+    auto BAR_AREADY = [&](int s) { return bar0 + 8u * (2 * PF_STAGES + s); };
+    auto BAR_ACCFULL = [&](int b) { return bar0 + 8u * (3 * PF_STAGES + b); };
+    auto BAR_ACCEMPTY = [&](int b) { return bar0 + 8u * (3 * PF_STAGES + 2 + b); };
+    u32 *s_tmem = reinterpret_cast<u32 *>(sm + PF_OFF_MISC);
+    volatile int *s_abort = reinterpret_cast<volatile int *>(sm + PF_OFF_MISC + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < PF_STAGES; ++s) {
+            mbar_init(BAR_FULL(s), 1);
+            mbar_init(BAR_EMPTY(s), 1);
+            mbar_init(BAR_AREADY(s), 4);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(BAR_ACCFULL(b), 1);
+            mbar_init(BAR_ACCEMPTY(b), 4);
+        }
+        *s_abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_x) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_w) : "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
+                     "r"(PF_TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    __syncthreads();
+    tc_fence_after();
+    const u32 tmem = *s_tmem;
+
+    const int total_tiles = p.n_tiles * p.m_tiles;
+    const int KS = p.k_stages;
+    const unsigned long long TO = p.timeout_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            long long it = 0;
+            bool failed = false;
+            for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x) {
+                const int nt = tile % p.n_tiles, mt = tile / p.n_tiles;
+                for (int ks = 0; ks < KS; ++ks, ++it) {
+                    const int s = (int)(it % PF_STAGES);
+                    const u32 ph = (u32)((it / PF_STAGES) & 1);
+                    if (!mbar_wait(BAR_EMPTY(s), ph ^ 1u, TO, s_abort)) {
+                        failed = true;
+                        break;
+                    }
+                    if (it == p.dbg_skip_iter) continue;  // test hook: this stage never arrives
+                    mbar_arrive_expect_tx(BAR_FULL(s), PF_B_BYTES + PF_P_BYTES);
+                    tma_load_2d(sbase + PF_OFF_B + s * PF_B_BYTES, &tm_x, ks * PF_BK, mt * PF_BN, BAR_FULL(s));
+                    tma_load_2d(sbase + PF_OFF_P + s * PF_P_BYTES, &tm_w, ks * (PF_BK / 4), nt * PF_BM, BAR_FULL(s));
+                }
+            }
+            if (failed) {
+                raise_device_error(DEVERR_TIMEOUT_PRODUCER);
+                *s_abort = 1;
+            }
+            // drain: the last PF_STAGES issued loads must have landed before exit
+            // (time-bounded only; the abort flag does not cut this wait short)
+            for (long long j = it - PF_STAGES; j < it; ++j) {
+                if (j < 0 || j == p.dbg_skip_iter) continue;
+                mbar_wait(BAR_FULL((int)(j % PF_STAGES)), (u32)((j / PF_STAGES) & 1), TO, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const u32 idesc = pf_idesc();
+            long long it = 0;
+            int tc = 0;
+            bool failed = false, issued = false;
+            u32 last_bar = 0, last_ph = 0;
+            for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x, ++tc) {
+                const int b = tc & 1;
+                const u32 aph = (u32)((tc >> 1) & 1);
+                if (!mbar_wait(BAR_ACCEMPTY(b), aph ^ 1u, TO, s_abort)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                const u32 d_tmem = tmem + PF_ACC_COL + b * PF_BN;
+                for (int ks = 0; ks < KS; ++ks, ++it) {
+                    const int s = (int)(it % PF_STAGES);
+                    const u32 ph = (u32)((it / PF_STAGES) & 1);
+                    if (!mbar_wait(BAR_FULL(s), ph, TO, s_abort) || !mbar_wait(BAR_AREADY(s), ph, TO, s_abort)) {
+                        failed = true;
+                        break;
+                    }
+                    tc_fence_after();
+                    const u32 bstage = sbase + PF_OFF_B + s * PF_B_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < PF_BK / 32; ++kk) {
+                        tc_mma_i8_ts(d_tmem, tmem + PF_A_COL + s * (PF_BK / 4) + kk * 8,
+                                     smem_desc_k_sw128(bstage + kk * 32), idesc, (ks | kk) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(BAR_EMPTY(s));
+                    issued = true;
+                    last_bar = BAR_EMPTY(s);
+                    last_ph = ph;
+                }
+                if (failed) break;
+                tc_commit(BAR_ACCFULL(b));
+            }
+            if (failed) {
+                raise_device_error(DEVERR_TIMEOUT_MMA);
+                *s_abort = 1;
+                // drain: every MMA issued so far completes before TMEM is freed
+                if (issued) mbar_wait(last_bar, last_ph, TO, nullptr);
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------------------------------------ expanders
+        const int q = warp & 3;
+        const int row = q * 32 + lane;
+        long long it = 0;
+        bool failed = false;
+        for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x) {
+            for (int ks = 0; ks < KS; ++ks, ++it) {
+                const int s = (int)(it % PF_STAGES);
+                const u32 ph = (u32)((it / PF_STAGES) & 1);
+                bool ok = mbar_wait(BAR_FULL(s), ph, TO, s_abort);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                const uint4 *src = reinterpret_cast<const uint4 *>(sm + PF_OFF_P + s * PF_P_BYTES + row * (PF_BK / 4));
+                const uint4 v0 = src[0], v1 = src[1];
+                const u32 w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+                u32 r[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    r[4 * i + 0] = (w[i] << 6) & 0xC0C0C0C0u;
+                    r[4 * i + 1] = (w[i] << 4) & 0xC0C0C0C0u;
+                    r[4 * i + 2] = (w[i] << 2) & 0xC0C0C0C0u;
+                    r[4 * i + 3] = w[i] & 0xC0C0C0C0u;
+                }
+                tc_st_32x32b_x32(tmem + ((u32)(q * 32) << 16) + PF_A_COL + s * (PF_BK / 4), r);
+                tc_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(BAR_AREADY(s));
+            }
+        }
+        if (failed && lane == 0) {
+            raise_device_error(DEVERR_TIMEOUT_EXPAND);
+            *s_abort = 1;
+        }
+    } else {
+        // ------------------------------------------------------------- epilogue
+        const int q = warp & 3;
+        const int ew = warp - 6;  // 0..3
+        const int row = q * 32 + lane;
+        float *fbuf = reinterpret_cast<float *>(sm + PF_OFF_F) + ew * 2 * PF_BN;
+        const float gamma = *p.gamma;
+        int tc = 0;
+        bool failed = false;
+        for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x, ++tc) {
+            const int nt = tile % p.n_tiles, mt = tile / p.n_tiles;
+            const int b = tc & 1;
+            const u32 aph = (u32)((tc >> 1) & 1);
+            float *f = fbuf + b * PF_BN;
+            // per-warp copy of float(gamma / s[m]) for this tile's tokens
+#pragma unroll
+            for (int j = 0; j < PF_BN / 32; ++j) {
+                const int c = j * 32 + lane;
+                const int m = mt * PF_BN + c;
+                f[c] = m < p.M ? __fdiv_rn(gamma, p.s[m]) : 0.f;
+            }
+            __syncwarp();
+            bool ok = mbar_wait(BAR_ACCFULL(b), aph, TO, s_abort);
+            if (!__all_sync(0xffffffffu, ok)) {
+                failed = true;
+                break;
+            }
+            tc_fence_after();
+            const int n = nt * PF_BM + row;
+            const bool nvalid = n < p.N;
+#pragma unroll 1
+            for (int c0 = 0; c0 < PF_BN; c0 += 32) {
+                u32 r[32];
+                tc_ld_32x32b_x32(tmem + ((u32)(q * 32) << 16) + PF_ACC_COL + b * PF_BN + c0, r);
+                tc_wait_ld();
+                if (c0 + 32 == PF_BN) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(BAR_ACCEMPTY(b));
+                }
+                const int mbase = mt * PF_BN + c0;
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int m = mbase + j;
+                    if (nvalid && m < p.M) {
+                        const int a = (int)r[j] >> 6;  // exact: the sum is a multiple of 64
+                        const size_t o = (size_t)m * p.N + n;
+                        p.Y[o] = __fmul_rn(__int2float_rn(a), f[c0 + j]);
+                        if (p.acc) p.acc[o] = a;
+                    }
+                }
+            }
+            __syncwarp();
+        }
+        if (failed && lane == 0) {
+            raise_device_error(DEVERR_TIMEOUT_EPILOGUE);
+            *s_abort = 1;
+        }
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(PF_TMEM_COLS)
+                     : "memory");
+    }
+}
+
+}  // namespace bl
+
+// ===========================================================================
+// Host side: tensor maps and launch.
+
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+namespace bl {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no
+// link-time dependency on libcuda).
+inline EncodeTiledFn encode_tiled_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+inline cudaError_t prefill_setup() {
+    if (encode_tiled_fn() == nullptr) return cudaErrorNotSupported;
+    return cudaFuncSetAttribute(k_prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM_BYTES);
+}
+
+constexpr unsigned long long PF_DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
+
+inline bl_status prefill_launch(int sms, const uint8_t *packed, const float *gamma, const int8_t *x_q, const float *s,
+                                int64_t M, int64_t N, int64_t K, float *Y, int32_t *acc_out, cudaStream_t st,
+                                unsigned long long timeout_ns = PF_DEFAULT_TIMEOUT_NS, long long dbg_skip_iter = -1) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (enc == nullptr) return BL_ERR_CUDA;
+    const int64_t n_tiles = (N + PF_BM - 1) / PF_BM, m_tiles = (M + PF_BN - 1) / PF_BN;
+    if (n_tiles * m_tiles > 0x7fffffffLL) return BL_ERR_SHAPE;
+    CUtensorMap tx, tw;
+    const cuuint32_t es[2] = {1, 1};
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)K};
+        const cuuint32_t box[2] = {(cuuint32_t)PF_BK, (cuuint32_t)PF_BN};
+        if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(x_q), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return BL_ERR_CUDA;
+    }
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
+        const cuuint64_t gstride[1] = {(cuuint64_t)(K / 4)};
+        const cuuint32_t box[2] = {(cuuint32_t)(PF_BK / 4), (cuuint32_t)PF_BM};
+        if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return BL_ERR_CUDA;
+    }
+    PrefillParams p;
+    p.gamma = gamma;
+    p.s = s;
+    p.Y = Y;
+    p.acc = acc_out;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.n_tiles = (int)n_tiles;
+    p.m_tiles = (int)m_tiles;
+    p.k_stages = (int)((K + PF_BK - 1) / PF_BK);
+    p.timeout_ns = timeout_ns;
+    p.dbg_skip_iter = dbg_skip_iter;
+    const int64_t tiles = n_tiles * m_tiles;
+    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    k_prefill_tc<<<grid, PF_THREADS, PF_SMEM_BYTES, st>>>(tx, tw, p);
+    return cudaGetLastError() == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+}  // namespace bl

@@ -12,7 +12,7 @@ import pytest
 
 from ternary_quantized_linear_bitlinear_b200 import api, build
 
-HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "bitlinear.h")
+INCLUDE = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
 
 OK, NULL, SHAPE, ALIGN, DTYPE, CUDA, TIMEOUT, WORKSPACE, DEVICE = range(9)
 A = 1 << 20  # a fake, 16-byte aligned "device address" (never dereferenced)
@@ -25,9 +25,13 @@ def L():
 
 
 def declared_functions():
-    text = open(HEADER).read()
-    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(bl_[a-z_0-9]+)\s*\(", text)))
+    names = set()
+    for h in sorted(os.listdir(INCLUDE)):
+        if h.endswith(".h"):
+            text = open(os.path.join(INCLUDE, h)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(bl_[a-z_0-9]+)\s*\(", text))
+    return sorted(names)
 
 
 def test_exports_every_declared_symbol(L):
@@ -114,22 +118,32 @@ def test_grouped_validation(L):
     P = (api.Problem * 2)()
     for i in range(2):
         P[i] = api.Problem(A, A, A, A, A, None, 64, 128)
-    g = L.bl_forward_grouped
-    assert g(None, 1, 1, None) == NULL
-    assert g(P, 0, 1, None) == SHAPE
-    assert g(P, api.BL_MAX_GROUP + 1, 1, None) == SHAPE
-    assert g(P, 2, 17, None) == SHAPE  # grouped decode is for M <= 16
+    def g(arr, count, M):
+        return L.bl_forward_grouped(arr, count, M, 0, None)
+    assert g(None, 1, 1) == NULL
+    assert g(P, 0, 1) == SHAPE
+    assert g(P, api.BL_MAX_GROUP + 1, 1) == SHAPE
+    assert g(P, 2, 17) == SHAPE  # grouped decode is for M <= 16
     P[1].K = 100
-    assert g(P, 2, 1, None) == SHAPE
+    assert g(P, 2, 1) == SHAPE
     P[1].K = 128
     P[1].Y = None
-    assert g(P, 2, 1, None) == NULL
+    assert g(P, 2, 1) == NULL
     P[1].Y = A
-    assert g(P, 2, 1, None) in (CUDA, DEVICE)
+    assert g(P, 2, 1) in (CUDA, DEVICE)
     Q = (api.ActProblem * 1)()
     Q[0] = api.ActProblem(A, None, A, A, 128)
     assert L.bl_quant_act_grouped(Q, 1, 5, 1, 1e-6, None) == DTYPE
     assert L.bl_quant_act_grouped(Q, 1, 1, 1, 1e-6, None) in (CUDA, DEVICE)
+
+
+def test_debug_prefill_validation(L):
+    f = L.bl_debug_forward_prefill
+    assert f(None, A, A, A, 1, 64, 128, A, None, -1, 1000, None) == NULL
+    assert f(A, A, A, A, 1, 64, 100, A, None, -1, 1000, None) == SHAPE
+    assert f(A, A, A, A, 1, 64, 128, A, None, -1, 0, None) == SHAPE
+    assert f(A, A, A, A, 1, 64, 128, A + 4, None, -1, 1000, None) == ALIGN
+    assert f(A, A, A, A, 1, 64, 128, A, None, 0, 1000, None) in (CUDA, DEVICE)
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

@@ -191,3 +191,68 @@ def test_linear_subln_qat4b_oproj_small():
     ref = oracle.linear(np32(W), np32(X), np32(gain), workloads.SUBLN_EPS)
     err = np.abs(Y.cpu().numpy().astype(np.float64) - ref["Y"])
     assert np.all(err <= 1e-6 * np.abs(ref["Y"]))
+
+
+# -- tcgen05 prefill engine at small M, and its bounded waits ----------------
+
+@pytest.mark.parametrize("M,N,K", [
+    (128, 128, 128), (1, 37, 64), (5, 300, 192), (16, 128, 1536), (200, 130, 768), (129, 257, 4096),
+    (300, 64, 8640),
+])
+def test_prefill_engine_forced(M, N, K):
+    W = workloads.normal((N, K), 0.02, 500 + K)
+    X = workloads.with_outlier_channels(workloads.normal((M, K), 1.0, 600 + M, torch.bfloat16), 2, 20.0, 4)
+    packed, gamma = api.bl_quant_weights(W.cuda())
+    x_q, s = api.bl_quant_act(X.cuda())
+    acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
+    Y = api.bl_debug_forward_prefill(packed, gamma, x_q, s, N, acc_out=acc)
+    api.bl_check_device_error()
+    wq_ref, g_ref = check_weights(W, packed, gamma)
+    xq_ref, s_ref = check_act(X, x_q, s)
+    check_forward_full(xq_ref, s_ref, wq_ref, g_ref, Y, acc)
+
+
+def test_prefill_bounded_wait_gives_up_and_context_survives():
+    M, N, K = 256, 256, 1024
+    W = workloads.normal((N, K), 0.02, 7)
+    X = workloads.normal((M, K), 1.0, 8, torch.bfloat16)
+    packed, gamma = api.bl_quant_weights(W.cuda())
+    x_q, s = api.bl_quant_act(X.cuda())
+    api.bl_check_device_error()
+    # the producer never issues k-iteration 0: every consumer's wait runs out
+    api.bl_debug_forward_prefill(packed, gamma, x_q, s, N, skip_iter=0, timeout_us=2000)
+    with pytest.raises(api.BitLinearError) as e:
+        api.bl_check_device_error()
+    assert e.value.status == 6  # BL_ERR_TIMEOUT
+    api.bl_check_device_error()  # the error word was cleared
+    acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
+    Y = api.bl_forward(packed, gamma, x_q, s, N, acc_out=acc)
+    api.bl_check_device_error()
+    wq_ref, g_ref = check_weights(W, packed, gamma)
+    xq_ref, s_ref = check_act(X, x_q, s)
+    check_forward_full(xq_ref, s_ref, wq_ref, g_ref, Y, acc)
+
+
+def test_grouped_decode_with_programmatic_launch():
+    M = 8
+    items = workloads.decode125m(M=M, layers=1)
+    acts, dev, refs = [], [], []
+    for name, W, X in items:
+        packed, gamma = gpu_quant_weights(W)
+        N, K = W.shape
+        Xd = X.cuda()
+        xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+        s = torch.empty(M, dtype=torch.float32, device="cuda")
+        acts.append((Xd, None, xq, s))
+        dev.append((packed, gamma, xq, s, torch.empty(M, N, device="cuda"),
+                    torch.empty(M, N, dtype=torch.int32, device="cuda"), N, K))
+        refs.append((W, X))
+    arr = api.make_problems(dev)
+    for _ in range(3):  # act quant immediately followed by the dependent GEMV
+        api.bl_quant_act_grouped(acts, torch.bfloat16)
+        api.bl_forward_grouped(arr, len(dev), M, flags=api.BL_FWD_WEIGHTS_READY)
+    api.bl_check_device_error()
+    for (packed, gamma, x_q, s, Y, acc, N, K), (W, X) in zip(dev, refs):
+        wq_ref, g_ref = check_weights(W, packed, gamma)
+        xq_ref, s_ref = check_act(X, x_q, s)
+        check_forward_full(xq_ref, s_ref, wq_ref, g_ref, Y, acc)
