@@ -184,6 +184,13 @@ bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st) {
         xq_off = xo > xq_off ? xo : xq_off;
     }
     P.xq_off = xq_off;
+    P.use_table = total <= DEC_CTA_TABLE ? 1 : 0;
+    if (P.use_table) {
+        for (int i = 0; i < P.count; ++i) {
+            const int end = i + 1 < P.count ? P.p[i + 1].cta_begin : total;
+            for (int c = P.p[i].cta_begin; c < end; ++c) P.cta_problem[c] = (unsigned char)i;
+        }
+    }
     const size_t smem = (size_t)xq_off + (size_t)P.M * rs_max;
     if (smem > DEC_SMEM_LIMIT) return BL_ERR_SHAPE;
     cudaLaunchConfig_t cfg = {};

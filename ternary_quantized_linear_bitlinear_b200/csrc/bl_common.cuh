@@ -177,14 +177,16 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(u32 bar, u32 bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
+// try_wait may suspend the thread up to the hint (ns) until the phase
+// completes, so waiting warps do not spin on the issue slots.
 __device__ __forceinline__ bool mbar_try_wait(u32 bar, u32 parity) {
     u32 ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(bar), "r"(parity)
+        : "r"(bar), "r"(parity), "r"(200000u)
         : "memory");
     return ok != 0;
 }
@@ -197,7 +199,7 @@ __device__ __forceinline__ bool mbar_wait(u32 bar, u32 parity, unsigned long lon
     const unsigned long long t0 = globaltimer();
     for (int it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 63) == 0) {
+        if ((it & 7) == 0) {
             if (abort_flag != nullptr && *abort_flag) return false;
             if (globaltimer() - t0 > timeout_ns) return false;
         }

@@ -7,8 +7,8 @@
 // weight).  Design:
 //   - A CTA (8 warps) owns T = 8/G consecutive 16-row tiles of one problem;
 //     their packed rows are one contiguous byte range, which one thread
-//     requests with cp.async.bulk copies into shared memory (completion on an
-//     mbarrier, bounded wait), so the memory system sees a few large requests
+//     requests with cp.async.bulk copies into shared memory (one mbarrier per
+//     tile, bounded waits), so the memory system sees a few large requests
 //     per CTA and the warps issue no global loads for weights.
 //   - A warp owns a 16-row tile; G warps split its K range (G picked per
 //     problem from K so that each warp has at most 4 steps of 256 k).
@@ -51,11 +51,15 @@ struct DecodeProblem {
     int cta_begin;  // first CTA of this problem in the grouped grid
 };
 
+constexpr int DEC_CTA_TABLE = 2048;  // grids up to this size look their problem up in a table
+
 struct DecodeParams {
     DecodeProblem p[BL_MAX_GROUP];
     int count;
     int M;
     int xq_off;  // shared-memory offset of the staged x_q (after the weight tiles)
+    int use_table;
+    unsigned char cta_problem[DEC_CTA_TABLE];
 };
 
 __host__ __device__ inline int dec_row_stride(int K) { return (K + 255) & ~255; }
@@ -88,54 +92,78 @@ template <int NT>
 __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ DecodeParams P) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_red[DEC_WARPS][NT][4][32];
-    __shared__ __align__(8) u64 s_bar;
+    __shared__ __align__(8) u64 s_bar[DEC_WARPS];
+    __shared__ float s_f[16];
 
-    // problem of this CTA: binary search over the CTA prefix
     const int b = blockIdx.x;
-    int lo = 0, hi = P.count - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (P.p[mid].cta_begin <= b) lo = mid; else hi = mid - 1;
+    int pi;
+    if (P.use_table) {
+        pi = P.cta_problem[b];
+    } else {  // binary search over the CTA prefix
+        int lo = 0, hi = P.count - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (P.p[mid].cta_begin <= b) lo = mid; else hi = mid - 1;
+        }
+        pi = lo;
     }
-    const DecodeProblem &pr = P.p[lo];
+    const DecodeProblem &pr = P.p[pi];
     const int M = P.M, N = pr.N, K = pr.K;
     const int glog = pr.g_log2, G = 1 << glog;
     const int T = DEC_WARPS >> glog;
     const int Kw = K >> 2;         // packed bytes per row
     const int row_base = (b - pr.cta_begin) * T * 16;
     const int rows = min(T * 16, N - row_base);
-    const u32 bar = smem_u32(&s_bar);
+    const int tiles = (rows + 15) >> 4;
 
-    // One thread requests the CTA's weight rows (contiguous bytes).
+    // One thread requests the CTA's weight rows, one bulk copy (and one
+    // mbarrier) per 16-row tile, so each warp starts as soon as its tile lands.
     if (threadIdx.x == 0) {
-        mbar_init(bar, 1);
+        for (int i = 0; i < tiles; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        const u32 bytes = (u32)rows * (u32)Kw;
-        mbar_arrive_expect_tx(bar, bytes);
         const uint8_t *src = pr.packed + (size_t)row_base * Kw;
         const u32 dst = smem_u32(smem);
-        for (u32 off = 0; off < bytes; off += 32768u) {
-            const u32 n = bytes - off < 32768u ? bytes - off : 32768u;
-            bulk_g2s(dst + off, src + off, n, bar);
+        for (int i = 0; i < tiles; ++i) {
+            const u32 nrows = (u32)min(16, rows - 16 * i);
+            const u32 bytes = nrows * (u32)Kw;
+            const u32 bar = smem_u32(&s_bar[i]);
+            mbar_arrive_expect_tx(bar, bytes);
+            const u32 off0 = (u32)(16 * i) * (u32)Kw;
+            for (u32 off = 0; off < bytes; off += 32768u) {
+                const u32 n = bytes - off < 32768u ? bytes - off : 32768u;
+                bulk_g2s(dst + off0 + off, src + off0 + off, n, bar);
+            }
         }
     }
 
-    // x_q may be produced by the kernel launched just before this one.
+    // x_q and s may be produced by the kernel launched just before this one.
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // Stage x_q rows [0, M) into shared memory, swizzled, zero-padded to RS.
+    // Stage x_q rows [0, M) into shared memory, swizzled, zero-padded to RS;
+    // float(gamma / s[m]) once per token.
     const int RS = dec_row_stride(K);
     uint8_t *s_xq = smem + P.xq_off;
     {
+        // every 16-byte chunk in flight at once (cp.async), one wait
         const int chunks = RS >> 4;
+        const int kchunks = K >> 4;
         for (int r = 0; r < M; ++r) {
+            const int8_t *src = pr.xq + (size_t)r * K;
+            uint8_t *dst = s_xq + r * RS;
             for (int L = threadIdx.x; L < chunks; L += DEC_THREADS) {
-                uint4 v = make_uint4(0, 0, 0, 0);
-                if (L * 16 < K) v = *reinterpret_cast<const uint4 *>(pr.xq + (size_t)r * K + L * 16);
                 const int x = (((L >> 3) & 1) << 1) | (r & 1);
-                *reinterpret_cast<uint4 *>(s_xq + r * RS + (((L & ~7) | ((L ^ x) & 7)) << 4)) = v;
+                uint8_t *d = dst + (((L & ~7) | ((L ^ x) & 7)) << 4);
+                if (L < kchunks) {
+                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(d)), "l"(src + L * 16)
+                                 : "memory");
+                } else {
+                    *reinterpret_cast<uint4 *>(d) = make_uint4(0, 0, 0, 0);
+                }
             }
         }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (threadIdx.x < M) s_f[threadIdx.x] = __fdiv_rn(*pr.gamma, pr.s[threadIdx.x]);
+        asm volatile("cp.async.wait_all;" ::: "memory");
     }
     __syncthreads();
 
@@ -146,16 +174,20 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
     const int steps = (K + 255) >> 8;
     const int nchunk64 = K >> 6;
 
-    int acc[NT][4];
+    // two independent accumulator chains (even / odd 16-k chunks)
+    int acc[NT][4], acc2[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][i] = 0;
+        for (int i = 0; i < 4; ++i) acc[nt][i] = acc2[nt][i] = 0;
 
-    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0, DEC_TIMEOUT_NS, nullptr));
-    if (!ok && lane == 0) raise_device_error(DEVERR_TIMEOUT_PRODUCER);
+    bool ok = true;
+    if (wt < tiles) {
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&s_bar[wt]), 0, DEC_TIMEOUT_NS, nullptr));
+        if (!ok && lane == 0) raise_device_error(DEVERR_TIMEOUT_PRODUCER);
+    }
 
-    if (ok && row0 < rows) {
+    if (ok && wt < tiles) {
         const uint8_t *wA = smem + (row0 + g) * Kw + t * 16;
         const uint8_t *wB = smem + (row0 + g + 8) * Kw + t * 16;
         // B fragments: token rows g (and g + 8); chunk c of a step sits at
@@ -165,31 +197,43 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
         const int xb1 = ((t >> 1) << 1) | ((g + 8) & 1);
         const uint8_t *xr0 = s_xq + g * RS + t * 64;
         const uint8_t *xr1 = s_xq + (g + 8) * RS + t * 64;
-#pragma unroll 4
+        int o0[4], o1[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            o0[c] = (c ^ xb0) << 4;
+            o1[c] = (c ^ xb1) << 4;
+        }
+#pragma unroll 2
         for (int s2 = kslot; s2 < steps; s2 += G) {
             const bool kv = (s2 * 4 + t) < nchunk64;
             const uint4 va = kv ? *reinterpret_cast<const uint4 *>(wA + s2 * 64) : make_uint4(0, 0, 0, 0);
             const uint4 vb = kv ? *reinterpret_cast<const uint4 *>(wB + s2 * 64) : make_uint4(0, 0, 0, 0);
             const u32 wa[4] = {va.x, va.y, va.z, va.w};
             const u32 wb[4] = {vb.x, vb.y, vb.z, vb.w};
+            const uint8_t *x0p = xr0 + s2 * 256;
+            const uint8_t *x1p = xr1 + s2 * 256;
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                const uint4 x0 = tv0 ? *reinterpret_cast<const uint4 *>(xr0 + s2 * 256 + ((c ^ xb0) << 4))
-                                     : make_uint4(0, 0, 0, 0);
+                const uint4 x0 = tv0 ? *reinterpret_cast<const uint4 *>(x0p + o0[c]) : make_uint4(0, 0, 0, 0);
                 uint4 x1 = make_uint4(0, 0, 0, 0);
-                if (NT > 1 && tv1) x1 = *reinterpret_cast<const uint4 *>(xr1 + s2 * 256 + ((c ^ xb1) << 4));
+                if (NT > 1 && tv1) x1 = *reinterpret_cast<const uint4 *>(x1p + o1[c]);
                 const u32 xq0[4] = {x0.x, x0.y, x0.z, x0.w};
                 const u32 xq1[4] = {x1.x, x1.y, x1.z, x1.w};
+                int(&A)[NT][4] = (c & 1) ? acc2 : acc;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const u32 a0 = dec_unpack(wa[c], 2 * h), a2 = dec_unpack(wa[c], 2 * h + 1);
                     const u32 a1 = dec_unpack(wb[c], 2 * h), a3 = dec_unpack(wb[c], 2 * h + 1);
-                    mma_s8_16832(acc[0], a0, a1, a2, a3, xq0[2 * h], xq0[2 * h + 1]);
-                    if (NT > 1) mma_s8_16832(acc[NT - 1], a0, a1, a2, a3, xq1[2 * h], xq1[2 * h + 1]);
+                    mma_s8_16832(A[0], a0, a1, a2, a3, xq0[2 * h], xq0[2 * h + 1]);
+                    if (NT > 1) mma_s8_16832(A[NT - 1], a0, a1, a2, a3, xq1[2 * h], xq1[2 * h + 1]);
                 }
             }
         }
     }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[nt][i] += acc2[nt][i];
 
     // split-K reduction through shared memory
     if (G > 1) {
@@ -206,16 +250,15 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
                     for (int i = 0; i < 4; ++i) acc[nt][i] += s_red[warp + q][nt][i][lane];
         }
     }
-    if (kslot != 0 || !ok || row0 >= rows) return;
+    if (kslot != 0 || !ok || wt >= tiles) return;
 
-    const float gamma = *pr.gamma;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
             const int m = nt * 8 + 2 * t + e;
             if (m >= M) continue;
-            const float f = __fdiv_rn(gamma, pr.s[m]);
+            const float f = s_f[m];
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 const int n = row_base + row0 + g + 8 * hh;

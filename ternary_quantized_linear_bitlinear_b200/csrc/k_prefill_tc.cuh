@@ -3,24 +3,31 @@
 // What it computes ("bitone" README, How 1.58-bit Works and Forward pass):
 //   acc[m, n] = sum_k x_q[m, k] * W_q[n, k];  Y[m, n] = acc * (gamma / s[m])
 //
-// One output tile = 128 weight rows (n) x 128 tokens (m), computed as
-// Y^T_tile = W_tile * x_q_tile^T on the 5th-generation tensor cores:
-//   A (M = 128, K = 32 per MMA) = 64 * W_q as int8, in TENSOR MEMORY: the
-//     packed 2-bit rows arrive by TMA, four expander warps unpack them
-//     ((word << (6 - 2j)) & 0xC0C0C0C0 gives four int8 lanes) and write them
-//     with tcgen05.st, so expanded weights never touch shared memory;
-//   B (N = 128 tokens, K = 32) = x_q, by TMA with 128-byte swizzle, K-major,
-//     read by the MMA from shared memory;
-//   D = int32 accumulators in TMEM, two buffers so the epilogue of one tile
-//     overlaps the MMAs of the next.
-// The exact sum is 64 * acc (no overflow: |64 acc| <= 2^28), shifted back
-// by 6 in the epilogue, which also applies float(gamma / s[m]).
+// One output tile = 128 weight rows (n) x 256 tokens (m), computed as
+// Y^T_tile = W_tile * x_q_tile^T with tcgen05.mma.cta_group::1.kind::i8,
+// M = 128, N = 256, K = 32 per instruction (the issue cost of one MMA is
+// nearly independent of N, so N = 256 is what reaches the tensor peak):
+//   A = 64 * W_q as int8 in shared memory: the packed 2-bit rows arrive by
+//     TMA, eight expander warps unpack them ((word << (6 - 2j)) & 0xC0C0C0C0
+//     gives four int8 lanes) and store them in the 128-byte-swizzled K-major
+//     layout the MMA reads, then fence the async proxy;
+//   B = x_q, by TMA with 128-byte swizzle, K-major;
+//   D = int32 accumulators in TMEM, two 256-column buffers so the epilogue
+//     of one tile overlaps the MMAs of the next.
+// The exact sum is 64 * acc (|64 acc| <= 2^28, exact in int32 and in
+// float), so Y = float(float(64 acc) * (f / 64)) with f = float(gamma / s[m])
+// (f / 64 is exact) -- the same bits as float(acc) * f.
+//
+// Pipelines: PF_STAGES shared-memory stages carry x_q and packed tiles from
+// TMA; PF_ASTAGES shared-memory stages carry the expanded weights from the
+// expanders to the MMA.  MMA completion frees both (two commits).
 //
 // Warp roles (persistent: one CTA per SM loops over tiles):
 //   warp 0       TMA producer (one thread)
 //   warp 1       TMEM allocator + MMA issuer (one thread)
-//   warps 2..5   expanders: TMEM lanes 32*(w % 4) .. +31 = weight rows
-//   warps 6..9   epilogue:  same lane quarters
+//   warps 2..9   expanders: weight rows 32*(w % 4) .. +31; two warps per
+//                row quarter take alternate pipeline stages
+//   warps 10..13 epilogue: TMEM lanes 32*(w % 4) .. +31 (= weight rows)
 // Every mbarrier wait is bounded (globaltimer); a wait that gives up raises
 // the device error word, sets a CTA abort flag and the CTA drains its
 // in-flight copies and MMAs (again with bounded waits) before it frees TMEM
@@ -33,28 +40,32 @@
 
 namespace bl {
 
-constexpr int PF_BM = 128;        // weight rows per tile (MMA M, TMEM lanes)
-constexpr int PF_BN = 128;        // tokens per tile (MMA N)
-constexpr int PF_BK = 128;        // k per pipeline stage (4 MMAs of K = 32)
-constexpr int PF_STAGES = 6;
-constexpr int PF_THREADS = 320;
-constexpr int PF_B_BYTES = PF_BN * PF_BK;          // x_q stage: 16 KiB
+constexpr int PF_BM = 128;         // weight rows per tile (MMA M, TMEM lanes)
+constexpr int PF_BN = 256;         // tokens per tile (MMA N)
+constexpr int PF_BK = 128;         // k per pipeline stage (4 MMAs of K = 32)
+constexpr int PF_STAGES = 4;       // TMA stages (x_q + packed)
+constexpr int PF_ASTAGES = 3;      // expanded-weight stages
+constexpr int PF_THREADS = 448;
+constexpr int PF_EXP_WARPS = 8;    // expander warps (2 per row quarter)
+constexpr int PF_EPI_WARP0 = 2 + PF_EXP_WARPS;
+constexpr int PF_B_BYTES = PF_BN * PF_BK;          // x_q stage: 32 KiB
+constexpr int PF_A_BYTES = PF_BM * PF_BK;          // expanded stage: 16 KiB
 constexpr int PF_P_BYTES = PF_BM * PF_BK / 4;      // packed stage: 4 KiB
-constexpr int PF_TMEM_COLS = 512;
-constexpr int PF_ACC_COL = 0;                      // 2 x 128 columns
-constexpr int PF_A_COL = 2 * PF_BN;                // PF_STAGES x 32 columns
-static_assert(PF_A_COL + PF_STAGES * (PF_BK / 4) <= PF_TMEM_COLS, "TMEM budget");
+constexpr int PF_TMEM_COLS = 512;                  // 2 x 256 accumulator columns
 
 // shared memory carve-up (offsets from a 1024-byte aligned base)
 constexpr int PF_OFF_B = 0;
-constexpr int PF_OFF_P = PF_OFF_B + PF_STAGES * PF_B_BYTES;
-constexpr int PF_OFF_F = PF_OFF_P + PF_STAGES * PF_P_BYTES;           // [4 warps][2][128] float
+constexpr int PF_OFF_A = PF_OFF_B + PF_STAGES * PF_B_BYTES;
+constexpr int PF_OFF_P = PF_OFF_A + PF_ASTAGES * PF_A_BYTES;
+constexpr int PF_OFF_F = PF_OFF_P + PF_STAGES * PF_P_BYTES;           // [4 warps][2][256] float
 constexpr int PF_OFF_BAR = PF_OFF_F + 4 * 2 * PF_BN * 4;
-constexpr int PF_NBAR = 3 * PF_STAGES + 4;                            // full, empty, aready, accfull x2, accempty x2
+constexpr int PF_NBAR = 2 * PF_STAGES + 2 * PF_ASTAGES + 4;           // full, empty, aready, aempty, accfull x2, accempty x2
 constexpr int PF_OFF_MISC = PF_OFF_BAR + PF_NBAR * 8;
 constexpr int PF_SMEM_USED = PF_OFF_MISC + 16;
 constexpr int PF_SMEM_BYTES = PF_SMEM_USED + 1024;                     // + alignment slack
 static_assert(PF_SMEM_BYTES > 116 * 1024, "keeps one CTA per SM, so the TMEM allocation never waits");
+static_assert(PF_SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(PF_ASTAGES >= 2, "expander warp pairs alternate stages");
 
 struct PrefillParams {
     const float *gamma;
@@ -80,32 +91,20 @@ __device__ __forceinline__ void tma_load_2d(u32 dst, const CUtensorMap *map, int
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[tmem] * B[smem desc], kind::i8, cta_group::1
-__device__ __forceinline__ void tc_mma_i8_ts(u32 d_tmem, u32 a_tmem, unsigned long long b_desc, u32 idesc,
-                                             u32 accumulate) {
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::i8, cta_group::1
+__device__ __forceinline__ void tc_mma_i8_ss(u32 d_tmem, unsigned long long a_desc, unsigned long long b_desc,
+                                             u32 idesc, u32 accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
 __device__ __forceinline__ void tc_commit(u32 bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                  : "memory");
-}
-
-__device__ __forceinline__ void tc_st_32x32b_x32(u32 taddr, const u32 (&r)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-        ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-        "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-        "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
 }
 
 __device__ __forceinline__ void tc_ld_32x32b_x32(u32 taddr, u32 (&r)[32]) {
@@ -121,7 +120,6 @@ __device__ __forceinline__ void tc_ld_32x32b_x32(u32 taddr, u32 (&r)[32]) {
         : "memory");
 }
 
-__device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
@@ -130,20 +128,20 @@ __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sy
 __device__ __forceinline__ unsigned long long smem_desc_k_sw128(u32 saddr) {
     unsigned long long d = 0;
     d |= (unsigned long long)((saddr >> 4) & 0x3FFFu);
-    d |= (unsigned long long)1u << 16;          // leading byte offset (unused for swizzled K-major) = 16 B
+    d |= (unsigned long long)1u << 16;            // leading byte offset (unused for swizzled K-major) = 16 B
     d |= (unsigned long long)(1024u >> 4) << 32;  // stride byte offset
-    d |= (unsigned long long)1u << 46;          // descriptor version
-    d |= (unsigned long long)2u << 61;          // SWIZZLE_128B
+    d |= (unsigned long long)1u << 46;            // descriptor version
+    d |= (unsigned long long)2u << 61;            // SWIZZLE_128B
     return d;
 }
 
 // Instruction descriptor, kind::i8: D s32, A s8, B s8, both K-major, N = PF_BN, M = 128.
-constexpr u32 pf_idesc() {
-    return (2u << 4)                 // D format: s32
-           | (1u << 7)               // A format: signed 8-bit
-           | (1u << 10)              // B format: signed 8-bit
+__host__ __device__ constexpr u32 pf_idesc() {
+    return (2u << 4)                    // D format: s32
+           | (1u << 7)                  // A format: signed 8-bit
+           | (1u << 10)                 // B format: signed 8-bit
            | ((u32)(PF_BN >> 3) << 17)  // N >> 3
-           | ((u32)(PF_BM >> 4) << 24);  // M >> 4
+           | ((u32)(PF_BM >> 4) << 24); // M >> 4
 }
 
 // ---------------------------------------------------------------------------
@@ -157,9 +155,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
     const u32 bar0 = sbase + PF_OFF_BAR;
     auto BAR_FULL = [&](int s) { return bar0 + 8u * s; };
     auto BAR_EMPTY = [&](int s) { return bar0 + 8u * (PF_STAGES + s); };
-    auto BAR_AREADY = [&](int s) { return bar0 + 8u * (2 * PF_STAGES + s); };
-    auto BAR_ACCFULL = [&](int b) { return bar0 + 8u * (3 * PF_STAGES + b); };
-    auto BAR_ACCEMPTY = [&](int b) { return bar0 + 8u * (3 * PF_STAGES + 2 + b); };
+    auto BAR_AREADY = [&](int a) { return bar0 + 8u * (2 * PF_STAGES + a); };
+    auto BAR_AEMPTY = [&](int a) { return bar0 + 8u * (2 * PF_STAGES + PF_ASTAGES + a); };
+    auto BAR_ACCFULL = [&](int b) { return bar0 + 8u * (2 * PF_STAGES + 2 * PF_ASTAGES + b); };
+    auto BAR_ACCEMPTY = [&](int b) { return bar0 + 8u * (2 * PF_STAGES + 2 * PF_ASTAGES + 2 + b); };
     u32 *s_tmem = reinterpret_cast<u32 *>(sm + PF_OFF_MISC);
     volatile int *s_abort = reinterpret_cast<volatile int *>(sm + PF_OFF_MISC + 4);
 
@@ -168,7 +167,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         for (int s = 0; s < PF_STAGES; ++s) {
             mbar_init(BAR_FULL(s), 1);
             mbar_init(BAR_EMPTY(s), 1);
-            mbar_init(BAR_AREADY(s), 4);
+        }
+        for (int a = 0; a < PF_ASTAGES; ++a) {
+            mbar_init(BAR_AREADY(a), 4);
+            mbar_init(BAR_AEMPTY(a), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(BAR_ACCFULL(b), 1);
@@ -234,28 +236,32 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
             u32 last_bar = 0, last_ph = 0;
             for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x, ++tc) {
                 const int b = tc & 1;
-                const u32 aph = (u32)((tc >> 1) & 1);
-                if (!mbar_wait(BAR_ACCEMPTY(b), aph ^ 1u, TO, s_abort)) {
+                const u32 cph = (u32)((tc >> 1) & 1);
+                if (!mbar_wait(BAR_ACCEMPTY(b), cph ^ 1u, TO, s_abort)) {
                     failed = true;
                     break;
                 }
                 tc_fence_after();
-                const u32 d_tmem = tmem + PF_ACC_COL + b * PF_BN;
+                const u32 d_tmem = tmem + b * PF_BN;
                 for (int ks = 0; ks < KS; ++ks, ++it) {
                     const int s = (int)(it % PF_STAGES);
                     const u32 ph = (u32)((it / PF_STAGES) & 1);
-                    if (!mbar_wait(BAR_FULL(s), ph, TO, s_abort) || !mbar_wait(BAR_AREADY(s), ph, TO, s_abort)) {
+                    const int a = (int)(it % PF_ASTAGES);
+                    const u32 aph = (u32)((it / PF_ASTAGES) & 1);
+                    if (!mbar_wait(BAR_FULL(s), ph, TO, s_abort) || !mbar_wait(BAR_AREADY(a), aph, TO, s_abort)) {
                         failed = true;
                         break;
                     }
                     tc_fence_after();
                     const u32 bstage = sbase + PF_OFF_B + s * PF_B_BYTES;
+                    const u32 astage = sbase + PF_OFF_A + a * PF_A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < PF_BK / 32; ++kk) {
-                        tc_mma_i8_ts(d_tmem, tmem + PF_A_COL + s * (PF_BK / 4) + kk * 8,
-                                     smem_desc_k_sw128(bstage + kk * 32), idesc, (ks | kk) != 0 ? 1u : 0u);
+                        tc_mma_i8_ss(d_tmem, smem_desc_k_sw128(astage + kk * 32), smem_desc_k_sw128(bstage + kk * 32),
+                                     idesc, (ks | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit(BAR_EMPTY(s));
+                    tc_commit(BAR_AEMPTY(a));
                     issued = true;
                     last_bar = BAR_EMPTY(s);
                     last_ph = ph;
@@ -270,38 +276,45 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                 if (issued) mbar_wait(last_bar, last_ph, TO, nullptr);
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < PF_EPI_WARP0) {
         // ------------------------------------------------------------ expanders
         const int q = warp & 3;
+        const int parity = (warp - 2) >> 2;  // this warp takes stages with it % 2 == parity
         const int row = q * 32 + lane;
+        const int rsw = row & 7;             // 128-byte swizzle phase of this row
         long long it = 0;
         bool failed = false;
         for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x) {
             for (int ks = 0; ks < KS; ++ks, ++it) {
+                if ((int)(it & 1) != parity) continue;
                 const int s = (int)(it % PF_STAGES);
                 const u32 ph = (u32)((it / PF_STAGES) & 1);
-                bool ok = mbar_wait(BAR_FULL(s), ph, TO, s_abort);
+                const int a = (int)(it % PF_ASTAGES);
+                const u32 aph = (u32)((it / PF_ASTAGES) & 1);
+                // the packed stage has landed and the MMAs that read this A stage before are done
+                bool ok = mbar_wait(BAR_FULL(s), ph, TO, s_abort) && mbar_wait(BAR_AEMPTY(a), aph ^ 1u, TO, s_abort);
                 if (!__all_sync(0xffffffffu, ok)) {
                     failed = true;
                     break;
                 }
-                tc_fence_after();
                 const uint4 *src = reinterpret_cast<const uint4 *>(sm + PF_OFF_P + s * PF_P_BYTES + row * (PF_BK / 4));
                 const uint4 v0 = src[0], v1 = src[1];
                 const u32 w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                u32 r[32];
+                uint8_t *arow = sm + PF_OFF_A + a * PF_A_BYTES + row * 128;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    r[4 * i + 0] = (w[i] << 6) & 0xC0C0C0C0u;
-                    r[4 * i + 1] = (w[i] << 4) & 0xC0C0C0C0u;
-                    r[4 * i + 2] = (w[i] << 2) & 0xC0C0C0C0u;
-                    r[4 * i + 3] = w[i] & 0xC0C0C0C0u;
+                    // packed word i = k 16i .. 16i+15 = 16-byte chunk i of the row
+                    uint4 o;
+                    o.x = (w[i] << 6) & 0xC0C0C0C0u;
+                    o.y = (w[i] << 4) & 0xC0C0C0C0u;
+                    o.z = (w[i] << 2) & 0xC0C0C0C0u;
+                    o.w = w[i] & 0xC0C0C0C0u;
+                    *reinterpret_cast<uint4 *>(arow + ((i ^ rsw) << 4)) = o;
                 }
-                tc_st_32x32b_x32(tmem + ((u32)(q * 32) << 16) + PF_A_COL + s * (PF_BK / 4), r);
-                tc_wait_st();
-                tc_fence_before();
+                // make the generic-proxy stores visible to the tensor core (async proxy)
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(BAR_AREADY(s));
+                if (lane == 0) mbar_arrive(BAR_AREADY(a));
             }
         }
         if (failed && lane == 0) {
@@ -311,7 +324,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
     } else {
         // ------------------------------------------------------------- epilogue
         const int q = warp & 3;
-        const int ew = warp - 6;  // 0..3
+        const int ew = warp - PF_EPI_WARP0;  // 0..3
         const int row = q * 32 + lane;
         float *fbuf = reinterpret_cast<float *>(sm + PF_OFF_F) + ew * 2 * PF_BN;
         const float gamma = *p.gamma;
@@ -320,45 +333,56 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x, ++tc) {
             const int nt = tile % p.n_tiles, mt = tile / p.n_tiles;
             const int b = tc & 1;
-            const u32 aph = (u32)((tc >> 1) & 1);
+            const u32 cph = (u32)((tc >> 1) & 1);
             float *f = fbuf + b * PF_BN;
-            // per-warp copy of float(gamma / s[m]) for this tile's tokens
+            // per-warp copy of float(gamma / s[m]) / 64 (exact) for this tile's tokens
 #pragma unroll
             for (int j = 0; j < PF_BN / 32; ++j) {
                 const int c = j * 32 + lane;
                 const int m = mt * PF_BN + c;
-                f[c] = m < p.M ? __fdiv_rn(gamma, p.s[m]) : 0.f;
+                f[c] = m < p.M ? __fmul_rn(__fdiv_rn(gamma, p.s[m]), 0.015625f) : 0.f;
             }
             __syncwarp();
-            bool ok = mbar_wait(BAR_ACCFULL(b), aph, TO, s_abort);
+            bool ok = mbar_wait(BAR_ACCFULL(b), cph, TO, s_abort);
             if (!__all_sync(0xffffffffu, ok)) {
                 failed = true;
                 break;
             }
             tc_fence_after();
             const int n = nt * PF_BM + row;
+            const int m0 = mt * PF_BN;
             const bool nvalid = n < p.N;
+            const bool full = m0 + PF_BN <= p.M;
+            float *yp = p.Y + (size_t)m0 * p.N + n;
+            int32_t *ap = p.acc ? p.acc + (size_t)m0 * p.N + n : nullptr;
 #pragma unroll 1
             for (int c0 = 0; c0 < PF_BN; c0 += 32) {
                 u32 r[32];
-                tc_ld_32x32b_x32(tmem + ((u32)(q * 32) << 16) + PF_ACC_COL + b * PF_BN + c0, r);
+                tc_ld_32x32b_x32(tmem + ((u32)(q * 32) << 16) + b * PF_BN + c0, r);
                 tc_wait_ld();
                 if (c0 + 32 == PF_BN) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(BAR_ACCEMPTY(b));
                 }
-                const int mbase = mt * PF_BN + c0;
+                if (nvalid) {
+                    const float4 *f4 = reinterpret_cast<const float4 *>(f + c0);
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int m = mbase + j;
-                    if (nvalid && m < p.M) {
-                        const int a = (int)r[j] >> 6;  // exact: the sum is a multiple of 64
-                        const size_t o = (size_t)m * p.N + n;
-                        p.Y[o] = __fmul_rn(__int2float_rn(a), f[c0 + j]);
-                        if (p.acc) p.acc[o] = a;
+                    for (int j4 = 0; j4 < 8; ++j4) {
+                        const float4 ff = f4[j4];
+                        const float fv[4] = {ff.x, ff.y, ff.z, ff.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = j4 * 4 + e;
+                            if (full || m0 + c0 + j < p.M) {
+                                const size_t o = (size_t)(c0 + j) * p.N;
+                                yp[o] = __fmul_rn(__int2float_rn((int)r[j]), fv[e]);
+                                if (ap) ap[o] = (int)r[j] >> 6;  // exact: the sum is a multiple of 64
+                            }
+                        }
                     }
                 }
+                __syncwarp();  // converged before the next tcgen05.ld
             }
             __syncwarp();
         }

@@ -112,52 +112,65 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const uint4 *__r
         s_whi[tid >> 5] = hi;
     }
     __syncthreads();
-    if (tid == 0) {
-        u64 L[WQ_PART_LIMBS] = {0, 0, 0, 0, 0, 0};
-        u64 blo = 0, bhi = 0;
-        for (int w = 0; w < WQ_THREADS / 32; ++w) {
-            u64 s = blo + s_wlo[w];
-            bhi += s_whi[w] + (s < blo ? 1ull : 0ull);
-            blo = s;
-        }
-        // term m << (e - base) stands for m * 2^(e - 150) = term * 2^(base - 1) units
-        limbs_add_u128_shl(L, blo, bhi, base - 1);
-        for (int e = 0; e < 256; ++e) {
-            u64 b = s_bins[e];
-            if (b) limbs_add_u128_shl(L, b, 0ull, e > 0 ? e - 1 : 0);
-        }
+    if (tid < 32) {
+        // warp 0: which exponent bins are non-empty (usually none)
+        u32 nz[8];
 #pragma unroll
-        for (int k = 0; k < WQ_PART_LIMBS; ++k) partials[(size_t)blockIdx.x * WQ_PART_LIMBS + k] = L[k];
+        for (int q = 0; q < 8; ++q) nz[q] = __ballot_sync(0xffffffffu, s_bins[q * 32 + tid] != 0ull);
+        if (tid == 0) {
+            u64 L[WQ_PART_LIMBS] = {0, 0, 0, 0, 0, 0};
+            u64 blo = 0, bhi = 0;
+            for (int w = 0; w < WQ_THREADS / 32; ++w) {
+                u64 sl = blo + s_wlo[w];
+                bhi += s_whi[w] + (sl < blo ? 1ull : 0ull);
+                blo = sl;
+            }
+            // term m << (e - base) stands for m * 2^(e - 150) = term * 2^(base - 1) units
+            limbs_add_u128_shl(L, blo, bhi, base - 1);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                u32 bits = nz[q];
+                while (bits) {
+                    const int e = q * 32 + __ffs(bits) - 1;
+                    bits &= bits - 1;
+                    limbs_add_u128_shl(L, s_bins[e], 0ull, e > 0 ? e - 1 : 0);
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < WQ_PART_LIMBS; ++k) partials[(size_t)blockIdx.x * WQ_PART_LIMBS + k] = L[k];
+        }
     }
 }
 
 // One warp.  Writes gamma and the threshold bits (as u32) into ws_thresh.
+// Each limb position is summed across the block partials as a 128-bit value
+// (lanes, then a shuffle tree), and lane 0 folds the limb sums with carries.
 __global__ void __launch_bounds__(32) k_gamma_finalize(const u64 *__restrict__ partials, int nblocks,
                                                          long long n, float *__restrict__ gamma_out,
                                                          u32 *__restrict__ ws_thresh) {
-    constexpr int NL = WQ_PART_LIMBS + 1;
-    __shared__ u64 s_L[32][NL];
+    constexpr int NL = WQ_PART_LIMBS;
     const int lane = threadIdx.x;
-    u64 L[NL];
+    u64 slo[NL], shi[NL];
 #pragma unroll
-    for (int k = 0; k < NL; ++k) L[k] = 0ull;
+    for (int k = 0; k < NL; ++k) slo[k] = shi[k] = 0ull;
     for (int b = lane; b < nblocks; b += 32) {
-        u64 R[NL];
 #pragma unroll
-        for (int k = 0; k < WQ_PART_LIMBS; ++k) R[k] = partials[(size_t)b * WQ_PART_LIMBS + k];
-        R[NL - 1] = 0ull;
-        limbs_add(L, R);
+        for (int k = 0; k < NL; ++k) {
+            const u64 v = partials[(size_t)b * NL + k];
+            const u64 t = slo[k] + v;
+            shi[k] += t < v ? 1ull : 0ull;
+            slo[k] = t;
+        }
     }
 #pragma unroll
-    for (int k = 0; k < NL; ++k) s_L[lane][k] = L[k];
-    __syncwarp();
+    for (int k = 0; k < NL; ++k) warp_sum_u128(slo[k], shi[k]);
     if (lane == 0) {
-        for (int l = 1; l < 32; ++l) {
-            u64 R[NL];
+        // S = sum_k (shi[k]:slo[k]) << 64k, folded into NL + 2 limbs
+        u64 L[NL + 2];
 #pragma unroll
-            for (int k = 0; k < NL; ++k) R[k] = s_L[l][k];
-            limbs_add(L, R);
-        }
+        for (int k = 0; k < NL + 2; ++k) L[k] = 0ull;
+#pragma unroll
+        for (int k = 0; k < NL; ++k) limbs_add_u128_shl(L, slo[k], shi[k], 64 * k);
         double S = limbs_to_double_rn(L, -149);
         float mean = __double2float_rn(__ddiv_rn(S, (double)n));
         float g = __fadd_rn(mean, 1e-5f);
