@@ -3,31 +3,34 @@
 // What it computes ("bitone" README, How 1.58-bit Works and Forward pass):
 //   acc[m, n] = sum_k x_q[m, k] * W_q[n, k];  Y[m, n] = acc * (gamma / s[m])
 //
-// One output tile = 128 weight rows (n) x 256 tokens (m), computed as
-// Y^T_tile = W_tile * x_q_tile^T with tcgen05.mma.cta_group::1.kind::i8,
-// M = 128, N = 256, K = 32 per instruction (the issue cost of one MMA is
-// nearly independent of N, so N = 256 is what reaches the tensor peak):
-//   A = 64 * W_q as int8 in shared memory: the packed 2-bit rows arrive by
-//     TMA, eight expander warps unpack them ((word << (6 - 2j)) & 0xC0C0C0C0
-//     gives four int8 lanes) and store them in the 128-byte-swizzled K-major
-//     layout the MMA reads, then fence the async proxy;
-//   B = x_q, by TMA with 128-byte swizzle, K-major;
-//   D = int32 accumulators in TMEM, two 256-column buffers so the epilogue
-//     of one tile overlaps the MMAs of the next.
+// One output tile = 128 tokens (m) x 256 weight rows (n), computed with
+// tcgen05.mma.cta_group::1.kind::i8, M = 128, N = 256, K = 32 per
+// instruction (the issue cost of one MMA is nearly independent of N, so
+// N = 256 is what reaches the tensor peak):
+//   A = x_q tile, by TMA with 128-byte swizzle, K-major;
+//   B = 64 * W_q as int8 in shared memory: the packed 2-bit rows arrive by
+//     TMA, eight expander warps (one weight row per thread) unpack them
+//     ((word << (6 - 2j)) & 0xC0C0C0C0 gives four int8 lanes), store them in
+//     the 128-byte-swizzled K-major layout the MMA reads, then fence the
+//     async proxy;
+//   D = int32 accumulators in TMEM (lane = token, column = weight row), two
+//     256-column buffers so the epilogue of one tile overlaps the MMAs of the
+//     next.  Each epilogue thread owns one token: one float(gamma / s[m])
+//     per tile and contiguous outputs, written with 16-byte stores.
 // The exact sum is 64 * acc (|64 acc| <= 2^28, exact in int32 and in
 // float), so Y = float(float(64 acc) * (f / 64)) with f = float(gamma / s[m])
 // (f / 64 is exact) -- the same bits as float(acc) * f.
 //
 // Pipelines: PF_STAGES shared-memory stages carry x_q and packed tiles from
-// TMA; PF_ASTAGES shared-memory stages carry the expanded weights from the
+// TMA; PF_BSTAGES shared-memory stages carry the expanded weights from the
 // expanders to the MMA.  MMA completion frees both (two commits).
 //
 // Warp roles (persistent: one CTA per SM loops over tiles):
-//   warp 0       TMA producer (one thread)
-//   warp 1       TMEM allocator + MMA issuer (one thread)
-//   warps 2..9   expanders: weight rows 32*(w % 4) .. +31; two warps per
-//                row quarter take alternate pipeline stages
-//   warps 10..13 epilogue: TMEM lanes 32*(w % 4) .. +31 (= weight rows)
+//   warp 0        TMA producer (one thread)
+//   warp 1        TMEM allocator + MMA issuer (one thread)
+//   warps 2..9    expanders: weight row 32*(w - 2) + lane of the tile
+//   warps 10..17  epilogue: TMEM lanes 32*(w % 4) .. +31 (tokens), columns
+//                 128*((w - 10) / 4) .. +127 (weight rows)
 // Every mbarrier wait is bounded (globaltimer); a wait that gives up raises
 // the device error word, sets a CTA abort flag and the CTA drains its
 // in-flight copies and MMAs (again with bounded waits) before it frees TMEM
@@ -40,32 +43,31 @@
 
 namespace bl {
 
-constexpr int PF_BM = 128;         // weight rows per tile (MMA M, TMEM lanes)
-constexpr int PF_BN = 256;         // tokens per tile (MMA N)
+constexpr int PF_BM = 128;         // tokens per tile (MMA M, TMEM lanes)
+constexpr int PF_BN = 256;         // weight rows per tile (MMA N, TMEM columns)
 constexpr int PF_BK = 128;         // k per pipeline stage (4 MMAs of K = 32)
 constexpr int PF_STAGES = 4;       // TMA stages (x_q + packed)
-constexpr int PF_ASTAGES = 3;      // expanded-weight stages
-constexpr int PF_THREADS = 448;
-constexpr int PF_EXP_WARPS = 8;    // expander warps (2 per row quarter)
+constexpr int PF_BSTAGES = 3;      // expanded-weight stages
+constexpr int PF_EXP_WARPS = PF_BN / 32;
+constexpr int PF_EPI_WARPS = 8;
 constexpr int PF_EPI_WARP0 = 2 + PF_EXP_WARPS;
-constexpr int PF_B_BYTES = PF_BN * PF_BK;          // x_q stage: 32 KiB
-constexpr int PF_A_BYTES = PF_BM * PF_BK;          // expanded stage: 16 KiB
-constexpr int PF_P_BYTES = PF_BM * PF_BK / 4;      // packed stage: 4 KiB
+constexpr int PF_THREADS = 32 * (PF_EPI_WARP0 + PF_EPI_WARPS);
+constexpr int PF_A_BYTES = PF_BM * PF_BK;          // x_q stage: 16 KiB
+constexpr int PF_P_BYTES = PF_BN * PF_BK / 4;      // packed stage: 8 KiB
+constexpr int PF_B_BYTES = PF_BN * PF_BK;          // expanded stage: 32 KiB
 constexpr int PF_TMEM_COLS = 512;                  // 2 x 256 accumulator columns
 
 // shared memory carve-up (offsets from a 1024-byte aligned base)
-constexpr int PF_OFF_B = 0;
-constexpr int PF_OFF_A = PF_OFF_B + PF_STAGES * PF_B_BYTES;
-constexpr int PF_OFF_P = PF_OFF_A + PF_ASTAGES * PF_A_BYTES;
-constexpr int PF_OFF_F = PF_OFF_P + PF_STAGES * PF_P_BYTES;           // [4 warps][2][256] float
-constexpr int PF_OFF_BAR = PF_OFF_F + 4 * 2 * PF_BN * 4;
-constexpr int PF_NBAR = 2 * PF_STAGES + 2 * PF_ASTAGES + 4;           // full, empty, aready, aempty, accfull x2, accempty x2
+constexpr int PF_OFF_A = 0;
+constexpr int PF_OFF_B = PF_OFF_A + PF_STAGES * PF_A_BYTES;
+constexpr int PF_OFF_P = PF_OFF_B + PF_BSTAGES * PF_B_BYTES;
+constexpr int PF_OFF_BAR = PF_OFF_P + PF_STAGES * PF_P_BYTES;
+constexpr int PF_NBAR = 2 * PF_STAGES + 2 * PF_BSTAGES + 4;  // full, empty, bready, bempty, accfull x2, accempty x2
 constexpr int PF_OFF_MISC = PF_OFF_BAR + PF_NBAR * 8;
 constexpr int PF_SMEM_USED = PF_OFF_MISC + 16;
 constexpr int PF_SMEM_BYTES = PF_SMEM_USED + 1024;                     // + alignment slack
 static_assert(PF_SMEM_BYTES > 116 * 1024, "keeps one CTA per SM, so the TMEM allocation never waits");
 static_assert(PF_SMEM_BYTES <= 227 * 1024, "shared memory budget");
-static_assert(PF_ASTAGES >= 2, "expander warp pairs alternate stages");
 
 struct PrefillParams {
     const float *gamma;
@@ -135,7 +137,7 @@ __device__ __forceinline__ unsigned long long smem_desc_k_sw128(u32 saddr) {
     return d;
 }
 
-// Instruction descriptor, kind::i8: D s32, A s8, B s8, both K-major, N = PF_BN, M = 128.
+// Instruction descriptor, kind::i8: D s32, A s8, B s8, both K-major, N = PF_BN, M = PF_BM.
 __host__ __device__ constexpr u32 pf_idesc() {
     return (2u << 4)                    // D format: s32
            | (1u << 7)                  // A format: signed 8-bit
@@ -155,10 +157,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
     const u32 bar0 = sbase + PF_OFF_BAR;
     auto BAR_FULL = [&](int s) { return bar0 + 8u * s; };
     auto BAR_EMPTY = [&](int s) { return bar0 + 8u * (PF_STAGES + s); };
-    auto BAR_AREADY = [&](int a) { return bar0 + 8u * (2 * PF_STAGES + a); };
-    auto BAR_AEMPTY = [&](int a) { return bar0 + 8u * (2 * PF_STAGES + PF_ASTAGES + a); };
-    auto BAR_ACCFULL = [&](int b) { return bar0 + 8u * (2 * PF_STAGES + 2 * PF_ASTAGES + b); };
-    auto BAR_ACCEMPTY = [&](int b) { return bar0 + 8u * (2 * PF_STAGES + 2 * PF_ASTAGES + 2 + b); };
+    auto BAR_BREADY = [&](int a) { return bar0 + 8u * (2 * PF_STAGES + a); };
+    auto BAR_BEMPTY = [&](int a) { return bar0 + 8u * (2 * PF_STAGES + PF_BSTAGES + a); };
+    auto BAR_ACCFULL = [&](int b) { return bar0 + 8u * (2 * PF_STAGES + 2 * PF_BSTAGES + b); };
+    auto BAR_ACCEMPTY = [&](int b) { return bar0 + 8u * (2 * PF_STAGES + 2 * PF_BSTAGES + 2 + b); };
     u32 *s_tmem = reinterpret_cast<u32 *>(sm + PF_OFF_MISC);
     volatile int *s_abort = reinterpret_cast<volatile int *>(sm + PF_OFF_MISC + 4);
 
@@ -168,13 +170,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
             mbar_init(BAR_FULL(s), 1);
             mbar_init(BAR_EMPTY(s), 1);
         }
-        for (int a = 0; a < PF_ASTAGES; ++a) {
-            mbar_init(BAR_AREADY(a), 4);
-            mbar_init(BAR_AEMPTY(a), 1);
+        for (int a = 0; a < PF_BSTAGES; ++a) {
+            mbar_init(BAR_BREADY(a), PF_EXP_WARPS);
+            mbar_init(BAR_BEMPTY(a), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(BAR_ACCFULL(b), 1);
-            mbar_init(BAR_ACCEMPTY(b), 4);
+            mbar_init(BAR_ACCEMPTY(b), PF_EPI_WARPS);
         }
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -210,9 +212,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                         break;
                     }
                     if (it == p.dbg_skip_iter) continue;  // test hook: this stage never arrives
-                    mbar_arrive_expect_tx(BAR_FULL(s), PF_B_BYTES + PF_P_BYTES);
-                    tma_load_2d(sbase + PF_OFF_B + s * PF_B_BYTES, &tm_x, ks * PF_BK, mt * PF_BN, BAR_FULL(s));
-                    tma_load_2d(sbase + PF_OFF_P + s * PF_P_BYTES, &tm_w, ks * (PF_BK / 4), nt * PF_BM, BAR_FULL(s));
+                    mbar_arrive_expect_tx(BAR_FULL(s), PF_A_BYTES + PF_P_BYTES);
+                    tma_load_2d(sbase + PF_OFF_A + s * PF_A_BYTES, &tm_x, ks * PF_BK, mt * PF_BM, BAR_FULL(s));
+                    tma_load_2d(sbase + PF_OFF_P + s * PF_P_BYTES, &tm_w, ks * (PF_BK / 4), nt * PF_BN, BAR_FULL(s));
                 }
             }
             if (failed) {
@@ -246,22 +248,22 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                 for (int ks = 0; ks < KS; ++ks, ++it) {
                     const int s = (int)(it % PF_STAGES);
                     const u32 ph = (u32)((it / PF_STAGES) & 1);
-                    const int a = (int)(it % PF_ASTAGES);
-                    const u32 aph = (u32)((it / PF_ASTAGES) & 1);
-                    if (!mbar_wait(BAR_FULL(s), ph, TO, s_abort) || !mbar_wait(BAR_AREADY(a), aph, TO, s_abort)) {
+                    const int a = (int)(it % PF_BSTAGES);
+                    const u32 aph = (u32)((it / PF_BSTAGES) & 1);
+                    if (!mbar_wait(BAR_FULL(s), ph, TO, s_abort) || !mbar_wait(BAR_BREADY(a), aph, TO, s_abort)) {
                         failed = true;
                         break;
                     }
                     tc_fence_after();
-                    const u32 bstage = sbase + PF_OFF_B + s * PF_B_BYTES;
-                    const u32 astage = sbase + PF_OFF_A + a * PF_A_BYTES;
+                    const u32 astage = sbase + PF_OFF_A + s * PF_A_BYTES;
+                    const u32 bstage = sbase + PF_OFF_B + a * PF_B_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < PF_BK / 32; ++kk) {
                         tc_mma_i8_ss(d_tmem, smem_desc_k_sw128(astage + kk * 32), smem_desc_k_sw128(bstage + kk * 32),
                                      idesc, (ks | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit(BAR_EMPTY(s));
-                    tc_commit(BAR_AEMPTY(a));
+                    tc_commit(BAR_BEMPTY(a));
                     issued = true;
                     last_bar = BAR_EMPTY(s);
                     last_ph = ph;
@@ -278,21 +280,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         }
     } else if (warp < PF_EPI_WARP0) {
         // ------------------------------------------------------------ expanders
-        const int q = warp & 3;
-        const int parity = (warp - 2) >> 2;  // this warp takes stages with it % 2 == parity
-        const int row = q * 32 + lane;
-        const int rsw = row & 7;             // 128-byte swizzle phase of this row
+        const int row = (warp - 2) * 32 + lane;  // weight row within the tile
+        const int rsw = row & 7;                 // 128-byte swizzle phase of this row
         long long it = 0;
         bool failed = false;
         for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x) {
             for (int ks = 0; ks < KS; ++ks, ++it) {
-                if ((int)(it & 1) != parity) continue;
                 const int s = (int)(it % PF_STAGES);
                 const u32 ph = (u32)((it / PF_STAGES) & 1);
-                const int a = (int)(it % PF_ASTAGES);
-                const u32 aph = (u32)((it / PF_ASTAGES) & 1);
-                // the packed stage has landed and the MMAs that read this A stage before are done
-                bool ok = mbar_wait(BAR_FULL(s), ph, TO, s_abort) && mbar_wait(BAR_AEMPTY(a), aph ^ 1u, TO, s_abort);
+                const int a = (int)(it % PF_BSTAGES);
+                const u32 aph = (u32)((it / PF_BSTAGES) & 1);
+                // the packed stage has landed and the MMAs that read this B stage before are done
+                bool ok = mbar_wait(BAR_FULL(s), ph, TO, s_abort) && mbar_wait(BAR_BEMPTY(a), aph ^ 1u, TO, s_abort);
                 if (!__all_sync(0xffffffffu, ok)) {
                     failed = true;
                     break;
@@ -300,7 +299,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                 const uint4 *src = reinterpret_cast<const uint4 *>(sm + PF_OFF_P + s * PF_P_BYTES + row * (PF_BK / 4));
                 const uint4 v0 = src[0], v1 = src[1];
                 const u32 w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                uint8_t *arow = sm + PF_OFF_A + a * PF_A_BYTES + row * 128;
+                uint8_t *brow = sm + PF_OFF_B + a * PF_B_BYTES + row * 128;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     // packed word i = k 16i .. 16i+15 = 16-byte chunk i of the row
@@ -309,12 +308,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                     o.y = (w[i] << 4) & 0xC0C0C0C0u;
                     o.z = (w[i] << 2) & 0xC0C0C0C0u;
                     o.w = w[i] & 0xC0C0C0C0u;
-                    *reinterpret_cast<uint4 *>(arow + ((i ^ rsw) << 4)) = o;
+                    *reinterpret_cast<uint4 *>(brow + ((i ^ rsw) << 4)) = o;
                 }
                 // make the generic-proxy stores visible to the tensor core (async proxy)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(BAR_AREADY(a));
+                if (lane == 0) mbar_arrive(BAR_BREADY(a));
             }
         }
         if (failed && lane == 0) {
@@ -323,68 +322,68 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         }
     } else {
         // ------------------------------------------------------------- epilogue
-        const int q = warp & 3;
-        const int ew = warp - PF_EPI_WARP0;  // 0..3
-        const int row = q * 32 + lane;
-        float *fbuf = reinterpret_cast<float *>(sm + PF_OFF_F) + ew * 2 * PF_BN;
+        const int q = warp & 3;                           // TMEM lane quarter = token block
+        const int half = (warp - PF_EPI_WARP0) >> 2;      // weight-row half of the tile
         const float gamma = *p.gamma;
+        const bool vec_ok = (p.N & 3) == 0;               // rows of Y 16-byte aligned
         int tc = 0;
         bool failed = false;
         for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x, ++tc) {
             const int nt = tile % p.n_tiles, mt = tile / p.n_tiles;
             const int b = tc & 1;
             const u32 cph = (u32)((tc >> 1) & 1);
-            float *f = fbuf + b * PF_BN;
-            // per-warp copy of float(gamma / s[m]) / 64 (exact) for this tile's tokens
-#pragma unroll
-            for (int j = 0; j < PF_BN / 32; ++j) {
-                const int c = j * 32 + lane;
-                const int m = mt * PF_BN + c;
-                f[c] = m < p.M ? __fmul_rn(__fdiv_rn(gamma, p.s[m]), 0.015625f) : 0.f;
-            }
-            __syncwarp();
+            const int m = mt * PF_BM + q * 32 + lane;     // this thread's token
+            const bool mvalid = m < p.M;
+            // float(gamma / s[m]) / 64 (exact)
+            const float f = mvalid ? __fmul_rn(__fdiv_rn(gamma, p.s[m]), 0.015625f) : 0.f;
             bool ok = mbar_wait(BAR_ACCFULL(b), cph, TO, s_abort);
             if (!__all_sync(0xffffffffu, ok)) {
                 failed = true;
                 break;
             }
             tc_fence_after();
-            const int n = nt * PF_BM + row;
-            const int m0 = mt * PF_BN;
-            const bool nvalid = n < p.N;
-            const bool full = m0 + PF_BN <= p.M;
-            float *yp = p.Y + (size_t)m0 * p.N + n;
-            int32_t *ap = p.acc ? p.acc + (size_t)m0 * p.N + n : nullptr;
+            const int n0 = nt * PF_BN + half * (PF_BN / 2);
+            const bool full = vec_ok && n0 + PF_BN / 2 <= p.N;
+            float *yrow = p.Y + (size_t)m * p.N + n0;
+            int32_t *arow = p.acc ? p.acc + (size_t)m * p.N + n0 : nullptr;
 #pragma unroll 1
-            for (int c0 = 0; c0 < PF_BN; c0 += 32) {
+            for (int c0 = 0; c0 < PF_BN / 2; c0 += 32) {
                 u32 r[32];
-                tc_ld_32x32b_x32(tmem + ((u32)(q * 32) << 16) + b * PF_BN + c0, r);
+                tc_ld_32x32b_x32(tmem + ((u32)(q * 32) << 16) + b * PF_BN + half * (PF_BN / 2) + c0, r);
                 tc_wait_ld();
-                if (c0 + 32 == PF_BN) {
+                if (c0 + 32 == PF_BN / 2) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(BAR_ACCEMPTY(b));
                 }
-                if (nvalid) {
-                    const float4 *f4 = reinterpret_cast<const float4 *>(f + c0);
+                if (mvalid) {
+                    if (full) {
 #pragma unroll
-                    for (int j4 = 0; j4 < 8; ++j4) {
-                        const float4 ff = f4[j4];
-                        const float fv[4] = {ff.x, ff.y, ff.z, ff.w};
+                        for (int j = 0; j < 32; j += 4) {
+                            float4 o;
+                            o.x = __fmul_rn(__int2float_rn((int)r[j + 0]), f);
+                            o.y = __fmul_rn(__int2float_rn((int)r[j + 1]), f);
+                            o.z = __fmul_rn(__int2float_rn((int)r[j + 2]), f);
+                            o.w = __fmul_rn(__int2float_rn((int)r[j + 3]), f);
+                            *reinterpret_cast<float4 *>(yrow + c0 + j) = o;
+                            if (arow) {
+                                // exact: the sums are multiples of 64
+                                *reinterpret_cast<int4 *>(arow + c0 + j) =
+                                    make_int4((int)r[j] >> 6, (int)r[j + 1] >> 6, (int)r[j + 2] >> 6, (int)r[j + 3] >> 6);
+                            }
+                        }
+                    } else {
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = j4 * 4 + e;
-                            if (full || m0 + c0 + j < p.M) {
-                                const size_t o = (size_t)(c0 + j) * p.N;
-                                yp[o] = __fmul_rn(__int2float_rn((int)r[j]), fv[e]);
-                                if (ap) ap[o] = (int)r[j] >> 6;  // exact: the sum is a multiple of 64
+                        for (int j = 0; j < 32; ++j) {
+                            if (n0 + c0 + j < p.N) {
+                                yrow[c0 + j] = __fmul_rn(__int2float_rn((int)r[j]), f);
+                                if (arow) arow[c0 + j] = (int)r[j] >> 6;
                             }
                         }
                     }
                 }
                 __syncwarp();  // converged before the next tcgen05.ld
             }
-            __syncwarp();
         }
         if (failed && lane == 0) {
             raise_device_error(DEVERR_TIMEOUT_EPILOGUE);
@@ -442,14 +441,14 @@ inline bl_status prefill_launch(int sms, const uint8_t *packed, const float *gam
                                 unsigned long long timeout_ns = PF_DEFAULT_TIMEOUT_NS, long long dbg_skip_iter = -1) {
     EncodeTiledFn enc = encode_tiled_fn();
     if (enc == nullptr) return BL_ERR_CUDA;
-    const int64_t n_tiles = (N + PF_BM - 1) / PF_BM, m_tiles = (M + PF_BN - 1) / PF_BN;
+    const int64_t n_tiles = (N + PF_BN - 1) / PF_BN, m_tiles = (M + PF_BM - 1) / PF_BM;
     if (n_tiles * m_tiles > 0x7fffffffLL) return BL_ERR_SHAPE;
     CUtensorMap tx, tw;
     const cuuint32_t es[2] = {1, 1};
     {
         const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
         const cuuint64_t gstride[1] = {(cuuint64_t)K};
-        const cuuint32_t box[2] = {(cuuint32_t)PF_BK, (cuuint32_t)PF_BN};
+        const cuuint32_t box[2] = {(cuuint32_t)PF_BK, (cuuint32_t)PF_BM};
         if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(x_q), gdim, gstride, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -458,7 +457,7 @@ inline bl_status prefill_launch(int sms, const uint8_t *packed, const float *gam
     {
         const cuuint64_t gdim[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
         const cuuint64_t gstride[1] = {(cuuint64_t)(K / 4)};
-        const cuuint32_t box[2] = {(cuuint32_t)(PF_BK / 4), (cuuint32_t)PF_BM};
+        const cuuint32_t box[2] = {(cuuint32_t)(PF_BK / 4), (cuuint32_t)PF_BN};
         if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
