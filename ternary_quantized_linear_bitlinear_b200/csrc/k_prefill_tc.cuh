@@ -15,8 +15,10 @@
 //     async proxy;
 //   D = int32 accumulators in TMEM (lane = token, column = weight row), two
 //     256-column buffers so the epilogue of one tile overlaps the MMAs of the
-//     next.  Each epilogue thread owns one token: one float(gamma / s[m])
-//     per tile and contiguous outputs, written with 16-byte stores.
+//     next.  Each epilogue thread owns one token (one float(gamma / s[m]) per
+//     tile); a warp converts a 32 x 32 block into a 128B-swizzled staging
+//     buffer and one lane writes it to Y with a TMA tensor store, so every
+//     store is a full-line bulk write (tails clipped by the tensor map).
 // The exact sum is 64 * acc (|64 acc| <= 2^28, exact in int32 and in
 // float), so Y = float(float(64 acc) * (f / 64)) with f = float(gamma / s[m])
 // (f / 64 is exact) -- the same bits as float(acc) * f.
@@ -46,7 +48,7 @@ namespace bl {
 constexpr int PF_BM = 128;         // tokens per tile (MMA M, TMEM lanes)
 constexpr int PF_BN = 256;         // weight rows per tile (MMA N, TMEM columns)
 constexpr int PF_BK = 128;         // k per pipeline stage (4 MMAs of K = 32)
-constexpr int PF_STAGES = 4;       // TMA stages (x_q + packed)
+constexpr int PF_STAGES = 3;       // TMA stages (x_q + packed)
 constexpr int PF_BSTAGES = 3;      // expanded-weight stages
 constexpr int PF_EXP_WARPS = PF_BN / 32;
 constexpr int PF_EPI_WARPS = 8;
@@ -56,12 +58,14 @@ constexpr int PF_A_BYTES = PF_BM * PF_BK;          // x_q stage: 16 KiB
 constexpr int PF_P_BYTES = PF_BN * PF_BK / 4;      // packed stage: 8 KiB
 constexpr int PF_B_BYTES = PF_BN * PF_BK;          // expanded stage: 32 KiB
 constexpr int PF_TMEM_COLS = 512;                  // 2 x 256 accumulator columns
+constexpr int PF_Y_BYTES = 32 * 32 * 4;            // per-epilogue-warp Y staging block (TMA store)
 
 // shared memory carve-up (offsets from a 1024-byte aligned base)
 constexpr int PF_OFF_A = 0;
 constexpr int PF_OFF_B = PF_OFF_A + PF_STAGES * PF_A_BYTES;
 constexpr int PF_OFF_P = PF_OFF_B + PF_BSTAGES * PF_B_BYTES;
-constexpr int PF_OFF_BAR = PF_OFF_P + PF_STAGES * PF_P_BYTES;
+constexpr int PF_OFF_Y = PF_OFF_P + PF_STAGES * PF_P_BYTES;             // [8 warps][32 x 32] float, 128B-swizzled
+constexpr int PF_OFF_BAR = PF_OFF_Y + PF_EPI_WARPS * PF_Y_BYTES;
 constexpr int PF_NBAR = 2 * PF_STAGES + 2 * PF_BSTAGES + 4;  // full, empty, bready, bempty, accfull x2, accempty x2
 constexpr int PF_OFF_MISC = PF_OFF_BAR + PF_NBAR * 8;
 constexpr int PF_SMEM_USED = PF_OFF_MISC + 16;
@@ -78,6 +82,7 @@ struct PrefillParams {
     int n_tiles, m_tiles, k_stages;
     unsigned long long timeout_ns;
     long long dbg_skip_iter;  // >= 0: the producer never issues this k-iteration (bounded-wait test)
+    int y_tma;                // 1: Y written by TMA stores through tm_y (N % 4 == 0 and no acc output)
 };
 
 // ---------------------------------------------------------------------------
@@ -88,6 +93,15 @@ __device__ __forceinline__ void tma_load_2d(u32 dst, const CUtensorMap *map, int
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
         ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar)
         : "memory");
+}
+
+// Y block store: shared (128B-swizzled 32 x 32 floats) -> global through the
+// tensor map; out-of-range rows / columns of the box are not written.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int y, u32 src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+                 ::"l"(map), "r"(x), "r"(y), "r"(src)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -150,6 +164,7 @@ __host__ __device__ constexpr u32 pf_idesc() {
 
 __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_constant__ CUtensorMap tm_x,
                                                                const __grid_constant__ CUtensorMap tm_w,
+                                                               const __grid_constant__ CUtensorMap tm_y,
                                                                const __grid_constant__ PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -182,6 +197,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_x) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_w) : "memory");
+        if (p.y_tma) asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_y) : "memory");
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
@@ -323,9 +339,12 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
     } else {
         // ------------------------------------------------------------- epilogue
         const int q = warp & 3;                           // TMEM lane quarter = token block
-        const int half = (warp - PF_EPI_WARP0) >> 2;      // weight-row half of the tile
+        const int ew = warp - PF_EPI_WARP0;               // 0..7
+        const int half = ew >> 2;                         // weight-row half of the tile
         const float gamma = *p.gamma;
         const bool vec_ok = (p.N & 3) == 0;               // rows of Y 16-byte aligned
+        uint8_t *ystage = sm + PF_OFF_Y + ew * PF_Y_BYTES;
+        const u32 ystage_s = smem_u32(ystage);
         int tc = 0;
         bool failed = false;
         for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x, ++tc) {
@@ -356,7 +375,23 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                     __syncwarp();
                     if (lane == 0) mbar_arrive(BAR_ACCEMPTY(b));
                 }
-                if (mvalid) {
+                if (p.y_tma) {
+                    // the previous TMA store from this block has finished reading it
+                    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    __syncwarp();
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        float4 o;
+                        o.x = __fmul_rn(__int2float_rn((int)r[4 * c + 0]), f);
+                        o.y = __fmul_rn(__int2float_rn((int)r[4 * c + 1]), f);
+                        o.z = __fmul_rn(__int2float_rn((int)r[4 * c + 2]), f);
+                        o.w = __fmul_rn(__int2float_rn((int)r[4 * c + 3]), f);
+                        *reinterpret_cast<float4 *>(ystage + lane * 128 + ((c ^ (lane & 7)) << 4)) = o;
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) tma_store_2d(&tm_y, n0 + c0, mt * PF_BM + q * 32, ystage_s);
+                } else if (mvalid) {
                     if (full) {
 #pragma unroll
                         for (int j = 0; j < 32; j += 4) {
@@ -385,6 +420,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                 __syncwarp();  // converged before the next tcgen05.ld
             }
         }
+        // every TMA store of this warp has completed before the CTA exits
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        __syncwarp();
         if (failed && lane == 0) {
             raise_device_error(DEVERR_TIMEOUT_EPILOGUE);
             *s_abort = 1;
@@ -406,6 +444,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
 
 #include <cudaTypedefs.h>
 
+#include <cstring>
 #include <mutex>
 
 namespace bl {
@@ -463,7 +502,21 @@ inline bl_status prefill_launch(int sms, const uint8_t *packed, const float *gam
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return BL_ERR_CUDA;
     }
+    // Y through TMA stores when its rows are 16-byte multiples and no acc output is requested
+    CUtensorMap ty;
+    memset(&ty, 0, sizeof(ty));
+    const int y_tma = (N % 4 == 0 && acc_out == nullptr) ? 1 : 0;
+    if (y_tma) {
+        const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)N * 4};
+        const cuuint32_t box[2] = {32, 32};
+        if (enc(&ty, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, Y, gdim, gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+            CUDA_SUCCESS)
+            return BL_ERR_CUDA;
+    }
     PrefillParams p;
+    p.y_tma = y_tma;
     p.gamma = gamma;
     p.s = s;
     p.Y = Y;
@@ -478,7 +531,7 @@ inline bl_status prefill_launch(int sms, const uint8_t *packed, const float *gam
     p.dbg_skip_iter = dbg_skip_iter;
     const int64_t tiles = n_tiles * m_tiles;
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    k_prefill_tc<<<grid, PF_THREADS, PF_SMEM_BYTES, st>>>(tx, tw, p);
+    k_prefill_tc<<<grid, PF_THREADS, PF_SMEM_BYTES, st>>>(tx, tw, ty, p);
     return cudaGetLastError() == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 
