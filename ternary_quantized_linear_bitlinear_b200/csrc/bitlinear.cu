@@ -174,7 +174,7 @@ bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st) {
     for (int i = 0; i < P.count; ++i) {
         DecodeProblem &q = P.p[i];
         q.g_log2 = dec_glog(q.K);
-        int tiles = (q.N + 15) / 16;
+        int tiles = (q.N + DEC_ROWS - 1) / DEC_ROWS;
         int per = DEC_WARPS >> q.g_log2;
         q.cta_begin = total;
         total += (tiles + per - 1) / per;

@@ -5,13 +5,14 @@
 //
 // The work is bound by streaming the packed weights from HBM (2 bits per
 // weight).  Design:
-//   - A CTA (8 warps) owns T = 8/G consecutive 16-row tiles of one problem;
+//   - A CTA (8 warps) owns 8/G consecutive 32-row groups of one problem;
 //     their packed rows are one contiguous byte range, which one thread
 //     requests with cp.async.bulk copies into shared memory (one mbarrier per
 //     tile, bounded waits), so the memory system sees a few large requests
 //     per CTA and the warps issue no global loads for weights.
-//   - A warp owns a 16-row tile; G warps split its K range (G picked per
-//     problem from K so that each warp has at most 4 steps of 256 k).
+//   - A warp owns 32 rows (two 16-row MMA tiles that share every x_q
+//     fragment); G warps split their K range (G picked per problem from K so
+//     that each warp has at most 4 steps of 256 k).
 //   - Unpacking costs 1-2 ALU ops per 4 weights: with the packed layout, word
 //     (w << (6 - 2j)) & 0xC0C0C0C0 puts the codes of k = 16w' + 4j .. 4j+3 in
 //     the top two bits of four bytes, i.e. the int8 values 64 * W_q.
@@ -71,8 +72,10 @@ __host__ __device__ inline int dec_glog(int K) {
     return g;
 }
 
+constexpr int DEC_ROWS = 32;  // weight rows per warp
+
 // bytes of packed weights one CTA stages
-__host__ __device__ inline int dec_w_bytes(int K) { return (DEC_WARPS >> dec_glog(K)) * 16 * (K >> 2); }
+__host__ __device__ inline int dec_w_bytes(int K) { return (DEC_WARPS >> dec_glog(K)) * DEC_ROWS * (K >> 2); }
 
 __device__ __forceinline__ u32 dec_unpack(u32 w, int j) {
     // codes of k = 4j .. 4j+3 of this 16-weight word -> int8 lanes holding 64 * W_q
@@ -91,9 +94,12 @@ __device__ __forceinline__ void mma_s8_16832(int (&c)[4], u32 a0, u32 a1, u32 a2
 template <int NT>
 __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ DecodeParams P) {
     extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int s_red[DEC_WARPS][NT][4][32];
+    __shared__ int s_red[DEC_WARPS][2][NT][4][32];
     __shared__ __align__(8) u64 s_bar[DEC_WARPS];
     __shared__ float s_f[16];
+
+    // a programmatically dependent launch that follows may start its prologue
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     const int b = blockIdx.x;
     int pi;
@@ -110,25 +116,25 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
     const DecodeProblem &pr = P.p[pi];
     const int M = P.M, N = pr.N, K = pr.K;
     const int glog = pr.g_log2, G = 1 << glog;
-    const int T = DEC_WARPS >> glog;
-    const int Kw = K >> 2;         // packed bytes per row
-    const int row_base = (b - pr.cta_begin) * T * 16;
-    const int rows = min(T * 16, N - row_base);
-    const int tiles = (rows + 15) >> 4;
+    const int T = DEC_WARPS >> glog;  // 32-row groups per CTA
+    const int Kw = K >> 2;            // packed bytes per row
+    const int row_base = (b - pr.cta_begin) * T * DEC_ROWS;
+    const int rows = min(T * DEC_ROWS, N - row_base);
+    const int groups = (rows + DEC_ROWS - 1) / DEC_ROWS;
 
     // One thread requests the CTA's weight rows, one bulk copy (and one
-    // mbarrier) per 16-row tile, so each warp starts as soon as its tile lands.
+    // mbarrier) per 32-row group, so each warp starts as soon as its rows land.
     if (threadIdx.x == 0) {
-        for (int i = 0; i < tiles; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
+        for (int i = 0; i < groups; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         const uint8_t *src = pr.packed + (size_t)row_base * Kw;
         const u32 dst = smem_u32(smem);
-        for (int i = 0; i < tiles; ++i) {
-            const u32 nrows = (u32)min(16, rows - 16 * i);
+        for (int i = 0; i < groups; ++i) {
+            const u32 nrows = (u32)min(DEC_ROWS, rows - DEC_ROWS * i);
             const u32 bytes = nrows * (u32)Kw;
             const u32 bar = smem_u32(&s_bar[i]);
             mbar_arrive_expect_tx(bar, bytes);
-            const u32 off0 = (u32)(16 * i) * (u32)Kw;
+            const u32 off0 = (u32)(DEC_ROWS * i) * (u32)Kw;
             for (u32 off = 0; off < bytes; off += 32768u) {
                 const u32 n = bytes - off < 32768u ? bytes - off : 32768u;
                 bulk_g2s(dst + off0 + off, src + off0 + off, n, bar);
@@ -169,27 +175,30 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int wt = warp >> glog, kslot = warp & (G - 1);
-    const int row0 = wt * 16;  // within the CTA
+    const int wg = warp >> glog, kslot = warp & (G - 1);
+    const int row0 = wg * DEC_ROWS;  // within the CTA
     const int steps = (K + 255) >> 8;
     const int nchunk64 = K >> 6;
 
-    // two independent accumulator chains (even / odd 16-k chunks)
-    int acc[NT][4], acc2[NT][4];
+    // acc[tile][nt][4]: two 16-row tiles, each with two independent chains
+    int acc[2][NT][4], acc2[2][NT][4];
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][i] = acc2[nt][i] = 0;
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[u][nt][i] = acc2[u][nt][i] = 0;
 
     bool ok = true;
-    if (wt < tiles) {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&s_bar[wt]), 0, DEC_TIMEOUT_NS, nullptr));
+    if (wg < groups) {
+        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&s_bar[wg]), 0, DEC_TIMEOUT_NS, nullptr));
         if (!ok && lane == 0) raise_device_error(DEVERR_TIMEOUT_PRODUCER);
     }
 
-    if (ok && wt < tiles) {
-        const uint8_t *wA = smem + (row0 + g) * Kw + t * 16;
-        const uint8_t *wB = smem + (row0 + g + 8) * Kw + t * 16;
+    if (ok && wg < groups) {
+        // rows g, g+8 (tile 0) and g+16, g+24 (tile 1)
+        const uint8_t *w0 = smem + (row0 + g) * Kw + t * 16;
+        const int Kw8 = 8 * Kw;
         // B fragments: token rows g (and g + 8); chunk c of a step sits at
         // 16 * (4t + (c ^ xb)) within the step's 256 bytes (the swizzle)
         const bool tv0 = g < M, tv1 = NT > 1 && g + 8 < M;
@@ -206,10 +215,10 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
 #pragma unroll 2
         for (int s2 = kslot; s2 < steps; s2 += G) {
             const bool kv = (s2 * 4 + t) < nchunk64;
-            const uint4 va = kv ? *reinterpret_cast<const uint4 *>(wA + s2 * 64) : make_uint4(0, 0, 0, 0);
-            const uint4 vb = kv ? *reinterpret_cast<const uint4 *>(wB + s2 * 64) : make_uint4(0, 0, 0, 0);
-            const u32 wa[4] = {va.x, va.y, va.z, va.w};
-            const u32 wb[4] = {vb.x, vb.y, vb.z, vb.w};
+            uint4 wv[4];
+#pragma unroll
+            for (int r4 = 0; r4 < 4; ++r4)
+                wv[r4] = kv ? *reinterpret_cast<const uint4 *>(w0 + r4 * Kw8 + s2 * 64) : make_uint4(0, 0, 0, 0);
             const uint8_t *x0p = xr0 + s2 * 256;
             const uint8_t *x1p = xr1 + s2 * 256;
 #pragma unroll
@@ -219,38 +228,48 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
                 if (NT > 1 && tv1) x1 = *reinterpret_cast<const uint4 *>(x1p + o1[c]);
                 const u32 xq0[4] = {x0.x, x0.y, x0.z, x0.w};
                 const u32 xq1[4] = {x1.x, x1.y, x1.z, x1.w};
-                int(&A)[NT][4] = (c & 1) ? acc2 : acc;
+                const u32 wr[4] = {(&wv[0].x)[c], (&wv[1].x)[c], (&wv[2].x)[c], (&wv[3].x)[c]};
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const u32 a0 = dec_unpack(wa[c], 2 * h), a2 = dec_unpack(wa[c], 2 * h + 1);
-                    const u32 a1 = dec_unpack(wb[c], 2 * h), a3 = dec_unpack(wb[c], 2 * h + 1);
-                    mma_s8_16832(A[0], a0, a1, a2, a3, xq0[2 * h], xq0[2 * h + 1]);
-                    if (NT > 1) mma_s8_16832(A[NT - 1], a0, a1, a2, a3, xq1[2 * h], xq1[2 * h + 1]);
+                for (int u = 0; u < 2; ++u) {
+                    int(&A)[NT][4] = (c & 1) ? acc2[u] : acc[u];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const u32 a0 = dec_unpack(wr[2 * u], 2 * h), a2 = dec_unpack(wr[2 * u], 2 * h + 1);
+                        const u32 a1 = dec_unpack(wr[2 * u + 1], 2 * h), a3 = dec_unpack(wr[2 * u + 1], 2 * h + 1);
+                        mma_s8_16832(A[0], a0, a1, a2, a3, xq0[2 * h], xq0[2 * h + 1]);
+                        if (NT > 1) mma_s8_16832(A[NT - 1], a0, a1, a2, a3, xq1[2 * h], xq1[2 * h + 1]);
+                    }
                 }
             }
         }
     }
 #pragma unroll
-    for (int nt = 0; nt < NT; ++nt)
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) acc[nt][i] += acc2[nt][i];
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[u][nt][i] += acc2[u][nt][i];
 
     // split-K reduction through shared memory
     if (G > 1) {
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+        for (int u = 0; u < 2; ++u)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) s_red[warp][nt][i][lane] = acc[nt][i];
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) s_red[warp][u][nt][i][lane] = acc[u][nt][i];
         __syncthreads();
         if (kslot == 0) {
             for (int q = 1; q < G; ++q)
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                for (int u = 0; u < 2; ++u)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[nt][i] += s_red[warp + q][nt][i][lane];
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) acc[u][nt][i] += s_red[warp + q][u][nt][i][lane];
         }
     }
-    if (kslot != 0 || !ok || wt >= tiles) return;
+    if (kslot != 0 || !ok || wg >= groups) return;
 
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
@@ -260,12 +279,15 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
             if (m >= M) continue;
             const float f = s_f[m];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                const int n = row_base + row0 + g + 8 * hh;
-                if (n < N) {
-                    const int a_ = acc[nt][2 * hh + e] >> 6;  // exact: the sum is a multiple of 64
-                    pr.Y[(size_t)m * N + n] = __fmul_rn(__int2float_rn(a_), f);
-                    if (pr.acc) pr.acc[(size_t)m * N + n] = a_;
+            for (int u = 0; u < 2; ++u) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int n = row_base + row0 + 16 * u + g + 8 * hh;
+                    if (n < N) {
+                        const int a_ = acc[u][nt][2 * hh + e] >> 6;  // exact: the sum is a multiple of 64
+                        pr.Y[(size_t)m * N + n] = __fmul_rn(__int2float_rn(a_), f);
+                        if (pr.acc) pr.acc[(size_t)m * N + n] = a_;
+                    }
                 }
             }
         }
