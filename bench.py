@@ -152,6 +152,20 @@ class Clocks:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def decode_traffic():
+    """DRAM bytes per grouped decode launch from the committed ncu capture, or
+    None when the kernel source changed since the counters were taken."""
+    import hashlib
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "decode_traffic.json")))
+        src = open(os.path.join(ROOT, rec["kernel_source"]), "rb").read()
+    except (OSError, ValueError, KeyError):
+        return None
+    if hashlib.sha256(src).hexdigest() != rec.get("kernel_source_sha256"):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def native(args, rank, world, local):
     from ternary_quantized_linear_bitlinear_b200 import api
 
@@ -299,13 +313,7 @@ def native(args, rank, world, local):
         pass
     peak = float(peaks.get("hbm_gbs", 6650.0))
     achieved = dec_bytes / (dec_us * 1e-6) / 1e9
-    traffic = None
-    tpath = os.path.join(ROOT, "profiles", "decode_traffic.json")
-    if os.path.exists(tpath):
-        try:
-            traffic = json.load(open(tpath)).get("dram_bytes_per_launch")
-        except (OSError, ValueError):
-            traffic = None
+    traffic = decode_traffic()
     roofline = {"bound": "hbm", "kernel": "k_decode (grouped GEMV, 84 problems)", "achieved": round(achieved, 1),
                 "peak": peak, "peak_source": "measured" if "hbm_gbs" in peaks else "fallback",
                 "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
