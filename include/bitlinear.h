@@ -166,7 +166,8 @@ bl_status bl_quant_act(const void *X, bl_dtype xdt, int64_t M, int64_t K,
 /*               (two float roundings: |Y - acc*gamma/s| <= 2^-23 |Y|)       */
 /*                                                                           */
 /* Engine: the bandwidth-bound decode GEMV when M <= 16 and its shared-     */
-/* memory staging fits (every M <= 16 for K <= 9728; M <= 2 at K = 32768),   */
+/* memory staging fits (M <= 16 for K <= 6144, M <= 13 at K = 9728, M <= 4 */
+/* at K = 16384, M <= 2 at K = 20480, none for K >= 24576),                  */
 /* otherwise the tcgen05 prefill GEMM.  Both give identical acc.             */
 /* packed [N, K/4] (format above); gamma [1]; x_q [M, K]; s [M]; Y [M, N]    */
 /* out; acc_out [M, N] int32 out or NULL.  All device.                       */
@@ -228,6 +229,41 @@ typedef struct {
 
 bl_status bl_quant_act_grouped(const bl_act_problem *problems, int count, bl_dtype xdt,
                                int64_t M, float subln_eps, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Grouped decode from raw activations: steps 2 + 3 + 4 in ONE launch.       */
+/*                                                                           */
+/* Defined by the same passages as bl_quant_act and bl_forward: for each     */
+/* problem, x_q and s are what bl_quant_act(X, subln_gain, subln_eps) would  */
+/* produce (bit for bit), and Y / acc what bl_forward would produce from     */
+/* them.  x_q never has to reach global memory: each CTA quantizes the rows  */
+/* it needs into on-chip memory while its packed weights stream in.          */
+/*                                                                           */
+/* X [M, K] of dtype xdt; subln_gain [K] float or NULL (RMSNorm before the   */
+/* quantizer, epsilon subln_eps); packed [N, K/4]; gamma [1]; Y [M, N] out.  */
+/* Optional outputs (NULL = not written): x_q [M, K] int8, s [M] float,      */
+/* acc_out [M, N] int32.  All device pointers, 16-byte aligned; `problems`   */
+/* is a HOST array read during the call only.  M <= 16 and every problem    */
+/* decode-eligible (see bl_forward), else BL_ERR_SHAPE.  flags: 0 or         */
+/* BL_FWD_WEIGHTS_READY (as for bl_forward_grouped; X may still be written  */
+/* by the kernel enqueued just before: it is read only after that kernel    */
+/* completes).                                                               */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    const uint8_t *packed;    /* [N, K/4] */
+    const float *gamma;       /* [1] */
+    const void *X;            /* [M, K] of the call's dtype */
+    const float *subln_gain;  /* [K] or NULL */
+    float *Y;                 /* [M, N] out */
+    int8_t *x_q;              /* [M, K] out or NULL */
+    float *s;                 /* [M] out or NULL */
+    int32_t *acc_out;         /* [M, N] out or NULL */
+    int64_t N;
+    int64_t K;
+} bl_decode_problem;
+
+bl_status bl_linear_decode_grouped(const bl_decode_problem *problems, int count, bl_dtype xdt,
+                                   int64_t M, float subln_eps, unsigned flags, bl_stream_t stream);
 
 #ifdef __cplusplus
 }

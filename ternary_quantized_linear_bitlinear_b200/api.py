@@ -46,6 +46,12 @@ class ActProblem(ctypes.Structure):
     _fields_ = [("X", _p), ("subln_gain", _p), ("x_q", _p), ("s", _p), ("K", _i64)]
 
 
+class DecodeProblem(ctypes.Structure):
+    """bl_decode_problem: one problem of the fused grouped decode (X in, Y out)."""
+    _fields_ = [("packed", _p), ("gamma", _p), ("X", _p), ("subln_gain", _p), ("Y", _p), ("x_q", _p),
+                ("s", _p), ("acc_out", _p), ("N", _i64), ("K", _i64)]
+
+
 _SIGS = {
     "bl_status_string": (ctypes.c_char_p, [_int]),
     "bl_version": (_int, []),
@@ -61,6 +67,8 @@ _SIGS = {
     "bl_debug_forward_prefill": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, ctypes.c_longlong,
                                         ctypes.c_uint32, _p]),
     "bl_quant_act_grouped": (_int, [ctypes.POINTER(ActProblem), _int, _int, _i64, _f32, _p]),
+    "bl_linear_decode_grouped": (_int, [ctypes.POINTER(DecodeProblem), _int, _int, _i64, _f32, ctypes.c_uint,
+                                        _p]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -214,6 +222,23 @@ def bl_forward_grouped(problems, count: int, M: int, flags: int = 0, stream=None
     """problems: ctypes array from make_problems (built once, launched many times)."""
     rc = lib().bl_forward_grouped(problems, count, M, flags, _stream(stream))
     _check(rc, "bl_forward_grouped")
+
+
+def make_decode_problems(items):
+    """items: list of (packed, gamma, X, subln_gain or None, Y, x_q or None, s or None, acc_out or None, N, K)
+    -> ctypes array for bl_linear_decode_grouped."""
+    arr = (DecodeProblem * len(items))()
+    for i, (packed, gamma, X, gain, Y, xq, s, acc, N, K) in enumerate(items):
+        arr[i] = DecodeProblem(packed.data_ptr(), gamma.data_ptr(), X.data_ptr(), _ptr(gain), Y.data_ptr(), _ptr(xq),
+                               _ptr(s), _ptr(acc), N, K)
+    return arr
+
+
+def bl_linear_decode_grouped(problems, count: int, M: int, dtype=torch.bfloat16, subln_eps: float = 1e-6,
+                             flags: int = 0, stream=None):
+    """Steps 2-4 fused: problems from make_decode_problems (X of `dtype`, same M)."""
+    rc = lib().bl_linear_decode_grouped(problems, count, _DTYPES[dtype], M, subln_eps, flags, _stream(stream))
+    _check(rc, "bl_linear_decode_grouped")
 
 
 # -- all four steps ------------------------------------------------------------

@@ -46,10 +46,10 @@ bl_status device_info(DeviceInfo **out) {
         if (d.ok) {
             // opt in to large dynamic shared memory once per device
             bool fail = false;
-            fail |= cudaFuncSetAttribute(k_decode<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         DEC_SMEM_LIMIT) != cudaSuccess;
-            fail |= cudaFuncSetAttribute(k_decode<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         DEC_SMEM_LIMIT) != cudaSuccess;
+            for (auto fn : {k_decode<1, DEC_SRC_XQ>, k_decode<2, DEC_SRC_XQ>, k_decode<1, DEC_SRC_BF16>,
+                            k_decode<2, DEC_SRC_BF16>, k_decode<1, DEC_SRC_F32>, k_decode<2, DEC_SRC_F32>})
+                fail |= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM_LIMIT) !=
+                        cudaSuccess;
             fail |= prefill_setup() != cudaSuccess;
             if (fail) return BL_ERR_CUDA;
         }
@@ -168,7 +168,7 @@ bool decode_eligible(int64_t M, int64_t K) {
     return M <= 16 && dec_xq_off(K) + M * dec_row_stride((int)K) <= DEC_SMEM_LIMIT;
 }
 
-bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st) {
+bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st, int src = DEC_SRC_XQ) {
     int total = 0;
     int rs_max = 0, xq_off = 0;
     for (int i = 0; i < P.count; ++i) {
@@ -203,7 +203,16 @@ bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    cudaError_t e = P.M <= 8 ? cudaLaunchKernelEx(&cfg, k_decode<1>, P) : cudaLaunchKernelEx(&cfg, k_decode<2>, P);
+    cudaError_t e;
+    if (src == DEC_SRC_BF16)
+        e = P.M <= 8 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_BF16>, P)
+                     : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_BF16>, P);
+    else if (src == DEC_SRC_F32)
+        e = P.M <= 8 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_F32>, P)
+                     : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_F32>, P);
+    else
+        e = P.M <= 8 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_XQ>, P)
+                     : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_XQ>, P);
     return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 
@@ -213,7 +222,9 @@ bl_status forward_impl(const DeviceInfo &d, const uint8_t *packed, const float *
         DecodeParams P;
         P.count = 1;
         P.M = (int)M;
-        P.p[0] = DecodeProblem{packed, gamma, x_q, s, Y, acc_out, (int)N, (int)K, 0, 0};
+        P.eps = 0.f;
+        P.p[0] = DecodeProblem{packed, gamma, x_q, const_cast<float *>(s), Y, acc_out, nullptr, nullptr,
+                               (int)N, (int)K, 0, 0};
         return decode_launch(P, false, st);
     }
     return prefill_launch(d.sms, packed, gamma, x_q, s, M, N, K, Y, acc_out, st);
@@ -332,14 +343,43 @@ bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, u
         if (!aligned16(q.packed) || !aligned16(q.gamma) || !aligned16(q.x_q) || !aligned16(q.s) || !aligned16(q.Y) ||
             (q.acc_out && !aligned16(q.acc_out)))
             return BL_ERR_ALIGN;
-        P.p[i] = DecodeProblem{q.packed, q.gamma, q.x_q, q.s, q.Y, q.acc_out, (int)q.N, (int)q.K, 0, 0};
+        P.p[i] = DecodeProblem{q.packed, q.gamma, q.x_q, const_cast<float *>(q.s), q.Y, q.acc_out, nullptr, nullptr,
+                               (int)q.N, (int)q.K, 0, 0};
         ctas += (q.N + 15) / 16;
     }
     if (ctas > 0x7fffffffLL) return BL_ERR_SHAPE;
+    P.eps = 0.f;
     DeviceInfo *d;
     bl_status rc = device_info(&d);
     if (rc) return rc;
     return decode_launch(P, (flags & BL_FWD_WEIGHTS_READY) != 0, (cudaStream_t)stream);
+}
+
+bl_status bl_linear_decode_grouped(const bl_decode_problem *problems, int count, bl_dtype xdt, int64_t M,
+                                   float subln_eps, unsigned flags, bl_stream_t stream) {
+    if (!problems) return BL_ERR_NULL;
+    if (count < 1 || count > BL_MAX_GROUP || M < 1 || M > 16) return BL_ERR_SHAPE;
+    if (xdt != BL_F32 && xdt != BL_BF16) return BL_ERR_DTYPE;
+    DecodeParams P;
+    P.count = count;
+    P.M = (int)M;
+    P.eps = subln_eps;
+    for (int i = 0; i < count; ++i) {
+        const bl_decode_problem &q = problems[i];
+        if (!q.packed || !q.gamma || !q.X || !q.Y) return BL_ERR_NULL;
+        if (q.N < 1 || q.N > 0x7fffffffLL || check_k(q.K) != BL_OK || !decode_eligible(M, q.K)) return BL_ERR_SHAPE;
+        if (!aligned16(q.packed) || !aligned16(q.gamma) || !aligned16(q.X) || !aligned16(q.Y) ||
+            (q.subln_gain && !aligned16(q.subln_gain)) || (q.x_q && !aligned16(q.x_q)) ||
+            (q.s && !aligned16(q.s)) || (q.acc_out && !aligned16(q.acc_out)))
+            return BL_ERR_ALIGN;
+        P.p[i] = DecodeProblem{q.packed, q.gamma, q.X, q.s, q.Y, q.acc_out, q.subln_gain, q.x_q,
+                               (int)q.N, (int)q.K, 0, 0};
+    }
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return decode_launch(P, (flags & BL_FWD_WEIGHTS_READY) != 0, (cudaStream_t)stream,
+                         xdt == BL_BF16 ? DEC_SRC_BF16 : DEC_SRC_F32);
 }
 
 size_t bl_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {

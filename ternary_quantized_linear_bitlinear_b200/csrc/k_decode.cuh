@@ -27,6 +27,13 @@
 //     bank conflicts).
 //   - acc = (sum of 64 * W_q * x_q) >> 6 exactly; the split-K partials meet
 //     in shared memory; the epilogue rescales and stores Y (and acc).
+//   - Fused variant (SRC = bf16 or f32 activations): step 2 runs inside the
+//     CTA instead of a separate launch.  One warp per token row computes
+//     s = 127 / max|y| (y = x, or the SubLN RMSNorm of x) and writes x_q
+//     straight into the swizzled staging rows, with the same arithmetic as
+//     the stand-alone activation quantizer, while the weights stream in.
+//     Every CTA of a problem quantizes the (L2-resident) rows itself; the
+//     problem's first CTA also writes x_q and s to global memory on request.
 #pragma once
 
 #include "bl_common.cuh"
@@ -37,15 +44,21 @@ constexpr int DEC_THREADS = 256;
 constexpr int DEC_WARPS = DEC_THREADS / 32;
 constexpr int DEC_SMEM_LIMIT = 200 * 1024;  // weight tiles + staged x_q, per CTA
 constexpr int DEC_PF = 4;                   // target 256-k steps per warp (G is chosen from it)
+constexpr int DEC_W_CAP = 48 * 1024;        // weight bytes per CTA above which G grows (3 CTAs per SM)
 constexpr unsigned long long DEC_TIMEOUT_NS = 2000000000ull;
+
+// Activation source of a launch: pre-quantized x_q, or X to quantize in-kernel.
+enum : int { DEC_SRC_XQ = 0, DEC_SRC_BF16 = 1, DEC_SRC_F32 = 2 };
 
 struct DecodeProblem {
     const uint8_t *packed;
     const float *gamma;
-    const int8_t *xq;
-    const float *s;
+    const void *x;         // DEC_SRC_XQ: x_q [M, K] int8; else X [M, K] bf16 / f32
+    float *s;              // DEC_SRC_XQ: s [M] in; else s [M] out or null
     float *Y;
     int32_t *acc;
+    const float *gain;     // fused: SubLN gain [K] or null
+    int8_t *xq_out;        // fused: x_q [M, K] out or null
     int N;
     int K;
     int g_log2;     // log2(G): warps per row tile
@@ -60,15 +73,19 @@ struct DecodeParams {
     int M;
     int xq_off;  // shared-memory offset of the staged x_q (after the weight tiles)
     int use_table;
+    float eps;   // fused: SubLN epsilon
     unsigned char cta_problem[DEC_CTA_TABLE];
 };
 
 __host__ __device__ inline int dec_row_stride(int K) { return (K + 255) & ~255; }
 
 __host__ __device__ inline int dec_glog(int K) {
-    // smallest G = 2^glog <= 8 with ceil(steps / G) <= DEC_PF
+    // smallest G = 2^glog <= 8 with ceil(steps / G) <= DEC_PF and at most
+    // DEC_W_CAP bytes of weights per CTA (8 / G groups of 32 rows), so that
+    // three CTAs fit on an SM and a grouped launch stays one wave
     int steps = (K + 255) >> 8, g = 0;
     while (g < 3 && ((steps + (1 << g) - 1) >> g) > DEC_PF) ++g;
+    while (g < 3 && (DEC_WARPS >> g) * 32 * (K >> 2) > DEC_W_CAP) ++g;
     return g;
 }
 
@@ -90,8 +107,141 @@ __device__ __forceinline__ void mma_s8_16832(int (&c)[4], u32 a0, u32 a1, u32 a2
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-// NT: 8-token column tiles (1: M <= 8, 2: M <= 16).
-template <int NT>
+// Float bits of element j of a 16-byte activation vector.
+template <bool BF16>
+__device__ __forceinline__ u32 dec_x_bits(const uint4 &v, int j) {
+    const u32 w = j < (BF16 ? 2 : 1) ? v.x : j < (BF16 ? 4 : 2) ? v.y : j < (BF16 ? 6 : 3) ? v.z : v.w;
+    return BF16 ? ((j & 1) ? (w & 0xffff0000u) : (w << 16)) : w;
+}
+
+// Exact sum of squares of one row, rounded once to double (valid on lane 0).
+// x^2 = mant^2 * 2^(2e - 300) with e >= 1 (subnormals: e = 1, no hidden
+// bit).  Each pass adds the values with e in [elo, ehi] (31 binades) as
+// mant^2 << 2(e - elo) into a 128-bit lane accumulator (< 2^108 per term,
+// at most 1024 terms per lane, a warp sum < 2^123), and lane 0 adds the warp
+// sum into 576-bit limbs in units of 2^-298; a pass repeats one window lower
+// only while some lane saw a smaller nonzero value (at most 9 passes).
+template <bool BF16>
+__device__ double dec_row_sumsq(const uint4 *xr, int nvec, int lane, u32 amax_bits) {
+    constexpr int EPV = BF16 ? 8 : 4;
+    u64 L[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+    int ehi = (int)(amax_bits >> 23);
+    if (ehi < 1) ehi = 1;
+    for (int pass = 0; pass < 10; ++pass) {
+        const int elo = ehi - 30 < 1 ? 1 : ehi - 30;
+        u64 lo = 0ull, hi = 0ull;
+        bool below = false;
+        for (int v = lane; v < nvec; v += 32) {
+            const uint4 raw = ldg_nc_v4(xr + v);
+#pragma unroll
+            for (int j = 0; j < EPV; ++j) {
+                const u32 u = dec_x_bits<BF16>(raw, j) & 0x7fffffffu;
+                const int e = (int)(u >> 23);
+                const int ee = e ? e : 1;
+                if (ee <= ehi && ee >= elo && u != 0u) {
+                    u64 mm = (u64)(e ? ((u & 0x7fffffu) | 0x800000u) : u);
+                    mm *= mm;
+                    const int sh = 2 * (ee - elo);  // <= 60
+                    const u64 plo = mm << sh;
+                    const u64 phi = sh ? (mm >> (64 - sh)) : 0ull;
+                    const u64 t = lo + plo;
+                    hi += phi + (t < lo ? 1ull : 0ull);
+                    lo = t;
+                } else if (ee < elo && u != 0u) {
+                    below = true;
+                }
+            }
+        }
+        warp_sum_u128(lo, hi);
+        if (lane == 0) limbs_add_u128_shl(L, lo, hi, 2 * (elo - 1));
+        if (!__any_sync(0xffffffffu, below) || elo == 1) break;
+        ehi = elo - 1;
+    }
+    return lane == 0 ? limbs_to_double_rn(L, -298) : 0.0;
+}
+
+// Step 2 for token row m by one warp, into the swizzled staging row (and,
+// when out is set, x_q / s in global memory).  Arithmetic identical to the
+// stand-alone quantizer:
+//   y = x, or y = float(float(x / r) * g), r = sqrtf(float(double(sum x^2) / K) + eps)
+//   s = float(127 / max(max|y|, 1e-5f)),  x_q = clamp(rne(float(y * s)), -128, 127)
+// Returns s (on every lane).
+template <bool BF16>
+__device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, uint8_t *s_xq, float eps, bool out,
+                               int lane) {
+    constexpr int EPV = BF16 ? 8 : 4;
+    const int nvec = K / EPV;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(pr.x) + (size_t)m * nvec;
+    const float4 *g4 = reinterpret_cast<const float4 *>(pr.gain);
+    u32 amax = 0;
+    for (int v = lane; v < nvec; v += 32) {
+        const uint4 raw = ldg_nc_v4(xr + v);
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) amax = max(amax, dec_x_bits<BF16>(raw, j) & 0x7fffffffu);
+    }
+    amax = warp_max_u32(amax);
+    float r = 1.f;
+    if (g4 != nullptr) {
+        const double S2 = dec_row_sumsq<BF16>(xr, nvec, lane, amax);
+        if (lane == 0) r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(S2, (double)K)), eps));
+        r = __shfl_sync(0xffffffffu, r, 0);
+        amax = 0;
+        for (int v = lane; v < nvec; v += 32) {
+            const uint4 raw = ldg_nc_v4(xr + v);
+#pragma unroll
+            for (int q = 0; q < EPV / 4; ++q) {
+                const float4 g = __ldg(g4 + v * (EPV / 4) + q);
+                const float gg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float y = __fmul_rn(__fdiv_rn(__uint_as_float(dec_x_bits<BF16>(raw, 4 * q + j)), r), gg[j]);
+                    amax = max(amax, __float_as_uint(y) & 0x7fffffffu);
+                }
+            }
+        }
+        amax = warp_max_u32(amax);
+    }
+    const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(amax), 1e-5f));
+    uint8_t *dst = s_xq + m * RS;
+    int8_t *gq = out && pr.xq_out != nullptr ? pr.xq_out + (size_t)m * K : nullptr;
+    for (int v = lane; v < nvec; v += 32) {
+        const uint4 raw = ldg_nc_v4(xr + v);
+        u32 word[EPV / 4];
+#pragma unroll
+        for (int q = 0; q < EPV / 4; ++q) {
+            float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
+            if (g4 != nullptr) g = __ldg(g4 + v * (EPV / 4) + q);
+            const float gg[4] = {g.x, g.y, g.z, g.w};
+            u32 w = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                float y = __uint_as_float(dec_x_bits<BF16>(raw, 4 * q + j));
+                if (g4 != nullptr) y = __fmul_rn(__fdiv_rn(y, r), gg[j]);
+                int qi = __float2int_rn(__fmul_rn(y, s));
+                qi = max(-128, min(127, qi));
+                w |= ((u32)qi & 0xffu) << (8 * j);
+            }
+            word[q] = w;
+        }
+        // 16-byte chunk L of the row holds k = 16L .. 16L + 15
+        const int L = BF16 ? (v >> 1) : (v >> 2);
+        const int within = BF16 ? (v & 1) * 8 : (v & 3) * 4;
+        const int x = (((L >> 3) & 1) << 1) | (m & 1);
+        uint8_t *d = dst + ((((L & ~7) | ((L ^ x) & 7)) << 4) + within);
+        if (BF16) {
+            *reinterpret_cast<uint2 *>(d) = make_uint2(word[0], word[EPV / 4 - 1]);
+            if (gq) *reinterpret_cast<uint2 *>(gq + (size_t)v * 8) = make_uint2(word[0], word[EPV / 4 - 1]);
+        } else {
+            *reinterpret_cast<u32 *>(d) = word[0];
+            if (gq) *reinterpret_cast<u32 *>(gq + (size_t)v * 4) = word[0];
+        }
+    }
+    if (out && lane == 0 && pr.s != nullptr) pr.s[m] = s;
+    return s;
+}
+
+// NT: 8-token column tiles (1: M <= 8, 2: M <= 16).  SRC: DEC_SRC_*.
+template <int NT, int SRC>
 __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ DecodeParams P) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_red[DEC_WARPS][2][NT][4][32];
@@ -149,12 +299,28 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
     // float(gamma / s[m]) once per token.
     const int RS = dec_row_stride(K);
     uint8_t *s_xq = smem + P.xq_off;
-    {
+    if (SRC != DEC_SRC_XQ) {
+        // fused step 2: warp w quantizes rows w, w + 8
+        const int lane = threadIdx.x & 31;
+        const bool out = b == pr.cta_begin;
+        for (int m = threadIdx.x >> 5; m < M; m += DEC_WARPS) {
+            const float s = dec_quant_row<SRC == DEC_SRC_BF16>(pr, m, K, RS, s_xq, P.eps, out, lane);
+            if (lane == 0) s_f[m] = __fdiv_rn(*pr.gamma, s);
+        }
+        const int chunks = RS >> 4, kchunks = K >> 4;
+        for (int r = 0; r < M; ++r) {
+            for (int L = kchunks + (int)threadIdx.x; L < chunks; L += DEC_THREADS) {
+                const int x = (((L >> 3) & 1) << 1) | (r & 1);
+                *reinterpret_cast<uint4 *>(s_xq + r * RS + (((L & ~7) | ((L ^ x) & 7)) << 4)) =
+                    make_uint4(0, 0, 0, 0);
+            }
+        }
+    } else {
         // every 16-byte chunk in flight at once (cp.async), one wait
         const int chunks = RS >> 4;
         const int kchunks = K >> 4;
         for (int r = 0; r < M; ++r) {
-            const int8_t *src = pr.xq + (size_t)r * K;
+            const int8_t *src = static_cast<const int8_t *>(pr.x) + (size_t)r * K;
             uint8_t *dst = s_xq + r * RS;
             for (int L = threadIdx.x; L < chunks; L += DEC_THREADS) {
                 const int x = (((L >> 3) & 1) << 1) | (r & 1);

@@ -137,6 +137,32 @@ def test_grouped_validation(L):
     assert L.bl_quant_act_grouped(Q, 1, 1, 1, 1e-6, None) in (CUDA, DEVICE)
 
 
+def test_fused_decode_validation(L):
+    P = (api.DecodeProblem * 2)()
+    for i in range(2):
+        P[i] = api.DecodeProblem(A, A, A, None, A, None, None, None, 64, 128)
+    def g(arr, count, M, dt=1):
+        return L.bl_linear_decode_grouped(arr, count, dt, M, 1e-6, 0, None)
+    assert g(None, 1, 1) == NULL
+    assert g(P, 0, 1) == SHAPE
+    assert g(P, api.BL_MAX_GROUP + 1, 1) == SHAPE
+    assert g(P, 2, 17) == SHAPE
+    assert g(P, 2, 1, dt=4) == DTYPE
+    P[1].X = None
+    assert g(P, 2, 1) == NULL
+    P[1].X = A
+    P[1].K = 96
+    assert g(P, 2, 1) == SHAPE
+    P[1].K = 32768
+    assert g(P, 2, 16) == SHAPE  # x_q staging of 16 rows of 32768 does not fit
+    P[1].K = 128
+    for field in ("subln_gain", "x_q", "s", "acc_out", "Y"):
+        setattr(P[1], field, A + 4)
+        assert g(P, 2, 1) == ALIGN, field
+        setattr(P[1], field, A if field == "Y" else None)
+    assert g(P, 2, 1) in (CUDA, DEVICE)
+
+
 def test_debug_prefill_validation(L):
     f = L.bl_debug_forward_prefill
     assert f(None, A, A, A, 1, 64, 128, A, None, -1, 1000, None) == NULL
