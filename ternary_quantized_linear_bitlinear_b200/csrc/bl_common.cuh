@@ -214,4 +214,19 @@ __device__ __forceinline__ void bulk_g2s(u32 dst, const void *src, u32 bytes, u3
                  : "memory");
 }
 
+// Same, with an L2 eviction-priority policy (from l2_policy_evict_first) for
+// data that is read exactly once, so it does not displace reused lines.
+__device__ __forceinline__ void bulk_g2s_hint(u32 dst, const void *src, u32 bytes, u32 bar, u64 policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;"
+        ::"r"(dst), "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ u64 l2_policy_evict_first() {
+    u64 p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
 }  // namespace bl

@@ -114,6 +114,19 @@ __device__ __forceinline__ u32 dec_x_bits(const uint4 &v, int j) {
     return BF16 ? ((j & 1) ? (w & 0xffff0000u) : (w << 16)) : w;
 }
 
+// A row of X is processed in blocks of 256 16-byte vectors, 8 per lane
+// (vector blk * 256 + 32 i + lane in register i, zero past the row end); a
+// row of at most one block is loaded once and every pass works on registers.
+constexpr int DEC_QV = 8;
+
+__device__ __forceinline__ void dec_load_block(uint4 (&c)[DEC_QV], const uint4 *xr, int nvec, int blk, int lane) {
+#pragma unroll
+    for (int i = 0; i < DEC_QV; ++i) {
+        const int v = blk * (32 * DEC_QV) + 32 * i + lane;
+        c[i] = v < nvec ? ldg_nc_v4(xr + v) : make_uint4(0, 0, 0, 0);
+    }
+}
+
 // Exact sum of squares of one row, rounded once to double (valid on lane 0).
 // x^2 = mant^2 * 2^(2e - 300) with e >= 1 (subnormals: e = 1, no hidden
 // bit).  Each pass adds the values with e in [elo, ehi] (31 binades) as
@@ -122,8 +135,9 @@ __device__ __forceinline__ u32 dec_x_bits(const uint4 &v, int j) {
 // sum into 576-bit limbs in units of 2^-298; a pass repeats one window lower
 // only while some lane saw a smaller nonzero value (at most 9 passes).
 template <bool BF16>
-__device__ double dec_row_sumsq(const uint4 *xr, int nvec, int lane, u32 amax_bits) {
+__device__ double dec_row_sumsq(uint4 (&c)[DEC_QV], const uint4 *xr, int nvec, int lane, u32 amax_bits) {
     constexpr int EPV = BF16 ? 8 : 4;
+    const int nblk = (nvec + 32 * DEC_QV - 1) / (32 * DEC_QV);
     u64 L[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
     int ehi = (int)(amax_bits >> 23);
     if (ehi < 1) ehi = 1;
@@ -131,24 +145,27 @@ __device__ double dec_row_sumsq(const uint4 *xr, int nvec, int lane, u32 amax_bi
         const int elo = ehi - 30 < 1 ? 1 : ehi - 30;
         u64 lo = 0ull, hi = 0ull;
         bool below = false;
-        for (int v = lane; v < nvec; v += 32) {
-            const uint4 raw = ldg_nc_v4(xr + v);
+        for (int blk = 0; blk < nblk; ++blk) {
+            if (nblk > 1) dec_load_block(c, xr, nvec, blk, lane);
 #pragma unroll
-            for (int j = 0; j < EPV; ++j) {
-                const u32 u = dec_x_bits<BF16>(raw, j) & 0x7fffffffu;
-                const int e = (int)(u >> 23);
-                const int ee = e ? e : 1;
-                if (ee <= ehi && ee >= elo && u != 0u) {
-                    u64 mm = (u64)(e ? ((u & 0x7fffffu) | 0x800000u) : u);
-                    mm *= mm;
-                    const int sh = 2 * (ee - elo);  // <= 60
-                    const u64 plo = mm << sh;
-                    const u64 phi = sh ? (mm >> (64 - sh)) : 0ull;
-                    const u64 t = lo + plo;
-                    hi += phi + (t < lo ? 1ull : 0ull);
-                    lo = t;
-                } else if (ee < elo && u != 0u) {
-                    below = true;
+            for (int i = 0; i < DEC_QV; ++i) {
+#pragma unroll
+                for (int j = 0; j < EPV; ++j) {
+                    const u32 u = dec_x_bits<BF16>(c[i], j) & 0x7fffffffu;
+                    const int e = (int)(u >> 23);
+                    const int ee = e ? e : 1;
+                    if (ee <= ehi && ee >= elo && u != 0u) {
+                        u64 mm = (u64)(e ? ((u & 0x7fffffu) | 0x800000u) : u);
+                        mm *= mm;
+                        const int sh = 2 * (ee - elo);  // <= 60
+                        const u64 plo = mm << sh;
+                        const u64 phi = sh ? (mm >> (64 - sh)) : 0ull;
+                        const u64 t = lo + plo;
+                        hi += phi + (t < lo ? 1ull : 0ull);
+                        lo = t;
+                    } else if (ee < elo && u != 0u) {
+                        below = true;
+                    }
                 }
             }
         }
@@ -158,6 +175,21 @@ __device__ double dec_row_sumsq(const uint4 *xr, int nvec, int lane, u32 amax_bi
         ehi = elo - 1;
     }
     return lane == 0 ? limbs_to_double_rn(L, -298) : 0.0;
+}
+
+// y of element j of vector v: x, or float(float(x / r) * g)
+template <bool BF16>
+__device__ __forceinline__ void dec_y4(const uint4 &raw, int q, const float4 *g4, int v, float r, float (&y)[4]) {
+    constexpr int EPV = BF16 ? 8 : 4;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) y[j] = __uint_as_float(dec_x_bits<BF16>(raw, 4 * q + j));
+    if (g4 != nullptr) {
+        const float4 g = __ldg(g4 + v * (EPV / 4) + q);
+        y[0] = __fmul_rn(__fdiv_rn(y[0], r), g.x);
+        y[1] = __fmul_rn(__fdiv_rn(y[1], r), g.y);
+        y[2] = __fmul_rn(__fdiv_rn(y[2], r), g.z);
+        y[3] = __fmul_rn(__fdiv_rn(y[3], r), g.w);
+    }
 }
 
 // Step 2 for token row m by one warp, into the swizzled staging row (and,
@@ -171,31 +203,39 @@ __device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, ui
                                int lane) {
     constexpr int EPV = BF16 ? 8 : 4;
     const int nvec = K / EPV;
+    const int nblk = (nvec + 32 * DEC_QV - 1) / (32 * DEC_QV);
     const uint4 *xr = reinterpret_cast<const uint4 *>(pr.x) + (size_t)m * nvec;
     const float4 *g4 = reinterpret_cast<const float4 *>(pr.gain);
+    uint4 c[DEC_QV];
+    dec_load_block(c, xr, nvec, 0, lane);
     u32 amax = 0;
-    for (int v = lane; v < nvec; v += 32) {
-        const uint4 raw = ldg_nc_v4(xr + v);
+    for (int blk = 0; blk < nblk; ++blk) {
+        if (blk > 0) dec_load_block(c, xr, nvec, blk, lane);
 #pragma unroll
-        for (int j = 0; j < EPV; ++j) amax = max(amax, dec_x_bits<BF16>(raw, j) & 0x7fffffffu);
+        for (int i = 0; i < DEC_QV; ++i)
+#pragma unroll
+            for (int j = 0; j < EPV; ++j) amax = max(amax, dec_x_bits<BF16>(c[i], j) & 0x7fffffffu);
     }
     amax = warp_max_u32(amax);
     float r = 1.f;
     if (g4 != nullptr) {
-        const double S2 = dec_row_sumsq<BF16>(xr, nvec, lane, amax);
+        if (nblk > 1) dec_load_block(c, xr, nvec, 0, lane);
+        const double S2 = dec_row_sumsq<BF16>(c, xr, nvec, lane, amax);
         if (lane == 0) r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(S2, (double)K)), eps));
         r = __shfl_sync(0xffffffffu, r, 0);
         amax = 0;
-        for (int v = lane; v < nvec; v += 32) {
-            const uint4 raw = ldg_nc_v4(xr + v);
+        for (int blk = 0; blk < nblk; ++blk) {
+            if (nblk > 1) dec_load_block(c, xr, nvec, blk, lane);
 #pragma unroll
-            for (int q = 0; q < EPV / 4; ++q) {
-                const float4 g = __ldg(g4 + v * (EPV / 4) + q);
-                const float gg[4] = {g.x, g.y, g.z, g.w};
+            for (int i = 0; i < DEC_QV; ++i) {
+                const int v = blk * (32 * DEC_QV) + 32 * i + lane;
+                if (v >= nvec) continue;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float y = __fmul_rn(__fdiv_rn(__uint_as_float(dec_x_bits<BF16>(raw, 4 * q + j)), r), gg[j]);
-                    amax = max(amax, __float_as_uint(y) & 0x7fffffffu);
+                for (int q = 0; q < EPV / 4; ++q) {
+                    float y[4];
+                    dec_y4<BF16>(c[i], q, g4, v, r, y);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) amax = max(amax, __float_as_uint(y[j]) & 0x7fffffffu);
                 }
             }
         }
@@ -204,36 +244,38 @@ __device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, ui
     const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(amax), 1e-5f));
     uint8_t *dst = s_xq + m * RS;
     int8_t *gq = out && pr.xq_out != nullptr ? pr.xq_out + (size_t)m * K : nullptr;
-    for (int v = lane; v < nvec; v += 32) {
-        const uint4 raw = ldg_nc_v4(xr + v);
-        u32 word[EPV / 4];
+    for (int blk = 0; blk < nblk; ++blk) {
+        if (nblk > 1) dec_load_block(c, xr, nvec, blk, lane);
 #pragma unroll
-        for (int q = 0; q < EPV / 4; ++q) {
-            float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
-            if (g4 != nullptr) g = __ldg(g4 + v * (EPV / 4) + q);
-            const float gg[4] = {g.x, g.y, g.z, g.w};
-            u32 w = 0;
+        for (int i = 0; i < DEC_QV; ++i) {
+            const int v = blk * (32 * DEC_QV) + 32 * i + lane;
+            if (v >= nvec) continue;
+            u32 word[EPV / 4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                float y = __uint_as_float(dec_x_bits<BF16>(raw, 4 * q + j));
-                if (g4 != nullptr) y = __fmul_rn(__fdiv_rn(y, r), gg[j]);
-                int qi = __float2int_rn(__fmul_rn(y, s));
-                qi = max(-128, min(127, qi));
-                w |= ((u32)qi & 0xffu) << (8 * j);
+            for (int q = 0; q < EPV / 4; ++q) {
+                float y[4];
+                dec_y4<BF16>(c[i], q, g4, v, r, y);
+                u32 w = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    int qi = __float2int_rn(__fmul_rn(y[j], s));
+                    qi = max(-128, min(127, qi));
+                    w |= ((u32)qi & 0xffu) << (8 * j);
+                }
+                word[q] = w;
             }
-            word[q] = w;
-        }
-        // 16-byte chunk L of the row holds k = 16L .. 16L + 15
-        const int L = BF16 ? (v >> 1) : (v >> 2);
-        const int within = BF16 ? (v & 1) * 8 : (v & 3) * 4;
-        const int x = (((L >> 3) & 1) << 1) | (m & 1);
-        uint8_t *d = dst + ((((L & ~7) | ((L ^ x) & 7)) << 4) + within);
-        if (BF16) {
-            *reinterpret_cast<uint2 *>(d) = make_uint2(word[0], word[EPV / 4 - 1]);
-            if (gq) *reinterpret_cast<uint2 *>(gq + (size_t)v * 8) = make_uint2(word[0], word[EPV / 4 - 1]);
-        } else {
-            *reinterpret_cast<u32 *>(d) = word[0];
-            if (gq) *reinterpret_cast<u32 *>(gq + (size_t)v * 4) = word[0];
+            // 16-byte chunk L of the row holds k = 16L .. 16L + 15
+            const int L = BF16 ? (v >> 1) : (v >> 2);
+            const int within = BF16 ? (v & 1) * 8 : (v & 3) * 4;
+            const int x = (((L >> 3) & 1) << 1) | (m & 1);
+            uint8_t *d = dst + ((((L & ~7) | ((L ^ x) & 7)) << 4) + within);
+            if (BF16) {
+                *reinterpret_cast<uint2 *>(d) = make_uint2(word[0], word[EPV / 4 - 1]);
+                if (gq) *reinterpret_cast<uint2 *>(gq + (size_t)v * 8) = make_uint2(word[0], word[EPV / 4 - 1]);
+            } else {
+                *reinterpret_cast<u32 *>(d) = word[0];
+                if (gq) *reinterpret_cast<u32 *>(gq + (size_t)v * 4) = word[0];
+            }
         }
     }
     if (out && lane == 0 && pr.s != nullptr) pr.s[m] = s;
@@ -242,7 +284,7 @@ __device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, ui
 
 // NT: 8-token column tiles (1: M <= 8, 2: M <= 16).  SRC: DEC_SRC_*.
 template <int NT, int SRC>
-__global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ DecodeParams P) {
+__global__ void __launch_bounds__(DEC_THREADS, 3) k_decode(const __grid_constant__ DecodeParams P) {
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int s_red[DEC_WARPS][2][NT][4][32];
     __shared__ __align__(8) u64 s_bar[DEC_WARPS];
@@ -279,6 +321,7 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         const uint8_t *src = pr.packed + (size_t)row_base * Kw;
         const u32 dst = smem_u32(smem);
+        const u64 policy = l2_policy_evict_first();  // weights are read once per launch
         for (int i = 0; i < groups; ++i) {
             const u32 nrows = (u32)min(DEC_ROWS, rows - DEC_ROWS * i);
             const u32 bytes = nrows * (u32)Kw;
@@ -287,7 +330,7 @@ __global__ void __launch_bounds__(DEC_THREADS) k_decode(const __grid_constant__ 
             const u32 off0 = (u32)(DEC_ROWS * i) * (u32)Kw;
             for (u32 off = 0; off < bytes; off += 32768u) {
                 const u32 n = bytes - off < 32768u ? bytes - off : 32768u;
-                bulk_g2s(dst + off0 + off, src + off0 + off, n, bar);
+                bulk_g2s_hint(dst + off0 + off, src + off0 + off, n, bar, policy);
             }
         }
     }
