@@ -91,21 +91,34 @@ bl_status quant_weights_impl(const DeviceInfo &d, const void *W, bl_dtype wdt, i
 
     u64 *partials = reinterpret_cast<u64 *>(ws);
     u32 *thresh = reinterpret_cast<u32 *>(reinterpret_cast<uint8_t *>(ws) + WQ_WS_PARTIALS);
+    u32 *ticket = reinterpret_cast<u32 *>(reinterpret_cast<uint8_t *>(ws) + WQ_WS_TICKET);
     const uint4 *Wv = reinterpret_cast<const uint4 *>(W);
+    if (cudaMemsetAsync(ticket, 0, sizeof(u32), st) != cudaSuccess) return BL_ERR_CUDA;
     if (bf16)
-        k_absmean_partial<true><<<(unsigned)grid, WQ_THREADS, 0, st>>>(Wv, nvec, partials);
+        k_absmean_partial<true><<<(unsigned)grid, WQ_THREADS, 0, st>>>(Wv, nvec, n, partials, gamma, thresh, ticket);
     else
-        k_absmean_partial<false><<<(unsigned)grid, WQ_THREADS, 0, st>>>(Wv, nvec, partials);
-    k_gamma_finalize<<<1, 32, 0, st>>>(partials, (int)grid, n, gamma, thresh);
+        k_absmean_partial<false><<<(unsigned)grid, WQ_THREADS, 0, st>>>(Wv, nvec, n, partials, gamma, thresh, ticket);
+    if (cudaGetLastError() != cudaSuccess) return BL_ERR_CUDA;
     const long long nwords = n / 16;
     long long pgrid = (nwords + 255) / 256;
     long long pcap = 8LL * d.sms;
     if (pgrid > pcap) pgrid = pcap;
-    if (bf16)
-        k_ternary_pack<true><<<(unsigned)pgrid, 256, 0, st>>>(Wv, nwords, thresh, reinterpret_cast<u32 *>(packed));
-    else
-        k_ternary_pack<false><<<(unsigned)pgrid, 256, 0, st>>>(Wv, nwords, thresh, reinterpret_cast<u32 *>(packed));
-    return launch_status();
+    // programmatic dependent launch: the pack grid starts loading W while the
+    // reduction finishes and waits for it (griddepcontrol.wait) before using T
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)pgrid);
+    cfg.blockDim = dim3(256);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    u32 *pk = reinterpret_cast<u32 *>(packed);
+    const u32 *th = thresh;
+    cudaError_t e = bf16 ? cudaLaunchKernelEx(&cfg, k_ternary_pack<true>, Wv, nwords, th, pk)
+                         : cudaLaunchKernelEx(&cfg, k_ternary_pack<false>, Wv, nwords, th, pk);
+    return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------
@@ -117,7 +130,7 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
     const long long nvec = Kmax / epv;
     bool subln = false;
     for (int i = 0; i < P.count; ++i) subln |= P.p[i].gain != nullptr;
-    if (!subln && nvec <= 8 * 32) {
+    if (!subln && nvec <= 16 * 32) {
         // short rows: one warp per row
         int vpl = 1;
         while (vpl * 32 < nvec) vpl *= 2;
@@ -132,10 +145,12 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
         BL_AQW_CASE(true, 2)
         BL_AQW_CASE(true, 4)
         BL_AQW_CASE(true, 8)
+        BL_AQW_CASE(true, 16)
         BL_AQW_CASE(false, 1)
         BL_AQW_CASE(false, 2)
         BL_AQW_CASE(false, 4)
         BL_AQW_CASE(false, 8)
+        BL_AQW_CASE(false, 16)
 #undef BL_AQW_CASE
     }
     int vec = 1;

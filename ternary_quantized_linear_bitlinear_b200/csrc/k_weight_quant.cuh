@@ -2,14 +2,17 @@
 // 2-bit packing ("Distillix" README, 1. BitNet b1.58 Core; "bitone" README,
 // Forward pass; "SLM750-Edge" section 3.1).
 //
-// Three launches, all on the caller's stream:
+// Two launches, both on the caller's stream:
 //   k_absmean_partial  one pass over W: exact per-block sum of |w| as a
-//                      384-bit fixed-point integer in units of 2^-149
-//   k_gamma_finalize   one warp: sums the block partials, rounds once to
-//                      double, gamma = float(S / n) + 1e-5f, and the float
-//                      threshold T with  |w| >= T  <=>  float(|w|/gamma) > 0.5
+//                      384-bit fixed-point integer in units of 2^-149; the
+//                      last block to finish (ticket counter) sums the block
+//                      partials, rounds once to double, gamma = float(S / n)
+//                      + 1e-5f, and the float threshold T with
+//                      |w| >= T  <=>  float(|w|/gamma) > 0.5
 //   k_ternary_pack     second pass over W: code = sign(w) * (|w| >= T), four
-//                      codes per byte in the packed word layout
+//                      codes per byte in the packed word layout; launched as
+//                      a programmatic dependent, it loads its first words of
+//                      W before waiting for gamma and T
 //
 // Exactness: every finite float is an integer multiple of 2^-149, so sum|w|
 // is an integer in those units.  Each thread accumulates m << (e - base) in a
@@ -29,7 +32,8 @@ constexpr int WQ_WINDOW = 25;       // fast path: base <= e <= base + 25
 constexpr int WQ_PART_LIMBS = 6;    // per-block partial, 384 bits
 constexpr int WQ_MAX_BLOCKS = 1024;
 constexpr size_t WQ_WS_PARTIALS = (size_t)WQ_MAX_BLOCKS * WQ_PART_LIMBS * 8;
-constexpr size_t WQ_WS_BYTES = WQ_WS_PARTIALS + 256;  // + threshold scratch
+constexpr size_t WQ_WS_BYTES = WQ_WS_PARTIALS + 256;  // + threshold word, ticket counter
+constexpr size_t WQ_WS_TICKET = WQ_WS_PARTIALS + 128;  // u32, zeroed by the host before each reduction
 
 // Float bits of the j-th element of a 16-byte vector.
 template <bool BF16>
@@ -43,9 +47,71 @@ __device__ __forceinline__ u32 vec_elem_bits(const uint4 &v, int j) {
     }
 }
 
+// Sums the block partials (one limb position per pass, 128 bits per limb
+// across the block), rounds the total to double and derives gamma and T.
+// Whole block; thread 0 writes the results.
+__device__ void wq_finalize_block(const u64 *partials, int nblocks, long long n, float *gamma_out,
+                                  u32 *ws_thresh) {
+    constexpr int NL = WQ_PART_LIMBS;
+    __shared__ u64 f_lo[NL][WQ_THREADS / 32], f_hi[NL][WQ_THREADS / 32];
+    const int tid = threadIdx.x;
+    u64 slo[NL], shi[NL];
+#pragma unroll
+    for (int k = 0; k < NL; ++k) slo[k] = shi[k] = 0ull;
+    for (int b = tid; b < nblocks; b += WQ_THREADS) {
+#pragma unroll
+        for (int k = 0; k < NL; ++k) {
+            // written by other blocks of this grid: bypass L1
+            const u64 v = __ldcg(partials + (size_t)b * NL + k);
+            const u64 t = slo[k] + v;
+            shi[k] += t < v ? 1ull : 0ull;
+            slo[k] = t;
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < NL; ++k) {
+        warp_sum_u128(slo[k], shi[k]);
+        if ((tid & 31) == 0) {
+            f_lo[k][tid >> 5] = slo[k];
+            f_hi[k][tid >> 5] = shi[k];
+        }
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // S = sum_k (hi:lo)_k << 64k over the warps, folded into NL + 2 limbs
+        u64 L[NL + 2];
+#pragma unroll
+        for (int k = 0; k < NL + 2; ++k) L[k] = 0ull;
+#pragma unroll
+        for (int k = 0; k < NL; ++k) {
+            u64 lo = 0ull, hi = 0ull;
+            for (int w = 0; w < WQ_THREADS / 32; ++w) {
+                const u64 t = lo + f_lo[k][w];
+                hi += f_hi[k][w] + (t < lo ? 1ull : 0ull);
+                lo = t;
+            }
+            limbs_add_u128_shl(L, lo, hi, 64 * k);
+        }
+        double S = limbs_to_double_rn(L, -149);
+        float mean = __double2float_rn(__ddiv_rn(S, (double)n));
+        float g = __fadd_rn(mean, 1e-5f);
+        // smallest t with float(t / g) > 0.5: start at g/2 (exact, quotient 0.5)
+        float t = __fmul_rn(0.5f, g);
+        for (int it = 0; it < 64 && !(__fdiv_rn(t, g) > 0.5f); ++it)
+            t = __uint_as_float(__float_as_uint(t) + 1u);
+        gamma_out[0] = g;
+        ws_thresh[0] = __float_as_uint(t);
+    }
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const uint4 *__restrict__ W, long long nvec,
-                                                                 u64 *__restrict__ partials) {
+                                                                 long long n, u64 *__restrict__ partials,
+                                                                 float *__restrict__ gamma_out,
+                                                                 u32 *__restrict__ ws_thresh,
+                                                                 u32 *__restrict__ ticket) {
+    // the pack kernel may start loading W while this grid runs
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int EPV = BF16 ? 8 : 4;  // elements per 16-byte vector
     __shared__ u64 s_bins[256];
     __shared__ u32 s_emax;
@@ -140,47 +206,20 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const uint4 *__r
             for (int k = 0; k < WQ_PART_LIMBS; ++k) partials[(size_t)blockIdx.x * WQ_PART_LIMBS + k] = L[k];
         }
     }
-}
 
-// One warp.  Writes gamma and the threshold bits (as u32) into ws_thresh.
-// Each limb position is summed across the block partials as a 128-bit value
-// (lanes, then a shuffle tree), and lane 0 folds the limb sums with carries.
-__global__ void __launch_bounds__(32) k_gamma_finalize(const u64 *__restrict__ partials, int nblocks,
-                                                         long long n, float *__restrict__ gamma_out,
-                                                         u32 *__restrict__ ws_thresh) {
-    constexpr int NL = WQ_PART_LIMBS;
-    const int lane = threadIdx.x;
-    u64 slo[NL], shi[NL];
-#pragma unroll
-    for (int k = 0; k < NL; ++k) slo[k] = shi[k] = 0ull;
-    for (int b = lane; b < nblocks; b += 32) {
-#pragma unroll
-        for (int k = 0; k < NL; ++k) {
-            const u64 v = partials[(size_t)b * NL + k];
-            const u64 t = slo[k] + v;
-            shi[k] += t < v ? 1ull : 0ull;
-            slo[k] = t;
-        }
+    // The last block to finish finalizes (partials published with a fence
+    // before the ticket; the ticket is zeroed by the host before the launch
+    // and reset here for the next call on the same workspace).
+    __shared__ bool s_last;
+    if (tid == 0) {
+        __threadfence();
+        s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
     }
-#pragma unroll
-    for (int k = 0; k < NL; ++k) warp_sum_u128(slo[k], shi[k]);
-    if (lane == 0) {
-        // S = sum_k (shi[k]:slo[k]) << 64k, folded into NL + 2 limbs
-        u64 L[NL + 2];
-#pragma unroll
-        for (int k = 0; k < NL + 2; ++k) L[k] = 0ull;
-#pragma unroll
-        for (int k = 0; k < NL; ++k) limbs_add_u128_shl(L, slo[k], shi[k], 64 * k);
-        double S = limbs_to_double_rn(L, -149);
-        float mean = __double2float_rn(__ddiv_rn(S, (double)n));
-        float g = __fadd_rn(mean, 1e-5f);
-        // smallest t with float(t / g) > 0.5: start at g/2 (exact, quotient 0.5)
-        float t = __fmul_rn(0.5f, g);
-        for (int it = 0; it < 64 && !(__fdiv_rn(t, g) > 0.5f); ++it)
-            t = __uint_as_float(__float_as_uint(t) + 1u);
-        gamma_out[0] = g;
-        ws_thresh[0] = __float_as_uint(t);
-    }
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    wq_finalize_block(partials, gridDim.x, n, gamma_out, ws_thresh);
+    if (tid == 0) *ticket = 0u;
 }
 
 // Each thread packs 16 consecutive weights into one 32-bit word per step.
@@ -189,12 +228,21 @@ __global__ void __launch_bounds__(256) k_ternary_pack(const uint4 *__restrict__ 
                                                         const u32 *__restrict__ ws_thresh,
                                                         u32 *__restrict__ packed) {
     constexpr int VPW = BF16 ? 2 : 4;  // 16-byte vectors per 16 weights
-    const u32 T = ws_thresh[0];
     const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long wi = (long long)blockIdx.x * blockDim.x + threadIdx.x; wi < nwords; wi += stride) {
-        uint4 v[VPW];
+    long long wi = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    // first words of W are requested before waiting for the reduction grid
+    uint4 v[VPW];
+    if (wi < nwords) {
 #pragma unroll
         for (int q = 0; q < VPW; ++q) v[q] = ldg_stream_v4(W + wi * VPW + q);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    const u32 T = __ldcg(ws_thresh);
+    for (; wi < nwords; wi += stride) {
+        if (wi != (long long)blockIdx.x * blockDim.x + threadIdx.x) {
+#pragma unroll
+            for (int q = 0; q < VPW; ++q) v[q] = ldg_stream_v4(W + wi * VPW + q);
+        }
         u32 word = 0;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {

@@ -68,6 +68,22 @@ def test_quant_weights(N, K, dtype, kind):
         assert int(packed.sum()) == 0
 
 
+def test_quant_weights_workspace_contents_ignored_and_reused():
+    """The workspace may hold anything on entry (here all 0xFF bytes), and back-to-back
+    calls on one workspace and stream (the second launched while the first may still
+    run) give each tensor's own result."""
+    Ws = [workloads.normal((300, 4096), 0.02, 31, torch.bfloat16), workloads.normal((37, 192), 0.03, 32),
+          workloads.normal((2048, 768), 0.02, 33, torch.bfloat16)]
+    ws = torch.full((api.quant_weights_workspace_bytes(2048, 4096),), 255, dtype=torch.uint8, device="cuda")
+    outs = []
+    for W in Ws:
+        Wd = W.cuda()
+        outs.append(api.bl_quant_weights(Wd, workspace=ws))
+    api.bl_check_device_error()
+    for W, (packed, gamma) in zip(Ws, outs):
+        check_weights(W, packed, gamma)
+
+
 # -- step 2 --------------------------------------------------------------------
 
 def _wide_rows(M, K, seed):
@@ -80,6 +96,9 @@ def _wide_rows(M, K, seed):
 @pytest.mark.parametrize("M,K,dtype,subln,kind", [
     (16, 768, torch.float32, False, "outlier"),
     (5, 3200, torch.bfloat16, False, "outlier"),
+    (3, 2048, torch.float32, False, "outlier"),
+    (7, 4096, torch.bfloat16, False, "student"),
+    (70, 4032, torch.bfloat16, False, "normal"),
     (3, 64, torch.float32, False, "normal"),
     (2, 32768, torch.float32, False, "normal"),
     (2, 32768, torch.bfloat16, True, "normal"),
