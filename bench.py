@@ -2,14 +2,16 @@
 
 One step = the decode hot path for every projection of all 12 layers
 (q,o 768x768; k,v 256x768; gate,up 2048x768; down 768x2048 -- 84 problems)
-at M = 1, 4 and 8 tokens: per M, one grouped activation-quant launch and one
-grouped ternary GEMV launch.  The ternary weights (29/42/29 split) are
-packed once at load time.  Weight bytes per step would fit in L2, so the
-packed weights are replicated and every step reads a different replica
-(the replicas total more than 3x the L2 size).
+at M = 1, 4 and 8 tokens: per M, ONE grouped launch that quantizes the bf16
+activations, runs the ternary GEMV and rescales (bl_linear_decode_grouped).
+The ternary weights (29/42/29 split) are packed once at load time.  Weight
+bytes per step would fit in L2, so the packed weights are replicated and
+every step reads a different replica (the replicas total more than 3x the
+L2 size).
 
-Metric: decode GB/s = (packed weight bytes + x_q bytes) per step / time,
-whole job, N GPUs = N independent replicas of the workload (weak scaling).
+Metric: decode GB/s = (packed weight bytes + bf16 activation bytes) per step
+/ time, whole job, N GPUs = N independent replicas of the workload (weak
+scaling).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 """
@@ -198,77 +200,89 @@ def native(args, rank, world, local):
         Xs = [X[:M].contiguous() for _, _, X in items]
         xin_host[M] = torch.cat([x.view(-1) for x in Xs]).pin_memory()
         xin[M] = xin_host[M].to(dev)
-        xq[M] = torch.empty(xin[M].numel(), dtype=torch.int8, device=dev)
-        sc[M] = torch.empty(len(items) * SPAD[M], dtype=torch.float32, device=dev)  # 16-byte aligned per problem
+        xq[M] = torch.empty(xin[M].numel(), dtype=torch.int8, device=dev)  # two-launch path only
+        sc[M] = torch.empty(len(items) * SPAD[M], dtype=torch.float32, device=dev)
         ytot = sum(M * N for N, _ in shapes)
         Y[M] = torch.empty(ytot + 4 * len(items), dtype=torch.float32, device=dev)
         y_host[M] = torch.empty_like(Y[M], device="cpu").pin_memory()
 
     def views(M):
         """Per-problem device views into the contiguous buffers (16-byte aligned)."""
-        act, fwd = [], []
+        out = []
         xo = yo = 0
         for i, (N, K) in enumerate(shapes):
-            xv = xin[M][xo:xo + M * K].view(M, K)
-            qv = xq[M][xo:xo + M * K].view(M, K)
-            sv = sc[M][i * SPAD[M]:i * SPAD[M] + M]
-            yv = Y[M][yo:yo + M * N].view(M, N)
-            act.append((xv, None, qv, sv))
-            fwd.append((qv, sv, yv, N, K))
+            out.append((xin[M][xo:xo + M * K], xq[M][xo:xo + M * K], sc[M][i * SPAD[M]:i * SPAD[M] + M],
+                        Y[M][yo:yo + M * N], N, K))
             xo += M * K
             yo += (M * N + 3) // 4 * 4
-        return act, fwd
+        return out
 
-    def act_problems(act):
-        arr = (api.ActProblem * len(act))()
-        for i, (X, g, q, s) in enumerate(act):
-            arr[i] = api.ActProblem(X.data_ptr(), None, q.data_ptr(), s.data_ptr(), X.shape[1])
-        return arr
-
-    def fwd_problems(fwd, rep):
-        arr = (api.Problem * len(fwd))()
+    def fused_problems(M, rep, sel=None):
+        v = views(M)
+        idx = range(len(v)) if sel is None else sel
+        arr = (api.DecodeProblem * len(idx))()
         base = replicas[rep].data_ptr()
-        for i, (q, s, y, N, K) in enumerate(fwd):
-            arr[i] = api.Problem(base + offs[i], gammas[i].data_ptr(), q.data_ptr(), s.data_ptr(), y.data_ptr(),
-                                 None, N, K)
+        for j, i in enumerate(idx):
+            X, _, _, y, N, K = v[i]
+            arr[j] = api.DecodeProblem(base + offs[i], gammas[i].data_ptr(), X.data_ptr(), None, y.data_ptr(), None,
+                                       None, None, N, K)
         return arr
+
+    def two_launch_problems(M, rep):
+        v = views(M)
+        acts = (api.ActProblem * len(v))()
+        fwd = (api.Problem * len(v))()
+        base = replicas[rep].data_ptr()
+        for i, (X, q, s_, y, N, K) in enumerate(v):
+            acts[i] = api.ActProblem(X.data_ptr(), None, q.data_ptr(), s_.data_ptr(), K)
+            fwd[i] = api.Problem(base + offs[i], gammas[i].data_ptr(), q.data_ptr(), s_.data_ptr(), y.data_ptr(), None,
+                                 N, K)
+        return acts, fwd
 
     L = api.lib()
-    acts = {M: act_problems(views(M)[0]) for M in MS}
-    fwds = {(M, r): fwd_problems(views(M)[1], r) for M in MS for r in range(R)}
     count = len(items)
+    fused = {(M, r): fused_problems(M, r) for M in MS for r in range(R)}
+    RDY = api.BL_FWD_WEIGHTS_READY
 
-    def launch_step(stream_ptr, rep, decode_only=False):
+    def launch_step(stream_ptr, rep):
+        """One step: per M, ONE fused launch (act quant + GEMV + rescale, 84 problems)."""
         for M in MS:
-            if not decode_only:
-                rc = L.bl_quant_act_grouped(acts[M], count, api.BL_BF16, M, 1e-6, stream_ptr)
-                if rc:
-                    raise api.BitLinearError(rc, "bl_quant_act_grouped")
-            rc = L.bl_forward_grouped(fwds[(M, rep)], count, M, api.BL_FWD_WEIGHTS_READY, stream_ptr)
+            rc = L.bl_linear_decode_grouped(fused[(M, rep)], count, api.BL_BF16, M, 1e-6, RDY, stream_ptr)
             if rc:
-                raise api.BitLinearError(rc, "bl_forward_grouped")
+                raise api.BitLinearError(rc, "bl_linear_decode_grouped")
 
-    # ---- capture one cycle (R steps, one per replica) as a CUDA graph ------
     stream = torch.cuda.Stream(device=dev)
     sp = stream.cuda_stream
-    with torch.cuda.stream(stream):
-        for r in range(R):  # eager warm-up: also runs the one-time device set-up
-            launch_step(sp, r)
-    torch.cuda.synchronize()
 
-    def capture(decode_only):
+    def graph_of(fn, reps):
+        with torch.cuda.stream(stream):  # eager warm-up: also runs the one-time device set-up
+            for r in range(reps):
+                fn(sp, r)
+        torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            for r in range(R):
-                launch_step(stream.cuda_stream, r, decode_only)
+            for r in range(reps):
+                fn(stream.cuda_stream, r)
+        torch.cuda.synchronize()
         return g
 
-    g_step = capture(False)
-    g_dec = capture(True)
-    torch.cuda.synchronize()
+    def time_graph(g, replays):
+        with torch.cuda.stream(stream):
+            g.replay()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(replays):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1)
 
-    K, Wm = args.steps, max(3, args.warmup)
-    cycles = max(1, (K + R - 1) // R)
+    # ---- capture one cycle (R steps, one per replica) as a CUDA graph ------
+    g_step = graph_of(launch_step, R)
+
+    K_, Wm = args.steps, max(3, args.warmup)
+    cycles = max(1, (K_ + R - 1) // R)
     steps_timed = cycles * R
     for _ in range(max(1, (Wm + R - 1) // R)):
         g_step.replay()
@@ -289,23 +303,13 @@ def native(args, rank, world, local):
     barrier(world)
     ms_total = max_over_ranks(ev0.elapsed_time(ev1), world)
     ms_per_step = ms_total / steps_timed
-    bytes_step = sum(wbytes + xbytes[M] for M in MS)
+    bytes_step = sum(wbytes + 2 * xbytes[M] for M in MS)  # packed W + bf16 X read by the fused kernel
     value = world * bytes_step * steps_timed / (ms_total * 1e-3) / 1e9
+    api.bl_check_device_error(stream)
 
-    # ---- dominant kernel alone: the grouped GEMV launches ------------------
-    with torch.cuda.stream(stream):
-        d0 = torch.cuda.Event(enable_timing=True)
-        d1 = torch.cuda.Event(enable_timing=True)
-        g_dec.replay()
-        d0.record(stream)
-        dec_cycles = max(1, cycles // 2)
-        for _ in range(dec_cycles):
-            g_dec.replay()
-        d1.record(stream)
-    torch.cuda.synchronize()
-    dec_launches = dec_cycles * R * len(MS)
-    dec_us = d0.elapsed_time(d1) * 1e3 / dec_launches
-    dec_bytes = sum(wbytes + xbytes[M] for M in MS) / len(MS)  # per launch, averaged over M
+    # ---- the dominant kernel: every launch of the step is the fused GEMV ---
+    dec_us = ev0.elapsed_time(ev1) * 1e3 / (steps_timed * len(MS))  # this rank's launches
+    dec_bytes = bytes_step / len(MS)  # per launch, averaged over M
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -313,15 +317,54 @@ def native(args, rank, world, local):
         pass
     peak = float(peaks.get("hbm_gbs", 6650.0))
     achieved = dec_bytes / (dec_us * 1e-6) / 1e9
-    traffic = decode_traffic()
-    roofline = {"bound": "hbm", "kernel": "k_decode (grouped GEMV, 84 problems)", "achieved": round(achieved, 1),
-                "peak": peak, "peak_source": "measured" if "hbm_gbs" in peaks else "fallback",
-                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": traffic,
-                "avg_launch_us": round(dec_us, 3)}
+    roofline = {"bound": "hbm", "kernel": "k_decode<1, bf16> (fused act quant + ternary GEMV + rescale, 84 problems)",
+                "achieved": round(achieved, 1), "peak": peak,
+                "peak_source": "measured" if "hbm_gbs" in peaks else "fallback",
+                "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": decode_traffic(),
+                "avg_launch_us": round(dec_us, 3), "algorithmic_bytes_per_launch": int(dec_bytes)}
+
+    # ---- secondary: the same step as two launches per M (act quant, GEMV) -
+    alt = {}
+    if not args.no_e2e:
+        tl = {(M, r): two_launch_problems(M, r) for M in MS for r in range(R)}
+
+        def two_step(stream_ptr, rep):
+            for M in MS:
+                acts, fwd = tl[(M, rep)]
+                if L.bl_quant_act_grouped(acts, count, api.BL_BF16, M, 1e-6, stream_ptr):
+                    raise RuntimeError("bl_quant_act_grouped")
+                if L.bl_forward_grouped(fwd, count, M, RDY, stream_ptr):
+                    raise RuntimeError("bl_forward_grouped")
+
+        g2 = graph_of(two_step, R)
+        alt["two_launch_us_per_step"] = round(time_graph(g2, max(1, cycles // 4)) * 1e3 / (R * max(1, cycles // 4)), 3)
+        del g2
+        # layer order at M = 1: per layer qkv | o | gate, up | down (4 grouped launches, 48 per step)
+        stages = []
+        per_layer = len(workloads.decode125m_layer_shapes())
+        for layer in range(count // per_layer):
+            b0 = layer * per_layer
+            for sel in ((0, 1, 2), (3,), (4, 5), (6,)):
+                stages.append([b0 + j for j in sel])
+        lay = {r: [fused_problems(1, r, sel) for sel in stages] for r in range(R)}
+
+        def layered_step(stream_ptr, rep):
+            for arr, sel in zip(lay[rep], stages):
+                if L.bl_linear_decode_grouped(arr, len(sel), api.BL_BF16, 1, 1e-6, RDY, stream_ptr):
+                    raise RuntimeError("bl_linear_decode_grouped")
+
+        g3 = graph_of(layered_step, R)
+        reps3 = max(1, cycles // 4)
+        us3 = time_graph(g3, reps3) * 1e3 / (R * reps3)
+        alt["layered_m1_us_per_step"] = round(us3, 3)
+        alt["layered_m1_gbs"] = round((wbytes + 2 * xbytes[1]) / (us3 * 1e-6) / 1e9, 1)
+        alt["layered_m1_launches_per_step"] = len(stages)
+        del g3
+        api.bl_check_device_error(stream)
+
     # ---- end to end through the C ABI with host buffers --------------------
     e2e = None
     if not args.no_e2e:
-        act_v = {M: views(M) for M in MS}
         h2d = sum(xin_host[M].numel() * 2 for M in MS)
         d2h = sum(y_host[M].numel() * 4 for M in MS)
         n_e2e = max(3, min(steps_timed, 300))
@@ -339,18 +382,18 @@ def native(args, rank, world, local):
         e2e_s = max_over_ranks(time.perf_counter() - t0, world)
         e2e = {"value": round(world * bytes_step * n_e2e / e2e_s / 1e9, 2), "unit": UNIT,
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
-        del act_v
 
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": steps_timed,
         "warmup": Wm, "ms_per_step": round(ms_per_step, 6), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
         "config": {"workload": WORKLOAD, "tokens_per_step": sum(MS), "projections": count,
-                   "weight_bytes_per_m": wbytes, "weight_replicas": R,
+                   "weight_bytes_per_m": wbytes, "activation_bytes_per_step": sum(2 * xbytes[M] for M in MS),
+                   "weight_replicas": R,
                    "l2": f"{R} rotating packed-weight replicas ({R * wbytes / 2**20:.0f} MiB > 3x L2)",
-                   "parallelism": f"replicas x{world}", "launch": "CUDA graph of whole steps"},
-        "roofline": roofline, "e2e": e2e,
-        "gpu_launches": steps_timed * 2 * len(MS),
+                   "parallelism": f"replicas x{world}", "launch": "CUDA graph of whole steps, 3 fused launches each"},
+        "roofline": roofline, "e2e": e2e, "alt_paths": alt,
+        "gpu_launches": steps_timed * len(MS),
     }
     out["clocks"] = clk.summary()
     return out
@@ -455,7 +498,7 @@ def cpu_baseline():
     wbytes, xbytes = step_bytes()
     items = oracle_items()
     secs = cpu_oracle_step(items, wbytes, xbytes)
-    bytes_step = sum(wbytes + xbytes[M] for M in MS)
+    bytes_step = sum(wbytes + 2 * xbytes[M] for M in MS)
     return {"value": round(bytes_step / secs / 1e9, 4), "unit": UNIT, "cores": oracle.num_threads(),
             "kind": "oracle",
             "sample": "one whole step (84 projections at M = 1, 4, 8: act quant, int64 contraction, rescale); "
@@ -492,7 +535,7 @@ def reference(args, rank, world):
         n = min(rows, wq.shape[0])
         xq, s = oracle.quant_act(X[:M])
         oracle.rescale(oracle.contract(xq, wq[:n]), g, s[:, None])
-        done_bytes += n * wq.shape[1] // 4 + M * wq.shape[1]
+        done_bytes += n * wq.shape[1] // 4 + 2 * M * wq.shape[1]
     secs = time.perf_counter() - t_start
     value = done_bytes / secs / 1e9
     return {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": world,
