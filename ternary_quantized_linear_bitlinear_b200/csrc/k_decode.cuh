@@ -316,7 +316,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) k_decode(const __grid_constant
 
     // One thread requests the CTA's weight rows, one bulk copy (and one
     // mbarrier) per 32-row group, so each warp starts as soon as its rows land.
-    if (threadIdx.x == 0) {
+    // It is lane 0 of the last warp: the fused path quantizes token row m in
+    // warp m, so for small M the first rows do not wait for the requests.
+    if (threadIdx.x == DEC_THREADS - 32) {
         for (int i = 0; i < groups; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         const uint8_t *src = pr.packed + (size_t)row_base * Kw;

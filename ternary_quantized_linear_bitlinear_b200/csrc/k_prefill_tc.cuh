@@ -48,8 +48,8 @@ namespace bl {
 constexpr int PF_BM = 128;         // tokens per tile (MMA M, TMEM lanes)
 constexpr int PF_BN = 256;         // weight rows per tile (MMA N, TMEM columns)
 constexpr int PF_BK = 128;         // k per pipeline stage (4 MMAs of K = 32)
-constexpr int PF_STAGES = 3;       // TMA stages (x_q + packed)
-constexpr int PF_BSTAGES = 3;      // expanded-weight stages
+constexpr int PF_STAGES = 4;       // TMA stages (x_q + packed)
+constexpr int PF_BSTAGES = 2;      // expanded-weight stages
 constexpr int PF_EXP_WARPS = PF_BN / 32;
 constexpr int PF_EPI_WARPS = 8;
 constexpr int PF_EPI_WARP0 = 2 + PF_EXP_WARPS;
