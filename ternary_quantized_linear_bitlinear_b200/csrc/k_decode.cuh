@@ -114,10 +114,12 @@ __device__ __forceinline__ u32 dec_x_bits(const uint4 &v, int j) {
     return BF16 ? ((j & 1) ? (w & 0xffff0000u) : (w << 16)) : w;
 }
 
-// A row of X is processed in blocks of 256 16-byte vectors, 8 per lane
-// (vector blk * 256 + 32 i + lane in register i, zero past the row end); a
+// A row of X is processed in blocks of 128 16-byte vectors, 4 per lane
+// (vector blk * 128 + 32 i + lane in register i, zero past the row end); a
 // row of at most one block is loaded once and every pass works on registers.
-constexpr int DEC_QV = 8;
+// (Four, not eight: the fused kernel runs once per CTA and its code is cold
+// in the instruction cache, so a shorter unrolled body is faster.)
+constexpr int DEC_QV = 4;
 
 __device__ __forceinline__ void dec_load_block(uint4 (&c)[DEC_QV], const uint4 *xr, int nvec, int blk, int lane) {
 #pragma unroll
@@ -423,7 +425,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) k_decode(const __grid_constant
             o0[c] = (c ^ xb0) << 4;
             o1[c] = (c ^ xb1) << 4;
         }
-#pragma unroll 2
+#pragma unroll 1
         for (int s2 = kslot; s2 < steps; s2 += G) {
             const bool kv = (s2 * 4 + t) < nchunk64;
             uint4 wv[4];
