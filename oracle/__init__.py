@@ -50,6 +50,7 @@ def _lib():
             "oracle_unpack": (ctypes.c_int, [_ptr, _i64, _i64, _ptr]),
             "oracle_rmsnorm": (ctypes.c_int, [_ptr, _i64, _ptr, _f32, _ptr]),
             "oracle_quant_act": (ctypes.c_int, [_ptr, _i64, _i64, _ptr, _f32, _ptr, _ptr, _ptr]),
+            "oracle_ffn_act": (None, [_ptr, _ptr, _i64, _ptr]),
             "oracle_contract": (None, [_ptr, _ptr, _i64, _i64, _i64, _ptr]),
             "oracle_contract_pairs": (None, [_ptr, _ptr, _i64, _ptr, _ptr, _i64, _ptr]),
             "oracle_rescale": (None, [_ptr, _i64, _f32, _ptr, _ptr]),
@@ -163,6 +164,23 @@ def quant_act(X, gain=None, eps: float = 1e-6):
         rc = _lib().oracle_quant_act(_p(X), M, K, _p(g), np.float32(eps), _p(xq), _p(s), _p(y))
     _check(rc, "quant_act")
     return xq, s
+
+
+def ffn_act(gate, up) -> np.ndarray:
+    """h = relu(gate)^2 * up elementwise, float32 ("SLM750-Edge", Key
+    Architectural Features: ReLU2; section 2.3: gate / up / down)."""
+    g = _f32c(gate)
+    u = _f32c(up)
+    if g.shape != u.shape:
+        raise OracleError("ffn_act: gate and up shapes differ")
+    h = np.zeros_like(g)
+    _lib().oracle_ffn_act(_p(g), _p(u), g.size, _p(h))
+    return h
+
+
+def ffn_act_quant(gate, up, gain=None, eps: float = 1e-6):
+    """(x_q, s) of the down projection's input: quant_act(ffn_act(gate, up))."""
+    return quant_act(ffn_act(gate, up), gain, eps)
 
 
 # -- steps 4, 5 -------------------------------------------------------------

@@ -301,6 +301,23 @@ int oracle_quant_act(const float *X, int64_t M, int64_t K, const float *gain, fl
 }
 
 /* ------------------------------------------------------------------------ */
+/* FFN activation between the up and down projections: "SLM750-Edge" model  */
+/* card, "Key Architectural Features" (FFN activation ReLU2, relu(x)^2) and   */
+/* section 2.3 (per-layer FFN gate, up and down projections).  Reading: the   */
+/* gated form h = relu(gate)^2 * up, each step a float operation:             */
+/*   r = gate > 0 ? gate : 0;  h = float(float(r * r) * up).                  */
+/* h is the input of the down projection's SubLN + activation quantizer       */
+/* ("BitDistill", Stage 1), i.e. oracle_quant_act on h.                       */
+/* ------------------------------------------------------------------------ */
+void oracle_ffn_act(const float *gate, const float *up, int64_t n, float *h) {
+    for (int64_t i = 0; i < n; ++i) {
+        float r = gate[i] > 0.0f ? gate[i] : 0.0f;
+        float sq = r * r;
+        h[i] = sq * up[i];
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Step 4: exact contraction; step 5: rescale.                                */
 /* ------------------------------------------------------------------------ */
 

@@ -349,3 +349,48 @@ def test_linear_small_golden():
     assert float(out["s"][0]) == float(rows["s"])
     assert out["acc"][0].tolist() == [int(v) for v in rows["acc"].split()]
     assert out["Y"][0].tolist() == [a * float(out["gamma"]) for a in (-6.0, -183.0)]
+
+
+# -- FFN activation (ReLU^2-gated) feeding the down projection ---------------
+
+def test_ffn_act_relu_closed_forms():
+    """relu(g)^2 * u: g <= 0 gives 0; g = 1 gives u; g = 2^k gives u * 4^k
+    exactly (SLM750-Edge, Key Architectural Features: ReLU2)."""
+    rng = np.random.default_rng(7)
+    u = rng.standard_normal(64).astype(np.float32)
+    for g0 in (-3.5, -1e-30, -0.0, 0.0):
+        h = oracle.ffn_act(np.full(64, g0, np.float32), u)
+        assert np.all(h == 0.0)
+    assert np.array_equal(oracle.ffn_act(np.ones(64, np.float32), u), u)
+    for k in range(-10, 11):
+        g = np.full(64, 2.0 ** k, np.float32)
+        assert np.array_equal(oracle.ffn_act(g, u), (u.astype(np.float64) * 4.0 ** k).astype(np.float32))
+
+
+def test_ffn_act_two_roundings_exact():
+    """Each product of two floats is exact in double (48-bit mantissa), so
+    float(float(r * r) * u) is two correctly rounded conversions of exact
+    products."""
+    rng = np.random.default_rng(8)
+    g = (rng.standard_normal(4096) * 3).astype(np.float32)
+    u = (rng.standard_normal(4096) * 2).astype(np.float32)
+    h = oracle.ffn_act(g, u)
+    for gi, ui, hi in zip(g.tolist(), u.tolist(), h.tolist()):
+        r = gi if gi > 0 else 0.0
+        sq = float(np.float32(r * r))          # r * r exact in double, one rounding to float
+        want = float(np.float32(sq * ui))      # sq * u exact in double, one rounding
+        assert hi == want or (hi == 0.0 and want == 0.0)
+
+
+def test_ffn_act_quant_constant_row():
+    """gate = 2, up = c on every element: h = 4c, so every x_q is +-127 and
+    s = 127 / (4|c|); with SubLN (gain 1) y = h / sqrt(h^2 + eps) per element."""
+    c = np.float32(0.375)
+    g = np.full((2, 256), 2.0, np.float32)
+    u = np.full((2, 256), c, np.float32)
+    u[1] = -c
+    xq, s = oracle.ffn_act_quant(g, u)
+    assert xq[0].tolist() == [127] * 256 and xq[1].tolist() == [-127] * 256
+    assert s.tolist() == [float(np.float32(127.0) / np.float32(1.5))] * 2
+    xq2, s2 = oracle.ffn_act_quant(g, u, np.ones(256, np.float32), 1e-6)
+    assert xq2[0].tolist() == [127] * 256 and xq2[1].tolist() == [-127] * 256
