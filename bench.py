@@ -451,12 +451,39 @@ def prefill(args, dev):
         torch.cuda.synchronize()
         ms = e0.elapsed_time(e1) / reps
         out[label] = {"ms_per_layer": round(ms, 4), "tops": round(ops / (ms * 1e-3) / 1e12, 1)}
+    # FFN activation + SubLN + act quant feeding the down projection (bl_ffn_act_quant)
+    F = workloads.PREFILL1B4["ffn"]
+    gate = workloads.normal((M, F), 1.5, 60).to(dev)
+    up = workloads.normal((M, F), 1.0, 61).to(dev)
+    fgain = workloads.uniform((F,), 0.9, 1.1, 62).to(dev)
+    fxq = torch.empty(M, F, dtype=torch.int8, device=dev)
+    fs = torch.empty(M, dtype=torch.float32, device=dev)
+
+    def ffn():
+        rc = L.bl_ffn_act_quant(gate.data_ptr(), up.data_ptr(), M, F, fgain.data_ptr(), 1e-6, fxq.data_ptr(),
+                                fs.data_ptr(), sp)
+        if rc:
+            raise api.BitLinearError(rc, "bl_ffn_act_quant")
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            ffn()
+        f0 = torch.cuda.Event(enable_timing=True)
+        f1 = torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(reps):
+            ffn()
+        f1.record(stream)
+    torch.cuda.synchronize()
+    ffn_us = f0.elapsed_time(f1) * 1e3 / reps
+    ffn_bytes = 2 * M * F * 4 + M * F + 4 * M
     api.bl_check_device_error(stream)
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
     except (OSError, ValueError):
         pass
+    hbm = float(peaks.get("hbm_gbs", 6650.0))
     # int8 dense peak = measured bf16 dense peak x the nominal int8:bf16 ratio (4.5 : 2.25)
     bf16 = float(peaks.get("bf16_tflops", 1590.0))
     peak = 2.0 * bf16
@@ -468,6 +495,9 @@ def prefill(args, dev):
                          "peak_source": ("measured bf16 x 2 (nominal int8:bf16)" if "bf16_tflops" in peaks
                                          else "fallback bf16 x 2"),
                          "frac": round(out["engine"]["tops"] / peak, 4)},
+            "ffn_act_quant": {"shape": f"gate, up [{M}, {F}] f32 -> x_q [{M}, {F}] (ReLU^2 gate, SubLN)",
+                              "us": round(ffn_us, 2), "gbs": round(ffn_bytes / (ffn_us * 1e-6) / 1e9, 1),
+                              "frac_hbm": round(ffn_bytes / (ffn_us * 1e-6) / 1e9 / hbm, 4)},
             "reps": reps, "l2": "inputs and outputs of the layer total > 700 MB"}
 
 

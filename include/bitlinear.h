@@ -155,6 +155,26 @@ bl_status bl_quant_act(const void *X, bl_dtype xdt, int64_t M, int64_t K,
                        int8_t *x_q, float *s, bl_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Step 2 for the down projection, fused with the FFN activation before it.  */
+/*                                                                           */
+/* Defined by: "SLM750-Edge" model card, "Key Architectural Features" (FFN   */
+/* activation ReLU2, relu(x)^2) and section 2.3 (gate, up and down           */
+/* projections per layer); the gated reading h = relu(gate)^2 * up; then the */
+/* SubLN + activation quantizer of bl_quant_act on h ("BitDistill", Stage 1: */
+/* SubLN before down_proj):                                                  */
+/*                                                                           */
+/*   h   = float(float(r * r) * up),  r = gate > 0 ? gate : 0                */
+/*   x_q, s = bl_quant_act(h, subln_gain, subln_eps)   (h never stored)      */
+/*                                                                           */
+/* gate, up [M, F] float32 (the gate / up projections' Y); subln_gain [F] or */
+/* NULL; x_q [M, F] int8 out; s [M] out.  All device, 16-byte aligned.      */
+/* F obeys the K limits (64 <= F <= 32768, F % 64 == 0).                     */
+/* ------------------------------------------------------------------------ */
+bl_status bl_ffn_act_quant(const float *gate, const float *up, int64_t M, int64_t F,
+                           const float *subln_gain, float subln_eps,
+                           int8_t *x_q, float *s, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Steps 3 + 4: exact ternary x INT8 contraction and rescale.                */
 /*                                                                           */
 /* Defined by: "bitone" README, "How 1.58-bit Works" (each weight adds,      */

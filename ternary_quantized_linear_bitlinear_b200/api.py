@@ -60,6 +60,7 @@ _SIGS = {
     "bl_quant_weights": (_int, [_p, _int, _i64, _i64, _p, _p, _p, _sz, _p]),
     "bl_quant_weights_noalloc": (_int, [_p, _int, _i64, _i64, _p, _p, _p]),
     "bl_quant_act": (_int, [_p, _int, _i64, _i64, _p, _f32, _p, _p, _p]),
+    "bl_ffn_act_quant": (_int, [_p, _p, _i64, _i64, _p, _f32, _p, _p, _p]),
     "bl_forward": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, _p]),
     "bl_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_linear": (_int, [_p, _int, _p, _int, _i64, _i64, _i64, _p, _f32, _p, _sz, _p, _p]),
@@ -197,6 +198,25 @@ def bl_quant_act_grouped(items, dtype=torch.bfloat16, subln_eps: float = 1e-6, s
 
 
 # -- steps 3 + 4 ---------------------------------------------------------------
+
+def bl_ffn_act_quant(gate: torch.Tensor, up: torch.Tensor, subln_gain=None, subln_eps: float = 1e-6, x_q=None, s=None,
+                     stream=None):
+    """Down-projection input from the gate / up outputs: (x_q int8 [M, F], s [M])
+    of relu(gate)^2 * up, after SubLN when a gain is given."""
+    _dev(gate, "gate", torch.float32)
+    _dev(up, "up", torch.float32)
+    if gate.shape != up.shape:
+        raise ValueError("gate and up must have the same shape")
+    M, F = gate.shape
+    if x_q is None:
+        x_q = torch.empty(M, F, dtype=torch.int8, device=gate.device)
+    if s is None:
+        s = torch.empty(max(M, 4), dtype=torch.float32, device=gate.device)[:M]
+    rc = lib().bl_ffn_act_quant(gate.data_ptr(), up.data_ptr(), M, F, _ptr(subln_gain), subln_eps, x_q.data_ptr(),
+                                s.data_ptr(), _stream(stream))
+    _check(rc, "bl_ffn_act_quant")
+    return x_q, s
+
 
 def bl_forward(packed, gamma, x_q, s, N: int, Y=None, acc_out=None, stream=None):
     """-> Y float32 [M, N] (acc_out int32 [M, N] filled when given)."""

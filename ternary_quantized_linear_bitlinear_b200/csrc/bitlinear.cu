@@ -126,6 +126,7 @@ bl_status quant_weights_impl(const DeviceInfo &d, const void *W, bl_dtype wdt, i
 
 bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStream_t st) {
     const bool bf16 = xdt == BL_BF16;
+    const bool glu = P.p[0].X2 != nullptr;  // all problems of a call alike (f32 only)
     const int epv = bf16 ? 8 : 4;
     const long long nvec = Kmax / epv;
     bool subln = false;
@@ -138,7 +139,10 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
         const unsigned grid = (unsigned)((rows + AQW_WARPS - 1) / AQW_WARPS);
 #define BL_AQW_CASE(B, V)                                                         \
         if (bf16 == B && vpl == V) {                                              \
-            k_act_quant_warp<B, V><<<grid, AQW_WARPS * 32, 0, st>>>(P);           \
+            if (glu)                                                              \
+                k_act_quant_warp<false, V, true><<<grid, AQW_WARPS * 32, 0, st>>>(P); \
+            else                                                                  \
+                k_act_quant_warp<B, V><<<grid, AQW_WARPS * 32, 0, st>>>(P);       \
             return launch_status();                                               \
         }
         BL_AQW_CASE(true, 1)
@@ -159,7 +163,10 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
     const unsigned grid = (unsigned)(P.count * P.M);
 #define BL_AQ_CASE(B, V)                                                        \
     if (bf16 == B && vec == V) {                                                \
-        k_act_quant<B, V><<<grid, T, 0, st>>>(P);                               \
+        if (glu)                                                                \
+            k_act_quant<false, V, true><<<grid, T, 0, st>>>(P);                 \
+        else                                                                    \
+            k_act_quant<B, V><<<grid, T, 0, st>>>(P);                           \
         return launch_status();                                                 \
     }
     // at most 32 values per thread (bf16: 4 vectors, f32: 8 vectors)
@@ -322,6 +329,24 @@ bl_status bl_quant_act_grouped(const bl_act_problem *problems, int count, bl_dty
     bl_status rc = device_info(&d);
     if (rc) return rc;
     return quant_act_impl(P, xdt, kmax, (cudaStream_t)stream);
+}
+
+bl_status bl_ffn_act_quant(const float *gate, const float *up, int64_t M, int64_t F, const float *subln_gain,
+                           float subln_eps, int8_t *x_q, float *s, bl_stream_t stream) {
+    if (!gate || !up || !x_q || !s) return BL_ERR_NULL;
+    if (M < 1 || M > 0x7fffffffLL || check_k(F) != BL_OK) return BL_ERR_SHAPE;
+    if (!aligned16(gate) || !aligned16(up) || !aligned16(x_q) || !aligned16(s) ||
+        (subln_gain && !aligned16(subln_gain)))
+        return BL_ERR_ALIGN;
+    ActParams P;
+    P.count = 1;
+    P.M = (int)M;
+    P.eps = subln_eps;
+    P.p[0] = ActProblem{gate, subln_gain, x_q, s, (int)F, 0, up};
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return quant_act_impl(P, BL_F32, F, (cudaStream_t)stream);
 }
 
 bl_status bl_quant_act(const void *X, bl_dtype xdt, int64_t M, int64_t K, const float *subln_gain, float subln_eps,

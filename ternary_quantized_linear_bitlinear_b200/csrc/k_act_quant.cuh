@@ -30,7 +30,24 @@ struct ActProblem {
     float *s;
     int K;
     int pad;
+    const float *X2;  // GLU: the up projection's output (X is the gate's), f32
 };
+
+// The FFN activation between the up and down projections ("SLM750-Edge",
+// Key Architectural Features: ReLU2; section 2.3: gate, up, down):
+// h = float(float(r * r) * u), r = g > 0 ? g : 0.  With GLU the quantizer's
+// input x is this h, computed as the row is loaded.
+__device__ __forceinline__ float glu_relu2(float g, float u) {
+    const float r = g > 0.f ? g : 0.f;
+    return __fmul_rn(__fmul_rn(r, r), u);
+}
+
+__device__ __forceinline__ uint4 glu_relu2_v4(const uint4 &g, const uint4 &u) {
+    return make_uint4(__float_as_uint(glu_relu2(__uint_as_float(g.x), __uint_as_float(u.x))),
+                      __float_as_uint(glu_relu2(__uint_as_float(g.y), __uint_as_float(u.y))),
+                      __float_as_uint(glu_relu2(__uint_as_float(g.z), __uint_as_float(u.z))),
+                      __float_as_uint(glu_relu2(__uint_as_float(g.w), __uint_as_float(u.w))));
+}
 
 struct ActParams {
     ActProblem p[AQ_MAX_GROUP];
@@ -52,8 +69,9 @@ __device__ __forceinline__ float block_max_f(float v, float *s_red) {
 }
 
 // VEC: 16-byte vectors per thread; EPV elements per vector.
-template <bool BF16, int VEC>
+template <bool BF16, int VEC, bool GLU = false>
 __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ ActParams P) {
+    static_assert(!(GLU && BF16), "GLU inputs are float32 projection outputs");
     constexpr int EPV = BF16 ? 8 : 4;
     constexpr int VPT = VEC * EPV;
     __shared__ float s_red[32];
@@ -78,6 +96,8 @@ __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ A
     for (int v = 0; v < VEC; ++v) {
         int vi = tid + v * T;
         uint4 raw = vi < nvec ? ldg_stream_v4(xr + vi) : make_uint4(0, 0, 0, 0);
+        if (GLU && vi < nvec)
+            raw = glu_relu2_v4(raw, ldg_stream_v4(reinterpret_cast<const uint4 *>(pr.X2) + (size_t)m * nvec + vi));
         const u32 w4[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
         for (int j = 0; j < EPV; ++j) {
@@ -187,8 +207,9 @@ __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ A
 // row in registers, absmax by a warp reduction -- no block barrier at all.
 constexpr int AQW_WARPS = 8;
 
-template <bool BF16, int VPL>
+template <bool BF16, int VPL, bool GLU = false>
 __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_constant__ ActParams P) {
+    static_assert(!(GLU && BF16), "GLU inputs are float32 projection outputs");
     constexpr int EPV = BF16 ? 8 : 4;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int gw = blockIdx.x * AQW_WARPS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
@@ -203,6 +224,8 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_
     for (int v = 0; v < VPL; ++v) {
         const int vi = lane + v * 32;
         raw[v] = vi < nvec ? ldg_stream_v4(xr + vi) : make_uint4(0, 0, 0, 0);
+        if (GLU && vi < nvec)
+            raw[v] = glu_relu2_v4(raw[v], ldg_stream_v4(reinterpret_cast<const uint4 *>(pr.X2) + (size_t)m * nvec + vi));
         const u32 w4[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
 #pragma unroll
         for (int j = 0; j < EPV; ++j) {

@@ -120,6 +120,7 @@ __device__ __forceinline__ u32 dec_x_bits(const uint4 &v, int j) {
 // (Four, not eight: the fused kernel runs once per CTA and its code is cold
 // in the instruction cache, so a shorter unrolled body is faster.)
 constexpr int DEC_QV = 4;
+constexpr int DEC_QB = 8;  // block-cooperative quantization: X vectors per thread (M * K / 8 <= 2048 for bf16)
 
 __device__ __forceinline__ void dec_load_block(uint4 (&c)[DEC_QV], const uint4 *xr, int nvec, int blk, int lane) {
 #pragma unroll
@@ -291,6 +292,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) k_decode(const __grid_constant
     __shared__ int s_red[DEC_WARPS][2][NT][4][32];
     __shared__ __align__(8) u64 s_bar[DEC_WARPS];
     __shared__ float s_f[16];
+    __shared__ u32 s_amax[16];
+    __shared__ float s_sc[16];
+    if (SRC != DEC_SRC_XQ && threadIdx.x < 16) s_amax[threadIdx.x] = 0u;
 
     // a programmatically dependent launch that follows may start its prologue
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -347,12 +351,89 @@ __global__ void __launch_bounds__(DEC_THREADS, 3) k_decode(const __grid_constant
     const int RS = dec_row_stride(K);
     uint8_t *s_xq = smem + P.xq_off;
     if (SRC != DEC_SRC_XQ) {
-        // fused step 2: warp w quantizes rows w, w + 8
-        const int lane = threadIdx.x & 31;
+        constexpr bool BF16 = SRC == DEC_SRC_BF16;
+        constexpr int EPV = BF16 ? 8 : 4;
         const bool out = b == pr.cta_begin;
-        for (int m = threadIdx.x >> 5; m < M; m += DEC_WARPS) {
-            const float s = dec_quant_row<SRC == DEC_SRC_BF16>(pr, m, K, RS, s_xq, P.eps, out, lane);
-            if (lane == 0) s_f[m] = __fdiv_rn(*pr.gamma, s);
+        const int nvec = K / EPV;
+        const int tot = M * nvec;  // 16-byte vectors of X, rows contiguous
+        if (pr.gain == nullptr && M <= 2 && tot <= DEC_QB * DEC_THREADS) {
+            // fused step 2 for one or two tokens, no SubLN, all of X in
+            // registers: thread t holds vectors t + 256 i; one load round
+            // trip, per-row max by a warp reduction and a shared atomic (max
+            // of the float bits of |x|).  (Measured: faster than a warp per
+            // row for M <= 2, slower from M = 4 on.)
+            const uint4 *xv = reinterpret_cast<const uint4 *>(pr.x);
+            uint4 c[DEC_QB];
+#pragma unroll
+            for (int i = 0; i < DEC_QB; ++i) {
+                const int idx = (int)threadIdx.x + DEC_THREADS * i;
+                c[i] = idx < tot ? ldg_nc_v4(xv + idx) : make_uint4(0, 0, 0, 0);
+            }
+            __syncthreads();  // s_amax cleared
+            const int lane = threadIdx.x & 31;
+#pragma unroll
+            for (int i = 0; i < DEC_QB; ++i) {
+                const int idx = (int)threadIdx.x + DEC_THREADS * i;
+                if (DEC_THREADS * i >= tot) break;  // uniform: no vector of this round is in range
+                u32 a = 0;
+                const int m = idx < tot ? idx / nvec : -1;
+#pragma unroll
+                for (int j = 0; j < EPV; ++j) a = max(a, dec_x_bits<BF16>(c[i], j) & 0x7fffffffu);
+                // one shared atomic per warp when the warp's 32 vectors lie in one row
+                const int m0 = __shfl_sync(0xffffffffu, m, 0);
+                if (__all_sync(0xffffffffu, m == m0)) {
+                    a = __reduce_max_sync(0xffffffffu, a);
+                    if (lane == 0 && m0 >= 0) atomicMax(&s_amax[m0], a);
+                } else if (m >= 0) {
+                    atomicMax(&s_amax[m], a);
+                }
+            }
+            __syncthreads();
+            if (threadIdx.x < M) {
+                const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(s_amax[threadIdx.x]), 1e-5f));
+                s_sc[threadIdx.x] = s;
+                s_f[threadIdx.x] = __fdiv_rn(*pr.gamma, s);
+                if (out && pr.s != nullptr) pr.s[threadIdx.x] = s;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int i = 0; i < DEC_QB; ++i) {
+                const int idx = (int)threadIdx.x + DEC_THREADS * i;
+                if (idx >= tot) continue;
+                const int m = idx / nvec, v = idx - m * nvec;
+                const float s = s_sc[m];
+                u32 word[EPV / 4];
+#pragma unroll
+                for (int q = 0; q < EPV / 4; ++q) {
+                    u32 w = 0;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        int qi = __float2int_rn(__fmul_rn(__uint_as_float(dec_x_bits<BF16>(c[i], 4 * q + j)), s));
+                        qi = max(-128, min(127, qi));
+                        w |= ((u32)qi & 0xffu) << (8 * j);
+                    }
+                    word[q] = w;
+                }
+                const int L = BF16 ? (v >> 1) : (v >> 2);
+                const int within = BF16 ? (v & 1) * 8 : (v & 3) * 4;
+                const int x = (((L >> 3) & 1) << 1) | (m & 1);
+                uint8_t *d = s_xq + m * RS + ((((L & ~7) | ((L ^ x) & 7)) << 4) + within);
+                int8_t *gq = out && pr.xq_out != nullptr ? pr.xq_out + (size_t)m * K : nullptr;
+                if (BF16) {
+                    *reinterpret_cast<uint2 *>(d) = make_uint2(word[0], word[EPV / 4 - 1]);
+                    if (gq) *reinterpret_cast<uint2 *>(gq + (size_t)v * 8) = make_uint2(word[0], word[EPV / 4 - 1]);
+                } else {
+                    *reinterpret_cast<u32 *>(d) = word[0];
+                    if (gq) *reinterpret_cast<u32 *>(gq + (size_t)v * 4) = word[0];
+                }
+            }
+        } else {
+            // fused step 2: warp w quantizes rows w, w + 8
+            const int lane = threadIdx.x & 31;
+            for (int m = threadIdx.x >> 5; m < M; m += DEC_WARPS) {
+                const float s = dec_quant_row<BF16>(pr, m, K, RS, s_xq, P.eps, out, lane);
+                if (lane == 0) s_f[m] = __fdiv_rn(*pr.gamma, s);
+            }
         }
         const int chunks = RS >> 4, kchunks = K >> 4;
         for (int r = 0; r < M; ++r) {

@@ -163,6 +163,18 @@ def test_fused_decode_validation(L):
     assert g(P, 2, 1) in (CUDA, DEVICE)
 
 
+def test_ffn_act_quant_validation(L):
+    f = L.bl_ffn_act_quant
+    assert f(None, A, 4, 128, None, 1e-6, A, A, None) == NULL
+    assert f(A, None, 4, 128, None, 1e-6, A, A, None) == NULL
+    assert f(A, A, 4, 128, None, 1e-6, None, A, None) == NULL
+    assert f(A, A, 0, 128, None, 1e-6, A, A, None) == SHAPE
+    assert f(A, A, 4, 100, None, 1e-6, A, A, None) == SHAPE
+    assert f(A, A + 4, 4, 128, None, 1e-6, A, A, None) == ALIGN
+    assert f(A, A, 4, 128, A + 8, 1e-6, A, A, None) == ALIGN
+    assert f(A, A, 4, 128, None, 1e-6, A, A, None) in (CUDA, DEVICE)
+
+
 def test_debug_prefill_validation(L):
     f = L.bl_debug_forward_prefill
     assert f(None, A, A, A, 1, 64, 128, A, None, -1, 1000, None) == NULL

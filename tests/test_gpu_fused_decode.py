@@ -76,6 +76,9 @@ def run_fused(items, M, dtype, eps=1e-6, outputs=True, flags=0):
     (4, 17, 128, torch.float32, True, "tiny"),
     (4, 17, 128, torch.float32, False, "tiny"),
     (9, 257, 64, torch.bfloat16, True, "normal"),
+    (2, 50, 1024, torch.float32, False, "wide"),
+    (1, 40, 4096, torch.bfloat16, False, "outlier"),
+    (2, 33, 192, torch.float32, False, "tiny"),
 ])
 def test_fused_decode_matches_oracle(M, N, K, dtype, subln, kind):
     W = workloads.normal((N, K), 0.02, 500 + K)
