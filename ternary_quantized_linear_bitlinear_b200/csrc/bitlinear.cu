@@ -131,30 +131,43 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
     const long long nvec = Kmax / epv;
     bool subln = false;
     for (int i = 0; i < P.count; ++i) subln |= P.p[i].gain != nullptr;
-    if (!subln && nvec <= 16 * 32) {
-        // short rows: one warp per row
+    const long long rows = (long long)P.count * P.M;
+    const unsigned wgrid = (unsigned)((rows + AQW_WARPS - 1) / AQW_WARPS);
+    if (subln) {
+        // one warp per row, chunked, any K (rows without a gain: plain)
+        if (glu)
+            k_act_quant_subln<false, true><<<wgrid, AQW_WARPS * 32, 0, st>>>(P);
+        else if (bf16)
+            k_act_quant_subln<true, false><<<wgrid, AQW_WARPS * 32, 0, st>>>(P);
+        else
+            k_act_quant_subln<false, false><<<wgrid, AQW_WARPS * 32, 0, st>>>(P);
+        return launch_status();
+    }
+    if (nvec <= 32 * 32) {
+        // rows up to 1024 16-byte vectors: one warp per row, row in registers
         int vpl = 1;
         while (vpl * 32 < nvec) vpl *= 2;
-        const long long rows = (long long)P.count * P.M;
-        const unsigned grid = (unsigned)((rows + AQW_WARPS - 1) / AQW_WARPS);
-#define BL_AQW_CASE(B, V)                                                         \
-        if (bf16 == B && vpl == V) {                                              \
-            if (glu)                                                              \
-                k_act_quant_warp<false, V, true><<<grid, AQW_WARPS * 32, 0, st>>>(P); \
-            else                                                                  \
-                k_act_quant_warp<B, V><<<grid, AQW_WARPS * 32, 0, st>>>(P);       \
-            return launch_status();                                               \
+        const unsigned grid = wgrid;
+#define BL_AQW_CASE(B, V)                                                              \
+        if (bf16 == B && vpl == V) {                                                   \
+            if (glu)                                                                   \
+                k_act_quant_warp<false, V, true><<<grid, AQW_WARPS * 32, 0, st>>>(P);  \
+            else                                                                       \
+                k_act_quant_warp<B, V><<<grid, AQW_WARPS * 32, 0, st>>>(P);            \
+            return launch_status();                                                    \
         }
         BL_AQW_CASE(true, 1)
         BL_AQW_CASE(true, 2)
         BL_AQW_CASE(true, 4)
         BL_AQW_CASE(true, 8)
         BL_AQW_CASE(true, 16)
+        BL_AQW_CASE(true, 32)
         BL_AQW_CASE(false, 1)
         BL_AQW_CASE(false, 2)
         BL_AQW_CASE(false, 4)
         BL_AQW_CASE(false, 8)
         BL_AQW_CASE(false, 16)
+        BL_AQW_CASE(false, 32)
 #undef BL_AQW_CASE
     }
     int vec = 1;

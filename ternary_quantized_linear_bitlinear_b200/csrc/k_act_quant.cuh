@@ -4,17 +4,17 @@
 // ("BitDistill", Stage 1; "SLM750-Edge" section 2.1, eps 1e-6 from its Key
 // Architectural Features).
 //
-// One CTA per token row; the row lives in registers (VPT values per thread),
-// so X is read from HBM exactly once and x_q written once.
 //   s   = float(127 / max(max|y|, 1e-5f))
 //   x_q = clamp(round_half_even(float(y * s)), -128, 127)
 // with y = x, or y = float(float(x / r) * g) and
 //   r = sqrtf(float(double(sum x^2) / K) + eps),
-// the sum of squares exact: x^2 = m^2 * 2^(2e - 300), accumulated as a 128-bit
-// integer per thread inside a window of 30 binades below the row's largest
-// exponent (m^2 < 2^48, shift <= 60, <= 32 terms per thread, so a warp sum
-// stays below 2^118), everything else added exactly into shared-memory bins
-// by exponent.
+// the sum of squares exact (see k_act_quant_subln).
+//
+// Kernels (all read X once from HBM and write x_q once):
+//   k_act_quant_warp   one warp per row, row in registers (up to 1024
+//                      16-byte vectors), no SubLN
+//   k_act_quant        one CTA per row, longer rows, no SubLN
+//   k_act_quant_subln  one warp per row, chunked, any length, SubLN
 #pragma once
 
 #include "bl_common.cuh"
@@ -68,16 +68,14 @@ __device__ __forceinline__ float block_max_f(float v, float *s_red) {
     return __uint_as_float(r);
 }
 
-// VEC: 16-byte vectors per thread; EPV elements per vector.
+// One CTA per row (rows longer than a warp holds), no SubLN.  VEC: 16-byte
+// vectors per thread; EPV elements per vector.
 template <bool BF16, int VEC, bool GLU = false>
 __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ ActParams P) {
     static_assert(!(GLU && BF16), "GLU inputs are float32 projection outputs");
     constexpr int EPV = BF16 ? 8 : 4;
     constexpr int VPT = VEC * EPV;
     __shared__ float s_red[32];
-    __shared__ u64 s_bins[256];
-    __shared__ u64 s_lo[32], s_hi[32];
-    __shared__ float s_r;
 
     // let a programmatically dependent launch (the GEMV) start streaming its
     // weights; it waits for this grid to finish before it reads x_q
@@ -105,71 +103,6 @@ __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ A
             float f = __uint_as_float(bits);
             x[v * EPV + j] = f;
             amax = fmaxf(amax, fabsf(f));
-        }
-    }
-
-    if (pr.gain != nullptr) {
-        // ---- exact sum of squares ------------------------------------------
-        for (int i = tid; i < 256; i += T) s_bins[i] = 0ull;
-        amax = block_max_f(amax, s_red);  // also orders the bin clear
-        int emax = (int)(__float_as_uint(amax) >> 23);
-        int elo = emax - 30;
-        if (elo < 1) elo = 1;
-        u64 lo = 0ull, hi = 0ull;
-#pragma unroll
-        for (int i = 0; i < VPT; ++i) {
-            u32 u = __float_as_uint(x[i]) & 0x7fffffffu;
-            int e = (int)(u >> 23);
-            u64 mm = (u64)((u & 0x7fffffu) | 0x800000u);
-            mm *= mm;  // < 2^48
-            int d = e - elo;
-            if (d >= 0) {
-                int sh = 2 * d;  // <= 60
-                u64 plo = sh < 64 ? (mm << sh) : 0ull;
-                u64 phi = sh == 0 ? 0ull : (sh < 64 ? (mm >> (64 - sh)) : (mm << (sh - 64)));
-                u64 s = lo + plo;
-                hi += phi + (s < lo ? 1ull : 0ull);
-                lo = s;
-            } else if (u != 0u) {
-                u64 mr = e ? mm : (u64)(u & 0x7fffffu) * (u64)(u & 0x7fffffu);
-                atomicAdd(&s_bins[e], mr);
-            }
-        }
-        warp_sum_u128(lo, hi);
-        if ((tid & 31) == 0) {
-            s_lo[tid >> 5] = lo;
-            s_hi[tid >> 5] = hi;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            u64 L[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
-            for (int w = 0; w < (T >> 5); ++w) limbs_add_u128_shl(L, s_lo[w], s_hi[w], 2 * (elo - 1));
-            for (int e = 0; e < 256; ++e) {
-                u64 b = s_bins[e];
-                if (b) limbs_add_u128_shl(L, b, 0ull, e > 0 ? 2 * (e - 1) : 0);
-            }
-            double S2 = limbs_to_double_rn(L, -298);
-            float ms = __double2float_rn(__ddiv_rn(S2, (double)K));
-            s_r = __fsqrt_rn(__fadd_rn(ms, P.eps));
-        }
-        __syncthreads();
-        const float r = s_r;
-        const float4 *g4 = reinterpret_cast<const float4 *>(pr.gain);
-        amax = 0.f;
-#pragma unroll
-        for (int v = 0; v < VEC; ++v) {
-            int vi = tid + v * T;
-#pragma unroll
-            for (int q = 0; q < EPV / 4; ++q) {
-                float4 g = vi < nvec ? __ldg(g4 + vi * (EPV / 4) + q) : make_float4(0.f, 0.f, 0.f, 0.f);
-                const float gg[4] = {g.x, g.y, g.z, g.w};
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    float &xv = x[v * EPV + q * 4 + j];
-                    xv = __fmul_rn(__fdiv_rn(xv, r), gg[j]);
-                    amax = fmaxf(amax, fabsf(xv));
-                }
-            }
         }
     }
 
@@ -203,9 +136,15 @@ __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ A
     }
 }
 
-// One warp per row, no SubLN (short rows): VPL 16-byte vectors per lane, the
-// row in registers, absmax by a warp reduction -- no block barrier at all.
+// One warp per row: VPL 16-byte vectors per lane, the row in registers,
+// reductions by warp shuffles -- no block barrier at all.
 constexpr int AQW_WARPS = 8;
+
+template <bool BF16>
+__device__ __forceinline__ u32 aq_bits(const uint4 &v, int j) {
+    const u32 w = j < (BF16 ? 2 : 1) ? v.x : j < (BF16 ? 4 : 2) ? v.y : j < (BF16 ? 6 : 3) ? v.z : v.w;
+    return BF16 ? ((j & 1) ? (w & 0xffff0000u) : (w << 16)) : w;
+}
 
 template <bool BF16, int VPL, bool GLU = false>
 __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_constant__ ActParams P) {
@@ -224,15 +163,19 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_
     for (int v = 0; v < VPL; ++v) {
         const int vi = lane + v * 32;
         raw[v] = vi < nvec ? ldg_stream_v4(xr + vi) : make_uint4(0, 0, 0, 0);
-        if (GLU && vi < nvec)
-            raw[v] = glu_relu2_v4(raw[v], ldg_stream_v4(reinterpret_cast<const uint4 *>(pr.X2) + (size_t)m * nvec + vi));
-        const u32 w4[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
+    }
+    if (GLU) {
 #pragma unroll
-        for (int j = 0; j < EPV; ++j) {
-            u32 bits = BF16 ? ((j & 1) ? (w4[j >> 1] & 0xffff0000u) : (w4[j >> 1] << 16)) : w4[j];
-            amax = max(amax, bits & 0x7fffffffu);
+        for (int v = 0; v < VPL; ++v) {
+            const int vi = lane + v * 32;
+            if (vi < nvec)
+                raw[v] = glu_relu2_v4(raw[v], ldg_stream_v4(reinterpret_cast<const uint4 *>(pr.X2) + (size_t)m * nvec + vi));
         }
     }
+#pragma unroll
+    for (int v = 0; v < VPL; ++v)
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) amax = max(amax, aq_bits<BF16>(raw[v], j) & 0x7fffffffu);
     amax = warp_max_u32(amax);
     const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(amax), 1e-5f));
     if (lane == 0) pr.s[m] = s;
@@ -241,16 +184,13 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_
     for (int v = 0; v < VPL; ++v) {
         const int vi = lane + v * 32;
         if (vi >= nvec) continue;
-        const u32 w4[4] = {raw[v].x, raw[v].y, raw[v].z, raw[v].w};
         u32 out[EPV / 4];
 #pragma unroll
         for (int q = 0; q < EPV / 4; ++q) {
             u32 word = 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int e = q * 4 + j;
-                u32 bits = BF16 ? ((e & 1) ? (w4[e >> 1] & 0xffff0000u) : (w4[e >> 1] << 16)) : w4[e];
-                int qi = __float2int_rn(__fmul_rn(__uint_as_float(bits), s));
+                int qi = __float2int_rn(__fmul_rn(__uint_as_float(aq_bits<BF16>(raw[v], 4 * q + j)), s));
                 qi = max(-128, min(127, qi));
                 word |= ((u32)qi & 0xffu) << (8 * j);
             }
@@ -260,6 +200,164 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_
             *reinterpret_cast<uint2 *>(qr + (size_t)vi * 8) = make_uint2(out[0], out[EPV / 4 - 1]);
         } else {
             *reinterpret_cast<u32 *>(qr + (size_t)vi * 4) = out[0];
+        }
+    }
+}
+
+// One warp per row with SubLN (rows without a gain are quantized plainly):
+// the row is processed in chunks of 128 16-byte vectors (AQS_V per lane),
+// re-read from L1/L2 for each pass unless it fits one chunk.  Few registers,
+// so many warps per SM hide the latency of the per-element divisions.
+//   pass 1  max|x| (the window of the exact sum)
+//   pass 2  exact sum x^2: each window adds the values with exponent e in
+//           [elo, ehi] (31 binades; subnormals count as e = 1 without the
+//           hidden bit) as mant^2 << 2(e - elo) into a 128-bit lane
+//           accumulator (< 2^108 per term, <= 2^12 terms per lane, warp sum
+//           < 2^125); lane 0 adds it into 576-bit limbs in units of 2^-298;
+//           the next window, 31 binades lower, runs only while some lane
+//           still holds a smaller nonzero value (normally never)
+//   pass 3  r = sqrtf(float(double(S) / K) + eps); max|y|, y = float(float(x / r) * g)
+//   pass 4  x_q = clamp(rne(float(y * s)), -128, 127), s = float(127 / max(max|y|, 1e-5f))
+constexpr int AQS_V = 4;
+
+template <bool BF16, bool GLU>
+__global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid_constant__ ActParams P) {
+    static_assert(!(GLU && BF16), "GLU inputs are float32 projection outputs");
+    constexpr int EPV = BF16 ? 8 : 4;
+    constexpr int CH = 32 * AQS_V;  // vectors per chunk
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int gw = blockIdx.x * AQW_WARPS + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+    if (gw >= P.count * P.M) return;
+    const int pi = gw / P.M, m = gw - pi * P.M;
+    const ActProblem &pr = P.p[pi];
+    const int K = pr.K, nvec = K / EPV;
+    const int nch = (nvec + CH - 1) / CH;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(pr.X) + (size_t)m * nvec;
+    const uint4 *ur = GLU ? reinterpret_cast<const uint4 *>(pr.X2) + (size_t)m * nvec : nullptr;
+    const float4 *g4 = reinterpret_cast<const float4 *>(pr.gain);
+    uint4 c[AQS_V];
+    auto load = [&](int ch) {
+#pragma unroll
+        for (int i = 0; i < AQS_V; ++i) {
+            const int vi = ch * CH + 32 * i + lane;
+            c[i] = make_uint4(0, 0, 0, 0);
+            if (vi < nvec) {
+                c[i] = ldg_nc_v4(xr + vi);
+                if (GLU) c[i] = glu_relu2_v4(c[i], ldg_nc_v4(ur + vi));
+            }
+        }
+    };
+    // pass 1
+    u32 amax = 0;
+    for (int ch = 0; ch < nch; ++ch) {
+        load(ch);
+#pragma unroll
+        for (int i = 0; i < AQS_V; ++i)
+#pragma unroll
+            for (int j = 0; j < EPV; ++j) amax = max(amax, aq_bits<BF16>(c[i], j) & 0x7fffffffu);
+    }
+    amax = warp_max_u32(amax);
+    float r = 1.f;
+    if (g4 != nullptr) {
+        // pass 2
+        u64 L[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+        int ehi = (int)(amax >> 23);
+        if (ehi < 1) ehi = 1;
+        for (int pass = 0; pass < 10; ++pass) {
+            const int elo = ehi - 30 < 1 ? 1 : ehi - 30;
+            u64 lo = 0ull, hi = 0ull;
+            bool below = false;
+            for (int ch = 0; ch < nch; ++ch) {
+                if (nch > 1 || pass > 0) load(ch);
+#pragma unroll
+                for (int i = 0; i < AQS_V; ++i) {
+#pragma unroll
+                    for (int j = 0; j < EPV; ++j) {
+                        const u32 u = aq_bits<BF16>(c[i], j) & 0x7fffffffu;
+                        const int e = (int)(u >> 23);
+                        const int ee = e ? e : 1;
+                        if (ee <= ehi && ee >= elo && u != 0u) {
+                            u64 mm = (u64)(e ? ((u & 0x7fffffu) | 0x800000u) : u);
+                            mm *= mm;
+                            const int sh = 2 * (ee - elo);  // <= 60
+                            const u64 plo = mm << sh;
+                            const u64 phi = sh ? (mm >> (64 - sh)) : 0ull;
+                            const u64 t = lo + plo;
+                            hi += phi + (t < lo ? 1ull : 0ull);
+                            lo = t;
+                        } else if (ee < elo && u != 0u) {
+                            below = true;
+                        }
+                    }
+                }
+            }
+            warp_sum_u128(lo, hi);
+            if (lane == 0) limbs_add_u128_shl(L, lo, hi, 2 * (elo - 1));
+            if (!__any_sync(0xffffffffu, below) || elo == 1) break;
+            ehi = elo - 1;
+        }
+        if (lane == 0)
+            r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(limbs_to_double_rn(L, -298), (double)K)), P.eps));
+        r = __shfl_sync(0xffffffffu, r, 0);
+        // pass 3
+        amax = 0;
+        for (int ch = 0; ch < nch; ++ch) {
+            if (nch > 1) load(ch);
+#pragma unroll
+            for (int i = 0; i < AQS_V; ++i) {
+                const int vi = ch * CH + 32 * i + lane;
+                if (vi >= nvec) continue;
+#pragma unroll
+                for (int q = 0; q < EPV / 4; ++q) {
+                    const float4 g = __ldg(g4 + vi * (EPV / 4) + q);
+                    const float gg[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const float y = __fmul_rn(__fdiv_rn(__uint_as_float(aq_bits<BF16>(c[i], 4 * q + j)), r), gg[j]);
+                        amax = max(amax, __float_as_uint(y) & 0x7fffffffu);
+                    }
+                }
+            }
+        }
+        amax = warp_max_u32(amax);
+    }
+    const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(amax), 1e-5f));
+    if (lane == 0) pr.s[m] = s;
+    // pass 4
+    int8_t *qr = pr.xq + (size_t)m * K;
+    for (int ch = 0; ch < nch; ++ch) {
+        if (nch > 1) load(ch);
+#pragma unroll
+        for (int i = 0; i < AQS_V; ++i) {
+            const int vi = ch * CH + 32 * i + lane;
+            if (vi >= nvec) continue;
+            u32 out[EPV / 4];
+#pragma unroll
+            for (int q = 0; q < EPV / 4; ++q) {
+                float gg[4] = {1.f, 1.f, 1.f, 1.f};
+                if (g4 != nullptr) {
+                    const float4 g = __ldg(g4 + vi * (EPV / 4) + q);
+                    gg[0] = g.x;
+                    gg[1] = g.y;
+                    gg[2] = g.z;
+                    gg[3] = g.w;
+                }
+                u32 word = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    float y = __uint_as_float(aq_bits<BF16>(c[i], 4 * q + j));
+                    if (g4 != nullptr) y = __fmul_rn(__fdiv_rn(y, r), gg[j]);
+                    int qi = __float2int_rn(__fmul_rn(y, s));
+                    qi = max(-128, min(127, qi));
+                    word |= ((u32)qi & 0xffu) << (8 * j);
+                }
+                out[q] = word;
+            }
+            if (BF16) {
+                *reinterpret_cast<uint2 *>(qr + (size_t)vi * 8) = make_uint2(out[0], out[EPV / 4 - 1]);
+            } else {
+                *reinterpret_cast<u32 *>(qr + (size_t)vi * 4) = out[0];
+            }
         }
     }
 }
