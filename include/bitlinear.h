@@ -208,10 +208,15 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt,
                     void *workspace, size_t workspace_bytes, float *Y, bl_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
-/* Grouped decode: up to BL_MAX_GROUP independent steps-3+4 problems that    */
-/* share M, in ONE kernel launch (e.g. every projection of a decode step).   */
-/* Same arithmetic as bl_forward; every problem must be decode-eligible      */
-/* (M <= 16 and the staging fits, see bl_forward), else BL_ERR_SHAPE.        */
+/* Grouped steps 3+4, ONE kernel launch, same arithmetic as bl_forward:      */
+/*  - decode: when every problem is decode-eligible (M <= 16 and the staging */
+/*    fits, see bl_forward), up to BL_MAX_GROUP independent problems that    */
+/*    share M (e.g. every projection of a decode step);                      */
+/*  - prefill: otherwise, up to BL_MAX_PREFILL_GROUP problems that share the */
+/*    same x_q, s and K (e.g. the q, k, v or the gate, up projections of one */
+/*    layer): their output tiles run in one persistent tcgen05 launch.       */
+/*    Problems with different x_q / s / K, or more of them, give             */
+/*    BL_ERR_SHAPE.                                                          */
 /* `problems` is a HOST array, read during the call only.                    */
 /* flags: 0, or BL_FWD_WEIGHTS_READY -- the caller promises that every       */
 /* problem's packed weights and gamma were complete before the kernel        */
@@ -220,6 +225,7 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt,
 /* finishes (it still waits for it before reading x_q and s).                */
 /* ------------------------------------------------------------------------ */
 #define BL_MAX_GROUP 128
+#define BL_MAX_PREFILL_GROUP 4
 #define BL_FWD_WEIGHTS_READY 1u
 
 typedef struct {

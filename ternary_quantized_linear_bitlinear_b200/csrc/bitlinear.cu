@@ -267,6 +267,28 @@ bl_status forward_impl(const DeviceInfo &d, const uint8_t *packed, const float *
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Prefill-sized groups: problems sharing one activation (x_q, s, K) in one
+// tcgen05 launch.
+bl_status forward_grouped_prefill(const bl_problem *problems, int count, int64_t M, cudaStream_t st) {
+    if (count > PF_MAX_PROB || M < 1 || M > 0x7fffffffLL) return BL_ERR_SHAPE;
+    const bl_problem &q0 = problems[0];
+    PrefillJob jobs[PF_MAX_PROB];
+    for (int i = 0; i < count; ++i) {
+        const bl_problem &q = problems[i];
+        if (!q.packed || !q.gamma || !q.x_q || !q.s || !q.Y) return BL_ERR_NULL;
+        if (q.x_q != q0.x_q || q.s != q0.s || q.K != q0.K) return BL_ERR_SHAPE;
+        if (q.N < 1 || q.N > 0x7fffffffLL || check_k(q.K) != BL_OK) return BL_ERR_SHAPE;
+        if (!aligned16(q.packed) || !aligned16(q.gamma) || !aligned16(q.x_q) || !aligned16(q.s) || !aligned16(q.Y) ||
+            (q.acc_out && !aligned16(q.acc_out)))
+            return BL_ERR_ALIGN;
+        jobs[i] = PrefillJob{q.packed, q.gamma, q.Y, q.acc_out, q.N};
+    }
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return prefill_launch_group(d->sms, jobs, count, q0.x_q, q0.s, M, q0.K, st);
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -384,7 +406,10 @@ bl_status bl_forward(const uint8_t *packed, const float *gamma, const int8_t *x_
 bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, unsigned flags,
                              bl_stream_t stream) {
     if (!problems) return BL_ERR_NULL;
-    if (count < 1 || count > BL_MAX_GROUP || M < 1 || M > 16) return BL_ERR_SHAPE;
+    if (count < 1 || count > BL_MAX_GROUP || M < 1) return BL_ERR_SHAPE;
+    bool decode = M <= 16;
+    for (int i = 0; i < count && decode; ++i) decode = check_k(problems[i].K) == BL_OK && decode_eligible(M, problems[i].K);
+    if (!decode) return forward_grouped_prefill(problems, count, M, (cudaStream_t)stream);
     DecodeParams P;
     P.count = count;
     P.M = (int)M;

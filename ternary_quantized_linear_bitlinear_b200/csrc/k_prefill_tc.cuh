@@ -73,16 +73,36 @@ constexpr int PF_SMEM_BYTES = PF_SMEM_USED + 1024;                     // + alig
 static_assert(PF_SMEM_BYTES > 116 * 1024, "keeps one CTA per SM, so the TMEM allocation never waits");
 static_assert(PF_SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
-struct PrefillParams {
+// Up to PF_MAX_PROB weight matrices that share one activation (e.g. the q,
+// k, v or the gate, up projections of a layer) in one launch: their output
+// tiles are numbered consecutively along N (problem p owns global n-tiles
+// nt_begin .. nt_begin + ceil(N / PF_BN) - 1).
+constexpr int PF_MAX_PROB = BL_MAX_PREFILL_GROUP;
+
+struct PrefillProb {
     const float *gamma;
-    const float *s;
     float *Y;
     int32_t *acc;
-    int M, N, K;
-    int n_tiles, m_tiles, k_stages;
+    int N;
+    int nt_begin;
+};
+
+// TMA descriptors: the shared x_q and, per problem, packed weights and Y.
+struct PrefillMaps {
+    CUtensorMap x;
+    CUtensorMap w[PF_MAX_PROB];
+    CUtensorMap y[PF_MAX_PROB];
+};
+
+struct PrefillParams {
+    PrefillProb prob[PF_MAX_PROB];
+    int nprob;
+    const float *s;
+    int M, K;
+    int n_tiles, m_tiles, k_stages;  // n_tiles: over all problems
     unsigned long long timeout_ns;
     long long dbg_skip_iter;  // >= 0: the producer never issues this k-iteration (bounded-wait test)
-    int y_tma;                // 1: Y written by TMA stores through tm_y (N % 4 == 0 and no acc output)
+    int y_tma;                // 1: Y written by TMA stores (every N % 4 == 0 and no acc output)
 };
 
 // ---------------------------------------------------------------------------
@@ -162,9 +182,14 @@ __host__ __device__ constexpr u32 pf_idesc() {
 
 // ---------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_constant__ CUtensorMap tm_x,
-                                                               const __grid_constant__ CUtensorMap tm_w,
-                                                               const __grid_constant__ CUtensorMap tm_y,
+// problem that owns global n-tile nt
+__device__ __forceinline__ int pf_prob_of(const PrefillParams &p, int nt) {
+    int pi = 0;
+    while (pi + 1 < p.nprob && nt >= p.prob[pi + 1].nt_begin) ++pi;
+    return pi;
+}
+
+__global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_constant__ PrefillMaps maps,
                                                                const __grid_constant__ PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -195,9 +220,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         }
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_x) : "memory");
-        asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_w) : "memory");
-        if (p.y_tma) asm volatile("prefetch.tensormap [%0];" ::"l"(&tm_y) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.x) : "memory");
+        for (int i = 0; i < p.nprob; ++i) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.w[i]) : "memory");
+            if (p.y_tma) asm volatile("prefetch.tensormap [%0];" ::"l"(&maps.y[i]) : "memory");
+        }
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
@@ -220,6 +247,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
             bool failed = false;
             for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x) {
                 const int nt = tile % p.n_tiles, mt = tile / p.n_tiles;
+                const int pi = pf_prob_of(p, nt);
+                const CUtensorMap *tmw = &maps.w[pi];
+                const int ntl = nt - p.prob[pi].nt_begin;
                 for (int ks = 0; ks < KS; ++ks, ++it) {
                     const int s = (int)(it % PF_STAGES);
                     const u32 ph = (u32)((it / PF_STAGES) & 1);
@@ -229,8 +259,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                     }
                     if (it == p.dbg_skip_iter) continue;  // test hook: this stage never arrives
                     mbar_arrive_expect_tx(BAR_FULL(s), PF_A_BYTES + PF_P_BYTES);
-                    tma_load_2d(sbase + PF_OFF_A + s * PF_A_BYTES, &tm_x, ks * PF_BK, mt * PF_BM, BAR_FULL(s));
-                    tma_load_2d(sbase + PF_OFF_P + s * PF_P_BYTES, &tm_w, ks * (PF_BK / 4), nt * PF_BN, BAR_FULL(s));
+                    tma_load_2d(sbase + PF_OFF_A + s * PF_A_BYTES, &maps.x, ks * PF_BK, mt * PF_BM, BAR_FULL(s));
+                    tma_load_2d(sbase + PF_OFF_P + s * PF_P_BYTES, tmw, ks * (PF_BK / 4), ntl * PF_BN, BAR_FULL(s));
                 }
             }
             if (failed) {
@@ -341,14 +371,18 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         const int q = warp & 3;                           // TMEM lane quarter = token block
         const int ew = warp - PF_EPI_WARP0;               // 0..7
         const int half = ew >> 2;                         // weight-row half of the tile
-        const float gamma = *p.gamma;
-        const bool vec_ok = (p.N & 3) == 0;               // rows of Y 16-byte aligned
+
         uint8_t *ystage = sm + PF_OFF_Y + ew * PF_Y_BYTES;
         const u32 ystage_s = smem_u32(ystage);
         int tc = 0;
         bool failed = false;
         for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x, ++tc) {
             const int nt = tile % p.n_tiles, mt = tile / p.n_tiles;
+            const PrefillProb &pp = p.prob[pf_prob_of(p, nt)];
+            const int pN = pp.N;
+            const int ntl = nt - pp.nt_begin;
+            const float gamma = *pp.gamma;
+            const bool vec_ok = (pN & 3) == 0;            // rows of Y 16-byte aligned
             const int b = tc & 1;
             const u32 cph = (u32)((tc >> 1) & 1);
             const int m = mt * PF_BM + q * 32 + lane;     // this thread's token
@@ -361,10 +395,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                 break;
             }
             tc_fence_after();
-            const int n0 = nt * PF_BN + half * (PF_BN / 2);
-            const bool full = vec_ok && n0 + PF_BN / 2 <= p.N;
-            float *yrow = p.Y + (size_t)m * p.N + n0;
-            int32_t *arow = p.acc ? p.acc + (size_t)m * p.N + n0 : nullptr;
+            const int n0 = ntl * PF_BN + half * (PF_BN / 2);  // within this problem
+            const bool full = vec_ok && n0 + PF_BN / 2 <= pN;
+            float *yrow = pp.Y + (size_t)m * pN + n0;
+            int32_t *arow = pp.acc ? pp.acc + (size_t)m * pN + n0 : nullptr;
 #pragma unroll 1
             for (int c0 = 0; c0 < PF_BN / 2; c0 += 32) {
                 u32 r[32];
@@ -390,7 +424,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
-                    if (lane == 0) tma_store_2d(&tm_y, n0 + c0, mt * PF_BM + q * 32, ystage_s);
+                    if (lane == 0) tma_store_2d(&maps.y[pf_prob_of(p, nt)], n0 + c0, mt * PF_BM + q * 32, ystage_s);
                 } else if (mvalid) {
                     if (full) {
 #pragma unroll
@@ -410,7 +444,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                     } else {
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
-                            if (n0 + c0 + j < p.N) {
+                            if (n0 + c0 + j < pN) {
                                 yrow[c0 + j] = __fmul_rn(__int2float_rn((int)r[j]), f);
                                 if (arow) arow[c0 + j] = (int)r[j] >> 6;
                             }
@@ -475,54 +509,69 @@ inline cudaError_t prefill_setup() {
 
 constexpr unsigned long long PF_DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
 
-inline bl_status prefill_launch(int sms, const uint8_t *packed, const float *gamma, const int8_t *x_q, const float *s,
-                                int64_t M, int64_t N, int64_t K, float *Y, int32_t *acc_out, cudaStream_t st,
-                                unsigned long long timeout_ns = PF_DEFAULT_TIMEOUT_NS, long long dbg_skip_iter = -1) {
+// One weight matrix of a grouped prefill launch (all share x_q, s, M, K).
+struct PrefillJob {
+    const uint8_t *packed;
+    const float *gamma;
+    float *Y;
+    int32_t *acc_out;
+    int64_t N;
+};
+
+inline bl_status prefill_launch_group(int sms, const PrefillJob *jobs, int count, const int8_t *x_q, const float *s,
+                                      int64_t M, int64_t K, cudaStream_t st,
+                                      unsigned long long timeout_ns = PF_DEFAULT_TIMEOUT_NS,
+                                      long long dbg_skip_iter = -1) {
     EncodeTiledFn enc = encode_tiled_fn();
     if (enc == nullptr) return BL_ERR_CUDA;
-    const int64_t n_tiles = (N + PF_BN - 1) / PF_BN, m_tiles = (M + PF_BM - 1) / PF_BM;
-    if (n_tiles * m_tiles > 0x7fffffffLL) return BL_ERR_SHAPE;
-    CUtensorMap tx, tw;
+    if (count < 1 || count > PF_MAX_PROB) return BL_ERR_SHAPE;
+    PrefillMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    PrefillParams p;
+    memset(&p, 0, sizeof(p));
     const cuuint32_t es[2] = {1, 1};
     {
         const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
         const cuuint64_t gstride[1] = {(cuuint64_t)K};
         const cuuint32_t box[2] = {(cuuint32_t)PF_BK, (cuuint32_t)PF_BM};
-        if (enc(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(x_q), gdim, gstride, box, es,
+        if (enc(&maps.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(x_q), gdim, gstride, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return BL_ERR_CUDA;
     }
-    {
-        const cuuint64_t gdim[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
-        const cuuint64_t gstride[1] = {(cuuint64_t)(K / 4)};
-        const cuuint32_t box[2] = {(cuuint32_t)(PF_BK / 4), (cuuint32_t)PF_BN};
-        if (enc(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride, box, es,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return BL_ERR_CUDA;
+    // Y through TMA stores when every Y row is a 16-byte multiple and no acc output is requested
+    int y_tma = 1;
+    for (int i = 0; i < count; ++i) y_tma &= (jobs[i].N % 4 == 0 && jobs[i].acc_out == nullptr) ? 1 : 0;
+    int64_t n_tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        const PrefillJob &j = jobs[i];
+        {
+            const cuuint64_t gdim[2] = {(cuuint64_t)(K / 4), (cuuint64_t)j.N};
+            const cuuint64_t gstride[1] = {(cuuint64_t)(K / 4)};
+            const cuuint32_t box[2] = {(cuuint32_t)(PF_BK / 4), (cuuint32_t)PF_BN};
+            if (enc(&maps.w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(j.packed), gdim, gstride, box,
+                    es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return BL_ERR_CUDA;
+        }
+        if (y_tma) {
+            const cuuint64_t gdim[2] = {(cuuint64_t)j.N, (cuuint64_t)M};
+            const cuuint64_t gstride[1] = {(cuuint64_t)j.N * 4};
+            const cuuint32_t box[2] = {32, 32};
+            if (enc(&maps.y[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, j.Y, gdim, gstride, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return BL_ERR_CUDA;
+        }
+        p.prob[i] = PrefillProb{j.gamma, j.Y, j.acc_out, (int)j.N, (int)n_tiles};
+        n_tiles += (j.N + PF_BN - 1) / PF_BN;
     }
-    // Y through TMA stores when its rows are 16-byte multiples and no acc output is requested
-    CUtensorMap ty;
-    memset(&ty, 0, sizeof(ty));
-    const int y_tma = (N % 4 == 0 && acc_out == nullptr) ? 1 : 0;
-    if (y_tma) {
-        const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
-        const cuuint64_t gstride[1] = {(cuuint64_t)N * 4};
-        const cuuint32_t box[2] = {32, 32};
-        if (enc(&ty, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, Y, gdim, gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-            CUDA_SUCCESS)
-            return BL_ERR_CUDA;
-    }
-    PrefillParams p;
+    const int64_t m_tiles = (M + PF_BM - 1) / PF_BM;
+    if (n_tiles * m_tiles > 0x7fffffffLL) return BL_ERR_SHAPE;
+    p.nprob = count;
     p.y_tma = y_tma;
-    p.gamma = gamma;
     p.s = s;
-    p.Y = Y;
-    p.acc = acc_out;
     p.M = (int)M;
-    p.N = (int)N;
     p.K = (int)K;
     p.n_tiles = (int)n_tiles;
     p.m_tiles = (int)m_tiles;
@@ -531,8 +580,15 @@ inline bl_status prefill_launch(int sms, const uint8_t *packed, const float *gam
     p.dbg_skip_iter = dbg_skip_iter;
     const int64_t tiles = n_tiles * m_tiles;
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    k_prefill_tc<<<grid, PF_THREADS, PF_SMEM_BYTES, st>>>(tx, tw, ty, p);
+    k_prefill_tc<<<grid, PF_THREADS, PF_SMEM_BYTES, st>>>(maps, p);
     return cudaGetLastError() == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+inline bl_status prefill_launch(int sms, const uint8_t *packed, const float *gamma, const int8_t *x_q, const float *s,
+                                int64_t M, int64_t N, int64_t K, float *Y, int32_t *acc_out, cudaStream_t st,
+                                unsigned long long timeout_ns = PF_DEFAULT_TIMEOUT_NS, long long dbg_skip_iter = -1) {
+    const PrefillJob job{packed, gamma, Y, acc_out, N};
+    return prefill_launch_group(sms, &job, 1, x_q, s, M, K, st, timeout_ns, dbg_skip_iter);
 }
 
 }  // namespace bl

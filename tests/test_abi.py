@@ -123,7 +123,6 @@ def test_grouped_validation(L):
     assert g(None, 1, 1) == NULL
     assert g(P, 0, 1) == SHAPE
     assert g(P, api.BL_MAX_GROUP + 1, 1) == SHAPE
-    assert g(P, 2, 17) == SHAPE  # grouped decode is for M <= 16
     P[1].K = 100
     assert g(P, 2, 1) == SHAPE
     P[1].K = 128
@@ -131,6 +130,17 @@ def test_grouped_validation(L):
     assert g(P, 2, 1) == NULL
     P[1].Y = A
     assert g(P, 2, 1) in (CUDA, DEVICE)
+    # prefill-sized groups share x_q, s and K, at most BL_MAX_PREFILL_GROUP of them
+    R = (api.Problem * 5)()
+    for i in range(5):
+        R[i] = api.Problem(A, A, A, A, A, None, 64, 128)
+    assert g(R, 5, 100) == SHAPE
+    assert g(R, 4, 100) in (CUDA, DEVICE)
+    R[1].x_q = A + 16
+    assert g(R, 2, 100) == SHAPE
+    R[1].x_q = A
+    R[1].K = 256
+    assert g(R, 2, 100) == SHAPE
     Q = (api.ActProblem * 1)()
     Q[0] = api.ActProblem(A, None, A, A, 128)
     assert L.bl_quant_act_grouped(Q, 1, 5, 1, 1e-6, None) == DTYPE

@@ -13,7 +13,8 @@ import torch
 
 import oracle
 from ternary_quantized_linear_bitlinear_b200 import api, workloads
-from _parity import check_act, check_forward_full, check_forward_sampled, check_weights, gpu_quant_weights, np32
+from _parity import (check_act, check_forward_full, check_forward_sampled, check_weights, check_y, gpu_quant_weights,
+                     np32)
 
 pytestmark = pytest.mark.gpu
 
@@ -178,6 +179,35 @@ def test_grouped_decode_125m(M):
         wq_ref, g_ref = check_weights(W, packed, gamma)
         xq_ref, s_ref = check_act(X, x_q, s)
         check_forward_full(xq_ref, s_ref, wq_ref, g_ref, Y, acc)
+
+
+@pytest.mark.parametrize("M,K,Ns,with_acc", [
+    (300, 768, (768, 256, 256), False),       # q, k, v of one layer sharing x_q; ragged M
+    (200, 1536, (4096, 4096), False),         # gate, up
+    (129, 192, (37, 300, 256, 64), True),     # ragged N, int32 outputs (plain stores)
+    (40, 64, (1,), False),                    # a one-problem group, N = 1
+])
+def test_grouped_prefill_shared_activation(M, K, Ns, with_acc):
+    """One tcgen05 launch over several weight matrices that share x_q."""
+    X = workloads.with_outlier_channels(workloads.normal((M, K), 1.0, 700 + M, torch.bfloat16), 2, 20.0, 5)
+    x_q, s = api.bl_quant_act(X.cuda())
+    probs, refs = [], []
+    for i, N in enumerate(Ns):
+        W = workloads.normal((N, K), 0.02, 710 + i)
+        packed, gamma = gpu_quant_weights(W)
+        Y = torch.empty(M, N, dtype=torch.float32, device="cuda")
+        acc = torch.empty(M, N, dtype=torch.int32, device="cuda") if with_acc else None
+        probs.append((packed, gamma, x_q, s, Y, acc, N, K))
+        refs.append(W)
+    api.bl_forward_grouped(api.make_problems(probs), len(probs), M)
+    api.bl_check_device_error()
+    xq_ref, s_ref = check_act(X, x_q, s)
+    for (packed, gamma, _, _, Y, acc, N, K_), W in zip(probs, refs):
+        wq_ref, g_ref = check_weights(W, packed, gamma)
+        if acc is None:
+            check_y(Y.cpu().numpy(), oracle.contract(xq_ref, wq_ref), g_ref, s_ref[:, None])
+        else:
+            check_forward_full(xq_ref, s_ref, wq_ref, g_ref, Y, acc)
 
 
 def test_grouped_act_quant_matches_single():
