@@ -197,7 +197,9 @@ bl_status bl_forward(const uint8_t *packed, const float *gamma, const int8_t *x_
                      int32_t *acc_out, bl_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
-/* All four steps in one call: bl_quant_weights, bl_quant_act, bl_forward.   */
+/* All four steps in one call: bl_quant_weights, bl_quant_act, bl_forward    */
+/* (for decode-eligible M, steps 2-4 run as one fused launch, with the same  */
+/* results).                                                                 */
 /* workspace >= bl_linear_workspace_bytes(M, N, K) holds packed W, gamma,    */
 /* x_q and s between the steps.                                              */
 /* ------------------------------------------------------------------------ */

@@ -493,6 +493,16 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt, in
     cudaStream_t st = (cudaStream_t)stream;
     rc = quant_weights_impl(*d, W, wdt, N, K, packed, gamma, wq_ws, st);
     if (rc) return rc;
+    if (decode_eligible(M, K)) {
+        // decode-sized: activation quant fused into the GEMV launch (x_q and s
+        // still land in the workspace)
+        DecodeParams P;
+        P.count = 1;
+        P.M = (int)M;
+        P.eps = subln_eps;
+        P.p[0] = DecodeProblem{packed, gamma, X, s, Y, nullptr, subln_gain, x_q, (int)N, (int)K, 0, 0};
+        return decode_launch(P, false, st, xdt == BL_BF16 ? DEC_SRC_BF16 : DEC_SRC_F32);
+    }
     ActParams P;
     P.count = 1;
     P.M = (int)M;
