@@ -124,7 +124,24 @@ bl_status quant_weights_impl(const DeviceInfo &d, const void *W, bl_dtype wdt, i
 // ---------------------------------------------------------------------------
 // Step 2
 
-bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStream_t st) {
+// Kernel launch, optionally as a programmatic dependent launch (it may
+// start while the kernel before it runs; the act-quant kernels end with
+// griddepcontrol.wait, so their completion still implies that kernel's).
+template <typename Kern>
+bl_status launch_act(Kern kernel, unsigned grid, unsigned block, cudaStream_t st, bool pdl, const ActParams &P) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, P) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStream_t st, bool pdl = false) {
     const bool bf16 = xdt == BL_BF16;
     const bool glu = P.p[0].X2 != nullptr;  // all problems of a call alike (f32 only)
     const int epv = bf16 ? 8 : 4;
@@ -135,26 +152,19 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
     const unsigned wgrid = (unsigned)((rows + AQW_WARPS - 1) / AQW_WARPS);
     if (subln) {
         // one warp per row, chunked, any K (rows without a gain: plain)
-        if (glu)
-            k_act_quant_subln<false, true><<<wgrid, AQW_WARPS * 32, 0, st>>>(P);
-        else if (bf16)
-            k_act_quant_subln<true, false><<<wgrid, AQW_WARPS * 32, 0, st>>>(P);
-        else
-            k_act_quant_subln<false, false><<<wgrid, AQW_WARPS * 32, 0, st>>>(P);
-        return launch_status();
+        if (glu) return launch_act(k_act_quant_subln<false, true>, wgrid, AQW_WARPS * 32, st, pdl, P);
+        if (bf16) return launch_act(k_act_quant_subln<true, false>, wgrid, AQW_WARPS * 32, st, pdl, P);
+        return launch_act(k_act_quant_subln<false, false>, wgrid, AQW_WARPS * 32, st, pdl, P);
     }
     if (nvec <= 32 * 32) {
         // rows up to 1024 16-byte vectors: one warp per row, row in registers
         int vpl = 1;
         while (vpl * 32 < nvec) vpl *= 2;
         const unsigned grid = wgrid;
-#define BL_AQW_CASE(B, V)                                                              \
-        if (bf16 == B && vpl == V) {                                                   \
-            if (glu)                                                                   \
-                k_act_quant_warp<false, V, true><<<grid, AQW_WARPS * 32, 0, st>>>(P);  \
-            else                                                                       \
-                k_act_quant_warp<B, V><<<grid, AQW_WARPS * 32, 0, st>>>(P);            \
-            return launch_status();                                                    \
+#define BL_AQW_CASE(B, V)                                                                       \
+        if (bf16 == B && vpl == V) {                                                            \
+            if (glu) return launch_act(k_act_quant_warp<false, V, true>, grid, AQW_WARPS * 32, st, pdl, P); \
+            return launch_act(k_act_quant_warp<B, V>, grid, AQW_WARPS * 32, st, pdl, P);       \
         }
         BL_AQW_CASE(true, 1)
         BL_AQW_CASE(true, 2)
@@ -174,13 +184,10 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
     while ((nvec + vec - 1) / vec > 1024) vec *= 2;
     int T = (int)(((nvec + vec - 1) / vec + 31) / 32 * 32);
     const unsigned grid = (unsigned)(P.count * P.M);
-#define BL_AQ_CASE(B, V)                                                        \
-    if (bf16 == B && vec == V) {                                                \
-        if (glu)                                                                \
-            k_act_quant<false, V, true><<<grid, T, 0, st>>>(P);                 \
-        else                                                                    \
-            k_act_quant<B, V><<<grid, T, 0, st>>>(P);                           \
-        return launch_status();                                                 \
+#define BL_AQ_CASE(B, V)                                                            \
+    if (bf16 == B && vec == V) {                                                    \
+        if (glu) return launch_act(k_act_quant<false, V, true>, grid, T, st, pdl, P); \
+        return launch_act(k_act_quant<B, V>, grid, T, st, pdl, P);                  \
     }
     // at most 32 values per thread (bf16: 4 vectors, f32: 8 vectors)
     BL_AQ_CASE(true, 1)
@@ -508,7 +515,9 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt, in
     P.M = (int)M;
     P.eps = subln_eps;
     P.p[0] = ActProblem{X, subln_gain, x_q, s, (int)K, 0};
-    rc = quant_act_impl(P, xdt, K, st);
+    // the act quant depends only on X: it may run while the weight pack
+    // finishes (programmatic dependent launch); the GEMM waits for both
+    rc = quant_act_impl(P, xdt, K, st, true);
     if (rc) return rc;
     return forward_impl(*d, packed, gamma, x_q, s, M, N, K, Y, nullptr, st);
 }

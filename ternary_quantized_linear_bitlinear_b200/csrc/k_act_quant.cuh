@@ -134,6 +134,9 @@ __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ A
             *reinterpret_cast<u32 *>(qr + (size_t)vi * 4) = out[0];
         }
     }
+    // as a programmatic dependent launch this grid completes only after the
+    // grid before it (no-op otherwise)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // One warp per row: VPL 16-byte vectors per lane, the row in registers,
@@ -202,6 +205,9 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_
             *reinterpret_cast<u32 *>(qr + (size_t)vi * 4) = out[0];
         }
     }
+    // as a programmatic dependent launch this grid completes only after the
+    // grid before it (no-op otherwise)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // One warp per row with SubLN (rows without a gain are quantized plainly):
@@ -360,6 +366,9 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid
             }
         }
     }
+    // as a programmatic dependent launch this grid completes only after the
+    // grid before it (no-op otherwise)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 }  // namespace bl

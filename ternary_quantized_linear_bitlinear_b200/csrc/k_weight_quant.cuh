@@ -124,9 +124,12 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const uint4 *__r
     const long long stride = (long long)gridDim.x * WQ_THREADS;
     const long long first = (long long)blockIdx.x * WQ_THREADS + tid;
 
-    // Window from a sample: the block's first vector per thread.
+    // Window from a sample: the block's first vector per thread.  The second
+    // vector is requested before the block reduction, so its latency overlaps.
     u32 emax = 0;
     uint4 v0 = make_uint4(0, 0, 0, 0);
+    const bool has1 = first + stride < nvec;
+    const uint4 v1 = has1 ? ldg_stream_v4(W + first + stride) : make_uint4(0, 0, 0, 0);
     if (first < nvec) {
         v0 = ldg_stream_v4(W + first);
 #pragma unroll
@@ -160,7 +163,8 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const uint4 *__r
         }
     };
     if (first < nvec) add_vec(v0);
-    long long i = first + stride;
+    if (has1) add_vec(v1);
+    long long i = first + 2 * stride;
     // two vectors in flight per iteration
     for (; i + stride < nvec; i += 2 * stride) {
         uint4 a = ldg_stream_v4(W + i);
@@ -228,6 +232,9 @@ __global__ void __launch_bounds__(256) k_ternary_pack(const uint4 *__restrict__ 
                                                         const u32 *__restrict__ ws_thresh,
                                                         u32 *__restrict__ packed) {
     constexpr int VPW = BF16 ? 2 : 4;  // 16-byte vectors per 16 weights
+    // a programmatically dependent launch after this one (bl_linear's act
+    // quant, which does not read the packed weights) may start now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const long long stride = (long long)gridDim.x * blockDim.x;
     long long wi = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     // first words of W are requested before waiting for the reduction grid

@@ -242,6 +242,28 @@ def test_linear_subln_qat4b_oproj_small():
     assert np.all(err <= 1e-6 * np.abs(ref["Y"]))
 
 
+def test_linear_back_to_back_calls_share_a_workspace():
+    """Prefill-sized bl_linear calls in a row on one stream and one workspace:
+    inside a call the act quant overlaps the weight pack (programmatic
+    dependent launch); each call must still see only its own inputs."""
+    cases = [(300, 130, 768, None), (200, 257, 1536, 21), (300, 64, 768, 22)]
+    ws = torch.empty(max(api.linear_workspace_bytes(M, N, K) for M, N, K, _ in cases), dtype=torch.uint8,
+                     device="cuda")
+    outs, refs = [], []
+    for i, (M, N, K, gseed) in enumerate(cases):
+        W = workloads.normal((N, K), 0.02, 40 + i, torch.bfloat16)
+        X = workloads.with_outlier_channels(workloads.normal((M, K), 1.0, 50 + i, torch.bfloat16), 2, 20.0, 60 + i)
+        gain = None if gseed is None else workloads.uniform((K,), 0.9, 1.1, gseed)
+        outs.append(api.bl_linear(W.cuda(), X.cuda(), None if gain is None else gain.cuda(), workloads.SUBLN_EPS,
+                                  workspace=ws))
+        refs.append((W, X, gain))
+    torch.cuda.synchronize()
+    for Y, (W, X, gain) in zip(outs, refs):
+        ref = oracle.linear(np32(W), np32(X), None if gain is None else np32(gain), workloads.SUBLN_EPS)
+        err = np.abs(Y.cpu().numpy().astype(np.float64) - ref["Y"])
+        assert np.all(err <= 1e-6 * np.abs(ref["Y"]))
+
+
 # -- tcgen05 prefill engine at small M, and its bounded waits ----------------
 
 @pytest.mark.parametrize("M,N,K", [
