@@ -259,7 +259,8 @@ bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st, int src = DE
 }
 
 bl_status forward_impl(const DeviceInfo &d, const uint8_t *packed, const float *gamma, const int8_t *x_q,
-                       const float *s, int64_t M, int64_t N, int64_t K, float *Y, int32_t *acc_out, cudaStream_t st) {
+                       const float *s, int64_t M, int64_t N, int64_t K, float *Y, int32_t *acc_out, cudaStream_t st,
+                       bool pdl = false) {
     if (decode_eligible(M, K)) {
         DecodeParams P;
         P.count = 1;
@@ -269,7 +270,7 @@ bl_status forward_impl(const DeviceInfo &d, const uint8_t *packed, const float *
                                (int)N, (int)K, 0, 0};
         return decode_launch(P, false, st);
     }
-    return prefill_launch(d.sms, packed, gamma, x_q, s, M, N, K, Y, acc_out, st);
+    return prefill_launch(d.sms, packed, gamma, x_q, s, M, N, K, Y, acc_out, st, PF_DEFAULT_TIMEOUT_NS, -1, pdl);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
@@ -519,7 +520,7 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt, in
     // finishes (programmatic dependent launch); the GEMM waits for both
     rc = quant_act_impl(P, xdt, K, st, true);
     if (rc) return rc;
-    return forward_impl(*d, packed, gamma, x_q, s, M, N, K, Y, nullptr, st);
+    return forward_impl(*d, packed, gamma, x_q, s, M, N, K, Y, nullptr, st, true);
 }
 
 }  // extern "C"

@@ -243,6 +243,9 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            // x_q and the packed weights may come from the kernel before this
+            // one (programmatic dependent launch; a no-op otherwise)
+            asm volatile("griddepcontrol.wait;" ::: "memory");
             long long it = 0;
             bool failed = false;
             for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x) {
@@ -368,6 +371,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         }
     } else {
         // ------------------------------------------------------------- epilogue
+        asm volatile("griddepcontrol.wait;" ::: "memory");  // s and gamma, as above
         const int q = warp & 3;                           // TMEM lane quarter = token block
         const int ew = warp - PF_EPI_WARP0;               // 0..7
         const int half = ew >> 2;                         // weight-row half of the tile
@@ -518,10 +522,13 @@ struct PrefillJob {
     int64_t N;
 };
 
+// pdl: launch as a programmatic dependent of the kernel before it (its
+// set-up -- barriers, TMEM, descriptor prefetch -- overlaps that kernel's
+// tail; the producer and the epilogue wait for it before touching inputs).
 inline bl_status prefill_launch_group(int sms, const PrefillJob *jobs, int count, const int8_t *x_q, const float *s,
                                       int64_t M, int64_t K, cudaStream_t st,
                                       unsigned long long timeout_ns = PF_DEFAULT_TIMEOUT_NS,
-                                      long long dbg_skip_iter = -1) {
+                                      long long dbg_skip_iter = -1, bool pdl = false) {
     EncodeTiledFn enc = encode_tiled_fn();
     if (enc == nullptr) return BL_ERR_CUDA;
     if (count < 1 || count > PF_MAX_PROB) return BL_ERR_SHAPE;
@@ -580,15 +587,25 @@ inline bl_status prefill_launch_group(int sms, const PrefillJob *jobs, int count
     p.dbg_skip_iter = dbg_skip_iter;
     const int64_t tiles = n_tiles * m_tiles;
     const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
-    k_prefill_tc<<<grid, PF_THREADS, PF_SMEM_BYTES, st>>>(maps, p);
-    return cudaGetLastError() == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(PF_THREADS);
+    cfg.dynamicSmemBytes = PF_SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_prefill_tc, maps, p) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 
 inline bl_status prefill_launch(int sms, const uint8_t *packed, const float *gamma, const int8_t *x_q, const float *s,
                                 int64_t M, int64_t N, int64_t K, float *Y, int32_t *acc_out, cudaStream_t st,
-                                unsigned long long timeout_ns = PF_DEFAULT_TIMEOUT_NS, long long dbg_skip_iter = -1) {
+                                unsigned long long timeout_ns = PF_DEFAULT_TIMEOUT_NS, long long dbg_skip_iter = -1,
+                                bool pdl = false) {
     const PrefillJob job{packed, gamma, Y, acc_out, N};
-    return prefill_launch_group(sms, &job, 1, x_q, s, M, K, st, timeout_ns, dbg_skip_iter);
+    return prefill_launch_group(sms, &job, 1, x_q, s, M, K, st, timeout_ns, dbg_skip_iter, pdl);
 }
 
 }  // namespace bl

@@ -51,7 +51,12 @@ def test_layer3b(M):
 @pytest.mark.parametrize("which", ["o", "gate", "down"])
 def test_qat4b_layer(which):
     name, W, X, gain = workloads.qat4b(which=(which,))[0]
-    run_projection(W, X, gain)
+    Y = run_projection(W, X, gain)
+    # the per-call path (weights re-quantized in the call, act quant overlapping
+    # the weight pack, TMA-stored Y) gives the same bits
+    Yl = api.bl_linear(W.cuda(), X.cuda(), None if gain is None else gain.cuda(), workloads.SUBLN_EPS)
+    torch.cuda.synchronize()
+    assert torch.equal(Yl.view(torch.int32), Y.view(torch.int32))
 
 
 def test_single_workload_full():
