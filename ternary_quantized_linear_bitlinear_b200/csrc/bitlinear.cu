@@ -210,19 +210,41 @@ bool decode_eligible(int64_t M, int64_t K) {
     return M <= 16 && dec_xq_off(K) + M * dec_row_stride((int)K) <= DEC_SMEM_LIMIT;
 }
 
-bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st, int src = DEC_SRC_XQ) {
+bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st, int src = DEC_SRC_XQ, int sms = 148) {
+    // G (warps per 32-row group) per problem: dec_glog's choice, raised while
+    // the launch would leave SMs idle and the problem has k steps to split
+    // (small launches, e.g. one layer's projections at a time, get more CTAs
+    // with fewer rows each)
+    for (int i = 0; i < P.count; ++i) P.p[i].g_log2 = dec_glog(P.p[i].K);
+    auto ctas_of = [&](const DecodeProblem &q) {
+        const int tiles = (q.N + DEC_ROWS - 1) / DEC_ROWS;
+        const int per = DEC_WARPS >> q.g_log2;
+        return (tiles + per - 1) / per;
+    };
+    for (;;) {
+        int total = 0;
+        for (int i = 0; i < P.count; ++i) total += ctas_of(P.p[i]);
+        if (total >= sms) break;
+        bool raised = false;
+        for (int i = 0; i < P.count; ++i) {
+            DecodeProblem &q = P.p[i];
+            const int steps = (q.K + 255) >> 8;
+            if (q.g_log2 < 3 && (2 << q.g_log2) <= steps) {
+                ++q.g_log2;
+                raised = true;
+            }
+        }
+        if (!raised) break;
+    }
     int total = 0;
     int rs_max = 0, xq_off = 0;
     for (int i = 0; i < P.count; ++i) {
         DecodeProblem &q = P.p[i];
-        q.g_log2 = dec_glog(q.K);
-        int tiles = (q.N + DEC_ROWS - 1) / DEC_ROWS;
-        int per = DEC_WARPS >> q.g_log2;
         q.cta_begin = total;
-        total += (tiles + per - 1) / per;
+        total += ctas_of(q);
         int rs = dec_row_stride(q.K);
         rs_max = rs > rs_max ? rs : rs_max;
-        int xo = dec_xq_off(q.K);
+        const int xo = (((DEC_WARPS >> q.g_log2) * DEC_ROWS * (q.K >> 2)) + 127) & ~127;  // this G's weight bytes
         xq_off = xo > xq_off ? xo : xq_off;
     }
     P.xq_off = xq_off;
@@ -268,7 +290,7 @@ bl_status forward_impl(const DeviceInfo &d, const uint8_t *packed, const float *
         P.eps = 0.f;
         P.p[0] = DecodeProblem{packed, gamma, x_q, const_cast<float *>(s), Y, acc_out, nullptr, nullptr,
                                (int)N, (int)K, 0, 0};
-        return decode_launch(P, false, st);
+        return decode_launch(P, false, st, DEC_SRC_XQ, d.sms);
     }
     return prefill_launch(d.sms, packed, gamma, x_q, s, M, N, K, Y, acc_out, st, PF_DEFAULT_TIMEOUT_NS, -1, pdl);
 }
@@ -438,7 +460,7 @@ bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, u
     DeviceInfo *d;
     bl_status rc = device_info(&d);
     if (rc) return rc;
-    return decode_launch(P, (flags & BL_FWD_WEIGHTS_READY) != 0, (cudaStream_t)stream);
+    return decode_launch(P, (flags & BL_FWD_WEIGHTS_READY) != 0, (cudaStream_t)stream, DEC_SRC_XQ, d->sms);
 }
 
 bl_status bl_linear_decode_grouped(const bl_decode_problem *problems, int count, bl_dtype xdt, int64_t M,
@@ -465,7 +487,7 @@ bl_status bl_linear_decode_grouped(const bl_decode_problem *problems, int count,
     bl_status rc = device_info(&d);
     if (rc) return rc;
     return decode_launch(P, (flags & BL_FWD_WEIGHTS_READY) != 0, (cudaStream_t)stream,
-                         xdt == BL_BF16 ? DEC_SRC_BF16 : DEC_SRC_F32);
+                         xdt == BL_BF16 ? DEC_SRC_BF16 : DEC_SRC_F32, d->sms);
 }
 
 size_t bl_linear_workspace_bytes(int64_t M, int64_t N, int64_t K) {
@@ -509,7 +531,7 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt, in
         P.M = (int)M;
         P.eps = subln_eps;
         P.p[0] = DecodeProblem{packed, gamma, X, s, Y, nullptr, subln_gain, x_q, (int)N, (int)K, 0, 0};
-        return decode_launch(P, false, st, xdt == BL_BF16 ? DEC_SRC_BF16 : DEC_SRC_F32);
+        return decode_launch(P, false, st, xdt == BL_BF16 ? DEC_SRC_BF16 : DEC_SRC_F32, d->sms);
     }
     ActParams P;
     P.count = 1;
