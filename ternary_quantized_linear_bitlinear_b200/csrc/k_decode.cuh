@@ -12,7 +12,8 @@
 //     per CTA and the warps issue no global loads for weights.
 //   - A warp owns 32 rows (two 16-row MMA tiles that share every x_q
 //     fragment); G warps split their K range (G picked per problem from K so
-//     that each warp has at most 4 steps of 256 k).
+//     that each warp has at most 4 steps of 256 k and a CTA at most 48 KiB
+//     of weights; the host raises G for launches too small to fill the GPU).
 //   - Unpacking costs 1-2 ALU ops per 4 weights: with the packed layout, word
 //     (w << (6 - 2j)) & 0xC0C0C0C0 puts the codes of k = 16w' + 4j .. 4j+3 in
 //     the top two bits of four bytes, i.e. the int8 values 64 * W_q.
@@ -28,10 +29,11 @@
 //   - acc = (sum of 64 * W_q * x_q) >> 6 exactly; the split-K partials meet
 //     in shared memory; the epilogue rescales and stores Y (and acc).
 //   - Fused variant (SRC = bf16 or f32 activations): step 2 runs inside the
-//     CTA instead of a separate launch.  One warp per token row computes
-//     s = 127 / max|y| (y = x, or the SubLN RMSNorm of x) and writes x_q
-//     straight into the swizzled staging rows, with the same arithmetic as
-//     the stand-alone activation quantizer, while the weights stream in.
+//     CTA instead of a separate launch.  One warp per token row (for one or
+//     two tokens without SubLN: the whole CTA) computes s = 127 / max|y|
+//     (y = x, or the SubLN RMSNorm of x) and writes x_q straight into the
+//     swizzled staging rows, with the same arithmetic as the stand-alone
+//     activation quantizer, while the weights stream in.
 //     Every CTA of a problem quantizes the (L2-resident) rows itself; the
 //     problem's first CTA also writes x_q and s to global memory on request.
 #pragma once
