@@ -210,7 +210,7 @@ bool decode_eligible(int64_t M, int64_t K) {
     return M <= 16 && dec_xq_off(K) + M * dec_row_stride((int)K) <= DEC_SMEM_LIMIT;
 }
 
-bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st, int src = DEC_SRC_XQ, int sms = 148) {
+bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st, int src, int sms) {
     // G (warps per 32-row group) per problem: dec_glog's choice, raised while
     // the launch would leave SMs idle and the problem has k steps to split
     // (small launches, e.g. one layer's projections at a time, get more CTAs
