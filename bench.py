@@ -6,8 +6,8 @@ at M = 1, 4 and 8 tokens: per M, ONE grouped launch that quantizes the bf16
 activations, runs the ternary GEMV and rescales (bl_linear_decode_grouped).
 The ternary weights (29/42/29 split) are packed once at load time.  Weight
 bytes per step would fit in L2, so the packed weights are replicated and
-every step reads a different replica (the replicas total more than 3x the
-L2 size).
+every launch reads a different replica than the launches around it (the
+replicas total more than 3x the L2 size).
 
 Metric: decode GB/s = (packed weight bytes + bf16 activation bytes) per step
 / time, whole job, N GPUs = N independent replicas of the workload (weak
@@ -253,10 +253,15 @@ def native(args, rank, world, local):
     fused = {(M, r): fused_problems(M, r) for M in MS for r in range(R)}
     RDY = api.BL_FWD_WEIGHTS_READY
 
+    def replica(step, j):
+        """Replica read by launch j of a step: consecutive launches never share
+        weights (the launches of one step included), so none is fed from L2."""
+        return (len(MS) * step + j) % R
+
     def launch_step(stream_ptr, rep):
         """One step: per M, ONE fused launch (act quant + GEMV + rescale, 84 problems)."""
-        for M in MS:
-            rc = L.bl_linear_decode_grouped(fused[(M, rep)], count, api.BL_BF16, M, 1e-6, RDY, stream_ptr)
+        for j, M in enumerate(MS):
+            rc = L.bl_linear_decode_grouped(fused[(M, replica(rep, j))], count, api.BL_BF16, M, 1e-6, RDY, stream_ptr)
             if rc:
                 raise api.BitLinearError(rc, "bl_linear_decode_grouped")
 
@@ -338,8 +343,8 @@ def native(args, rank, world, local):
         tl = {(M, r): two_launch_problems(M, r) for M in MS for r in range(R)}
 
         def two_step(stream_ptr, rep):
-            for M in MS:
-                acts, fwd = tl[(M, rep)]
+            for j, M in enumerate(MS):
+                acts, fwd = tl[(M, replica(rep, j))]
                 if L.bl_quant_act_grouped(acts, count, api.BL_BF16, M, 1e-6, stream_ptr):
                     raise RuntimeError("bl_quant_act_grouped")
                 if L.bl_forward_grouped(fwd, count, M, RDY, stream_ptr):
@@ -412,8 +417,8 @@ def native(args, rank, world, local):
                 ev_up[k].record(s_up)
             stream.wait_event(ev_up[k])
             stream.wait_event(ev_dn[k])              # this slot's previous Y has been read back
-            for M in MS:
-                rc = L.bl_linear_decode_grouped(slot_arrs[k][(M, it % R)], count, api.BL_BF16, M, 1e-6, RDY, sp)
+            for j, M in enumerate(MS):
+                rc = L.bl_linear_decode_grouped(slot_arrs[k][(M, replica(it, j))], count, api.BL_BF16, M, 1e-6, RDY, sp)
                 if rc:
                     raise api.BitLinearError(rc, "bl_linear_decode_grouped")
             ev_comp[k].record(stream)
@@ -435,7 +440,7 @@ def native(args, rank, world, local):
         "config": {"workload": WORKLOAD, "tokens_per_step": sum(MS), "projections": count,
                    "weight_bytes_per_m": wbytes, "activation_bytes_per_step": sum(2 * xbytes[M] for M in MS),
                    "weight_replicas": R,
-                   "l2": f"{R} rotating packed-weight replicas ({R * wbytes / 2**20:.0f} MiB > 3x L2)",
+                   "l2": f"{R} rotating packed-weight replicas ({R * wbytes / 2**20:.0f} MiB > 3x L2), a different one for every launch",
                    "parallelism": f"replicas x{world}", "launch": "CUDA graph of whole steps, 3 fused launches each"},
         "roofline": roofline, "e2e": e2e, "alt_paths": alt,
         "gpu_launches": steps_timed * len(MS),
