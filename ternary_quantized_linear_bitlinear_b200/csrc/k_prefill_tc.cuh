@@ -3,40 +3,51 @@
 // What it computes ("bitone" README, How 1.58-bit Works and Forward pass):
 //   acc[m, n] = sum_k x_q[m, k] * W_q[n, k];  Y[m, n] = acc * (gamma / s[m])
 //
-// One output tile = 128 tokens (m) x 256 weight rows (n), computed with
-// tcgen05.mma.cta_group::1.kind::i8, M = 128, N = 256, K = 32 per
-// instruction (the issue cost of one MMA is nearly independent of N, so
-// N = 256 is what reaches the tensor peak):
-//   A = x_q tile, by TMA with 128-byte swizzle, K-major;
-//   B = 64 * W_q as int8 in shared memory: the packed 2-bit rows arrive by
-//     TMA, eight expander warps (one weight row per thread) unpack them
-//     ((word << (6 - 2j)) & 0xC0C0C0C0 gives four int8 lanes), store them in
-//     the 128-byte-swizzled K-major layout the MMA reads, then fence the
-//     async proxy;
-//   D = int32 accumulators in TMEM (lane = token, column = weight row), two
-//     256-column buffers so the epilogue of one tile overlaps the MMAs of the
-//     next.  Each epilogue thread owns one token (one float(gamma / s[m]) per
-//     tile); a warp converts a 32 x 32 block into a 128B-swizzled staging
-//     buffer and one lane writes it to Y with a TMA tensor store, so every
-//     store is a full-line bulk write (tails clipped by the tensor map).
-// The exact sum is 64 * acc (|64 acc| <= 2^28, exact in int32 and in
+// Two CTAs (a cluster pair on two SMs) compute one output tile of 256 tokens
+// (m) x 256 weight rows (n) with tcgen05.mma.cta_group::2.kind::i8, M = 256,
+// N = 256, K = 32 per instruction, issued by one thread of the pair's first
+// CTA (the leader).  Each CTA holds its own half of both operands:
+//   A = its 128 tokens of x_q, by TMA with 128-byte swizzle, K-major;
+//   B = 64 * W_q of its 128 of the 256 weight rows as int8: the packed 2-bit
+//     rows arrive by TMA, four expander warps (one weight row per thread)
+//     unpack them ((word << (6 - 2j)) & 0xC0C0C0C0 gives four int8 lanes),
+//     store them in the 128-byte-swizzled K-major layout the MMA reads, then
+//     fence the async proxy;
+//   D = int32 accumulators in each CTA's TMEM (lane = its token, column =
+//     weight row of the full 256), two 256-column buffers so the epilogue of
+//     one tile overlaps the MMAs of the next.
+// The pair reads each B half once for both token halves, so every CTA
+// expands, stores and feeds the tensor core half the weight bytes of a
+// one-CTA 128 x 256 tile for the same number of MACs per SM: the shared
+// memory traffic per MAC (TMA writes, expansion, operand reads), which bounds
+// the one-CTA design, drops by about a third.
+// Each epilogue thread owns one token (one float(gamma / s[m]) per tile); a
+// warp converts a 32 x 32 block into a 128B-swizzled staging buffer and one
+// lane writes it to Y with a TMA tensor store (tails clipped by the tensor
+// map).  The exact sum is 64 * acc (|64 acc| <= 2^28, exact in int32 and in
 // float), so Y = float(float(64 acc) * (f / 64)) with f = float(gamma / s[m])
 // (f / 64 is exact) -- the same bits as float(acc) * f.
 //
 // Pipelines: PF_STAGES shared-memory stages carry x_q and packed tiles from
-// TMA; PF_BSTAGES shared-memory stages carry the expanded weights from the
-// expanders to the MMA.  MMA completion frees both (two commits).
+// TMA (per CTA, own barriers); PF_BSTAGES stages carry the expanded weights
+// to the MMA: both CTAs' expanders arrive on the leader's "ready" barrier.
+// MMA completion is committed to the barriers of both CTAs at once
+// (tcgen05.commit multicast), which frees both kinds of stage and signals the
+// epilogues; both CTAs' epilogues arrive on the leader's "accumulator empty"
+// barrier.  The leader's "ready" arrival from the peer's expanders also
+// implies that the peer's x_q stage has landed (they waited for it).
 //
-// Warp roles (persistent: one CTA per SM loops over tiles):
+// Warp roles (persistent: one cluster pair per two SMs loops over tiles):
 //   warp 0        TMA producer (one thread)
-//   warp 1        TMEM allocator + MMA issuer (one thread)
-//   warps 2..9    expanders: weight row 32*(w - 2) + lane of the tile
-//   warps 10..17  epilogue: TMEM lanes 32*(w % 4) .. +31 (tokens), columns
-//                 128*((w - 10) / 4) .. +127 (weight rows)
+//   warp 1        TMEM allocator (both CTAs) + MMA issuer (leader, one thread)
+//   warps 2..5    expanders: weight row 32*(w - 2) + lane of this CTA's half
+//   warps 6..13   epilogue: TMEM lanes 32*(w % 4) .. +31 (tokens), columns
+//                 128*((w - 6) / 4) .. +127 (weight rows)
 // Every mbarrier wait is bounded (globaltimer); a wait that gives up raises
-// the device error word, sets a CTA abort flag and the CTA drains its
-// in-flight copies and MMAs (again with bounded waits) before it frees TMEM
-// and exits.  No wait is unbounded and nothing traps.
+// the device error word, sets the CTA's abort flag and the CTA drains its
+// in-flight copies and MMAs (again with bounded waits) before the pair meets
+// at a cluster barrier, frees TMEM and exits.  No wait is unbounded and
+// nothing traps.  No copy uses cluster multicast.
 #pragma once
 
 #include <cuda.h>
@@ -45,22 +56,24 @@
 
 namespace bl {
 
-constexpr int PF_BM = 128;         // tokens per tile (MMA M, TMEM lanes)
-constexpr int PF_BN = 256;         // weight rows per tile (MMA N, TMEM columns)
-constexpr int PF_BK = 128;         // k per pipeline stage (4 MMAs of K = 32)
-constexpr int PF_STAGES = 4;       // TMA stages (x_q + packed)
-constexpr int PF_BSTAGES = 2;      // expanded-weight stages
-constexpr int PF_EXP_WARPS = PF_BN / 32;
+constexpr int PF_BM = 128;          // tokens per CTA (MMA M = 2 x 128, TMEM lanes)
+constexpr int PF_BN = 256;          // weight rows per pair tile (MMA N, TMEM columns)
+constexpr int PF_BNH = PF_BN / 2;   // weight rows expanded per CTA
+constexpr int PF_BK = 128;          // k per pipeline stage (4 MMAs of K = 32)
+constexpr int PF_STAGES = 6;        // TMA stages (x_q + packed)
+constexpr int PF_BSTAGES = 4;       // expanded-weight stages
+constexpr int PF_EXP_WARPS = PF_BNH / 32;
 constexpr int PF_EPI_WARPS = 8;
 constexpr int PF_EPI_WARP0 = 2 + PF_EXP_WARPS;
 constexpr int PF_THREADS = 32 * (PF_EPI_WARP0 + PF_EPI_WARPS);
 constexpr int PF_A_BYTES = PF_BM * PF_BK;          // x_q stage: 16 KiB
-constexpr int PF_P_BYTES = PF_BN * PF_BK / 4;      // packed stage: 8 KiB
-constexpr int PF_B_BYTES = PF_BN * PF_BK;          // expanded stage: 32 KiB
+constexpr int PF_P_BYTES = PF_BNH * PF_BK / 4;     // packed stage: 4 KiB
+constexpr int PF_B_BYTES = PF_BNH * PF_BK;         // expanded stage: 16 KiB
 constexpr int PF_TMEM_COLS = 512;                  // 2 x 256 accumulator columns
 constexpr int PF_Y_BYTES = 32 * 32 * 4;            // per-epilogue-warp Y staging block (TMA store)
 
-// shared memory carve-up (offsets from a 1024-byte aligned base)
+// shared memory carve-up (offsets from a 1024-byte aligned base; identical in
+// both CTAs of a pair, which the pair MMA relies on)
 constexpr int PF_OFF_A = 0;
 constexpr int PF_OFF_B = PF_OFF_A + PF_STAGES * PF_A_BYTES;
 constexpr int PF_OFF_P = PF_OFF_B + PF_BSTAGES * PF_B_BYTES;
@@ -72,6 +85,8 @@ constexpr int PF_SMEM_USED = PF_OFF_MISC + 16;
 constexpr int PF_SMEM_BYTES = PF_SMEM_USED + 1024;                     // + alignment slack
 static_assert(PF_SMEM_BYTES > 116 * 1024, "keeps one CTA per SM, so the TMEM allocation never waits");
 static_assert(PF_SMEM_BYTES <= 227 * 1024, "shared memory budget");
+static_assert(PF_OFF_B % 1024 == 0 && PF_OFF_Y % 1024 == 0 && PF_A_BYTES % 1024 == 0 && PF_B_BYTES % 1024 == 0,
+              "128-byte swizzled stages start on 1024-byte boundaries");
 
 // Up to PF_MAX_PROB weight matrices that share one activation (e.g. the q,
 // k, v or the gate, up projections of a layer) in one launch: their output
@@ -99,9 +114,9 @@ struct PrefillParams {
     int nprob;
     const float *s;
     int M, K;
-    int n_tiles, m_tiles, k_stages;  // n_tiles: over all problems
+    int n_tiles, m_tiles, k_stages;  // n_tiles: over all problems; m_tiles: 256-token pair tiles
     unsigned long long timeout_ns;
-    long long dbg_skip_iter;  // >= 0: the producer never issues this k-iteration (bounded-wait test)
+    long long dbg_skip_iter;  // >= 0: the producers never issue this k-iteration (bounded-wait test)
     int y_tma;                // 1: Y written by TMA stores (every N % 4 == 0 and no acc output)
 };
 
@@ -127,20 +142,65 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, int x, int 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc], kind::i8, cta_group::1
-__device__ __forceinline__ void tc_mma_i8_ss(u32 d_tmem, unsigned long long a_desc, unsigned long long b_desc,
-                                             u32 idesc, u32 accumulate) {
+__device__ __forceinline__ u32 cluster_ctarank() {
+    u32 r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ u32 cluster_idx() {
+    u32 r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ u32 cluster_count() {
+    u32 r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+
+// every thread of both CTAs; orders the barrier initialisation (release) before
+// any arrival from the peer, and at the end keeps a CTA resident while its peer
+// may still touch its shared memory
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// arrive on the barrier at the same shared-memory offset in CTA `rank` of the
+// cluster (this CTA included).  Default (CTA-scope release) semantics: what the
+// arrival publishes is shared memory for the tensor core, ordered by the
+// async-proxy fence before it, or TMEM reads ordered by tcgen05.fence; a
+// cluster-scope release here (a fence per expander warp per k block) measured
+// 40 % slower.
+__device__ __forceinline__ void mbar_arrive_cluster(u32 bar, u32 rank) {
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.shared::cluster.b64 _, [ra];\n\t}"
+        ::"r"(bar), "r"(rank)
+        : "memory");
+}
+
+// D[tmem of both CTAs] (+)= A[smem desc, each CTA's half] * B[smem desc, each
+// CTA's half of N], kind::i8, cta_group::2
+__device__ __forceinline__ void tc2_mma_i8_ss(u32 d_tmem, unsigned long long a_desc, unsigned long long b_desc,
+                                              u32 idesc, u32 accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}"
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
-__device__ __forceinline__ void tc_commit(u32 bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
+// arrive (once the MMAs issued so far complete) on the barrier at this
+// shared-memory offset in both CTAs of the pair
+__device__ __forceinline__ void tc2_commit_pair(u32 bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+        ::"r"(bar), "h"((unsigned short)3)
+        : "memory");
 }
 
 __device__ __forceinline__ void tc_ld_32x32b_x32(u32 taddr, u32 (&r)[32]) {
@@ -171,13 +231,14 @@ __device__ __forceinline__ unsigned long long smem_desc_k_sw128(u32 saddr) {
     return d;
 }
 
-// Instruction descriptor, kind::i8: D s32, A s8, B s8, both K-major, N = PF_BN, M = PF_BM.
+// Instruction descriptor, kind::i8: D s32, A s8, B s8, both K-major,
+// N = PF_BN, M = 2 x PF_BM (the pair).
 __host__ __device__ constexpr u32 pf_idesc() {
-    return (2u << 4)                    // D format: s32
-           | (1u << 7)                  // A format: signed 8-bit
-           | (1u << 10)                 // B format: signed 8-bit
-           | ((u32)(PF_BN >> 3) << 17)  // N >> 3
-           | ((u32)(PF_BM >> 4) << 24); // M >> 4
+    return (2u << 4)                          // D format: s32
+           | (1u << 7)                        // A format: signed 8-bit
+           | (1u << 10)                       // B format: signed 8-bit
+           | ((u32)(PF_BN >> 3) << 17)        // N >> 3
+           | ((u32)((2 * PF_BM) >> 4) << 24); // M >> 4
 }
 
 // ---------------------------------------------------------------------------
@@ -189,8 +250,8 @@ __device__ __forceinline__ int pf_prob_of(const PrefillParams &p, int nt) {
     return pi;
 }
 
-__global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_constant__ PrefillMaps maps,
-                                                               const __grid_constant__ PrefillParams p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
+    k_prefill_tc(const __grid_constant__ PrefillMaps maps, const __grid_constant__ PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     const u32 sbase = smem_u32(sm);
@@ -205,18 +266,19 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
     volatile int *s_abort = reinterpret_cast<volatile int *>(sm + PF_OFF_MISC + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const u32 rank = cluster_ctarank();  // 0: the leader, which issues the pair's MMAs
     if (threadIdx.x == 0) {
         for (int s = 0; s < PF_STAGES; ++s) {
             mbar_init(BAR_FULL(s), 1);
             mbar_init(BAR_EMPTY(s), 1);
         }
         for (int a = 0; a < PF_BSTAGES; ++a) {
-            mbar_init(BAR_BREADY(a), PF_EXP_WARPS);
+            mbar_init(BAR_BREADY(a), 2 * PF_EXP_WARPS);  // used in the leader: both CTAs' expanders
             mbar_init(BAR_BEMPTY(a), 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(BAR_ACCFULL(b), 1);
-            mbar_init(BAR_ACCEMPTY(b), PF_EPI_WARPS);
+            mbar_init(BAR_ACCEMPTY(b), 2 * PF_EPI_WARPS);  // used in the leader: both CTAs' epilogues
         }
         *s_abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -227,18 +289,22 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         }
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
+        // both CTAs, same warp: the pair's columns are allocated in both TMEMs
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(s_tmem)),
                      "r"(PF_TMEM_COLS)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
+    tc_fence_before();
     __syncthreads();
+    cluster_sync_all();
     tc_fence_after();
     const u32 tmem = *s_tmem;
 
     const int total_tiles = p.n_tiles * p.m_tiles;
     const int KS = p.k_stages;
     const unsigned long long TO = p.timeout_ns;
+    const int cid = (int)cluster_idx(), ncl = (int)cluster_count();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
@@ -248,11 +314,13 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
             asm volatile("griddepcontrol.wait;" ::: "memory");
             long long it = 0;
             bool failed = false;
-            for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x) {
+            for (int tile = cid; tile < total_tiles && !failed; tile += ncl) {
                 const int nt = tile % p.n_tiles, mt = tile / p.n_tiles;
                 const int pi = pf_prob_of(p, nt);
                 const CUtensorMap *tmw = &maps.w[pi];
                 const int ntl = nt - p.prob[pi].nt_begin;
+                const int arow = mt * (2 * PF_BM) + (int)rank * PF_BM;   // this CTA's tokens
+                const int brow = ntl * PF_BN + (int)rank * PF_BNH;       // this CTA's weight rows
                 for (int ks = 0; ks < KS; ++ks, ++it) {
                     const int s = (int)(it % PF_STAGES);
                     const u32 ph = (u32)((it / PF_STAGES) & 1);
@@ -262,8 +330,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                     }
                     if (it == p.dbg_skip_iter) continue;  // test hook: this stage never arrives
                     mbar_arrive_expect_tx(BAR_FULL(s), PF_A_BYTES + PF_P_BYTES);
-                    tma_load_2d(sbase + PF_OFF_A + s * PF_A_BYTES, &maps.x, ks * PF_BK, mt * PF_BM, BAR_FULL(s));
-                    tma_load_2d(sbase + PF_OFF_P + s * PF_P_BYTES, tmw, ks * (PF_BK / 4), ntl * PF_BN, BAR_FULL(s));
+                    tma_load_2d(sbase + PF_OFF_A + s * PF_A_BYTES, &maps.x, ks * PF_BK, arow, BAR_FULL(s));
+                    tma_load_2d(sbase + PF_OFF_P + s * PF_P_BYTES, tmw, ks * (PF_BK / 4), brow, BAR_FULL(s));
                 }
             }
             if (failed) {
@@ -279,15 +347,16 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
+        if (lane == 0 && rank == 0) {
             const u32 idesc = pf_idesc();
             long long it = 0;
             int tc = 0;
             bool failed = false, issued = false;
             u32 last_bar = 0, last_ph = 0;
-            for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x, ++tc) {
+            for (int tile = cid; tile < total_tiles && !failed; tile += ncl, ++tc) {
                 const int b = tc & 1;
                 const u32 cph = (u32)((tc >> 1) & 1);
+                // both CTAs' epilogues have drained this accumulator buffer
                 if (!mbar_wait(BAR_ACCEMPTY(b), cph ^ 1u, TO, s_abort)) {
                     failed = true;
                     break;
@@ -299,7 +368,10 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                     const u32 ph = (u32)((it / PF_STAGES) & 1);
                     const int a = (int)(it % PF_BSTAGES);
                     const u32 aph = (u32)((it / PF_BSTAGES) & 1);
-                    if (!mbar_wait(BAR_FULL(s), ph, TO, s_abort) || !mbar_wait(BAR_BREADY(a), aph, TO, s_abort)) {
+                    // own x_q stage landed; both CTAs' expanded halves ready
+                    // (the peer's expanders waited for the peer's x_q stage)
+                    if (!mbar_wait(BAR_FULL(s), ph, TO, s_abort) ||
+                        !mbar_wait(BAR_BREADY(a), aph, TO, s_abort)) {
                         failed = true;
                         break;
                     }
@@ -308,17 +380,17 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                     const u32 bstage = sbase + PF_OFF_B + a * PF_B_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < PF_BK / 32; ++kk) {
-                        tc_mma_i8_ss(d_tmem, smem_desc_k_sw128(astage + kk * 32), smem_desc_k_sw128(bstage + kk * 32),
-                                     idesc, (ks | kk) != 0 ? 1u : 0u);
+                        tc2_mma_i8_ss(d_tmem, smem_desc_k_sw128(astage + kk * 32), smem_desc_k_sw128(bstage + kk * 32),
+                                      idesc, (ks | kk) != 0 ? 1u : 0u);
                     }
-                    tc_commit(BAR_EMPTY(s));
-                    tc_commit(BAR_BEMPTY(a));
+                    tc2_commit_pair(BAR_EMPTY(s));
+                    tc2_commit_pair(BAR_BEMPTY(a));
                     issued = true;
                     last_bar = BAR_EMPTY(s);
                     last_ph = ph;
                 }
                 if (failed) break;
-                tc_commit(BAR_ACCFULL(b));
+                tc2_commit_pair(BAR_ACCFULL(b));
             }
             if (failed) {
                 raise_device_error(DEVERR_TIMEOUT_MMA);
@@ -329,11 +401,11 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         }
     } else if (warp < PF_EPI_WARP0) {
         // ------------------------------------------------------------ expanders
-        const int row = (warp - 2) * 32 + lane;  // weight row within the tile
+        const int row = (warp - 2) * 32 + lane;  // weight row within this CTA's half
         const int rsw = row & 7;                 // 128-byte swizzle phase of this row
         long long it = 0;
         bool failed = false;
-        for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x) {
+        for (int tile = cid; tile < total_tiles && !failed; tile += ncl) {
             for (int ks = 0; ks < KS; ++ks, ++it) {
                 const int s = (int)(it % PF_STAGES);
                 const u32 ph = (u32)((it / PF_STAGES) & 1);
@@ -362,7 +434,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                 // make the generic-proxy stores visible to the tensor core (async proxy)
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                 __syncwarp();
-                if (lane == 0) mbar_arrive(BAR_BREADY(a));
+                if (lane == 0) mbar_arrive_cluster(BAR_BREADY(a), 0);
             }
         }
         if (failed && lane == 0) {
@@ -380,7 +452,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         const u32 ystage_s = smem_u32(ystage);
         int tc = 0;
         bool failed = false;
-        for (int tile = blockIdx.x; tile < total_tiles && !failed; tile += gridDim.x, ++tc) {
+        for (int tile = cid; tile < total_tiles && !failed; tile += ncl, ++tc) {
             const int nt = tile % p.n_tiles, mt = tile / p.n_tiles;
             const PrefillProb &pp = p.prob[pf_prob_of(p, nt)];
             const int pN = pp.N;
@@ -389,7 +461,8 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
             const bool vec_ok = (pN & 3) == 0;            // rows of Y 16-byte aligned
             const int b = tc & 1;
             const u32 cph = (u32)((tc >> 1) & 1);
-            const int m = mt * PF_BM + q * 32 + lane;     // this thread's token
+            const int mrow0 = mt * (2 * PF_BM) + (int)rank * PF_BM + q * 32;  // this warp's first token
+            const int m = mrow0 + lane;                   // this thread's token
             const bool mvalid = m < p.M;
             // float(gamma / s[m]) / 64 (exact)
             const float f = mvalid ? __fmul_rn(__fdiv_rn(gamma, p.s[m]), 0.015625f) : 0.f;
@@ -411,7 +484,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                 if (c0 + 32 == PF_BN / 2) {
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(BAR_ACCEMPTY(b));
+                    if (lane == 0) mbar_arrive_cluster(BAR_ACCEMPTY(b), 0);
                 }
                 if (p.y_tma) {
                     // the previous TMA store from this block has finished reading it
@@ -428,7 +501,7 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();
-                    if (lane == 0) tma_store_2d(&maps.y[pf_prob_of(p, nt)], n0 + c0, mt * PF_BM + q * 32, ystage_s);
+                    if (lane == 0) tma_store_2d(&maps.y[pf_prob_of(p, nt)], n0 + c0, mrow0, ystage_s);
                 } else if (mvalid) {
                     if (full) {
 #pragma unroll
@@ -467,10 +540,14 @@ __global__ void __launch_bounds__(PF_THREADS, 1) k_prefill_tc(const __grid_const
         }
     }
 
+    tc_fence_before();
     __syncthreads();
+    // neither CTA leaves (or frees TMEM) while its peer may still arrive on its
+    // barriers, read its shared memory through the pair MMA or write its TMEM
+    cluster_sync_all();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(PF_TMEM_COLS)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(PF_TMEM_COLS)
                      : "memory");
     }
 }
@@ -509,6 +586,27 @@ inline EncodeTiledFn encode_tiled_fn() {
 inline cudaError_t prefill_setup() {
     if (encode_tiled_fn() == nullptr) return cudaErrorNotSupported;
     return cudaFuncSetAttribute(k_prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM_BYTES);
+}
+
+// Cluster pairs that can be resident at once on the current device (the
+// persistent grid never exceeds it, so every pair runs in the first wave).
+inline int prefill_max_pairs(int sms) {
+    static int cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sms / 2;
+    if (cache[dev] > 0) return cache[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * (sms / 2)));
+    cfg.blockDim = dim3(PF_THREADS);
+    cfg.dynamicSmemBytes = PF_SMEM_BYTES;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_prefill_tc, &cfg) != cudaSuccess || n < 1) {
+        (void)cudaGetLastError();
+        n = sms / 2;
+    }
+    if (n > sms / 2) n = sms / 2;
+    cache[dev] = n;
+    return n;
 }
 
 constexpr unsigned long long PF_DEFAULT_TIMEOUT_NS = 2000000000ull;  // 2 s per wait
@@ -555,7 +653,7 @@ inline bl_status prefill_launch_group(int sms, const PrefillJob *jobs, int count
         {
             const cuuint64_t gdim[2] = {(cuuint64_t)(K / 4), (cuuint64_t)j.N};
             const cuuint64_t gstride[1] = {(cuuint64_t)(K / 4)};
-            const cuuint32_t box[2] = {(cuuint32_t)(PF_BK / 4), (cuuint32_t)PF_BN};
+            const cuuint32_t box[2] = {(cuuint32_t)(PF_BK / 4), (cuuint32_t)PF_BNH};  // one CTA's half of a tile
             if (enc(&maps.w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(j.packed), gdim, gstride, box,
                     es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -573,7 +671,7 @@ inline bl_status prefill_launch_group(int sms, const PrefillJob *jobs, int count
         p.prob[i] = PrefillProb{j.gamma, j.Y, j.acc_out, (int)j.N, (int)n_tiles};
         n_tiles += (j.N + PF_BN - 1) / PF_BN;
     }
-    const int64_t m_tiles = (M + PF_BM - 1) / PF_BM;
+    const int64_t m_tiles = (M + 2 * PF_BM - 1) / (2 * PF_BM);  // 256-token pair tiles
     if (n_tiles * m_tiles > 0x7fffffffLL) return BL_ERR_SHAPE;
     p.nprob = count;
     p.y_tma = y_tma;
@@ -586,7 +684,8 @@ inline bl_status prefill_launch_group(int sms, const PrefillJob *jobs, int count
     p.timeout_ns = timeout_ns;
     p.dbg_skip_iter = dbg_skip_iter;
     const int64_t tiles = n_tiles * m_tiles;
-    const unsigned grid = (unsigned)(tiles < sms ? tiles : sms);
+    const int pairs = prefill_max_pairs(sms);
+    const unsigned grid = 2u * (unsigned)(tiles < pairs ? tiles : pairs);  // cluster pairs (__cluster_dims__)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(PF_THREADS);
