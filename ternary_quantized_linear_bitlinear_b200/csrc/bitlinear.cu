@@ -51,8 +51,10 @@ bl_status device_info(DeviceInfo **out) {
                 fail |= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM_LIMIT) !=
                         cudaSuccess;
             fail |= prefill_setup() != cudaSuccess;
-            fail |= cudaFuncSetAttribute(k_act_quant_subln_smem<false, true>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, AQM_SMEM_BYTES) != cudaSuccess;
+            for (auto fn : {k_act_quant_subln_row<false, true>, k_act_quant_subln_row<true, false>,
+                            k_act_quant_subln_row<false, false>})
+                fail |= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, AQR_MAX_K * 4) !=
+                        cudaSuccess;
             if (fail) return BL_ERR_CUDA;
         }
         d.init = true;
@@ -152,30 +154,28 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
     for (int i = 0; i < P.count; ++i) subln |= P.p[i].gain != nullptr;
     const long long rows = (long long)P.count * P.M;
     const unsigned wgrid = (unsigned)((rows + AQW_WARPS - 1) / AQW_WARPS);
-    if (subln && glu && nvec > 32 * AQS_V) {
-        // gated FFN rows longer than one chunk: one warp per row, h cached in
-        // shared memory as float (gate and up read once, each element divided
-        // once).  Measured faster than the chunked kernel for these rows and
-        // slower for plain long rows, whose occupancy it halves.
-        const int kmax = (int)Kmax;
-        int wpc = (int)((AQM_SMEM_BYTES / 4) / kmax);
-        if (wpc > AQW_WARPS) wpc = AQW_WARPS;
-        if (wpc >= 1) {
-            const unsigned sgrid = (unsigned)((rows + wpc - 1) / wpc);
-            const size_t smem = (size_t)wpc * kmax * 4;
-            cudaLaunchConfig_t cfg = {};
-            cfg.gridDim = dim3(sgrid);
-            cfg.blockDim = dim3(AQW_WARPS * 32);
-            cfg.dynamicSmemBytes = smem;
-            cfg.stream = st;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-            attr[0].val.programmaticStreamSerializationAllowed = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = pdl ? 1 : 0;
-            return cudaLaunchKernelEx(&cfg, k_act_quant_subln_smem<false, true>, P, wpc) == cudaSuccess ? BL_OK
-                                                                                                 : BL_ERR_CUDA;
-        }
+    if (subln && nvec > (glu ? 32 * AQS_V : 256) && Kmax <= AQR_MAX_K) {
+        // SubLN rows (gated FFN rows longer than one chunk, plain rows longer
+        // than 256 vectors): one CTA per row, the row cached in shared memory
+        // as float (read once, each element divided once), four warps per
+        // row.  Measured 1.9x faster than a warp per row for the gated
+        // [8192, 4096] input, 2-10 % faster for bf16 rows of 2560 and 9728,
+        // slower for bf16 rows of 1536 (which the chunked warp kernel keeps).
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)rows);
+        cfg.blockDim = dim3(AQR_THREADS);
+        cfg.dynamicSmemBytes = (size_t)Kmax * 4;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = pdl ? 1 : 0;
+        cudaError_t e;
+        if (glu) e = cudaLaunchKernelEx(&cfg, k_act_quant_subln_row<false, true>, P);
+        else if (bf16) e = cudaLaunchKernelEx(&cfg, k_act_quant_subln_row<true, false>, P);
+        else e = cudaLaunchKernelEx(&cfg, k_act_quant_subln_row<false, false>, P);
+        return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
     }
     if (subln) {
         // one warp per row, chunked, any K (rows without a gain: plain)

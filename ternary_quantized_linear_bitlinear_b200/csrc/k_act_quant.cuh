@@ -15,8 +15,9 @@
 //                      16-byte vectors), no SubLN
 //   k_act_quant        one CTA per row, longer rows, no SubLN
 //   k_act_quant_subln  one warp per row, chunked, any length, SubLN
-//   k_act_quant_subln_smem  one warp per row cached in shared memory,
-//                      SubLN, for the gated FFN input (bl_ffn_act_quant)
+//   k_act_quant_subln_row   one CTA per row cached in shared memory,
+//                      SubLN, rows longer than 256 vectors and the gated
+//                      FFN input (bl_ffn_act_quant)
 #pragma once
 
 #include "bl_common.cuh"
@@ -227,7 +228,6 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_
 //   pass 3  r = sqrtf(float(double(S) / K) + eps); max|y|, y = float(float(x / r) * g)
 //   pass 4  x_q = clamp(rne(float(y * s)), -128, 127), s = float(127 / max(max|y|, 1e-5f))
 constexpr int AQS_V = 4;
-constexpr int AQM_SMEM_BYTES = 110 * 1024;  // row cache of k_act_quant_subln_smem per CTA (two CTAs per SM)
 
 template <bool BF16, bool GLU>
 __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid_constant__ ActParams P) {
@@ -374,62 +374,77 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
-// One warp per row with SubLN, the row cached in shared memory as float32
-// (used for the gated FFN input h): gate and up are read from HBM once and
-// each element is divided once -- pass 3 stores y over h in place and pass 4
-// quantizes it.  Same arithmetic and passes as k_act_quant_subln;
-// warps_per_cta rows per CTA, each owning K floats of dynamic shared memory.
+// One CTA (AQR_THREADS threads) per row with SubLN, the row cached in shared
+// memory as float32: the same arithmetic and passes as k_act_quant_subln,
+// with the row's elements spread over four warps and the reductions (max,
+// the windowed exact sum of squares and its "smaller values remain" flag)
+// combined through shared memory.  A warp per row left too few independent
+// chains per SM to hide the latency of the exact arithmetic.
+constexpr int AQR_THREADS = 128;
+constexpr int AQR_WARPS = AQR_THREADS / 32;
+constexpr int AQR_MAX_K = 24 * 1024;  // rows cached per CTA: K * 4 bytes of dynamic shared memory
+
+__device__ __forceinline__ u32 aqr_block_max(u32 v, u32 *s_u) {
+    v = warp_max_u32(v);
+    __syncthreads();  // s_u free (a previous reduction has been read)
+    if ((threadIdx.x & 31) == 0) s_u[threadIdx.x >> 5] = v;
+    __syncthreads();
+    u32 r = s_u[0];
+#pragma unroll
+    for (int w = 1; w < AQR_WARPS; ++w) r = max(r, s_u[w]);
+    return r;
+}
+
 template <bool BF16, bool GLU>
-__global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln_smem(const __grid_constant__ ActParams P,
-                                                                          int warps_per_cta) {
+__global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __grid_constant__ ActParams P) {
     static_assert(!(GLU && BF16), "GLU inputs are float32 projection outputs");
     constexpr int EPV = BF16 ? 8 : 4;
-    extern __shared__ __align__(16) float s_rows[];
+    constexpr int U = 4;  // 16-byte vectors in flight per thread in pass 1
+    extern __shared__ __align__(16) float s_row[];
+    __shared__ u32 s_u[AQR_WARPS];
+    __shared__ u64 s_lo[AQR_WARPS], s_hi[AQR_WARPS];
+    __shared__ float s_r;
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int gw = blockIdx.x * warps_per_cta + warp;
-    if (warp >= warps_per_cta || gw >= P.count * P.M) {
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-        return;
-    }
-    const int pi = gw / P.M, m = gw - pi * P.M;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int pi = blockIdx.x / P.M, m = blockIdx.x - pi * P.M;
     const ActProblem &pr = P.p[pi];
     const int K = pr.K, nvec = K / EPV;
-    float *row = s_rows + (size_t)warp * K;
     const uint4 *xr = reinterpret_cast<const uint4 *>(pr.X) + (size_t)m * nvec;
     const uint4 *ur = GLU ? reinterpret_cast<const uint4 *>(pr.X2) + (size_t)m * nvec : nullptr;
     const float4 *g4 = reinterpret_cast<const float4 *>(pr.gain);
     // pass 1: load (once), cache as float, max|x|
     u32 amax = 0;
-    for (int v0 = 0; v0 < nvec; v0 += 32 * AQS_V) {
-        uint4 c[AQS_V];
+    for (int v0 = 0; v0 < nvec; v0 += AQR_THREADS * U) {
+        uint4 c[U];
 #pragma unroll
-        for (int i = 0; i < AQS_V; ++i) {
-            const int vi = v0 + 32 * i + lane;
+        for (int i = 0; i < U; ++i) {
+            const int vi = v0 + AQR_THREADS * i + tid;
             c[i] = vi < nvec ? ldg_stream_v4(xr + vi) : make_uint4(0, 0, 0, 0);
         }
         if (GLU) {
 #pragma unroll
-            for (int i = 0; i < AQS_V; ++i) {
-                const int vi = v0 + 32 * i + lane;
+            for (int i = 0; i < U; ++i) {
+                const int vi = v0 + AQR_THREADS * i + tid;
                 if (vi < nvec) c[i] = glu_relu2_v4(c[i], ldg_stream_v4(ur + vi));
             }
         }
 #pragma unroll
-        for (int i = 0; i < AQS_V; ++i) {
-            const int vi = v0 + 32 * i + lane;
+        for (int i = 0; i < U; ++i) {
+            const int vi = v0 + AQR_THREADS * i + tid;
             if (vi >= nvec) continue;
+            float f[EPV];
 #pragma unroll
             for (int j = 0; j < EPV; ++j) {
                 const u32 b = aq_bits<BF16>(c[i], j);
                 amax = max(amax, b & 0x7fffffffu);
-                row[vi * EPV + j] = __uint_as_float(b);
+                f[j] = __uint_as_float(b);
             }
+#pragma unroll
+            for (int j = 0; j < EPV; j += 4)
+                reinterpret_cast<float4 *>(s_row)[(vi * EPV + j) >> 2] = make_float4(f[j], f[j + 1], f[j + 2], f[j + 3]);
         }
     }
-    amax = warp_max_u32(amax);
-    __syncwarp();
-    float r = 1.f;
+    amax = aqr_block_max(amax, s_u);  // also orders the row cache writes before the reads below
     if (g4 != nullptr) {
         // pass 2: exact sum of squares, 31-binade windows (normally one)
         u64 L[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
@@ -438,9 +453,9 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln_smem(const _
         for (int pass = 0; pass < 10; ++pass) {
             const int elo = ehi - 30 < 1 ? 1 : ehi - 30;
             u64 lo = 0ull, hi = 0ull;
-            bool below = false;
-            for (int k = lane; k < K; k += 32) {
-                const u32 u = __float_as_uint(row[k]) & 0x7fffffffu;
+            int below = 0;
+            for (int k = tid; k < K; k += AQR_THREADS) {
+                const u32 u = __float_as_uint(s_row[k]) & 0x7fffffffu;
                 const int e = (int)(u >> 23);
                 const int ee = e ? e : 1;
                 if (ee <= ehi && ee >= elo && u != 0u) {
@@ -453,39 +468,46 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln_smem(const _
                     hi += phi + (t < lo ? 1ull : 0ull);
                     lo = t;
                 } else if (ee < elo && u != 0u) {
-                    below = true;
+                    below = 1;
                 }
             }
-            warp_sum_u128(lo, hi);
-            if (lane == 0) limbs_add_u128_shl(L, lo, hi, 2 * (elo - 1));
-            if (!__any_sync(0xffffffffu, below) || elo == 1) break;
+            warp_sum_u128(lo, hi);  // < 2^108 per term, < 2^116 per thread, < 2^123 per CTA
+            if (lane == 0) {
+                s_lo[warp] = lo;
+                s_hi[warp] = hi;
+            }
+            const int any_below = __syncthreads_or(below);
+            if (tid == 0)
+                for (int w = 0; w < AQR_WARPS; ++w) limbs_add_u128_shl(L, s_lo[w], s_hi[w], 2 * (elo - 1));
+            if (!any_below || elo == 1) break;
             ehi = elo - 1;
+            __syncthreads();  // s_lo / s_hi read before the next window writes them
         }
-        if (lane == 0)
-            r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(limbs_to_double_rn(L, -298), (double)K)), P.eps));
-        r = __shfl_sync(0xffffffffu, r, 0);
+        if (tid == 0)
+            s_r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(limbs_to_double_rn(L, -298), (double)K)), P.eps));
+        __syncthreads();
+        const float r = s_r;
         // pass 3: y = float(float(x / r) * g) in place, max|y|
         amax = 0;
-        for (int q = lane; q < K / 4; q += 32) {
+        for (int q = tid; q < K / 4; q += AQR_THREADS) {
             const float4 g = __ldg(g4 + q);
-            float4 x = reinterpret_cast<float4 *>(row)[q];
+            float4 x = reinterpret_cast<float4 *>(s_row)[q];
             x.x = __fmul_rn(__fdiv_rn(x.x, r), g.x);
             x.y = __fmul_rn(__fdiv_rn(x.y, r), g.y);
             x.z = __fmul_rn(__fdiv_rn(x.z, r), g.z);
             x.w = __fmul_rn(__fdiv_rn(x.w, r), g.w);
-            reinterpret_cast<float4 *>(row)[q] = x;
+            reinterpret_cast<float4 *>(s_row)[q] = x;
             amax = max(amax, max(max(__float_as_uint(x.x) & 0x7fffffffu, __float_as_uint(x.y) & 0x7fffffffu),
                                  max(__float_as_uint(x.z) & 0x7fffffffu, __float_as_uint(x.w) & 0x7fffffffu)));
         }
-        amax = warp_max_u32(amax);
-        __syncwarp();
+        amax = aqr_block_max(amax, s_u);  // each thread quantizes the elements it wrote: no further barrier
     }
     const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(amax), 1e-5f));
-    if (lane == 0) pr.s[m] = s;
+    if (tid == 0) pr.s[m] = s;
     // pass 4: quantize, four elements -> one 32-bit word
     u32 *qr = reinterpret_cast<u32 *>(pr.xq + (size_t)m * K);
-    for (int q = lane; q < K / 4; q += 32) {
-        const float4 y = reinterpret_cast<const float4 *>(row)[q];
+    for (int q = tid; q < K / 4; q += AQR_THREADS) {
+        const float4 y = reinterpret_cast<const float4 *>(s_row)[q];
         const float yy[4] = {y.x, y.y, y.z, y.w};
         u32 w = 0;
 #pragma unroll

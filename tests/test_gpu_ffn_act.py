@@ -26,7 +26,7 @@ def _check(gate, up, gain, x_q, s, eps=1e-6):
 
 @pytest.mark.parametrize("M,F,subln", [
     (1, 4096, True), (7, 1536, False), (300, 4096, True), (33, 64, False), (5, 9728, True), (2, 32768, False),
-    (64, 2048, False), (3, 8640, True),
+    (64, 2048, False), (3, 8640, True), (2, 32768, True),
 ])
 def test_ffn_act_quant_matches_oracle(M, F, subln):
     gate = workloads.normal((M, F), 2.0, 40 + F)

@@ -108,6 +108,8 @@ def _wide_rows(M, K, seed):
     (4, 9728, torch.float32, True, "normal"),
     (6, 1024, torch.float32, True, "wide"),
     (7, 9728, torch.bfloat16, True, "student"),
+    (6, 4096, torch.float32, True, "wide"),
+    (3, 2560, torch.bfloat16, True, "wide"),
 ])
 def test_quant_act(M, K, dtype, subln, kind):
     if kind == "outlier":
