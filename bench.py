@@ -22,6 +22,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -108,7 +109,8 @@ class Clocks:
             if vis:
                 self.index = vis.split(",")[index]
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{index}.csv")
+        # the raw samples go to $BL_CLOCKS_DIR (default: the temp directory)
+        self.path = os.path.join(os.environ.get("BL_CLOCKS_DIR") or tempfile.gettempdir(), f"clocks_rank{index}.csv")
 
     def __enter__(self):
         os.makedirs(os.path.dirname(self.path), exist_ok=True)
