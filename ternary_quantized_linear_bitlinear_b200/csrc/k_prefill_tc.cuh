@@ -60,8 +60,8 @@ constexpr int PF_BM = 128;          // tokens per CTA (MMA M = 2 x 128, TMEM lan
 constexpr int PF_BN = 256;          // weight rows per pair tile (MMA N, TMEM columns)
 constexpr int PF_BNH = PF_BN / 2;   // weight rows expanded per CTA
 constexpr int PF_BK = 128;          // k per pipeline stage (4 MMAs of K = 32)
-constexpr int PF_STAGES = 6;        // TMA stages (x_q + packed)
-constexpr int PF_BSTAGES = 4;       // expanded-weight stages
+constexpr int PF_STAGES = 8;        // TMA stages (x_q + packed)
+constexpr int PF_BSTAGES = 2;       // expanded-weight stages (8 + 2 measured best of 5+5, 6+4, 7+3, 8+2)
 constexpr int PF_EXP_WARPS = PF_BNH / 32;
 constexpr int PF_EPI_WARPS = 8;
 constexpr int PF_EPI_WARP0 = 2 + PF_EXP_WARPS;
