@@ -559,6 +559,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
 
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -591,10 +592,11 @@ inline cudaError_t prefill_setup() {
 // Cluster pairs that can be resident at once on the current device (the
 // persistent grid never exceeds it, so every pair runs in the first wave).
 inline int prefill_max_pairs(int sms) {
-    static int cache[64];
+    static std::atomic<int> cache[64];  // per device; 0 = not queried yet (a race only repeats the query)
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sms / 2;
-    if (cache[dev] > 0) return cache[dev];
+    const int known = cache[dev].load(std::memory_order_relaxed);
+    if (known > 0) return known;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * (sms / 2)));
     cfg.blockDim = dim3(PF_THREADS);
@@ -605,7 +607,7 @@ inline int prefill_max_pairs(int sms) {
         n = sms / 2;
     }
     if (n > sms / 2) n = sms / 2;
-    cache[dev] = n;
+    cache[dev].store(n, std::memory_order_relaxed);
     return n;
 }
 
