@@ -66,11 +66,6 @@ bl_status device_info(DeviceInfo **out) {
 
 inline bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
-inline bl_status launch_status() {
-    cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
-}
-
 bl_status check_k(int64_t K) {
     if (K < 64 || K > K_MAX || (K % 64) != 0) return BL_ERR_SHAPE;
     return BL_OK;
