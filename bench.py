@@ -41,6 +41,13 @@ SPAD = {M: (M + 3) // 4 * 4 for M in MS}
 WORKLOAD = "decode125m: 12 layers x {q,o 768x768; k,v 256x768; gate,up 2048x768; down 768x2048}, M in {1,4,8}"
 
 
+def replica_of(step: int, j: int, replicas: int) -> int:
+    """Weight replica read by launch j (the j-th M) of a step: consecutive
+    launches never share weights (the launches of one step included), so no
+    launch is fed from L2; a replica comes back every `replicas` launches."""
+    return (len(MS) * step + j) % replicas
+
+
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -49,6 +56,8 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--ref-budget-s", type=float, default=90.0,
+                    help="reference arm: seconds of oracle work over the whole run")
     ap.add_argument("--mode", default="all", choices=["all", "decode", "prefill"],
                     help="decode: the headline decode workload only; prefill: only the prefill measurement")
     return ap.parse_args()
@@ -256,9 +265,7 @@ def native(args, rank, world, local):
     RDY = api.BL_FWD_WEIGHTS_READY
 
     def replica(step, j):
-        """Replica read by launch j of a step: consecutive launches never share
-        weights (the launches of one step included), so none is fed from L2."""
-        return (len(MS) * step + j) % R
+        return replica_of(step, j, R)
 
     def launch_step(stream_ptr, rep):
         """One step: per M, ONE fused launch (act quant + GEMV + rescale, 84 problems)."""
@@ -623,7 +630,7 @@ def reference(args, rank, world):
     items = oracle_items()
     jobs = [(M, i) for M in MS for i in range(len(items))]
     total_steps = args.steps + max(3, args.warmup)
-    budget_s = 90.0 / max(1, total_steps)
+    budget_s = args.ref_budget_s / max(1, total_steps)
     # calibrate the oracle's rows-per-second on one projection (not timed)
     wq, g, X = items[4]
     t0 = time.perf_counter()
