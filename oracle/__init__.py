@@ -54,6 +54,8 @@ def _lib():
             "oracle_contract": (None, [_ptr, _ptr, _i64, _i64, _i64, _ptr]),
             "oracle_contract_pairs": (None, [_ptr, _ptr, _i64, _ptr, _ptr, _i64, _ptr]),
             "oracle_rescale": (None, [_ptr, _i64, _f32, _ptr, _ptr]),
+            "oracle_bwd_dx": (None, [_ptr, _ptr, _f32, _i64, _i64, _i64, _ptr]),
+            "oracle_bwd_dw": (ctypes.c_int, [_ptr, _ptr, _ptr, _ptr, _f32, ctypes.c_double, _i64, _i64, _i64, _ptr]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -222,6 +224,40 @@ def linear(W, X, gain=None, eps: float = 1e-6):
     acc = contract(xq, wq)
     Y = rescale(acc, gamma, s[:, None])
     return dict(packed=packed, gamma=gamma, wq=wq, xq=xq, s=s, acc=acc, Y=Y)
+
+
+# -- backward under the straight-through estimator (next step of the path) --
+
+def bwd_dx(dY, wq: np.ndarray, gamma) -> np.ndarray:
+    """dX [M, K] float64 = dY @ (gamma W_q): the activation quantizer passed
+    straight through ("BitDistill", Evaluation and results)."""
+    dY = _f32c(dY)
+    wq = np.ascontiguousarray(wq, dtype=np.int8)
+    M, N = dY.shape
+    if wq.shape[0] != N:
+        raise OracleError("bwd_dx: dY and W_q disagree on N")
+    K = wq.shape[1]
+    dX = np.zeros((M, K), dtype=np.float64)
+    _lib().oracle_bwd_dx(_p(dY), _p(wq), np.float32(gamma), M, N, K, _p(dX))
+    return dX
+
+
+def bwd_dw(dY, xq: np.ndarray, s, W, gamma, beta: float = 0.0) -> np.ndarray:
+    """dW [N, K] float64 = (dY^T @ (x_q / s)) * scale(W / gamma), scale the
+    hard STE mask (beta <= 0) or the soft 1 - tanh^2(beta W / gamma) ("bitone"
+    README, Soft-STE notes)."""
+    dY = _f32c(dY)
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    s = _f32c(s).ravel()
+    W = _f32c(W)
+    M, N = dY.shape
+    K = xq.shape[1]
+    if xq.shape[0] != M or s.size != M or W.shape != (N, K):
+        raise OracleError("bwd_dw: shapes disagree")
+    dW = np.zeros((N, K), dtype=np.float64)
+    _check(_lib().oracle_bwd_dw(_p(dY), _p(xq), _p(s), _p(W), np.float32(gamma), float(beta), M, N, K, _p(dW)),
+           "bwd_dw")
+    return dW
 
 
 def num_threads() -> int:

@@ -1,5 +1,6 @@
 /*
- * BitLinear (BitNet b1.58) forward -- plain CPU oracle.
+ * BitLinear (BitNet b1.58) forward, and its straight-through backward (at
+ * the end of this file) -- plain CPU oracle.
  *
  * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the
  * benchmark's CPU-baseline leg may load this library.  The product path never
@@ -353,4 +354,61 @@ void oracle_rescale(const int64_t *acc, int64_t count, float gamma, const float 
                     double *Y) {
     for (int64_t i = 0; i < count; ++i)
         Y[i] = (double)acc[i] * (double)gamma / (double)s_per_item[i];
+}
+
+/* ------------------------------------------------------------------------
+ * Backward of the quantization-aware BitLinear (straight-through estimator).
+ *
+ * The pages fix only the rule: gradients pass through the quantizers
+ * unchanged ("Distillix" README, 1. BitNet b1.58 Core: "STE"; "BitDistill",
+ * Evaluation and results: gradients through the activation quantizer use the
+ * straight-through estimator), the weight gradient optionally masked by the
+ * hard or the soft STE scale of "bitone" README, Soft-STE notes:
+ *   hard:  scale = 1 if |w / gamma| <= 1, else 0
+ *   soft:  scale = 1 - tanh^2(beta * w / gamma)        (beta = 2 by default)
+ * Readings (the plainest ones; listed in the design notes):
+ *   - the forward is Y = (x_q / s) @ (gamma W_q)^T, so with both quantizers
+ *     passed straight through, dX = dY @ (gamma W_q) and the weight receives
+ *     dW = (dY^T @ (x_q / s)) * scale(W / gamma); gamma's own dependence on W
+ *     is not differentiated (it is part of the quantizer);
+ *   - w / gamma is the float division of the forward (the mask is an integer
+ *     decision, taken in the forward's precision); everything else is double.
+ * ------------------------------------------------------------------------ */
+
+/* dX [M, K] = dY [M, N] @ (gamma * W_q) [N, K], in double, n ascending. */
+void oracle_bwd_dx(const float *dY, const int8_t *wq, float gamma, int64_t M, int64_t N, int64_t K,
+                   double *dX) {
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) {
+            double a = 0.0;
+            for (int64_t n = 0; n < N; ++n)
+                a += (double)dY[m * N + n] * (double)wq[n * K + k];
+            dX[m * K + k] = a * (double)gamma;
+        }
+}
+
+/* STE scale of one latent weight: beta <= 0 selects the hard mask. */
+static double ste_scale(float w, float gamma, double beta) {
+    const float ws = w / gamma; /* float division, as in the forward */
+    if (beta <= 0.0) return fabsf(ws) <= 1.0f ? 1.0 : 0.0;
+    const double t = tanh(beta * (double)ws);
+    return 1.0 - t * t;
+}
+
+/* dW [N, K] = (dY^T @ (x_q / s)) * scale(W / gamma), in double, m ascending. */
+int oracle_bwd_dw(const float *dY, const int8_t *xq, const float *s, const float *W, float gamma,
+                  double beta, int64_t M, int64_t N, int64_t K, double *dW) {
+    if (!(gamma > 0.0f)) return OR_ERR_SHAPE;
+    for (int64_t m = 0; m < M; ++m)
+        if (!(s[m] > 0.0f)) return OR_ERR_SHAPE;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            double a = 0.0;
+            for (int64_t m = 0; m < M; ++m)
+                a += (double)dY[m * N + n] * ((double)xq[m * K + k] / (double)s[m]);
+            dW[n * K + k] = a * ste_scale(W[n * K + k], gamma, beta);
+        }
+    return OR_OK;
 }
