@@ -1,4 +1,5 @@
-"""CPU oracle for the BitLinear (BitNet b1.58) forward -- TEST INFRASTRUCTURE.
+"""CPU oracle for the BitLinear (BitNet b1.58) forward and its
+straight-through backward -- TEST INFRASTRUCTURE.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
 ``bench.py`` may import this package.  It never touches the CUDA library and
