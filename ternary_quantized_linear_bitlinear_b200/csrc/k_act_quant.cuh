@@ -487,15 +487,33 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
             s_r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(limbs_to_double_rn(L, -298), (double)K)), P.eps));
         __syncthreads();
         const float r = s_r;
-        // pass 3: y = float(float(x / r) * g) in place, max|y|
+        // pass 3: y = float(float(x / r) * g) in place, max|y|.  For the gated
+        // FFN input, x / r is correctly rounded by Markstein's method from the
+        // correctly rounded reciprocal of the row constant r (q0 = x * (1/r),
+        // remainder by FMA, one correction FMA), exact for normal dividends
+        // and normal quotients (checked against IEEE division for every
+        // dividend mantissa and 2016 divisors).  A nonzero subnormal dividend
+        // (its remainder is not exact) or an r that is not a finite normal
+        // number takes the IEEE division; a subnormal quotient cannot change
+        // x_q or s (y * s rounds to 0 and s is floored at 127 / 1e-5).
+        // Measured 172 -> 136 us for [8192, 4096]; bf16 rows were 1-2 %
+        // slower with it, so they keep the IEEE division.
+        const float ry = __frcp_rn(r);
+        const bool mk = GLU && __float_as_uint(r) >= 0x00800000u && __float_as_uint(r) < 0x7f800000u;
+        auto div_r = [&](float x) {
+            const u32 ax = __float_as_uint(x) & 0x7fffffffu;
+            if (!mk || (ax != 0u && ax < 0x00800000u)) return __fdiv_rn(x, r);
+            const float q0 = __fmul_rn(x, ry);
+            return __fmaf_rn(__fmaf_rn(-q0, r, x), ry, q0);
+        };
         amax = 0;
         for (int q = tid; q < K / 4; q += AQR_THREADS) {
             const float4 g = __ldg(g4 + q);
             float4 x = reinterpret_cast<float4 *>(s_row)[q];
-            x.x = __fmul_rn(__fdiv_rn(x.x, r), g.x);
-            x.y = __fmul_rn(__fdiv_rn(x.y, r), g.y);
-            x.z = __fmul_rn(__fdiv_rn(x.z, r), g.z);
-            x.w = __fmul_rn(__fdiv_rn(x.w, r), g.w);
+            x.x = __fmul_rn(div_r(x.x), g.x);
+            x.y = __fmul_rn(div_r(x.y), g.y);
+            x.z = __fmul_rn(div_r(x.z), g.z);
+            x.w = __fmul_rn(div_r(x.w), g.w);
             reinterpret_cast<float4 *>(s_row)[q] = x;
             amax = max(amax, max(max(__float_as_uint(x.x) & 0x7fffffffu, __float_as_uint(x.y) & 0x7fffffffu),
                                  max(__float_as_uint(x.z) & 0x7fffffffu, __float_as_uint(x.w) & 0x7fffffffu)));
