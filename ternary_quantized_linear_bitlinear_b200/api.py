@@ -114,14 +114,29 @@ def _ptr(t):
     return None if t is None else t.data_ptr()
 
 
-def _dev(t: torch.Tensor, name: str, dtype=None):
-    if not t.is_cuda:
+def _is_cuda(t: torch.Tensor) -> bool:
+    return t.is_cuda
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None, min_numel: int = 0):
+    """A device buffer the library reads or writes: CUDA, contiguous, of the
+    given dtype and at least min_numel elements (so that no kernel touches
+    host memory or runs past the end of a caller's buffer)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not _is_cuda(t):
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs at least {min_numel}")
     return t
+
+
+def _opt(t, name: str, dtype=None, min_numel: int = 0):
+    return None if t is None else _dev(t, name, dtype, min_numel)
 
 
 # -- workspace queries ---------------------------------------------------------
@@ -146,6 +161,9 @@ def bl_quant_weights(W: torch.Tensor, packed=None, gamma=None, workspace=None, s
         gamma = torch.empty(4, dtype=torch.float32, device=W.device)[:1]
     if workspace is None:
         workspace = torch.empty(quant_weights_workspace_bytes(N, K), dtype=torch.uint8, device=W.device)
+    _dev(packed, "packed", torch.uint8, N * K // 4)
+    _dev(gamma, "gamma", torch.float32, 1)
+    _dev(workspace, "workspace", torch.uint8)
     rc = lib().bl_quant_weights(W.data_ptr(), _DTYPES.get(W.dtype, -1), N, K, packed.data_ptr(), gamma.data_ptr(),
                                 workspace.data_ptr(), workspace.numel(), _stream(stream))
     _check(rc, "bl_quant_weights")
@@ -163,6 +181,8 @@ def bl_quant_weights_noalloc(W: torch.Tensor, packed=None, gamma=None, stream=No
         packed = torch.empty(N, K // 4, dtype=torch.uint8, device=W.device)
     if gamma is None:
         gamma = torch.empty(4, dtype=torch.float32, device=W.device)[:1]
+    _dev(packed, "packed", torch.uint8, N * K // 4)
+    _dev(gamma, "gamma", torch.float32, 1)
     rc = lib().bl_quant_weights_noalloc(W.data_ptr(), _DTYPES.get(W.dtype, -1), N, K, packed.data_ptr(),
                                         gamma.data_ptr(), _stream(stream))
     _check(rc, "bl_quant_weights_noalloc")
@@ -179,8 +199,9 @@ def bl_quant_act(X: torch.Tensor, subln_gain=None, subln_eps: float = 1e-6, x_q=
         x_q = torch.empty(M, K, dtype=torch.int8, device=X.device)
     if s is None:
         s = torch.empty(M, dtype=torch.float32, device=X.device)
-    if subln_gain is not None:
-        _dev(subln_gain, "subln_gain", torch.float32)
+    _dev(x_q, "x_q", torch.int8, M * K)
+    _dev(s, "s", torch.float32, M)
+    _opt(subln_gain, "subln_gain", torch.float32, K)
     rc = lib().bl_quant_act(X.data_ptr(), _DTYPES.get(X.dtype, -1), M, K, _ptr(subln_gain), subln_eps,
                             x_q.data_ptr(), s.data_ptr(), _stream(stream))
     _check(rc, "bl_quant_act")
@@ -192,6 +213,10 @@ def bl_quant_act_grouped(items, dtype=torch.bfloat16, subln_eps: float = 1e-6, s
     arr = (ActProblem * len(items))()
     M = items[0][0].shape[0]
     for i, (X, gain, xq, s) in enumerate(items):
+        _dev(X, f"items[{i}].X", dtype, M * X.shape[1])
+        _opt(gain, f"items[{i}].gain", torch.float32, X.shape[1])
+        _dev(xq, f"items[{i}].x_q", torch.int8, M * X.shape[1])
+        _dev(s, f"items[{i}].s", torch.float32, M)
         arr[i] = ActProblem(X.data_ptr(), _ptr(gain), xq.data_ptr(), s.data_ptr(), X.shape[1])
     rc = lib().bl_quant_act_grouped(arr, len(items), _DTYPES.get(dtype, -1), M, subln_eps, _stream(stream))
     _check(rc, "bl_quant_act_grouped")
@@ -212,6 +237,9 @@ def bl_ffn_act_quant(gate: torch.Tensor, up: torch.Tensor, subln_gain=None, subl
         x_q = torch.empty(M, F, dtype=torch.int8, device=gate.device)
     if s is None:
         s = torch.empty(max(M, 4), dtype=torch.float32, device=gate.device)[:M]
+    _dev(x_q, "x_q", torch.int8, M * F)
+    _dev(s, "s", torch.float32, M)
+    _opt(subln_gain, "subln_gain", torch.float32, F)
     rc = lib().bl_ffn_act_quant(gate.data_ptr(), up.data_ptr(), M, F, _ptr(subln_gain), subln_eps, x_q.data_ptr(),
                                 s.data_ptr(), _stream(stream))
     _check(rc, "bl_ffn_act_quant")
@@ -220,19 +248,31 @@ def bl_ffn_act_quant(gate: torch.Tensor, up: torch.Tensor, subln_gain=None, subl
 
 def bl_forward(packed, gamma, x_q, s, N: int, Y=None, acc_out=None, stream=None):
     """-> Y float32 [M, N] (acc_out int32 [M, N] filled when given)."""
+    _dev(x_q, "x_q", torch.int8)
     M, K = x_q.shape
     if Y is None:
         Y = torch.empty(M, N, dtype=torch.float32, device=x_q.device)
+    _check_forward_args(packed, gamma, s, Y, acc_out, M, N, K)
     rc = lib().bl_forward(packed.data_ptr(), gamma.data_ptr(), x_q.data_ptr(), s.data_ptr(), M, N, K, Y.data_ptr(),
                           _ptr(acc_out), _stream(stream))
     _check(rc, "bl_forward")
     return Y
 
 
+def _check_forward_args(packed, gamma, s, Y, acc_out, M, N, K):
+    _dev(packed, "packed", torch.uint8, N * K // 4)
+    _dev(gamma, "gamma", torch.float32, 1)
+    _dev(s, "s", torch.float32, M)
+    _dev(Y, "Y", torch.float32, M * N)
+    _opt(acc_out, "acc_out", torch.int32, M * N)
+
+
 def make_problems(items):
     """items: list of (packed, gamma, x_q, s, Y, acc_out or None, N, K) -> ctypes array."""
     arr = (Problem * len(items))()
     for i, (packed, gamma, xq, s, Y, acc, N, K) in enumerate(items):
+        for nm, t in (("packed", packed), ("gamma", gamma), ("x_q", xq), ("s", s), ("Y", Y), ("acc_out", acc)):
+            _opt(t, f"items[{i}].{nm}")
         arr[i] = Problem(packed.data_ptr(), gamma.data_ptr(), xq.data_ptr(), s.data_ptr(), Y.data_ptr(),
                          _ptr(acc), N, K)
     return arr
@@ -249,6 +289,9 @@ def make_decode_problems(items):
     -> ctypes array for bl_linear_decode_grouped."""
     arr = (DecodeProblem * len(items))()
     for i, (packed, gamma, X, gain, Y, xq, s, acc, N, K) in enumerate(items):
+        for nm, t in (("packed", packed), ("gamma", gamma), ("X", X), ("subln_gain", gain), ("Y", Y), ("x_q", xq),
+                      ("s", s), ("acc_out", acc)):
+            _opt(t, f"items[{i}].{nm}")
         arr[i] = DecodeProblem(packed.data_ptr(), gamma.data_ptr(), X.data_ptr(), _ptr(gain), Y.data_ptr(), _ptr(xq),
                                _ptr(s), _ptr(acc), N, K)
     return arr
@@ -273,6 +316,9 @@ def bl_linear(W, X, subln_gain=None, subln_eps: float = 1e-6, Y=None, workspace=
         Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
     if workspace is None:
         workspace = torch.empty(linear_workspace_bytes(M, N, K), dtype=torch.uint8, device=X.device)
+    _dev(Y, "Y", torch.float32, M * N)
+    _dev(workspace, "workspace", torch.uint8)
+    _opt(subln_gain, "subln_gain", torch.float32, K)
     rc = lib().bl_linear(W.data_ptr(), _DTYPES.get(W.dtype, -1), X.data_ptr(), _DTYPES.get(X.dtype, -1), M, N, K,
                          _ptr(subln_gain), subln_eps, workspace.data_ptr(), workspace.numel(), Y.data_ptr(),
                          _stream(stream))
@@ -285,9 +331,11 @@ def bl_debug_forward_prefill(packed, gamma, x_q, s, N: int, Y=None, acc_out=None
     """Test hook (include/bitlinear_debug.h): bl_forward forced through the
     tcgen05 prefill engine, with bounded waits of timeout_us and an optional
     stalled k-iteration."""
+    _dev(x_q, "x_q", torch.int8)
     M, K = x_q.shape
     if Y is None:
         Y = torch.empty(M, N, dtype=torch.float32, device=x_q.device)
+    _check_forward_args(packed, gamma, s, Y, acc_out, M, N, K)
     rc = lib().bl_debug_forward_prefill(packed.data_ptr(), gamma.data_ptr(), x_q.data_ptr(), s.data_ptr(), M, N, K,
                                         Y.data_ptr(), _ptr(acc_out), skip_iter, timeout_us, _stream(stream))
     _check(rc, "bl_debug_forward_prefill")
