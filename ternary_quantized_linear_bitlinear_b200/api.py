@@ -1,7 +1,8 @@
 """Python binding of libbitlinear.so (include/bitlinear.h).
 
 Argument marshalling only: every function here checks that torch tensors are
-CUDA, contiguous and of the right dtype, allocates outputs with torch when
+CUDA tensors on the current device, contiguous, of the right dtype and large
+enough for the call, allocates outputs with torch when
 the caller passes none, and calls the C entry point of the same name with
 raw device pointers and the current torch stream.  All arithmetic runs in
 the library's kernels; if the library is missing, loading fails loudly.
@@ -105,9 +106,19 @@ def _check(status: int, where: str):
         raise BitLinearError(status, where)
 
 
+def _current_device() -> int:
+    return torch.cuda.current_device()
+
+
 def _stream(stream) -> int:
-    s = torch.cuda.current_stream() if stream is None else stream
-    return s.cuda_stream
+    """Raw handle of `stream` (default: torch's current stream).  The library
+    launches on the current device, so an explicit stream must belong to it."""
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if stream.device_index != _current_device():
+        raise ValueError(f"stream belongs to cuda:{stream.device_index}, the current device is "
+                         f"cuda:{_current_device()}")
+    return stream.cuda_stream
 
 
 def _ptr(t):
@@ -118,14 +129,22 @@ def _is_cuda(t: torch.Tensor) -> bool:
     return t.is_cuda
 
 
+def _device_index(t: torch.Tensor) -> int:
+    return t.device.index
+
+
 def _dev(t: torch.Tensor, name: str, dtype=None, min_numel: int = 0):
-    """A device buffer the library reads or writes: CUDA, contiguous, of the
-    given dtype and at least min_numel elements (so that no kernel touches
-    host memory or runs past the end of a caller's buffer)."""
+    """A device buffer the library reads or writes: CUDA, on the current
+    device (the library launches there, so every buffer of a call lives on
+    one GPU), contiguous, of the given dtype and at least min_numel elements
+    (so that no kernel touches host memory, another GPU's memory, or runs
+    past the end of a caller's buffer)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not _is_cuda(t):
         raise ValueError(f"{name} must be a CUDA tensor")
+    if _device_index(t) != _current_device():
+        raise ValueError(f"{name} lives on cuda:{_device_index(t)}, the current device is cuda:{_current_device()}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
@@ -137,6 +156,22 @@ def _dev(t: torch.Tensor, name: str, dtype=None, min_numel: int = 0):
 
 def _opt(t, name: str, dtype=None, min_numel: int = 0):
     return None if t is None else _dev(t, name, dtype, min_numel)
+
+
+def _mat(t: torch.Tensor, name: str, cols: int | None = None, rows: int | None = None):
+    """A 2-D float32 or bfloat16 input matrix ([N, K] weights or [M, K]
+    activations) on the current device, optionally with a fixed column
+    (and row) count -> (rows, cols)."""
+    _dev(t, name)
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D, got shape {tuple(t.shape)}")
+    if t.dtype not in _DTYPES:
+        raise ValueError(f"{name} must be float32 or bfloat16, got {t.dtype}")
+    if cols is not None and t.shape[1] != cols:
+        raise ValueError(f"{name} has {t.shape[1]} columns, expected {cols}")
+    if rows is not None and t.shape[0] != rows:
+        raise ValueError(f"{name} has {t.shape[0]} rows, expected {rows}")
+    return t.shape[0], t.shape[1]
 
 
 # -- workspace queries ---------------------------------------------------------
@@ -153,8 +188,7 @@ def linear_workspace_bytes(M: int, N: int, K: int) -> int:
 
 def bl_quant_weights(W: torch.Tensor, packed=None, gamma=None, workspace=None, stream=None):
     """-> (packed uint8 [N, K/4], gamma float32 [1])."""
-    _dev(W, "W")
-    N, K = W.shape
+    N, K = _mat(W, "W")
     if packed is None:
         packed = torch.empty(N, K // 4, dtype=torch.uint8, device=W.device)
     if gamma is None:
@@ -175,8 +209,7 @@ def bl_quant_weights_noalloc(W: torch.Tensor, packed=None, gamma=None, stream=No
     device scratch is used instead (for callers that cannot allocate device
     memory; see include/bitlinear.h).  Outputs are allocated here only when
     the caller passes none."""
-    _dev(W, "W")
-    N, K = W.shape
+    N, K = _mat(W, "W")
     if packed is None:
         packed = torch.empty(N, K // 4, dtype=torch.uint8, device=W.device)
     if gamma is None:
@@ -193,8 +226,7 @@ def bl_quant_weights_noalloc(W: torch.Tensor, packed=None, gamma=None, stream=No
 
 def bl_quant_act(X: torch.Tensor, subln_gain=None, subln_eps: float = 1e-6, x_q=None, s=None, stream=None):
     """-> (x_q int8 [M, K], s float32 [M])."""
-    _dev(X, "X")
-    M, K = X.shape
+    M, K = _mat(X, "X")
     if x_q is None:
         x_q = torch.empty(M, K, dtype=torch.int8, device=X.device)
     if s is None:
@@ -210,10 +242,13 @@ def bl_quant_act(X: torch.Tensor, subln_gain=None, subln_eps: float = 1e-6, x_q=
 
 def bl_quant_act_grouped(items, dtype=torch.bfloat16, subln_eps: float = 1e-6, stream=None):
     """items: list of (X [M, K], gain or None, x_q [M, K], s [M]), same M and dtype."""
+    if dtype not in _DTYPES:
+        raise ValueError(f"dtype must be float32 or bfloat16, got {dtype}")
     arr = (ActProblem * len(items))()
     M = items[0][0].shape[0]
     for i, (X, gain, xq, s) in enumerate(items):
-        _dev(X, f"items[{i}].X", dtype, M * X.shape[1])
+        _mat(X, f"items[{i}].X", rows=M)
+        _dev(X, f"items[{i}].X", dtype)
         _opt(gain, f"items[{i}].gain", torch.float32, X.shape[1])
         _dev(xq, f"items[{i}].x_q", torch.int8, M * X.shape[1])
         _dev(s, f"items[{i}].s", torch.float32, M)
@@ -230,8 +265,8 @@ def bl_ffn_act_quant(gate: torch.Tensor, up: torch.Tensor, subln_gain=None, subl
     of relu(gate)^2 * up, after SubLN when a gain is given."""
     _dev(gate, "gate", torch.float32)
     _dev(up, "up", torch.float32)
-    if gate.shape != up.shape:
-        raise ValueError("gate and up must have the same shape")
+    if gate.dim() != 2 or gate.shape != up.shape:
+        raise ValueError("gate and up must be 2-D [M, F] of the same shape")
     M, F = gate.shape
     if x_q is None:
         x_q = torch.empty(M, F, dtype=torch.int8, device=gate.device)
@@ -248,8 +283,7 @@ def bl_ffn_act_quant(gate: torch.Tensor, up: torch.Tensor, subln_gain=None, subl
 
 def bl_forward(packed, gamma, x_q, s, N: int, Y=None, acc_out=None, stream=None):
     """-> Y float32 [M, N] (acc_out int32 [M, N] filled when given)."""
-    _dev(x_q, "x_q", torch.int8)
-    M, K = x_q.shape
+    M, K = _xq2d(x_q)
     if Y is None:
         Y = torch.empty(M, N, dtype=torch.float32, device=x_q.device)
     _check_forward_args(packed, gamma, s, Y, acc_out, M, N, K)
@@ -257,6 +291,13 @@ def bl_forward(packed, gamma, x_q, s, N: int, Y=None, acc_out=None, stream=None)
                           _ptr(acc_out), _stream(stream))
     _check(rc, "bl_forward")
     return Y
+
+
+def _xq2d(x_q):
+    _dev(x_q, "x_q", torch.int8)
+    if x_q.dim() != 2:
+        raise ValueError(f"x_q must be 2-D [M, K], got shape {tuple(x_q.shape)}")
+    return x_q.shape[0], x_q.shape[1]
 
 
 def _check_forward_args(packed, gamma, s, Y, acc_out, M, N, K):
@@ -267,39 +308,90 @@ def _check_forward_args(packed, gamma, s, Y, acc_out, M, N, K):
     _opt(acc_out, "acc_out", torch.int32, M * N)
 
 
-def make_problems(items):
-    """items: list of (packed, gamma, x_q, s, Y, acc_out or None, N, K) -> ctypes array."""
+def _rows_of(t, name: str) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dim() != 2:
+        raise ValueError(f"{name} must be 2-D [M, K] when M is not given")
+    return t.shape[0]
+
+
+def make_problems(items, M: int | None = None):
+    """items: list of (packed, gamma, x_q, s, Y, acc_out or None, N, K) -> ctypes
+    array for bl_forward_grouped at token count M (default: the first x_q's
+    row count).  Every buffer is checked against N, K and M: packed uint8
+    >= N*K/4, gamma float32 >= 1, x_q int8 >= M*K, s float32 >= M, Y float32
+    and acc_out int32 >= M*N."""
+    if M is None:
+        M = _rows_of(items[0][2], "items[0].x_q")
     arr = (Problem * len(items))()
     for i, (packed, gamma, xq, s, Y, acc, N, K) in enumerate(items):
-        for nm, t in (("packed", packed), ("gamma", gamma), ("x_q", xq), ("s", s), ("Y", Y), ("acc_out", acc)):
-            _opt(t, f"items[{i}].{nm}")
+        _dev(packed, f"items[{i}].packed", torch.uint8, N * K // 4)
+        _dev(gamma, f"items[{i}].gamma", torch.float32, 1)
+        _dev(xq, f"items[{i}].x_q", torch.int8, M * K)
+        _dev(s, f"items[{i}].s", torch.float32, M)
+        _dev(Y, f"items[{i}].Y", torch.float32, M * N)
+        _opt(acc, f"items[{i}].acc_out", torch.int32, M * N)
         arr[i] = Problem(packed.data_ptr(), gamma.data_ptr(), xq.data_ptr(), s.data_ptr(), Y.data_ptr(),
                          _ptr(acc), N, K)
+    arr.bl_M = M
     return arr
+
+
+def _check_array(problems, count: int, M: int, dtype=None):
+    """A problem array built by make_problems / make_decode_problems was
+    validated for one M (and dtype): launching it with another, or with more
+    problems than it holds, would let a kernel run past a buffer."""
+    if count < 0 or count > len(problems):
+        raise ValueError(f"count {count} outside the {len(problems)} problems of the array")
+    checked_M = getattr(problems, "bl_M", None)
+    if checked_M is not None and M != checked_M:
+        raise ValueError(f"the problem array was checked for M = {checked_M}, called with M = {M}")
+    checked_dt = getattr(problems, "bl_dtype", None)
+    if dtype is not None and checked_dt is not None and dtype != checked_dt:
+        raise ValueError(f"the problem array was checked for X of {checked_dt}, called with {dtype}")
 
 
 def bl_forward_grouped(problems, count: int, M: int, flags: int = 0, stream=None):
     """problems: ctypes array from make_problems (built once, launched many times)."""
+    _check_array(problems, count, M)
     rc = lib().bl_forward_grouped(problems, count, M, flags, _stream(stream))
     _check(rc, "bl_forward_grouped")
 
 
-def make_decode_problems(items):
+def make_decode_problems(items, M: int | None = None):
     """items: list of (packed, gamma, X, subln_gain or None, Y, x_q or None, s or None, acc_out or None, N, K)
-    -> ctypes array for bl_linear_decode_grouped."""
+    -> ctypes array for bl_linear_decode_grouped at token count M (default:
+    the first X's row count).  Every X must have the first one's dtype
+    (float32 or bfloat16); every buffer is checked against N, K and M."""
+    if M is None:
+        M = _rows_of(items[0][2], "items[0].X")
+    dtype = items[0][2].dtype if isinstance(items[0][2], torch.Tensor) else None
+    if dtype not in _DTYPES:
+        raise ValueError(f"X must be float32 or bfloat16, got {dtype}")
     arr = (DecodeProblem * len(items))()
     for i, (packed, gamma, X, gain, Y, xq, s, acc, N, K) in enumerate(items):
-        for nm, t in (("packed", packed), ("gamma", gamma), ("X", X), ("subln_gain", gain), ("Y", Y), ("x_q", xq),
-                      ("s", s), ("acc_out", acc)):
-            _opt(t, f"items[{i}].{nm}")
+        _dev(packed, f"items[{i}].packed", torch.uint8, N * K // 4)
+        _dev(gamma, f"items[{i}].gamma", torch.float32, 1)
+        _dev(X, f"items[{i}].X", dtype, M * K)
+        _opt(gain, f"items[{i}].subln_gain", torch.float32, K)
+        _dev(Y, f"items[{i}].Y", torch.float32, M * N)
+        _opt(xq, f"items[{i}].x_q", torch.int8, M * K)
+        _opt(s, f"items[{i}].s", torch.float32, M)
+        _opt(acc, f"items[{i}].acc_out", torch.int32, M * N)
         arr[i] = DecodeProblem(packed.data_ptr(), gamma.data_ptr(), X.data_ptr(), _ptr(gain), Y.data_ptr(), _ptr(xq),
                                _ptr(s), _ptr(acc), N, K)
+    arr.bl_M = M
+    arr.bl_dtype = dtype
     return arr
 
 
 def bl_linear_decode_grouped(problems, count: int, M: int, dtype=torch.bfloat16, subln_eps: float = 1e-6,
                              flags: int = 0, stream=None):
     """Steps 2-4 fused: problems from make_decode_problems (X of `dtype`, same M)."""
+    if dtype not in _DTYPES:
+        raise ValueError(f"dtype must be float32 or bfloat16, got {dtype}")
+    _check_array(problems, count, M, dtype)
     rc = lib().bl_linear_decode_grouped(problems, count, _DTYPES[dtype], M, subln_eps, flags, _stream(stream))
     _check(rc, "bl_linear_decode_grouped")
 
@@ -308,10 +400,8 @@ def bl_linear_decode_grouped(problems, count: int, M: int, dtype=torch.bfloat16,
 
 def bl_linear(W, X, subln_gain=None, subln_eps: float = 1e-6, Y=None, workspace=None, stream=None):
     """-> Y float32 [M, N] = BitLinear(X) with weights W quantized in the call."""
-    _dev(W, "W")
-    _dev(X, "X")
-    N, K = W.shape
-    M = X.shape[0]
+    N, K = _mat(W, "W")
+    M, _ = _mat(X, "X", cols=K)
     if Y is None:
         Y = torch.empty(M, N, dtype=torch.float32, device=X.device)
     if workspace is None:
@@ -331,8 +421,7 @@ def bl_debug_forward_prefill(packed, gamma, x_q, s, N: int, Y=None, acc_out=None
     """Test hook (include/bitlinear_debug.h): bl_forward forced through the
     tcgen05 prefill engine, with bounded waits of timeout_us and an optional
     stalled k-iteration."""
-    _dev(x_q, "x_q", torch.int8)
-    M, K = x_q.shape
+    M, K = _xq2d(x_q)
     if Y is None:
         Y = torch.empty(M, N, dtype=torch.float32, device=x_q.device)
     _check_forward_args(packed, gamma, s, Y, acc_out, M, N, K)

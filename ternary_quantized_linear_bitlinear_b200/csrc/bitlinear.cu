@@ -71,6 +71,10 @@ bl_status check_k(int64_t K) {
     return BL_OK;
 }
 
+// N * K < 2^31 without forming the product (N may be anything up to
+// INT64_MAX; K has passed check_k, so 64 <= K <= K_MAX).
+bool nk_fits(int64_t N, int64_t K) { return N <= ((1LL << 31) - 1) / K; }
+
 // ---------------------------------------------------------------------------
 // Step 1
 
@@ -383,7 +387,7 @@ bl_status bl_quant_weights(const void *W, bl_dtype wdt, int64_t N, int64_t K, ui
                            void *workspace, size_t workspace_bytes, bl_stream_t stream) {
     if (!W || !packed || !gamma) return BL_ERR_NULL;
     if (wdt != BL_F32 && wdt != BL_BF16) return BL_ERR_DTYPE;
-    if (N < 1 || check_k(K) != BL_OK || N * K >= (1LL << 31)) return BL_ERR_SHAPE;
+    if (N < 1 || check_k(K) != BL_OK || !nk_fits(N, K)) return BL_ERR_SHAPE;
     if (!aligned16(W) || !aligned16(packed) || !aligned16(gamma)) return BL_ERR_ALIGN;
     if (!workspace || workspace_bytes < bl_quant_weights_workspace_bytes(N, K)) return BL_ERR_WORKSPACE;
     if (!aligned16(workspace)) return BL_ERR_ALIGN;
@@ -524,7 +528,7 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt, in
     if (!W || !X || !Y) return BL_ERR_NULL;
     if (wdt != BL_F32 && wdt != BL_BF16) return BL_ERR_DTYPE;
     if (xdt != BL_F32 && xdt != BL_BF16) return BL_ERR_DTYPE;
-    if (M < 1 || N < 1 || M > 0x7fffffffLL || check_k(K) != BL_OK || N * K >= (1LL << 31)) return BL_ERR_SHAPE;
+    if (M < 1 || N < 1 || M > 0x7fffffffLL || check_k(K) != BL_OK || !nk_fits(N, K)) return BL_ERR_SHAPE;
     if (!aligned16(W) || !aligned16(X) || !aligned16(Y) || (subln_gain && !aligned16(subln_gain)))
         return BL_ERR_ALIGN;
     if (!workspace || workspace_bytes < bl_linear_workspace_bytes(M, N, K)) return BL_ERR_WORKSPACE;
@@ -605,7 +609,7 @@ extern "C" bl_status bl_quant_weights_noalloc(const void *W, bl_dtype wdt, int64
                                               float *gamma, bl_stream_t stream) {
     if (!W || !packed || !gamma) return BL_ERR_NULL;
     if (wdt != BL_F32 && wdt != BL_BF16) return BL_ERR_DTYPE;
-    if (N < 1 || check_k(K) != BL_OK || N * K >= (1LL << 31)) return BL_ERR_SHAPE;
+    if (N < 1 || check_k(K) != BL_OK || !nk_fits(N, K)) return BL_ERR_SHAPE;
     if (!aligned16(W) || !aligned16(packed) || !aligned16(gamma)) return BL_ERR_ALIGN;
     DeviceInfo *d;
     bl_status rc = device_info(&d);

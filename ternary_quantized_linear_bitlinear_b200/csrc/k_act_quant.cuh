@@ -490,12 +490,17 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
         // pass 3: y = float(float(x / r) * g) in place, max|y|.  For the gated
         // FFN input, x / r is correctly rounded by Markstein's method from the
         // correctly rounded reciprocal of the row constant r (q0 = x * (1/r),
-        // remainder by FMA, one correction FMA), exact for normal dividends
-        // and normal quotients (checked against IEEE division for every
-        // dividend mantissa and 2016 divisors).  A nonzero subnormal dividend
-        // (its remainder is not exact) or an r that is not a finite normal
-        // number takes the IEEE division; a subnormal quotient cannot change
-        // x_q or s (y * s rounds to 0 and s is floored at 127 / 1e-5).
+        // remainder x - r * q0 by FMA, one correction FMA).  The method is
+        // exact whenever that remainder is representable, which holds for
+        // quotients well above 2^-126 * 2^24 (checked against IEEE division
+        // for every dividend mantissa and 2016 divisors); nearer underflow
+        // the remainder can need bits below 2^-149 and q1 may be one ulp off.
+        // A nonzero subnormal dividend or an r that is not a finite normal
+        // number takes the IEEE division.  The underflow band cannot change
+        // x_q or s: there |y| < 2^-100, so y * s (s <= 127 / 1e-5 < 2^24)
+        // rounds to 0 either way, and such a y is the row maximum only when
+        // every |y| of the row is below 1e-5, where s is floored at
+        // 127 / 1e-5 whatever the maximum is.
         // Measured 172 -> 136 us for [8192, 4096]; bf16 rows were 1-2 %
         // slower with it, so they keep the IEEE division.
         const float ry = __frcp_rn(r);

@@ -1,10 +1,13 @@
 /* Markstein's division from a correctly rounded reciprocal, against IEEE
  * float division: for b with y = RN(1/b),
  *     q0 = RN(x * y);  e = RN(x - b * q0) (one FMA, exact);  q1 = RN(q0 + e * y)
- * must equal RN(x / b) for normal dividends with normal quotients.  Checks
- * every dividend mantissa x in [1, 2) against nb divisors in [1, 2) and
- * [2, 4) (edge significands first, then a xorshift sequence); scaling by
- * powers of two carries the result to every normal exponent.  Prints the
+ * must equal RN(x / b) whenever the remainder x - b * q0 is representable.
+ * Checks every dividend mantissa x in [1, 2) against nb divisors in [1, 2)
+ * and [2, 4) (edge significands first, then a xorshift sequence); scaling
+ * by powers of two carries the result to every exponent at which the
+ * remainder stays representable, i.e. quotients well above 2^-126 * 2^24.
+ * Nearer underflow the remainder can need bits below 2^-149 (and a
+ * subnormal dividend never has an exact one: the second mode shows it).  Prints the
  * count of quotients and of mismatches.  Build: gcc -O2 -std=c11
  * -ffp-contract=off -fno-fast-math -fopenmp markstein_check.c -lm */
 #include <math.h>

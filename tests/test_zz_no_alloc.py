@@ -4,7 +4,7 @@ tensors it owns, a fixed device-memory budget).  It runs the same kernels as
 bl_quant_weights with the library's static device scratch instead of a
 caller workspace, so its packed weights and gamma must equal
 bl_quant_weights' bit for bit -- on two calls in a row, because the static
-scratch keeps the previous call's contents.
+scratch keeps the previous call's contents -- and the CPU oracle's.
 
 This file is collected last on purpose: it must pass alone in a fresh process
 and after every other test."""
@@ -13,6 +13,9 @@ from __future__ import annotations
 import pytest
 import torch
 
+import numpy as np
+
+import oracle
 from ternary_quantized_linear_bitlinear_b200 import api, workloads
 
 pytestmark = pytest.mark.gpu
@@ -31,6 +34,10 @@ def test_noalloc_matches_workspace_entry_point_twice():
             torch.cuda.synchronize()
             assert torch.equal(packed, ref_packed)
             assert gamma.view(torch.int32).item() == ref_gamma.view(torch.int32).item()
+        # and directly against the CPU oracle, so the check stands on its own
+        o_packed, o_gamma, _ = oracle.quant_weights(W_cpu.float().numpy())
+        assert np.array_equal(packed.cpu().numpy(), o_packed)
+        assert gamma.cpu().numpy().view(np.uint32)[0] == np.float32(o_gamma).view(np.uint32)
 
 
 def test_noalloc_rejects_oversize_on_host():
