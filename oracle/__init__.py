@@ -19,6 +19,8 @@ Parity status per function (what pins it, see tests/test_oracle_pins.py):
   rmsnorm         pinned: constant-row closed form, exact sum vs Fraction
   contract        pinned: add/subtract identity (bitone "How 1.58-bit Works"),
                   int64 matmul, brute force over all ternary rows for tiny K
+  contract_blas   pinned: equals contract (int64 loop) on ragged shapes and
+                  at the extreme |acc| = 128 K; rejects K beyond its bound
   rescale         pinned: closed form on hand values
 """
 from __future__ import annotations
@@ -57,6 +59,7 @@ def _lib():
             "oracle_rescale": (None, [_ptr, _i64, _f32, _ptr, _ptr]),
             "oracle_bwd_dx": (None, [_ptr, _ptr, _f32, _i64, _i64, _i64, _ptr]),
             "oracle_bwd_dw": (ctypes.c_int, [_ptr, _ptr, _ptr, _ptr, _f32, ctypes.c_double, _i64, _i64, _i64, _ptr]),
+            "oracle_set_num_threads": (None, [ctypes.c_int]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(lib, name)
@@ -199,6 +202,26 @@ def contract(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:
     return acc
 
 
+def contract_blas(xq: np.ndarray, wq: np.ndarray) -> np.ndarray:
+    """acc [M, N] int64 = x_q @ W_q^T, exact, through a library float32
+    matmul (numpy / BLAS): the same definition as ``contract`` with the
+    matmul as its one step, fast enough for the full-size workloads.
+
+    Exact because every product x_q * W_q is an integer in [-128, 128] and
+    every partial sum an integer of magnitude <= 128 * K < 2^24, so each
+    float32 addition (or fused multiply-add) is exact whatever order the
+    library sums in.  Refuses K >= 2^24 / 128."""
+    xq = np.ascontiguousarray(xq, dtype=np.int8)
+    wq = np.ascontiguousarray(wq, dtype=np.int8)
+    K = xq.shape[1]
+    if wq.shape[1] != K:
+        raise OracleError("contract_blas: x_q and W_q disagree on K")
+    if 128 * K >= (1 << 24):
+        raise OracleError("contract_blas: K too large for exact float32 sums")
+    acc = np.matmul(xq.astype(np.float32), wq.astype(np.float32).T)
+    return np.rint(acc).astype(np.int64)
+
+
 def contract_pairs(xq: np.ndarray, wq: np.ndarray, ms, ns) -> np.ndarray:
     xq = np.ascontiguousarray(xq, dtype=np.int8)
     wq = np.ascontiguousarray(wq, dtype=np.int8)
@@ -259,6 +282,12 @@ def bwd_dw(dY, xq: np.ndarray, s, W, gamma, beta: float = 0.0) -> np.ndarray:
     _check(_lib().oracle_bwd_dw(_p(dY), _p(xq), _p(s), _p(W), np.float32(gamma), float(beta), M, N, K, _p(dW)),
            "bwd_dw")
     return dW
+
+
+def set_num_threads(n: int) -> None:
+    """Threads the OpenMP loops use from now on (timing only: every output is
+    computed by one thread, in the same order, whatever the count)."""
+    _lib().oracle_set_num_threads(int(n))
 
 
 def num_threads() -> int:

@@ -53,6 +53,7 @@
  *        -fPIC oracle.c -o liboracle.so  (see build.py beside this file).
  */
 #include <math.h>
+#include <omp.h>
 #include <stdint.h>
 #include <string.h>
 
@@ -60,6 +61,10 @@
 #define OR_ERR_NONFINITE 1
 #define OR_ERR_SHAPE 2
 #define OR_ERR_RANGE 3
+
+/* Threads of the OpenMP loops below (a timing knob; results do not depend
+ * on it: each output is computed by one thread in a fixed order). */
+void oracle_set_num_threads(int n) { omp_set_num_threads(n > 0 ? n : 1); }
 
 /* ------------------------------------------------------------------------ */
 /* Exact big-integer helpers (little-endian uint64 limbs).                   */

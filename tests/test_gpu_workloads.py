@@ -1,8 +1,11 @@
-"""Full-size workloads on the GPU, checked against the oracle.
+"""Full-size workloads on the GPU, checked against the oracle element by
+element: every packed weight byte and gamma, every row of x_q and s, every
+int32 accumulator and every Y of each projection run (the accumulators from
+the oracle's exact contraction, its BLAS form at these sizes).
 
-Weights, gamma: every byte.  x_q, s: every row for decode, sampled rows for
-prefill.  acc and Y: every output for decode, 4096 sampled (m, n) pairs plus
-corners for prefill.
+Each projection runs twice through the contraction: once with the int32
+accumulators requested (plain stores in the prefill epilogue) and once
+without (Y by TMA tensor stores); both Y must carry the same bits.
 """
 from __future__ import annotations
 
@@ -10,33 +13,40 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from ternary_quantized_linear_bitlinear_b200 import api, workloads
-from _parity import check_act, check_forward_full, check_forward_sampled, check_weights, np32
+from _parity import check_act, check_weights, check_y
 
 pytestmark = pytest.mark.gpu
 
 
-def run_projection(W, X, gain=None, full=False, sample_rows=256, seed=0):
+def check_acc_full(acc_got: torch.Tensor, acc_ref: np.ndarray):
+    got = acc_got.cpu().numpy()
+    if not np.array_equal(got, acc_ref):
+        bad = np.argwhere(got != acc_ref)
+        raise AssertionError(f"acc mismatch at {len(bad)} of {acc_ref.size} entries, first {bad[:5].tolist()}")
+
+
+def run_projection(W, X, gain=None):
     Wd, Xd = W.cuda(), X.cuda()
     packed, gamma = api.bl_quant_weights(Wd)
     x_q, s = api.bl_quant_act(Xd, None if gain is None else gain.cuda(), workloads.SUBLN_EPS)
     M, N = X.shape[0], W.shape[0]
     acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
     Y = api.bl_forward(packed, gamma, x_q, s, N, acc_out=acc)
+    Y2 = api.bl_forward(packed, gamma, x_q, s, N)
     api.bl_check_device_error()
+    assert torch.equal(Y.view(torch.int32), Y2.view(torch.int32)), "Y differs between the two store paths"
+    del Y2
     wq_ref, g_ref = check_weights(W, packed, gamma)
-    if full:
-        xq_ref, s_ref = check_act(X, x_q, s, gain)
-        check_forward_full(xq_ref, s_ref, wq_ref, g_ref, Y, acc)
-    else:
-        rng = np.random.default_rng(seed)
-        rows = np.unique(np.concatenate([rng.integers(0, M, sample_rows), [0, M - 1]]))
-        xq_ref, s_ref = check_act(X, x_q, s, gain, rows=rows)
-        check_forward_sampled(xq_ref, s_ref, wq_ref, g_ref, Y, acc, xq_rows=rows, seed=seed)
+    xq_ref, s_ref = check_act(X, x_q, s, gain)
+    acc_ref = oracle.contract_blas(xq_ref, wq_ref)
+    check_acc_full(acc, acc_ref)
+    check_y(Y.cpu().numpy(), acc_ref, g_ref, s_ref[:, None])
     return Y
 
 
-@pytest.mark.parametrize("which", ["q", "k", "o", "gate", "down"])
+@pytest.mark.parametrize("which", ["q", "k", "v", "o", "gate", "up", "down"])
 def test_prefill1b4_layer(which):
     name, W, X = workloads.prefill1b4(which=(which,))[0]
     run_projection(W, X)
@@ -45,7 +55,7 @@ def test_prefill1b4_layer(which):
 @pytest.mark.parametrize("M", [1, 2048])
 def test_layer3b(M):
     for name, W, X in workloads.layer3b(M=M):
-        run_projection(W, X, full=(M == 1))
+        run_projection(W, X)
 
 
 @pytest.mark.parametrize("which", ["o", "gate", "down"])
@@ -59,6 +69,15 @@ def test_qat4b_layer(which):
     assert torch.equal(Yl.view(torch.int32), Y.view(torch.int32))
 
 
+def test_prefill_every_pair_runs_several_tiles():
+    """M = 4096, N = 4096, K = 768: 16 x 16 = 256 output tiles of 256 x 256 on
+    at most 74 CTA pairs, so every pair runs 3 or 4 tiles: both TMEM
+    accumulator buffers and their phase flips are used, every output checked."""
+    W = workloads.normal((4096, 768), 0.02, 501)
+    X = workloads.with_outlier_channels(workloads.normal((4096, 768), 1.0, 502, torch.bfloat16), 8, 20.0, 503)
+    run_projection(W, X)
+
+
 def test_single_workload_full():
     W, X = workloads.single()
-    run_projection(W, X, full=True)
+    run_projection(W, X)

@@ -328,6 +328,38 @@ def test_contraction_brute_force_tiny():
             assert acc[m, n] == s
 
 
+def test_contract_blas_equals_the_integer_loop():
+    """The BLAS form of the contraction (float32 matmul, exact below 2^24)
+    against the int64 loop and the add/subtract identity, on ragged
+    non-square shapes (a transposed operand or a dropped column fails)."""
+    rng = np.random.default_rng(7)
+    for M, N, K in ((37, 53, 448), (1, 5, 64), (9, 300, 2048)):
+        xq = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
+        wq = rng.integers(-1, 2, size=(N, K)).astype(np.int8)
+        got = oracle.contract_blas(xq, wq)
+        assert got.shape == (M, N) and got.dtype == np.int64
+        assert np.array_equal(got, oracle.contract(xq, wq))
+    x64 = xq.astype(np.int64)
+    ident = np.stack([(x64 * (wq[n] == 1)).sum(1) - (x64 * (wq[n] == -1)).sum(1) for n in range(N)], axis=1)
+    assert np.array_equal(got, ident)
+
+
+def test_contract_blas_extreme_sums_and_bound():
+    """|acc| = 128 K at the largest K the library takes (closed form), and
+    refusal where float32 partial sums could round."""
+    K = 32768
+    xq = np.full((2, K), -128, dtype=np.int8)
+    xq[1] = 127
+    wq = np.full((3, K), -1, dtype=np.int8)
+    wq[1] = 1
+    wq[2, ::2] = 0
+    got = oracle.contract_blas(xq, wq)
+    want = np.array([[128 * K, -128 * K, 64 * K], [-127 * K, 127 * K, -127 * K // 2]], dtype=np.int64)
+    assert np.array_equal(got, want)
+    with pytest.raises(oracle.OracleError):
+        oracle.contract_blas(np.zeros((1, 1 << 17), np.int8), np.zeros((1, 1 << 17), np.int8))
+
+
 def test_rescale_hand_values():
     acc = np.array([254, 0, -6], dtype=np.int64)
     Y = oracle.rescale(acc, np.float32(0.5), np.array([127.0, 3.0, 1.0], dtype=np.float32))
