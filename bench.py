@@ -74,6 +74,7 @@ def parse(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-alt", action="store_true", help="skip the secondary decode paths (per-M, two-launch, chains)")
     ap.add_argument("--min-timed-ms", type=float, default=300.0,
                     help="each measurement repeats its timed region until this much device time is timed")
     ap.add_argument("--ref-budget-s", type=float, default=90.0,
@@ -467,7 +468,7 @@ def bench_decode125m(args, rank, world, local, dev, pk):
 
     # per M: K launches of that M alone
     per_m = {}
-    for M in MS:
+    for M in (() if args.no_alt else MS):
         g = graph_of(steps_fn(K_, (M,)), stream)
         msm = time_regions(g.replay, stream, world, min_ms=args.min_timed_ms / 3)
         us = statistics.median(msm) * 1e3 / K_
@@ -480,6 +481,8 @@ def bench_decode125m(args, rank, world, local, dev, pk):
     # ---- secondary: two launches per M; layer order at M = 1 ---------------
     alt = {}
     nalt = max(1, min(K_, 2 * R))
+    if args.no_alt:
+        nalt = 0
     tl = {(M, r): two_launch_problems(M, r) for M in MS for r in range(R)}
 
     def two_step(sp):
@@ -489,31 +492,46 @@ def bench_decode125m(args, rank, world, local, dev, pk):
                 ok(L.bl_quant_act_grouped(acts, count, api.BL_BF16, M, 1e-6, sp), "bl_quant_act_grouped")
                 ok(L.bl_forward_grouped(fwd, count, M, RDY, sp), "bl_forward_grouped")
 
-    g2 = graph_of(two_step, stream)
-    alt["two_launch_us_per_step"] = round(statistics.median(time_regions(g2.replay, stream, world, min_reps=10,
-                                                                         min_ms=50)) * 1e3 / nalt, 3)
-    del g2
-    stages = []
-    per_layer = len(workloads.decode125m_layer_shapes())
-    for layer in range(count // per_layer):
-        b0 = layer * per_layer
-        for sel in ((0, 1, 2), (3,), (4, 5), (6,)):
-            stages.append([b0 + j for j in sel])
-    lay = {r: [fused_problems(1, r, sel) for sel in stages] for r in range(R)}
+    if nalt:
+        g2 = graph_of(two_step, stream)
+        alt["two_launch_us_per_step"] = round(statistics.median(time_regions(g2.replay, stream, world, min_reps=10,
+                                                                             min_ms=50)) * 1e3 / nalt, 3)
+        del g2
+    # the real dependent step: each layer reads the previous layer's output
+    # (chain.DecodeChain), one chain per weight replica so that no step finds
+    # its weights in L2
+    from ternary_quantized_linear_bitlinear_b200.chain import PROJ, DecodeChain
+    per_layer = len(PROJ)
+    nlay = count // per_layer
+    gains = [(workloads.uniform((768,), 0.9, 1.1, 30 + li).to(dev), workloads.uniform((2048,), 0.9, 1.1, 60 + li).to(dev))
+             for li in range(nlay)]
+    for Mc in ((1, 4) if nalt else ()):
+        chains = []
+        for r in range(R):
+            layers = []
+            for li in range(nlay):
+                lay = {}
+                for j, name in enumerate(PROJ):
+                    i = li * per_layer + j
+                    N, K = shapes[i]
+                    lay[name] = (replicas[r][offs[i]:offs[i] + N * K // 4].view(N, K // 4), gammas[i], N, K)
+                layers.append(lay)
+            ch = DecodeChain(layers, gains, Mc)
+            ch.x0.copy_(items[0][2][:Mc].float().to(dev))
+            chains.append(ch)
 
-    def layered(sp):
-        for st in range(nalt):
-            for arr, sel in zip(lay[st % R], stages):
-                ok(L.bl_linear_decode_grouped(arr, len(sel), api.BL_BF16, 1, 1e-6, RDY, sp),
-                   "bl_linear_decode_grouped")
+        def chained(sp, chains=chains):
+            for st in range(nalt):
+                chains[st % R].run(sp)
 
-    g3 = graph_of(layered, stream)
-    us3 = statistics.median(time_regions(g3.replay, stream, world, min_reps=10, min_ms=50)) * 1e3 / nalt
-    alt["layered_m1_us_per_step"] = round(us3, 3)
-    alt["layered_m1_gbs"] = round((wbytes + 2 * xbytes[1]) / (us3 * 1e-6) / 1e9, 1)
-    alt["layered_m1_launches_per_step"] = len(stages)
-    alt["layered_m1_note"] = "per layer qkv | o | gate,up | down, launches ordered but fed no data by each other"
-    del g3
+        g3 = graph_of(chained, stream)
+        us3 = statistics.median(time_regions(g3.replay, stream, world, min_reps=10, min_ms=50)) * 1e3 / nalt
+        abytes = wbytes + 4 * Mc * sum(K for _, K in shapes)  # packed W + the f32 activations each layer reads
+        alt[f"chain_m{Mc}"] = {"us_per_token_step": round(us3, 3), "gbs": round(abytes / (us3 * 1e-6) / 1e9, 1),
+                               "launches_per_step": chains[0].launches_per_step(),
+                               "note": "12 dependent layers: qkv | o (SubLN) | gate,up | FFN act quant (SubLN) "
+                                       "| down, each reading the previous launch's output"}
+        del g3, chains
     api.bl_check_device_error(stream)
 
     # ---- end to end through the C ABI with host buffers --------------------

@@ -131,6 +131,33 @@ bl_status bl_quant_weights_noalloc(const void *W, bl_dtype wdt, int64_t N, int64
                                    uint8_t *packed, float *gamma, bl_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Step 1 for several weight matrices in two launches (one reduction grid    */
+/* and one pack grid over all of them), e.g. the projections of a layer      */
+/* that are re-quantized every call: their reduction latency chains overlap  */
+/* instead of running one after the other.  Same definition and the same    */
+/* bits as bl_quant_weights for each matrix.                                 */
+/*                                                                           */
+/* problems  HOST array of `count` (1 <= count <= BL_MAX_WQ_GROUP) matrices, */
+/*           read during the call only; each W of dtype wdt, each with its    */
+/*           own packed and gamma outputs (device); limits per matrix as for */
+/*           bl_quant_weights                                                */
+/* workspace device scratch of at least bl_quant_weights_workspace_bytes()   */
+/*           (the same size as for one matrix), clobbered                    */
+/* ------------------------------------------------------------------------ */
+#define BL_MAX_WQ_GROUP 8
+
+typedef struct {
+    const void *W;    /* [N, K] of the call's dtype */
+    int64_t N;
+    int64_t K;
+    uint8_t *packed;  /* [N, K/4] out */
+    float *gamma;     /* [1] out */
+} bl_weight_problem;
+
+bl_status bl_quant_weights_grouped(const bl_weight_problem *problems, int count, bl_dtype wdt,
+                                   void *workspace, size_t workspace_bytes, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Step 2: per-token absmax INT8 activation quantization, optionally fused  */
 /* with a preceding SubLN RMSNorm.                                           */
 /*                                                                           */
@@ -185,16 +212,59 @@ bl_status bl_ffn_act_quant(const float *gate, const float *up, int64_t M, int64_
 /*   Y[m, n]   = float(float(acc) * float(gamma / s[m]))                     */
 /*               (two float roundings: |Y - acc*gamma/s| <= 2^-23 |Y|)       */
 /*                                                                           */
-/* Engine: the bandwidth-bound decode GEMV when M <= 16 and its shared-     */
-/* memory staging fits (M <= 16 for K <= 6144, M <= 13 at K = 9728, M <= 4 */
-/* at K = 16384, M <= 2 at K = 20480, none for K >= 24576),                  */
-/* otherwise the tcgen05 prefill GEMM.  Both give identical acc.             */
+/* Engine: the bandwidth-bound decode GEMV when M <= 16 and the staged     */
+/* activations fit, M * round_up(K, 256) <= 153600 bytes (M <= 16 for      */
+/* K <= 9472, M <= 15 at K = 9728, M <= 9 at K = 16384, M <= 4 at           */
+/* K = 32768), otherwise the tcgen05 prefill GEMM.  Both give identical acc. */
 /* packed [N, K/4] (format above); gamma [1]; x_q [M, K]; s [M]; Y [M, N]    */
 /* out; acc_out [M, N] int32 out or NULL.  All device.                       */
 /* ------------------------------------------------------------------------ */
 bl_status bl_forward(const uint8_t *packed, const float *gamma, const int8_t *x_q,
                      const float *s, int64_t M, int64_t N, int64_t K, float *Y,
                      int32_t *acc_out, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Steps 3 + 4 of the gate and up projections of an FFN, fused with the FFN  */
+/* activation between them and the down projection, in ONE tcgen05 launch:  */
+/*                                                                           */
+/*   h = float(float(r * r) * Y_up),  r = max(Y_gate, 0)                     */
+/*                                                                           */
+/* with Y_gate and Y_up the bits bl_forward would give for the two          */
+/* projections on the shared x_q, s; only h is written (the gate and up     */
+/* outputs never reach memory).  Defined by: "SLM750-Edge" model card, "Key */
+/* Architectural Features" (FFN activation ReLU2) and section 2.3 (gate,    */
+/* up, down); "bitone" README, Forward pass (Y = X @ W_q^T * gamma).        */
+/* h then feeds bl_quant_act (with the down projection's SubLN gain).       */
+/*                                                                           */
+/* packed_gate, packed_up [F, K/4]; gamma_gate, gamma_up [1]; x_q [M, K];    */
+/* s [M]; h [M, F] float32 out.  All device, 16-byte aligned.  F % 64 == 0  */
+/* and 64 <= F <= 2^31 - 1 (F is the down projection's K); K as for        */
+/* bl_forward.  Any M (the tcgen05 engine; decode-sized calls do better     */
+/* with bl_linear_decode_grouped + bl_ffn_act_quant).                        */
+/* ------------------------------------------------------------------------ */
+bl_status bl_forward_glu(const uint8_t *packed_gate, const float *gamma_gate, const uint8_t *packed_up,
+                         const float *gamma_up, const int8_t *x_q, const float *s, int64_t M, int64_t F,
+                         int64_t K, float *h, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Backward of the quantization-aware BitLinear, activation gradient, with  */
+/* the straight-through estimator ("Distillix" README, 1. BitNet b1.58      */
+/* Core: STE; "BitDistill", Evaluation and results: gradients pass the      */
+/* activation quantizer unchanged).  With the forward Y = (x_q/s) (gamma    */
+/* W_q)^T and both quantizers passed straight through:                       */
+/*                                                                           */
+/*   dX[m, k] = float(gamma * float(sum_n dY[m, n] * W_q[n, k]))             */
+/*                                                                           */
+/* the sum in float32 on the tensor cores (bf16 x ternary products are      */
+/* exact; the accumulation order is the hardware's, so dX agrees with the   */
+/* exact value within about N * 2^-23 of sum_n |dY[m, n] W_q[n, k]| gamma). */
+/*                                                                           */
+/* dY [M, N] bfloat16 (N % 8 == 0); packed [N, K/4] and gamma [1] as the    */
+/* forward's (bl_quant_weights); dX [M, K] float32 out.  All device, 16-byte */
+/* aligned.  K as for bl_forward.                                            */
+/* ------------------------------------------------------------------------ */
+bl_status bl_backward_dx(const void *dY, const uint8_t *packed, const float *gamma, int64_t M, int64_t N,
+                         int64_t K, float *dX, bl_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* All four steps in one call: bl_quant_weights, bl_quant_act, bl_forward    */
@@ -292,6 +362,32 @@ typedef struct {
 
 bl_status bl_linear_decode_grouped(const bl_decode_problem *problems, int count, bl_dtype xdt,
                                    int64_t M, float subln_eps, unsigned flags, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* All four steps for up to BL_MAX_PREFILL_GROUP weight matrices that share  */
+/* one input X (the q, k, v or the gate, up projections of a layer), every  */
+/* weight re-quantized in the call: one grouped weight quantization (two     */
+/* launches), ONE activation quantization of X, and one grouped contraction */
+/* launch (the tcgen05 GEMM over all matrices' output tiles, or for         */
+/* decode-sized M the fused decode launch, which quantizes X itself).  Each  */
+/* Y_i carries the bits bl_linear(W_i, X) gives.                             */
+/*                                                                           */
+/* problems  HOST array of `count` matrices, read during the call only      */
+/* X         [M, K] of dtype xdt, device; subln_gain [K] or NULL             */
+/* workspace >= bl_linear_grouped_workspace_bytes(problems, count, M, K):    */
+/*           packed weights, gammas, x_q and s between the steps             */
+/* Errors: as bl_linear; BL_ERR_SHAPE for count outside [1, 4].              */
+/* ------------------------------------------------------------------------ */
+typedef struct {
+    const void *W;  /* [N, K] of the call's weight dtype */
+    float *Y;       /* [M, N] out */
+    int64_t N;
+} bl_linear_problem;
+
+size_t bl_linear_grouped_workspace_bytes(const bl_linear_problem *problems, int count, int64_t M, int64_t K);
+bl_status bl_linear_grouped(const bl_linear_problem *problems, int count, bl_dtype wdt, const void *X,
+                            bl_dtype xdt, int64_t M, int64_t K, const float *subln_gain, float subln_eps,
+                            void *workspace, size_t workspace_bytes, bl_stream_t stream);
 
 #ifdef __cplusplus
 }

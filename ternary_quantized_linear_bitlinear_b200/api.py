@@ -47,6 +47,16 @@ class ActProblem(ctypes.Structure):
     _fields_ = [("X", _p), ("subln_gain", _p), ("x_q", _p), ("s", _p), ("K", _i64)]
 
 
+class WeightProblem(ctypes.Structure):
+    """bl_weight_problem: one weight matrix of a grouped weight quantization."""
+    _fields_ = [("W", _p), ("N", _i64), ("K", _i64), ("packed", _p), ("gamma", _p)]
+
+
+class LinearProblem(ctypes.Structure):
+    """bl_linear_problem: one weight matrix (and its output) of a grouped bl_linear."""
+    _fields_ = [("W", _p), ("Y", _p), ("N", _i64)]
+
+
 class DecodeProblem(ctypes.Structure):
     """bl_decode_problem: one problem of the fused grouped decode (X in, Y out)."""
     _fields_ = [("packed", _p), ("gamma", _p), ("X", _p), ("subln_gain", _p), ("Y", _p), ("x_q", _p),
@@ -71,6 +81,12 @@ _SIGS = {
     "bl_quant_act_grouped": (_int, [ctypes.POINTER(ActProblem), _int, _int, _i64, _f32, _p]),
     "bl_linear_decode_grouped": (_int, [ctypes.POINTER(DecodeProblem), _int, _int, _i64, _f32, ctypes.c_uint,
                                         _p]),
+    "bl_quant_weights_grouped": (_int, [ctypes.POINTER(WeightProblem), _int, _int, _p, _sz, _p]),
+    "bl_forward_glu": (_int, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _p]),
+    "bl_backward_dx": (_int, [_p, _p, _p, _i64, _i64, _i64, _p, _p]),
+    "bl_linear_grouped_workspace_bytes": (_sz, [ctypes.POINTER(LinearProblem), _int, _i64, _i64]),
+    "bl_linear_grouped": (_int, [ctypes.POINTER(LinearProblem), _int, _int, _p, _int, _i64, _i64, _p, _f32, _p, _sz,
+                                 _p]),
 }
 
 EXPORTED = tuple(_SIGS)
@@ -222,6 +238,35 @@ def bl_quant_weights_noalloc(W: torch.Tensor, packed=None, gamma=None, stream=No
     return packed, gamma
 
 
+def bl_quant_weights_grouped(Ws, packed=None, gammas=None, workspace=None, stream=None):
+    """Several weight matrices (same dtype) in two launches -> ([packed], [gamma]),
+    each as bl_quant_weights(W) would give it."""
+    Ws = list(Ws)
+    if not 1 <= len(Ws) <= 8:
+        raise ValueError("between 1 and 8 weight matrices")
+    dtype = Ws[0].dtype
+    shapes = [_mat(W, f"Ws[{i}]") for i, W in enumerate(Ws)]
+    for i, W in enumerate(Ws):
+        _dev(W, f"Ws[{i}]", dtype)
+    dev = Ws[0].device
+    if packed is None:
+        packed = [torch.empty(N, K // 4, dtype=torch.uint8, device=dev) for N, K in shapes]
+    if gammas is None:
+        gammas = [torch.empty(4, dtype=torch.float32, device=dev)[:1] for _ in Ws]
+    if workspace is None:
+        workspace = torch.empty(quant_weights_workspace_bytes(1, 64), dtype=torch.uint8, device=dev)
+    _dev(workspace, "workspace", torch.uint8)
+    arr = (WeightProblem * len(Ws))()
+    for i, ((N, K), W, pk, g) in enumerate(zip(shapes, Ws, packed, gammas)):
+        _dev(pk, f"packed[{i}]", torch.uint8, N * K // 4)
+        _dev(g, f"gammas[{i}]", torch.float32, 1)
+        arr[i] = WeightProblem(W.data_ptr(), N, K, pk.data_ptr(), g.data_ptr())
+    rc = lib().bl_quant_weights_grouped(arr, len(Ws), _DTYPES[dtype], workspace.data_ptr(), workspace.numel(),
+                                        _stream(stream))
+    _check(rc, "bl_quant_weights_grouped")
+    return packed, gammas
+
+
 # -- step 2 --------------------------------------------------------------------
 
 def bl_quant_act(X: torch.Tensor, subln_gain=None, subln_eps: float = 1e-6, x_q=None, s=None, stream=None):
@@ -298,6 +343,42 @@ def _xq2d(x_q):
     if x_q.dim() != 2:
         raise ValueError(f"x_q must be 2-D [M, K], got shape {tuple(x_q.shape)}")
     return x_q.shape[0], x_q.shape[1]
+
+
+def bl_forward_glu(packed_gate, gamma_gate, packed_up, gamma_up, x_q, s, F: int, h=None, stream=None):
+    """h float32 [M, F] = relu(Y_gate)^2 * Y_up of the gate and up projections
+    on the shared (x_q, s), from one launch that never stores Y_gate or Y_up."""
+    M, K = _xq2d(x_q)
+    if h is None:
+        h = torch.empty(M, F, dtype=torch.float32, device=x_q.device)
+    _dev(packed_gate, "packed_gate", torch.uint8, F * K // 4)
+    _dev(packed_up, "packed_up", torch.uint8, F * K // 4)
+    _dev(gamma_gate, "gamma_gate", torch.float32, 1)
+    _dev(gamma_up, "gamma_up", torch.float32, 1)
+    _dev(s, "s", torch.float32, M)
+    _dev(h, "h", torch.float32, M * F)
+    rc = lib().bl_forward_glu(packed_gate.data_ptr(), gamma_gate.data_ptr(), packed_up.data_ptr(), gamma_up.data_ptr(),
+                              x_q.data_ptr(), s.data_ptr(), M, F, K, h.data_ptr(), _stream(stream))
+    _check(rc, "bl_forward_glu")
+    return h
+
+
+def bl_backward_dx(dY, packed, gamma, K: int, dX=None, stream=None):
+    """dX float32 [M, K] = dY @ (gamma W_q) (straight-through backward of the
+    activation), dY bfloat16 [M, N]."""
+    _dev(dY, "dY", torch.bfloat16)
+    if dY.dim() != 2:
+        raise ValueError("dY must be 2-D [M, N]")
+    M, N = dY.shape
+    if dX is None:
+        dX = torch.empty(M, K, dtype=torch.float32, device=dY.device)
+    _dev(packed, "packed", torch.uint8, N * K // 4)
+    _dev(gamma, "gamma", torch.float32, 1)
+    _dev(dX, "dX", torch.float32, M * K)
+    rc = lib().bl_backward_dx(dY.data_ptr(), packed.data_ptr(), gamma.data_ptr(), M, N, K, dX.data_ptr(),
+                              _stream(stream))
+    _check(rc, "bl_backward_dx")
+    return dX
 
 
 def _check_forward_args(packed, gamma, s, Y, acc_out, M, N, K):
@@ -414,6 +495,36 @@ def bl_linear(W, X, subln_gain=None, subln_eps: float = 1e-6, Y=None, workspace=
                          _stream(stream))
     _check(rc, "bl_linear")
     return Y
+
+
+def bl_linear_grouped(Ws, X, subln_gain=None, subln_eps: float = 1e-6, Ys=None, workspace=None, stream=None):
+    """Up to 4 weight matrices sharing the input X (e.g. q, k, v), all steps,
+    weights quantized in the call -> [Y_i float32 [M, N_i]]."""
+    Ws = list(Ws)
+    if not 1 <= len(Ws) <= 4:
+        raise ValueError("between 1 and 4 weight matrices")
+    wdt = Ws[0].dtype
+    shapes = [_mat(W, f"Ws[{i}]") for i, W in enumerate(Ws)]
+    K = shapes[0][1]
+    for i, W in enumerate(Ws):
+        _mat(W, f"Ws[{i}]", cols=K)
+        _dev(W, f"Ws[{i}]", wdt)
+    M, _ = _mat(X, "X", cols=K)
+    if Ys is None:
+        Ys = [torch.empty(M, N, dtype=torch.float32, device=X.device) for N, _ in shapes]
+    arr = (LinearProblem * len(Ws))()
+    for i, ((N, _), W, Y) in enumerate(zip(shapes, Ws, Ys)):
+        _dev(Y, f"Ys[{i}]", torch.float32, M * N)
+        arr[i] = LinearProblem(W.data_ptr(), Y.data_ptr(), N)
+    need = int(lib().bl_linear_grouped_workspace_bytes(arr, len(Ws), M, K))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=X.device)
+    _dev(workspace, "workspace", torch.uint8, need)
+    _opt(subln_gain, "subln_gain", torch.float32, K)
+    rc = lib().bl_linear_grouped(arr, len(Ws), _DTYPES[wdt], X.data_ptr(), _DTYPES[X.dtype], M, K, _ptr(subln_gain),
+                                 subln_eps, workspace.data_ptr(), workspace.numel(), _stream(stream))
+    _check(rc, "bl_linear_grouped")
+    return Ys
 
 
 def bl_debug_forward_prefill(packed, gamma, x_q, s, N: int, Y=None, acc_out=None, skip_iter: int = -1,

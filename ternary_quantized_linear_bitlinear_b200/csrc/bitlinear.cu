@@ -5,7 +5,10 @@
 // (except bl_check_device_error, which is documented to).
 #include <cuda_runtime.h>
 
+#include <cmath>
+#include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "bitlinear.h"
 #include "bitlinear_debug.h"
@@ -22,6 +25,9 @@ namespace {
 constexpr int BL_VERSION = 100;
 constexpr int64_t K_MAX = 32768;
 constexpr int MAX_DEVICES = 64;
+constexpr size_t DEC_SMEM_ATTR = (size_t)dec_fixed_smem(2) + DEC_X_MAX + 1024;
+static_assert(DEC_SMEM_ATTR <= 227 * 1024, "decode engine shared memory");
+static_assert(sizeof(DecodeParams) <= 32764, "decode parameters exceed the kernel parameter limit");
 
 struct DeviceInfo {
     bool init = false;
@@ -48,7 +54,7 @@ bl_status device_info(DeviceInfo **out) {
             bool fail = false;
             for (auto fn : {k_decode<1, DEC_SRC_XQ>, k_decode<2, DEC_SRC_XQ>, k_decode<1, DEC_SRC_BF16>,
                             k_decode<2, DEC_SRC_BF16>, k_decode<1, DEC_SRC_F32>, k_decode<2, DEC_SRC_F32>})
-                fail |= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, DEC_SMEM_LIMIT) !=
+                fail |= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DEC_SMEM_ATTR) !=
                         cudaSuccess;
             fail |= prefill_setup() != cudaSuccess;
             for (auto fn : {k_act_quant_subln_row<false, true>, k_act_quant_subln_row<true, false>,
@@ -78,33 +84,73 @@ bool nk_fits(int64_t N, int64_t K) { return N <= ((1LL << 31) - 1) / K; }
 // ---------------------------------------------------------------------------
 // Step 1
 
-bl_status quant_weights_impl(const DeviceInfo &d, const void *W, bl_dtype wdt, int64_t N, int64_t K,
-                             uint8_t *packed, float *gamma, void *ws, cudaStream_t st) {
-    const long long n = (long long)N * K;
+// One weight matrix to quantize (all matrices of a launch share the dtype).
+struct WqIn {
+    const void *W;
+    int64_t N, K;
+    uint8_t *packed;
+    float *gamma;
+};
+
+// Reduction blocks per matrix: a share of 2 x SMs proportional to its size,
+// at least enough that no thread sums more than 2^14 terms (which keeps each
+// 64-bit window accumulator exact), at most one vector per thread, and at
+// most WQ_MAX_BLOCKS over the launch.
+bl_status quant_weights_impl(const DeviceInfo &d, const WqIn *in, int count, bl_dtype wdt, void *ws,
+                             cudaStream_t st) {
+    if (count < 1 || count > WQ_MAX_JOBS) return BL_ERR_SHAPE;
     const bool bf16 = wdt == BL_BF16;
     const int epv = bf16 ? 8 : 4;
-    const long long nvec = n / epv;
-    long long grid = 2LL * d.sms;
-    long long need = (nvec + WQ_THREADS - 1) / WQ_THREADS;
-    if (grid > need) grid = need;
-    if (grid < 1) grid = 1;
-    // at most 2^14 terms per thread keeps each 64-bit window accumulator exact
-    while (grid < WQ_MAX_BLOCKS && ((nvec + grid * WQ_THREADS - 1) / (grid * WQ_THREADS)) * epv > 16384) grid *= 2;
-    if (grid > WQ_MAX_BLOCKS) grid = WQ_MAX_BLOCKS;
-
-    u64 *partials = reinterpret_cast<u64 *>(ws);
-    u32 *thresh = reinterpret_cast<u32 *>(reinterpret_cast<uint8_t *>(ws) + WQ_WS_PARTIALS);
-    u32 *ticket = reinterpret_cast<u32 *>(reinterpret_cast<uint8_t *>(ws) + WQ_WS_TICKET);
-    const uint4 *Wv = reinterpret_cast<const uint4 *>(W);
-    if (cudaMemsetAsync(ticket, 0, sizeof(u32), st) != cudaSuccess) return BL_ERR_CUDA;
+    const long long vec_cap = 16384 / epv;  // vectors per thread
+    WqParams P;
+    memset(&P, 0, sizeof(P));
+    P.count = count;
+    P.partials = reinterpret_cast<u64 *>(ws);
+    P.thresh = reinterpret_cast<u32 *>(reinterpret_cast<uint8_t *>(ws) + WQ_WS_PARTIALS);
+    P.tickets = reinterpret_cast<u32 *>(reinterpret_cast<uint8_t *>(ws) + WQ_WS_TICKET);
+    double total = 0.0;
+    for (int i = 0; i < count; ++i) total += (double)in[i].N * (double)in[i].K;
+    long long blocks = 0, words = 0;
+    long long mins = 0;
+    for (int i = 0; i < count; ++i) {
+        const long long n = (long long)in[i].N * in[i].K;
+        const long long nvec = n / epv;
+        const long long need = (nvec + WQ_THREADS - 1) / WQ_THREADS;
+        const long long minb = (nvec + (long long)WQ_THREADS * vec_cap - 1) / ((long long)WQ_THREADS * vec_cap);
+        long long nb = (long long)std::llround(2.0 * d.sms * ((double)n / total));
+        if (nb > need) nb = need;
+        if (nb < minb) nb = minb;
+        if (nb < 1) nb = 1;
+        mins += minb;
+        P.j[i] = WqJob{reinterpret_cast<const uint4 *>(in[i].W), nvec, n, in[i].gamma,
+                       reinterpret_cast<u32 *>(in[i].packed), n / 16, words, (int)blocks, (int)nb};
+        blocks += nb;
+        words += n / 16;
+    }
+    if (mins > WQ_MAX_BLOCKS) return BL_ERR_SHAPE;
+    if (blocks > WQ_MAX_BLOCKS) {
+        // scale the shares down (never below a matrix's minimum)
+        blocks = 0;
+        for (int i = 0; i < count; ++i) {
+            const long long minb = (P.j[i].nvec + (long long)WQ_THREADS * vec_cap - 1) / ((long long)WQ_THREADS * vec_cap);
+            long long nb = (long long)((double)P.j[i].nblk * (WQ_MAX_BLOCKS - mins) / (double)WQ_MAX_BLOCKS);
+            if (nb < minb) nb = minb;
+            if (nb < 1) nb = 1;
+            P.j[i].blk0 = (int)blocks;
+            P.j[i].nblk = (int)nb;
+            blocks += nb;
+        }
+        if (blocks > WQ_MAX_BLOCKS) return BL_ERR_SHAPE;
+    }
+    P.total_words = words;
+    if (cudaMemsetAsync(P.tickets, 0, sizeof(u32) * count, st) != cudaSuccess) return BL_ERR_CUDA;
     if (bf16)
-        k_absmean_partial<true><<<(unsigned)grid, WQ_THREADS, 0, st>>>(Wv, nvec, n, partials, gamma, thresh, ticket);
+        k_absmean_partial<true><<<(unsigned)blocks, WQ_THREADS, 0, st>>>(P);
     else
-        k_absmean_partial<false><<<(unsigned)grid, WQ_THREADS, 0, st>>>(Wv, nvec, n, partials, gamma, thresh, ticket);
+        k_absmean_partial<false><<<(unsigned)blocks, WQ_THREADS, 0, st>>>(P);
     if (cudaGetLastError() != cudaSuccess) return BL_ERR_CUDA;
-    const long long nwords = n / 16;
-    long long pgrid = (nwords + 255) / 256;
-    long long pcap = 8LL * d.sms;
+    long long pgrid = (words + 255) / 256;
+    const long long pcap = 8LL * d.sms;
     if (pgrid > pcap) pgrid = pcap;
     // programmatic dependent launch: the pack grid starts loading W while the
     // reduction finishes and waits for it (griddepcontrol.wait) before using T
@@ -117,11 +163,15 @@ bl_status quant_weights_impl(const DeviceInfo &d, const void *W, bl_dtype wdt, i
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    u32 *pk = reinterpret_cast<u32 *>(packed);
-    const u32 *th = thresh;
-    cudaError_t e = bf16 ? cudaLaunchKernelEx(&cfg, k_ternary_pack<true>, Wv, nwords, th, pk)
-                         : cudaLaunchKernelEx(&cfg, k_ternary_pack<false>, Wv, nwords, th, pk);
+    cudaError_t e = bf16 ? cudaLaunchKernelEx(&cfg, k_ternary_pack<true>, P)
+                         : cudaLaunchKernelEx(&cfg, k_ternary_pack<false>, P);
     return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+bl_status quant_weights_one(const DeviceInfo &d, const void *W, bl_dtype wdt, int64_t N, int64_t K, uint8_t *packed,
+                            float *gamma, void *ws, cudaStream_t st) {
+    const WqIn in{W, N, K, packed, gamma};
+    return quant_weights_impl(d, &in, 1, wdt, ws, st);
 }
 
 // ---------------------------------------------------------------------------
@@ -230,61 +280,137 @@ bl_status quant_act_impl(const ActParams &P, bl_dtype xdt, int64_t Kmax, cudaStr
 // ---------------------------------------------------------------------------
 // Steps 3 + 4
 
-int dec_xq_off(int64_t K) { return (dec_w_bytes((int)K) + 127) & ~127; }
+bool decode_eligible(int64_t M, int64_t K) { return M <= 16 && M * dec_row_stride((int)K) <= DEC_X_MAX; }
 
-bool decode_eligible(int64_t M, int64_t K) {
-    return M <= 16 && dec_xq_off(K) + M * dec_row_stride((int)K) <= DEC_SMEM_LIMIT;
+
+// One problem of a decode launch, as the entry points receive it.
+struct DecodeJob {
+    const uint8_t *packed;
+    const float *gamma;
+    const void *x;        // x_q (DEC_SRC_XQ) or X
+    float *s;
+    float *Y;
+    int32_t *acc;
+    const float *gain;
+    int8_t *xq_out;
+    int64_t N, K;
+};
+
+// Tensor maps of packed weight matrices ({K/4 bytes, N rows}, box 128 x 32,
+// 128-byte swizzle), cached by (address, N, K): encoding one costs about a
+// microsecond of host time, and a decode launch may need a hundred.
+struct WmapKey {
+    const void *p;
+    int64_t N, K;
+    bool operator==(const WmapKey &o) const { return p == o.p && N == o.N && K == o.K; }
+};
+struct WmapHash {
+    size_t operator()(const WmapKey &k) const {
+        return std::hash<const void *>()(k.p) ^ (std::hash<int64_t>()(k.N) * 31u) ^ (std::hash<int64_t>()(k.K) * 131u);
+    }
+};
+std::mutex g_wmap_mu;
+std::unordered_map<WmapKey, CUtensorMap, WmapHash> g_wmap;
+
+bl_status dec_wmap(const uint8_t *packed, int64_t N, int64_t K, CUtensorMap *out) {
+    const WmapKey key{packed, N, K};
+    std::lock_guard<std::mutex> lk(g_wmap_mu);
+    auto it = g_wmap.find(key);
+    if (it != g_wmap.end()) {
+        *out = it->second;
+        return BL_OK;
+    }
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (enc == nullptr) return BL_ERR_CUDA;
+    const cuuint64_t gdim[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
+    const cuuint64_t gstride[1] = {(cuuint64_t)(K / 4)};
+    const cuuint32_t box[2] = {(cuuint32_t)DEC_CB, (cuuint32_t)DEC_ROWS};
+    const cuuint32_t es[2] = {1, 1};
+    CUtensorMap m;
+    if (enc(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return BL_ERR_CUDA;
+    if (g_wmap.size() >= 8192) g_wmap.clear();
+    g_wmap.emplace(key, m);
+    *out = m;
+    return BL_OK;
 }
 
-bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st, int src, int sms) {
-    // G (warps per 32-row group) per problem: dec_glog's choice, raised while
-    // the launch would leave SMs idle and the problem has k steps to split
-    // (small launches, e.g. one layer's projections at a time, get more CTAs
-    // with fewer rows each)
-    for (int i = 0; i < P.count; ++i) P.p[i].g_log2 = dec_glog(P.p[i].K);
-    auto ctas_of = [&](const DecodeProblem &q) {
-        const int tiles = (q.N + DEC_ROWS - 1) / DEC_ROWS;
-        const int per = DEC_WARPS >> q.g_log2;
-        return (tiles + per - 1) / per;
-    };
-    for (;;) {
-        int total = 0;
-        for (int i = 0; i < P.count; ++i) total += ctas_of(P.p[i]);
-        if (total >= sms) break;
-        bool raised = false;
-        for (int i = 0; i < P.count; ++i) {
-            DecodeProblem &q = P.p[i];
-            const int steps = (q.K + 255) >> 8;
-            if (q.g_log2 < 3 && (2 << q.g_log2) <= steps) {
-                ++q.g_log2;
-                raised = true;
+// Decode launch: groups of 32 weight rows over all problems, cut into one
+// contiguous range per CTA with about equal packed bytes (cut before the
+// first group whose midpoint passes the next multiple of total / SMs), then
+// split further at problem boundaries so that no CTA stages more than
+// DEC_MAX_PSLOTS problems' activations or, when it can be avoided, more than
+// DEC_X_PAIR bytes of them (two CTAs per SM).
+bl_status decode_launch(const DecodeJob *jobs, int count, int M, float eps, bool pdl, cudaStream_t st, int src,
+                        int sms) {
+    thread_local DecodeParams P;
+    P.count = count;
+    P.M = M;
+    P.eps = eps;
+    int64_t G = 0;
+    double total = 0.0;
+    for (int i = 0; i < count; ++i) {
+        const DecodeJob &j = jobs[i];
+        bl_status rc = dec_wmap(j.packed, j.N, j.K, &P.wmap[i]);
+        if (rc) return rc;
+        P.p[i] = DecodeProblem{j.gamma, j.x, j.s, j.Y, j.acc, j.gain, j.xq_out, (int)j.N, (int)j.K, (int)G};
+        G += (j.N + DEC_ROWS - 1) / DEC_ROWS;
+        if (G > 0x7fffffffLL) return BL_ERR_SHAPE;
+        total += (double)j.N * (double)(j.K / 4);
+    }
+    P.ngroups = (int)G;
+    const int base_ctas = sms < 1 ? 1 : (sms > DEC_MAX_CTAS - BL_MAX_GROUP ? DEC_MAX_CTAS - BL_MAX_GROUP : sms);
+    const double target = total / base_ctas;
+    int cuts[DEC_MAX_CTAS + 1];
+    int ncut = 0;
+    cuts[ncut++] = 0;
+    double c0 = 0.0, next = target;
+    for (int i = 0; i < count; ++i) {
+        const int64_t ng = (jobs[i].N + DEC_ROWS - 1) / DEC_ROWS;
+        const double gb = (double)DEC_ROWS * (double)(jobs[i].K / 4);
+        while (next < c0 + (double)ng * gb && ncut < base_ctas) {
+            int64_t k = (int64_t)std::floor((next - c0) / gb - 0.5) + 1;
+            if (k < 0) k = 0;
+            const int64_t g = P.p[i].gbase + k;
+            if (k < ng && g > cuts[ncut - 1]) cuts[ncut++] = (int)g;
+            next += target;
+        }
+        c0 += (double)ng * gb;
+    }
+    cuts[ncut] = (int)G;  // end sentinel (not a CTA start)
+    // split at problem boundaries for the activation staging
+    int nc = 0;
+    int max_x = 0;
+    for (int c = 0; c < ncut; ++c) {
+        const int a = cuts[c], b = cuts[c + 1];
+        P.cta_g[nc++] = a;
+        // problems of [a, b)
+        int pi = 0;
+        while (pi + 1 < count && P.p[pi + 1].gbase <= a) ++pi;
+        int xb = 0, np = 0;
+        for (; pi < count && P.p[pi].gbase < b; ++pi) {
+            const int xp = M * dec_row_stride(P.p[pi].K);
+            if (np > 0 && (np == DEC_MAX_PSLOTS || xb + xp > DEC_X_PAIR)) {
+                if (nc >= DEC_MAX_CTAS) return BL_ERR_SHAPE;
+                max_x = xb > max_x ? xb : max_x;
+                P.cta_g[nc++] = P.p[pi].gbase;
+                xb = 0;
+                np = 0;
             }
+            xb += xp;
+            ++np;
         }
-        if (!raised) break;
+        max_x = xb > max_x ? xb : max_x;
     }
-    int total = 0;
-    int rs_max = 0, xq_off = 0;
-    for (int i = 0; i < P.count; ++i) {
-        DecodeProblem &q = P.p[i];
-        q.cta_begin = total;
-        total += ctas_of(q);
-        int rs = dec_row_stride(q.K);
-        rs_max = rs > rs_max ? rs : rs_max;
-        const int xo = (((DEC_WARPS >> q.g_log2) * DEC_ROWS * (q.K >> 2)) + 127) & ~127;  // this G's weight bytes
-        xq_off = xo > xq_off ? xo : xq_off;
-    }
-    P.xq_off = xq_off;
-    P.use_table = total <= DEC_CTA_TABLE ? 1 : 0;
-    if (P.use_table) {
-        for (int i = 0; i < P.count; ++i) {
-            const int end = i + 1 < P.count ? P.p[i + 1].cta_begin : total;
-            for (int c = P.p[i].cta_begin; c < end; ++c) P.cta_problem[c] = (unsigned char)i;
-        }
-    }
-    const size_t smem = (size_t)xq_off + (size_t)P.M * rs_max;
-    if (smem > DEC_SMEM_LIMIT) return BL_ERR_SHAPE;
+    P.cta_g[nc] = (int)G;
+    P.ncta = nc;
+    const int NT = M <= 8 ? 1 : 2;
+    const size_t smem = (size_t)dec_fixed_smem(NT) + (size_t)max_x + 1024;
+    if (max_x > DEC_X_MAX || smem > DEC_SMEM_ATTR) return BL_ERR_SHAPE;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)total);
+    cfg.gridDim = dim3((unsigned)nc);
     cfg.blockDim = dim3(DEC_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = st;
@@ -295,14 +421,14 @@ bl_status decode_launch(DecodeParams &P, bool pdl, cudaStream_t st, int src, int
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t e;
     if (src == DEC_SRC_BF16)
-        e = P.M <= 8 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_BF16>, P)
-                     : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_BF16>, P);
+        e = NT == 1 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_BF16>, P)
+                    : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_BF16>, P);
     else if (src == DEC_SRC_F32)
-        e = P.M <= 8 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_F32>, P)
-                     : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_F32>, P);
+        e = NT == 1 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_F32>, P)
+                    : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_F32>, P);
     else
-        e = P.M <= 8 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_XQ>, P)
-                     : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_XQ>, P);
+        e = NT == 1 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_XQ>, P)
+                    : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_XQ>, P);
     return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 
@@ -310,13 +436,8 @@ bl_status forward_impl(const DeviceInfo &d, const uint8_t *packed, const float *
                        const float *s, int64_t M, int64_t N, int64_t K, float *Y, int32_t *acc_out, cudaStream_t st,
                        bool pdl = false) {
     if (decode_eligible(M, K)) {
-        DecodeParams P;
-        P.count = 1;
-        P.M = (int)M;
-        P.eps = 0.f;
-        P.p[0] = DecodeProblem{packed, gamma, x_q, const_cast<float *>(s), Y, acc_out, nullptr, nullptr,
-                               (int)N, (int)K, 0, 0};
-        return decode_launch(P, false, st, DEC_SRC_XQ, d.sms);
+        const DecodeJob job{packed, gamma, x_q, const_cast<float *>(s), Y, acc_out, nullptr, nullptr, N, K};
+        return decode_launch(&job, 1, (int)M, 0.f, false, st, DEC_SRC_XQ, d.sms);
     }
     return prefill_launch(d.sms, packed, gamma, x_q, s, M, N, K, Y, acc_out, st, PF_DEFAULT_TIMEOUT_NS, -1, pdl);
 }
@@ -394,7 +515,28 @@ bl_status bl_quant_weights(const void *W, bl_dtype wdt, int64_t N, int64_t K, ui
     DeviceInfo *d;
     bl_status rc = device_info(&d);
     if (rc) return rc;
-    return quant_weights_impl(*d, W, wdt, N, K, packed, gamma, workspace, (cudaStream_t)stream);
+    return quant_weights_one(*d, W, wdt, N, K, packed, gamma, workspace, (cudaStream_t)stream);
+}
+
+bl_status bl_quant_weights_grouped(const bl_weight_problem *problems, int count, bl_dtype wdt, void *workspace,
+                                   size_t workspace_bytes, bl_stream_t stream) {
+    if (!problems) return BL_ERR_NULL;
+    if (count < 1 || count > BL_MAX_WQ_GROUP) return BL_ERR_SHAPE;
+    if (wdt != BL_F32 && wdt != BL_BF16) return BL_ERR_DTYPE;
+    WqIn in[BL_MAX_WQ_GROUP];
+    for (int i = 0; i < count; ++i) {
+        const bl_weight_problem &q = problems[i];
+        if (!q.W || !q.packed || !q.gamma) return BL_ERR_NULL;
+        if (q.N < 1 || check_k(q.K) != BL_OK || !nk_fits(q.N, q.K)) return BL_ERR_SHAPE;
+        if (!aligned16(q.W) || !aligned16(q.packed) || !aligned16(q.gamma)) return BL_ERR_ALIGN;
+        in[i] = WqIn{q.W, q.N, q.K, q.packed, q.gamma};
+    }
+    if (!workspace || workspace_bytes < bl_quant_weights_workspace_bytes(1, 64)) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGN;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return quant_weights_impl(*d, in, count, wdt, workspace, (cudaStream_t)stream);
 }
 
 bl_status bl_quant_act_grouped(const bl_act_problem *problems, int count, bl_dtype xdt, int64_t M, float subln_eps,
@@ -459,6 +601,34 @@ bl_status bl_forward(const uint8_t *packed, const float *gamma, const int8_t *x_
     return forward_impl(*d, packed, gamma, x_q, s, M, N, K, Y, acc_out, (cudaStream_t)stream);
 }
 
+bl_status bl_forward_glu(const uint8_t *packed_gate, const float *gamma_gate, const uint8_t *packed_up,
+                         const float *gamma_up, const int8_t *x_q, const float *s, int64_t M, int64_t F, int64_t K,
+                         float *h, bl_stream_t stream) {
+    if (!packed_gate || !gamma_gate || !packed_up || !gamma_up || !x_q || !s || !h) return BL_ERR_NULL;
+    if (M < 1 || M > 0x7fffffffLL || F < 64 || F > 0x7fffffffLL || (F % 64) != 0 || check_k(K) != BL_OK)
+        return BL_ERR_SHAPE;
+    if (!aligned16(packed_gate) || !aligned16(gamma_gate) || !aligned16(packed_up) || !aligned16(gamma_up) ||
+        !aligned16(x_q) || !aligned16(s) || !aligned16(h))
+        return BL_ERR_ALIGN;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return prefill_launch_glu(d->sms, packed_gate, gamma_gate, packed_up, gamma_up, x_q, s, M, F, K, h,
+                              (cudaStream_t)stream);
+}
+
+bl_status bl_backward_dx(const void *dY, const uint8_t *packed, const float *gamma, int64_t M, int64_t N, int64_t K,
+                         float *dX, bl_stream_t stream) {
+    if (!dY || !packed || !gamma || !dX) return BL_ERR_NULL;
+    if (M < 1 || M > 0x7fffffffLL || N < 8 || N > 0x7fffffffLL || (N % 8) != 0 || check_k(K) != BL_OK)
+        return BL_ERR_SHAPE;
+    if (!aligned16(dY) || !aligned16(packed) || !aligned16(gamma) || !aligned16(dX)) return BL_ERR_ALIGN;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    return prefill_launch_bwd(d->sms, dY, packed, gamma, M, N, K, dX, (cudaStream_t)stream);
+}
+
 bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, unsigned flags,
                              bl_stream_t stream) {
     if (!problems) return BL_ERR_NULL;
@@ -466,10 +636,7 @@ bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, u
     bool decode = M <= 16;
     for (int i = 0; i < count && decode; ++i) decode = check_k(problems[i].K) == BL_OK && decode_eligible(M, problems[i].K);
     if (!decode) return forward_grouped_prefill(problems, count, M, (cudaStream_t)stream);
-    DecodeParams P;
-    P.count = count;
-    P.M = (int)M;
-    long long ctas = 0;
+    DecodeJob jobs[BL_MAX_GROUP];
     for (int i = 0; i < count; ++i) {
         const bl_problem &q = problems[i];
         if (!q.packed || !q.gamma || !q.x_q || !q.s || !q.Y) return BL_ERR_NULL;
@@ -477,16 +644,14 @@ bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, u
         if (!aligned16(q.packed) || !aligned16(q.gamma) || !aligned16(q.x_q) || !aligned16(q.s) || !aligned16(q.Y) ||
             (q.acc_out && !aligned16(q.acc_out)))
             return BL_ERR_ALIGN;
-        P.p[i] = DecodeProblem{q.packed, q.gamma, q.x_q, const_cast<float *>(q.s), q.Y, q.acc_out, nullptr, nullptr,
-                               (int)q.N, (int)q.K, 0, 0};
-        ctas += (q.N + 15) / 16;
+        jobs[i] = DecodeJob{q.packed, q.gamma, q.x_q, const_cast<float *>(q.s), q.Y, q.acc_out, nullptr, nullptr,
+                            q.N, q.K};
     }
-    if (ctas > 0x7fffffffLL) return BL_ERR_SHAPE;
-    P.eps = 0.f;
     DeviceInfo *d;
     bl_status rc = device_info(&d);
     if (rc) return rc;
-    return decode_launch(P, (flags & BL_FWD_WEIGHTS_READY) != 0, (cudaStream_t)stream, DEC_SRC_XQ, d->sms);
+    return decode_launch(jobs, count, (int)M, 0.f, (flags & BL_FWD_WEIGHTS_READY) != 0, (cudaStream_t)stream,
+                         DEC_SRC_XQ, d->sms);
 }
 
 bl_status bl_linear_decode_grouped(const bl_decode_problem *problems, int count, bl_dtype xdt, int64_t M,
@@ -494,10 +659,7 @@ bl_status bl_linear_decode_grouped(const bl_decode_problem *problems, int count,
     if (!problems) return BL_ERR_NULL;
     if (count < 1 || count > BL_MAX_GROUP || M < 1 || M > 16) return BL_ERR_SHAPE;
     if (xdt != BL_F32 && xdt != BL_BF16) return BL_ERR_DTYPE;
-    DecodeParams P;
-    P.count = count;
-    P.M = (int)M;
-    P.eps = subln_eps;
+    DecodeJob jobs[BL_MAX_GROUP];
     for (int i = 0; i < count; ++i) {
         const bl_decode_problem &q = problems[i];
         if (!q.packed || !q.gamma || !q.X || !q.Y) return BL_ERR_NULL;
@@ -506,13 +668,12 @@ bl_status bl_linear_decode_grouped(const bl_decode_problem *problems, int count,
             (q.subln_gain && !aligned16(q.subln_gain)) || (q.x_q && !aligned16(q.x_q)) ||
             (q.s && !aligned16(q.s)) || (q.acc_out && !aligned16(q.acc_out)))
             return BL_ERR_ALIGN;
-        P.p[i] = DecodeProblem{q.packed, q.gamma, q.X, q.s, q.Y, q.acc_out, q.subln_gain, q.x_q,
-                               (int)q.N, (int)q.K, 0, 0};
+        jobs[i] = DecodeJob{q.packed, q.gamma, q.X, q.s, q.Y, q.acc_out, q.subln_gain, q.x_q, q.N, q.K};
     }
     DeviceInfo *d;
     bl_status rc = device_info(&d);
     if (rc) return rc;
-    return decode_launch(P, (flags & BL_FWD_WEIGHTS_READY) != 0, (cudaStream_t)stream,
+    return decode_launch(jobs, count, (int)M, subln_eps, (flags & BL_FWD_WEIGHTS_READY) != 0, (cudaStream_t)stream,
                          xdt == BL_BF16 ? DEC_SRC_BF16 : DEC_SRC_F32, d->sms);
 }
 
@@ -547,17 +708,14 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt, in
     p += align256((size_t)M * (size_t)K);
     float *s = reinterpret_cast<float *>(p);
     cudaStream_t st = (cudaStream_t)stream;
-    rc = quant_weights_impl(*d, W, wdt, N, K, packed, gamma, wq_ws, st);
+    rc = quant_weights_one(*d, W, wdt, N, K, packed, gamma, wq_ws, st);
     if (rc) return rc;
     if (decode_eligible(M, K)) {
         // decode-sized: activation quant fused into the GEMV launch (x_q and s
         // still land in the workspace)
-        DecodeParams P;
-        P.count = 1;
-        P.M = (int)M;
-        P.eps = subln_eps;
-        P.p[0] = DecodeProblem{packed, gamma, X, s, Y, nullptr, subln_gain, x_q, (int)N, (int)K, 0, 0};
-        return decode_launch(P, false, st, xdt == BL_BF16 ? DEC_SRC_BF16 : DEC_SRC_F32, d->sms);
+        const DecodeJob job{packed, gamma, X, s, Y, nullptr, subln_gain, x_q, N, K};
+        return decode_launch(&job, 1, (int)M, subln_eps, false, st, xdt == BL_BF16 ? DEC_SRC_BF16 : DEC_SRC_F32,
+                             d->sms);
     }
     ActParams P;
     P.count = 1;
@@ -569,6 +727,78 @@ bl_status bl_linear(const void *W, bl_dtype wdt, const void *X, bl_dtype xdt, in
     rc = quant_act_impl(P, xdt, K, st, true);
     if (rc) return rc;
     return forward_impl(*d, packed, gamma, x_q, s, M, N, K, Y, nullptr, st, true);
+}
+
+size_t bl_linear_grouped_workspace_bytes(const bl_linear_problem *problems, int count, int64_t M, int64_t K) {
+    if (!problems || count < 1 || count > BL_MAX_PREFILL_GROUP || M < 1 || K < 1) return 0;
+    size_t b = align256(WQ_WS_BYTES) + 256 + align256((size_t)M * (size_t)K) + align256((size_t)M * 4);
+    for (int i = 0; i < count; ++i) {
+        if (problems[i].N < 1) return 0;
+        b += align256((size_t)problems[i].N * (size_t)K / 4);
+    }
+    return b;
+}
+
+bl_status bl_linear_grouped(const bl_linear_problem *problems, int count, bl_dtype wdt, const void *X, bl_dtype xdt,
+                            int64_t M, int64_t K, const float *subln_gain, float subln_eps, void *workspace,
+                            size_t workspace_bytes, bl_stream_t stream) {
+    if (!problems || !X) return BL_ERR_NULL;
+    if (count < 1 || count > BL_MAX_PREFILL_GROUP) return BL_ERR_SHAPE;
+    if (wdt != BL_F32 && wdt != BL_BF16) return BL_ERR_DTYPE;
+    if (xdt != BL_F32 && xdt != BL_BF16) return BL_ERR_DTYPE;
+    if (M < 1 || M > 0x7fffffffLL || check_k(K) != BL_OK) return BL_ERR_SHAPE;
+    if (!aligned16(X) || (subln_gain && !aligned16(subln_gain))) return BL_ERR_ALIGN;
+    for (int i = 0; i < count; ++i) {
+        const bl_linear_problem &q = problems[i];
+        if (!q.W || !q.Y) return BL_ERR_NULL;
+        if (q.N < 1 || !nk_fits(q.N, K)) return BL_ERR_SHAPE;
+        if (!aligned16(q.W) || !aligned16(q.Y)) return BL_ERR_ALIGN;
+    }
+    if (!workspace || workspace_bytes < bl_linear_grouped_workspace_bytes(problems, count, M, K))
+        return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGN;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    // workspace: [weight-quant scratch | gammas (16 B apart) | x_q | s | packed_0 | packed_1 ...]
+    uint8_t *p = reinterpret_cast<uint8_t *>(workspace);
+    void *wq_ws = p;
+    p += align256(WQ_WS_BYTES);
+    float *gammas = reinterpret_cast<float *>(p);
+    p += 256;
+    int8_t *x_q = reinterpret_cast<int8_t *>(p);
+    p += align256((size_t)M * (size_t)K);
+    float *s = reinterpret_cast<float *>(p);
+    p += align256((size_t)M * 4);
+    WqIn in[BL_MAX_PREFILL_GROUP];
+    for (int i = 0; i < count; ++i) {
+        in[i] = WqIn{problems[i].W, problems[i].N, K, p, gammas + 4 * i};
+        p += align256((size_t)problems[i].N * (size_t)K / 4);
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    rc = quant_weights_impl(*d, in, count, wdt, wq_ws, st);
+    if (rc) return rc;
+    if (decode_eligible(M, K)) {
+        // decode-sized: the fused launch quantizes X itself (per CTA)
+        DecodeJob jobs[BL_MAX_PREFILL_GROUP];
+        for (int i = 0; i < count; ++i)
+            jobs[i] = DecodeJob{in[i].packed, in[i].gamma, X, nullptr, problems[i].Y, nullptr, subln_gain, nullptr,
+                                problems[i].N, K};
+        return decode_launch(jobs, count, (int)M, subln_eps, false, st, xdt == BL_BF16 ? DEC_SRC_BF16 : DEC_SRC_F32,
+                             d->sms);
+    }
+    ActParams P;
+    P.count = 1;
+    P.M = (int)M;
+    P.eps = subln_eps;
+    P.p[0] = ActProblem{X, subln_gain, x_q, s, (int)K, 0};
+    // the act quant depends only on X: it may run while the weight pack
+    // finishes (programmatic dependent launch); the GEMM waits for both
+    rc = quant_act_impl(P, xdt, K, st, true);
+    if (rc) return rc;
+    PrefillJob jobs[BL_MAX_PREFILL_GROUP];
+    for (int i = 0; i < count; ++i) jobs[i] = PrefillJob{in[i].packed, in[i].gamma, problems[i].Y, nullptr, problems[i].N};
+    return prefill_launch_group(d->sms, jobs, count, x_q, s, M, K, st, PF_DEFAULT_TIMEOUT_NS, -1, true);
 }
 
 }  // extern "C"
@@ -617,7 +847,7 @@ extern "C" bl_status bl_quant_weights_noalloc(const void *W, bl_dtype wdt, int64
     void *scratch = nullptr;
     rc = noalloc_scratch(&scratch);
     if (rc) return rc;
-    return quant_weights_impl(*d, W, wdt, N, K, packed, gamma, scratch, (cudaStream_t)stream);
+    return quant_weights_one(*d, W, wdt, N, K, packed, gamma, scratch, (cudaStream_t)stream);
 }
 
 extern "C" bl_status bl_debug_forward_prefill(const uint8_t *packed, const float *gamma, const int8_t *x_q,

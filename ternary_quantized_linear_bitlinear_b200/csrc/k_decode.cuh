@@ -4,56 +4,80 @@
 //   acc[m, n] = sum_k x_q[m, k] * W_q[n, k];  Y[m, n] = acc * (gamma / s[m])
 //
 // The work is bound by streaming the packed weights from HBM (2 bits per
-// weight).  Design:
-//   - A CTA (8 warps) owns 8/G consecutive 32-row groups of one problem;
-//     their packed rows are one contiguous byte range, which one thread
-//     requests with cp.async.bulk copies into shared memory (one mbarrier per
-//     tile, bounded waits), so the memory system sees a few large requests
-//     per CTA and the warps issue no global loads for weights.
-//   - A warp owns 32 rows (two 16-row MMA tiles that share every x_q
-//     fragment); G warps split their K range (G picked per problem from K so
-//     that each warp has at most 4 steps of 256 k and a CTA at most 48 KiB
-//     of weights; the host raises G for launches too small to fill the GPU).
+// weight).  Design (one CTA per SM and launch, small enough that the CTA of
+// the next launch fits beside it):
+//   - Work unit: a group of 32 weight rows of one problem; its packed bytes
+//     are cut into chunks of 32 rows x 128 bytes (512 k), which a producer
+//     thread streams with 2-D TMA tensor loads (128-byte swizzle, L2
+//     evict-first: each byte is read once) through a ring of DEC_STAGES
+//     shared-memory stages, in group order.  The host cuts the flattened
+//     group list of all problems into one contiguous range per CTA with
+//     equal bytes.
+//   - Consumers: DEC_CWARPS warps take the ring's chunks round-robin
+//     (chunk j -> warp j mod DEC_CWARPS), so every warp streams at the same
+//     rate whatever the problems' K.  A warp's partial sums of a chunk go
+//     into the group's accumulator slot in shared memory (integer atomics:
+//     exact, any order); the warp that completes a group's last chunk
+//     rescales the slot and writes Y (lane = weight row: coalesced stores),
+//     zeroes the slot and only then frees its ring stage, which keeps a slot
+//     from being reused (slot = group ordinal mod DEC_STAGES) before its
+//     group is written out.
+//   - MACs on the tensor cores (mma.sync m16n8k32 s8): weight rows as A (two
+//     16-row tiles per chunk share every x_q fragment), tokens as B (8
+//     columns per tile, zero for m >= M).  The int32 sum is exact, so the k
+//     order inside a 256-k step may be permuted as long as A and B use the
+//     same permutation: the lane with k-slot t holds the packed bytes
+//     64t .. 64t + 15 of the step, and its B fragment reads those x_q bytes.
 //   - Unpacking costs 1-2 ALU ops per 4 weights: with the packed layout, word
 //     (w << (6 - 2j)) & 0xC0C0C0C0 puts the codes of k = 16w' + 4j .. 4j+3 in
-//     the top two bits of four bytes, i.e. the int8 values 64 * W_q.
-//   - The MACs run on the tensor cores (mma.sync m16n8k32 s8): W tile as A
-//     (16 rows), tokens as B (8 columns, zero for m >= M).  Because the
-//     int32 sum is exact, the k order inside a step may be permuted as long
-//     as A and B use the same permutation: thread t's A fragment for step
-//     pair c holds k = 64t + 16c + (0..15), and its B fragment reads exactly
-//     those x_q bytes.
-//   - x_q is staged once per CTA in shared memory (rows of round_up(K, 256)
-//     bytes, 16-byte chunks XOR-swizzled so that the B loads are free of
-//     bank conflicts).
-//   - acc = (sum of 64 * W_q * x_q) >> 6 exactly; the split-K partials meet
-//     in shared memory; the epilogue rescales and stores Y (and acc).
-//   - Fused variant (SRC = bf16 or f32 activations): step 2 runs inside the
-//     CTA instead of a separate launch.  One warp per token row (for one or
-//     two tokens without SubLN: the whole CTA) computes s = 127 / max|y|
-//     (y = x, or the SubLN RMSNorm of x) and writes x_q straight into the
-//     swizzled staging rows, with the same arithmetic as the stand-alone
-//     activation quantizer, while the weights stream in.
-//     Every CTA of a problem quantizes the (L2-resident) rows itself; the
-//     problem's first CTA also writes x_q and s to global memory on request.
+//     the top two bits of four bytes, i.e. the int8 values 64 * W_q; the sum
+//     is 64 * acc, exactly.
+//   - Lane (g, t) of an MMA tile reads weight rows pi(g) and pi(g) + 8 with
+//     pi(g) = (g >> 1) | ((g & 1) << 2): with the 128-byte swizzle, the eight
+//     lanes of each quarter warp then hit eight different bank quads.
+//   - x_q is staged once per CTA and problem in shared memory (rows of
+//     round_up(K, 256) bytes, 16-byte chunks XOR-swizzled so that the B loads
+//     are free of bank conflicts).  Fused variant (SRC = bf16 or f32
+//     activations): step 2 runs inside the CTA, one warp per token row, with
+//     the same arithmetic as the stand-alone activation quantizer; the CTA
+//     holding a problem's first group also writes x_q and s on request.
+//   - Launched as a programmatic dependent (BL_FWD_WEIGHTS_READY), the
+//     producer fills the ring before griddepcontrol.wait, so a launch streams
+//     its weights while the launch before it finishes; activations and s are
+//     read only after the wait.
+//   - Every mbarrier wait is bounded (globaltimer); a wait that gives up
+//     raises the device error word and the CTA's abort flag; the producer
+//     then waits (bounded) for its in-flight copies before the CTA exits.
 #pragma once
+
+#include <cuda.h>
 
 #include "bl_common.cuh"
 
 namespace bl {
 
-constexpr int DEC_THREADS = 256;
-constexpr int DEC_WARPS = DEC_THREADS / 32;
-constexpr int DEC_SMEM_LIMIT = 200 * 1024;  // weight tiles + staged x_q, per CTA
-constexpr int DEC_PF = 4;                   // target 256-k steps per warp (G is chosen from it)
-constexpr int DEC_W_CAP = 48 * 1024;        // weight bytes per CTA above which G grows (3 CTAs per SM)
+constexpr int DEC_CWARPS = 8;                         // consumer warps
+constexpr int DEC_THREADS = 32 * (DEC_CWARPS + 1);    // + the producer warp
+constexpr int DEC_ROWS = 32;                          // weight rows per group (two MMA tiles)
+constexpr int DEC_CB = 128;                           // packed bytes per row per chunk (512 k)
+constexpr int DEC_CHUNK = DEC_ROWS * DEC_CB;          // 4 KiB
+constexpr int DEC_STAGES = 12;                        // ring stages = accumulator slots
+constexpr int DEC_SLOT_LD = 36;                       // words per token row of a slot (bank spread)
+constexpr int DEC_MAX_PSLOTS = 8;                     // problems per CTA
+constexpr int DEC_MAX_CTAS = 320;
+constexpr int DEC_X_MAX = 150 * 1024;                 // staged activations per CTA
+constexpr int DEC_X_PAIR = 36 * 1024;                 // ... at most this keeps two CTAs per SM
 constexpr unsigned long long DEC_TIMEOUT_NS = 2000000000ull;
+
+__host__ __device__ constexpr int dec_slot_bytes(int nt) { return 8 * nt * DEC_SLOT_LD * 4; }
+__host__ __device__ constexpr int dec_fixed_smem(int nt) {
+    return DEC_STAGES * DEC_CHUNK + DEC_STAGES * dec_slot_bytes(nt);
+}
 
 // Activation source of a launch: pre-quantized x_q, or X to quantize in-kernel.
 enum : int { DEC_SRC_XQ = 0, DEC_SRC_BF16 = 1, DEC_SRC_F32 = 2 };
 
 struct DecodeProblem {
-    const uint8_t *packed;
     const float *gamma;
     const void *x;         // DEC_SRC_XQ: x_q [M, K] int8; else X [M, K] bf16 / f32
     float *s;              // DEC_SRC_XQ: s [M] in; else s [M] out or null
@@ -63,38 +87,21 @@ struct DecodeProblem {
     int8_t *xq_out;        // fused: x_q [M, K] out or null
     int N;
     int K;
-    int g_log2;     // log2(G): warps per row tile
-    int cta_begin;  // first CTA of this problem in the grouped grid
+    int gbase;             // first group of this problem in the flattened group list
 };
 
-constexpr int DEC_CTA_TABLE = 2048;  // grids up to this size look their problem up in a table
-
 struct DecodeParams {
+    CUtensorMap wmap[BL_MAX_GROUP];  // packed weights per problem: {K/4 bytes, N rows}, box 128 x 32, 128B swizzle
     DecodeProblem p[BL_MAX_GROUP];
     int count;
     int M;
-    int xq_off;  // shared-memory offset of the staged x_q (after the weight tiles)
-    int use_table;
-    float eps;   // fused: SubLN epsilon
-    unsigned char cta_problem[DEC_CTA_TABLE];
+    int ngroups;
+    int ncta;
+    float eps;                        // fused: SubLN epsilon
+    int cta_g[DEC_MAX_CTAS + 1];      // CTA c owns groups [cta_g[c], cta_g[c + 1])
 };
 
 __host__ __device__ inline int dec_row_stride(int K) { return (K + 255) & ~255; }
-
-__host__ __device__ inline int dec_glog(int K) {
-    // smallest G = 2^glog <= 8 with ceil(steps / G) <= DEC_PF and at most
-    // DEC_W_CAP bytes of weights per CTA (8 / G groups of 32 rows), so that
-    // three CTAs fit on an SM and a grouped launch stays one wave
-    int steps = (K + 255) >> 8, g = 0;
-    while (g < 3 && ((steps + (1 << g) - 1) >> g) > DEC_PF) ++g;
-    while (g < 3 && (DEC_WARPS >> g) * 32 * (K >> 2) > DEC_W_CAP) ++g;
-    return g;
-}
-
-constexpr int DEC_ROWS = 32;  // weight rows per warp
-
-// bytes of packed weights one CTA stages
-__host__ __device__ inline int dec_w_bytes(int K) { return (DEC_WARPS >> dec_glog(K)) * DEC_ROWS * (K >> 2); }
 
 __device__ __forceinline__ u32 dec_unpack(u32 w, int j) {
     // codes of k = 4j .. 4j+3 of this 16-weight word -> int8 lanes holding 64 * W_q
@@ -122,7 +129,6 @@ __device__ __forceinline__ u32 dec_x_bits(const uint4 &v, int j) {
 // (Four, not eight: the fused kernel runs once per CTA and its code is cold
 // in the instruction cache, so a shorter unrolled body is faster.)
 constexpr int DEC_QV = 4;
-constexpr int DEC_QB = 8;  // block-cooperative quantization: X vectors per thread (M * K / 8 <= 2048 for bf16)
 
 __device__ __forceinline__ void dec_load_block(uint4 (&c)[DEC_QV], const uint4 *xr, int nvec, int blk, int lane) {
 #pragma unroll
@@ -287,306 +293,407 @@ __device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, ui
     return s;
 }
 
+// Step 2 for all (problem, token) rows of a CTA at once, rows without SubLN:
+// every thread takes the 16-byte vectors t, t + DEC_THREADS, ... of the
+// concatenated rows with all its loads in flight together (one memory round
+// trip for the CTA instead of one per row and warp), the row maxima meet in
+// shared memory (max of the float bits of |x|), and each thread then
+// quantizes its vectors into the staging rows.  Same arithmetic as
+// dec_quant_row.  vbase[ps] = first vector of problem slot ps (vbase[np] =
+// the total, at most DEC_QBV * DEC_THREADS); s_amax[np * M] zeroed before.
+constexpr int DEC_QBV = 12;
+
+template <bool BF16>
+__device__ void dec_quant_block(const DecodeParams &P, int p_lo, int np, int g_begin, const int *s_xoff,
+                                const int *vbase, uint8_t *s_x, u32 *s_amax, float *s_sc, float (*s_f)[16]) {
+    constexpr int EPV = BF16 ? 8 : 4;
+    const int M = P.M, T = vbase[np];
+    const int lane = threadIdx.x & 31;
+    uint4 c[DEC_QBV];
+    int meta[DEC_QBV];  // (slot << 20) | (m << 16) | vector within the row; -1 past the end
+#pragma unroll
+    for (int i = 0; i < DEC_QBV; ++i) {
+        const int idx = (int)threadIdx.x + DEC_THREADS * i;
+        meta[i] = -1;
+        c[i] = make_uint4(0, 0, 0, 0);
+        if (idx < T) {
+            int ps = 0;
+            while (ps + 1 < np && idx >= vbase[ps + 1]) ++ps;
+            const int nvec = P.p[p_lo + ps].K / EPV;
+            const int local = idx - vbase[ps];
+            const int m = local / nvec, v = local - m * nvec;
+            meta[i] = (ps << 20) | (m << 16) | v;
+            c[i] = ldg_nc_v4(reinterpret_cast<const uint4 *>(P.p[p_lo + ps].x) + (size_t)m * nvec + v);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < DEC_QBV; ++i) {
+        if (DEC_THREADS * i >= T) break;  // uniform: no vector of this round is in range
+        u32 a = 0;
+#pragma unroll
+        for (int j = 0; j < EPV; ++j) a = max(a, dec_x_bits<BF16>(c[i], j) & 0x7fffffffu);
+        const int row = meta[i] < 0 ? -1 : ((meta[i] >> 20) * M + ((meta[i] >> 16) & 15));
+        const int row0 = __shfl_sync(0xffffffffu, row, 0);
+        if (__all_sync(0xffffffffu, row == row0)) {
+            a = __reduce_max_sync(0xffffffffu, a);
+            if (lane == 0 && row0 >= 0) atomicMax(&s_amax[row0], a);
+        } else if (row >= 0) {
+            atomicMax(&s_amax[row], a);
+        }
+    }
+    __syncthreads();
+    for (int r = threadIdx.x; r < np * M; r += DEC_THREADS) {
+        const int ps = r / M, m = r - ps * M;
+        const DecodeProblem &pr = P.p[p_lo + ps];
+        const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(s_amax[r]), 1e-5f));
+        s_sc[r] = s;
+        s_f[ps][m] = __fdiv_rn(*pr.gamma, s);
+        if (g_begin <= pr.gbase && pr.s != nullptr) pr.s[m] = s;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < DEC_QBV; ++i) {
+        if (meta[i] < 0) continue;
+        const int ps = meta[i] >> 20, m = (meta[i] >> 16) & 15, v = meta[i] & 0xffff;
+        const DecodeProblem &pr = P.p[p_lo + ps];
+        const int K = pr.K, RS = dec_row_stride(K);
+        const float s = s_sc[ps * M + m];
+        u32 word[EPV / 4];
+#pragma unroll
+        for (int q = 0; q < EPV / 4; ++q) {
+            u32 w = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                int qi = __float2int_rn(__fmul_rn(__uint_as_float(dec_x_bits<BF16>(c[i], 4 * q + j)), s));
+                qi = max(-128, min(127, qi));
+                w |= ((u32)qi & 0xffu) << (8 * j);
+            }
+            word[q] = w;
+        }
+        const int L = BF16 ? (v >> 1) : (v >> 2);
+        const int within = BF16 ? (v & 1) * 8 : (v & 3) * 4;
+        const int x = (((L >> 3) & 1) << 1) | (m & 1);
+        uint8_t *d = s_x + s_xoff[ps] + m * RS + ((((L & ~7) | ((L ^ x) & 7)) << 4) + within);
+        int8_t *gq = (g_begin <= pr.gbase && pr.xq_out != nullptr) ? pr.xq_out + (size_t)m * K : nullptr;
+        if (BF16) {
+            *reinterpret_cast<uint2 *>(d) = make_uint2(word[0], word[EPV / 4 - 1]);
+            if (gq) *reinterpret_cast<uint2 *>(gq + (size_t)v * 8) = make_uint2(word[0], word[EPV / 4 - 1]);
+        } else {
+            *reinterpret_cast<u32 *>(d) = word[0];
+            if (gq) *reinterpret_cast<u32 *>(gq + (size_t)v * 4) = word[0];
+        }
+    }
+}
+
+// problem owning flattened group g (binary search over the group bases)
+__device__ __forceinline__ int dec_problem_of(const DecodeParams &P, int g) {
+    int lo = 0, hi = P.count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.p[mid].gbase <= g) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ int dec_nchunks(int K) { return (K + 4 * DEC_CB - 1) / (4 * DEC_CB); }
+
+// Chunk cursor over a CTA's groups: group g of problem p, chunk kc.
+struct DecCursor {
+    int g, p, kc;
+};
+
+__device__ __forceinline__ void dec_advance(const DecodeParams &P, DecCursor &c, int by, int g_end) {
+    c.kc += by;
+    while (c.g < g_end) {
+        const int nch = dec_nchunks(P.p[c.p].K);
+        if (c.kc < nch) break;
+        c.kc -= nch;
+        ++c.g;
+        if (c.p + 1 < P.count && c.g >= P.p[c.p + 1].gbase) ++c.p;
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d_hint(u32 dst, const CUtensorMap *map, int x, int y, u32 bar, u64 pol) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3}], [%4], %5;"
+        ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar), "l"(pol)
+        : "memory");
+}
+
 // NT: 8-token column tiles (1: M <= 8, 2: M <= 16).  SRC: DEC_SRC_*.
 template <int NT, int SRC>
-__global__ void __launch_bounds__(DEC_THREADS, 3) k_decode(const __grid_constant__ DecodeParams P) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    __shared__ int s_red[DEC_WARPS][2][NT][4][32];
-    __shared__ __align__(8) u64 s_bar[DEC_WARPS];
-    __shared__ float s_f[16];
-    __shared__ u32 s_amax[16];
-    __shared__ float s_sc[16];
-    if (SRC != DEC_SRC_XQ && threadIdx.x < 16) s_amax[threadIdx.x] = 0u;
+__global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant__ DecodeParams P) {
+    extern __shared__ uint8_t dsm_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~(uintptr_t)1023);
+    __shared__ __align__(8) u64 s_full[DEC_STAGES];
+    __shared__ __align__(8) u64 s_empty[DEC_STAGES];
+    __shared__ int s_cnt[DEC_STAGES];
+    __shared__ float s_f[DEC_MAX_PSLOTS][16];
+    __shared__ int s_xoff[DEC_MAX_PSLOTS + 1];
+    __shared__ int s_vbase[DEC_MAX_PSLOTS + 1];
+    __shared__ u32 s_amax[DEC_MAX_PSLOTS * 16];
+    __shared__ float s_sc[DEC_MAX_PSLOTS * 16];
+    __shared__ volatile int s_abort;
 
     // a programmatically dependent launch that follows may start its prologue
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    const int b = blockIdx.x;
-    int pi;
-    if (P.use_table) {
-        pi = P.cta_problem[b];
-    } else {  // binary search over the CTA prefix
-        int lo = 0, hi = P.count - 1;
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (P.p[mid].cta_begin <= b) lo = mid; else hi = mid - 1;
-        }
-        pi = lo;
-    }
-    const DecodeProblem &pr = P.p[pi];
-    const int M = P.M, N = pr.N, K = pr.K;
-    const int glog = pr.g_log2, G = 1 << glog;
-    const int T = DEC_WARPS >> glog;  // 32-row groups per CTA
-    const int Kw = K >> 2;            // packed bytes per row
-    const int row_base = (b - pr.cta_begin) * T * DEC_ROWS;
-    const int rows = min(T * DEC_ROWS, N - row_base);
-    const int groups = (rows + DEC_ROWS - 1) / DEC_ROWS;
+    constexpr int SLOT_WORDS = dec_slot_bytes(NT) / 4;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g_begin = P.cta_g[blockIdx.x], g_end = P.cta_g[blockIdx.x + 1];
+    const int p_lo = dec_problem_of(P, g_begin), p_hi = dec_problem_of(P, g_end - 1);
+    const int np = p_hi - p_lo + 1;
+    const int M = P.M;
+    int *slots = reinterpret_cast<int *>(sm + DEC_STAGES * DEC_CHUNK);
+    uint8_t *s_x = sm + dec_fixed_smem(NT);
 
-    // One thread requests the CTA's weight rows, one bulk copy (and one
-    // mbarrier) per 32-row group, so each warp starts as soon as its rows land.
-    // It is lane 0 of the last warp: the fused path quantizes token row m in
-    // warp m, so for small M the first rows do not wait for the requests.
-    if (threadIdx.x == DEC_THREADS - 32) {
-        for (int i = 0; i < groups; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        const uint8_t *src = pr.packed + (size_t)row_base * Kw;
-        const u32 dst = smem_u32(smem);
-        const u64 policy = l2_policy_evict_first();  // weights are read once per launch
-        for (int i = 0; i < groups; ++i) {
-            const u32 nrows = (u32)min(DEC_ROWS, rows - DEC_ROWS * i);
-            const u32 bytes = nrows * (u32)Kw;
-            const u32 bar = smem_u32(&s_bar[i]);
-            mbar_arrive_expect_tx(bar, bytes);
-            const u32 off0 = (u32)(DEC_ROWS * i) * (u32)Kw;
-            for (u32 off = 0; off < bytes; off += 32768u) {
-                const u32 n = bytes - off < 32768u ? bytes - off : 32768u;
-                bulk_g2s_hint(dst + off0 + off, src + off0 + off, n, bar, policy);
-            }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < DEC_STAGES; ++s) {
+            mbar_init(smem_u32(&s_full[s]), 1);
+            mbar_init(smem_u32(&s_empty[s]), 1);
         }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        s_abort = 0;
+        int off = 0, vb = 0;
+        for (int i = 0; i < np; ++i) {
+            s_xoff[i] = off;
+            s_vbase[i] = vb;
+            off += M * dec_row_stride(P.p[p_lo + i].K);
+            vb += M * (P.p[p_lo + i].K / (SRC == DEC_SRC_F32 ? 4 : 8));
+        }
+        s_xoff[np] = off;
+        s_vbase[np] = vb;
+    }
+    if (threadIdx.x < DEC_MAX_PSLOTS * 16) s_amax[threadIdx.x] = 0u;
+    for (int i = threadIdx.x; i < DEC_STAGES * SLOT_WORDS; i += DEC_THREADS) slots[i] = 0;
+    if (threadIdx.x < DEC_STAGES) s_cnt[threadIdx.x] = 0;
+    __syncthreads();
+
+    // chunks of this CTA
+    long long total = 0;
+    {
+        int g = g_begin;
+        for (int p = p_lo; p <= p_hi; ++p) {
+            const int gnext = p + 1 < P.count ? min(P.p[p + 1].gbase, g_end) : g_end;
+            total += (long long)(gnext - g) * dec_nchunks(P.p[p].K);
+            g = gnext;
+        }
+    }
+
+    // ---- producer: the first ring-full before waiting for the previous grid
+    const bool producer = warp == DEC_CWARPS && lane == 0;
+    u64 policy = 0;
+    DecCursor pc{g_begin, p_lo, 0};
+    long long issued = 0;
+    auto issue = [&](long long j) {
+        const int s = (int)(j % DEC_STAGES);
+        const u32 bar = smem_u32(&s_full[s]);
+        mbar_arrive_expect_tx(bar, DEC_CHUNK);
+        tma_load_2d_hint(smem_u32(sm + s * DEC_CHUNK), &P.wmap[pc.p], pc.kc * DEC_CB,
+                         (pc.g - P.p[pc.p].gbase) * DEC_ROWS, bar, policy);
+        dec_advance(P, pc, 1, g_end);
+    };
+    if (producer) {
+        policy = l2_policy_evict_first();
+        for (int p = p_lo; p <= p_hi; ++p) asm volatile("prefetch.tensormap [%0];" ::"l"(&P.wmap[p]) : "memory");
+        for (; issued < total && issued < DEC_STAGES; ++issued) issue(issued);
     }
 
     // x_q and s may be produced by the kernel launched just before this one.
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // Stage x_q rows [0, M) into shared memory, swizzled, zero-padded to RS;
-    // float(gamma / s[m]) once per token.
-    const int RS = dec_row_stride(K);
-    uint8_t *s_xq = smem + P.xq_off;
+    // ---- activations of this CTA's problems, staged (and quantized) --------
+    bool block_quant = false;
     if (SRC != DEC_SRC_XQ) {
-        constexpr bool BF16 = SRC == DEC_SRC_BF16;
-        constexpr int EPV = BF16 ? 8 : 4;
-        const bool out = b == pr.cta_begin;
-        const int nvec = K / EPV;
-        const int tot = M * nvec;  // 16-byte vectors of X, rows contiguous
-        if (pr.gain == nullptr && M <= 2 && tot <= DEC_QB * DEC_THREADS) {
-            // fused step 2 for one or two tokens, no SubLN, all of X in
-            // registers: thread t holds vectors t + 256 i; one load round
-            // trip, per-row max by a warp reduction and a shared atomic (max
-            // of the float bits of |x|).  (Measured: faster than a warp per
-            // row for M <= 2, slower from M = 4 on.)
-            const uint4 *xv = reinterpret_cast<const uint4 *>(pr.x);
-            uint4 c[DEC_QB];
-#pragma unroll
-            for (int i = 0; i < DEC_QB; ++i) {
-                const int idx = (int)threadIdx.x + DEC_THREADS * i;
-                c[i] = idx < tot ? ldg_nc_v4(xv + idx) : make_uint4(0, 0, 0, 0);
-            }
-            __syncthreads();  // s_amax cleared
-            const int lane = threadIdx.x & 31;
-#pragma unroll
-            for (int i = 0; i < DEC_QB; ++i) {
-                const int idx = (int)threadIdx.x + DEC_THREADS * i;
-                if (DEC_THREADS * i >= tot) break;  // uniform: no vector of this round is in range
-                u32 a = 0;
-                const int m = idx < tot ? idx / nvec : -1;
-#pragma unroll
-                for (int j = 0; j < EPV; ++j) a = max(a, dec_x_bits<BF16>(c[i], j) & 0x7fffffffu);
-                // one shared atomic per warp when the warp's 32 vectors lie in one row
-                const int m0 = __shfl_sync(0xffffffffu, m, 0);
-                if (__all_sync(0xffffffffu, m == m0)) {
-                    a = __reduce_max_sync(0xffffffffu, a);
-                    if (lane == 0 && m0 >= 0) atomicMax(&s_amax[m0], a);
-                } else if (m >= 0) {
-                    atomicMax(&s_amax[m], a);
-                }
-            }
-            __syncthreads();
-            if (threadIdx.x < M) {
-                const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(s_amax[threadIdx.x]), 1e-5f));
-                s_sc[threadIdx.x] = s;
-                s_f[threadIdx.x] = __fdiv_rn(*pr.gamma, s);
-                if (out && pr.s != nullptr) pr.s[threadIdx.x] = s;
-            }
-            __syncthreads();
-#pragma unroll
-            for (int i = 0; i < DEC_QB; ++i) {
-                const int idx = (int)threadIdx.x + DEC_THREADS * i;
-                if (idx >= tot) continue;
-                const int m = idx / nvec, v = idx - m * nvec;
-                const float s = s_sc[m];
-                u32 word[EPV / 4];
-#pragma unroll
-                for (int q = 0; q < EPV / 4; ++q) {
-                    u32 w = 0;
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        int qi = __float2int_rn(__fmul_rn(__uint_as_float(dec_x_bits<BF16>(c[i], 4 * q + j)), s));
-                        qi = max(-128, min(127, qi));
-                        w |= ((u32)qi & 0xffu) << (8 * j);
-                    }
-                    word[q] = w;
-                }
-                const int L = BF16 ? (v >> 1) : (v >> 2);
-                const int within = BF16 ? (v & 1) * 8 : (v & 3) * 4;
+        bool gain = false;
+        for (int i = 0; i < np; ++i) gain |= P.p[p_lo + i].gain != nullptr;
+        block_quant = !gain && s_vbase[np] <= DEC_QBV * DEC_THREADS;
+    }
+    if (block_quant) {
+        dec_quant_block<SRC == DEC_SRC_BF16>(P, p_lo, np, g_begin, s_xoff, s_vbase, s_x, s_amax, s_sc, s_f);
+        // zero the padding chunks K .. round_up(K, 256) of every row
+        for (int r = warp; r < np * M; r += DEC_CWARPS + 1) {
+            const int ps = r / M, m = r - ps * M;
+            const int K = P.p[p_lo + ps].K, RS = dec_row_stride(K);
+            uint8_t *xs = s_x + s_xoff[ps];
+            for (int L = (K >> 4) + lane; L < (RS >> 4); L += 32) {
                 const int x = (((L >> 3) & 1) << 1) | (m & 1);
-                uint8_t *d = s_xq + m * RS + ((((L & ~7) | ((L ^ x) & 7)) << 4) + within);
-                int8_t *gq = out && pr.xq_out != nullptr ? pr.xq_out + (size_t)m * K : nullptr;
-                if (BF16) {
-                    *reinterpret_cast<uint2 *>(d) = make_uint2(word[0], word[EPV / 4 - 1]);
-                    if (gq) *reinterpret_cast<uint2 *>(gq + (size_t)v * 8) = make_uint2(word[0], word[EPV / 4 - 1]);
-                } else {
-                    *reinterpret_cast<u32 *>(d) = word[0];
-                    if (gq) *reinterpret_cast<u32 *>(gq + (size_t)v * 4) = word[0];
-                }
+                *reinterpret_cast<uint4 *>(xs + m * RS + (((L & ~7) | ((L ^ x) & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+    for (int r = warp; r < (block_quant ? 0 : np * M); r += DEC_CWARPS + 1) {
+        const int ps = r / M, m = r - ps * M;
+        const DecodeProblem &pr = P.p[p_lo + ps];
+        const int K = pr.K, RS = dec_row_stride(K);
+        uint8_t *xs = s_x + s_xoff[ps];
+        if (SRC != DEC_SRC_XQ) {
+            constexpr bool BF16 = SRC == DEC_SRC_BF16;
+            const bool out = g_begin <= pr.gbase;  // this CTA holds the problem's first group
+            const float s = dec_quant_row<BF16>(pr, m, K, RS, xs, P.eps, out, lane);
+            if (lane == 0) s_f[ps][m] = __fdiv_rn(*pr.gamma, s);
+            for (int L = (K >> 4) + lane; L < (RS >> 4); L += 32) {
+                const int x = (((L >> 3) & 1) << 1) | (m & 1);
+                *reinterpret_cast<uint4 *>(xs + m * RS + (((L & ~7) | ((L ^ x) & 7)) << 4)) = make_uint4(0, 0, 0, 0);
             }
         } else {
-            // fused step 2: warp w quantizes rows w, w + 8
-            const int lane = threadIdx.x & 31;
-            for (int m = threadIdx.x >> 5; m < M; m += DEC_WARPS) {
-                const float s = dec_quant_row<BF16>(pr, m, K, RS, s_xq, P.eps, out, lane);
-                if (lane == 0) s_f[m] = __fdiv_rn(*pr.gamma, s);
-            }
-        }
-        const int chunks = RS >> 4, kchunks = K >> 4;
-        for (int r = 0; r < M; ++r) {
-            for (int L = kchunks + (int)threadIdx.x; L < chunks; L += DEC_THREADS) {
-                const int x = (((L >> 3) & 1) << 1) | (r & 1);
-                *reinterpret_cast<uint4 *>(s_xq + r * RS + (((L & ~7) | ((L ^ x) & 7)) << 4)) =
-                    make_uint4(0, 0, 0, 0);
-            }
-        }
-    } else {
-        // every 16-byte chunk in flight at once (cp.async), one wait
-        const int chunks = RS >> 4;
-        const int kchunks = K >> 4;
-        for (int r = 0; r < M; ++r) {
-            const int8_t *src = static_cast<const int8_t *>(pr.x) + (size_t)r * K;
-            uint8_t *dst = s_xq + r * RS;
-            for (int L = threadIdx.x; L < chunks; L += DEC_THREADS) {
-                const int x = (((L >> 3) & 1) << 1) | (r & 1);
-                uint8_t *d = dst + (((L & ~7) | ((L ^ x) & 7)) << 4);
-                if (L < kchunks) {
+            const int8_t *src = static_cast<const int8_t *>(pr.x) + (size_t)m * K;
+            for (int L = lane; L < (RS >> 4); L += 32) {
+                const int x = (((L >> 3) & 1) << 1) | (m & 1);
+                uint8_t *d = xs + m * RS + (((L & ~7) | ((L ^ x) & 7)) << 4);
+                if (L < (K >> 4))
                     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(d)), "l"(src + L * 16)
                                  : "memory");
-                } else {
+                else
                     *reinterpret_cast<uint4 *>(d) = make_uint4(0, 0, 0, 0);
-                }
             }
+            if (lane == 0) s_f[ps][m] = __fdiv_rn(*pr.gamma, pr.s[m]);
         }
+    }
+    if (SRC == DEC_SRC_XQ) {
         asm volatile("cp.async.commit_group;" ::: "memory");
-        if (threadIdx.x < M) s_f[threadIdx.x] = __fdiv_rn(*pr.gamma, pr.s[threadIdx.x]);
         asm volatile("cp.async.wait_all;" ::: "memory");
     }
     __syncthreads();
 
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, t = lane & 3;
-    const int wg = warp >> glog, kslot = warp & (G - 1);
-    const int row0 = wg * DEC_ROWS;  // within the CTA
-    const int steps = (K + 255) >> 8;
-    const int nchunk64 = K >> 6;
-
-    // acc[tile][nt][4]: two 16-row tiles, each with two independent chains
-    int acc[2][NT][4], acc2[2][NT][4];
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[u][nt][i] = acc2[u][nt][i] = 0;
-
-    bool ok = true;
-    if (wg < groups) {
-        ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&s_bar[wg]), 0, DEC_TIMEOUT_NS, nullptr));
-        if (!ok && lane == 0) raise_device_error(DEVERR_TIMEOUT_PRODUCER);
+    if (warp == DEC_CWARPS) {
+        // ---------------------------------------------------------- producer
+        if (producer) {
+            bool failed = false;
+            for (; issued < total; ++issued) {
+                const int s = (int)(issued % DEC_STAGES);
+                // the stage's previous chunk has been consumed
+                if (!mbar_wait(smem_u32(&s_empty[s]), (u32)(((issued / DEC_STAGES) & 1) ^ 1), DEC_TIMEOUT_NS,
+                               &s_abort)) {
+                    failed = true;
+                    break;
+                }
+                issue(issued);
+            }
+            if (failed) {
+                raise_device_error(DEVERR_TIMEOUT_PRODUCER);
+                s_abort = 1;
+            }
+            if (s_abort) {
+                // drain: the last copies issued land before the CTA exits
+                for (long long j = issued - DEC_STAGES; j < issued; ++j)
+                    if (j >= 0)
+                        mbar_wait(smem_u32(&s_full[(int)(j % DEC_STAGES)]), (u32)((j / DEC_STAGES) & 1),
+                                  DEC_TIMEOUT_NS, nullptr);
+            }
+        }
+        return;
     }
 
-    if (ok && wg < groups) {
-        // rows g, g+8 (tile 0) and g+16, g+24 (tile 1)
-        const uint8_t *w0 = smem + (row0 + g) * Kw + t * 16;
-        const int Kw8 = 8 * Kw;
-        // B fragments: token rows g (and g + 8); chunk c of a step sits at
-        // 16 * (4t + (c ^ xb)) within the step's 256 bytes (the swizzle)
-        const bool tv0 = g < M, tv1 = NT > 1 && g + 8 < M;
-        const int xb0 = ((t >> 1) << 1) | (g & 1);
-        const int xb1 = ((t >> 1) << 1) | ((g + 8) & 1);
-        const uint8_t *xr0 = s_xq + g * RS + t * 64;
-        const uint8_t *xr1 = s_xq + (g + 8) * RS + t * 64;
-        int o0[4], o1[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            o0[c] = (c ^ xb0) << 4;
-            o1[c] = (c ^ xb1) << 4;
+    // ------------------------------------------------------------- consumers
+    const int g8 = lane >> 2, t = lane & 3;
+    const int pg = (g8 >> 1) | ((g8 & 1) << 2);       // physical row phase of MMA row g8
+    const int xb = ((t >> 1) << 1) | (g8 & 1);        // x_q swizzle of this lane's token rows
+    DecCursor cc{g_begin, p_lo, 0};
+    dec_advance(P, cc, warp, g_end);
+    for (long long j = warp; j < total; j += DEC_CWARPS) {
+        const int s = (int)(j % DEC_STAGES);
+        const bool ok = mbar_wait(smem_u32(&s_full[s]), (u32)((j / DEC_STAGES) & 1), DEC_TIMEOUT_NS, &s_abort);
+        if (!__all_sync(0xffffffffu, ok)) {
+            if (lane == 0) {
+                raise_device_error(DEVERR_TIMEOUT_MMA);
+                s_abort = 1;
+            }
+            break;
         }
+        const DecodeProblem &pr = P.p[cc.p];
+        const int ps = cc.p - p_lo;
+        const int K = pr.K, RS = dec_row_stride(K);
+        const int vb = min(DEC_CB, (K >> 2) - cc.kc * DEC_CB);  // valid packed bytes per row (>= 16)
+        const uint8_t *st = sm + s * DEC_CHUNK;
+        const uint8_t *xs = s_x + s_xoff[ps];
+        // two accumulator chains per tile at M <= 8 (alternate planes), one at
+        // M <= 16 (two token tiles already give four independent chains)
+        constexpr int CH = NT == 1 ? 2 : 1;
+        int acc[CH][2][NT][4];
+#pragma unroll
+        for (int c = 0; c < CH; ++c)
+#pragma unroll
+            for (int u = 0; u < 2; ++u)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) acc[c][u][nt][i] = 0;
 #pragma unroll 1
-        for (int s2 = kslot; s2 < steps; s2 += G) {
-            const bool kv = (s2 * 4 + t) < nchunk64;
+        for (int h2 = 0; h2 < 2; ++h2) {
+            if (64 * h2 >= vb) break;
+            // weights: physical rows pg + 8a (a = 0..3), this lane's 16 bytes of the half
             uint4 wv[4];
 #pragma unroll
-            for (int r4 = 0; r4 < 4; ++r4)
-                wv[r4] = kv ? *reinterpret_cast<const uint4 *>(w0 + r4 * Kw8 + s2 * 64) : make_uint4(0, 0, 0, 0);
-            const uint8_t *x0p = xr0 + s2 * 256;
-            const uint8_t *x1p = xr1 + s2 * 256;
+            for (int a = 0; a < 4; ++a)
+                wv[a] = *reinterpret_cast<const uint4 *>(st + (pg + 8 * a) * DEC_CB + (((4 * h2 + t) ^ pg) << 4));
+            // x_q of tokens g8 (+ 8): the 64 bytes of k-slot t in 256-k step s2
+            const int s2 = 2 * cc.kc + h2;
+            uint4 xv[NT][4];
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const uint4 x0 = tv0 ? *reinterpret_cast<const uint4 *>(x0p + o0[c]) : make_uint4(0, 0, 0, 0);
-                uint4 x1 = make_uint4(0, 0, 0, 0);
-                if (NT > 1 && tv1) x1 = *reinterpret_cast<const uint4 *>(x1p + o1[c]);
-                const u32 xq0[4] = {x0.x, x0.y, x0.z, x0.w};
-                const u32 xq1[4] = {x1.x, x1.y, x1.z, x1.w};
-                const u32 wr[4] = {(&wv[0].x)[c], (&wv[1].x)[c], (&wv[2].x)[c], (&wv[3].x)[c]};
+            for (int nt = 0; nt < NT; ++nt) {
+                const int m = g8 + 8 * nt;
+                const uint8_t *xr = xs + m * RS + s2 * 256 + t * 64;
 #pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    int(&A)[NT][4] = (c & 1) ? acc2[u] : acc[u];
+                for (int c = 0; c < 4; ++c)
+                    xv[nt][c] = m < M ? *reinterpret_cast<const uint4 *>(xr + ((c ^ xb) << 4)) : make_uint4(0, 0, 0, 0);
+            }
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const u32 a0 = dec_unpack(wr[2 * u], 2 * h), a2 = dec_unpack(wr[2 * u], 2 * h + 1);
-                        const u32 a1 = dec_unpack(wr[2 * u + 1], 2 * h), a3 = dec_unpack(wr[2 * u + 1], 2 * h + 1);
-                        mma_s8_16832(A[0], a0, a1, a2, a3, xq0[2 * h], xq0[2 * h + 1]);
-                        if (NT > 1) mma_s8_16832(A[NT - 1], a0, a1, a2, a3, xq1[2 * h], xq1[2 * h + 1]);
+            for (int u = 0; u < 2; ++u) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const u32 wa0 = (&wv[2 * u].x)[2 * hh], wa2 = (&wv[2 * u].x)[2 * hh + 1];
+                    const u32 wa1 = (&wv[2 * u + 1].x)[2 * hh], wa3 = (&wv[2 * u + 1].x)[2 * hh + 1];
+#pragma unroll
+                    for (int jp = 0; jp < 4; ++jp) {
+                        const u32 a0 = dec_unpack(wa0, jp), a1 = dec_unpack(wa1, jp);
+                        const u32 a2 = dec_unpack(wa2, jp), a3 = dec_unpack(wa3, jp);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            int(&A)[4] = acc[(jp & 1) % CH][u][nt];
+                            mma_s8_16832(A, a0, a1, a2, a3, (&xv[nt][2 * hh].x)[jp], (&xv[nt][2 * hh + 1].x)[jp]);
+                        }
                     }
                 }
             }
         }
-    }
-#pragma unroll
-    for (int u = 0; u < 2; ++u)
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) acc[u][nt][i] += acc2[u][nt][i];
-
-    // split-K reduction through shared memory
-    if (G > 1) {
+        // partial sums into the group's slot: row pg + 16u + 8(i >> 1), token 8nt + 2t + (i & 1)
+        const int go = cc.g - g_begin;
+        int *slot = slots + (go % DEC_STAGES) * SLOT_WORDS;
 #pragma unroll
         for (int u = 0; u < 2; ++u)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) s_red[warp][u][nt][i][lane] = acc[u][nt][i];
-        __syncthreads();
-        if (kslot == 0) {
-            for (int q = 1; q < G; ++q)
-#pragma unroll
-                for (int u = 0; u < 2; ++u)
-#pragma unroll
-                    for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) acc[u][nt][i] += s_red[warp + q][u][nt][i][lane];
+                for (int i = 0; i < 4; ++i) {
+                    const int v = CH == 2 ? acc[0][u][nt][i] + acc[CH - 1][u][nt][i] : acc[0][u][nt][i];
+                    atomicAdd(slot + (8 * nt + 2 * t + (i & 1)) * DEC_SLOT_LD + pg + 16 * u + 8 * (i >> 1), v);
+                }
+        __syncwarp();
+        int last = 0;
+        if (lane == 0) {
+            __threadfence_block();
+            last = atomicAdd(&s_cnt[go % DEC_STAGES], 1) == dec_nchunks(K) - 1;
         }
-    }
-    if (kslot != 0 || !ok || wg >= groups) return;
-
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) {
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            const int m = nt * 8 + 2 * t + e;
-            if (m >= M) continue;
-            const float f = s_f[m];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const int n = row_base + row0 + 16 * u + g + 8 * hh;
-                    if (n < N) {
-                        const int a_ = acc[u][nt][2 * hh + e] >> 6;  // exact: the sum is a multiple of 64
-                        pr.Y[(size_t)m * N + n] = __fmul_rn(__int2float_rn(a_), f);
-                        if (pr.acc) pr.acc[(size_t)m * N + n] = a_;
-                    }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+            // every chunk of the group has been added: rescale and write it out
+            __threadfence_block();
+            const int n = (cc.g - pr.gbase) * DEC_ROWS + lane;
+            for (int m = 0; m < M; ++m) {
+                const int a = slot[m * DEC_SLOT_LD + lane] >> 6;  // exact: the sum is a multiple of 64
+                slot[m * DEC_SLOT_LD + lane] = 0;
+                if (n < pr.N) {
+                    pr.Y[(size_t)m * pr.N + n] = __fmul_rn(__int2float_rn(a), s_f[ps][m]);
+                    if (pr.acc) pr.acc[(size_t)m * pr.N + n] = a;
                 }
             }
+            if (lane == 0) s_cnt[go % DEC_STAGES] = 0;
+            __syncwarp();
         }
+        if (lane == 0) mbar_arrive(smem_u32(&s_empty[s]));
+        dec_advance(P, cc, DEC_CWARPS, g_end);
     }
 }
 

@@ -118,6 +118,7 @@ struct PrefillParams {
     unsigned long long timeout_ns;
     long long dbg_skip_iter;  // >= 0: the producers never issue this k-iteration (bounded-wait test)
     int y_tma;                // 1: Y written by TMA stores (every N % 4 == 0 and no acc output)
+    int glu;                  // 1: gated FFN tiles (below): problem 0 = gate, 1 = up, output h
 };
 
 // ---------------------------------------------------------------------------
@@ -194,6 +195,18 @@ __device__ __forceinline__ void tc2_mma_i8_ss(u32 d_tmem, unsigned long long a_d
         : "memory");
 }
 
+// Same with bf16 operands and f32 accumulation (kind::f16): the backward
+// product dX = dY (gamma W_q).
+__device__ __forceinline__ void tc2_mma_f16_ss(u32 d_tmem, unsigned long long a_desc, unsigned long long b_desc,
+                                               u32 idesc, u32 accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // arrive (once the MMAs issued so far complete) on the barrier at this
 // shared-memory offset in both CTAs of the pair
 __device__ __forceinline__ void tc2_commit_pair(u32 bar) {
@@ -232,14 +245,22 @@ __device__ __forceinline__ unsigned long long smem_desc_k_sw128(u32 saddr) {
 }
 
 // Instruction descriptor, kind::i8: D s32, A s8, B s8, both K-major,
-// N = PF_BN, M = 2 x PF_BM (the pair).
+// N = PF_BN, M = 2 x PF_BM (the pair).  BWD (kind::f16): D f32, A bf16,
+// B bf16, same shape.
+template <bool BWD>
 __host__ __device__ constexpr u32 pf_idesc() {
-    return (2u << 4)                          // D format: s32
-           | (1u << 7)                        // A format: signed 8-bit
-           | (1u << 10)                       // B format: signed 8-bit
+    return (BWD ? (1u << 4) : (2u << 4))      // D format: f32 / s32
+           | (1u << 7)                        // A format: bf16 / signed 8-bit
+           | (1u << 10)                       // B format: bf16 / signed 8-bit
            | ((u32)(PF_BN >> 3) << 17)        // N >> 3
            | ((u32)((2 * PF_BM) >> 4) << 24); // M >> 4
 }
+
+// Backward mode: a pipeline stage covers 64 of the reduction index n (bf16:
+// the same 128 bytes per operand row as 128 int8); its packed stage holds
+// 64 rows n x 128 k of the forward's packed matrix (32 bytes per row).
+constexpr int PF_BWD_BK = 64;
+constexpr int PF_BWD_P_BYTES = PF_BWD_BK * PF_BNH / 4;  // 2 KiB
 
 // ---------------------------------------------------------------------------
 
@@ -250,6 +271,14 @@ __device__ __forceinline__ int pf_prob_of(const PrefillParams &p, int nt) {
     return pi;
 }
 
+// BWD = false: the forward (int8 x_q against expanded 64 * W_q, acc int32).
+// BWD = true: the backward product dX = dY (gamma W_q): A = dY bf16 [M, N]
+// (the reduction index n contiguous), B = W_q^T as bf16 +-1 / 0, expanded
+// from the forward's packed rows (each B row is an input feature k, read
+// across 64 packed rows n per stage), f32 accumulators; epilogue dX =
+// float(acc * gamma).  Everything else (pairs, pipelines, TMEM, waits) is
+// shared.
+template <bool BWD>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
     k_prefill_tc(const __grid_constant__ PrefillMaps maps, const __grid_constant__ PrefillParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -316,11 +345,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
             bool failed = false;
             for (int tile = cid; tile < total_tiles && !failed; tile += ncl) {
                 const int nt = tile % p.n_tiles, mt = tile / p.n_tiles;
-                const int pi = pf_prob_of(p, nt);
+                // gated tiles: the leader's half of B is 128 gate rows, the
+                // peer's the same 128 rows of up
+                const int pi = (!BWD && p.glu) ? (int)rank : pf_prob_of(p, nt);
                 const CUtensorMap *tmw = &maps.w[pi];
-                const int ntl = nt - p.prob[pi].nt_begin;
+                const int ntl = (!BWD && p.glu) ? nt : nt - p.prob[pi].nt_begin;
                 const int arow = mt * (2 * PF_BM) + (int)rank * PF_BM;   // this CTA's tokens
-                const int brow = ntl * PF_BN + (int)rank * PF_BNH;       // this CTA's weight rows
+                const int brow = (!BWD && p.glu) ? ntl * PF_BNH : ntl * PF_BN + (int)rank * PF_BNH;  // this CTA's B rows
                 for (int ks = 0; ks < KS; ++ks, ++it) {
                     const int s = (int)(it % PF_STAGES);
                     const u32 ph = (u32)((it / PF_STAGES) & 1);
@@ -329,9 +360,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
                         break;
                     }
                     if (it == p.dbg_skip_iter) continue;  // test hook: this stage never arrives
-                    mbar_arrive_expect_tx(BAR_FULL(s), PF_A_BYTES + PF_P_BYTES);
-                    tma_load_2d(sbase + PF_OFF_A + s * PF_A_BYTES, &maps.x, ks * PF_BK, arow, BAR_FULL(s));
-                    tma_load_2d(sbase + PF_OFF_P + s * PF_P_BYTES, tmw, ks * (PF_BK / 4), brow, BAR_FULL(s));
+                    if (BWD) {
+                        // dY columns n = 64 ks ..; packed rows n = 64 ks .., bytes of k = brow .. brow + 127
+                        mbar_arrive_expect_tx(BAR_FULL(s), PF_A_BYTES + PF_BWD_P_BYTES);
+                        tma_load_2d(sbase + PF_OFF_A + s * PF_A_BYTES, &maps.x, ks * PF_BWD_BK, arow, BAR_FULL(s));
+                        tma_load_2d(sbase + PF_OFF_P + s * PF_P_BYTES, tmw, brow / 4, ks * PF_BWD_BK, BAR_FULL(s));
+                    } else {
+                        mbar_arrive_expect_tx(BAR_FULL(s), PF_A_BYTES + PF_P_BYTES);
+                        tma_load_2d(sbase + PF_OFF_A + s * PF_A_BYTES, &maps.x, ks * PF_BK, arow, BAR_FULL(s));
+                        tma_load_2d(sbase + PF_OFF_P + s * PF_P_BYTES, tmw, ks * (PF_BK / 4), brow, BAR_FULL(s));
+                    }
                 }
             }
             if (failed) {
@@ -348,7 +386,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0 && rank == 0) {
-            const u32 idesc = pf_idesc();
+            const u32 idesc = pf_idesc<BWD>();
             long long it = 0;
             int tc = 0;
             bool failed = false, issued = false;
@@ -380,8 +418,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
                     const u32 bstage = sbase + PF_OFF_B + a * PF_B_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < PF_BK / 32; ++kk) {
-                        tc2_mma_i8_ss(d_tmem, smem_desc_k_sw128(astage + kk * 32), smem_desc_k_sw128(bstage + kk * 32),
-                                      idesc, (ks | kk) != 0 ? 1u : 0u);
+                        if (BWD)
+                            tc2_mma_f16_ss(d_tmem, smem_desc_k_sw128(astage + kk * 32),
+                                           smem_desc_k_sw128(bstage + kk * 32), idesc, (ks | kk) != 0 ? 1u : 0u);
+                        else
+                            tc2_mma_i8_ss(d_tmem, smem_desc_k_sw128(astage + kk * 32),
+                                          smem_desc_k_sw128(bstage + kk * 32), idesc, (ks | kk) != 0 ? 1u : 0u);
                     }
                     tc2_commit_pair(BAR_EMPTY(s));
                     tc2_commit_pair(BAR_BEMPTY(a));
@@ -417,10 +459,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
                     failed = true;
                     break;
                 }
+                uint8_t *brow = sm + PF_OFF_B + a * PF_B_BYTES + row * 128;
+                if (BWD) {
+                    // B row = input feature k (this thread's `row` of the tile's
+                    // 128): the codes of (n, k) for the stage's 64 n, from word
+                    // k / 16 of each packed row n (32 bytes per row in the
+                    // stage; the warp's 32 rows share two words: broadcasts),
+                    // as bf16 0 / +1 / -1, 8 n per 16-byte chunk
+                    const u32 *pw = reinterpret_cast<const u32 *>(sm + PF_OFF_P + s * PF_P_BYTES) + (row >> 4);
+                    const int sh = 8 * (row & 3) + 2 * ((row >> 2) & 3);
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        u32 o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const u32 c0 = (pw[8 * (8 * c + 2 * e)] >> sh) & 3u;
+                            const u32 c1 = (pw[8 * (8 * c + 2 * e + 1)] >> sh) & 3u;
+                            const u32 b0 = (c0 & 1u) * 0x3F80u | ((c0 & 2u) << 14);
+                            const u32 b1 = (c1 & 1u) * 0x3F80u | ((c1 & 2u) << 14);
+                            o[e] = b0 | (b1 << 16);
+                        }
+                        *reinterpret_cast<uint4 *>(brow + ((c ^ rsw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(BAR_BREADY(a), 0);
+                    continue;
+                }
                 const uint4 *src = reinterpret_cast<const uint4 *>(sm + PF_OFF_P + s * PF_P_BYTES + row * (PF_BK / 4));
                 const uint4 v0 = src[0], v1 = src[1];
                 const u32 w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-                uint8_t *brow = sm + PF_OFF_B + a * PF_B_BYTES + row * 128;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     // packed word i = k 16i .. 16i+15 = 16-byte chunk i of the row
@@ -454,6 +522,61 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
         bool failed = false;
         for (int tile = cid; tile < total_tiles && !failed; tile += ncl, ++tc) {
             const int nt = tile % p.n_tiles, mt = tile / p.n_tiles;
+            if (!BWD && p.glu) {
+                // Gated FFN tile: TMEM columns 0..127 hold gate, 128..255 up,
+                // for the same 128 rows (n).  Each thread owns one token:
+                //   h = float(float(r * r) * u), r = max(g, 0), with
+                //   g = float(float(acc_g) * float(gamma_g / s)), u likewise,
+                // the bits the plain epilogue would store for gate and up.
+                // This warp writes h columns 64 * half .. + 63 of the tile.
+                const int b = tc & 1;
+                const u32 cph = (u32)((tc >> 1) & 1);
+                const int mrow0 = mt * (2 * PF_BM) + (int)rank * PF_BM + q * 32;
+                const int m = mrow0 + lane;
+                const float sm_ = m < p.M ? p.s[m] : 1.f;
+                const float fg = __fmul_rn(__fdiv_rn(*p.prob[0].gamma, sm_), 0.015625f);
+                const float fu = __fmul_rn(__fdiv_rn(*p.prob[1].gamma, sm_), 0.015625f);
+                bool ok = mbar_wait(BAR_ACCFULL(b), cph, TO, s_abort);
+                if (!__all_sync(0xffffffffu, ok)) {
+                    failed = true;
+                    break;
+                }
+                tc_fence_after();
+                const int n0 = nt * PF_BNH + half * (PF_BNH / 2);
+#pragma unroll 1
+                for (int c0 = 0; c0 < PF_BNH / 2; c0 += 32) {
+                    u32 rg[32], ru[32];
+                    const u32 ta = tmem + ((u32)(q * 32) << 16) + b * PF_BN + half * (PF_BNH / 2) + c0;
+                    tc_ld_32x32b_x32(ta, rg);
+                    tc_ld_32x32b_x32(ta + PF_BNH, ru);
+                    tc_wait_ld();
+                    if (c0 + 32 == PF_BNH / 2) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(BAR_ACCEMPTY(b), 0);
+                    }
+                    if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    __syncwarp();
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        float hv[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float g = __fmul_rn(__int2float_rn((int)rg[4 * c + e]), fg);
+                            const float u = __fmul_rn(__int2float_rn((int)ru[4 * c + e]), fu);
+                            const float r = g > 0.f ? g : 0.f;
+                            hv[e] = __fmul_rn(__fmul_rn(r, r), u);
+                        }
+                        *reinterpret_cast<float4 *>(ystage + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                            make_float4(hv[0], hv[1], hv[2], hv[3]);
+                    }
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) tma_store_2d(&maps.y[0], n0 + c0, mrow0, ystage_s);
+                    __syncwarp();
+                }
+                continue;
+            }
             const PrefillProb &pp = p.prob[pf_prob_of(p, nt)];
             const int pN = pp.N;
             const int ntl = nt - pp.nt_begin;
@@ -464,8 +587,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
             const int mrow0 = mt * (2 * PF_BM) + (int)rank * PF_BM + q * 32;  // this warp's first token
             const int m = mrow0 + lane;                   // this thread's token
             const bool mvalid = m < p.M;
-            // float(gamma / s[m]) / 64 (exact)
-            const float f = mvalid ? __fmul_rn(__fdiv_rn(gamma, p.s[m]), 0.015625f) : 0.f;
+            // forward: float(gamma / s[m]) / 64 (exact); backward: gamma
+            const float f = BWD ? gamma : (mvalid ? __fmul_rn(__fdiv_rn(gamma, p.s[m]), 0.015625f) : 0.f);
+            auto cvt = [&](u32 v) {
+                return BWD ? __fmul_rn(__uint_as_float(v), f) : __fmul_rn(__int2float_rn((int)v), f);
+            };
             bool ok = mbar_wait(BAR_ACCFULL(b), cph, TO, s_abort);
             if (!__all_sync(0xffffffffu, ok)) {
                 failed = true;
@@ -493,10 +619,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
                     for (int c = 0; c < 8; ++c) {
                         float4 o;
-                        o.x = __fmul_rn(__int2float_rn((int)r[4 * c + 0]), f);
-                        o.y = __fmul_rn(__int2float_rn((int)r[4 * c + 1]), f);
-                        o.z = __fmul_rn(__int2float_rn((int)r[4 * c + 2]), f);
-                        o.w = __fmul_rn(__int2float_rn((int)r[4 * c + 3]), f);
+                        o.x = cvt(r[4 * c + 0]);
+                        o.y = cvt(r[4 * c + 1]);
+                        o.z = cvt(r[4 * c + 2]);
+                        o.w = cvt(r[4 * c + 3]);
                         *reinterpret_cast<float4 *>(ystage + lane * 128 + ((c ^ (lane & 7)) << 4)) = o;
                     }
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -507,10 +633,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
                         for (int j = 0; j < 32; j += 4) {
                             float4 o;
-                            o.x = __fmul_rn(__int2float_rn((int)r[j + 0]), f);
-                            o.y = __fmul_rn(__int2float_rn((int)r[j + 1]), f);
-                            o.z = __fmul_rn(__int2float_rn((int)r[j + 2]), f);
-                            o.w = __fmul_rn(__int2float_rn((int)r[j + 3]), f);
+                            o.x = cvt(r[j + 0]);
+                            o.y = cvt(r[j + 1]);
+                            o.z = cvt(r[j + 2]);
+                            o.w = cvt(r[j + 3]);
                             *reinterpret_cast<float4 *>(yrow + c0 + j) = o;
                             if (arow) {
                                 // exact: the sums are multiples of 64
@@ -522,7 +648,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
 #pragma unroll
                         for (int j = 0; j < 32; ++j) {
                             if (n0 + c0 + j < pN) {
-                                yrow[c0 + j] = __fmul_rn(__int2float_rn((int)r[j]), f);
+                                yrow[c0 + j] = cvt(r[j]);
                                 if (arow) arow[c0 + j] = (int)r[j] >> 6;
                             }
                         }
@@ -586,7 +712,10 @@ inline EncodeTiledFn encode_tiled_fn() {
 
 inline cudaError_t prefill_setup() {
     if (encode_tiled_fn() == nullptr) return cudaErrorNotSupported;
-    return cudaFuncSetAttribute(k_prefill_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM_BYTES);
+    if (cudaFuncSetAttribute(k_prefill_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM_BYTES) !=
+        cudaSuccess)
+        return cudaErrorUnknown;
+    return cudaFuncSetAttribute(k_prefill_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM_BYTES);
 }
 
 // Cluster pairs that can be resident at once on the current device (the
@@ -602,7 +731,7 @@ inline int prefill_max_pairs(int sms) {
     cfg.blockDim = dim3(PF_THREADS);
     cfg.dynamicSmemBytes = PF_SMEM_BYTES;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, k_prefill_tc, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, k_prefill_tc<false>, &cfg) != cudaSuccess || n < 1) {
         (void)cudaGetLastError();
         n = sms / 2;
     }
@@ -698,7 +827,142 @@ inline bl_status prefill_launch_group(int sms, const PrefillJob *jobs, int count
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, k_prefill_tc, maps, p) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, k_prefill_tc<false>, maps, p) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+// Gated FFN: h [M, F] = relu(Y_gate)^2 * Y_up from one launch whose pair
+// tiles hold 128 gate and the same 128 up rows (F % 64 == 0: every h row is
+// a multiple of 16 bytes, stored by TMA).
+inline bl_status prefill_launch_glu(int sms, const uint8_t *packed_gate, const float *gamma_gate,
+                                    const uint8_t *packed_up, const float *gamma_up, const int8_t *x_q,
+                                    const float *s, int64_t M, int64_t F, int64_t K, float *h, cudaStream_t st,
+                                    bool pdl = false) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (enc == nullptr) return BL_ERR_CUDA;
+    PrefillMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    PrefillParams p;
+    memset(&p, 0, sizeof(p));
+    const cuuint32_t es[2] = {1, 1};
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)K};
+        const cuuint32_t box[2] = {(cuuint32_t)PF_BK, (cuuint32_t)PF_BM};
+        if (enc(&maps.x, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t *>(x_q), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return BL_ERR_CUDA;
+    }
+    const uint8_t *pk[2] = {packed_gate, packed_up};
+    for (int i = 0; i < 2; ++i) {
+        const cuuint64_t gdim[2] = {(cuuint64_t)(K / 4), (cuuint64_t)F};
+        const cuuint64_t gstride[1] = {(cuuint64_t)(K / 4)};
+        const cuuint32_t box[2] = {(cuuint32_t)(PF_BK / 4), (cuuint32_t)PF_BNH};
+        if (enc(&maps.w[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(pk[i]), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return BL_ERR_CUDA;
+    }
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)F, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)F * 4};
+        const cuuint32_t box[2] = {32, 32};
+        if (enc(&maps.y[0], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, h, gdim, gstride, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+            CUDA_SUCCESS)
+            return BL_ERR_CUDA;
+    }
+    p.prob[0] = PrefillProb{gamma_gate, h, nullptr, (int)F, 0};
+    p.prob[1] = PrefillProb{gamma_up, h, nullptr, (int)F, 0};
+    p.nprob = 2;
+    p.glu = 1;
+    p.y_tma = 1;
+    p.s = s;
+    p.M = (int)M;
+    p.K = (int)K;
+    const int64_t n_tiles = (F + PF_BNH - 1) / PF_BNH;
+    const int64_t m_tiles = (M + 2 * PF_BM - 1) / (2 * PF_BM);
+    if (n_tiles * m_tiles > 0x7fffffffLL) return BL_ERR_SHAPE;
+    p.n_tiles = (int)n_tiles;
+    p.m_tiles = (int)m_tiles;
+    p.k_stages = (int)((K + PF_BK - 1) / PF_BK);
+    p.timeout_ns = PF_DEFAULT_TIMEOUT_NS;
+    p.dbg_skip_iter = -1;
+    const int64_t tiles = n_tiles * m_tiles;
+    const int pairs = prefill_max_pairs(sms);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2u * (unsigned)(tiles < pairs ? tiles : pairs));
+    cfg.blockDim = dim3(PF_THREADS);
+    cfg.dynamicSmemBytes = PF_SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, k_prefill_tc<false>, maps, p) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+}
+
+// Backward dX [M, K] = dY [M, N] (gamma W_q) on the tensor cores: bf16 dY,
+// the forward's packed W [N, K/4], f32 accumulation (N % 8 == 0: the dY
+// rows are multiples of 16 bytes for TMA).
+inline bl_status prefill_launch_bwd(int sms, const void *dY, const uint8_t *packed, const float *gamma, int64_t M,
+                                    int64_t N, int64_t K, float *dX, cudaStream_t st) {
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (enc == nullptr) return BL_ERR_CUDA;
+    PrefillMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    PrefillParams p;
+    memset(&p, 0, sizeof(p));
+    const cuuint32_t es[2] = {1, 1};
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)N, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)N * 2};
+        const cuuint32_t box[2] = {(cuuint32_t)PF_BWD_BK, (cuuint32_t)PF_BM};
+        if (enc(&maps.x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(dY), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return BL_ERR_CUDA;
+    }
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
+        const cuuint64_t gstride[1] = {(cuuint64_t)(K / 4)};
+        const cuuint32_t box[2] = {(cuuint32_t)(PF_BNH / 4), (cuuint32_t)PF_BWD_BK};  // 128 k x 64 n
+        if (enc(&maps.w[0], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return BL_ERR_CUDA;
+    }
+    {
+        const cuuint64_t gdim[2] = {(cuuint64_t)K, (cuuint64_t)M};
+        const cuuint64_t gstride[1] = {(cuuint64_t)K * 4};
+        const cuuint32_t box[2] = {32, 32};
+        if (enc(&maps.y[0], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dX, gdim, gstride, box, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return BL_ERR_CUDA;
+    }
+    p.prob[0] = PrefillProb{gamma, dX, nullptr, (int)K, 0};
+    p.nprob = 1;
+    p.y_tma = 1;
+    p.M = (int)M;
+    p.K = (int)N;
+    const int64_t n_tiles = (K + PF_BN - 1) / PF_BN;
+    const int64_t m_tiles = (M + 2 * PF_BM - 1) / (2 * PF_BM);
+    if (n_tiles * m_tiles > 0x7fffffffLL) return BL_ERR_SHAPE;
+    p.n_tiles = (int)n_tiles;
+    p.m_tiles = (int)m_tiles;
+    p.k_stages = (int)((N + PF_BWD_BK - 1) / PF_BWD_BK);
+    p.timeout_ns = PF_DEFAULT_TIMEOUT_NS;
+    p.dbg_skip_iter = -1;
+    const int64_t tiles = n_tiles * m_tiles;
+    const int pairs = prefill_max_pairs(sms);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2u * (unsigned)(tiles < pairs ? tiles : pairs));
+    cfg.blockDim = dim3(PF_THREADS);
+    cfg.dynamicSmemBytes = PF_SMEM_BYTES;
+    cfg.stream = st;
+    return cudaLaunchKernelEx(&cfg, k_prefill_tc<true>, maps, p) == cudaSuccess ? BL_OK : BL_ERR_CUDA;
 }
 
 inline bl_status prefill_launch(int sms, const uint8_t *packed, const float *gamma, const int8_t *x_q, const float *s,

@@ -2,12 +2,15 @@
 // 2-bit packing ("Distillix" README, 1. BitNet b1.58 Core; "bitone" README,
 // Forward pass; "SLM750-Edge" section 3.1).
 //
-// Two launches, both on the caller's stream:
+// Two launches, both on the caller's stream, each over one or several
+// weight matrices (up to WQ_MAX_JOBS: e.g. the projections of a layer, so
+// their reduction latency chains overlap):
 //   k_absmean_partial  one pass over W: exact per-block sum of |w| as a
 //                      384-bit fixed-point integer in units of 2^-149; the
-//                      last block to finish (ticket counter) sums the block
-//                      partials, rounds once to double, gamma = float(S / n)
-//                      + 1e-5f, and the float threshold T with
+//                      last block of a matrix to finish (ticket counter)
+//                      sums its block partials, rounds once to double,
+//                      gamma = float(S / n) + 1e-5f, and the float
+//                      threshold T with
 //                      |w| >= T  <=>  float(|w|/gamma) > 0.5
 //   k_ternary_pack     second pass over W: code = sign(w) * (|w| >= T), four
 //                      codes per byte in the packed word layout; launched as
@@ -30,10 +33,35 @@ namespace bl {
 constexpr int WQ_THREADS = 512;
 constexpr int WQ_WINDOW = 25;       // fast path: base <= e <= base + 25
 constexpr int WQ_PART_LIMBS = 6;    // per-block partial, 384 bits
-constexpr int WQ_MAX_BLOCKS = 1024;
+constexpr int WQ_MAX_BLOCKS = 1024; // over all matrices of a launch
+constexpr int WQ_MAX_JOBS = 8;      // weight matrices per launch
 constexpr size_t WQ_WS_PARTIALS = (size_t)WQ_MAX_BLOCKS * WQ_PART_LIMBS * 8;
-constexpr size_t WQ_WS_BYTES = WQ_WS_PARTIALS + 256;  // + threshold word, ticket counter
-constexpr size_t WQ_WS_TICKET = WQ_WS_PARTIALS + 128;  // u32, zeroed by the host before each reduction
+constexpr size_t WQ_WS_BYTES = WQ_WS_PARTIALS + 256;  // + threshold words, ticket counters
+constexpr size_t WQ_WS_TICKET = WQ_WS_PARTIALS + 128;  // u32 per matrix, zeroed by the host before each reduction
+
+// One weight matrix of a (grouped) quantization launch: blocks
+// [blk0, blk0 + nblk) of the reduction grid sum it; its packed words are
+// words [word0, word0 + nwords) of the pack grid's index space.
+struct WqJob {
+    const uint4 *W;
+    long long nvec;   // 16-byte vectors
+    long long n;      // weights
+    float *gamma;
+    u32 *packed;
+    long long nwords; // packed 32-bit words (16 weights each)
+    long long word0;
+    int blk0;
+    int nblk;
+};
+
+struct WqParams {
+    WqJob j[WQ_MAX_JOBS];
+    int count;
+    long long total_words;
+    u64 *partials;    // [WQ_MAX_BLOCKS][WQ_PART_LIMBS]
+    u32 *thresh;      // [WQ_MAX_JOBS]
+    u32 *tickets;     // [WQ_MAX_JOBS]
+};
 
 // Float bits of the j-th element of a 16-byte vector.
 template <bool BF16>
@@ -105,11 +133,7 @@ __device__ void wq_finalize_block(const u64 *partials, int nblocks, long long n,
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const uint4 *__restrict__ W, long long nvec,
-                                                                 long long n, u64 *__restrict__ partials,
-                                                                 float *__restrict__ gamma_out,
-                                                                 u32 *__restrict__ ws_thresh,
-                                                                 u32 *__restrict__ ticket) {
+__global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const __grid_constant__ WqParams P) {
     // the pack kernel may start loading W while this grid runs
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int EPV = BF16 ? 8 : 4;  // elements per 16-byte vector
@@ -117,12 +141,20 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const uint4 *__r
     __shared__ u32 s_emax;
     __shared__ u64 s_wlo[WQ_THREADS / 32], s_whi[WQ_THREADS / 32];
 
+    // the matrix this block sums
+    int ji = 0;
+    while (ji + 1 < P.count && (int)blockIdx.x >= P.j[ji + 1].blk0) ++ji;
+    const WqJob &job = P.j[ji];
+    const uint4 *__restrict__ W = job.W;
+    const long long nvec = job.nvec;
+    u64 *__restrict__ partials = P.partials;
+
     const int tid = threadIdx.x;
     for (int i = tid; i < 256; i += WQ_THREADS) s_bins[i] = 0ull;
     if (tid == 0) s_emax = 0;
 
-    const long long stride = (long long)gridDim.x * WQ_THREADS;
-    const long long first = (long long)blockIdx.x * WQ_THREADS + tid;
+    const long long stride = (long long)job.nblk * WQ_THREADS;
+    const long long first = (long long)((int)blockIdx.x - job.blk0) * WQ_THREADS + tid;
 
     // Window from a sample: the block's first vector per thread.  The second
     // vector is requested before the block reduction, so its latency overlaps.
@@ -211,45 +243,55 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const uint4 *__r
         }
     }
 
-    // The last block to finish finalizes (partials published with a fence
-    // before the ticket; the ticket is zeroed by the host before the launch
-    // and reset here for the next call on the same workspace).
+    // The last block of this matrix to finish finalizes it (partials
+    // published with a fence before the ticket; the ticket is zeroed by the
+    // host before the launch and reset here for the next call on the same
+    // workspace).
     __shared__ bool s_last;
     if (tid == 0) {
         __threadfence();
-        s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+        s_last = atomicAdd(&P.tickets[ji], 1u) == (u32)job.nblk - 1;
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    wq_finalize_block(partials, gridDim.x, n, gamma_out, ws_thresh);
-    if (tid == 0) *ticket = 0u;
+    wq_finalize_block(partials + (size_t)job.blk0 * WQ_PART_LIMBS, job.nblk, job.n, job.gamma, &P.thresh[ji]);
+    if (tid == 0) P.tickets[ji] = 0u;
 }
 
-// Each thread packs 16 consecutive weights into one 32-bit word per step.
+// Each thread packs 16 consecutive weights into one 32-bit word per step;
+// the words of all matrices of the launch form one index space.
 template <bool BF16>
-__global__ void __launch_bounds__(256) k_ternary_pack(const uint4 *__restrict__ W, long long nwords,
-                                                        const u32 *__restrict__ ws_thresh,
-                                                        u32 *__restrict__ packed) {
+__global__ void __launch_bounds__(256) k_ternary_pack(const __grid_constant__ WqParams P) {
     constexpr int VPW = BF16 ? 2 : 4;  // 16-byte vectors per 16 weights
     // a programmatically dependent launch after this one (bl_linear's act
     // quant, which does not read the packed weights) may start now
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const long long stride = (long long)gridDim.x * blockDim.x;
-    long long wi = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long first = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    auto job_of = [&](long long w) {
+        int i = 0;
+        while (i + 1 < P.count && w >= P.j[i + 1].word0) ++i;
+        return i;
+    };
     // first words of W are requested before waiting for the reduction grid
     uint4 v[VPW];
-    if (wi < nwords) {
+    if (first < P.total_words) {
+        const WqJob &jb = P.j[job_of(first)];
+        const long long wl = first - jb.word0;
 #pragma unroll
-        for (int q = 0; q < VPW; ++q) v[q] = ldg_stream_v4(W + wi * VPW + q);
+        for (int q = 0; q < VPW; ++q) v[q] = ldg_stream_v4(jb.W + wl * VPW + q);
     }
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const u32 T = __ldcg(ws_thresh);
-    for (; wi < nwords; wi += stride) {
-        if (wi != (long long)blockIdx.x * blockDim.x + threadIdx.x) {
+    for (long long wi = first; wi < P.total_words; wi += stride) {
+        const int ji = job_of(wi);
+        const WqJob &jb = P.j[ji];
+        const long long wl = wi - jb.word0;
+        if (wi != first) {
 #pragma unroll
-            for (int q = 0; q < VPW; ++q) v[q] = ldg_stream_v4(W + wi * VPW + q);
+            for (int q = 0; q < VPW; ++q) v[q] = ldg_stream_v4(jb.W + wl * VPW + q);
         }
+        const u32 T = __ldcg(P.thresh + ji);
         u32 word = 0;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
@@ -260,7 +302,7 @@ __global__ void __launch_bounds__(256) k_ternary_pack(const uint4 *__restrict__ 
             int i = k & 3, j = k >> 2;
             word |= code << (8 * i + 2 * j);
         }
-        packed[wi] = word;
+        jb.packed[wl] = word;
     }
 }
 

@@ -199,3 +199,72 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(build, "LIB", str(tmp_path / "libbitlinear.so"))
     with pytest.raises(RuntimeError, match="missing"):
         api.lib()
+
+
+def test_grouped_weight_quant_validation(L):
+    def call(count=1, wdt=0, ws=A, wsb=1 << 20, **kw):
+        p = dict(W=A, N=64, K=128, packed=A, gamma=A)
+        p.update(kw)
+        arr = (api.WeightProblem * 8)()
+        for i in range(8):
+            arr[i] = api.WeightProblem(p["W"], p["N"], p["K"], p["packed"], p["gamma"])
+        return L.bl_quant_weights_grouped(arr, count, wdt, ws, wsb, None)
+
+    assert L.bl_quant_weights_grouped(None, 1, 0, A, 1 << 20, None) == NULL
+    assert call(count=0) == SHAPE
+    assert call(count=9) == SHAPE
+    assert call(wdt=3) == DTYPE
+    assert call(W=None) == NULL
+    assert call(gamma=None) == NULL
+    assert call(K=96) == SHAPE
+    assert call(N=1 << 17, K=1 << 14) == SHAPE
+    assert call(packed=A + 8) == ALIGN
+    assert call(ws=None) == WORKSPACE
+    assert call(wsb=100) == WORKSPACE
+    assert call(count=8) in (CUDA, DEVICE)
+
+
+def test_grouped_linear_validation_and_workspace(L):
+    M, K = 64, 768
+    arr = (api.LinearProblem * 4)()
+    for i, N in enumerate((768, 256, 256, 2048)):
+        arr[i] = api.LinearProblem(A, A, N)
+    ws = L.bl_linear_grouped_workspace_bytes(arr, 3, M, K)
+    assert ws >= L.bl_quant_weights_workspace_bytes(1, 64) + (768 + 256 + 256) * K // 4 + M * K + 4 * M
+    assert L.bl_linear_grouped_workspace_bytes(arr, 5, M, K) == 0
+
+    def call(count=3, wdt=1, X=A, xdt=1, M=M, K=K, gain=None, wsp=A, wsb=ws):
+        return L.bl_linear_grouped(arr, count, wdt, X, xdt, M, K, gain, 1e-6, wsp, wsb, None)
+
+    assert call(X=None) == NULL
+    assert call(count=5) == SHAPE
+    assert call(wdt=2) == DTYPE
+    assert call(xdt=2) == DTYPE
+    assert call(K=100) == SHAPE
+    assert call(M=0) == SHAPE
+    assert call(X=A + 4) == ALIGN
+    assert call(gain=A + 4) == ALIGN
+    assert call(wsb=ws - 1) == WORKSPACE
+    assert call() in (CUDA, DEVICE)
+
+
+def test_backward_and_gated_validation(L):
+    def bdx(dY=A, packed=A, gamma=A, M=64, N=128, K=256, dX=A):
+        return L.bl_backward_dx(dY, packed, gamma, M, N, K, dX, None)
+
+    assert bdx(dY=None) == NULL
+    assert bdx(dX=None) == NULL
+    assert bdx(N=12) == SHAPE       # dY rows must be multiples of 16 bytes
+    assert bdx(K=100) == SHAPE
+    assert bdx(M=0) == SHAPE
+    assert bdx(dY=A + 8) == ALIGN
+    assert bdx() in (CUDA, DEVICE)
+
+    def glu(pg=A, gg=A, pu=A, gu=A, xq=A, s=A, M=64, F=256, K=256, h=A):
+        return L.bl_forward_glu(pg, gg, pu, gu, xq, s, M, F, K, h, None)
+
+    assert glu(pu=None) == NULL
+    assert glu(F=100) == SHAPE      # F is the down projection's K: a multiple of 64
+    assert glu(K=96) == SHAPE
+    assert glu(h=A + 4) == ALIGN
+    assert glu() in (CUDA, DEVICE)
