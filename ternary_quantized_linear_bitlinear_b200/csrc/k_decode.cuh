@@ -45,6 +45,10 @@
 //     producer fills the ring before griddepcontrol.wait, so a launch streams
 //     its weights while the launch before it finishes; activations and s are
 //     read only after the wait.
+//   - A consumer tests a stage's phase parity only after the producer has
+//     issued its chunk (a shared issue counter): the stage's previous chunk
+//     belongs to another warp and may still be in flight, and a parity test
+//     two phases behind would pass.
 //   - Every mbarrier wait is bounded (globaltimer); a wait that gives up
 //     raises the device error word and the CTA's abort flag; the producer
 //     then waits (bounded) for its in-flight copies before the CTA exits.
@@ -435,6 +439,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
     __shared__ u32 s_amax[DEC_MAX_PSLOTS * 16];
     __shared__ float s_sc[DEC_MAX_PSLOTS * 16];
     __shared__ volatile int s_abort;
+    __shared__ volatile int s_issued;  // chunks the producer has issued
 
     // a programmatically dependent launch that follows may start its prologue
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -455,6 +460,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_abort = 0;
+        s_issued = 0;
         int off = 0, vb = 0;
         for (int i = 0; i < np; ++i) {
             s_xoff[i] = off;
@@ -498,6 +504,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
         policy = l2_policy_evict_first();
         for (int p = p_lo; p <= p_hi; ++p) asm volatile("prefetch.tensormap [%0];" ::"l"(&P.wmap[p]) : "memory");
         for (; issued < total && issued < DEC_STAGES; ++issued) issue(issued);
+        __threadfence_block();
+        s_issued = (int)issued;
     }
 
     // x_q and s may be produced by the kernel launched just before this one.
@@ -570,6 +578,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
                     break;
                 }
                 issue(issued);
+                __threadfence_block();  // the stage's earlier phases are ordered before the count
+                s_issued = (int)issued + 1;
             }
             if (failed) {
                 raise_device_error(DEVERR_TIMEOUT_PRODUCER);
@@ -594,7 +604,23 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
     dec_advance(P, cc, warp, g_end);
     for (long long j = warp; j < total; j += DEC_CWARPS) {
         const int s = (int)(j % DEC_STAGES);
-        const bool ok = mbar_wait(smem_u32(&s_full[s]), (u32)((j / DEC_STAGES) & 1), DEC_TIMEOUT_NS, &s_abort);
+        // Wait until chunk j has been issued before testing its stage's
+        // phase parity: warps take chunks round-robin, so this stage's
+        // previous chunk (j - DEC_STAGES) belongs to another warp and may
+        // not have landed yet, and a parity test two phases behind would
+        // pass.  Once j is issued, j - DEC_STAGES has been consumed.
+        bool ok = true;
+        if (s_issued <= j) {
+            const unsigned long long t0 = globaltimer();
+            while (s_issued <= j) {
+                if (s_abort || globaltimer() - t0 > DEC_TIMEOUT_NS) {
+                    ok = false;
+                    break;
+                }
+            }
+        }
+        __threadfence_block();
+        ok = ok && mbar_wait(smem_u32(&s_full[s]), (u32)((j / DEC_STAGES) & 1), DEC_TIMEOUT_NS, &s_abort);
         if (!__all_sync(0xffffffffu, ok)) {
             if (lane == 0) {
                 raise_device_error(DEVERR_TIMEOUT_MMA);
