@@ -213,8 +213,8 @@ bl_status bl_ffn_act_quant(const float *gate, const float *up, int64_t M, int64_
 /*               (two float roundings: |Y - acc*gamma/s| <= 2^-23 |Y|)       */
 /*                                                                           */
 /* Engine: the bandwidth-bound decode GEMV when M <= 16 and the staged     */
-/* activations fit, M * round_up(K, 256) <= 153600 bytes (M <= 16 for      */
-/* K <= 9472, M <= 15 at K = 9728, M <= 9 at K = 16384, M <= 4 at           */
+/* activations fit, M * round_up(K, 256) <= 147456 bytes (M <= 16 for      */
+/* K <= 9216, M <= 15 at K = 9728, M <= 9 at K = 16384, M <= 4 at           */
 /* K = 32768), otherwise the tcgen05 prefill GEMM.  Both give identical acc. */
 /* packed [N, K/4] (format above); gamma [1]; x_q [M, K]; s [M]; Y [M, N]    */
 /* out; acc_out [M, N] int32 out or NULL.  All device.                       */

@@ -26,7 +26,9 @@ constexpr int BL_VERSION = 100;
 constexpr int64_t K_MAX = 32768;
 constexpr int MAX_DEVICES = 64;
 constexpr size_t DEC_SMEM_ATTR = (size_t)dec_fixed_smem(2) + DEC_X_MAX + 1024;
-static_assert(DEC_SMEM_ATTR <= 227 * 1024, "decode engine shared memory");
+// dynamic + static shared memory of one CTA within the 227 KiB opt-in limit
+// (the kernel's static shared memory is under 4 KiB)
+static_assert(DEC_SMEM_ATTR + 4 * 1024 <= 227 * 1024, "decode engine shared memory");
 static_assert(sizeof(DecodeParams) <= 32764, "decode parameters exceed the kernel parameter limit");
 
 struct DeviceInfo {

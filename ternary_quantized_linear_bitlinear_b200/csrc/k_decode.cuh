@@ -69,7 +69,7 @@ constexpr int DEC_STAGES = 12;                        // ring stages = accumulat
 constexpr int DEC_SLOT_LD = 36;                       // words per token row of a slot (bank spread)
 constexpr int DEC_MAX_PSLOTS = 8;                     // problems per CTA
 constexpr int DEC_MAX_CTAS = 320;
-constexpr int DEC_X_MAX = 150 * 1024;                 // staged activations per CTA
+constexpr int DEC_X_MAX = 144 * 1024;                 // staged activations per CTA
 constexpr int DEC_X_PAIR = 36 * 1024;                 // ... at most this keeps two CTAs per SM
 constexpr unsigned long long DEC_TIMEOUT_NS = 2000000000ull;
 
