@@ -267,6 +267,32 @@ bl_status bl_backward_dx(const void *dY, const uint8_t *packed, const float *gam
                          int64_t K, float *dX, bl_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Backward of the quantization-aware BitLinear, weight gradient, with the  */
+/* straight-through estimator and the hard or soft STE scale ("Distillix"   */
+/* README, 1. BitNet b1.58 Core: STE; "bitone" README, Soft-STE notes:      */
+/* hard mask |w / gamma| <= 1, soft scale 1 - tanh^2(beta w / gamma)):      */
+/*                                                                           */
+/*   dW[n, k] = float(float(sum_m dY[m, n] * xs[m, k]) * scale(r))           */
+/*   xs = bf16(float(x_q / s)), r = float(W[n, k] / gamma)                   */
+/*   scale(r) = |r| <= 1 ? 1 : 0 (beta <= 0),  1 - tanhf(beta r)^2 otherwise */
+/*                                                                           */
+/* the sum over the tokens in float32 on the tensor cores after both         */
+/* operands are laid out with the tokens contiguous (two transposes into    */
+/* the workspace); xs is rounded to bf16 (2^-9 relative), so dW agrees with */
+/* the exact value within about (2^-8 + M * 2^-23) of                       */
+/* sum_m |dY[m, n] x_q[m, k] / s[m]| * scale.                                */
+/*                                                                           */
+/* dY [M, N] bfloat16; x_q [M, K], s [M] from the forward's bl_quant_act;    */
+/* W [N, K] the latent weights (wdt), gamma [1] their forward scale;         */
+/* dW [N, K] float32 out; workspace >= bl_backward_dw_workspace_bytes(M, N,  */
+/* K).  All device, 16-byte aligned.  K as for bl_forward, N >= 1.           */
+/* ------------------------------------------------------------------------ */
+size_t bl_backward_dw_workspace_bytes(int64_t M, int64_t N, int64_t K);
+bl_status bl_backward_dw(const void *dY, const int8_t *x_q, const float *s, const void *W, bl_dtype wdt,
+                         const float *gamma, float beta, int64_t M, int64_t N, int64_t K, void *workspace,
+                         size_t workspace_bytes, float *dW, bl_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* All four steps in one call: bl_quant_weights, bl_quant_act, bl_forward    */
 /* (for decode-eligible M, steps 2-4 run as one fused launch, with the same  */
 /* results).                                                                 */

@@ -84,6 +84,8 @@ _SIGS = {
     "bl_quant_weights_grouped": (_int, [ctypes.POINTER(WeightProblem), _int, _int, _p, _sz, _p]),
     "bl_forward_glu": (_int, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _p, _p]),
     "bl_backward_dx": (_int, [_p, _p, _p, _i64, _i64, _i64, _p, _p]),
+    "bl_backward_dw_workspace_bytes": (_sz, [_i64, _i64, _i64]),
+    "bl_backward_dw": (_int, [_p, _p, _p, _p, _int, _p, _f32, _i64, _i64, _i64, _p, _sz, _p, _p]),
     "bl_linear_grouped_workspace_bytes": (_sz, [ctypes.POINTER(LinearProblem), _int, _i64, _i64]),
     "bl_linear_grouped": (_int, [ctypes.POINTER(LinearProblem), _int, _int, _p, _int, _i64, _i64, _p, _f32, _p, _sz,
                                  _p]),
@@ -379,6 +381,34 @@ def bl_backward_dx(dY, packed, gamma, K: int, dX=None, stream=None):
                               _stream(stream))
     _check(rc, "bl_backward_dx")
     return dX
+
+
+def bl_backward_dw(dY, x_q, s, W, gamma, beta: float = 0.0, dW=None, workspace=None, stream=None):
+    """dW float32 [N, K] = (dY^T @ (x_q / s)) * scale(W / gamma): the weight
+    gradient under the hard (beta <= 0) or soft STE scale; dY bfloat16 [M, N],
+    x_q, s from the forward's activation quantization, W the latent weights."""
+    _dev(dY, "dY", torch.bfloat16)
+    if dY.dim() != 2:
+        raise ValueError("dY must be 2-D [M, N]")
+    M, N = dY.shape
+    Mx, K = _xq2d(x_q)
+    if Mx != M:
+        raise ValueError("x_q and dY disagree on M")
+    _mat(W, "W", cols=K, rows=N)
+    _dev(s, "s", torch.float32, M)
+    _dev(gamma, "gamma", torch.float32, 1)
+    if dW is None:
+        dW = torch.empty(N, K, dtype=torch.float32, device=dY.device)
+    _dev(dW, "dW", torch.float32, N * K)
+    need = int(lib().bl_backward_dw_workspace_bytes(M, N, K))
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dY.device)
+    _dev(workspace, "workspace", torch.uint8, need)
+    rc = lib().bl_backward_dw(dY.data_ptr(), x_q.data_ptr(), s.data_ptr(), W.data_ptr(), _DTYPES[W.dtype],
+                              gamma.data_ptr(), float(beta), M, N, K, workspace.data_ptr(), workspace.numel(), dW.data_ptr(),
+                              _stream(stream))
+    _check(rc, "bl_backward_dw")
+    return dW
 
 
 def _check_forward_args(packed, gamma, s, Y, acc_out, M, N, K):

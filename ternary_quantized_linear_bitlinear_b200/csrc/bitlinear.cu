@@ -16,6 +16,7 @@
 #include "k_act_quant.cuh"
 #include "k_decode.cuh"
 #include "k_prefill_tc.cuh"
+#include "k_dense_tc.cuh"
 #include "k_weight_quant.cuh"
 
 using namespace bl;
@@ -59,6 +60,7 @@ bl_status device_info(DeviceInfo **out) {
                 fail |= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)DEC_SMEM_ATTR) !=
                         cudaSuccess;
             fail |= prefill_setup() != cudaSuccess;
+            fail |= dense_setup() != cudaSuccess;
             for (auto fn : {k_act_quant_subln_row<false, true>, k_act_quant_subln_row<true, false>,
                             k_act_quant_subln_row<false, false>})
                 fail |= cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, AQR_MAX_K * 4) !=
@@ -629,6 +631,29 @@ bl_status bl_backward_dx(const void *dY, const uint8_t *packed, const float *gam
     bl_status rc = device_info(&d);
     if (rc) return rc;
     return prefill_launch_bwd(d->sms, dY, packed, gamma, M, N, K, dX, (cudaStream_t)stream);
+}
+
+size_t bl_backward_dw_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    if (M < 1 || N < 1 || K < 1) return 0;
+    return dw_workspace_bytes(M, N, K);
+}
+
+bl_status bl_backward_dw(const void *dY, const int8_t *x_q, const float *s, const void *W, bl_dtype wdt,
+                         const float *gamma, float beta, int64_t M, int64_t N, int64_t K, void *workspace,
+                         size_t workspace_bytes, float *dW, bl_stream_t stream) {
+    if (!dY || !x_q || !s || !W || !gamma || !dW) return BL_ERR_NULL;
+    if (wdt != BL_F32 && wdt != BL_BF16) return BL_ERR_DTYPE;
+    if (M < 1 || M > 0x7fffffffLL - 64 || N < 1 || check_k(K) != BL_OK || !nk_fits(N, K)) return BL_ERR_SHAPE;
+    if (!aligned16(dY) || !aligned16(x_q) || !aligned16(s) || !aligned16(W) || !aligned16(gamma) || !aligned16(dW))
+        return BL_ERR_ALIGN;
+    if (!workspace || workspace_bytes < dw_workspace_bytes(M, N, K)) return BL_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return BL_ERR_ALIGN;
+    DeviceInfo *d;
+    bl_status rc = device_info(&d);
+    if (rc) return rc;
+    EncodeTiledFn enc = encode_tiled_fn();
+    if (enc == nullptr) return BL_ERR_CUDA;
+    return dw_launch(enc, dY, x_q, s, W, wdt == BL_BF16, gamma, beta, M, N, K, workspace, dW, (cudaStream_t)stream);
 }
 
 bl_status bl_forward_grouped(const bl_problem *problems, int count, int64_t M, unsigned flags,

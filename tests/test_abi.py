@@ -268,3 +268,22 @@ def test_backward_and_gated_validation(L):
     assert glu(K=96) == SHAPE
     assert glu(h=A + 4) == ALIGN
     assert glu() in (CUDA, DEVICE)
+
+
+def test_weight_gradient_validation(L):
+    M, N, K = 300, 256, 512
+    ws = L.bl_backward_dw_workspace_bytes(M, N, K)
+    assert ws >= 2 * (N + K) * 320  # dY^T and (x_q / s)^T in bf16 over 320 padded tokens
+    assert L.bl_backward_dw_workspace_bytes(0, N, K) == 0
+
+    def dw(dY=A, xq=A, s=A, W=A, wdt=0, g=A, M=M, N=N, K=K, wsp=A, wsb=ws, out=A):
+        return L.bl_backward_dw(dY, xq, s, W, wdt, g, 2.0, M, N, K, wsp, wsb, out, None)
+
+    assert dw(dY=None) == NULL
+    assert dw(out=None) == NULL
+    assert dw(wdt=5) == DTYPE
+    assert dw(K=100) == SHAPE
+    assert dw(N=0) == SHAPE
+    assert dw(xq=A + 2) == ALIGN
+    assert dw(wsb=ws - 1) == WORKSPACE
+    assert dw() in (CUDA, DEVICE)
