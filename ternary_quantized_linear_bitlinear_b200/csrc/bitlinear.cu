@@ -375,10 +375,13 @@ bl_status decode_launch(const DecodeJob *jobs, int count, int M, float eps, bool
         const int64_t ng = (jobs[i].N + DEC_ROWS - 1) / DEC_ROWS;
         const double gb = (double)DEC_ROWS * (double)(jobs[i].K / 4);
         while (next < c0 + (double)ng * gb && ncut < base_ctas) {
+            // the first group whose byte midpoint lies past `next` (the next
+            // problem's first group when it is none of this problem's)
             int64_t k = (int64_t)std::floor((next - c0) / gb - 0.5) + 1;
             if (k < 0) k = 0;
+            if (k > ng) k = ng;
             const int64_t g = P.p[i].gbase + k;
-            if (k < ng && g > cuts[ncut - 1]) cuts[ncut++] = (int)g;
+            if (g < G && g > cuts[ncut - 1]) cuts[ncut++] = (int)g;
             next += target;
         }
         c0 += (double)ng * gb;

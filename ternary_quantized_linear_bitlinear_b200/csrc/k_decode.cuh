@@ -6,28 +6,28 @@
 // The work is bound by streaming the packed weights from HBM (2 bits per
 // weight).  Design (one CTA per SM and launch, small enough that the CTA of
 // the next launch fits beside it):
-//   - Work unit: a group of 32 weight rows of one problem; its packed bytes
-//     are cut into chunks of 32 rows x 128 bytes (512 k), which a producer
-//     thread streams with 2-D TMA tensor loads (128-byte swizzle, L2
-//     evict-first: each byte is read once) through a ring of DEC_STAGES
-//     shared-memory stages, in group order.  The host cuts the flattened
-//     group list of all problems into one contiguous range per CTA with
-//     equal bytes.
-//   - Consumers: DEC_CWARPS warps take the ring's chunks round-robin
-//     (chunk j -> warp j mod DEC_CWARPS), so every warp streams at the same
-//     rate whatever the problems' K.  A warp's partial sums of a chunk go
-//     into the group's accumulator slot in shared memory (integer atomics:
-//     exact, any order); the warp that completes a group's last chunk
-//     rescales the slot and writes Y (lane = weight row: coalesced stores),
-//     zeroes the slot and only then frees its ring stage, which keeps a slot
-//     from being reused (slot = group ordinal mod DEC_STAGES) before its
-//     group is written out.
+//   - Work unit: a group of 32 weight rows of one problem.  The host cuts the
+//     flattened group list of all problems into one contiguous range per CTA
+//     with about equal packed bytes.  Inside the CTA every warp takes whole
+//     groups: its first one by its index, the next ones from a shared
+//     counter as it needs them, so warps that meet short groups take more.
+//   - Streaming: each warp owns a ring of DEC_WSTAGES shared-memory stages.
+//     Its lane 0 cuts its groups into chunks of 32 rows x 128 bytes (512 k)
+//     and requests each with a 2-D TMA tensor load (per-problem tensor map,
+//     128-byte swizzle, L2 evict-first: each byte is read once) as soon as
+//     the warp has consumed the stage, DEC_WSTAGES chunks ahead of its
+//     compute; the first requests go out before griddepcontrol.wait, so a
+//     programmatic dependent launch (BL_FWD_WEIGHTS_READY) streams its
+//     weights while the launch before it finishes.  A warp consumes only its
+//     own stages, in order: no cross-warp synchronization on the stream.
 //   - MACs on the tensor cores (mma.sync m16n8k32 s8): weight rows as A (two
 //     16-row tiles per chunk share every x_q fragment), tokens as B (8
 //     columns per tile, zero for m >= M).  The int32 sum is exact, so the k
 //     order inside a 256-k step may be permuted as long as A and B use the
 //     same permutation: the lane with k-slot t holds the packed bytes
 //     64t .. 64t + 15 of the step, and its B fragment reads those x_q bytes.
+//     A group's accumulators stay in the warp's registers over its chunks;
+//     the warp rescales them and writes Y when the group's last chunk is in.
 //   - Unpacking costs 1-2 ALU ops per 4 weights: with the packed layout, word
 //     (w << (6 - 2j)) & 0xC0C0C0C0 puts the codes of k = 16w' + 4j .. 4j+3 in
 //     the top two bits of four bytes, i.e. the int8 values 64 * W_q; the sum
@@ -38,20 +38,13 @@
 //   - x_q is staged once per CTA and problem in shared memory (rows of
 //     round_up(K, 256) bytes, 16-byte chunks XOR-swizzled so that the B loads
 //     are free of bank conflicts).  Fused variant (SRC = bf16 or f32
-//     activations): step 2 runs inside the CTA, one warp per token row, with
-//     the same arithmetic as the stand-alone activation quantizer; the CTA
-//     holding a problem's first group also writes x_q and s on request.
-//   - Launched as a programmatic dependent (BL_FWD_WEIGHTS_READY), the
-//     producer fills the ring before griddepcontrol.wait, so a launch streams
-//     its weights while the launch before it finishes; activations and s are
-//     read only after the wait.
-//   - A consumer tests a stage's phase parity only after the producer has
-//     issued its chunk (a shared issue counter): the stage's previous chunk
-//     belongs to another warp and may still be in flight, and a parity test
-//     two phases behind would pass.
+//     activations): step 2 runs inside the CTA with the same arithmetic as
+//     the stand-alone activation quantizer (rows without SubLN by the whole
+//     CTA at once, SubLN rows one warp per row); the CTA holding a problem's
+//     first group also writes x_q and s on request.
 //   - Every mbarrier wait is bounded (globaltimer); a wait that gives up
-//     raises the device error word and the CTA's abort flag; the producer
-//     then waits (bounded) for its in-flight copies before the CTA exits.
+//     raises the device error word and the CTA's abort flag, and each warp
+//     then waits (bounded) for its own copies in flight before it exits.
 #pragma once
 
 #include <cuda.h>
@@ -60,23 +53,19 @@
 
 namespace bl {
 
-constexpr int DEC_CWARPS = 8;                         // consumer warps
-constexpr int DEC_THREADS = 32 * (DEC_CWARPS + 1);    // + the producer warp
+constexpr int DEC_WARPS = 8;
+constexpr int DEC_THREADS = 32 * DEC_WARPS;
 constexpr int DEC_ROWS = 32;                          // weight rows per group (two MMA tiles)
 constexpr int DEC_CB = 128;                           // packed bytes per row per chunk (512 k)
 constexpr int DEC_CHUNK = DEC_ROWS * DEC_CB;          // 4 KiB
-constexpr int DEC_STAGES = 12;                        // ring stages = accumulator slots
-constexpr int DEC_SLOT_LD = 36;                       // words per token row of a slot (bank spread)
+constexpr int DEC_WSTAGES = 2;                        // ring stages per warp
 constexpr int DEC_MAX_PSLOTS = 8;                     // problems per CTA
 constexpr int DEC_MAX_CTAS = 320;
 constexpr int DEC_X_MAX = 144 * 1024;                 // staged activations per CTA
 constexpr int DEC_X_PAIR = 36 * 1024;                 // ... at most this keeps two CTAs per SM
 constexpr unsigned long long DEC_TIMEOUT_NS = 2000000000ull;
 
-__host__ __device__ constexpr int dec_slot_bytes(int nt) { return 8 * nt * DEC_SLOT_LD * 4; }
-__host__ __device__ constexpr int dec_fixed_smem(int nt) {
-    return DEC_STAGES * DEC_CHUNK + DEC_STAGES * dec_slot_bytes(nt);
-}
+__host__ __device__ constexpr int dec_fixed_smem(int) { return DEC_WARPS * DEC_WSTAGES * DEC_CHUNK; }
 
 // Activation source of a launch: pre-quantized x_q, or X to quantize in-kernel.
 enum : int { DEC_SRC_XQ = 0, DEC_SRC_BF16 = 1, DEC_SRC_F32 = 2 };
@@ -401,22 +390,6 @@ __device__ __forceinline__ int dec_problem_of(const DecodeParams &P, int g) {
 
 __device__ __forceinline__ int dec_nchunks(int K) { return (K + 4 * DEC_CB - 1) / (4 * DEC_CB); }
 
-// Chunk cursor over a CTA's groups: group g of problem p, chunk kc.
-struct DecCursor {
-    int g, p, kc;
-};
-
-__device__ __forceinline__ void dec_advance(const DecodeParams &P, DecCursor &c, int by, int g_end) {
-    c.kc += by;
-    while (c.g < g_end) {
-        const int nch = dec_nchunks(P.p[c.p].K);
-        if (c.kc < nch) break;
-        c.kc -= nch;
-        ++c.g;
-        if (c.p + 1 < P.count && c.g >= P.p[c.p + 1].gbase) ++c.p;
-    }
-}
-
 __device__ __forceinline__ void tma_load_2d_hint(u32 dst, const CUtensorMap *map, int x, int y, u32 bar, u64 pol) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
@@ -430,37 +403,33 @@ template <int NT, int SRC>
 __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant__ DecodeParams P) {
     extern __shared__ uint8_t dsm_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~(uintptr_t)1023);
-    __shared__ __align__(8) u64 s_full[DEC_STAGES];
-    __shared__ __align__(8) u64 s_empty[DEC_STAGES];
-    __shared__ int s_cnt[DEC_STAGES];
+    __shared__ __align__(8) u64 s_full[DEC_WARPS][DEC_WSTAGES];
+    __shared__ int s_queue[DEC_WARPS][DEC_WSTAGES + 2];  // groups a warp has started requesting, in order
+    __shared__ int s_next;                               // next group to hand out
     __shared__ float s_f[DEC_MAX_PSLOTS][16];
     __shared__ int s_xoff[DEC_MAX_PSLOTS + 1];
     __shared__ int s_vbase[DEC_MAX_PSLOTS + 1];
     __shared__ u32 s_amax[DEC_MAX_PSLOTS * 16];
     __shared__ float s_sc[DEC_MAX_PSLOTS * 16];
     __shared__ volatile int s_abort;
-    __shared__ volatile int s_issued;  // chunks the producer has issued
 
     // a programmatically dependent launch that follows may start its prologue
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    constexpr int SLOT_WORDS = dec_slot_bytes(NT) / 4;
+    constexpr int QN = DEC_WSTAGES + 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g_begin = P.cta_g[blockIdx.x], g_end = P.cta_g[blockIdx.x + 1];
     const int p_lo = dec_problem_of(P, g_begin), p_hi = dec_problem_of(P, g_end - 1);
     const int np = p_hi - p_lo + 1;
     const int M = P.M;
-    int *slots = reinterpret_cast<int *>(sm + DEC_STAGES * DEC_CHUNK);
     uint8_t *s_x = sm + dec_fixed_smem(NT);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < DEC_STAGES; ++s) {
-            mbar_init(smem_u32(&s_full[s]), 1);
-            mbar_init(smem_u32(&s_empty[s]), 1);
-        }
+        for (int w = 0; w < DEC_WARPS; ++w)
+            for (int s = 0; s < DEC_WSTAGES; ++s) mbar_init(smem_u32(&s_full[w][s]), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         s_abort = 0;
-        s_issued = 0;
+        s_next = g_begin + DEC_WARPS;
         int off = 0, vb = 0;
         for (int i = 0; i < np; ++i) {
             s_xoff[i] = off;
@@ -472,41 +441,54 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
         s_vbase[np] = vb;
     }
     if (threadIdx.x < DEC_MAX_PSLOTS * 16) s_amax[threadIdx.x] = 0u;
-    for (int i = threadIdx.x; i < DEC_STAGES * SLOT_WORDS; i += DEC_THREADS) slots[i] = 0;
-    if (threadIdx.x < DEC_STAGES) s_cnt[threadIdx.x] = 0;
     __syncthreads();
 
-    // chunks of this CTA
-    long long total = 0;
-    {
-        int g = g_begin;
-        for (int p = p_lo; p <= p_hi; ++p) {
-            const int gnext = p + 1 < P.count ? min(P.p[p + 1].gbase, g_end) : g_end;
-            total += (long long)(gnext - g) * dec_nchunks(P.p[p].K);
-            g = gnext;
-        }
-    }
-
-    // ---- producer: the first ring-full before waiting for the previous grid
-    const bool producer = warp == DEC_CWARPS && lane == 0;
-    u64 policy = 0;
-    DecCursor pc{g_begin, p_lo, 0};
+    // ---- this warp's request stream: its groups' chunks, in order ---------
+    // (warp-uniform state; lane 0 issues the copies)
+    uint8_t *ring = sm + warp * (DEC_WSTAGES * DEC_CHUNK);
+    const u64 policy = l2_policy_evict_first();
+    int i_g = -1, i_p = p_lo, i_k = 0, i_nch = 0;  // request cursor: group, problem, chunk, chunks of group
+    int q_tail = 0;                                // groups queued for the consumer side
     long long issued = 0;
-    auto issue = [&](long long j) {
-        const int s = (int)(j % DEC_STAGES);
-        const u32 bar = smem_u32(&s_full[s]);
-        mbar_arrive_expect_tx(bar, DEC_CHUNK);
-        tma_load_2d_hint(smem_u32(sm + s * DEC_CHUNK), &P.wmap[pc.p], pc.kc * DEC_CB,
-                         (pc.g - P.p[pc.p].gbase) * DEC_ROWS, bar, policy);
-        dec_advance(P, pc, 1, g_end);
+    auto next_group = [&]() -> int {
+        int g;
+        if (i_g < 0) {
+            g = g_begin + warp;
+        } else {
+            g = 0;
+            if (lane == 0) g = atomicAdd(&s_next, 1);
+            g = __shfl_sync(0xffffffffu, g, 0);
+        }
+        return g < g_end ? g : -2;
     };
-    if (producer) {
-        policy = l2_policy_evict_first();
+    auto issue_next = [&]() {
+        if (i_g == -2) return;
+        if (i_g < 0 || i_k == i_nch) {
+            const int g = next_group();
+            if (g < 0) {
+                i_g = -2;
+                return;
+            }
+            while (i_p + 1 < P.count && g >= P.p[i_p + 1].gbase) ++i_p;
+            i_g = g;
+            i_k = 0;
+            i_nch = dec_nchunks(P.p[i_p].K);
+            s_queue[warp][q_tail % QN] = g;  // every lane writes (and later reads) its own copy
+            ++q_tail;
+        }
+        const int s = (int)(issued % DEC_WSTAGES);
+        if (lane == 0) {
+            const u32 bar = smem_u32(&s_full[warp][s]);
+            mbar_arrive_expect_tx(bar, DEC_CHUNK);
+            tma_load_2d_hint(smem_u32(ring + s * DEC_CHUNK), &P.wmap[i_p], i_k * DEC_CB,
+                             (i_g - P.p[i_p].gbase) * DEC_ROWS, bar, policy);
+        }
+        ++i_k;
+        ++issued;
+    };
+    if (lane == 0)
         for (int p = p_lo; p <= p_hi; ++p) asm volatile("prefetch.tensormap [%0];" ::"l"(&P.wmap[p]) : "memory");
-        for (; issued < total && issued < DEC_STAGES; ++issued) issue(issued);
-        __threadfence_block();
-        s_issued = (int)issued;
-    }
+    for (int i = 0; i < DEC_WSTAGES; ++i) issue_next();
 
     // x_q and s may be produced by the kernel launched just before this one.
     asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -521,7 +503,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
     if (block_quant) {
         dec_quant_block<SRC == DEC_SRC_BF16>(P, p_lo, np, g_begin, s_xoff, s_vbase, s_x, s_amax, s_sc, s_f);
         // zero the padding chunks K .. round_up(K, 256) of every row
-        for (int r = warp; r < np * M; r += DEC_CWARPS + 1) {
+        for (int r = warp; r < np * M; r += DEC_WARPS) {
             const int ps = r / M, m = r - ps * M;
             const int K = P.p[p_lo + ps].K, RS = dec_row_stride(K);
             uint8_t *xs = s_x + s_xoff[ps];
@@ -531,7 +513,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
             }
         }
     }
-    for (int r = warp; r < (block_quant ? 0 : np * M); r += DEC_CWARPS + 1) {
+    for (int r = warp; r < (block_quant ? 0 : np * M); r += DEC_WARPS) {
         const int ps = r / M, m = r - ps * M;
         const DecodeProblem &pr = P.p[p_lo + ps];
         const int K = pr.K, RS = dec_row_stride(K);
@@ -565,78 +547,25 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
     }
     __syncthreads();
 
-    if (warp == DEC_CWARPS) {
-        // ---------------------------------------------------------- producer
-        if (producer) {
-            bool failed = false;
-            for (; issued < total; ++issued) {
-                const int s = (int)(issued % DEC_STAGES);
-                // the stage's previous chunk has been consumed
-                if (!mbar_wait(smem_u32(&s_empty[s]), (u32)(((issued / DEC_STAGES) & 1) ^ 1), DEC_TIMEOUT_NS,
-                               &s_abort)) {
-                    failed = true;
-                    break;
-                }
-                issue(issued);
-                __threadfence_block();  // the stage's earlier phases are ordered before the count
-                s_issued = (int)issued + 1;
-            }
-            if (failed) {
-                raise_device_error(DEVERR_TIMEOUT_PRODUCER);
-                s_abort = 1;
-            }
-            if (s_abort) {
-                // drain: the last copies issued land before the CTA exits
-                for (long long j = issued - DEC_STAGES; j < issued; ++j)
-                    if (j >= 0)
-                        mbar_wait(smem_u32(&s_full[(int)(j % DEC_STAGES)]), (u32)((j / DEC_STAGES) & 1),
-                                  DEC_TIMEOUT_NS, nullptr);
-            }
-        }
-        return;
-    }
-
     // ------------------------------------------------------------- consumers
     const int g8 = lane >> 2, t = lane & 3;
     const int pg = (g8 >> 1) | ((g8 & 1) << 2);       // physical row phase of MMA row g8
     const int xb = ((t >> 1) << 1) | (g8 & 1);        // x_q swizzle of this lane's token rows
-    DecCursor cc{g_begin, p_lo, 0};
-    dec_advance(P, cc, warp, g_end);
-    for (long long j = warp; j < total; j += DEC_CWARPS) {
-        const int s = (int)(j % DEC_STAGES);
-        // Wait until chunk j has been issued before testing its stage's
-        // phase parity: warps take chunks round-robin, so this stage's
-        // previous chunk (j - DEC_STAGES) belongs to another warp and may
-        // not have landed yet, and a parity test two phases behind would
-        // pass.  Once j is issued, j - DEC_STAGES has been consumed.
-        bool ok = true;
-        if (s_issued <= j) {
-            const unsigned long long t0 = globaltimer();
-            while (s_issued <= j) {
-                if (s_abort || globaltimer() - t0 > DEC_TIMEOUT_NS) {
-                    ok = false;
-                    break;
-                }
-            }
-        }
-        __threadfence_block();
-        ok = ok && mbar_wait(smem_u32(&s_full[s]), (u32)((j / DEC_STAGES) & 1), DEC_TIMEOUT_NS, &s_abort);
-        if (!__all_sync(0xffffffffu, ok)) {
-            if (lane == 0) {
-                raise_device_error(DEVERR_TIMEOUT_MMA);
-                s_abort = 1;
-            }
-            break;
-        }
-        const DecodeProblem &pr = P.p[cc.p];
-        const int ps = cc.p - p_lo;
+    // two accumulator chains per tile at M <= 8 (alternate planes), one at
+    // M <= 16 (two token tiles already give four independent chains)
+    constexpr int CH = NT == 1 ? 2 : 1;
+    long long consumed = 0;
+    int q_head = 0, c_p = p_lo;
+    bool ok = true;
+    while (ok && q_head < q_tail) {
+        const int g = s_queue[warp][q_head % QN];
+        ++q_head;
+        while (c_p + 1 < P.count && g >= P.p[c_p + 1].gbase) ++c_p;
+        const DecodeProblem &pr = P.p[c_p];
+        const int ps = c_p - p_lo;
         const int K = pr.K, RS = dec_row_stride(K);
-        const int vb = min(DEC_CB, (K >> 2) - cc.kc * DEC_CB);  // valid packed bytes per row (>= 16)
-        const uint8_t *st = sm + s * DEC_CHUNK;
         const uint8_t *xs = s_x + s_xoff[ps];
-        // two accumulator chains per tile at M <= 8 (alternate planes), one at
-        // M <= 16 (two token tiles already give four independent chains)
-        constexpr int CH = NT == 1 ? 2 : 1;
+        const int nch = dec_nchunks(K);
         int acc[CH][2][NT][4];
 #pragma unroll
         for (int c = 0; c < CH; ++c)
@@ -646,80 +575,85 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) acc[c][u][nt][i] = 0;
-#pragma unroll 1
-        for (int h2 = 0; h2 < 2; ++h2) {
-            if (64 * h2 >= vb) break;
-            // weights: physical rows pg + 8a (a = 0..3), this lane's 16 bytes of the half
-            uint4 wv[4];
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-                wv[a] = *reinterpret_cast<const uint4 *>(st + (pg + 8 * a) * DEC_CB + (((4 * h2 + t) ^ pg) << 4));
-            // x_q of tokens g8 (+ 8): the 64 bytes of k-slot t in 256-k step s2
-            const int s2 = 2 * cc.kc + h2;
-            uint4 xv[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                const int m = g8 + 8 * nt;
-                const uint8_t *xr = xs + m * RS + s2 * 256 + t * 64;
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    xv[nt][c] = m < M ? *reinterpret_cast<const uint4 *>(xr + ((c ^ xb) << 4)) : make_uint4(0, 0, 0, 0);
+        for (int kc = 0; kc < nch; ++kc, ++consumed) {
+            const int s = (int)(consumed % DEC_WSTAGES);
+            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&s_full[warp][s]), (u32)((consumed / DEC_WSTAGES) & 1),
+                                                  DEC_TIMEOUT_NS, &s_abort));
+            if (!ok) {
+                if (lane == 0) {
+                    raise_device_error(DEVERR_TIMEOUT_MMA);
+                    s_abort = 1;
+                }
+                break;
             }
+            const int vb = min(DEC_CB, (K >> 2) - kc * DEC_CB);  // valid packed bytes per row (>= 16)
+            const uint8_t *st = ring + s * DEC_CHUNK;
+#pragma unroll 1
+            for (int h2 = 0; h2 < 2; ++h2) {
+                if (64 * h2 >= vb) break;
+                // weights: physical rows pg + 8a (a = 0..3), this lane's 16 bytes of the half
+                uint4 wv[4];
 #pragma unroll
-            for (int u = 0; u < 2; ++u) {
+                for (int a = 0; a < 4; ++a)
+                    wv[a] = *reinterpret_cast<const uint4 *>(st + (pg + 8 * a) * DEC_CB + (((4 * h2 + t) ^ pg) << 4));
+                // x_q of tokens g8 (+ 8): the 64 bytes of k-slot t in 256-k step s2
+                const int s2 = 2 * kc + h2;
+                uint4 xv[NT][4];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    const u32 wa0 = (&wv[2 * u].x)[2 * hh], wa2 = (&wv[2 * u].x)[2 * hh + 1];
-                    const u32 wa1 = (&wv[2 * u + 1].x)[2 * hh], wa3 = (&wv[2 * u + 1].x)[2 * hh + 1];
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int m = g8 + 8 * nt;
+                    const uint8_t *xr = xs + m * RS + s2 * 256 + t * 64;
 #pragma unroll
-                    for (int jp = 0; jp < 4; ++jp) {
-                        const u32 a0 = dec_unpack(wa0, jp), a1 = dec_unpack(wa1, jp);
-                        const u32 a2 = dec_unpack(wa2, jp), a3 = dec_unpack(wa3, jp);
+                    for (int c = 0; c < 4; ++c)
+                        xv[nt][c] = m < M ? *reinterpret_cast<const uint4 *>(xr + ((c ^ xb) << 4))
+                                          : make_uint4(0, 0, 0, 0);
+                }
 #pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            int(&A)[4] = acc[(jp & 1) % CH][u][nt];
-                            mma_s8_16832(A, a0, a1, a2, a3, (&xv[nt][2 * hh].x)[jp], (&xv[nt][2 * hh + 1].x)[jp]);
+                for (int u = 0; u < 2; ++u) {
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        const u32 wa0 = (&wv[2 * u].x)[2 * hh], wa2 = (&wv[2 * u].x)[2 * hh + 1];
+                        const u32 wa1 = (&wv[2 * u + 1].x)[2 * hh], wa3 = (&wv[2 * u + 1].x)[2 * hh + 1];
+#pragma unroll
+                        for (int jp = 0; jp < 4; ++jp) {
+                            const u32 a0 = dec_unpack(wa0, jp), a1 = dec_unpack(wa1, jp);
+                            const u32 a2 = dec_unpack(wa2, jp), a3 = dec_unpack(wa3, jp);
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+                                mma_s8_16832(acc[(jp & 1) % CH][u][nt], a0, a1, a2, a3, (&xv[nt][2 * hh].x)[jp],
+                                             (&xv[nt][2 * hh + 1].x)[jp]);
                         }
                     }
                 }
             }
+            // the stage is free again: request this warp's next chunk into it
+            __syncwarp();
+            issue_next();
         }
-        // partial sums into the group's slot: row pg + 16u + 8(i >> 1), token 8nt + 2t + (i & 1)
-        const int go = cc.g - g_begin;
-        int *slot = slots + (go % DEC_STAGES) * SLOT_WORDS;
+        if (!ok) break;
+        // epilogue: rows pg + 16u + 8(i >> 1), tokens 8nt + 2t + (i & 1)
+        const int n_base = (g - pr.gbase) * DEC_ROWS + pg;
 #pragma unroll
         for (int u = 0; u < 2; ++u)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const int v = CH == 2 ? acc[0][u][nt][i] + acc[CH - 1][u][nt][i] : acc[0][u][nt][i];
-                    atomicAdd(slot + (8 * nt + 2 * t + (i & 1)) * DEC_SLOT_LD + pg + 16 * u + 8 * (i >> 1), v);
+                    const int m = 8 * nt + 2 * t + (i & 1);
+                    const int n = n_base + 16 * u + 8 * (i >> 1);
+                    if (m < M && n < pr.N) {
+                        const int v = CH == 2 ? acc[0][u][nt][i] + acc[CH - 1][u][nt][i] : acc[0][u][nt][i];
+                        const int a_ = v >> 6;  // exact: the sum is a multiple of 64
+                        pr.Y[(size_t)m * pr.N + n] = __fmul_rn(__int2float_rn(a_), s_f[ps][m]);
+                        if (pr.acc) pr.acc[(size_t)m * pr.N + n] = a_;
+                    }
                 }
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-            __threadfence_block();
-            last = atomicAdd(&s_cnt[go % DEC_STAGES], 1) == dec_nchunks(K) - 1;
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-            // every chunk of the group has been added: rescale and write it out
-            __threadfence_block();
-            const int n = (cc.g - pr.gbase) * DEC_ROWS + lane;
-            for (int m = 0; m < M; ++m) {
-                const int a = slot[m * DEC_SLOT_LD + lane] >> 6;  // exact: the sum is a multiple of 64
-                slot[m * DEC_SLOT_LD + lane] = 0;
-                if (n < pr.N) {
-                    pr.Y[(size_t)m * pr.N + n] = __fmul_rn(__int2float_rn(a), s_f[ps][m]);
-                    if (pr.acc) pr.acc[(size_t)m * pr.N + n] = a;
-                }
-            }
-            if (lane == 0) s_cnt[go % DEC_STAGES] = 0;
-            __syncwarp();
-        }
-        if (lane == 0) mbar_arrive(smem_u32(&s_empty[s]));
-        dec_advance(P, cc, DEC_CWARPS, g_end);
+    }
+    if (!ok) {
+        // drain: this warp's copies in flight land before it exits
+        for (long long j = consumed; j < issued; ++j)
+            mbar_wait(smem_u32(&s_full[warp][(int)(j % DEC_WSTAGES)]), (u32)((j / DEC_WSTAGES) & 1), DEC_TIMEOUT_NS,
+                      nullptr);
     }
 }
 
