@@ -37,8 +37,9 @@
  * ~1.6 bits): 2 bits per weight, N * K / 4 bytes.  Row n occupies K/4
  * contiguous bytes = K/16 little-endian 32-bit words.  Weight k = 16*w + 4*j
  * + i (0 <= i, j < 4) has its code in word w at bits [8*i + 2*j,
- * 8*i + 2*j + 1].  Codes: 00 = 0, 01 = +1, 11 = -1 (2-bit two's complement);
- * 10 is never written.  So byte i of a word holds the codes of k = i, i+4,
+ * 8*i + 2*j + 1].  The code is 1 - W_q as a 2-bit unsigned number: 00 = +1,
+ * 01 = 0, 10 = -1; 11 is never written (a zero weight matrix packs to 0x55
+ * bytes).  So byte i of a word holds the codes of k = i, i+4,
  * i+8, i+12 of its 16-weight group.
  */
 #ifndef BITLINEAR_H

@@ -46,8 +46,8 @@
  *   - the 2-bit packing (a format of this library; the pages only say two
  *     bits or fewer per weight): row n is K/4 bytes = K/16 little-endian
  *     32-bit words; weight k = 16*w + 4*j + i has its code in word w at bits
- *     8*i + 2*j (low) and 8*i + 2*j + 1 (high); code 00 = 0, 01 = +1,
- *     11 = -1, 10 never written.
+ *     8*i + 2*j (low) and 8*i + 2*j + 1 (high); the code is 1 - W_q as a
+ *     2-bit unsigned number: 00 = +1, 01 = 0, 10 = -1, 11 never written.
  *
  * Build: gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -shared
  *        -fPIC oracle.c -o liboracle.so  (see build.py beside this file).
@@ -192,10 +192,10 @@ int oracle_pack(const int8_t *q, int64_t N, int64_t K, uint8_t *packed) {
         uint8_t *row = packed + n * (K / 4);
         for (int64_t k = 0; k < K; ++k) {
             int8_t v = q[n * K + k];
-            unsigned code;
-            if (v == 0) code = 0u;
-            else if (v == 1) code = 1u;
-            else if (v == -1) code = 3u;
+            unsigned code;  /* 1 - v */
+            if (v == 1) code = 0u;
+            else if (v == 0) code = 1u;
+            else if (v == -1) code = 2u;
             else return OR_ERR_RANGE;
             int64_t byte; int bit;
             code_position(k, &byte, &bit);
@@ -205,7 +205,7 @@ int oracle_pack(const int8_t *q, int64_t N, int64_t K, uint8_t *packed) {
     return OR_OK;
 }
 
-/* Inverse of oracle_pack; the reserved code 10 is reported as an error. */
+/* Inverse of oracle_pack; the reserved code 11 is reported as an error. */
 int oracle_unpack(const uint8_t *packed, int64_t N, int64_t K, int8_t *q) {
     if (N <= 0 || K <= 0 || K % 16) return OR_ERR_SHAPE;
     for (int64_t n = 0; n < N; ++n) {
@@ -214,8 +214,8 @@ int oracle_unpack(const uint8_t *packed, int64_t N, int64_t K, int8_t *q) {
             int64_t byte; int bit;
             code_position(k, &byte, &bit);
             unsigned code = (row[byte] >> bit) & 3u;
-            if (code == 2u) return OR_ERR_RANGE;
-            q[n * K + k] = code == 0u ? 0 : (code == 1u ? 1 : -1);
+            if (code == 3u) return OR_ERR_RANGE;
+            q[n * K + k] = (int8_t)(1 - (int)code);
         }
     }
     return OR_OK;

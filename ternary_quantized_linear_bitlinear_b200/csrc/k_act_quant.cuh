@@ -487,8 +487,9 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
             s_r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(limbs_to_double_rn(L, -298), (double)K)), P.eps));
         __syncthreads();
         const float r = s_r;
-        // pass 3: y = float(float(x / r) * g) in place, max|y|.  For the gated
-        // FFN input, x / r is correctly rounded by Markstein's method from the
+        // pass 3: y = float(float(x / r) * g) in place, max|y|.  For float32
+        // rows (the gated FFN input and h from the gated GEMM), x / r is
+        // correctly rounded by Markstein's method from the
         // correctly rounded reciprocal of the row constant r (q0 = x * (1/r),
         // remainder x - r * q0 by FMA, one correction FMA).  The method is
         // exact whenever that remainder is representable, which holds for
@@ -504,7 +505,7 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
         // Measured 172 -> 136 us for [8192, 4096]; bf16 rows were 1-2 %
         // slower with it, so they keep the IEEE division.
         const float ry = __frcp_rn(r);
-        const bool mk = GLU && __float_as_uint(r) >= 0x00800000u && __float_as_uint(r) < 0x7f800000u;
+        const bool mk = (GLU || !BF16) && __float_as_uint(r) >= 0x00800000u && __float_as_uint(r) < 0x7f800000u;
         auto div_r = [&](float x) {
             const u32 ax = __float_as_uint(x) & 0x7fffffffu;
             if (!mk || (ax != 0u && ax < 0x00800000u)) return __fdiv_rn(x, r);

@@ -28,10 +28,15 @@
 //     64t .. 64t + 15 of the step, and its B fragment reads those x_q bytes.
 //     A group's accumulators stay in the warp's registers over its chunks;
 //     the warp rescales them and writes Y when the group's last chunk is in.
-//   - Unpacking costs 1-2 ALU ops per 4 weights: with the packed layout, word
-//     (w << (6 - 2j)) & 0xC0C0C0C0 puts the codes of k = 16w' + 4j .. 4j+3 in
-//     the top two bits of four bytes, i.e. the int8 values 64 * W_q; the sum
-//     is 64 * acc, exactly.
+//   - Unpacking costs one AND per 4 weights: a packed word holds the codes
+//     c = 1 - W_q in {0, 1, 2}; word & (0x03030303 << 2j) leaves the codes of
+//     k = 16w' + 4j .. 4j+3 in four bytes as the unsigned values 4^j c, which
+//     the MMA takes as u8 (A) against the s8 activations (B), one accumulator
+//     per plane j.  Then sum_k W_q x = sum_k x - sum_j D_j / 4^j (each D_j a
+//     multiple of 4^j, so the shifts are exact), with sum_k x the row sum of
+//     the staged x_q.  At M > 8 (two token tiles) the planes are moved to the
+//     top two bits instead ((w << (6 - 2j)) & 0xC0C0C0C0, 64 c) and share one
+//     accumulator per tile, to keep the registers of the second tile.
 //   - Lane (g, t) of an MMA tile reads weight rows pi(g) and pi(g) + 8 with
 //     pi(g) = (g >> 1) | ((g & 1) << 2): with the 128-byte swizzle, the eight
 //     lanes of each quarter warp then hit eight different bank quads.
@@ -96,18 +101,21 @@ struct DecodeParams {
 
 __host__ __device__ inline int dec_row_stride(int K) { return (K + 255) & ~255; }
 
-__device__ __forceinline__ u32 dec_unpack(u32 w, int j) {
-    // codes of k = 4j .. 4j+3 of this 16-weight word -> int8 lanes holding 64 * W_q
-    return (w << (6 - 2 * j)) & 0xC0C0C0C0u;
-}
+// codes of k = 4j .. 4j+3 of this 16-weight word as u8 lanes 4^j * (1 - W_q)
+__device__ __forceinline__ u32 dec_plane(u32 w, int j) { return w & (0x03030303u << (2 * j)); }
 
-__device__ __forceinline__ void mma_s8_16832(int (&c)[4], u32 a0, u32 a1, u32 a2, u32 a3, u32 b0, u32 b1) {
+// the same codes moved to the top two bits: u8 lanes 64 * (1 - W_q)
+__device__ __forceinline__ u32 dec_plane_top(u32 w, int j) { return (w << (6 - 2 * j)) & 0xC0C0C0C0u; }
+
+// unsigned 8-bit A (the weight codes), signed 8-bit B (x_q)
+__device__ __forceinline__ void mma_u8s8_16832(int (&c)[4], u32 a0, u32 a1, u32 a2, u32 a3, u32 b0, u32 b1) {
     asm volatile(
-        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 "
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 "
         "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
         : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
+
 
 // Float bits of element j of a 16-byte activation vector.
 template <bool BF16>
@@ -204,7 +212,7 @@ __device__ __forceinline__ void dec_y4(const uint4 &raw, int q, const float4 *g4
 // Returns s (on every lane).
 template <bool BF16>
 __device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, uint8_t *s_xq, float eps, bool out,
-                               int lane) {
+                               int lane, int *rowsum) {
     constexpr int EPV = BF16 ? 8 : 4;
     const int nvec = K / EPV;
     const int nblk = (nvec + 32 * DEC_QV - 1) / (32 * DEC_QV);
@@ -248,6 +256,7 @@ __device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, ui
     const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(amax), 1e-5f));
     uint8_t *dst = s_xq + m * RS;
     int8_t *gq = out && pr.xq_out != nullptr ? pr.xq_out + (size_t)m * K : nullptr;
+    int rs = 0;
     for (int blk = 0; blk < nblk; ++blk) {
         if (nblk > 1) dec_load_block(c, xr, nvec, blk, lane);
 #pragma unroll
@@ -264,6 +273,7 @@ __device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, ui
                 for (int j = 0; j < 4; ++j) {
                     int qi = __float2int_rn(__fmul_rn(y[j], s));
                     qi = max(-128, min(127, qi));
+                    rs += qi;
                     w |= ((u32)qi & 0xffu) << (8 * j);
                 }
                 word[q] = w;
@@ -283,6 +293,8 @@ __device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, ui
         }
     }
     if (out && lane == 0 && pr.s != nullptr) pr.s[m] = s;
+    rs = __reduce_add_sync(0xffffffffu, rs);
+    if (lane == 0) *rowsum = rs;
     return s;
 }
 
@@ -298,7 +310,8 @@ constexpr int DEC_QBV = 12;
 
 template <bool BF16>
 __device__ void dec_quant_block(const DecodeParams &P, int p_lo, int np, int g_begin, const int *s_xoff,
-                                const int *vbase, uint8_t *s_x, u32 *s_amax, float *s_sc, float (*s_f)[16]) {
+                                const int *vbase, uint8_t *s_x, u32 *s_amax, float *s_sc, float (*s_f)[16],
+                                int *s_rs) {
     constexpr int EPV = BF16 ? 8 : 4;
     const int M = P.M, T = vbase[np];
     const int lane = threadIdx.x & 31;
@@ -346,7 +359,10 @@ __device__ void dec_quant_block(const DecodeParams &P, int p_lo, int np, int g_b
     __syncthreads();
 #pragma unroll
     for (int i = 0; i < DEC_QBV; ++i) {
-        if (meta[i] < 0) continue;
+        if (DEC_THREADS * i >= T) break;  // uniform: no vector of this round is in range
+        int rsum = 0;
+        const int row = meta[i] < 0 ? -1 : ((meta[i] >> 20) * M + ((meta[i] >> 16) & 15));
+        if (meta[i] >= 0) {
         const int ps = meta[i] >> 20, m = (meta[i] >> 16) & 15, v = meta[i] & 0xffff;
         const DecodeProblem &pr = P.p[p_lo + ps];
         const int K = pr.K, RS = dec_row_stride(K);
@@ -359,6 +375,7 @@ __device__ void dec_quant_block(const DecodeParams &P, int p_lo, int np, int g_b
             for (int j = 0; j < 4; ++j) {
                 int qi = __float2int_rn(__fmul_rn(__uint_as_float(dec_x_bits<BF16>(c[i], 4 * q + j)), s));
                 qi = max(-128, min(127, qi));
+                rsum += qi;
                 w |= ((u32)qi & 0xffu) << (8 * j);
             }
             word[q] = w;
@@ -374,6 +391,15 @@ __device__ void dec_quant_block(const DecodeParams &P, int p_lo, int np, int g_b
         } else {
             *reinterpret_cast<u32 *>(d) = word[0];
             if (gq) *reinterpret_cast<u32 *>(gq + (size_t)v * 4) = word[0];
+        }
+        }
+        // the row sums of x_q, one shared atomic per warp when its vectors share a row
+        const int row0 = __shfl_sync(0xffffffffu, row, 0);
+        if (__all_sync(0xffffffffu, row == row0)) {
+            rsum = __reduce_add_sync(0xffffffffu, rsum);
+            if ((threadIdx.x & 31) == 0 && row0 >= 0) atomicAdd(&s_rs[row0], rsum);
+        } else if (row >= 0) {
+            atomicAdd(&s_rs[row], rsum);
         }
     }
 }
@@ -411,6 +437,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
     __shared__ int s_vbase[DEC_MAX_PSLOTS + 1];
     __shared__ u32 s_amax[DEC_MAX_PSLOTS * 16];
     __shared__ float s_sc[DEC_MAX_PSLOTS * 16];
+    __shared__ int s_rs[DEC_MAX_PSLOTS * 16];  // row sums of the staged x_q
     __shared__ volatile int s_abort;
 
     // a programmatically dependent launch that follows may start its prologue
@@ -440,7 +467,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
         s_xoff[np] = off;
         s_vbase[np] = vb;
     }
-    if (threadIdx.x < DEC_MAX_PSLOTS * 16) s_amax[threadIdx.x] = 0u;
+    if (threadIdx.x < DEC_MAX_PSLOTS * 16) {
+        s_amax[threadIdx.x] = 0u;
+        s_rs[threadIdx.x] = 0;
+    }
     __syncthreads();
 
     // ---- this warp's request stream: its groups' chunks, in order ---------
@@ -501,7 +531,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
         block_quant = !gain && s_vbase[np] <= DEC_QBV * DEC_THREADS;
     }
     if (block_quant) {
-        dec_quant_block<SRC == DEC_SRC_BF16>(P, p_lo, np, g_begin, s_xoff, s_vbase, s_x, s_amax, s_sc, s_f);
+        dec_quant_block<SRC == DEC_SRC_BF16>(P, p_lo, np, g_begin, s_xoff, s_vbase, s_x, s_amax, s_sc, s_f, s_rs);
         // zero the padding chunks K .. round_up(K, 256) of every row
         for (int r = warp; r < np * M; r += DEC_WARPS) {
             const int ps = r / M, m = r - ps * M;
@@ -521,7 +551,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
         if (SRC != DEC_SRC_XQ) {
             constexpr bool BF16 = SRC == DEC_SRC_BF16;
             const bool out = g_begin <= pr.gbase;  // this CTA holds the problem's first group
-            const float s = dec_quant_row<BF16>(pr, m, K, RS, xs, P.eps, out, lane);
+            const float s = dec_quant_row<BF16>(pr, m, K, RS, xs, P.eps, out, lane, &s_rs[ps * M + m]);
             if (lane == 0) s_f[ps][m] = __fdiv_rn(*pr.gamma, s);
             for (int L = (K >> 4) + lane; L < (RS >> 4); L += 32) {
                 const int x = (((L >> 3) & 1) << 1) | (m & 1);
@@ -544,6 +574,24 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
     if (SRC == DEC_SRC_XQ) {
         asm volatile("cp.async.commit_group;" ::: "memory");
         asm volatile("cp.async.wait_all;" ::: "memory");
+        __syncthreads();
+        // row sums of the staged x_q (the padding is zero; the order of the
+        // 16-byte chunks does not matter)
+        for (int r = warp; r < np * M; r += DEC_WARPS) {
+            const int ps = r / M, m = r - ps * M;
+            const int RS = dec_row_stride(P.p[p_lo + ps].K);
+            const uint4 *row = reinterpret_cast<const uint4 *>(s_x + s_xoff[ps] + m * RS);
+            int sum = 0;
+            for (int L = lane; L < (RS >> 4); L += 32) {
+                const uint4 v = row[L];
+                sum = __dp4a((int)v.x, 0x01010101, sum);
+                sum = __dp4a((int)v.y, 0x01010101, sum);
+                sum = __dp4a((int)v.z, 0x01010101, sum);
+                sum = __dp4a((int)v.w, 0x01010101, sum);
+            }
+            sum = __reduce_add_sync(0xffffffffu, sum);
+            if (lane == 0) s_rs[r] = sum;
+        }
     }
     __syncthreads();
 
@@ -551,9 +599,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
     const int g8 = lane >> 2, t = lane & 3;
     const int pg = (g8 >> 1) | ((g8 & 1) << 2);       // physical row phase of MMA row g8
     const int xb = ((t >> 1) << 1) | (g8 & 1);        // x_q swizzle of this lane's token rows
-    // two accumulator chains per tile at M <= 8 (alternate planes), one at
-    // M <= 16 (two token tiles already give four independent chains)
-    constexpr int CH = NT == 1 ? 2 : 1;
+    // M <= 8: one accumulator per code plane and tile (plane j at scale 4^j);
+    // M <= 16: the planes moved to scale 64, one accumulator per tile
+    constexpr int PL = NT == 1 ? 4 : 1;
     long long consumed = 0;
     int q_head = 0, c_p = p_lo;
     bool ok = true;
@@ -566,9 +614,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
         const int K = pr.K, RS = dec_row_stride(K);
         const uint8_t *xs = s_x + s_xoff[ps];
         const int nch = dec_nchunks(K);
-        int acc[CH][2][NT][4];
+        int acc[PL][2][NT][4];
 #pragma unroll
-        for (int c = 0; c < CH; ++c)
+        for (int c = 0; c < PL; ++c)
 #pragma unroll
             for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -616,12 +664,22 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
                         const u32 wa1 = (&wv[2 * u + 1].x)[2 * hh], wa3 = (&wv[2 * u + 1].x)[2 * hh + 1];
 #pragma unroll
                         for (int jp = 0; jp < 4; ++jp) {
-                            const u32 a0 = dec_unpack(wa0, jp), a1 = dec_unpack(wa1, jp);
-                            const u32 a2 = dec_unpack(wa2, jp), a3 = dec_unpack(wa3, jp);
+                            u32 a0, a1, a2, a3;
+                            if (PL == 4) {
+                                a0 = dec_plane(wa0, jp);
+                                a1 = dec_plane(wa1, jp);
+                                a2 = dec_plane(wa2, jp);
+                                a3 = dec_plane(wa3, jp);
+                            } else {
+                                a0 = dec_plane_top(wa0, jp);
+                                a1 = dec_plane_top(wa1, jp);
+                                a2 = dec_plane_top(wa2, jp);
+                                a3 = dec_plane_top(wa3, jp);
+                            }
 #pragma unroll
                             for (int nt = 0; nt < NT; ++nt)
-                                mma_s8_16832(acc[(jp & 1) % CH][u][nt], a0, a1, a2, a3, (&xv[nt][2 * hh].x)[jp],
-                                             (&xv[nt][2 * hh + 1].x)[jp]);
+                                mma_u8s8_16832(acc[jp % PL][u][nt], a0, a1, a2, a3, (&xv[nt][2 * hh].x)[jp],
+                                               (&xv[nt][2 * hh + 1].x)[jp]);
                         }
                     }
                 }
@@ -642,8 +700,12 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
                     const int m = 8 * nt + 2 * t + (i & 1);
                     const int n = n_base + 16 * u + 8 * (i >> 1);
                     if (m < M && n < pr.N) {
-                        const int v = CH == 2 ? acc[0][u][nt][i] + acc[CH - 1][u][nt][i] : acc[0][u][nt][i];
-                        const int a_ = v >> 6;  // exact: the sum is a multiple of 64
+                        // sum_k c x with c = 1 - W_q, each plane's sum a multiple of its scale
+                        const int cx = PL == 4 ? acc[0][u][nt][i] + (acc[PL > 1 ? 1 : 0][u][nt][i] >> 2) +
+                                                     (acc[PL > 2 ? 2 : 0][u][nt][i] >> 4) +
+                                                     (acc[PL > 3 ? 3 : 0][u][nt][i] >> 6)
+                                               : acc[0][u][nt][i] >> 6;
+                        const int a_ = s_rs[ps * M + m] - cx;
                         pr.Y[(size_t)m * pr.N + n] = __fmul_rn(__int2float_rn(a_), s_f[ps][m]);
                         if (pr.acc) pr.acc[(size_t)m * pr.N + n] = a_;
                     }

@@ -10,7 +10,8 @@
 //   A = its 128 tokens of x_q, by TMA with 128-byte swizzle, K-major;
 //   B = 64 * W_q of its 128 of the 256 weight rows as int8: the packed 2-bit
 //     rows arrive by TMA, four expander warps (one weight row per thread)
-//     unpack them ((word << (6 - 2j)) & 0xC0C0C0C0 gives four int8 lanes),
+//     unpack them (((word << (6 - 2j)) & 0xC0C0C0C0) ^ 0x40404040 gives
+//     four int8 lanes 64 * W_q from the codes 1 - W_q),
 //     store them in the 128-byte-swizzled K-major layout the MMA reads, then
 //     fence the async proxy;
 //   D = int32 accumulators in each CTA's TMEM (lane = its token, column =
@@ -475,8 +476,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
                         for (int e = 0; e < 4; ++e) {
                             const u32 c0 = (pw[8 * (8 * c + 2 * e)] >> sh) & 3u;
                             const u32 c1 = (pw[8 * (8 * c + 2 * e + 1)] >> sh) & 3u;
-                            const u32 b0 = (c0 & 1u) * 0x3F80u | ((c0 & 2u) << 14);
-                            const u32 b1 = (c1 & 1u) * 0x3F80u | ((c1 & 2u) << 14);
+                            // code 1 - W_q -> bf16: 00 -> +1 (0x3F80), 01 -> 0, 10 -> -1 (0xBF80)
+                            const u32 b0 = ((c0 & 1u) ^ 1u) * 0x3F80u | ((c0 & 2u) << 14);
+                            const u32 b1 = ((c1 & 1u) ^ 1u) * 0x3F80u | ((c1 & 2u) << 14);
                             o[e] = b0 | (b1 << 16);
                         }
                         *reinterpret_cast<uint4 *>(brow + ((c ^ rsw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
@@ -491,12 +493,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PF_THREADS, 1)
                 const u32 w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    // packed word i = k 16i .. 16i+15 = 16-byte chunk i of the row
+                    // packed word i = k 16i .. 16i+15 = 16-byte chunk i of the row.
+                    // Code c = 1 - W_q moved to the top two bits of a byte, its
+                    // low bit flipped, is W_q in two's complement there, i.e.
+                    // the int8 64 * W_q (one AND and XOR, one LOP3, per four)
                     uint4 o;
-                    o.x = (w[i] << 6) & 0xC0C0C0C0u;
-                    o.y = (w[i] << 4) & 0xC0C0C0C0u;
-                    o.z = (w[i] << 2) & 0xC0C0C0C0u;
-                    o.w = w[i] & 0xC0C0C0C0u;
+                    o.x = ((w[i] << 6) & 0xC0C0C0C0u) ^ 0x40404040u;
+                    o.y = ((w[i] << 4) & 0xC0C0C0C0u) ^ 0x40404040u;
+                    o.z = ((w[i] << 2) & 0xC0C0C0C0u) ^ 0x40404040u;
+                    o.w = (w[i] & 0xC0C0C0C0u) ^ 0x40404040u;
                     *reinterpret_cast<uint4 *>(brow + ((i ^ rsw) << 4)) = o;
                 }
                 // make the generic-proxy stores visible to the tensor core (async proxy)

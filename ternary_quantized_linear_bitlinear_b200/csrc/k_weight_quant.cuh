@@ -12,8 +12,9 @@
 //                      gamma = float(S / n) + 1e-5f, and the float
 //                      threshold T with
 //                      |w| >= T  <=>  float(|w|/gamma) > 0.5
-//   k_ternary_pack     second pass over W: code = sign(w) * (|w| >= T), four
-//                      codes per byte in the packed word layout; launched as
+//   k_ternary_pack     second pass over W: W_q = sign(w) * (|w| >= T), stored
+//                      as the code 1 - W_q, four codes per byte in the
+//                      packed word layout; launched as
 //                      a programmatic dependent, it loads its first words of
 //                      W before waiting for gamma and T
 //
@@ -298,7 +299,7 @@ __global__ void __launch_bounds__(256) k_ternary_pack(const __grid_constant__ Wq
             constexpr int EPV = BF16 ? 8 : 4;
             u32 bits = vec_elem_bits<BF16>(v[k / EPV], k % EPV);
             u32 nz = (bits & 0x7fffffffu) >= T ? 1u : 0u;
-            u32 code = nz | ((bits >> 30) & 2u & (nz << 1));  // 01 = +1, 11 = -1
+            u32 code = (nz ^ 1u) | ((bits >> 30) & 2u & (nz << 1));  // 1 - W_q: 00 = +1, 01 = 0, 10 = -1
             int i = k & 3, j = k >> 2;
             word |= code << (8 * i + 2 * j);
         }

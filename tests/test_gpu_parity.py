@@ -66,7 +66,7 @@ def test_quant_weights(N, K, dtype, kind):
     check_weights(W, packed, gamma)
     if kind == "zeros":
         assert gamma.item() == np.float32(1e-5)
-        assert int(packed.sum()) == 0
+        assert bool(torch.all(packed == 0x55))  # code 01 = 0 for every weight
 
 
 def test_quant_weights_workspace_contents_ignored_and_reused():

@@ -207,8 +207,9 @@ def test_pack_roundtrip_and_bits_per_weight():
 
 
 def test_unpack_rejects_reserved_code():
-    p = np.zeros((1, 4), dtype=np.uint8)
-    p[0, 0] = 0b10
+    p = np.full((1, 4), 0x55, dtype=np.uint8)  # sixteen zero weights
+    assert np.array_equal(oracle.unpack(p, 16), np.zeros((1, 16), np.int8))
+    p[0, 2] = 0x57  # k = 2 gets code 11
     with pytest.raises(oracle.OracleError):
         oracle.unpack(p, 16)
 
