@@ -8,7 +8,6 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
-#include <unordered_map>
 
 #include "bitlinear.h"
 #include "bitlinear_debug.h"
@@ -26,10 +25,13 @@ namespace {
 constexpr int BL_VERSION = 100;
 constexpr int64_t K_MAX = 32768;
 constexpr int MAX_DEVICES = 64;
-constexpr size_t DEC_SMEM_ATTR = (size_t)dec_fixed_smem(2) + DEC_X_MAX + 1024;
-// dynamic + static shared memory of one CTA within the 227 KiB opt-in limit
-// (the kernel's static shared memory is under 4 KiB)
-static_assert(DEC_SMEM_ATTR + 4 * 1024 <= 227 * 1024, "decode engine shared memory");
+// dynamic shared memory of the largest decode launch: weights of a CTA
+// (whole rows up to DEC_W_CAP bytes, or one row group up to 32 x 1536 bytes,
+// or a 32 x DEC_KCH_B chunk) plus padding, x_q, the sums, alignment slack
+constexpr size_t DEC_SMEM_ATTR = (size_t)DEC_ROWS * DEC_KCH_B + DEC_W_PAD + DEC_X_MAX + DEC_WARPS * DEC_ROWS * 16 * 4 + 512;
+// ... within the 227 KiB opt-in limit with the kernel's static shared memory (under 1 KiB)
+static_assert(DEC_SMEM_ATTR + 1024 <= 227 * 1024, "decode engine shared memory");
+static_assert(DEC_ROWS * (DEC_K_WHOLE / 4) <= DEC_ROWS * DEC_KCH_B, "decode weight staging");
 static_assert(sizeof(DecodeParams) <= 32764, "decode parameters exceed the kernel parameter limit");
 
 struct DeviceInfo {
@@ -300,143 +302,87 @@ struct DecodeJob {
     int64_t N, K;
 };
 
-// Tensor maps of packed weight matrices ({K/4 bytes, N rows}, box 128 x 32,
-// 128-byte swizzle), cached by (address, N, K): encoding one costs about a
-// microsecond of host time, and a decode launch may need a hundred.
-struct WmapKey {
-    const void *p;
-    int64_t N, K;
-    bool operator==(const WmapKey &o) const { return p == o.p && N == o.N && K == o.K; }
-};
-struct WmapHash {
-    size_t operator()(const WmapKey &k) const {
-        return std::hash<const void *>()(k.p) ^ (std::hash<int64_t>()(k.N) * 31u) ^ (std::hash<int64_t>()(k.K) * 131u);
-    }
-};
-std::mutex g_wmap_mu;
-std::unordered_map<WmapKey, CUtensorMap, WmapHash> g_wmap;
-
-bl_status dec_wmap(const uint8_t *packed, int64_t N, int64_t K, CUtensorMap *out) {
-    const WmapKey key{packed, N, K};
-    std::lock_guard<std::mutex> lk(g_wmap_mu);
-    auto it = g_wmap.find(key);
-    if (it != g_wmap.end()) {
-        *out = it->second;
-        return BL_OK;
-    }
-    EncodeTiledFn enc = encode_tiled_fn();
-    if (enc == nullptr) return BL_ERR_CUDA;
-    const cuuint64_t gdim[2] = {(cuuint64_t)(K / 4), (cuuint64_t)N};
-    const cuuint64_t gstride[1] = {(cuuint64_t)(K / 4)};
-    const cuuint32_t box[2] = {(cuuint32_t)DEC_CB, (cuuint32_t)DEC_ROWS};
-    const cuuint32_t es[2] = {1, 1};
-    CUtensorMap m;
-    if (enc(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t *>(packed), gdim, gstride, box, es,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return BL_ERR_CUDA;
-    if (g_wmap.size() >= 8192) g_wmap.clear();
-    g_wmap.emplace(key, m);
-    *out = m;
-    return BL_OK;
-}
-
-// Decode launch: groups of 32 weight rows over all problems, cut into one
-// contiguous range per CTA with about equal packed bytes (cut before the
-// first group whose midpoint passes the next multiple of total / SMs), then
-// split further at problem boundaries so that no CTA stages more than
-// DEC_MAX_PSLOTS problems' activations or, when it can be avoided, more than
-// DEC_X_PAIR bytes of them (two CTAs per SM).
+// Decode launches: each problem's 32-row groups cut into CTAs of T = 8 / G
+// groups (G from K, raised to 8 when the problems are too few to fill the
+// GPU); a CTA table maps each CTA to its problem.  A call with more CTAs or
+// problems than one launch holds is split into several launches (a problem
+// by row ranges).
 bl_status decode_launch(const DecodeJob *jobs, int count, int M, float eps, bool pdl, cudaStream_t st, int src,
                         int sms) {
     thread_local DecodeParams P;
-    P.count = count;
+    int glog[BL_MAX_GROUP];
+    int64_t total = 0;
+    for (int i = 0; i < count; ++i) {
+        glog[i] = dec_glog_p((int)jobs[i].K);
+        const int64_t ng = (jobs[i].N + DEC_ROWS - 1) / DEC_ROWS;
+        total += (ng + (DEC_WARPS >> glog[i]) - 1) / (DEC_WARPS >> glog[i]);
+    }
+    if (total < sms)
+        for (int i = 0; i < count; ++i) glog[i] = 3;
+    const int NT = M <= 8 ? 1 : 2;
     P.M = M;
     P.eps = eps;
-    int64_t G = 0;
-    double total = 0.0;
+    P.count = 0;
+    int nc = 0, w_max = 0, rs_max = 0, t_max = 0;
+    bool first = true;
+    auto flush = [&]() -> bl_status {
+        if (P.count == 0) return BL_OK;
+        P.x_off = (w_max + DEC_W_PAD + 127) & ~127;
+        P.acc_off = P.x_off + ((M * rs_max + 127) & ~127);
+        const size_t smem = (size_t)P.acc_off + (size_t)t_max * DEC_ROWS * M * 4;
+        if (M * rs_max > DEC_X_MAX || smem > DEC_SMEM_ATTR) return BL_ERR_SHAPE;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)nc);
+        cfg.blockDim = dim3(DEC_THREADS);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = pdl || !first ? 1 : 0;
+        cudaError_t e;
+        if (src == DEC_SRC_BF16)
+            e = NT == 1 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_BF16>, P)
+                        : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_BF16>, P);
+        else if (src == DEC_SRC_F32)
+            e = NT == 1 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_F32>, P)
+                        : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_F32>, P);
+        else
+            e = NT == 1 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_XQ>, P)
+                        : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_XQ>, P);
+        if (e != cudaSuccess) return BL_ERR_CUDA;
+        first = false;
+        P.count = 0;
+        nc = w_max = rs_max = t_max = 0;
+        return BL_OK;
+    };
     for (int i = 0; i < count; ++i) {
         const DecodeJob &j = jobs[i];
-        bl_status rc = dec_wmap(j.packed, j.N, j.K, &P.wmap[i]);
-        if (rc) return rc;
-        P.p[i] = DecodeProblem{j.gamma, j.x, j.s, j.Y, j.acc, j.gain, j.xq_out, (int)j.N, (int)j.K, (int)G};
-        G += (j.N + DEC_ROWS - 1) / DEC_ROWS;
-        if (G > 0x7fffffffLL) return BL_ERR_SHAPE;
-        total += (double)j.N * (double)(j.K / 4);
-    }
-    P.ngroups = (int)G;
-    const int base_ctas = sms < 1 ? 1 : (sms > DEC_MAX_CTAS - BL_MAX_GROUP ? DEC_MAX_CTAS - BL_MAX_GROUP : sms);
-    const double target = total / base_ctas;
-    int cuts[DEC_MAX_CTAS + 1];
-    int ncut = 0;
-    cuts[ncut++] = 0;
-    double c0 = 0.0, next = target;
-    for (int i = 0; i < count; ++i) {
-        const int64_t ng = (jobs[i].N + DEC_ROWS - 1) / DEC_ROWS;
-        const double gb = (double)DEC_ROWS * (double)(jobs[i].K / 4);
-        while (next < c0 + (double)ng * gb && ncut < base_ctas) {
-            // the first group whose byte midpoint lies past `next` (the next
-            // problem's first group when it is none of this problem's)
-            int64_t k = (int64_t)std::floor((next - c0) / gb - 0.5) + 1;
-            if (k < 0) k = 0;
-            if (k > ng) k = ng;
-            const int64_t g = P.p[i].gbase + k;
-            if (g < G && g > cuts[ncut - 1]) cuts[ncut++] = (int)g;
-            next += target;
-        }
-        c0 += (double)ng * gb;
-    }
-    cuts[ncut] = (int)G;  // end sentinel (not a CTA start)
-    // split at problem boundaries for the activation staging
-    int nc = 0;
-    int max_x = 0;
-    for (int c = 0; c < ncut; ++c) {
-        const int a = cuts[c], b = cuts[c + 1];
-        P.cta_g[nc++] = a;
-        // problems of [a, b)
-        int pi = 0;
-        while (pi + 1 < count && P.p[pi + 1].gbase <= a) ++pi;
-        int xb = 0, np = 0;
-        for (; pi < count && P.p[pi].gbase < b; ++pi) {
-            const int xp = M * dec_row_stride(P.p[pi].K);
-            if (np > 0 && (np == DEC_MAX_PSLOTS || xb + xp > DEC_X_PAIR)) {
-                if (nc >= DEC_MAX_CTAS) return BL_ERR_SHAPE;
-                max_x = xb > max_x ? xb : max_x;
-                P.cta_g[nc++] = P.p[pi].gbase;
-                xb = 0;
-                np = 0;
+        const int N = (int)j.N, K = (int)j.K;
+        const int T = DEC_WARPS >> glog[i];
+        const int kch = dec_kch(K);
+        const int wb = kch > 1 ? DEC_ROWS * DEC_KCH_B : T * DEC_ROWS * (K >> 2);
+        for (int row = 0; row < N;) {
+            if (P.count == BL_MAX_GROUP || nc == DEC_MAX_CTAS) {
+                bl_status rc = flush();
+                if (rc) return rc;
             }
-            xb += xp;
-            ++np;
+            const int need = (N - row + T * DEC_ROWS - 1) / (T * DEC_ROWS);
+            const int cn = need < DEC_MAX_CTAS - nc ? need : DEC_MAX_CTAS - nc;
+            const int nrows = cn * T * DEC_ROWS < N - row ? cn * T * DEC_ROWS : N - row;
+            P.p[P.count] = DecodeProblem{j.packed, j.gamma, j.x, j.s, j.Y, j.acc, j.gain, j.xq_out,
+                                         N, K, row, nrows, glog[i], nc, kch};
+            for (int c = 0; c < cn; ++c) P.cta_problem[nc + c] = (unsigned char)P.count;
+            nc += cn;
+            ++P.count;
+            row += nrows;
+            w_max = wb > w_max ? wb : w_max;
+            rs_max = dec_row_stride(K) > rs_max ? dec_row_stride(K) : rs_max;
+            t_max = T > t_max ? T : t_max;
         }
-        max_x = xb > max_x ? xb : max_x;
     }
-    P.cta_g[nc] = (int)G;
-    P.ncta = nc;
-    const int NT = M <= 8 ? 1 : 2;
-    const size_t smem = (size_t)dec_fixed_smem(NT) + (size_t)max_x + 1024;
-    if (max_x > DEC_X_MAX || smem > DEC_SMEM_ATTR) return BL_ERR_SHAPE;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)nc);
-    cfg.blockDim = dim3(DEC_THREADS);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    cudaError_t e;
-    if (src == DEC_SRC_BF16)
-        e = NT == 1 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_BF16>, P)
-                    : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_BF16>, P);
-    else if (src == DEC_SRC_F32)
-        e = NT == 1 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_F32>, P)
-                    : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_F32>, P);
-    else
-        e = NT == 1 ? cudaLaunchKernelEx(&cfg, k_decode<1, DEC_SRC_XQ>, P)
-                    : cudaLaunchKernelEx(&cfg, k_decode<2, DEC_SRC_XQ>, P);
-    return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
+    return flush();
 }
 
 bl_status forward_impl(const DeviceInfo &d, const uint8_t *packed, const float *gamma, const int8_t *x_q,

@@ -4,55 +4,43 @@
 //   acc[m, n] = sum_k x_q[m, k] * W_q[n, k];  Y[m, n] = acc * (gamma / s[m])
 //
 // The work is bound by streaming the packed weights from HBM (2 bits per
-// weight).  Design (one CTA per SM and launch, small enough that the CTA of
-// the next launch fits beside it):
-//   - Work unit: a group of 32 weight rows of one problem.  The host cuts the
-//     flattened group list of all problems into one contiguous range per CTA
-//     with about equal packed bytes.  Inside the CTA every warp takes whole
-//     groups: its first one by its index, the next ones from a shared
-//     counter as it needs them, so warps that meet short groups take more.
-//   - Streaming: each warp owns a ring of DEC_WSTAGES shared-memory stages.
-//     Its lane 0 cuts its groups into chunks of 32 rows x 128 bytes (512 k)
-//     and requests each with a 2-D TMA tensor load (per-problem tensor map,
-//     128-byte swizzle, L2 evict-first: each byte is read once) as soon as
-//     the warp has consumed the stage, DEC_WSTAGES chunks ahead of its
-//     compute; the first requests go out before griddepcontrol.wait, so a
-//     programmatic dependent launch (BL_FWD_WEIGHTS_READY) streams its
-//     weights while the launch before it finishes.  A warp consumes only its
-//     own stages, in order: no cross-warp synchronization on the stream.
-//   - MACs on the tensor cores (mma.sync m16n8k32 s8): weight rows as A (two
-//     16-row tiles per chunk share every x_q fragment), tokens as B (8
-//     columns per tile, zero for m >= M).  The int32 sum is exact, so the k
-//     order inside a 256-k step may be permuted as long as A and B use the
-//     same permutation: the lane with k-slot t holds the packed bytes
-//     64t .. 64t + 15 of the step, and its B fragment reads those x_q bytes.
-//     A group's accumulators stay in the warp's registers over its chunks;
-//     the warp rescales them and writes Y when the group's last chunk is in.
-//   - Unpacking costs one AND per 4 weights: a packed word holds the codes
-//     c = 1 - W_q in {0, 1, 2}; word & (0x03030303 << 2j) leaves the codes of
-//     k = 16w' + 4j .. 4j+3 in four bytes as the unsigned values 4^j c, which
-//     the MMA takes as u8 (A) against the s8 activations (B), one accumulator
-//     per plane j.  Then sum_k W_q x = sum_k x - sum_j D_j / 4^j (each D_j a
-//     multiple of 4^j, so the shifts are exact), with sum_k x the row sum of
-//     the staged x_q.  At M > 8 (two token tiles) the planes are moved to the
-//     top two bits instead ((w << (6 - 2j)) & 0xC0C0C0C0, 64 c) and share one
-//     accumulator per tile, to keep the registers of the second tile.
-//   - Lane (g, t) of an MMA tile reads weight rows pi(g) and pi(g) + 8 with
-//     pi(g) = (g >> 1) | ((g & 1) << 2): with the 128-byte swizzle, the eight
-//     lanes of each quarter warp then hit eight different bank quads.
-//   - x_q is staged once per CTA and problem in shared memory (rows of
-//     round_up(K, 256) bytes, 16-byte chunks XOR-swizzled so that the B loads
-//     are free of bank conflicts).  Fused variant (SRC = bf16 or f32
-//     activations): step 2 runs inside the CTA with the same arithmetic as
-//     the stand-alone activation quantizer (rows without SubLN by the whole
-//     CTA at once, SubLN rows one warp per row); the CTA holding a problem's
-//     first group also writes x_q and s on request.
-//   - Every mbarrier wait is bounded (globaltimer); a wait that gives up
-//     raises the device error word and the CTA's abort flag, and each warp
-//     then waits (bounded) for its own copies in flight before it exits.
+// weight).  Design:
+//   - A CTA owns a contiguous range of whole 32-row groups of one problem,
+//     at most DEC_W_CAP packed bytes, so that three CTAs (of this launch or
+//     of the next) share an SM.  Its rows are one contiguous byte range of
+//     the packed matrix: lane 0 of the last warp requests them with one bulk
+//     copy (cp.async.bulk, L2 evict-first) per group into shared memory, one
+//     mbarrier per group, before waiting on the launch before this one: the
+//     weights are static, so with BL_FWD_WEIGHTS_READY (a programmatic
+//     dependent launch) a CTA that lands on an SM while that launch finishes
+//     streams its weights at once.
+//   - The CTA's 8 warps split its groups: G = 8 / T warps per group (T
+//     groups per CTA) take every G-th 256-k step of it, G chosen per problem
+//     from K so that a warp has a few steps.  Partial sums meet in shared
+//     memory (int32, exact), and the CTA writes Y with a thread per (token,
+//     row), 32 consecutive floats per warp and token.
+//   - MACs on the tensor cores (mma.sync m16n8k32, u8 x s8): weight rows as
+//     A (two 16-row tiles per group share every x_q fragment), tokens as B (8
+//     columns per tile; the columns m >= M read token M - 1 and are never
+//     stored).  The int32 sum is exact, so the k order inside a step may be
+//     permuted as long as A and B use the same permutation: the lane with
+//     k-slot t holds the packed bytes 16t .. 16t + 15 of the step (k = 64t ..
+//     64t + 63), and its B fragment reads those x_q bytes.
+//   - Unpacking: a packed word holds the codes c = 1 - W_q in {0, 1, 2};
+//     (word << (6 - 2j)) & 0xC0C0C0C0 leaves the codes of k = 16w' + 4j ..
+//     4j+3 in the top two bits of four bytes, the unsigned values 64 c, so
+//     every plane shares one accumulator per tile:
+//     sum_k W_q x = sum_k x - (sum_k 64 c x) / 64, exact (a multiple of 64),
+//     with sum_k x the row sum of the staged x_q.
+//   - x_q is staged once per CTA in shared memory (rows of round_up(K, 256)
+//     bytes, 16-byte chunks XOR-swizzled so that the B loads are free of
+//     bank conflicts).  Fused variant (SRC = bf16 or f32 activations): step
+//     2 runs inside the CTA with the same arithmetic as the stand-alone
+//     activation quantizer (a warp per row without SubLN, from registers
+//     after one load, or the whole CTA in rounds for long rows; SubLN rows a
+//     warp per row); the problem's first CTA also writes x_q and s on
+//     request.
 #pragma once
-
-#include <cuda.h>
 
 #include "bl_common.cuh"
 
@@ -60,44 +48,63 @@ namespace bl {
 
 constexpr int DEC_WARPS = 8;
 constexpr int DEC_THREADS = 32 * DEC_WARPS;
-constexpr int DEC_ROWS = 32;                          // weight rows per group (two MMA tiles)
-constexpr int DEC_CB = 128;                           // packed bytes per row per chunk (512 k)
-constexpr int DEC_CHUNK = DEC_ROWS * DEC_CB;          // 4 KiB
-constexpr int DEC_WSTAGES = 2;                        // ring stages per warp
-constexpr int DEC_MAX_PSLOTS = 8;                     // problems per CTA
-constexpr int DEC_MAX_CTAS = 320;
-constexpr int DEC_X_MAX = 144 * 1024;                 // staged activations per CTA
-constexpr int DEC_X_PAIR = 36 * 1024;                 // ... at most this keeps two CTAs per SM
+constexpr int DEC_ROWS = 32;                // weight rows per group (two MMA tiles)
+constexpr int DEC_PF = 4;                   // target 256-k steps per warp (G is chosen from it)
+constexpr int DEC_W_CAP = 48 * 1024;        // packed bytes per CTA above which G grows (three CTAs per SM)
+constexpr int DEC_MAX_CTAS = 2048;          // CTAs per launch (larger calls are split into launches)
+constexpr int DEC_X_MAX = 144 * 1024;       // staged activations per CTA
+constexpr int DEC_MAX_PSLOTS = 1;           // problems per CTA (the staging helpers take a slot array)
 constexpr unsigned long long DEC_TIMEOUT_NS = 2000000000ull;
-
-__host__ __device__ constexpr int dec_fixed_smem(int) { return DEC_WARPS * DEC_WSTAGES * DEC_CHUNK; }
 
 // Activation source of a launch: pre-quantized x_q, or X to quantize in-kernel.
 enum : int { DEC_SRC_XQ = 0, DEC_SRC_BF16 = 1, DEC_SRC_F32 = 2 };
 
 struct DecodeProblem {
+    const uint8_t *packed; // [N, K/4], 16-byte aligned
     const float *gamma;
     const void *x;         // DEC_SRC_XQ: x_q [M, K] int8; else X [M, K] bf16 / f32
     float *s;              // DEC_SRC_XQ: s [M] in; else s [M] out or null
-    float *Y;
-    int32_t *acc;
+    float *Y;              // [M, N]
+    int32_t *acc;          // [M, N] or null
     const float *gain;     // fused: SubLN gain [K] or null
     int8_t *xq_out;        // fused: x_q [M, K] out or null
-    int N;
-    int K;
-    int gbase;             // first group of this problem in the flattened group list
+    int N, K;
+    int row0;              // first row of this launch's part of the problem
+    int rows;              // rows of that part
+    int glog;              // log2(G): warps per group
+    int cta_begin;         // first CTA of this problem in the launch
+    int kch;               // K chunks: 1, or (K > DEC_K_WHOLE) one group per CTA in chunks of DEC_KCH_B bytes a row
 };
 
 struct DecodeParams {
-    CUtensorMap wmap[BL_MAX_GROUP];  // packed weights per problem: {K/4 bytes, N rows}, box 128 x 32, 128B swizzle
     DecodeProblem p[BL_MAX_GROUP];
     int count;
     int M;
-    int ngroups;
-    int ncta;
-    float eps;                        // fused: SubLN epsilon
-    int cta_g[DEC_MAX_CTAS + 1];      // CTA c owns groups [cta_g[c], cta_g[c + 1])
+    float eps;                                 // fused: SubLN epsilon
+    int x_off;                                 // shared-memory offsets of the staged x_q and of the sums
+    int acc_off;
+    unsigned char cta_problem[DEC_MAX_CTAS];   // problem of each CTA
 };
+
+// A problem as one CTA sees it, in shared memory.
+struct DecSlot {
+    const void *x;
+    float *s;
+    const float *gain;
+    int8_t *xq_out;
+    int K;
+    int first;  // this CTA holds the problem's first rows (writes x_q and s on request)
+};
+
+__host__ __device__ inline int dec_glog(int K) {
+    // smallest G = 2^glog <= 8 with ceil(steps / G) <= DEC_PF and at most
+    // DEC_W_CAP bytes of weights per CTA (8 / G groups of 32 rows)
+    const int steps = (K + 255) >> 8;
+    int g = 0;
+    while (g < 3 && ((steps + (1 << g) - 1) >> g) > DEC_PF) ++g;
+    while (g < 3 && (DEC_WARPS >> g) * DEC_ROWS * (K >> 2) > DEC_W_CAP) ++g;
+    return g;
+}
 
 __host__ __device__ inline int dec_row_stride(int K) { return (K + 255) & ~255; }
 
@@ -211,7 +218,7 @@ __device__ __forceinline__ void dec_y4(const uint4 &raw, int q, const float4 *g4
 //   s = float(127 / max(max|y|, 1e-5f)),  x_q = clamp(rne(float(y * s)), -128, 127)
 // Returns s (on every lane).
 template <bool BF16>
-__device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, uint8_t *s_xq, float eps, bool out,
+__device__ float dec_quant_row(const DecSlot &pr, int m, int K, int RS, uint8_t *s_xq, float eps, bool out,
                                int lane, int *rowsum) {
     constexpr int EPV = BF16 ? 8 : 4;
     const int nvec = K / EPV;
@@ -299,398 +306,449 @@ __device__ float dec_quant_row(const DecodeProblem &pr, int m, int K, int RS, ui
 }
 
 // Step 2 for all (problem, token) rows of a CTA at once, rows without SubLN:
-// every thread takes the 16-byte vectors t, t + DEC_THREADS, ... of the
-// concatenated rows with all its loads in flight together (one memory round
-// trip for the CTA instead of one per row and warp), the row maxima meet in
-// shared memory (max of the float bits of |x|), and each thread then
-// quantizes its vectors into the staging rows.  Same arithmetic as
-// dec_quant_row.  vbase[ps] = first vector of problem slot ps (vbase[np] =
-// the total, at most DEC_QBV * DEC_THREADS); s_amax[np * M] zeroed before.
-constexpr int DEC_QBV = 12;
+// the concatenated rows are taken in rounds of DEC_QBV * DEC_THREADS 16-byte
+// vectors, every thread holding the vectors t, t + DEC_THREADS, ... of a
+// round with all its loads in flight together (one memory round trip per
+// round for the CTA, not one per row and warp).  Pass 1 meets the row maxima
+// in shared memory (max of the float bits of |x|); pass 2 quantizes each
+// vector into the staging rows, the rounds in reverse order so that the one
+// still in registers is not loaded again.  Same arithmetic as dec_quant_row.
+// vbase[ps] = first vector of problem slot ps (vbase[np] = the total);
+// s_amax[np * M] and s_rs[np * M] zeroed before.
+constexpr int DEC_QBV = 8;
 
 template <bool BF16>
-__device__ void dec_quant_block(const DecodeParams &P, int p_lo, int np, int g_begin, const int *s_xoff,
-                                const int *vbase, uint8_t *s_x, u32 *s_amax, float *s_sc, float (*s_f)[16],
-                                int *s_rs) {
+__device__ void dec_quant_block(const DecSlot *sl, int np, int M, const int *s_xoff, const int *vbase, uint8_t *s_x,
+                                u32 *s_amax, float *s_sc, const float *s_gam, float (*s_f)[16], int *s_rs) {
     constexpr int EPV = BF16 ? 8 : 4;
-    const int M = P.M, T = vbase[np];
+    constexpr int RV = DEC_QBV * DEC_THREADS;  // vectors per round
+    const int T = vbase[np];
+    const int rounds = (T + RV - 1) / RV;
     const int lane = threadIdx.x & 31;
     uint4 c[DEC_QBV];
     int meta[DEC_QBV];  // (slot << 20) | (m << 16) | vector within the row; -1 past the end
+    auto load_round = [&](int rd) {
 #pragma unroll
-    for (int i = 0; i < DEC_QBV; ++i) {
-        const int idx = (int)threadIdx.x + DEC_THREADS * i;
-        meta[i] = -1;
-        c[i] = make_uint4(0, 0, 0, 0);
-        if (idx < T) {
-            int ps = 0;
-            while (ps + 1 < np && idx >= vbase[ps + 1]) ++ps;
-            const int nvec = P.p[p_lo + ps].K / EPV;
-            const int local = idx - vbase[ps];
-            const int m = local / nvec, v = local - m * nvec;
-            meta[i] = (ps << 20) | (m << 16) | v;
-            c[i] = ldg_nc_v4(reinterpret_cast<const uint4 *>(P.p[p_lo + ps].x) + (size_t)m * nvec + v);
+        for (int i = 0; i < DEC_QBV; ++i) {
+            const int idx = rd * RV + (int)threadIdx.x + DEC_THREADS * i;
+            meta[i] = -1;
+            c[i] = make_uint4(0, 0, 0, 0);
+            if (idx < T) {
+                int ps = 0;
+                while (ps + 1 < np && idx >= vbase[ps + 1]) ++ps;
+                const int nvec = sl[ps].K / EPV;
+                const int local = idx - vbase[ps];
+                const int m = local / nvec, v = local - m * nvec;
+                meta[i] = (ps << 20) | (m << 16) | v;
+                c[i] = ldg_nc_v4(reinterpret_cast<const uint4 *>(sl[ps].x) + (size_t)m * nvec + v);
+            }
         }
-    }
+    };
+    for (int rd = 0; rd < rounds; ++rd) {
+        load_round(rd);
 #pragma unroll
-    for (int i = 0; i < DEC_QBV; ++i) {
-        if (DEC_THREADS * i >= T) break;  // uniform: no vector of this round is in range
-        u32 a = 0;
+        for (int i = 0; i < DEC_QBV; ++i) {
+            if (rd * RV + DEC_THREADS * i >= T) break;  // uniform: no vector of this row of the round is in range
+            u32 a = 0;
 #pragma unroll
-        for (int j = 0; j < EPV; ++j) a = max(a, dec_x_bits<BF16>(c[i], j) & 0x7fffffffu);
-        const int row = meta[i] < 0 ? -1 : ((meta[i] >> 20) * M + ((meta[i] >> 16) & 15));
-        const int row0 = __shfl_sync(0xffffffffu, row, 0);
-        if (__all_sync(0xffffffffu, row == row0)) {
-            a = __reduce_max_sync(0xffffffffu, a);
-            if (lane == 0 && row0 >= 0) atomicMax(&s_amax[row0], a);
-        } else if (row >= 0) {
-            atomicMax(&s_amax[row], a);
+            for (int j = 0; j < EPV; ++j) a = max(a, dec_x_bits<BF16>(c[i], j) & 0x7fffffffu);
+            const int row = meta[i] < 0 ? -1 : ((meta[i] >> 20) * M + ((meta[i] >> 16) & 15));
+            const int row0 = __shfl_sync(0xffffffffu, row, 0);
+            if (__all_sync(0xffffffffu, row == row0)) {
+                a = __reduce_max_sync(0xffffffffu, a);
+                if (lane == 0 && row0 >= 0) atomicMax(&s_amax[row0], a);
+            } else if (row >= 0) {
+                atomicMax(&s_amax[row], a);
+            }
         }
     }
     __syncthreads();
     for (int r = threadIdx.x; r < np * M; r += DEC_THREADS) {
         const int ps = r / M, m = r - ps * M;
-        const DecodeProblem &pr = P.p[p_lo + ps];
         const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(s_amax[r]), 1e-5f));
         s_sc[r] = s;
-        s_f[ps][m] = __fdiv_rn(*pr.gamma, s);
-        if (g_begin <= pr.gbase && pr.s != nullptr) pr.s[m] = s;
+        s_f[ps][m] = __fdiv_rn(s_gam[ps], s);
+        if (sl[ps].first && sl[ps].s != nullptr) sl[ps].s[m] = s;
     }
     __syncthreads();
+    for (int rd = rounds - 1; rd >= 0; --rd) {
+        if (rd != rounds - 1) load_round(rd);
 #pragma unroll
-    for (int i = 0; i < DEC_QBV; ++i) {
-        if (DEC_THREADS * i >= T) break;  // uniform: no vector of this round is in range
-        int rsum = 0;
-        const int row = meta[i] < 0 ? -1 : ((meta[i] >> 20) * M + ((meta[i] >> 16) & 15));
-        if (meta[i] >= 0) {
-        const int ps = meta[i] >> 20, m = (meta[i] >> 16) & 15, v = meta[i] & 0xffff;
-        const DecodeProblem &pr = P.p[p_lo + ps];
-        const int K = pr.K, RS = dec_row_stride(K);
-        const float s = s_sc[ps * M + m];
-        u32 word[EPV / 4];
+        for (int i = 0; i < DEC_QBV; ++i) {
+            if (rd * RV + DEC_THREADS * i >= T) break;  // uniform
+            int rsum = 0;
+            const int row = meta[i] < 0 ? -1 : ((meta[i] >> 20) * M + ((meta[i] >> 16) & 15));
+            if (meta[i] >= 0) {
+                const int ps = meta[i] >> 20, m = (meta[i] >> 16) & 15, v = meta[i] & 0xffff;
+                const DecSlot &pr = sl[ps];
+                const int K = pr.K, RS = dec_row_stride(K);
+                const float s = s_sc[ps * M + m];
+                u32 word[EPV / 4];
 #pragma unroll
-        for (int q = 0; q < EPV / 4; ++q) {
-            u32 w = 0;
+                for (int q = 0; q < EPV / 4; ++q) {
+                    u32 w = 0;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                int qi = __float2int_rn(__fmul_rn(__uint_as_float(dec_x_bits<BF16>(c[i], 4 * q + j)), s));
-                qi = max(-128, min(127, qi));
-                rsum += qi;
-                w |= ((u32)qi & 0xffu) << (8 * j);
+                    for (int j = 0; j < 4; ++j) {
+                        int qi = __float2int_rn(__fmul_rn(__uint_as_float(dec_x_bits<BF16>(c[i], 4 * q + j)), s));
+                        qi = max(-128, min(127, qi));
+                        rsum += qi;
+                        w |= ((u32)qi & 0xffu) << (8 * j);
+                    }
+                    word[q] = w;
+                }
+                const int L = BF16 ? (v >> 1) : (v >> 2);
+                const int within = BF16 ? (v & 1) * 8 : (v & 3) * 4;
+                const int x = (((L >> 3) & 1) << 1) | (m & 1);
+                uint8_t *d = s_x + s_xoff[ps] + m * RS + ((((L & ~7) | ((L ^ x) & 7)) << 4) + within);
+                int8_t *gq = (pr.first && pr.xq_out != nullptr) ? pr.xq_out + (size_t)m * K : nullptr;
+                if (BF16) {
+                    *reinterpret_cast<uint2 *>(d) = make_uint2(word[0], word[EPV / 4 - 1]);
+                    if (gq) *reinterpret_cast<uint2 *>(gq + (size_t)v * 8) = make_uint2(word[0], word[EPV / 4 - 1]);
+                } else {
+                    *reinterpret_cast<u32 *>(d) = word[0];
+                    if (gq) *reinterpret_cast<u32 *>(gq + (size_t)v * 4) = word[0];
+                }
             }
-            word[q] = w;
+            // the row sums of x_q, one shared atomic per warp when its vectors share a row
+            const int row0 = __shfl_sync(0xffffffffu, row, 0);
+            if (__all_sync(0xffffffffu, row == row0)) {
+                rsum = __reduce_add_sync(0xffffffffu, rsum);
+                if (lane == 0 && row0 >= 0) atomicAdd(&s_rs[row0], rsum);
+            } else if (row >= 0) {
+                atomicAdd(&s_rs[row], rsum);
+            }
         }
-        const int L = BF16 ? (v >> 1) : (v >> 2);
-        const int within = BF16 ? (v & 1) * 8 : (v & 3) * 4;
-        const int x = (((L >> 3) & 1) << 1) | (m & 1);
-        uint8_t *d = s_x + s_xoff[ps] + m * RS + ((((L & ~7) | ((L ^ x) & 7)) << 4) + within);
-        int8_t *gq = (g_begin <= pr.gbase && pr.xq_out != nullptr) ? pr.xq_out + (size_t)m * K : nullptr;
+    }
+}
+
+// Step 2 for rows without SubLN of at most DEC_RJ 16-byte vectors per lane
+// (K <= 2048 for bf16, 1024 for f32): warp w quantizes the rows w, w +
+// DEC_WARPS, ... (row = slot * M + token) from registers after one load
+// each.
+// Same arithmetic as dec_quant_row: s = float(127 / max(max|x|, 1e-5f)),
+// x_q = clamp(rne(float(x * s)), -128, 127).
+constexpr int DEC_RJ = 8;
+
+template <bool BF16>
+__device__ __forceinline__ void dec_row_load(uint4 (&c)[DEC_RJ], const DecSlot *sl, int M, int r, int lane) {
+    constexpr int EPV = BF16 ? 8 : 4;
+    const int ps = r / M, m = r - ps * M;
+    const int nvec = sl[ps].K / EPV;
+    const uint4 *xr = reinterpret_cast<const uint4 *>(sl[ps].x) + (size_t)m * nvec;
+#pragma unroll
+    for (int j = 0; j < DEC_RJ; ++j) {
+        const int v = lane + 32 * j;
+        c[j] = v < nvec ? ldg_nc_v4(xr + v) : make_uint4(0, 0, 0, 0);
+    }
+}
+
+// four products x * s rounded to the nearest even integer, saturated to
+// int8 and packed, the first in the low byte
+__device__ __forceinline__ u32 dec_q4(u32 a, u32 b, u32 c, u32 d, float s) {
+    const int qa = __float2int_rn(__fmul_rn(__uint_as_float(a), s));
+    const int qb = __float2int_rn(__fmul_rn(__uint_as_float(b), s));
+    const int qc = __float2int_rn(__fmul_rn(__uint_as_float(c), s));
+    const int qd = __float2int_rn(__fmul_rn(__uint_as_float(d), s));
+    u32 hi, w;
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(qd), "r"(qc));
+    asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(w) : "r"(qb), "r"(qa), "r"(hi));
+    return w;
+}
+
+template <bool BF16>
+__device__ __forceinline__ void dec_row_quant(const uint4 (&c)[DEC_RJ], const DecSlot *sl, int M, int r,
+                                              uint8_t *s_x, const int *s_xoff, const float *s_gam, float (*s_f)[16],
+                                              int *s_rs, int lane) {
+    constexpr int EPV = BF16 ? 8 : 4;
+    const int ps = r / M, m = r - ps * M;
+    const DecSlot &pr = sl[ps];
+    const int K = pr.K, nvec = K / EPV, RS = dec_row_stride(K);
+    // max |x| as float bits (bf16: 16-bit magnitudes, two per word)
+    u32 am = 0;
+#pragma unroll
+    for (int j = 0; j < DEC_RJ; ++j) {
         if (BF16) {
-            *reinterpret_cast<uint2 *>(d) = make_uint2(word[0], word[EPV / 4 - 1]);
-            if (gq) *reinterpret_cast<uint2 *>(gq + (size_t)v * 8) = make_uint2(word[0], word[EPV / 4 - 1]);
+            const u32 p = __vmaxu2(__vmaxu2(c[j].x & 0x7fff7fffu, c[j].y & 0x7fff7fffu),
+                                   __vmaxu2(c[j].z & 0x7fff7fffu, c[j].w & 0x7fff7fffu));
+            am = __vmaxu2(am, p);
         } else {
-            *reinterpret_cast<u32 *>(d) = word[0];
-            if (gq) *reinterpret_cast<u32 *>(gq + (size_t)v * 4) = word[0];
+            am = max(am, max(max(c[j].x & 0x7fffffffu, c[j].y & 0x7fffffffu),
+                             max(c[j].z & 0x7fffffffu, c[j].w & 0x7fffffffu)));
         }
+    }
+    if (BF16) am = max(am >> 16, am & 0xffffu) << 16;
+    am = __reduce_max_sync(0xffffffffu, am);
+    const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(am), 1e-5f));
+    uint8_t *dst = s_x + s_xoff[ps] + m * RS;
+    int8_t *gq = pr.first && pr.xq_out != nullptr ? pr.xq_out + (size_t)m * K : nullptr;
+    int rs = 0;
+#pragma unroll
+    for (int j = 0; j < DEC_RJ; ++j) {
+        const int v = lane + 32 * j;
+        if (v < nvec) {
+            // 16-byte chunk L of the row holds k = 16L .. 16L + 15
+            const int L = BF16 ? (v >> 1) : (v >> 2);
+            const int within = BF16 ? (v & 1) * 8 : (v & 3) * 4;
+            const int x = (((L >> 3) & 1) << 1) | (m & 1);
+            uint8_t *d = dst + ((((L & ~7) | ((L ^ x) & 7)) << 4) + within);
+            if (BF16) {
+                const u32 w0 = dec_q4(c[j].x << 16, c[j].x & 0xffff0000u, c[j].y << 16, c[j].y & 0xffff0000u, s);
+                const u32 w1 = dec_q4(c[j].z << 16, c[j].z & 0xffff0000u, c[j].w << 16, c[j].w & 0xffff0000u, s);
+                rs = __dp4a((int)w1, 0x01010101, __dp4a((int)w0, 0x01010101, rs));
+                *reinterpret_cast<uint2 *>(d) = make_uint2(w0, w1);
+                if (gq) *reinterpret_cast<uint2 *>(gq + (size_t)v * 8) = make_uint2(w0, w1);
+            } else {
+                const u32 w0 = dec_q4(c[j].x, c[j].y, c[j].z, c[j].w, s);
+                rs = __dp4a((int)w0, 0x01010101, rs);
+                *reinterpret_cast<u32 *>(d) = w0;
+                if (gq) *reinterpret_cast<u32 *>(gq + (size_t)v * 4) = w0;
+            }
         }
-        // the row sums of x_q, one shared atomic per warp when its vectors share a row
-        const int row0 = __shfl_sync(0xffffffffu, row, 0);
-        if (__all_sync(0xffffffffu, row == row0)) {
-            rsum = __reduce_add_sync(0xffffffffu, rsum);
-            if ((threadIdx.x & 31) == 0 && row0 >= 0) atomicAdd(&s_rs[row0], rsum);
-        } else if (row >= 0) {
-            atomicAdd(&s_rs[row], rsum);
-        }
+    }
+    rs = __reduce_add_sync(0xffffffffu, rs);
+    if (lane == 0) {
+        s_rs[r] = rs;
+        s_f[ps][m] = __fdiv_rn(s_gam[ps], s);
+        if (pr.first && pr.s != nullptr) pr.s[m] = s;
     }
 }
 
-// problem owning flattened group g (binary search over the group bases)
-__device__ __forceinline__ int dec_problem_of(const DecodeParams &P, int g) {
-    int lo = 0, hi = P.count - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (P.p[mid].gbase <= g) lo = mid; else hi = mid - 1;
+template <bool BF16>
+__device__ void dec_quant_rows(const DecSlot *sl, int np, int M, uint8_t *s_x, const int *s_xoff, const float *s_gam,
+                               float (*s_f)[16], int *s_rs, int warp, int lane) {
+    uint4 c[DEC_RJ];
+    for (int r = warp; r < np * M; r += DEC_WARPS) {
+        dec_row_load<BF16>(c, sl, M, r, lane);
+        dec_row_quant<BF16>(c, sl, M, r, s_x, s_xoff, s_gam, s_f, s_rs, lane);
     }
-    return lo;
 }
 
-__device__ __forceinline__ int dec_nchunks(int K) { return (K + 4 * DEC_CB - 1) / (4 * DEC_CB); }
+__device__ __forceinline__ int dec_nsteps(int K) { return (K + 255) >> 8; }
 
-__device__ __forceinline__ void tma_load_2d_hint(u32 dst, const CUtensorMap *map, int x, int y, u32 bar, u64 pol) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
-        " [%0], [%1, {%2, %3}], [%4], %5;"
-        ::"r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar), "l"(pol)
-        : "memory");
+// Shared memory of a launch: the CTA's packed weights (at most
+// dec_w_bytes(K) + DEC_W_PAD), then at x_off the staged x_q (M rows of
+// round_up(K, 256) bytes), then at acc_off the sums (T groups x 32 rows x M).
+// Rows longer than DEC_K_WHOLE / 4 bytes are staged in chunks of DEC_KCH_B
+// bytes (one group per CTA; a bulk copy per row and chunk).
+constexpr int DEC_W_PAD = 256;  // reads of a row's last step may run past the copied bytes
+constexpr int DEC_K_WHOLE = 6144;
+constexpr int DEC_KCH_B = 2048;
+__host__ __device__ inline int dec_kch(int K) { return K <= DEC_K_WHOLE ? 1 : ((K >> 2) + DEC_KCH_B - 1) / DEC_KCH_B; }
+__host__ __device__ inline int dec_glog_p(int K) { return dec_kch(K) > 1 ? 3 : dec_glog(K); }
+__host__ __device__ inline int dec_w_bytes(int K) {
+    return dec_kch(K) > 1 ? DEC_ROWS * DEC_KCH_B : (DEC_WARPS >> dec_glog(K)) * DEC_ROWS * (K >> 2);
 }
 
 // NT: 8-token column tiles (1: M <= 8, 2: M <= 16).  SRC: DEC_SRC_*.
 template <int NT, int SRC>
-__global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant__ DecodeParams P) {
-    extern __shared__ uint8_t dsm_raw[];
-    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~(uintptr_t)1023);
-    __shared__ __align__(8) u64 s_full[DEC_WARPS][DEC_WSTAGES];
-    __shared__ int s_queue[DEC_WARPS][DEC_WSTAGES + 2];  // groups a warp has started requesting, in order
-    __shared__ int s_next;                               // next group to hand out
-    __shared__ float s_f[DEC_MAX_PSLOTS][16];
-    __shared__ int s_xoff[DEC_MAX_PSLOTS + 1];
-    __shared__ int s_vbase[DEC_MAX_PSLOTS + 1];
-    __shared__ u32 s_amax[DEC_MAX_PSLOTS * 16];
-    __shared__ float s_sc[DEC_MAX_PSLOTS * 16];
-    __shared__ int s_rs[DEC_MAX_PSLOTS * 16];  // row sums of the staged x_q
-    __shared__ volatile int s_abort;
+__global__ void __launch_bounds__(DEC_THREADS, 3) k_decode(const __grid_constant__ DecodeParams P) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ __align__(8) u64 s_bar[DEC_WARPS];
+    __shared__ DecSlot s_sl[1];
+    __shared__ float s_f[1][16];
+    __shared__ float s_gam[1];
+    __shared__ int s_xoff[2];
+    __shared__ int s_vbase[2];
+    __shared__ u32 s_amax[16];
+    __shared__ float s_sc[16];
+    __shared__ int s_rs[16];  // row sums of the staged x_q
 
     // a programmatically dependent launch that follows may start its prologue
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-    constexpr int QN = DEC_WSTAGES + 2;
+    const int b = blockIdx.x;
+    const DecodeProblem &pr = P.p[P.cta_problem[b]];
+    const int M = P.M, N = pr.N, K = pr.K;
+    const int glog = pr.glog, G = 1 << glog;
+    const int T = DEC_WARPS >> glog;  // 32-row groups per CTA
+    const int RB = K >> 2;            // packed bytes per row
+    const int rbase = pr.row0 + (b - pr.cta_begin) * T * DEC_ROWS;  // first row of this CTA
+    const int rows = min(T * DEC_ROWS, pr.row0 + pr.rows - rbase);
+    const int groups = (rows + DEC_ROWS - 1) / DEC_ROWS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g_begin = P.cta_g[blockIdx.x], g_end = P.cta_g[blockIdx.x + 1];
-    const int p_lo = dec_problem_of(P, g_begin), p_hi = dec_problem_of(P, g_end - 1);
-    const int np = p_hi - p_lo + 1;
-    const int M = P.M;
-    uint8_t *s_x = sm + dec_fixed_smem(NT);
+    uint8_t *s_x = smem + P.x_off;
+    int *s_acc = reinterpret_cast<int *>(smem + P.acc_off);
 
-    if (threadIdx.x == 0) {
-        for (int w = 0; w < DEC_WARPS; ++w)
-            for (int s = 0; s < DEC_WSTAGES; ++s) mbar_init(smem_u32(&s_full[w][s]), 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-        s_abort = 0;
-        s_next = g_begin + DEC_WARPS;
-        int off = 0, vb = 0;
-        for (int i = 0; i < np; ++i) {
-            s_xoff[i] = off;
-            s_vbase[i] = vb;
-            off += M * dec_row_stride(P.p[p_lo + i].K);
-            vb += M * (P.p[p_lo + i].K / (SRC == DEC_SRC_F32 ? 4 : 8));
+    // The weights are static: one thread requests the CTA's rows (one bulk
+    // copy per group, each with its own mbarrier) before the wait below.  It
+    // is lane 0 of the last warp, so that the first warps start staging the
+    // activations at once.
+    const int kch = pr.kch;
+    const int WS = kch > 1 ? DEC_KCH_B : RB;  // shared-memory row stride of the weights
+    const u64 policy = l2_policy_evict_first();  // read once per launch
+    // chunk c of the single group (kch > 1): row r's bytes [c DEC_KCH_B, ...)
+    // by lane r of the last warp, after lane 0 has set the expected bytes
+    auto request_chunk = [&](int c) {
+        const u32 cb = (u32)min(DEC_KCH_B, RB - c * DEC_KCH_B);
+        const u32 bar = smem_u32(&s_bar[0]);
+        if (lane == 0) mbar_arrive_expect_tx(bar, cb * (u32)rows);
+        __syncwarp();
+        if (lane < rows)
+            bulk_g2s_hint(smem_u32(smem + lane * DEC_KCH_B), pr.packed + (size_t)(rbase + lane) * RB + (size_t)c * DEC_KCH_B,
+                          cb, bar, policy);
+    };
+    if (warp == DEC_WARPS - 1) {
+        if (lane == 0) {
+            for (int i = 0; i < groups; ++i) mbar_init(smem_u32(&s_bar[i]), 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         }
-        s_xoff[np] = off;
-        s_vbase[np] = vb;
+        __syncwarp();
+        if (kch > 1) {
+            request_chunk(0);
+        } else if (lane == 0) {
+            const uint8_t *src = pr.packed + (size_t)rbase * RB;
+            const u32 dst = smem_u32(smem);
+            for (int i = 0; i < groups; ++i) {
+                const u32 bytes = (u32)min(DEC_ROWS, rows - DEC_ROWS * i) * (u32)RB;
+                const u32 bar = smem_u32(&s_bar[i]);
+                mbar_arrive_expect_tx(bar, bytes);
+                const u32 off0 = (u32)(DEC_ROWS * i) * (u32)RB;
+                for (u32 off = 0; off < bytes; off += 32768u)
+                    bulk_g2s_hint(dst + off0 + off, src + off0 + off, bytes - off < 32768u ? bytes - off : 32768u,
+                                  bar, policy);
+            }
+        }
     }
-    if (threadIdx.x < DEC_MAX_PSLOTS * 16) {
+    if (threadIdx.x == 0) {
+        DecSlot &d = s_sl[0];
+        d.x = pr.x;
+        d.s = pr.s;
+        d.gain = pr.gain;
+        d.xq_out = pr.xq_out;
+        d.K = K;
+        d.first = rbase == 0;
+        s_xoff[0] = 0;
+        s_xoff[1] = M * dec_row_stride(K);
+        s_vbase[0] = 0;
+        s_vbase[1] = M * (K / (SRC == DEC_SRC_F32 ? 4 : 8));
+    }
+    if (threadIdx.x == 32) s_gam[0] = *pr.gamma;
+    if (threadIdx.x < 16) {
         s_amax[threadIdx.x] = 0u;
         s_rs[threadIdx.x] = 0;
     }
+    if (G > 1)
+        for (int i = threadIdx.x; i < T * DEC_ROWS * M; i += DEC_THREADS) s_acc[i] = 0;
     __syncthreads();
-
-    // ---- this warp's request stream: its groups' chunks, in order ---------
-    // (warp-uniform state; lane 0 issues the copies)
-    uint8_t *ring = sm + warp * (DEC_WSTAGES * DEC_CHUNK);
-    const u64 policy = l2_policy_evict_first();
-    int i_g = -1, i_p = p_lo, i_k = 0, i_nch = 0;  // request cursor: group, problem, chunk, chunks of group
-    int q_tail = 0;                                // groups queued for the consumer side
-    long long issued = 0;
-    auto next_group = [&]() -> int {
-        int g;
-        if (i_g < 0) {
-            g = g_begin + warp;
-        } else {
-            g = 0;
-            if (lane == 0) g = atomicAdd(&s_next, 1);
-            g = __shfl_sync(0xffffffffu, g, 0);
-        }
-        return g < g_end ? g : -2;
-    };
-    auto issue_next = [&]() {
-        if (i_g == -2) return;
-        if (i_g < 0 || i_k == i_nch) {
-            const int g = next_group();
-            if (g < 0) {
-                i_g = -2;
-                return;
-            }
-            while (i_p + 1 < P.count && g >= P.p[i_p + 1].gbase) ++i_p;
-            i_g = g;
-            i_k = 0;
-            i_nch = dec_nchunks(P.p[i_p].K);
-            s_queue[warp][q_tail % QN] = g;  // every lane writes (and later reads) its own copy
-            ++q_tail;
-        }
-        const int s = (int)(issued % DEC_WSTAGES);
-        if (lane == 0) {
-            const u32 bar = smem_u32(&s_full[warp][s]);
-            mbar_arrive_expect_tx(bar, DEC_CHUNK);
-            tma_load_2d_hint(smem_u32(ring + s * DEC_CHUNK), &P.wmap[i_p], i_k * DEC_CB,
-                             (i_g - P.p[i_p].gbase) * DEC_ROWS, bar, policy);
-        }
-        ++i_k;
-        ++issued;
-    };
-    if (lane == 0)
-        for (int p = p_lo; p <= p_hi; ++p) asm volatile("prefetch.tensormap [%0];" ::"l"(&P.wmap[p]) : "memory");
-    for (int i = 0; i < DEC_WSTAGES; ++i) issue_next();
 
     // x_q and s may be produced by the kernel launched just before this one.
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // ---- activations of this CTA's problems, staged (and quantized) --------
-    bool block_quant = false;
+    // ---- activations, staged (and quantized) -------------------------------
+    const int RS = dec_row_stride(K);
     if (SRC != DEC_SRC_XQ) {
-        bool gain = false;
-        for (int i = 0; i < np; ++i) gain |= P.p[p_lo + i].gain != nullptr;
-        block_quant = !gain && s_vbase[np] <= DEC_QBV * DEC_THREADS;
-    }
-    if (block_quant) {
-        dec_quant_block<SRC == DEC_SRC_BF16>(P, p_lo, np, g_begin, s_xoff, s_vbase, s_x, s_amax, s_sc, s_f, s_rs);
-        // zero the padding chunks K .. round_up(K, 256) of every row
-        for (int r = warp; r < np * M; r += DEC_WARPS) {
-            const int ps = r / M, m = r - ps * M;
-            const int K = P.p[p_lo + ps].K, RS = dec_row_stride(K);
-            uint8_t *xs = s_x + s_xoff[ps];
-            for (int L = (K >> 4) + lane; L < (RS >> 4); L += 32) {
-                const int x = (((L >> 3) & 1) << 1) | (m & 1);
-                *reinterpret_cast<uint4 *>(xs + m * RS + (((L & ~7) | ((L ^ x) & 7)) << 4)) = make_uint4(0, 0, 0, 0);
-            }
-        }
-    }
-    for (int r = warp; r < (block_quant ? 0 : np * M); r += DEC_WARPS) {
-        const int ps = r / M, m = r - ps * M;
-        const DecodeProblem &pr = P.p[p_lo + ps];
-        const int K = pr.K, RS = dec_row_stride(K);
-        uint8_t *xs = s_x + s_xoff[ps];
-        if (SRC != DEC_SRC_XQ) {
-            constexpr bool BF16 = SRC == DEC_SRC_BF16;
-            const bool out = g_begin <= pr.gbase;  // this CTA holds the problem's first group
-            const float s = dec_quant_row<BF16>(pr, m, K, RS, xs, P.eps, out, lane, &s_rs[ps * M + m]);
-            if (lane == 0) s_f[ps][m] = __fdiv_rn(*pr.gamma, s);
-            for (int L = (K >> 4) + lane; L < (RS >> 4); L += 32) {
-                const int x = (((L >> 3) & 1) << 1) | (m & 1);
-                *reinterpret_cast<uint4 *>(xs + m * RS + (((L & ~7) | ((L ^ x) & 7)) << 4)) = make_uint4(0, 0, 0, 0);
-            }
+        constexpr bool BF16 = SRC == DEC_SRC_BF16;
+        if (pr.gain == nullptr) {
+            if (K <= DEC_RJ * 32 * (BF16 ? 8 : 4))
+                dec_quant_rows<BF16>(s_sl, 1, M, s_x, s_xoff, s_gam, s_f, s_rs, warp, lane);
+            else
+                dec_quant_block<BF16>(s_sl, 1, M, s_xoff, s_vbase, s_x, s_amax, s_sc, s_gam, s_f, s_rs);
         } else {
-            const int8_t *src = static_cast<const int8_t *>(pr.x) + (size_t)m * K;
-            for (int L = lane; L < (RS >> 4); L += 32) {
-                const int x = (((L >> 3) & 1) << 1) | (m & 1);
-                uint8_t *d = xs + m * RS + (((L & ~7) | ((L ^ x) & 7)) << 4);
-                if (L < (K >> 4))
-                    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(d)), "l"(src + L * 16)
-                                 : "memory");
-                else
-                    *reinterpret_cast<uint4 *>(d) = make_uint4(0, 0, 0, 0);
+            for (int m = warp; m < M; m += DEC_WARPS) {
+                const float s = dec_quant_row<BF16>(s_sl[0], m, K, RS, s_x, P.eps, s_sl[0].first, lane, &s_rs[m]);
+                if (lane == 0) s_f[0][m] = __fdiv_rn(s_gam[0], s);
             }
-            if (lane == 0) s_f[ps][m] = __fdiv_rn(*pr.gamma, pr.s[m]);
         }
-    }
-    if (SRC == DEC_SRC_XQ) {
-        asm volatile("cp.async.commit_group;" ::: "memory");
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        __syncthreads();
-        // row sums of the staged x_q (the padding is zero; the order of the
-        // 16-byte chunks does not matter)
-        for (int r = warp; r < np * M; r += DEC_WARPS) {
-            const int ps = r / M, m = r - ps * M;
-            const int RS = dec_row_stride(P.p[p_lo + ps].K);
-            const uint4 *row = reinterpret_cast<const uint4 *>(s_x + s_xoff[ps] + m * RS);
+        // zero the padding chunks K .. round_up(K, 256) of every row
+        for (int m = warp; m < M; m += DEC_WARPS)
+            for (int L = (K >> 4) + lane; L < (RS >> 4); L += 32) {
+                const int x = (((L >> 3) & 1) << 1) | (m & 1);
+                *reinterpret_cast<uint4 *>(s_x + m * RS + (((L & ~7) | ((L ^ x) & 7)) << 4)) = make_uint4(0, 0, 0, 0);
+            }
+    } else {
+        // plain loads, a warp per row
+        for (int m = warp; m < M; m += DEC_WARPS) {
+            const int8_t *src = static_cast<const int8_t *>(pr.x) + (size_t)m * K;
             int sum = 0;
             for (int L = lane; L < (RS >> 4); L += 32) {
-                const uint4 v = row[L];
+                const int x = (((L >> 3) & 1) << 1) | (m & 1);
+                const uint4 v = L < (K >> 4) ? ldg_nc_v4(src + L * 16) : make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(s_x + m * RS + (((L & ~7) | ((L ^ x) & 7)) << 4)) = v;
                 sum = __dp4a((int)v.x, 0x01010101, sum);
                 sum = __dp4a((int)v.y, 0x01010101, sum);
                 sum = __dp4a((int)v.z, 0x01010101, sum);
                 sum = __dp4a((int)v.w, 0x01010101, sum);
             }
             sum = __reduce_add_sync(0xffffffffu, sum);
-            if (lane == 0) s_rs[r] = sum;
+            if (lane == 0) {
+                s_rs[m] = sum;
+                s_f[0][m] = __fdiv_rn(s_gam[0], pr.s[m]);
+            }
         }
     }
     __syncthreads();
 
-    // ------------------------------------------------------------- consumers
+    // ------------------------------------------------------------- the GEMV
     const int g8 = lane >> 2, t = lane & 3;
-    const int pg = (g8 >> 1) | ((g8 & 1) << 2);       // physical row phase of MMA row g8
-    const int xb = ((t >> 1) << 1) | (g8 & 1);        // x_q swizzle of this lane's token rows
-    // M <= 8: one accumulator per code plane and tile (plane j at scale 4^j);
-    // M <= 16: the planes moved to scale 64, one accumulator per tile
-    constexpr int PL = NT == 1 ? 4 : 1;
-    long long consumed = 0;
-    int q_head = 0, c_p = p_lo;
+    const int xb = ((t >> 1) << 1) | (g8 & 1);  // x_q swizzle of this lane's token rows
+    const int wg = warp >> glog, kslot = warp & (G - 1);
     bool ok = true;
-    while (ok && q_head < q_tail) {
-        const int g = s_queue[warp][q_head % QN];
-        ++q_head;
-        while (c_p + 1 < P.count && g >= P.p[c_p + 1].gbase) ++c_p;
-        const DecodeProblem &pr = P.p[c_p];
-        const int ps = c_p - p_lo;
-        const int K = pr.K, RS = dec_row_stride(K);
-        const uint8_t *xs = s_x + s_xoff[ps];
-        const int nch = dec_nchunks(K);
-        int acc[PL][2][NT][4];
+    int acc[2][NT][4];
 #pragma unroll
-        for (int c = 0; c < PL; ++c)
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-            for (int u = 0; u < 2; ++u)
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc[u][nt][i] = 0;
+    const int steps = dec_nsteps(K);
+    const int SC = kch > 1 ? DEC_KCH_B / 64 : steps;  // steps per chunk
+    // rows g8 + 8a of the group; a step's slice of a row past its end reads
+    // the next row's bytes (or the padding): their k are past K, where x_q is
+    // zero
+    const uint8_t *w0 = smem + (wg * DEC_ROWS + g8) * WS + t * 16;
+    const uint8_t *xr[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) xr[nt] = s_x + min(g8 + 8 * nt, M - 1) * RS + t * 64;
+    int last_c = 0;  // last chunk requested
+    for (int c = 0; c < kch; ++c) {
+        if (wg < groups) {
+            ok = ok && __all_sync(0xffffffffu, mbar_wait(smem_u32(&s_bar[wg]), (u32)(c & 1), DEC_TIMEOUT_NS, nullptr));
+            if (!ok && lane == 0) raise_device_error(DEVERR_TIMEOUT_PRODUCER);
+        }
+        if (ok && wg < groups) {
+            const int st_end = min(steps, (c + 1) * SC);
+#pragma unroll 1
+            for (int st = c * SC + kslot; st < st_end; st += G) {
+                const int so = (st - c * SC) * 64;
+                uint4 wv[4];
+#pragma unroll
+                for (int a = 0; a < 4; ++a) wv[a] = *reinterpret_cast<const uint4 *>(w0 + a * 8 * WS + so);
+                uint4 xv[NT][4];
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) acc[c][u][nt][i] = 0;
-        for (int kc = 0; kc < nch; ++kc, ++consumed) {
-            const int s = (int)(consumed % DEC_WSTAGES);
-            ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&s_full[warp][s]), (u32)((consumed / DEC_WSTAGES) & 1),
-                                                  DEC_TIMEOUT_NS, &s_abort));
-            if (!ok) {
-                if (lane == 0) {
-                    raise_device_error(DEVERR_TIMEOUT_MMA);
-                    s_abort = 1;
-                }
-                break;
-            }
-            const int vb = min(DEC_CB, (K >> 2) - kc * DEC_CB);  // valid packed bytes per row (>= 16)
-            const uint8_t *st = ring + s * DEC_CHUNK;
-#pragma unroll 1
-            for (int h2 = 0; h2 < 2; ++h2) {
-                if (64 * h2 >= vb) break;
-                // weights: physical rows pg + 8a (a = 0..3), this lane's 16 bytes of the half
-                uint4 wv[4];
+                    for (int q = 0; q < 4; ++q)
+                        xv[nt][q] = *reinterpret_cast<const uint4 *>(xr[nt] + st * 256 + ((q ^ xb) << 4));
 #pragma unroll
-                for (int a = 0; a < 4; ++a)
-                    wv[a] = *reinterpret_cast<const uint4 *>(st + (pg + 8 * a) * DEC_CB + (((4 * h2 + t) ^ pg) << 4));
-                // x_q of tokens g8 (+ 8): the 64 bytes of k-slot t in 256-k step s2
-                const int s2 = 2 * kc + h2;
-                uint4 xv[NT][4];
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    const int m = g8 + 8 * nt;
-                    const uint8_t *xr = xs + m * RS + s2 * 256 + t * 64;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c)
-                        xv[nt][c] = m < M ? *reinterpret_cast<const uint4 *>(xr + ((c ^ xb) << 4))
-                                          : make_uint4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
+                for (int u = 0; u < 2; ++u)
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const u32 wa0 = (&wv[2 * u].x)[2 * hh], wa2 = (&wv[2 * u].x)[2 * hh + 1];
                         const u32 wa1 = (&wv[2 * u + 1].x)[2 * hh], wa3 = (&wv[2 * u + 1].x)[2 * hh + 1];
 #pragma unroll
                         for (int jp = 0; jp < 4; ++jp) {
-                            u32 a0, a1, a2, a3;
-                            if (PL == 4) {
-                                a0 = dec_plane(wa0, jp);
-                                a1 = dec_plane(wa1, jp);
-                                a2 = dec_plane(wa2, jp);
-                                a3 = dec_plane(wa3, jp);
-                            } else {
-                                a0 = dec_plane_top(wa0, jp);
-                                a1 = dec_plane_top(wa1, jp);
-                                a2 = dec_plane_top(wa2, jp);
-                                a3 = dec_plane_top(wa3, jp);
-                            }
+                            const u32 a0 = dec_plane_top(wa0, jp), a1 = dec_plane_top(wa1, jp);
+                            const u32 a2 = dec_plane_top(wa2, jp), a3 = dec_plane_top(wa3, jp);
 #pragma unroll
                             for (int nt = 0; nt < NT; ++nt)
-                                mma_u8s8_16832(acc[jp % PL][u][nt], a0, a1, a2, a3, (&xv[nt][2 * hh].x)[jp],
+                                mma_u8s8_16832(acc[u][nt], a0, a1, a2, a3, (&xv[nt][2 * hh].x)[jp],
                                                (&xv[nt][2 * hh + 1].x)[jp]);
                         }
                     }
-                }
             }
-            // the stage is free again: request this warp's next chunk into it
-            __syncwarp();
-            issue_next();
         }
-        if (!ok) break;
-        // epilogue: rows pg + 16u + 8(i >> 1), tokens 8nt + 2t + (i & 1)
-        const int n_base = (g - pr.gbase) * DEC_ROWS + pg;
+        if (c + 1 < kch) {
+            // every warp is done with this chunk before the next one lands
+            __syncthreads();
+            if (warp == DEC_WARPS - 1 && ok) {
+                request_chunk(c + 1);
+                last_c = c + 1;
+            }
+        }
+    }
+    if (ok && wg < groups) {
+        // this warp's sums of 64 c x into the CTA's [row][token] table (the
+        // only writer when G == 1)
 #pragma unroll
         for (int u = 0; u < 2; ++u)
 #pragma unroll
@@ -698,24 +756,36 @@ __global__ void __launch_bounds__(DEC_THREADS, 2) k_decode(const __grid_constant
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int m = 8 * nt + 2 * t + (i & 1);
-                    const int n = n_base + 16 * u + 8 * (i >> 1);
-                    if (m < M && n < pr.N) {
-                        // sum_k c x with c = 1 - W_q, each plane's sum a multiple of its scale
-                        const int cx = PL == 4 ? acc[0][u][nt][i] + (acc[PL > 1 ? 1 : 0][u][nt][i] >> 2) +
-                                                     (acc[PL > 2 ? 2 : 0][u][nt][i] >> 4) +
-                                                     (acc[PL > 3 ? 3 : 0][u][nt][i] >> 6)
-                                               : acc[0][u][nt][i] >> 6;
-                        const int a_ = s_rs[ps * M + m] - cx;
-                        pr.Y[(size_t)m * pr.N + n] = __fmul_rn(__int2float_rn(a_), s_f[ps][m]);
-                        if (pr.acc) pr.acc[(size_t)m * pr.N + n] = a_;
+                    const int r = wg * DEC_ROWS + g8 + 16 * u + 8 * (i >> 1);
+                    if (m < M) {
+                        if (G == 1)
+                            s_acc[r * M + m] = acc[u][nt][i];
+                        else
+                            atomicAdd(&s_acc[r * M + m], acc[u][nt][i]);
                     }
                 }
     }
-    if (!ok) {
-        // drain: this warp's copies in flight land before it exits
-        for (long long j = consumed; j < issued; ++j)
-            mbar_wait(smem_u32(&s_full[warp][(int)(j % DEC_WSTAGES)]), (u32)((j / DEC_WSTAGES) & 1), DEC_TIMEOUT_NS,
-                      nullptr);
+    __syncthreads();
+    // Y[m, rbase + r] = (sum_k x - (sum_k 64 c x) / 64) * (gamma / s[m]); 32
+    // consecutive rows per warp and token
+    float *Y = pr.Y;
+    int32_t *accp = pr.acc;
+    const int TR = T * DEC_ROWS;
+    for (int e = threadIdx.x; e < M * TR; e += DEC_THREADS) {
+        const int m = e / TR, r = e - m * TR;
+        if (r < rows) {
+            const int a_ = s_rs[m] - (s_acc[r * M + m] >> 6);
+            Y[(size_t)m * N + rbase + r] = __fmul_rn(__int2float_rn(a_), s_f[0][m]);
+            if (accp) accp[(size_t)m * N + rbase + r] = a_;
+        }
+    }
+    // a wait that gave up: the copies still in flight land (bounded) before
+    // the CTA exits
+    if (__syncthreads_or(!ok) && threadIdx.x == DEC_THREADS - 32) {
+        if (kch > 1)
+            mbar_wait(smem_u32(&s_bar[0]), (u32)(last_c & 1), DEC_TIMEOUT_NS, nullptr);
+        else
+            for (int i = 0; i < groups; ++i) mbar_wait(smem_u32(&s_bar[i]), 0, DEC_TIMEOUT_NS, nullptr);
     }
 }
 
