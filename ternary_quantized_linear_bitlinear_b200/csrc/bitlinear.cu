@@ -25,13 +25,17 @@ namespace {
 constexpr int BL_VERSION = 100;
 constexpr int64_t K_MAX = 32768;
 constexpr int MAX_DEVICES = 64;
-// dynamic shared memory of the largest decode launch: weights of a CTA
-// (whole rows up to DEC_W_CAP bytes, or one row group up to 32 x 1536 bytes,
-// or a 32 x DEC_KCH_B chunk) plus padding, x_q, the sums, alignment slack
+// dynamic shared memory a decode launch may use: the CTA's weights (whole
+// groups, or a 32 x DEC_KCH_B chunk) plus padding, x_q and the sums; a
+// problem whose whole group does not fit beside its x_q is chunked, and
+// problems whose combined layout would not fit go to separate launches
 constexpr size_t DEC_SMEM_ATTR = (size_t)DEC_ROWS * DEC_KCH_B + DEC_W_PAD + DEC_X_MAX + DEC_WARPS * DEC_ROWS * 16 * 4 + 512;
 // ... within the 227 KiB opt-in limit with the kernel's static shared memory (under 1 KiB)
 static_assert(DEC_SMEM_ATTR + 1024 <= 227 * 1024, "decode engine shared memory");
-static_assert(DEC_ROWS * (DEC_K_WHOLE / 4) <= DEC_ROWS * DEC_KCH_B, "decode weight staging");
+// dynamic shared memory of a CTA that still fits three to an SM (228 KiB,
+// 1 KiB reserved per CTA, static shared memory under 1 KiB)
+constexpr size_t DEC_SMEM_3 = 228 * 1024 / 3 - 2 * 1024;
+
 static_assert(sizeof(DecodeParams) <= 32764, "decode parameters exceed the kernel parameter limit");
 
 struct DeviceInfo {
@@ -310,10 +314,11 @@ struct DecodeJob {
 bl_status decode_launch(const DecodeJob *jobs, int count, int M, float eps, bool pdl, cudaStream_t st, int src,
                         int sms) {
     thread_local DecodeParams P;
-    int glog[BL_MAX_GROUP];
+    int glog[BL_MAX_GROUP], kchs[BL_MAX_GROUP];
     int64_t total = 0;
     for (int i = 0; i < count; ++i) {
-        glog[i] = dec_glog_p((int)jobs[i].K);
+        kchs[i] = dec_kch((int)jobs[i].K, M, DEC_SMEM_ATTR);
+        glog[i] = kchs[i] > 1 ? 3 : dec_glog((int)jobs[i].K);
         const int64_t ng = (jobs[i].N + DEC_ROWS - 1) / DEC_ROWS;
         total += (ng + (DEC_WARPS >> glog[i]) - 1) / (DEC_WARPS >> glog[i]);
     }
@@ -361,10 +366,22 @@ bl_status decode_launch(const DecodeJob *jobs, int count, int M, float eps, bool
         const DecodeJob &j = jobs[i];
         const int N = (int)j.N, K = (int)j.K;
         const int T = DEC_WARPS >> glog[i];
-        const int kch = dec_kch(K);
+        const int kch = kchs[i];
         const int wb = kch > 1 ? DEC_ROWS * DEC_KCH_B : T * DEC_ROWS * (K >> 2);
         for (int row = 0; row < N;) {
-            if (P.count == BL_MAX_GROUP || nc == DEC_MAX_CTAS) {
+            // the launch's layout with this problem in it must fit
+            const int w2 = wb > w_max ? wb : w_max;
+            const int r2 = dec_row_stride(K) > rs_max ? dec_row_stride(K) : rs_max;
+            const int t2 = T > t_max ? T : t_max;
+            const size_t need_smem = (size_t)((w2 + DEC_W_PAD + 127) & ~127) + (size_t)((M * r2 + 127) & ~127) +
+                                     (size_t)t2 * DEC_ROWS * M * 4;
+            // (and a launch whose CTAs fit three to an SM is not given a
+            // problem that would take that away from all of them)
+            const size_t cur_smem = (size_t)((w_max + DEC_W_PAD + 127) & ~127) +
+                                    (size_t)((M * rs_max + 127) & ~127) + (size_t)t_max * DEC_ROWS * M * 4;
+            const bool lose3 = cur_smem <= DEC_SMEM_3 && need_smem > DEC_SMEM_3;
+            if (P.count == BL_MAX_GROUP || nc == DEC_MAX_CTAS ||
+                (P.count > 0 && (need_smem > DEC_SMEM_ATTR || lose3))) {
                 bl_status rc = flush();
                 if (rc) return rc;
             }

@@ -50,7 +50,7 @@ constexpr int DEC_WARPS = 8;
 constexpr int DEC_THREADS = 32 * DEC_WARPS;
 constexpr int DEC_ROWS = 32;                // weight rows per group (two MMA tiles)
 constexpr int DEC_PF = 4;                   // target 256-k steps per warp (G is chosen from it)
-constexpr int DEC_W_CAP = 48 * 1024;        // packed bytes per CTA above which G grows (three CTAs per SM)
+constexpr int DEC_W_CAP = 56 * 1024;        // packed bytes per CTA above which G grows (three CTAs per SM)
 constexpr int DEC_MAX_CTAS = 2048;          // CTAs per launch (larger calls are split into launches)
 constexpr int DEC_X_MAX = 144 * 1024;       // staged activations per CTA
 constexpr int DEC_MAX_PSLOTS = 1;           // problems per CTA (the staging helpers take a slot array)
@@ -73,7 +73,7 @@ struct DecodeProblem {
     int rows;              // rows of that part
     int glog;              // log2(G): warps per group
     int cta_begin;         // first CTA of this problem in the launch
-    int kch;               // K chunks: 1, or (K > DEC_K_WHOLE) one group per CTA in chunks of DEC_KCH_B bytes a row
+    int kch;               // K chunks: 1, or one group per CTA in chunks of DEC_KCH_B bytes a row
 };
 
 struct DecodeParams {
@@ -525,18 +525,20 @@ __device__ void dec_quant_rows(const DecSlot *sl, int np, int M, uint8_t *s_x, c
 
 __device__ __forceinline__ int dec_nsteps(int K) { return (K + 255) >> 8; }
 
-// Shared memory of a launch: the CTA's packed weights (at most
-// dec_w_bytes(K) + DEC_W_PAD), then at x_off the staged x_q (M rows of
-// round_up(K, 256) bytes), then at acc_off the sums (T groups x 32 rows x M).
-// Rows longer than DEC_K_WHOLE / 4 bytes are staged in chunks of DEC_KCH_B
-// bytes (one group per CTA; a bulk copy per row and chunk).
+// Shared memory of a launch: the CTA's packed weights plus DEC_W_PAD, then
+// at x_off the staged x_q (M rows of round_up(K, 256) bytes), then at
+// acc_off the sums (T groups x 32 rows x M).  A group of whole rows is
+// staged when it is at most DEC_W_WHOLE bytes and fits beside x_q in the
+// budget; longer rows are staged in chunks of DEC_KCH_B bytes (one group per
+// CTA; a bulk copy per row and chunk).
 constexpr int DEC_W_PAD = 256;  // reads of a row's last step may run past the copied bytes
-constexpr int DEC_K_WHOLE = 6144;
+constexpr int DEC_W_WHOLE = 48 * 1024;
 constexpr int DEC_KCH_B = 2048;
-__host__ __device__ inline int dec_kch(int K) { return K <= DEC_K_WHOLE ? 1 : ((K >> 2) + DEC_KCH_B - 1) / DEC_KCH_B; }
-__host__ __device__ inline int dec_glog_p(int K) { return dec_kch(K) > 1 ? 3 : dec_glog(K); }
-__host__ __device__ inline int dec_w_bytes(int K) {
-    return dec_kch(K) > 1 ? DEC_ROWS * DEC_KCH_B : (DEC_WARPS >> dec_glog(K)) * DEC_ROWS * (K >> 2);
+inline int dec_kch(int K, int M, size_t budget) {
+    const size_t whole = (size_t)DEC_ROWS * (K >> 2);
+    if (whole <= DEC_W_WHOLE && whole + DEC_W_PAD + (size_t)M * dec_row_stride(K) + DEC_ROWS * M * 4 + 256 <= budget)
+        return 1;
+    return ((K >> 2) + DEC_KCH_B - 1) / DEC_KCH_B;
 }
 
 // NT: 8-token column tiles (1: M <= 8, 2: M <= 16).  SRC: DEC_SRC_*.

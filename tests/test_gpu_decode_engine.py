@@ -1,12 +1,14 @@
-"""The decode engine's work partition, against the CPU oracle element by
-element: the host cuts the groups of 32 weight rows of all problems into
-one byte-balanced range per CTA and splits ranges at problem boundaries for
-the activation staging; inside a CTA the chunks of 32 rows x 512 k stream
-through a ring and the warps' partial sums meet in per-group accumulator
-slots.  These cases drive the corners of that: many tiny problems in one
-range, one group of many chunks, chunks with only part of their 512 k in
-range, slot reuse over hundreds of one-chunk groups, and launches repeated
-on the same buffers (the slots must come back clean).
+"""The decode engine's work split, against the CPU oracle element by
+element: a CTA stages T = 8 / G whole 32-row groups of one problem (G warps
+per group split its k steps; partial sums meet in a shared-memory table),
+groups too long for shared memory are staged in 2 KiB chunks of their rows,
+launches too small to fill the GPU take one group per CTA, and a call is
+split into several launches when it holds more CTAs than one launch maps,
+when its problems' shared-memory layouts do not fit together, or when a
+problem would take the third CTA slot per SM from the others.  These cases
+drive the corners of that: many tiny problems, one group of many chunks,
+steps with only part of their 256 k in range, whole groups up to 96 KiB,
+the splits, and launches repeated on the same buffers.
 """
 from __future__ import annotations
 
@@ -44,29 +46,30 @@ def _xq_path(shapes, M, seed, repeat=1):
 
 def test_many_tiny_problems_share_a_range():
     """120 small problems (one group each, ragged N, K from 64 to 512) ahead
-    of one large one: the first byte-balanced range holds all of them and is
-    split at problem boundaries (at most eight problems' activations per
-    CTA)."""
+    of one large one: 121 problems in one launch, most of them one CTA of a
+    single partial group."""
     shapes = [(1 + (7 * i) % 64, 64 * (1 + i % 8)) for i in range(120)] + [(8192, 4096)]
     _xq_path(shapes, 4, 1000)
 
 
 def test_one_group_of_many_chunks():
-    """K = 32768 at M = 1: 64 chunks per group, N ragged (three groups, the
-    last with 4 rows)."""
+    """K = 32768 at M = 1: a group of whole rows (256 KiB) exceeds shared
+    memory, so each CTA stages its group in 4 chunks of 2 KiB per row; N
+    ragged (three groups, the last with 4 rows)."""
     _xq_path([(68, 32768)], 1, 1100)
 
 
 def test_partial_chunks_and_slot_reuse():
-    """K = 256 and K = 832: chunks with 64 or 80 of their 128 bytes in range;
-    N = 8192 gives hundreds of one-chunk groups per launch, each CTA reusing
-    every accumulator slot many times; run twice on the same buffers."""
+    """K = 256 and K = 832: one-step rows, and a last step with 64 of its
+    256 k in range (the lanes past the row read the next row's bytes against
+    zero x_q); N = 8192 gives 32 CTAs of eight groups; run twice on the same
+    buffers (the sums table must come back clean)."""
     _xq_path([(8192, 256), (333, 832)], 3, 1200, repeat=2)
 
 
 def test_m16_wide_activations_one_problem_per_cta():
-    """M = 16, K = 2048 (32 KiB of staged activations per problem): ranges
-    hold one problem each; fused act quant with SubLN."""
+    """M = 16, K = 2048 (32 KiB of staged activations per CTA), two token
+    tiles; fused act quant with SubLN."""
     M = 16
     dev, refs = [], []
     for i in range(5):
@@ -88,3 +91,18 @@ def test_m16_wide_activations_one_problem_per_cta():
         wq_ref, g_ref = check_weights(W, d[0], d[1])
         xq_ref, s_ref = check_act(X, d[5], d[6], gain)
         check_forward_full(xq_ref, s_ref, wq_ref, g_ref, d[4], d[7])
+
+
+def test_whole_and_chunked_groups_and_a_layout_split():
+    """K = 6144 at M = 4: whole groups of 48 KiB; K = 8640 and 12288 chunked
+    (2160- and 3072-byte rows); K = 32768 (128 KiB of x_q at M = 4) with the
+    others' layouts does not fit one launch, so the call is split into
+    launches."""
+    _xq_path([(70, 8640), (65, 12288), (40, 32768), (33, 768), (50, 6144)], 4, 1400)
+
+
+def test_more_ctas_than_one_launch_maps():
+    """N = 600,000 rows of K = 64 at M = 2: 2344 CTAs of eight groups, more
+    than the 2048 one launch maps, so the problem is split by row ranges
+    over two launches."""
+    _xq_path([(600000, 64)], 2, 1500)
