@@ -57,6 +57,7 @@ MS = (1, 4, 8)
 SPAD = {M: (M + 3) // 4 * 4 for M in MS}
 WORKLOAD = "decode125m: 12 layers x {q,o 768x768; k,v 256x768; gate,up 2048x768; down 768x2048}, M in {1,4,8}"
 CONFIGS = ("single", "decode125m", "prefill1b4", "layer3b", "qat4b")
+PER_CALL = ("per_call", "per_call_grouped", "per_call_layer")  # per-call paths of the prefill workloads
 
 
 def replica_of(step: int, j: int, replicas: int) -> int:
@@ -835,6 +836,30 @@ class PrefillLayer:
                                         None if r0["gain"] is None else r0["gain"].data_ptr(), workloads.SUBLN_EPS,
                                         self._lg_ws.data_ptr(), self._lg_ws.numel(), sp), "bl_linear_grouped")
 
+    def per_call_layer(self, sp):
+        """The per-call path with the layer's weights quantized together: one
+        bl_quant_weights_grouped over all projections (at most eight), then
+        per group of projections sharing an input one act quant and one
+        grouped GEMM."""
+        api = self.api
+        if not hasattr(self, "_pl"):
+            n = len(self.rows)
+            warr = (api.WeightProblem * n)()
+            for i, r in enumerate(self.rows):
+                warr[i] = api.WeightProblem(r["W"].data_ptr(), r["N"], r["K"], r["packed"].data_ptr(),
+                                            r["gamma"].data_ptr())
+            wsz = int(self.L.bl_quant_weights_workspace_bytes(self.rows[0]["N"], self.rows[0]["K"]))
+            self._pl = (warr, n, torch.empty(wsz, dtype=torch.uint8, device=self.dev))
+        warr, n, wws = self._pl
+        ok(self.L.bl_quant_weights_grouped(warr, n, self.rows[0]["wdt"], wws.data_ptr(), wws.numel(), sp),
+           "bl_quant_weights_grouped")
+        for g, (arr, ng) in zip(self.groups, self.garrs):
+            r0 = self.rows[g[0]]
+            ok(self.L.bl_quant_act(r0["X"].data_ptr(), r0["xdt"], self.M, r0["K"],
+                                   None if r0["gain"] is None else r0["gain"].data_ptr(), workloads.SUBLN_EPS,
+                                   r0["x_q"].data_ptr(), r0["s"].data_ptr(), sp), "bl_quant_act")
+            ok(self.L.bl_forward_grouped(arr, ng, self.M, 0, sp), "bl_forward_grouped")
+
     def per_call(self, sp, rows=None, Ws=None, Xs=None, Ys=None):
         for i, r in enumerate(self.rows):
             W = r["W"] if Ws is None else Ws[i]
@@ -906,7 +931,8 @@ def bench_prefill1b4(args, world, local, dev, pk):
     stream = torch.cuda.Stream(device=dev)
     with Clocks(local, "prefill1b4") as clk:
         res = time_layer_fns(layer, {"engine": layer.engine, "engine_grouped": layer.engine_grouped,
-                                     "per_call": layer.per_call, "per_call_grouped": layer.per_call_grouped},
+                                     "per_call": layer.per_call, "per_call_grouped": layer.per_call_grouped,
+                                     "per_call_layer": layer.per_call_layer},
                              stream, world, args)
         # FFN activation + SubLN + act quant feeding the down projection (bl_ffn_act_quant)
         M, F = layer.M, workloads.PREFILL1B4["ffn"]
@@ -956,12 +982,15 @@ def bench_prefill1b4(args, world, local, dev, pk):
                                   "down 1536x4096, M = 8192; W bf16 ~N(0, 0.02^2), X bf16 = 0.5 t(3)",
                       "ops_per_layer": layer.ops,
                       "l2": "inputs and outputs of the layer total > 700 MB"},
-           "value": max(res["per_call"]["tops"], res["per_call_grouped"]["tops"]),
+           "value": max(res[k]["tops"] for k in PER_CALL),
            "unit": "TOPS (per-call path: weights quantized in the call)",
            **res,
            "engine_grouped_launches": "q,k,v | o | gate,up | down (shared-input projections in one launch)",
            "roofline": roofline_tensor("k_prefill_tc", layer.ops, res[best]["ms_per_layer"], pk, best),
-           "per_call_frac": round(max(res["per_call"]["tops"], res["per_call_grouped"]["tops"]) / pk["int8"], 4),
+           "per_call_frac": round(max(res[k]["tops"] for k in PER_CALL) / pk["int8"], 4),
+           "per_call_paths": "per_call: bl_linear x7; per_call_grouped: bl_linear_grouped per group of "
+                             "projections sharing an input; per_call_layer: one bl_quant_weights_grouped over "
+                             "the layer's 7 matrices, then per group bl_quant_act + bl_forward_grouped",
            "ffn_act_quant": {"shape": f"gate, up [{M}, {F}] f32 -> x_q [{M}, {F}] (ReLU^2 gate, SubLN)",
                              "us": round(ffn_us, 2), "gbs": round(ffn_bytes / (ffn_us * 1e-6) / 1e9, 1),
                              "frac_hbm": round(ffn_bytes / (ffn_us * 1e-6) / 1e9 / pk["hbm"], 4)},
@@ -1138,18 +1167,17 @@ def bench_qat4b(args, world, local, dev, pk):
     stream = torch.cuda.Stream(device=dev)
     with Clocks(local, "qat4b") as clk:
         res = time_layer_fns(layer, {"per_call": layer.per_call, "per_call_grouped": layer.per_call_grouped,
+                                     "per_call_layer": layer.per_call_layer,
                                      "engine_grouped": layer.engine_grouped}, stream, world, args)
     api.bl_check_device_error(stream)
     out = {"config": {"workload": "qat4b: hidden 2560, FFN 9728, q,k,v,o 2560^2, gate,up 9728x2560, down 2560x9728, "
                                   "M = 16 x 2048 = 32768; bf16 master W ~N(0, 0.02^2) re-quantized every call; SubLN "
                                   "(gain ~U(0.9, 1.1), eps 1e-6) fused into the act quant before o_proj and "
                                   "down_proj", "ops_per_layer": layer.ops},
-           "value": max(res["per_call"]["tops"], res["per_call_grouped"]["tops"]), "unit": "TOPS (per-call path)",
+           "value": max(res[k]["tops"] for k in PER_CALL), "unit": "TOPS (per-call path)",
            **res,
-           "roofline": roofline_tensor("k_prefill_tc", layer.ops,
-                                       min(res["per_call"]["ms_per_layer"], res["per_call_grouped"]["ms_per_layer"]),
-                                       pk, "per_call" if res["per_call"]["tops"] >= res["per_call_grouped"]["tops"]
-                                       else "per_call_grouped"),
+           "roofline": roofline_tensor("k_prefill_tc", layer.ops, min(res[k]["ms_per_layer"] for k in PER_CALL), pk,
+                                       max(PER_CALL, key=lambda k: res[k]["tops"])),
            "engine_frac": round(res["engine_grouped"]["tops"] / pk["int8"], 4),
            "clocks": clk.summary()}
     if not args.no_e2e:

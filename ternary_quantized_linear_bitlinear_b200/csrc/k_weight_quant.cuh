@@ -106,21 +106,28 @@ __device__ void wq_finalize_block(const u64 *partials, int nblocks, long long n,
         }
     }
     __syncthreads();
+    // limb position k summed over the warps by lane k of warp 0 (128 bits:
+    // a thread adds at most two 64-bit limbs, a warp's sum is below 2^70,
+    // the sixteen warps' below 2^74)
+    __shared__ u64 f_sum[NL][2];
+    if (tid < NL) {
+        u64 lo = 0ull, hi = 0ull;
+        for (int w = 0; w < WQ_THREADS / 32; ++w) {
+            const u64 t = lo + f_lo[tid][w];
+            hi += f_hi[tid][w] + (t < lo ? 1ull : 0ull);
+            lo = t;
+        }
+        f_sum[tid][0] = lo;
+        f_sum[tid][1] = hi;
+    }
+    __syncwarp();
     if (tid == 0) {
-        // S = sum_k (hi:lo)_k << 64k over the warps, folded into NL + 2 limbs
+        // S = sum_k (hi:lo)_k << 64k, folded into NL + 2 limbs
         u64 L[NL + 2];
 #pragma unroll
         for (int k = 0; k < NL + 2; ++k) L[k] = 0ull;
 #pragma unroll
-        for (int k = 0; k < NL; ++k) {
-            u64 lo = 0ull, hi = 0ull;
-            for (int w = 0; w < WQ_THREADS / 32; ++w) {
-                const u64 t = lo + f_lo[k][w];
-                hi += f_hi[k][w] + (t < lo ? 1ull : 0ull);
-                lo = t;
-            }
-            limbs_add_u128_shl(L, lo, hi, 64 * k);
-        }
+        for (int k = 0; k < NL; ++k) limbs_add_u128_shl(L, f_sum[k][0], f_sum[k][1], 64 * k);
         double S = limbs_to_double_rn(L, -149);
         float mean = __double2float_rn(__ddiv_rn(S, (double)n));
         float g = __fadd_rn(mean, 1e-5f);
@@ -198,14 +205,18 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const __grid_con
     if (first < nvec) add_vec(v0);
     if (has1) add_vec(v1);
     long long i = first + 2 * stride;
-    // two vectors in flight per iteration
-    for (; i + stride < nvec; i += 2 * stride) {
-        uint4 a = ldg_stream_v4(W + i);
-        uint4 b = ldg_stream_v4(W + i + stride);
+    // four vectors in flight per iteration
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+        const uint4 a = ldg_stream_v4(W + i);
+        const uint4 b = ldg_stream_v4(W + i + stride);
+        const uint4 c = ldg_stream_v4(W + i + 2 * stride);
+        const uint4 d = ldg_stream_v4(W + i + 3 * stride);
         add_vec(a);
         add_vec(b);
+        add_vec(c);
+        add_vec(d);
     }
-    if (i < nvec) add_vec(ldg_stream_v4(W + i));
+    for (; i < nvec; i += stride) add_vec(ldg_stream_v4(W + i));
 
     // Block sum of the 64-bit window accumulators as 128 bits.
     u64 lo = acc, hi = 0ull;
