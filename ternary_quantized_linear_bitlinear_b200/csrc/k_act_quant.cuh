@@ -383,6 +383,7 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid
 constexpr int AQR_THREADS = 128;
 constexpr int AQR_WARPS = AQR_THREADS / 32;
 constexpr int AQR_MAX_K = 24 * 1024;  // rows cached per CTA: K * 4 bytes of dynamic shared memory
+constexpr int AQR_FAST_SPAN = 19;     // bf16 rows: exponent span of the 64-bit exact sum of squares
 
 __device__ __forceinline__ u32 aqr_block_max(u32 v, u32 *s_u) {
     v = warp_max_u32(v);
@@ -412,8 +413,9 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
     const uint4 *xr = reinterpret_cast<const uint4 *>(pr.X) + (size_t)m * nvec;
     const uint4 *ur = GLU ? reinterpret_cast<const uint4 *>(pr.X2) + (size_t)m * nvec : nullptr;
     const float4 *g4 = reinterpret_cast<const float4 *>(pr.gain);
-    // pass 1: load (once), cache as float, max|x|
-    u32 amax = 0;
+    // pass 1: load (once), cache as float, max|x| (bf16 rows also the
+    // smallest nonzero |x|'s exponent, 255 - e carried as a max)
+    u32 amax = 0, inv_emin = 0;
     for (int v0 = 0; v0 < nvec; v0 += AQR_THREADS * U) {
         uint4 c[U];
 #pragma unroll
@@ -437,6 +439,8 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
             for (int j = 0; j < EPV; ++j) {
                 const u32 b = aq_bits<BF16>(c[i], j);
                 amax = max(amax, b & 0x7fffffffu);
+                // (a subnormal counts as exponent 0: below any window)
+                if (BF16 && (b & 0x7fffffffu) != 0u) inv_emin = max(inv_emin, 255u - ((b >> 23) & 0xffu));
                 f[j] = __uint_as_float(b);
             }
 #pragma unroll
@@ -445,11 +449,38 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
         }
     }
     amax = aqr_block_max(amax, s_u);  // also orders the row cache writes before the reads below
+    if (BF16 && g4 != nullptr) inv_emin = aqr_block_max(inv_emin, s_u);
     if (g4 != nullptr) {
-        // pass 2: exact sum of squares, 31-binade windows (normally one)
+        // pass 2: exact sum of squares
         u64 L[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
         int ehi = (int)(amax >> 23);
         if (ehi < 1) ehi = 1;
+        const int emin = 255 - (int)inv_emin;
+        // bf16 rows whose nonzero |x| span at most AQR_FAST_SPAN binades (no
+        // subnormal): x^2 = m^2 * 2^(2e - 268) with the 8-bit mantissa m, so
+        // m^2 << 2(e - emin) < 2^(16 + 38) and at most 2^8 terms per thread
+        // stay below 2^62: one 64-bit accumulator per thread, no window pass
+        if (BF16 && emin >= 1 && ehi - emin <= AQR_FAST_SPAN && K <= AQR_THREADS * 256) {
+            u64 acc = 0ull;
+            for (int k = tid; k < K; k += AQR_THREADS) {
+                const u32 u = __float_as_uint(s_row[k]) & 0x7fffffffu;
+                const u32 m = ((u >> 16) & 0x7fu) | 0x80u;
+                const int sh = 2 * ((int)(u >> 23) - emin);  // 0 .. 2 AQR_FAST_SPAN for u != 0
+                const u64 t = (u64)(m * m) << (sh & 63);
+                acc += u != 0u ? t : 0ull;
+            }
+            u64 lo = acc, hi = 0ull;
+            warp_sum_u128(lo, hi);
+            if (lane == 0) {
+                s_lo[warp] = lo;
+                s_hi[warp] = hi;
+            }
+            __syncthreads();
+            // term = m^2 << 2(e - emin) stands for x^2 = term * 2^(2 emin - 268),
+            // i.e. term << (2 emin + 30) units of 2^-298
+            if (tid == 0)
+                for (int w = 0; w < AQR_WARPS; ++w) limbs_add_u128_shl(L, s_lo[w], s_hi[w], 2 * emin + 30);
+        } else
         for (int pass = 0; pass < 10; ++pass) {
             const int elo = ehi - 30 < 1 ? 1 : ehi - 30;
             u64 lo = 0ull, hi = 0ull;
@@ -502,8 +533,11 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
         // rounds to 0 either way, and such a y is the row maximum only when
         // every |y| of the row is below 1e-5, where s is floored at
         // 127 / 1e-5 whatever the maximum is.
-        // Measured 172 -> 136 us for [8192, 4096]; bf16 rows were 1-2 %
-        // slower with it, so they keep the IEEE division.
+        // Measured 172 -> 136 us for [8192, 4096].  A bf16 row without
+        // subnormal values (known from pass 1) takes Markstein for every
+        // element without the per-element test (717 -> 638 us for [32768,
+        // 9728]); other bf16 rows keep the IEEE division, which with the
+        // per-element test was as fast.
         const float ry = __frcp_rn(r);
         const bool mk = (GLU || !BF16) && __float_as_uint(r) >= 0x00800000u && __float_as_uint(r) < 0x7f800000u;
         auto div_r = [&](float x) {
@@ -513,6 +547,24 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
             return __fmaf_rn(__fmaf_rn(-q0, r, x), ry, q0);
         };
         amax = 0;
+        if (BF16 && emin >= 1 && __float_as_uint(r) >= 0x00800000u && __float_as_uint(r) < 0x7f800000u) {
+            // a bf16 row without subnormal values: Markstein for every element, no branch
+            for (int q = tid; q < K / 4; q += AQR_THREADS) {
+                const float4 g = __ldg(g4 + q);
+                float4 x = reinterpret_cast<float4 *>(s_row)[q];
+                float q0 = __fmul_rn(x.x, ry);
+                x.x = __fmul_rn(__fmaf_rn(__fmaf_rn(-q0, r, x.x), ry, q0), g.x);
+                q0 = __fmul_rn(x.y, ry);
+                x.y = __fmul_rn(__fmaf_rn(__fmaf_rn(-q0, r, x.y), ry, q0), g.y);
+                q0 = __fmul_rn(x.z, ry);
+                x.z = __fmul_rn(__fmaf_rn(__fmaf_rn(-q0, r, x.z), ry, q0), g.z);
+                q0 = __fmul_rn(x.w, ry);
+                x.w = __fmul_rn(__fmaf_rn(__fmaf_rn(-q0, r, x.w), ry, q0), g.w);
+                reinterpret_cast<float4 *>(s_row)[q] = x;
+                amax = max(amax, max(max(__float_as_uint(x.x) & 0x7fffffffu, __float_as_uint(x.y) & 0x7fffffffu),
+                                     max(__float_as_uint(x.z) & 0x7fffffffu, __float_as_uint(x.w) & 0x7fffffffu)));
+            }
+        } else
         for (int q = tid; q < K / 4; q += AQR_THREADS) {
             const float4 g = __ldg(g4 + q);
             float4 x = reinterpret_cast<float4 *>(s_row)[q];

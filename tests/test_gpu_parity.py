@@ -110,6 +110,12 @@ def _wide_rows(M, K, seed):
     (7, 9728, torch.bfloat16, True, "student"),
     (6, 4096, torch.float32, True, "wide"),
     (3, 2560, torch.bfloat16, True, "wide"),
+    # bf16 SubLN rows of the CTA-per-row kernel: its one-accumulator exact
+    # sum of squares (nonzero |x| within 19 binades, no subnormal) and the
+    # windowed one it falls back to
+    (4, 4096, torch.bfloat16, True, "tiny"),
+    (3, 24576, torch.bfloat16, True, "normal"),
+    (5, 2560, torch.bfloat16, True, "span"),
 ])
 def test_quant_act(M, K, dtype, subln, kind):
     if kind == "outlier":
@@ -120,6 +126,16 @@ def test_quant_act(M, K, dtype, subln, kind):
         X = workloads.student_t((M, K), 3, 0.5, 10, dtype)
     elif kind == "wide":
         X = _wide_rows(M, K, 11).to(dtype)
+    elif kind == "span":
+        # rows whose nonzero |x| span exactly 19 binades (the one-accumulator
+        # limit), 20 binades, one subnormal, and huge values (2^60)
+        X = workloads.normal((M, K), 1.0, 14).to(dtype).float()
+        X = X.sign() * (X.abs().clamp(2.0 ** -8, 2.0 ** 8 - 1))
+        X[0, 0], X[0, 1] = 2.0 ** 10, 2.0 ** -9          # exponents 10 .. -9: span 19
+        X[1, 0], X[1, 1] = 2.0 ** 10, -(2.0 ** -10)      # span 20
+        X[2, 5] = 2.0 ** -130                            # a subnormal (bf16 keeps it)
+        X[3] = X[3] * 2.0 ** 52                          # up to 2^60
+        X = X.to(dtype)
     else:  # rows below the 1e-5 floor, and an all-zero row
         X = (workloads.normal((M, K), 1.0, 12) * 1e-7).to(dtype)
         X[1] = 0
