@@ -76,6 +76,7 @@ _SIGS = {
     "bl_linear_workspace_bytes": (_sz, [_i64, _i64, _i64]),
     "bl_linear": (_int, [_p, _int, _p, _int, _i64, _i64, _i64, _p, _f32, _p, _sz, _p, _p]),
     "bl_forward_grouped": (_int, [ctypes.POINTER(Problem), _int, _i64, ctypes.c_uint, _p]),
+    "bl_debug_decode_plan": (_int, [_p, _int, _i64, _int, _p, _int, _p]),
     "bl_debug_forward_prefill": (_int, [_p, _p, _p, _p, _i64, _i64, _i64, _p, _p, ctypes.c_longlong,
                                         ctypes.c_uint32, _p]),
     "bl_quant_act_grouped": (_int, [ctypes.POINTER(ActProblem), _int, _int, _i64, _f32, _p]),
@@ -555,6 +556,31 @@ def bl_linear_grouped(Ws, X, subln_gain=None, subln_eps: float = 1e-6, Ys=None, 
                                  subln_eps, workspace.data_ptr(), workspace.numel(), _stream(stream))
     _check(rc, "bl_linear_grouped")
     return Ys
+
+
+def bl_debug_decode_plan(shapes, M: int, sms: int = 148):
+    """Host-side plan of a decode call over problems of the given (N, K)
+    shapes at M tokens on a GPU with `sms` SMs (nothing is launched; no GPU
+    needed): a list of launches, each {"ctas", "smem", "problems": [{"job",
+    "row0", "rows", "glog", "kch", "cta_begin"}]}."""
+    shapes = list(shapes)
+    arr = (ctypes.c_int64 * (2 * len(shapes)))(*[int(v) for nk in shapes for v in nk])
+    cap = 64 + 16 * 6 * max(1, len(shapes)) * 8
+    out = (ctypes.c_int * cap)()
+    written = ctypes.c_int(0)
+    rc = lib().bl_debug_decode_plan(arr, len(shapes), int(M), int(sms), out, cap, ctypes.byref(written))
+    _check(rc, "bl_debug_decode_plan")
+    vals, launches, i = list(out[:written.value]), [], 0
+    while i < len(vals):
+        ctas, smem, n = vals[i:i + 3]
+        i += 3
+        probs = []
+        for _ in range(n):
+            job, row0, rows, glog, kch, cta0 = vals[i:i + 6]
+            i += 6
+            probs.append(dict(job=job, row0=row0, rows=rows, glog=glog, kch=kch, cta_begin=cta0))
+        launches.append(dict(ctas=ctas, smem=smem, problems=probs))
+    return launches
 
 
 def bl_debug_forward_prefill(packed, gamma, x_q, s, N: int, Y=None, acc_out=None, skip_iter: int = -1,

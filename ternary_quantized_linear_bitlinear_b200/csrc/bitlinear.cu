@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "bitlinear.h"
 #include "bitlinear_debug.h"
@@ -311,9 +312,13 @@ struct DecodeJob {
 // GPU); a CTA table maps each CTA to its problem.  A call with more CTAs or
 // problems than one launch holds is split into several launches (a problem
 // by row ranges).
+// With `plan` set nothing is launched: each launch the call would make is
+// appended to it as {CTAs, dynamic shared memory bytes, problems, then per
+// problem: job index, first row, rows, glog, K chunks, first CTA}.
 bl_status decode_launch(const DecodeJob *jobs, int count, int M, float eps, bool pdl, cudaStream_t st, int src,
-                        int sms) {
+                        int sms, std::vector<int> *plan = nullptr) {
     thread_local DecodeParams P;
+    int pjob[BL_MAX_GROUP];
     int glog[BL_MAX_GROUP], kchs[BL_MAX_GROUP];
     int64_t total = 0;
     for (int i = 0; i < count; ++i) {
@@ -336,6 +341,14 @@ bl_status decode_launch(const DecodeJob *jobs, int count, int M, float eps, bool
         P.acc_off = P.x_off + ((M * rs_max + 127) & ~127);
         const size_t smem = (size_t)P.acc_off + (size_t)t_max * DEC_ROWS * M * 4;
         if (M * rs_max > DEC_X_MAX || smem > DEC_SMEM_ATTR) return BL_ERR_SHAPE;
+        if (plan != nullptr) {
+            plan->insert(plan->end(), {nc, (int)smem, P.count});
+            for (int q = 0; q < P.count; ++q)
+                plan->insert(plan->end(), {pjob[q], P.p[q].row0, P.p[q].rows, P.p[q].glog, P.p[q].kch, P.p[q].cta_begin});
+            P.count = 0;
+            nc = w_max = rs_max = t_max = 0;
+            return BL_OK;
+        }
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)nc);
         cfg.blockDim = dim3(DEC_THREADS);
@@ -391,6 +404,7 @@ bl_status decode_launch(const DecodeJob *jobs, int count, int M, float eps, bool
             P.p[P.count] = DecodeProblem{j.packed, j.gamma, j.x, j.s, j.Y, j.acc, j.gain, j.xq_out,
                                          N, K, row, nrows, glog[i], nc, kch};
             for (int c = 0; c < cn; ++c) P.cta_problem[nc + c] = (unsigned char)P.count;
+            pjob[P.count] = i;
             nc += cn;
             ++P.count;
             row += nrows;
@@ -859,3 +873,27 @@ extern "C" bl_status bl_debug_forward_prefill(const uint8_t *packed, const float
     return prefill_launch(d->sms, packed, gamma, x_q, s, M, N, K, Y, acc_out, (cudaStream_t)stream,
                           (unsigned long long)timeout_us * 1000ull, skip_iter < 0 ? -1 : skip_iter);
 }
+
+extern "C" bl_status bl_debug_decode_plan(const int64_t *shapes, int count, int64_t M, int sms, int *out,
+                                          int out_len, int *written) {
+    if (!shapes || !out || !written) return BL_ERR_NULL;
+    if (count < 1 || count > BL_MAX_GROUP || M < 1 || M > 16 || sms < 1 || out_len < 1) return BL_ERR_SHAPE;
+    DecodeJob jobs[BL_MAX_GROUP];
+    // placeholder addresses: the plan reads only the shapes
+    static const float dummy[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < count; ++i) {
+        const int64_t N = shapes[2 * i], K = shapes[2 * i + 1];
+        if (N < 1 || N > 0x7fffffffLL || check_k(K) != BL_OK || !nk_fits(N, K) || !decode_eligible(M, K))
+            return BL_ERR_SHAPE;
+        jobs[i] = DecodeJob{reinterpret_cast<const uint8_t *>(dummy), dummy, dummy, nullptr, nullptr, nullptr,
+                            nullptr, nullptr, N, K};
+    }
+    std::vector<int> plan;
+    bl_status rc = decode_launch(jobs, count, (int)M, 0.f, false, nullptr, DEC_SRC_XQ, sms, &plan);
+    if (rc) return rc;
+    if ((int)plan.size() > out_len) return BL_ERR_WORKSPACE;
+    std::memcpy(out, plan.data(), plan.size() * sizeof(int));
+    *written = (int)plan.size();
+    return BL_OK;
+}
+

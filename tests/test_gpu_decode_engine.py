@@ -4,8 +4,8 @@ per group split its k steps; partial sums meet in a shared-memory table),
 groups too long for shared memory are staged in 2 KiB chunks of their rows,
 launches too small to fill the GPU take one group per CTA, and a call is
 split into several launches when it holds more CTAs than one launch maps,
-when its problems' shared-memory layouts do not fit together, or when a
-problem would take the third CTA slot per SM from the others.  These cases
+or when a problem would take the third CTA slot per SM from the others
+(the host-side planner's cases are in test_decode_plan.py).  These cases
 drive the corners of that: many tiny problems, one group of many chunks,
 steps with only part of their 256 k in range, whole groups up to 96 KiB,
 the splits, and launches repeated on the same buffers.
@@ -93,11 +93,10 @@ def test_m16_wide_activations_one_problem_per_cta():
         check_forward_full(xq_ref, s_ref, wq_ref, g_ref, d[4], d[7])
 
 
-def test_whole_and_chunked_groups_and_a_layout_split():
+def test_whole_and_chunked_groups_in_one_launch():
     """K = 6144 at M = 4: whole groups of 48 KiB; K = 8640 and 12288 chunked
-    (2160- and 3072-byte rows); K = 32768 (128 KiB of x_q at M = 4) with the
-    others' layouts does not fit one launch, so the call is split into
-    launches."""
+    (2160- and 3072-byte rows); K = 32768 (128 KiB of x_q at M = 4) beside
+    them: the largest layouts share one launch (a few CTAs, one group each)."""
     _xq_path([(70, 8640), (65, 12288), (40, 32768), (33, 768), (50, 6144)], 4, 1400)
 
 
