@@ -106,7 +106,8 @@ struct WqIn {
 // Reduction blocks per matrix: a share of 2 x SMs proportional to its size,
 // at least enough that no thread sums more than 2^14 terms (which keeps each
 // 64-bit window accumulator exact), at most one vector per thread, and at
-// most WQ_MAX_BLOCKS over the launch.
+// most WQ_MAX_BLOCKS over the launch.  Pack blocks: a share of 8 x SMs (at
+// most one word per thread), at least one per matrix.
 bl_status quant_weights_impl(const DeviceInfo &d, const WqIn *in, int count, bl_dtype wdt, void *ws,
                              cudaStream_t st) {
     if (count < 1 || count > WQ_MAX_JOBS) return BL_ERR_SHAPE;
@@ -118,7 +119,6 @@ bl_status quant_weights_impl(const DeviceInfo &d, const WqIn *in, int count, bl_
     P.count = count;
     P.partials = reinterpret_cast<u64 *>(ws);
     P.thresh = reinterpret_cast<u32 *>(reinterpret_cast<uint8_t *>(ws) + WQ_WS_PARTIALS);
-    P.tickets = reinterpret_cast<u32 *>(reinterpret_cast<uint8_t *>(ws) + WQ_WS_TICKET);
     double total = 0.0;
     for (int i = 0; i < count; ++i) total += (double)in[i].N * (double)in[i].K;
     long long blocks = 0, words = 0;
@@ -134,7 +134,7 @@ bl_status quant_weights_impl(const DeviceInfo &d, const WqIn *in, int count, bl_
         if (nb < 1) nb = 1;
         mins += minb;
         P.j[i] = WqJob{reinterpret_cast<const uint4 *>(in[i].W), nvec, n, in[i].gamma,
-                       reinterpret_cast<u32 *>(in[i].packed), n / 16, words, (int)blocks, (int)nb};
+                       reinterpret_cast<u32 *>(in[i].packed), n / 16, (int)blocks, (int)nb, 0, 0};
         blocks += nb;
         words += n / 16;
     }
@@ -153,27 +153,36 @@ bl_status quant_weights_impl(const DeviceInfo &d, const WqIn *in, int count, bl_
         }
         if (blocks > WQ_MAX_BLOCKS) return BL_ERR_SHAPE;
     }
-    P.total_words = words;
-    if (cudaMemsetAsync(P.tickets, 0, sizeof(u32) * count, st) != cudaSuccess) return BL_ERR_CUDA;
+    const long long pcap = 8LL * d.sms;
+    long long pblocks = 0;
+    for (int i = 0; i < count; ++i) {
+        const long long need = (P.j[i].nwords + WQ_PACK_THREADS - 1) / WQ_PACK_THREADS;
+        long long nb = (long long)std::llround((double)pcap * ((double)P.j[i].nwords / (double)words));
+        if (nb > need) nb = need;
+        if (nb < 1) nb = 1;
+        P.j[i].pblk0 = (int)pblocks;
+        P.j[i].pnblk = (int)nb;
+        pblocks += nb;
+    }
     if (bf16)
         k_absmean_partial<true><<<(unsigned)blocks, WQ_THREADS, 0, st>>>(P);
     else
         k_absmean_partial<false><<<(unsigned)blocks, WQ_THREADS, 0, st>>>(P);
     if (cudaGetLastError() != cudaSuccess) return BL_ERR_CUDA;
-    long long pgrid = (words + 255) / 256;
-    const long long pcap = 8LL * d.sms;
-    if (pgrid > pcap) pgrid = pcap;
-    // programmatic dependent launch: the pack grid starts loading W while the
-    // reduction finishes and waits for it (griddepcontrol.wait) before using T
+    // programmatic dependent launches: the final grid waits for the
+    // reduction (griddepcontrol.wait) before it reads the partials; the pack
+    // grid starts loading W while both run and waits for T
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)pgrid);
-    cfg.blockDim = dim3(256);
+    cfg.blockDim = dim3(WQ_PACK_THREADS);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    cfg.gridDim = dim3((unsigned)count);
+    if (cudaLaunchKernelEx(&cfg, k_absmean_final, P) != cudaSuccess) return BL_ERR_CUDA;
+    cfg.gridDim = dim3((unsigned)pblocks);
     cudaError_t e = bf16 ? cudaLaunchKernelEx(&cfg, k_ternary_pack<true>, P)
                          : cudaLaunchKernelEx(&cfg, k_ternary_pack<false>, P);
     return e == cudaSuccess ? BL_OK : BL_ERR_CUDA;
@@ -812,9 +821,9 @@ bl_status bl_linear_grouped(const bl_linear_problem *problems, int count, bl_dty
 
 // ---------------------------------------------------------------------------
 // Weight quantization without caller-provided scratch (see the header): the
-// reduction's per-block partials and the threshold word live in this static
-// array.  Host code must not hand the symbol itself to a kernel -- in host
-// code it names a host-side stand-in -- so the device address is looked up
+// reduction's per-block partials live in this static array.  Host code must
+// not hand the symbol itself to a kernel -- in host code it names a
+// host-side stand-in -- so the device address is looked up
 // once per device with cudaGetSymbolAddress.
 
 namespace {

@@ -2,21 +2,23 @@
 // 2-bit packing ("Distillix" README, 1. BitNet b1.58 Core; "bitone" README,
 // Forward pass; "SLM750-Edge" section 3.1).
 //
-// Two launches, both on the caller's stream, each over one or several
-// weight matrices (up to WQ_MAX_JOBS: e.g. the projections of a layer, so
-// their reduction latency chains overlap):
+// Three launches on the caller's stream, each over one or several weight
+// matrices (up to WQ_MAX_JOBS: e.g. the projections of a layer, so their
+// reduction latency chains overlap), chained as programmatic dependents:
 //   k_absmean_partial  one pass over W: exact per-block sum of |w| as a
-//                      384-bit fixed-point integer in units of 2^-149; the
-//                      last block of a matrix to finish (ticket counter)
-//                      sums its block partials, rounds once to double,
-//                      gamma = float(S / n) + 1e-5f, and the float
-//                      threshold T with
-//                      |w| >= T  <=>  float(|w|/gamma) > 0.5
-//   k_ternary_pack     second pass over W: W_q = sign(w) * (|w| >= T), stored
+//                      384-bit fixed-point integer in units of 2^-149,
+//                      written to the workspace
+//   k_absmean_final    one CTA per matrix: sums its block partials, rounds
+//                      once to double, gamma = float(S / n) + 1e-5f, and the
+//                      float threshold T with
+//                        |w| >= T  <=>  float(|w|/gamma) > 0.5
+//   k_ternary_pack     second pass over W (its first words requested before
+//                      the wait for T): W_q = sign(w) * (|w| >= T), stored
 //                      as the code 1 - W_q, four codes per byte in the
-//                      packed word layout; launched as
-//                      a programmatic dependent, it loads its first words of
-//                      W before waiting for gamma and T
+//                      packed word layout
+// No CTA waits on another CTA of its own launch, and nothing in the
+// workspace needs clearing: every word a launch reads there was written by
+// the launch before it.
 //
 // Exactness: every finite float is an integer multiple of 2^-149, so sum|w|
 // is an integer in those units.  Each thread accumulates m << (e - base) in a
@@ -32,17 +34,18 @@
 namespace bl {
 
 constexpr int WQ_THREADS = 512;
+constexpr int WQ_PACK_THREADS = 256;
 constexpr int WQ_WINDOW = 25;       // fast path: base <= e <= base + 25
 constexpr int WQ_PART_LIMBS = 6;    // per-block partial, 384 bits
 constexpr int WQ_MAX_BLOCKS = 1024; // over all matrices of a launch
 constexpr int WQ_MAX_JOBS = 8;      // weight matrices per launch
 constexpr size_t WQ_WS_PARTIALS = (size_t)WQ_MAX_BLOCKS * WQ_PART_LIMBS * 8;
-constexpr size_t WQ_WS_BYTES = WQ_WS_PARTIALS + 256;  // + threshold words, ticket counters
-constexpr size_t WQ_WS_TICKET = WQ_WS_PARTIALS + 128;  // u32 per matrix, zeroed by the host before each reduction
+constexpr size_t WQ_WS_BYTES = WQ_WS_PARTIALS + 256;  // + threshold words
 
 // One weight matrix of a (grouped) quantization launch: blocks
-// [blk0, blk0 + nblk) of the reduction grid sum it; its packed words are
-// words [word0, word0 + nwords) of the pack grid's index space.
+// [blk0, blk0 + nblk) of the reduction grid sum it, block j of the final
+// grid derives its gamma and T, blocks [pblk0, pblk0 + pnblk) of the pack
+// grid pack it.
 struct WqJob {
     const uint4 *W;
     long long nvec;   // 16-byte vectors
@@ -50,18 +53,17 @@ struct WqJob {
     float *gamma;
     u32 *packed;
     long long nwords; // packed 32-bit words (16 weights each)
-    long long word0;
     int blk0;
     int nblk;
+    int pblk0;
+    int pnblk;
 };
 
 struct WqParams {
     WqJob j[WQ_MAX_JOBS];
     int count;
-    long long total_words;
     u64 *partials;    // [WQ_MAX_BLOCKS][WQ_PART_LIMBS]
-    u32 *thresh;      // [WQ_MAX_JOBS]
-    u32 *tickets;     // [WQ_MAX_JOBS]
+    u32 *thresh;      // [WQ_MAX_JOBS] float bits of T
 };
 
 // Float bits of the j-th element of a 16-byte vector.
@@ -76,21 +78,24 @@ __device__ __forceinline__ u32 vec_elem_bits(const uint4 &v, int j) {
     }
 }
 
-// Sums the block partials (one limb position per pass, 128 bits per limb
-// across the block), rounds the total to double and derives gamma and T.
-// Whole block; thread 0 writes the results.
-__device__ void wq_finalize_block(const u64 *partials, int nblocks, long long n, float *gamma_out,
-                                  u32 *ws_thresh) {
+// Sums a matrix's block partials (one limb position per pass, 128 bits per
+// limb across the block), rounds the total to double and derives gamma and
+// T.  Whole block of NT threads; every thread returns with s_out[0] = gamma
+// bits and s_out[1] = T bits.
+template <int NT>
+__device__ void wq_gamma_threshold(const u64 *partials, int nblocks, long long n, u32 *s_out) {
     constexpr int NL = WQ_PART_LIMBS;
-    __shared__ u64 f_lo[NL][WQ_THREADS / 32], f_hi[NL][WQ_THREADS / 32];
+    constexpr int NW = NT / 32;
+    __shared__ u64 f_lo[NL][NW], f_hi[NL][NW];
+    __shared__ u64 f_sum[NL][2];
     const int tid = threadIdx.x;
     u64 slo[NL], shi[NL];
 #pragma unroll
     for (int k = 0; k < NL; ++k) slo[k] = shi[k] = 0ull;
-    for (int b = tid; b < nblocks; b += WQ_THREADS) {
+    for (int b = tid; b < nblocks; b += NT) {
 #pragma unroll
         for (int k = 0; k < NL; ++k) {
-            // written by other blocks of this grid: bypass L1
+            // written by the reduction grid: bypass L1
             const u64 v = __ldcg(partials + (size_t)b * NL + k);
             const u64 t = slo[k] + v;
             shi[k] += t < v ? 1ull : 0ull;
@@ -107,12 +112,11 @@ __device__ void wq_finalize_block(const u64 *partials, int nblocks, long long n,
     }
     __syncthreads();
     // limb position k summed over the warps by lane k of warp 0 (128 bits:
-    // a thread adds at most two 64-bit limbs, a warp's sum is below 2^70,
-    // the sixteen warps' below 2^74)
-    __shared__ u64 f_sum[NL][2];
+    // a thread adds at most four 64-bit limbs, the block's sum is below 2^74)
     if (tid < NL) {
         u64 lo = 0ull, hi = 0ull;
-        for (int w = 0; w < WQ_THREADS / 32; ++w) {
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
             const u64 t = lo + f_lo[tid][w];
             hi += f_hi[tid][w] + (t < lo ? 1ull : 0ull);
             lo = t;
@@ -135,13 +139,14 @@ __device__ void wq_finalize_block(const u64 *partials, int nblocks, long long n,
         float t = __fmul_rn(0.5f, g);
         for (int it = 0; it < 64 && !(__fdiv_rn(t, g) > 0.5f); ++it)
             t = __uint_as_float(__float_as_uint(t) + 1u);
-        gamma_out[0] = g;
-        ws_thresh[0] = __float_as_uint(t);
+        s_out[0] = __float_as_uint(g);
+        s_out[1] = __float_as_uint(t);
     }
+    __syncthreads();
 }
 
 template <bool BF16>
-__global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const __grid_constant__ WqParams P) {
+__global__ void __launch_bounds__(WQ_THREADS, 2) k_absmean_partial(const __grid_constant__ WqParams P) {
     // the pack kernel may start loading W while this grid runs
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int EPV = BF16 ? 8 : 4;  // elements per 16-byte vector
@@ -155,7 +160,6 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const __grid_con
     const WqJob &job = P.j[ji];
     const uint4 *__restrict__ W = job.W;
     const long long nvec = job.nvec;
-    u64 *__restrict__ partials = P.partials;
 
     const int tid = threadIdx.x;
     for (int i = tid; i < 256; i += WQ_THREADS) s_bins[i] = 0ull;
@@ -164,19 +168,23 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const __grid_con
     const long long stride = (long long)job.nblk * WQ_THREADS;
     const long long first = (long long)((int)blockIdx.x - job.blk0) * WQ_THREADS + tid;
 
-    // Window from a sample: the block's first vector per thread.  The second
-    // vector is requested before the block reduction, so its latency overlaps.
+    // Window from a sample: the block's first vector per thread.  The next
+    // four vectors are requested before the block reduction, so their
+    // latency overlaps it.
     u32 emax = 0;
     uint4 v0 = make_uint4(0, 0, 0, 0);
-    const bool has1 = first + stride < nvec;
-    const uint4 v1 = has1 ? ldg_stream_v4(W + first + stride) : make_uint4(0, 0, 0, 0);
     if (first < nvec) {
         v0 = ldg_stream_v4(W + first);
+    }
+    uint4 a[4];
+    long long i = first + stride;
 #pragma unroll
-        for (int j = 0; j < EPV; ++j) {
-            u32 e = (vec_elem_bits<BF16>(v0, j) & 0x7fffffffu) >> 23;
-            emax = e > emax ? e : emax;
-        }
+    for (int q = 0; q < 4; ++q)
+        a[q] = i + q * stride < nvec ? ldg_stream_v4(W + i + q * stride) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int j = 0; j < EPV; ++j) {
+        u32 e = (vec_elem_bits<BF16>(v0, j) & 0x7fffffffu) >> 23;
+        emax = e > emax ? e : emax;
     }
     emax = warp_max_u32(emax);
     __syncthreads();
@@ -202,21 +210,24 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const __grid_con
             }
         }
     };
-    if (first < nvec) add_vec(v0);
-    if (has1) add_vec(v1);
-    long long i = first + 2 * stride;
-    // four vectors in flight per iteration
-    for (; i + 3 * stride < nvec; i += 4 * stride) {
-        const uint4 a = ldg_stream_v4(W + i);
-        const uint4 b = ldg_stream_v4(W + i + stride);
-        const uint4 c = ldg_stream_v4(W + i + 2 * stride);
-        const uint4 d = ldg_stream_v4(W + i + 3 * stride);
-        add_vec(a);
-        add_vec(b);
-        add_vec(c);
-        add_vec(d);
+    add_vec(v0);  // zero when first >= nvec
+    // Two stages of four vectors: the next four are in flight while the
+    // current four are summed.  a[] holds vectors i + q * stride (zero where
+    // past the end; zeros add nothing).
+    while (i + 4 * stride < nvec) {
+        const long long inext = i + 4 * stride;
+        uint4 b[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            b[q] = inext + q * stride < nvec ? ldg_stream_v4(W + inext + q * stride) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) add_vec(a[q]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) a[q] = b[q];
+        i = inext;
     }
-    for (; i < nvec; i += stride) add_vec(ldg_stream_v4(W + i));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) add_vec(a[q]);
 
     // Block sum of the 64-bit window accumulators as 128 bits.
     u64 lo = acc, hi = 0ull;
@@ -250,64 +261,60 @@ __global__ void __launch_bounds__(WQ_THREADS) k_absmean_partial(const __grid_con
                     limbs_add_u128_shl(L, s_bins[e], 0ull, e > 0 ? e - 1 : 0);
                 }
             }
+            // read by the pack grid after its griddepcontrol.wait (which
+            // returns once this grid has completed and its writes are visible)
 #pragma unroll
-            for (int k = 0; k < WQ_PART_LIMBS; ++k) partials[(size_t)blockIdx.x * WQ_PART_LIMBS + k] = L[k];
+            for (int k = 0; k < WQ_PART_LIMBS; ++k) P.partials[(size_t)blockIdx.x * WQ_PART_LIMBS + k] = L[k];
         }
     }
-
-    // The last block of this matrix to finish finalizes it (partials
-    // published with a fence before the ticket; the ticket is zeroed by the
-    // host before the launch and reset here for the next call on the same
-    // workspace).
-    __shared__ bool s_last;
-    if (tid == 0) {
-        __threadfence();
-        s_last = atomicAdd(&P.tickets[ji], 1u) == (u32)job.nblk - 1;
-    }
-    __syncthreads();
-    if (!s_last) return;
-    __threadfence();
-    wq_finalize_block(partials + (size_t)job.blk0 * WQ_PART_LIMBS, job.nblk, job.n, job.gamma, &P.thresh[ji]);
-    if (tid == 0) P.tickets[ji] = 0u;
 }
 
-// Each thread packs 16 consecutive weights into one 32-bit word per step;
-// the words of all matrices of the launch form one index space.
+// Block j derives gamma and T of matrix j from its reduction blocks'
+// partials (read after the reduction grid has completed).
+__global__ void __launch_bounds__(WQ_PACK_THREADS) k_absmean_final(const __grid_constant__ WqParams P) {
+    // the pack grid may start loading W now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    __shared__ u32 s_gt[2];
+    const WqJob &jb = P.j[blockIdx.x];
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    wq_gamma_threshold<WQ_PACK_THREADS>(P.partials + (size_t)jb.blk0 * WQ_PART_LIMBS, jb.nblk, jb.n, s_gt);
+    if (threadIdx.x == 0) {
+        jb.gamma[0] = __uint_as_float(s_gt[0]);
+        P.thresh[blockIdx.x] = s_gt[1];
+    }
+}
+
+// A CTA packs words of one matrix (grid-stride over its block range); each
+// thread packs 16 consecutive weights into one 32-bit word per step, the
+// next word's vectors in flight while it packs the current one.  T is read
+// after the final grid has completed (griddepcontrol.wait).
 template <bool BF16>
-__global__ void __launch_bounds__(256) k_ternary_pack(const __grid_constant__ WqParams P) {
+__global__ void __launch_bounds__(WQ_PACK_THREADS) k_ternary_pack(const __grid_constant__ WqParams P) {
     constexpr int VPW = BF16 ? 2 : 4;  // 16-byte vectors per 16 weights
+    constexpr int EPV = BF16 ? 8 : 4;
     // a programmatically dependent launch after this one (bl_linear's act
     // quant, which does not read the packed weights) may start now
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    const long long first = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    auto job_of = [&](long long w) {
-        int i = 0;
-        while (i + 1 < P.count && w >= P.j[i + 1].word0) ++i;
-        return i;
-    };
-    // first words of W are requested before waiting for the reduction grid
+    int ji = 0;
+    while (ji + 1 < P.count && (int)blockIdx.x >= P.j[ji + 1].pblk0) ++ji;
+    const WqJob &jb = P.j[ji];
+    const long long stride = (long long)jb.pnblk * WQ_PACK_THREADS;
+    long long wl = (long long)((int)blockIdx.x - jb.pblk0) * WQ_PACK_THREADS + threadIdx.x;
+    const long long nwords = jb.nwords;
+    // the first words of W are requested before waiting for the reduction grid
     uint4 v[VPW];
-    if (first < P.total_words) {
-        const WqJob &jb = P.j[job_of(first)];
-        const long long wl = first - jb.word0;
 #pragma unroll
-        for (int q = 0; q < VPW; ++q) v[q] = ldg_stream_v4(jb.W + wl * VPW + q);
-    }
+    for (int q = 0; q < VPW; ++q) v[q] = wl < nwords ? ldg_stream_v4(jb.W + wl * VPW + q) : make_uint4(0, 0, 0, 0);
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    for (long long wi = first; wi < P.total_words; wi += stride) {
-        const int ji = job_of(wi);
-        const WqJob &jb = P.j[ji];
-        const long long wl = wi - jb.word0;
-        if (wi != first) {
+    const u32 T = __ldcg(P.thresh + ji);  // written by the final grid
+    for (; wl < nwords; wl += stride) {
+        const long long wn = wl + stride;
+        uint4 nx[VPW];
 #pragma unroll
-            for (int q = 0; q < VPW; ++q) v[q] = ldg_stream_v4(jb.W + wl * VPW + q);
-        }
-        const u32 T = __ldcg(P.thresh + ji);
+        for (int q = 0; q < VPW; ++q) nx[q] = wn < nwords ? ldg_stream_v4(jb.W + wn * VPW + q) : make_uint4(0, 0, 0, 0);
         u32 word = 0;
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-            constexpr int EPV = BF16 ? 8 : 4;
             u32 bits = vec_elem_bits<BF16>(v[k / EPV], k % EPV);
             u32 nz = (bits & 0x7fffffffu) >= T ? 1u : 0u;
             u32 code = (nz ^ 1u) | ((bits >> 30) & 2u & (nz << 1));  // 1 - W_q: 00 = +1, 01 = 0, 10 = -1
@@ -315,6 +322,8 @@ __global__ void __launch_bounds__(256) k_ternary_pack(const __grid_constant__ Wq
             word |= code << (8 * i + 2 * j);
         }
         jb.packed[wl] = word;
+#pragma unroll
+        for (int q = 0; q < VPW; ++q) v[q] = nx[q];
     }
 }
 
