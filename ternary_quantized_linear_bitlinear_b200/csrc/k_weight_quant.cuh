@@ -307,19 +307,46 @@ __global__ void __launch_bounds__(WQ_PACK_THREADS) k_ternary_pack(const __grid_c
     for (int q = 0; q < VPW; ++q) v[q] = wl < nwords ? ldg_stream_v4(jb.W + wl * VPW + q) : make_uint4(0, 0, 0, 0);
     asm volatile("griddepcontrol.wait;" ::: "memory");
     const u32 T = __ldcg(P.thresh + ji);  // written by the final grid
+    // bf16: |w| >= T <=> the magnitude's 15 bits >= T16 = ceil(T / 2^16),
+    // tested on both halves of a word at once: (w & 0x7fff7fff) + C with
+    // C = (0x8000 - T16) per half has bit 15 (31) set exactly when the low
+    // (high) half is >= T16, and no carry crosses the halves (T16 >= 1, as
+    // gamma >= 1e-5)
+    const u32 T16 = (T + 0xffffu) >> 16;
+    const u32 C = (0x8000u - T16) * 0x00010001u;
     for (; wl < nwords; wl += stride) {
         const long long wn = wl + stride;
         uint4 nx[VPW];
 #pragma unroll
         for (int q = 0; q < VPW; ++q) nx[q] = wn < nwords ? ldg_stream_v4(jb.W + wn * VPW + q) : make_uint4(0, 0, 0, 0);
         u32 word = 0;
+        if (BF16) {
+            // pair p = weights 2p (low half) and 2p + 1: j = p / 2, i = 2 (p & 1) + half
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            u32 bits = vec_elem_bits<BF16>(v[k / EPV], k % EPV);
-            u32 nz = (bits & 0x7fffffffu) >= T ? 1u : 0u;
-            u32 code = (nz ^ 1u) | ((bits >> 30) & 2u & (nz << 1));  // 1 - W_q: 00 = +1, 01 = 0, 10 = -1
-            int i = k & 3, j = k >> 2;
-            word |= code << (8 * i + 2 * j);
+            for (int jp = 0; jp < 4; ++jp) {
+                u32 t[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int p = 2 * jp + h;
+                    const u32 w = (&v[p >> 2].x)[p & 3];
+                    const u32 nz = ((w & 0x7fff7fffu) + C) & 0x80008000u;
+                    // code 1 - W_q at bits 14-15 (low weight) and 30-31: bit 0 = zero, bit 1 = negative
+                    t[h] = ((nz ^ 0x80008000u) >> 1) | (nz & w);
+                }
+                // bytes 1 and 3 of t[0] (i = 0, 1) and of t[1] (i = 2, 3) hold the codes in
+                // their top two bits; word byte i takes code (4 jp + i) at bits 2 jp
+                const u32 b = __byte_perm(t[0], t[1], 0x7531u);
+                word |= (b >> (6 - 2 * jp)) & (0x03030303u << (2 * jp));
+            }
+        } else {
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                u32 bits = vec_elem_bits<BF16>(v[k / EPV], k % EPV);
+                u32 nz = (bits & 0x7fffffffu) >= T ? 1u : 0u;
+                u32 code = (nz ^ 1u) | ((bits >> 30) & 2u & (nz << 1));  // 1 - W_q: 00 = +1, 01 = 0, 10 = -1
+                int i = k & 3, j = k >> 2;
+                word |= code << (8 * i + 2 * j);
+            }
         }
         jb.packed[wl] = word;
 #pragma unroll
