@@ -44,6 +44,9 @@ def chain(W_cpu, X_cpu, gain_cpu=None, eps=1e-6, want_acc=True):
     (48, 512, torch.float32, "zeros"),
     (33, 320, torch.bfloat16, "ternary"),
     (9728, 2560, torch.bfloat16, "normal"),
+    (64, 1024, torch.bfloat16, "wide"),
+    (48, 512, torch.bfloat16, "zeros"),
+    (512, 2048, torch.bfloat16, "outliers"),
 ])
 def test_quant_weights(N, K, dtype, kind):
     if kind == "normal":
@@ -60,6 +63,16 @@ def test_quant_weights(N, K, dtype, kind):
         W = W.to(dtype)
     elif kind == "zeros":
         W = torch.zeros(N, K, dtype=dtype)
+    elif kind == "outliers":
+        # a few values outside the summing window of their block (tiny, a
+        # subnormal, huge) among normal ones: only the threads that meet
+        # them take the exact slow path
+        W = workloads.normal((N, K), 0.02, 7, torch.float32)
+        W[3, 7] = 1e-30
+        W[100, 5] = -(2.0 ** -130)
+        W[200, 1000] = 1e20
+        W[511, 2047] = 0.0
+        W = W.to(dtype)
     else:
         W = workloads.ternary_weights(N, K, seed=3, dtype=dtype)
     packed, gamma = gpu_quant_weights(W)
