@@ -146,6 +146,26 @@ __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ A
 // reductions by warp shuffles -- no block barrier at all.
 constexpr int AQW_WARPS = 8;
 
+// Per-half unsigned max of two 16-bit lanes.
+__device__ __forceinline__ u32 vmax_u16x2(u32 a, u32 b) {
+    u32 r;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// x_q bytes of four finite values with |x * s| <= 127: p = float(x * s),
+// then p + 1.5 * 2^23 rounds p to the nearest integer, ties to even (the
+// addend is even and its ulp is 1), and leaves that integer in two's
+// complement in the low byte of the sum's bits (|p| < 2^22).
+__device__ __forceinline__ u32 aq_pack4(float a, float b, float c, float d, float s) {
+    constexpr float RND = 12582912.0f;  // 1.5 * 2^23
+    const u32 ra = __float_as_uint(__fadd_rn(__fmul_rn(a, s), RND));
+    const u32 rb = __float_as_uint(__fadd_rn(__fmul_rn(b, s), RND));
+    const u32 rc = __float_as_uint(__fadd_rn(__fmul_rn(c, s), RND));
+    const u32 rd = __float_as_uint(__fadd_rn(__fmul_rn(d, s), RND));
+    return __byte_perm(__byte_perm(ra, rb, 0x0040u), __byte_perm(rc, rd, 0x0040u), 0x5410u);
+}
+
 template <bool BF16>
 __device__ __forceinline__ u32 aq_bits(const uint4 &v, int j) {
     const u32 w = j < (BF16 ? 2 : 1) ? v.x : j < (BF16 ? 4 : 2) ? v.y : j < (BF16 ? 6 : 3) ? v.z : v.w;
@@ -178,29 +198,57 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_
                 raw[v] = glu_relu2_v4(raw[v], ldg_stream_v4(reinterpret_cast<const uint4 *>(pr.X2) + (size_t)m * nvec + vi));
         }
     }
+    if (BF16) {
+        // both halves of a word at once: max of the 15-bit magnitudes
+        u32 m2 = 0;
 #pragma unroll
-    for (int v = 0; v < VPL; ++v)
+        for (int v = 0; v < VPL; ++v) {
+            m2 = vmax_u16x2(m2, raw[v].x & 0x7fff7fffu);
+            m2 = vmax_u16x2(m2, raw[v].y & 0x7fff7fffu);
+            m2 = vmax_u16x2(m2, raw[v].z & 0x7fff7fffu);
+            m2 = vmax_u16x2(m2, raw[v].w & 0x7fff7fffu);
+        }
+        amax = max(m2 << 16, m2 & 0xffff0000u);
+    } else {
 #pragma unroll
-        for (int j = 0; j < EPV; ++j) amax = max(amax, aq_bits<BF16>(raw[v], j) & 0x7fffffffu);
+        for (int v = 0; v < VPL; ++v)
+#pragma unroll
+            for (int j = 0; j < EPV; ++j) amax = max(amax, aq_bits<BF16>(raw[v], j) & 0x7fffffffu);
+    }
     amax = warp_max_u32(amax);
     const float s = __fdiv_rn(127.f, fmaxf(__uint_as_float(amax), 1e-5f));
     if (lane == 0) pr.s[m] = s;
     int8_t *qr = pr.xq + (size_t)m * K;
+    // finite rows: |x * s| <= 127, so rne and the int8 byte come from one
+    // addend (aq_pack4) and no clamp applies; a row with inf / NaN takes the
+    // converting path
+    const bool finite = amax < 0x7f800000u;
 #pragma unroll
     for (int v = 0; v < VPL; ++v) {
         const int vi = lane + v * 32;
         if (vi >= nvec) continue;
         u32 out[EPV / 4];
+        if (finite) {
 #pragma unroll
-        for (int q = 0; q < EPV / 4; ++q) {
-            u32 word = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                int qi = __float2int_rn(__fmul_rn(__uint_as_float(aq_bits<BF16>(raw[v], 4 * q + j)), s));
-                qi = max(-128, min(127, qi));
-                word |= ((u32)qi & 0xffu) << (8 * j);
+            for (int q = 0; q < EPV / 4; ++q) {
+                const float a = __uint_as_float(aq_bits<BF16>(raw[v], 4 * q + 0));
+                const float b = __uint_as_float(aq_bits<BF16>(raw[v], 4 * q + 1));
+                const float c = __uint_as_float(aq_bits<BF16>(raw[v], 4 * q + 2));
+                const float d = __uint_as_float(aq_bits<BF16>(raw[v], 4 * q + 3));
+                out[q] = aq_pack4(a, b, c, d, s);
             }
-            out[q] = word;
+        } else {
+#pragma unroll
+            for (int q = 0; q < EPV / 4; ++q) {
+                u32 word = 0;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    int qi = __float2int_rn(__fmul_rn(__uint_as_float(aq_bits<BF16>(raw[v], 4 * q + j)), s));
+                    qi = max(-128, min(127, qi));
+                    word |= ((u32)qi & 0xffu) << (8 * j);
+                }
+                out[q] = word;
+            }
         }
         if (BF16) {
             *reinterpret_cast<uint2 *>(qr + (size_t)vi * 8) = make_uint2(out[0], out[EPV / 4 - 1]);
