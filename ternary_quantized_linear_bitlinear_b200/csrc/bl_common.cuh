@@ -53,6 +53,22 @@ __device__ __forceinline__ u64 mad_wide_u32(u32 a, u32 b, u64 c) {
     return d;
 }
 
+// INT8 activation codes of four finite values whose |x * s| is at most 127
+// (s = 127 / max|x| of their row): p = float(x * s), then p + 1.5 * 2^23
+// rounds p to the nearest integer, ties to even (the addend is even and
+// its ulp is 1), and leaves that integer in two's complement in the low
+// byte of the sum's bits (|p| < 2^22); the four bytes are packed first in
+// the low byte.  Equal to clamp(rne(float(x * s)), -128, 127), which needs
+// no clamp there.
+__device__ __forceinline__ u32 pack4_s8_rne(float a, float b, float c, float d, float s) {
+    constexpr float RND = 12582912.0f;  // 1.5 * 2^23
+    const u32 ra = __float_as_uint(__fadd_rn(__fmul_rn(a, s), RND));
+    const u32 rb = __float_as_uint(__fadd_rn(__fmul_rn(b, s), RND));
+    const u32 rc = __float_as_uint(__fadd_rn(__fmul_rn(c, s), RND));
+    const u32 rd = __float_as_uint(__fadd_rn(__fmul_rn(d, s), RND));
+    return __byte_perm(__byte_perm(ra, rb, 0x0040u), __byte_perm(rc, rd, 0x0040u), 0x5410u);
+}
+
 // ---------------------------------------------------------------------------
 // Exact multi-limb fixed point (little-endian u64 limbs).
 

@@ -153,19 +153,6 @@ __device__ __forceinline__ u32 vmax_u16x2(u32 a, u32 b) {
     return r;
 }
 
-// x_q bytes of four finite values with |x * s| <= 127: p = float(x * s),
-// then p + 1.5 * 2^23 rounds p to the nearest integer, ties to even (the
-// addend is even and its ulp is 1), and leaves that integer in two's
-// complement in the low byte of the sum's bits (|p| < 2^22).
-__device__ __forceinline__ u32 aq_pack4(float a, float b, float c, float d, float s) {
-    constexpr float RND = 12582912.0f;  // 1.5 * 2^23
-    const u32 ra = __float_as_uint(__fadd_rn(__fmul_rn(a, s), RND));
-    const u32 rb = __float_as_uint(__fadd_rn(__fmul_rn(b, s), RND));
-    const u32 rc = __float_as_uint(__fadd_rn(__fmul_rn(c, s), RND));
-    const u32 rd = __float_as_uint(__fadd_rn(__fmul_rn(d, s), RND));
-    return __byte_perm(__byte_perm(ra, rb, 0x0040u), __byte_perm(rc, rd, 0x0040u), 0x5410u);
-}
-
 template <bool BF16>
 __device__ __forceinline__ u32 aq_bits(const uint4 &v, int j) {
     const u32 w = j < (BF16 ? 2 : 1) ? v.x : j < (BF16 ? 4 : 2) ? v.y : j < (BF16 ? 6 : 3) ? v.z : v.w;
@@ -235,7 +222,7 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_warp(const __grid_
                 const float b = __uint_as_float(aq_bits<BF16>(raw[v], 4 * q + 1));
                 const float c = __uint_as_float(aq_bits<BF16>(raw[v], 4 * q + 2));
                 const float d = __uint_as_float(aq_bits<BF16>(raw[v], 4 * q + 3));
-                out[q] = aq_pack4(a, b, c, d, s);
+                out[q] = pack4_s8_rne(a, b, c, d, s);
             }
         } else {
 #pragma unroll
@@ -630,8 +617,13 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
     if (tid == 0) pr.s[m] = s;
     // pass 4: quantize, four elements -> one 32-bit word
     u32 *qr = reinterpret_cast<u32 *>(pr.xq + (size_t)m * K);
+    const bool finite = amax < 0x7f800000u;  // else the converting path (inf / NaN in the row)
     for (int q = tid; q < K / 4; q += AQR_THREADS) {
         const float4 y = reinterpret_cast<const float4 *>(s_row)[q];
+        if (finite) {
+            qr[q] = pack4_s8_rne(y.x, y.y, y.z, y.w, s);
+            continue;
+        }
         const float yy[4] = {y.x, y.y, y.z, y.w};
         u32 w = 0;
 #pragma unroll
