@@ -153,6 +153,13 @@ __device__ __forceinline__ u32 vmax_u16x2(u32 a, u32 b) {
     return r;
 }
 
+// Per-half unsigned min of two 16-bit lanes.
+__device__ __forceinline__ u32 vmin_u16x2(u32 a, u32 b) {
+    u32 r;
+    asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 template <bool BF16>
 __device__ __forceinline__ u32 aq_bits(const uint4 &v, int j) {
     const u32 w = j < (BF16 ? 2 : 1) ? v.x : j < (BF16 ? 4 : 2) ? v.y : j < (BF16 ? 6 : 3) ? v.z : v.w;
@@ -410,15 +417,40 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid
 }
 
 // One CTA (AQR_THREADS threads) per row with SubLN, the row cached in shared
-// memory as float32: the same arithmetic and passes as k_act_quant_subln,
-// with the row's elements spread over four warps and the reductions (max,
-// the windowed exact sum of squares and its "smaller values remain" flag)
-// combined through shared memory.  A warp per row left too few independent
-// chains per SM to hide the latency of the exact arithmetic.
+// memory as float32: the same result as k_act_quant_subln, with the row's
+// elements spread over four warps and the reductions combined through
+// shared memory.  A warp per row left too few independent chains per SM to
+// hide the latency of the arithmetic.
+//
+// r needs f = float(double(S) / K) for the exact S = sum x^2.  The square of
+// a float (24-bit significand) is exact in double and no float's square
+// over- or underflows there, so pass 1 also sums the squares in double as
+// it loads the row: S_hat, within beta * S_hat of the sum of the squares it
+// was given (beta = 2 (K + 256) 2^-53 covers every rounding of the
+// non-negative sum: at most K + 256 additions on any path), which are the
+// exact squares except that zero and subnormal x enter as values below
+// 2^-125, i.e. within A = K 2^-250 above S.  Hence S lies in
+// [S_hat (1 - beta) - A, S_hat (1 + beta)]; f is monotone in S, so when both
+// ends give the same f that is f(S), bit for bit.  Rows where they differ
+// (S / K within about 10^-12 of a float rounding boundary) or with inf /
+// NaN sum the squares exactly by windows over the cached row, as
+// k_act_quant_subln does.
 constexpr int AQR_THREADS = 128;
 constexpr int AQR_WARPS = AQR_THREADS / 32;
 constexpr int AQR_MAX_K = 24 * 1024;  // rows cached per CTA: K * 4 bytes of dynamic shared memory
-constexpr int AQR_FAST_SPAN = 19;     // bf16 rows: exponent span of the 64-bit exact sum of squares
+
+// |x| of a float's bits as a double: exponent rebiased, mantissa moved;
+// exact for normal x, below 2^-125 for zero and subnormal x.
+__device__ __forceinline__ double aqr_abs_double(u32 b) {
+    const u32 a = b & 0x7fffffffu;
+    return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
+}
 
 __device__ __forceinline__ u32 aqr_block_max(u32 v, u32 *s_u) {
     v = warp_max_u32(v);
@@ -448,9 +480,13 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
     const uint4 *xr = reinterpret_cast<const uint4 *>(pr.X) + (size_t)m * nvec;
     const uint4 *ur = GLU ? reinterpret_cast<const uint4 *>(pr.X2) + (size_t)m * nvec : nullptr;
     const float4 *g4 = reinterpret_cast<const float4 *>(pr.gain);
-    // pass 1: load (once), cache as float, max|x| (bf16 rows also the
-    // smallest nonzero |x|'s exponent, 255 - e carried as a max)
-    u32 amax = 0, inv_emin = 0;
+    // pass 1: load (once), cache as float, max|x|, and (SubLN rows) the
+    // double sum of squares S_hat
+    // (bf16: also the smallest exponent field, two halves at a time; 0 means
+    // the row holds a zero or a subnormal value)
+    const bool sub = g4 != nullptr;
+    u32 amax = 0, emin2 = 0xffffffffu;
+    double dsq = 0.0;
     for (int v0 = 0; v0 < nvec; v0 += AQR_THREADS * U) {
         uint4 c[U];
 #pragma unroll
@@ -469,13 +505,21 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
         for (int i = 0; i < U; ++i) {
             const int vi = v0 + AQR_THREADS * i + tid;
             if (vi >= nvec) continue;
+            if (BF16) {
+                emin2 = vmin_u16x2(emin2, c[i].x & 0x7f807f80u);
+                emin2 = vmin_u16x2(emin2, c[i].y & 0x7f807f80u);
+                emin2 = vmin_u16x2(emin2, c[i].z & 0x7f807f80u);
+                emin2 = vmin_u16x2(emin2, c[i].w & 0x7f807f80u);
+            }
             float f[EPV];
 #pragma unroll
             for (int j = 0; j < EPV; ++j) {
                 const u32 b = aq_bits<BF16>(c[i], j);
                 amax = max(amax, b & 0x7fffffffu);
-                // (a subnormal counts as exponent 0: below any window)
-                if (BF16 && (b & 0x7fffffffu) != 0u) inv_emin = max(inv_emin, 255u - ((b >> 23) & 0xffu));
+                if (sub) {
+                    const double xd = aqr_abs_double(b);
+                    dsq = __fma_rn(xd, xd, dsq);
+                }
                 f[j] = __uint_as_float(b);
             }
 #pragma unroll
@@ -484,38 +528,44 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
         }
     }
     amax = aqr_block_max(amax, s_u);  // also orders the row cache writes before the reads below
-    if (BF16 && g4 != nullptr) inv_emin = aqr_block_max(inv_emin, s_u);
-    if (g4 != nullptr) {
-        // pass 2: exact sum of squares
+    // bf16 rows without zero or subnormal values take Markstein's division
+    // in pass 3 without a per-element test
+    const bool bf16_normal = BF16 && sub && !__syncthreads_or((emin2 & 0xffffu) == 0u || (emin2 >> 16) == 0u);
+    if (sub) {
+        // f = float(double(S) / K) from S_hat when its bounds agree
+        __shared__ double s_d[AQR_WARPS];
+        __shared__ float s_f;
+        __shared__ int s_exact;
+        dsq = warp_sum_f64(dsq);
+        if (lane == 0) s_d[warp] = dsq;
+        __syncthreads();
+        if (tid == 0) {
+            double sh = s_d[0];
+            for (int w = 1; w < AQR_WARPS; ++w) sh = __dadd_rn(sh, s_d[w]);
+            int exact = 1;
+            if (amax < 0x7f800000u) {
+                const double beta = 2.0 * (double)(K + 256) * 0x1p-53;
+                const double A = (double)K * 0x1p-250;
+                double lo = __dsub_rd(__dmul_rd(sh, 1.0 - beta), A);
+                lo = lo > 0.0 ? lo : 0.0;
+                const double hi = __dmul_ru(sh, 1.0 + beta);
+                const float flo = __double2float_rn(__ddiv_rn(lo, (double)K));
+                const float fhi = __double2float_rn(__ddiv_rn(hi, (double)K));
+                if (flo == fhi) {
+                    s_f = flo;
+                    exact = 0;
+                }
+            }
+            s_exact = exact;
+        }
+        __syncthreads();
+        if (!s_exact) {
+            if (tid == 0) s_r = __fsqrt_rn(__fadd_rn(s_f, P.eps));
+        } else {
+        // exact sum of squares by windows over the cached row
         u64 L[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
         int ehi = (int)(amax >> 23);
         if (ehi < 1) ehi = 1;
-        const int emin = 255 - (int)inv_emin;
-        // bf16 rows whose nonzero |x| span at most AQR_FAST_SPAN binades (no
-        // subnormal): x^2 = m^2 * 2^(2e - 268) with the 8-bit mantissa m, so
-        // m^2 << 2(e - emin) < 2^(16 + 38) and at most 2^8 terms per thread
-        // stay below 2^62: one 64-bit accumulator per thread, no window pass
-        if (BF16 && emin >= 1 && ehi - emin <= AQR_FAST_SPAN && K <= AQR_THREADS * 256) {
-            u64 acc = 0ull;
-            for (int k = tid; k < K; k += AQR_THREADS) {
-                const u32 u = __float_as_uint(s_row[k]) & 0x7fffffffu;
-                const u32 m = ((u >> 16) & 0x7fu) | 0x80u;
-                const int sh = 2 * ((int)(u >> 23) - emin);  // 0 .. 2 AQR_FAST_SPAN for u != 0
-                const u64 t = (u64)(m * m) << (sh & 63);
-                acc += u != 0u ? t : 0ull;
-            }
-            u64 lo = acc, hi = 0ull;
-            warp_sum_u128(lo, hi);
-            if (lane == 0) {
-                s_lo[warp] = lo;
-                s_hi[warp] = hi;
-            }
-            __syncthreads();
-            // term = m^2 << 2(e - emin) stands for x^2 = term * 2^(2 emin - 268),
-            // i.e. term << (2 emin + 30) units of 2^-298
-            if (tid == 0)
-                for (int w = 0; w < AQR_WARPS; ++w) limbs_add_u128_shl(L, s_lo[w], s_hi[w], 2 * emin + 30);
-        } else
         for (int pass = 0; pass < 10; ++pass) {
             const int elo = ehi - 30 < 1 ? 1 : ehi - 30;
             u64 lo = 0ull, hi = 0ull;
@@ -551,6 +601,7 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
         }
         if (tid == 0)
             s_r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(limbs_to_double_rn(L, -298), (double)K)), P.eps));
+        }
         __syncthreads();
         const float r = s_r;
         // pass 3: y = float(float(x / r) * g) in place, max|y|.  For float32
@@ -568,7 +619,7 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
         // rounds to 0 either way, and such a y is the row maximum only when
         // every |y| of the row is below 1e-5, where s is floored at
         // 127 / 1e-5 whatever the maximum is.
-        // Measured 172 -> 136 us for [8192, 4096].  A bf16 row without
+        // Measured 172 -> 136 us for [8192, 4096].  A bf16 row without zero or
         // subnormal values (known from pass 1) takes Markstein for every
         // element without the per-element test (717 -> 638 us for [32768,
         // 9728]); other bf16 rows keep the IEEE division, which with the
@@ -582,8 +633,8 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
             return __fmaf_rn(__fmaf_rn(-q0, r, x), ry, q0);
         };
         amax = 0;
-        if (BF16 && emin >= 1 && __float_as_uint(r) >= 0x00800000u && __float_as_uint(r) < 0x7f800000u) {
-            // a bf16 row without subnormal values: Markstein for every element, no branch
+        if (bf16_normal && __float_as_uint(r) >= 0x00800000u && __float_as_uint(r) < 0x7f800000u) {
+            // a bf16 row without zero or subnormal values: Markstein for every element, no branch
             for (int q = tid; q < K / 4; q += AQR_THREADS) {
                 const float4 g = __ldg(g4 + q);
                 float4 x = reinterpret_cast<float4 *>(s_row)[q];

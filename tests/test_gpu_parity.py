@@ -129,6 +129,11 @@ def _wide_rows(M, K, seed):
     (4, 4096, torch.bfloat16, True, "tiny"),
     (3, 24576, torch.bfloat16, True, "normal"),
     (5, 2560, torch.bfloat16, True, "span"),
+    # rows whose sum of squares / K lies exactly on, or just off, a float
+    # rounding boundary: the double-sum estimate cannot decide them, the
+    # exact windowed sum does
+    (4, 4096, torch.bfloat16, True, "midpoint"),
+    (4, 2048, torch.float32, True, "midpoint"),
 ])
 def test_quant_act(M, K, dtype, subln, kind):
     if kind == "outlier":
@@ -148,6 +153,16 @@ def test_quant_act(M, K, dtype, subln, kind):
         X[1, 0], X[1, 1] = 2.0 ** 10, -(2.0 ** -10)      # span 20
         X[2, 5] = 2.0 ** -130                            # a subnormal (bf16 keeps it)
         X[3] = X[3] * 2.0 ** 52                          # up to 2^60
+        X = X.to(dtype)
+    elif kind == "midpoint":
+        # sum x^2 = 64 + 2^-18 with K = 2^12 (or 2^11): S / K = 2^-6 (1 + 2^-24)
+        # (or 2^-5 (1 + 2^-24)), halfway between two floats; then a row just
+        # above it, its negation, and a normal row
+        X = torch.zeros(M, K, dtype=torch.float32)
+        X[0, 0], X[0, 1] = 8.0, 2.0 ** -9
+        X[1, 0], X[1, 1], X[1, 2] = 8.0, 2.0 ** -9, 2.0 ** -30
+        X[2] = -X[0]
+        X[3] = workloads.normal((1, K), 1.0, 15)[0]
         X = X.to(dtype)
     else:  # rows below the 1e-5 floor, and an all-zero row
         X = (workloads.normal((M, K), 1.0, 12) * 1e-7).to(dtype)
