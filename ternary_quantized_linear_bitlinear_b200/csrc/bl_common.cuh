@@ -69,6 +69,42 @@ __device__ __forceinline__ u32 pack4_s8_rne(float a, float b, float c, float d, 
     return __byte_perm(__byte_perm(ra, rb, 0x0040u), __byte_perm(rc, rd, 0x0040u), 0x5410u);
 }
 
+// SubLN's f = float(double(S) / K) for S = sum x^2 from a double estimate.
+// The square of a float is exact in double and cannot over- or underflow
+// there; sq_abs_double gives |x| for the estimate (exact for normal x, below
+// 2^-125 for zero and subnormal x, so no per-element test).  An estimate
+// S_hat summed from those squares with at most K + 256 roundings of a
+// non-negative sum lies within beta * S_hat of their sum, beta = 2 (K + 256)
+// 2^-53, and their sum within K 2^-250 above S: S lies in
+// [S_hat (1 - beta) - K 2^-250, S_hat (1 + beta)].  f is monotone in S, so
+// when both ends give the same f it is f(S) bit for bit: returns true with
+// *f set.  False (the caller sums exactly) when they differ -- S / K within
+// about 10^-12 of a float rounding boundary -- or when amax_bits (max |x|
+// of the row as float bits) says the row holds inf / NaN.
+__device__ __forceinline__ double sq_abs_double(u32 bits) {
+    const u32 a = bits & 0x7fffffffu;
+    return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
+}
+
+__device__ __forceinline__ bool subln_mean_sq_from_estimate(double s_hat, int K, u32 amax_bits, float *f) {
+    if (amax_bits >= 0x7f800000u) return false;
+    const double beta = 2.0 * (double)(K + 256) * 0x1p-53;
+    const double A = (double)K * 0x1p-250;
+    double lo = __dsub_rd(__dmul_rd(s_hat, 1.0 - beta), A);
+    lo = lo > 0.0 ? lo : 0.0;
+    const double hi = __dmul_ru(s_hat, 1.0 + beta);
+    const float flo = __double2float_rn(__ddiv_rn(lo, (double)K));
+    const float fhi = __double2float_rn(__ddiv_rn(hi, (double)K));
+    *f = flo;
+    return flo == fhi;
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
+    return v;
+}
+
 // ---------------------------------------------------------------------------
 // Exact multi-limb fixed point (little-endian u64 limbs).
 

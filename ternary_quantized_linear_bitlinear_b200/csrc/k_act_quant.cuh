@@ -298,19 +298,36 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid
             }
         }
     };
-    // pass 1
+    // pass 1 (SubLN rows: also the double estimate of sum x^2)
     u32 amax = 0;
+    double dsq = 0.0;
     for (int ch = 0; ch < nch; ++ch) {
         load(ch);
 #pragma unroll
         for (int i = 0; i < AQS_V; ++i)
 #pragma unroll
-            for (int j = 0; j < EPV; ++j) amax = max(amax, aq_bits<BF16>(c[i], j) & 0x7fffffffu);
+            for (int j = 0; j < EPV; ++j) {
+                const u32 b = aq_bits<BF16>(c[i], j);
+                amax = max(amax, b & 0x7fffffffu);
+                if (g4 != nullptr) {
+                    const double xd = sq_abs_double(b);
+                    dsq = __fma_rn(xd, xd, dsq);
+                }
+            }
     }
     amax = warp_max_u32(amax);
     float r = 1.f;
+    float fest = 0.f;
+    bool decided = false;
     if (g4 != nullptr) {
-        // pass 2
+        dsq = warp_sum_f64(dsq);
+        decided = subln_mean_sq_from_estimate(dsq, K, amax, &fest);
+        decided = __shfl_sync(0xffffffffu, decided, 0);  // lane 0's sum decides (lanes may round differently)
+        fest = __shfl_sync(0xffffffffu, fest, 0);
+    }
+    if (g4 != nullptr && decided) r = __fsqrt_rn(__fadd_rn(fest, P.eps));
+    if (g4 != nullptr && !decided) {
+        // pass 2: exact, by windows
         u64 L[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
         int ehi = (int)(amax >> 23);
         if (ehi < 1) ehi = 1;
@@ -350,6 +367,8 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid
         if (lane == 0)
             r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(limbs_to_double_rn(L, -298), (double)K)), P.eps));
         r = __shfl_sync(0xffffffffu, r, 0);
+    }
+    if (g4 != nullptr) {
         // pass 3
         amax = 0;
         for (int ch = 0; ch < nch; ++ch) {
@@ -422,35 +441,15 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid
 // shared memory.  A warp per row left too few independent chains per SM to
 // hide the latency of the arithmetic.
 //
-// r needs f = float(double(S) / K) for the exact S = sum x^2.  The square of
-// a float (24-bit significand) is exact in double and no float's square
-// over- or underflows there, so pass 1 also sums the squares in double as
-// it loads the row: S_hat, within beta * S_hat of the sum of the squares it
-// was given (beta = 2 (K + 256) 2^-53 covers every rounding of the
-// non-negative sum: at most K + 256 additions on any path), which are the
-// exact squares except that zero and subnormal x enter as values below
-// 2^-125, i.e. within A = K 2^-250 above S.  Hence S lies in
-// [S_hat (1 - beta) - A, S_hat (1 + beta)]; f is monotone in S, so when both
-// ends give the same f that is f(S), bit for bit.  Rows where they differ
-// (S / K within about 10^-12 of a float rounding boundary) or with inf /
-// NaN sum the squares exactly by windows over the cached row, as
+// r needs f = float(double(S) / K) for the exact S = sum x^2: pass 1 also
+// sums the squares in double as it loads the row (sq_abs_double), and
+// subln_mean_sq_from_estimate decides f from that estimate for all but rows
+// within about 10^-12 of a float rounding boundary or with inf / NaN, which
+// sum the squares exactly by windows over the cached row, as
 // k_act_quant_subln does.
 constexpr int AQR_THREADS = 128;
 constexpr int AQR_WARPS = AQR_THREADS / 32;
 constexpr int AQR_MAX_K = 24 * 1024;  // rows cached per CTA: K * 4 bytes of dynamic shared memory
-
-// |x| of a float's bits as a double: exponent rebiased, mantissa moved;
-// exact for normal x, below 2^-125 for zero and subnormal x.
-__device__ __forceinline__ double aqr_abs_double(u32 b) {
-    const u32 a = b & 0x7fffffffu;
-    return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
-}
-
-__device__ __forceinline__ double warp_sum_f64(double v) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, off));
-    return v;
-}
 
 __device__ __forceinline__ u32 aqr_block_max(u32 v, u32 *s_u) {
     v = warp_max_u32(v);
@@ -517,7 +516,7 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
                 const u32 b = aq_bits<BF16>(c[i], j);
                 amax = max(amax, b & 0x7fffffffu);
                 if (sub) {
-                    const double xd = aqr_abs_double(b);
+                    const double xd = sq_abs_double(b);
                     dsq = __fma_rn(xd, xd, dsq);
                 }
                 f[j] = __uint_as_float(b);
@@ -542,21 +541,10 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
         if (tid == 0) {
             double sh = s_d[0];
             for (int w = 1; w < AQR_WARPS; ++w) sh = __dadd_rn(sh, s_d[w]);
-            int exact = 1;
-            if (amax < 0x7f800000u) {
-                const double beta = 2.0 * (double)(K + 256) * 0x1p-53;
-                const double A = (double)K * 0x1p-250;
-                double lo = __dsub_rd(__dmul_rd(sh, 1.0 - beta), A);
-                lo = lo > 0.0 ? lo : 0.0;
-                const double hi = __dmul_ru(sh, 1.0 + beta);
-                const float flo = __double2float_rn(__ddiv_rn(lo, (double)K));
-                const float fhi = __double2float_rn(__ddiv_rn(hi, (double)K));
-                if (flo == fhi) {
-                    s_f = flo;
-                    exact = 0;
-                }
-            }
-            s_exact = exact;
+            float f;
+            const bool ok = subln_mean_sq_from_estimate(sh, K, amax, &f);
+            s_f = f;
+            s_exact = ok ? 0 : 1;
         }
         __syncthreads();
         if (!s_exact) {

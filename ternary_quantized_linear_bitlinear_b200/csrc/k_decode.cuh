@@ -228,20 +228,37 @@ __device__ float dec_quant_row(const DecSlot &pr, int m, int K, int RS, uint8_t 
     uint4 c[DEC_QV];
     dec_load_block(c, xr, nvec, 0, lane);
     u32 amax = 0;
+    double dsq = 0.0;  // SubLN rows: the double estimate of sum x^2
     for (int blk = 0; blk < nblk; ++blk) {
         if (blk > 0) dec_load_block(c, xr, nvec, blk, lane);
 #pragma unroll
         for (int i = 0; i < DEC_QV; ++i)
 #pragma unroll
-            for (int j = 0; j < EPV; ++j) amax = max(amax, dec_x_bits<BF16>(c[i], j) & 0x7fffffffu);
+            for (int j = 0; j < EPV; ++j) {
+                const u32 b = dec_x_bits<BF16>(c[i], j);
+                amax = max(amax, b & 0x7fffffffu);
+                if (g4 != nullptr) {
+                    const double xd = sq_abs_double(b);
+                    dsq = __fma_rn(xd, xd, dsq);
+                }
+            }
     }
     amax = warp_max_u32(amax);
     float r = 1.f;
     if (g4 != nullptr) {
-        if (nblk > 1) dec_load_block(c, xr, nvec, 0, lane);
-        const double S2 = dec_row_sumsq<BF16>(c, xr, nvec, lane, amax);
-        if (lane == 0) r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(S2, (double)K)), eps));
-        r = __shfl_sync(0xffffffffu, r, 0);
+        dsq = warp_sum_f64(dsq);
+        float f;
+        bool decided = subln_mean_sq_from_estimate(dsq, K, amax, &f);
+        decided = __shfl_sync(0xffffffffu, decided, 0);  // lane 0's sum decides (lanes may round differently)
+        f = __shfl_sync(0xffffffffu, f, 0);
+        if (decided) {
+            r = __fsqrt_rn(__fadd_rn(f, eps));
+        } else {
+            if (nblk > 1) dec_load_block(c, xr, nvec, 0, lane);
+            const double S2 = dec_row_sumsq<BF16>(c, xr, nvec, lane, amax);
+            if (lane == 0) r = __fsqrt_rn(__fadd_rn(__double2float_rn(__ddiv_rn(S2, (double)K)), eps));
+            r = __shfl_sync(0xffffffffu, r, 0);
+        }
         amax = 0;
         for (int blk = 0; blk < nblk; ++blk) {
             if (nblk > 1) dec_load_block(c, xr, nvec, blk, lane);

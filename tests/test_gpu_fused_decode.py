@@ -40,6 +40,16 @@ def _inputs(M, K, dtype, kind, seed):
         if dtype == torch.float32:
             X[0, :8] = torch.tensor([1e-40, -3e-39, 2e-45, 0.0, 5e-41, -1e-44, 7e-39, 1e-38])
         return X
+    if kind == "midpoint":
+        # sum x^2 / K exactly halfway between two floats (K a power of two),
+        # a row just above it, its negation and a normal row: the double
+        # estimate of sum x^2 cannot decide the first and third, the exact sum does
+        X = torch.zeros(M, K, dtype=torch.float32)
+        X[0, 0], X[0, 1] = 8.0, 2.0 ** -9
+        X[1, 0], X[1, 1], X[1, 2] = 8.0, 2.0 ** -9, 2.0 ** -30
+        X[2] = -X[0]
+        X[3] = workloads.normal((1, K), 1.0, seed)[0]
+        return X.to(dtype)
     return workloads.normal((M, K), 1.0, seed, dtype)
 
 
@@ -79,6 +89,8 @@ def run_fused(items, M, dtype, eps=1e-6, outputs=True, flags=0):
     (2, 50, 1024, torch.float32, False, "wide"),
     (1, 40, 4096, torch.bfloat16, False, "outlier"),
     (2, 33, 192, torch.float32, False, "tiny"),
+    (4, 64, 4096, torch.bfloat16, True, "midpoint"),
+    (4, 64, 2048, torch.float32, True, "midpoint"),
 ])
 def test_fused_decode_matches_oracle(M, N, K, dtype, subln, kind):
     W = workloads.normal((N, K), 0.02, 500 + K)

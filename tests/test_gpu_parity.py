@@ -134,6 +134,9 @@ def _wide_rows(M, K, seed):
     # exact windowed sum does
     (4, 4096, torch.bfloat16, True, "midpoint"),
     (4, 2048, torch.float32, True, "midpoint"),
+    # the same rows short enough for the warp-per-row SubLN quantizer
+    (4, 2048, torch.bfloat16, True, "midpoint"),
+    (4, 1024, torch.float32, True, "midpoint"),
 ])
 def test_quant_act(M, K, dtype, subln, kind):
     if kind == "outlier":
