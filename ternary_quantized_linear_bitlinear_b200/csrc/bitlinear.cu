@@ -134,7 +134,7 @@ bl_status quant_weights_impl(const DeviceInfo &d, const WqIn *in, int count, bl_
         if (nb < 1) nb = 1;
         mins += minb;
         P.j[i] = WqJob{reinterpret_cast<const uint4 *>(in[i].W), nvec, n, in[i].gamma,
-                       reinterpret_cast<u32 *>(in[i].packed), n / 16, (int)blocks, (int)nb, 0, 0};
+                       reinterpret_cast<u32 *>(in[i].packed), n / 16, (int)blocks, (int)nb, 0, 0, 0};
         blocks += nb;
         words += n / 16;
     }
@@ -152,6 +152,13 @@ bl_status quant_weights_impl(const DeviceInfo &d, const WqIn *in, int count, bl_
             blocks += nb;
         }
         if (blocks > WQ_MAX_BLOCKS) return BL_ERR_SHAPE;
+    }
+    // roundings a term of a matrix's double sum passes through: its thread's
+    // chain (half of its elements per accumulator) plus the reduction trees
+    for (int i = 0; i < count; ++i) {
+        const long long per = (long long)P.j[i].nblk * WQ_THREADS;
+        const long long vpt = (P.j[i].nvec + per - 1) / per;
+        P.j[i].depth = (int)(vpt * epv / 2 + 64 + (P.j[i].nblk + WQ_PACK_THREADS - 1) / WQ_PACK_THREADS);
     }
     const long long pcap = 8LL * d.sms;
     long long pblocks = 0;
@@ -181,7 +188,9 @@ bl_status quant_weights_impl(const DeviceInfo &d, const WqIn *in, int count, bl_
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cfg.gridDim = dim3((unsigned)count);
-    if (cudaLaunchKernelEx(&cfg, k_absmean_final, P) != cudaSuccess) return BL_ERR_CUDA;
+    if ((bf16 ? cudaLaunchKernelEx(&cfg, k_absmean_final<true>, P) : cudaLaunchKernelEx(&cfg, k_absmean_final<false>, P)) !=
+        cudaSuccess)
+        return BL_ERR_CUDA;
     cfg.gridDim = dim3((unsigned)pblocks);
     cudaError_t e = bf16 ? cudaLaunchKernelEx(&cfg, k_ternary_pack<true>, P)
                          : cudaLaunchKernelEx(&cfg, k_ternary_pack<false>, P);

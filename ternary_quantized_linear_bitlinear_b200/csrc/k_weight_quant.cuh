@@ -5,13 +5,10 @@
 // Three launches on the caller's stream, each over one or several weight
 // matrices (up to WQ_MAX_JOBS: e.g. the projections of a layer, so their
 // reduction latency chains overlap), chained as programmatic dependents:
-//   k_absmean_partial  one pass over W: exact per-block sum of |w| as a
-//                      384-bit fixed-point integer in units of 2^-149,
-//                      written to the workspace
-//   k_absmean_final    one CTA per matrix: sums its block partials, rounds
-//                      once to double, gamma = float(S / n) + 1e-5f, and the
-//                      float threshold T with
-//                        |w| >= T  <=>  float(|w|/gamma) > 0.5
+//   k_absmean_partial  one pass over W: each block's sum of |w| in double
+//   k_absmean_final    one CTA per matrix: gamma = float(double(S) / n) +
+//                      1e-5f for the exact S = sum |w| and the float
+//                      threshold T with |w| >= T <=> float(|w|/gamma) > 0.5
 //   k_ternary_pack     second pass over W (its first words requested before
 //                      the wait for T): W_q = sign(w) * (|w| >= T), stored
 //                      as the code 1 - W_q, four codes per byte in the
@@ -20,13 +17,23 @@
 // workspace needs clearing: every word a launch reads there was written by
 // the launch before it.
 //
-// Exactness: every finite float is an integer multiple of 2^-149, so sum|w|
-// is an integer in those units.  Each thread accumulates m << (e - base) in a
-// 64-bit register for exponents inside a 26-binade window chosen per block
-// from a sample of its data (term < 2^49, at most 2^14 terms per thread).
-// Anything outside the window (tiny, huge or subnormal values) is added
-// exactly into per-block shared-memory bins indexed by exponent.  The result
-// does not depend on the window, the grid or the order of the additions.
+// gamma from a double estimate.  A float is exact in double, so the sum of
+// |w| in double, S_hat, is within beta * S_hat of the sum of its terms when
+// no term passes through more than D roundings on its way to the total
+// (beta = 2 D 2^-53 for a non-negative sum; D is the longest chain of a
+// thread plus the reduction tree, counted on the host).  The terms are the
+// exact |w| except that zero and subnormal w enter as values below 2^-126
+// (no per-element test), i.e. within A = n 2^-126 above S.  gamma is
+// monotone in S, so when both ends of [S_hat (1 - beta) - A, S_hat (1 + beta)]
+// give the same gamma that is gamma(S), bit for bit (tiny sums, e.g. an
+// all-zero matrix, give 1e-5f at both ends).  Otherwise -- the mean within
+// about 10^-14 of a float rounding boundary, or S_hat >= 2^127 (inf / NaN
+// weights) -- the final CTA sums |w| exactly: every finite float is an
+// integer multiple of 2^-149, so S is an integer in those units; each thread
+// adds m << (e - base) for exponents in a 26-binade window chosen from a
+// sample of the matrix into 128 bits, anything outside the window into exact
+// shared-memory bins by exponent, and the block folds it all into 384-bit
+// limbs, rounded once to double.
 #pragma once
 
 #include "bl_common.cuh"
@@ -35,8 +42,8 @@ namespace bl {
 
 constexpr int WQ_THREADS = 512;
 constexpr int WQ_PACK_THREADS = 256;
-constexpr int WQ_WINDOW = 25;       // fast path: base <= e <= base + 25
-constexpr int WQ_PART_LIMBS = 6;    // per-block partial, 384 bits
+constexpr int WQ_WINDOW = 25;       // exact sum: base <= e <= base + 25
+constexpr int WQ_PART_LIMBS = 6;    // workspace words per reduction block (one double used)
 constexpr int WQ_MAX_BLOCKS = 1024; // over all matrices of a launch
 constexpr int WQ_MAX_JOBS = 8;      // weight matrices per launch
 constexpr size_t WQ_WS_PARTIALS = (size_t)WQ_MAX_BLOCKS * WQ_PART_LIMBS * 8;
@@ -45,7 +52,8 @@ constexpr size_t WQ_WS_BYTES = WQ_WS_PARTIALS + 256;  // + threshold words
 // One weight matrix of a (grouped) quantization launch: blocks
 // [blk0, blk0 + nblk) of the reduction grid sum it, block j of the final
 // grid derives its gamma and T, blocks [pblk0, pblk0 + pnblk) of the pack
-// grid pack it.
+// grid pack it.  depth bounds the roundings any term of its double sum
+// passes through.
 struct WqJob {
     const uint4 *W;
     long long nvec;   // 16-byte vectors
@@ -57,12 +65,13 @@ struct WqJob {
     int nblk;
     int pblk0;
     int pnblk;
+    int depth;
 };
 
 struct WqParams {
     WqJob j[WQ_MAX_JOBS];
     int count;
-    u64 *partials;    // [WQ_MAX_BLOCKS][WQ_PART_LIMBS]
+    u64 *partials;    // [WQ_MAX_BLOCKS][WQ_PART_LIMBS]: word 0 of a block holds its double sum
     u32 *thresh;      // [WQ_MAX_JOBS] float bits of T
 };
 
@@ -78,113 +87,46 @@ __device__ __forceinline__ u32 vec_elem_bits(const uint4 &v, int j) {
     }
 }
 
-// Sums a matrix's block partials (one limb position per pass, 128 bits per
-// limb across the block), rounds the total to double and derives gamma and
-// T.  Whole block of NT threads; every thread returns with s_out[0] = gamma
-// bits and s_out[1] = T bits.
-template <int NT>
-__device__ void wq_gamma_threshold(const u64 *partials, int nblocks, long long n, u32 *s_out) {
-    constexpr int NL = WQ_PART_LIMBS;
-    constexpr int NW = NT / 32;
-    __shared__ u64 f_lo[NL][NW], f_hi[NL][NW];
-    __shared__ u64 f_sum[NL][2];
-    const int tid = threadIdx.x;
-    u64 slo[NL], shi[NL];
-#pragma unroll
-    for (int k = 0; k < NL; ++k) slo[k] = shi[k] = 0ull;
-    for (int b = tid; b < nblocks; b += NT) {
-#pragma unroll
-        for (int k = 0; k < NL; ++k) {
-            // written by the reduction grid: bypass L1
-            const u64 v = __ldcg(partials + (size_t)b * NL + k);
-            const u64 t = slo[k] + v;
-            shi[k] += t < v ? 1ull : 0ull;
-            slo[k] = t;
-        }
-    }
-#pragma unroll
-    for (int k = 0; k < NL; ++k) {
-        warp_sum_u128(slo[k], shi[k]);
-        if ((tid & 31) == 0) {
-            f_lo[k][tid >> 5] = slo[k];
-            f_hi[k][tid >> 5] = shi[k];
-        }
-    }
-    __syncthreads();
-    // limb position k summed over the warps by lane k of warp 0 (128 bits:
-    // a thread adds at most four 64-bit limbs, the block's sum is below 2^74)
-    if (tid < NL) {
-        u64 lo = 0ull, hi = 0ull;
-#pragma unroll
-        for (int w = 0; w < NW; ++w) {
-            const u64 t = lo + f_lo[tid][w];
-            hi += f_hi[tid][w] + (t < lo ? 1ull : 0ull);
-            lo = t;
-        }
-        f_sum[tid][0] = lo;
-        f_sum[tid][1] = hi;
-    }
-    __syncwarp();
-    if (tid == 0) {
-        // S = sum_k (hi:lo)_k << 64k, folded into NL + 2 limbs
-        u64 L[NL + 2];
-#pragma unroll
-        for (int k = 0; k < NL + 2; ++k) L[k] = 0ull;
-#pragma unroll
-        for (int k = 0; k < NL; ++k) limbs_add_u128_shl(L, f_sum[k][0], f_sum[k][1], 64 * k);
-        double S = limbs_to_double_rn(L, -149);
-        float mean = __double2float_rn(__ddiv_rn(S, (double)n));
-        float g = __fadd_rn(mean, 1e-5f);
-        // smallest t with float(t / g) > 0.5: start at g/2 (exact, quotient 0.5)
-        float t = __fmul_rn(0.5f, g);
-        for (int it = 0; it < 64 && !(__fdiv_rn(t, g) > 0.5f); ++it)
-            t = __uint_as_float(__float_as_uint(t) + 1u);
-        s_out[0] = __float_as_uint(g);
-        s_out[1] = __float_as_uint(t);
-    }
-    __syncthreads();
+// |w| of a float's bits as a double: exponent rebiased, mantissa moved;
+// exact for normal w, in [2^-127, 2^-126) for zero and subnormal w.
+__device__ __forceinline__ double wq_abs_double(u32 bits) {
+    const u32 a = bits & 0x7fffffffu;
+    return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
 }
 
-template <bool BF16>
-__global__ void __launch_bounds__(WQ_THREADS, 2) k_absmean_partial(const __grid_constant__ WqParams P) {
-    // the pack kernel may start loading W while this grid runs
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    constexpr int EPV = BF16 ? 8 : 4;  // elements per 16-byte vector
+// gamma = float(S / n) + 1e-5f (S already rounded to double) and the
+// smallest float t with float(t / gamma) > 0.5.
+__device__ __forceinline__ void wq_gamma_threshold_of(double S, long long n, float *g_out, u32 *t_out) {
+    const float mean = __double2float_rn(__ddiv_rn(S, (double)n));
+    const float g = __fadd_rn(mean, 1e-5f);
+    // start at g/2 (exact, quotient 0.5)
+    float t = __fmul_rn(0.5f, g);
+    for (int it = 0; it < 64 && !(__fdiv_rn(t, g) > 0.5f); ++it) t = __uint_as_float(__float_as_uint(t) + 1u);
+    *g_out = g;
+    *t_out = __float_as_uint(t);
+}
+
+// Exact sum of |w| over vectors first, first + stride, ... < nvec by the
+// whole block (NT threads), as 384-bit limbs in units of 2^-149 in thread 0.
+template <bool BF16, int NT>
+__device__ void wq_exact_block_sum(const uint4 *__restrict__ W, long long first, long long stride, long long nvec,
+                                   u64 (&L)[WQ_PART_LIMBS]) {
+    constexpr int EPV = BF16 ? 8 : 4;
     __shared__ u64 s_bins[256];
     __shared__ u32 s_emax;
-    __shared__ u64 s_wlo[WQ_THREADS / 32], s_whi[WQ_THREADS / 32];
-
-    // the matrix this block sums
-    int ji = 0;
-    while (ji + 1 < P.count && (int)blockIdx.x >= P.j[ji + 1].blk0) ++ji;
-    const WqJob &job = P.j[ji];
-    const uint4 *__restrict__ W = job.W;
-    const long long nvec = job.nvec;
-
+    __shared__ u64 s_wlo[NT / 32], s_whi[NT / 32];
     const int tid = threadIdx.x;
-    for (int i = tid; i < 256; i += WQ_THREADS) s_bins[i] = 0ull;
+    for (int i = tid; i < 256; i += NT) s_bins[i] = 0ull;
     if (tid == 0) s_emax = 0;
-
-    const long long stride = (long long)job.nblk * WQ_THREADS;
-    const long long first = (long long)((int)blockIdx.x - job.blk0) * WQ_THREADS + tid;
-
-    // Window from a sample: the block's first vector per thread.  The next
-    // four vectors are requested before the block reduction, so their
-    // latency overlaps it.
+    // window from a sample: the first vector per thread
     u32 emax = 0;
-    uint4 v0 = make_uint4(0, 0, 0, 0);
     if (first < nvec) {
-        v0 = ldg_stream_v4(W + first);
-    }
-    uint4 a[4];
-    long long i = first + stride;
+        const uint4 v = ldg_stream_v4(W + first);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-        a[q] = i + q * stride < nvec ? ldg_stream_v4(W + i + q * stride) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-    for (int j = 0; j < EPV; ++j) {
-        u32 e = (vec_elem_bits<BF16>(v0, j) & 0x7fffffffu) >> 23;
-        emax = e > emax ? e : emax;
+        for (int j = 0; j < EPV; ++j) {
+            const u32 e = (vec_elem_bits<BF16>(v, j) & 0x7fffffffu) >> 23;
+            emax = e > emax ? e : emax;
+        }
     }
     emax = warp_max_u32(emax);
     __syncthreads();
@@ -194,26 +136,69 @@ __global__ void __launch_bounds__(WQ_THREADS, 2) k_absmean_partial(const __grid_
     if (top > 254) top = 254;
     int base = top - WQ_WINDOW;
     if (base < 1) base = 1;
-
-    u64 acc = 0ull;
-    auto add_vec = [&](const uint4 &v) {
+    // 128-bit per-thread sum of m << (e - base) (< 2^49 per term)
+    u64 lo = 0ull, hi = 0ull;
+    for (long long i = first; i < nvec; i += stride) {
+        const uint4 v = ldg_stream_v4(W + i);
 #pragma unroll
         for (int j = 0; j < EPV; ++j) {
-            u32 u = vec_elem_bits<BF16>(v, j) & 0x7fffffffu;
-            u32 e = u >> 23;
-            u32 m = (u & 0x7fffffu) | 0x800000u;
-            u32 d = e - (u32)base;
+            const u32 u = vec_elem_bits<BF16>(v, j) & 0x7fffffffu;
+            const u32 e = u >> 23;
+            const u32 m = (u & 0x7fffffu) | 0x800000u;
+            const u32 d = e - (u32)base;
             if (d <= (u32)WQ_WINDOW) {
-                acc = mad_wide_u32(m, 1u << d, acc);
+                const u64 t = (u64)m << d;
+                const u64 s2 = lo + t;
+                hi += s2 < lo ? 1ull : 0ull;
+                lo = s2;
             } else if (u != 0u) {
                 atomicAdd(&s_bins[e], (u64)(e ? m : (u & 0x7fffffu)));
             }
         }
+    }
+    warp_sum_u128(lo, hi);
+    if ((tid & 31) == 0) {
+        s_wlo[tid >> 5] = lo;
+        s_whi[tid >> 5] = hi;
+    }
+    __syncthreads();
+    if (tid == 0) {
+#pragma unroll
+        for (int k = 0; k < WQ_PART_LIMBS; ++k) L[k] = 0ull;
+        for (int w = 0; w < NT / 32; ++w) limbs_add_u128_shl(L, s_wlo[w], s_whi[w], base - 1);
+        // term m << (e - base) stands for m * 2^(e - 150) = term * 2^(base - 1) units
+        for (int e = 0; e < 256; ++e)
+            if (s_bins[e] != 0ull) limbs_add_u128_shl(L, s_bins[e], 0ull, e > 0 ? e - 1 : 0);
+    }
+}
+
+template <bool BF16>
+__global__ void __launch_bounds__(WQ_THREADS, 2) k_absmean_partial(const __grid_constant__ WqParams P) {
+    // the next grids may start now (the final grid waits for this one)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    constexpr int EPV = BF16 ? 8 : 4;
+    __shared__ double s_d[WQ_THREADS / 32];
+    int ji = 0;
+    while (ji + 1 < P.count && (int)blockIdx.x >= P.j[ji + 1].blk0) ++ji;
+    const WqJob &job = P.j[ji];
+    const uint4 *__restrict__ W = job.W;
+    const long long nvec = job.nvec;
+    const int tid = threadIdx.x;
+    const long long stride = (long long)job.nblk * WQ_THREADS;
+    long long i = (long long)((int)blockIdx.x - job.blk0) * WQ_THREADS + tid;
+    // two accumulators (even / odd elements of a vector), four vectors in
+    // flight while four are summed
+    double d0 = 0.0, d1 = 0.0;
+    auto add_vec = [&](const uint4 &v) {
+#pragma unroll
+        for (int j = 0; j < EPV; j += 2) {
+            d0 = __dadd_rn(d0, wq_abs_double(vec_elem_bits<BF16>(v, j)));
+            d1 = __dadd_rn(d1, wq_abs_double(vec_elem_bits<BF16>(v, j + 1)));
+        }
     };
-    add_vec(v0);  // zero when first >= nvec
-    // Two stages of four vectors: the next four are in flight while the
-    // current four are summed.  a[] holds vectors i + q * stride (zero where
-    // past the end; zeros add nothing).
+    uint4 a[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) a[q] = i + q * stride < nvec ? ldg_stream_v4(W + i + q * stride) : make_uint4(0, 0, 0, 0);
     while (i + 4 * stride < nvec) {
         const long long inext = i + 4 * stride;
         uint4 b[4];
@@ -226,61 +211,82 @@ __global__ void __launch_bounds__(WQ_THREADS, 2) k_absmean_partial(const __grid_
         for (int q = 0; q < 4; ++q) a[q] = b[q];
         i = inext;
     }
+    // the last vectors (zeros past the end: 2^-127 each, inside the bound)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) add_vec(a[q]);
-
-    // Block sum of the 64-bit window accumulators as 128 bits.
-    u64 lo = acc, hi = 0ull;
-    warp_sum_u128(lo, hi);
-    if ((tid & 31) == 0) {
-        s_wlo[tid >> 5] = lo;
-        s_whi[tid >> 5] = hi;
-    }
+    for (int q = 0; q < 4; ++q)
+        if (i + q * stride < nvec) add_vec(a[q]);
+    double d = warp_sum_f64(__dadd_rn(d0, d1));
+    if ((tid & 31) == 0) s_d[tid >> 5] = d;
     __syncthreads();
-    if (tid < 32) {
-        // warp 0: which exponent bins are non-empty (usually none)
-        u32 nz[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) nz[q] = __ballot_sync(0xffffffffu, s_bins[q * 32 + tid] != 0ull);
-        if (tid == 0) {
-            u64 L[WQ_PART_LIMBS] = {0, 0, 0, 0, 0, 0};
-            u64 blo = 0, bhi = 0;
-            for (int w = 0; w < WQ_THREADS / 32; ++w) {
-                u64 sl = blo + s_wlo[w];
-                bhi += s_whi[w] + (sl < blo ? 1ull : 0ull);
-                blo = sl;
-            }
-            // term m << (e - base) stands for m * 2^(e - 150) = term * 2^(base - 1) units
-            limbs_add_u128_shl(L, blo, bhi, base - 1);
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                u32 bits = nz[q];
-                while (bits) {
-                    const int e = q * 32 + __ffs(bits) - 1;
-                    bits &= bits - 1;
-                    limbs_add_u128_shl(L, s_bins[e], 0ull, e > 0 ? e - 1 : 0);
-                }
-            }
-            // read by the pack grid after its griddepcontrol.wait (which
-            // returns once this grid has completed and its writes are visible)
-#pragma unroll
-            for (int k = 0; k < WQ_PART_LIMBS; ++k) P.partials[(size_t)blockIdx.x * WQ_PART_LIMBS + k] = L[k];
-        }
+    if (tid == 0) {
+        double t = s_d[0];
+        for (int w = 1; w < WQ_THREADS / 32; ++w) t = __dadd_rn(t, s_d[w]);
+        // read by the final grid after its griddepcontrol.wait
+        P.partials[(size_t)blockIdx.x * WQ_PART_LIMBS] = (u64)__double_as_longlong(t);
     }
 }
 
-// Block j derives gamma and T of matrix j from its reduction blocks'
-// partials (read after the reduction grid has completed).
+// Block j derives gamma and T of matrix j: from the reduction blocks'
+// double sums when their bound decides gamma, else from the exact sum
+// (read after the reduction grid has completed).
+template <bool BF16>
 __global__ void __launch_bounds__(WQ_PACK_THREADS) k_absmean_final(const __grid_constant__ WqParams P) {
     // the pack grid may start loading W now
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    __shared__ u32 s_gt[2];
+    __shared__ double s_d[WQ_PACK_THREADS / 32];
+    __shared__ int s_decided;
+    __shared__ float s_g;
+    __shared__ u32 s_t;
     const WqJob &jb = P.j[blockIdx.x];
+    const int tid = threadIdx.x;
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    wq_gamma_threshold<WQ_PACK_THREADS>(P.partials + (size_t)jb.blk0 * WQ_PART_LIMBS, jb.nblk, jb.n, s_gt);
-    if (threadIdx.x == 0) {
-        jb.gamma[0] = __uint_as_float(s_gt[0]);
-        P.thresh[blockIdx.x] = s_gt[1];
+    double d = 0.0;
+    for (int b = tid; b < jb.nblk; b += WQ_PACK_THREADS)
+        d = __dadd_rn(d, __longlong_as_double((long long)__ldcg(P.partials + (size_t)(jb.blk0 + b) * WQ_PART_LIMBS)));
+    d = warp_sum_f64(d);
+    if ((tid & 31) == 0) s_d[tid >> 5] = d;
+    __syncthreads();
+    if (tid == 0) {
+        double sh = s_d[0];
+        for (int w = 1; w < WQ_PACK_THREADS / 32; ++w) sh = __dadd_rn(sh, s_d[w]);
+        int decided = 0;
+        if (sh < 0x1p127) {
+            const double beta = 2.0 * (double)jb.depth * 0x1p-53;
+            const double A = (double)jb.n * 0x1p-126;
+            double lo = __dsub_rd(__dmul_rd(sh, 1.0 - beta), A);
+            lo = lo > 0.0 ? lo : 0.0;
+            const double hi = __dmul_ru(sh, 1.0 + beta);
+            float glo, ghi;
+            u32 tlo, thi;
+            wq_gamma_threshold_of(lo, jb.n, &glo, &tlo);
+            wq_gamma_threshold_of(hi, jb.n, &ghi, &thi);
+            if (__float_as_uint(glo) == __float_as_uint(ghi)) {
+                s_g = glo;
+                s_t = tlo;
+                decided = 1;
+            }
+        }
+        s_decided = decided;
+    }
+    __syncthreads();
+    if (!s_decided) {
+        u64 L[WQ_PART_LIMBS];
+        wq_exact_block_sum<BF16, WQ_PACK_THREADS>(jb.W, tid, WQ_PACK_THREADS, jb.nvec, L);
+        if (tid == 0) {
+            u64 L2[WQ_PART_LIMBS + 2];
+#pragma unroll
+            for (int k = 0; k < WQ_PART_LIMBS; ++k) L2[k] = L[k];
+            L2[WQ_PART_LIMBS] = L2[WQ_PART_LIMBS + 1] = 0ull;
+            float g;
+            u32 t;
+            wq_gamma_threshold_of(limbs_to_double_rn(L2, -149), jb.n, &g, &t);
+            s_g = g;
+            s_t = t;
+        }
+    }
+    if (tid == 0) {
+        jb.gamma[0] = s_g;
+        P.thresh[blockIdx.x] = s_t;
     }
 }
 

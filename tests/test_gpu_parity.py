@@ -47,6 +47,11 @@ def chain(W_cpu, X_cpu, gain_cpu=None, eps=1e-6, want_acc=True):
     (64, 1024, torch.bfloat16, "wide"),
     (48, 512, torch.bfloat16, "zeros"),
     (512, 2048, torch.bfloat16, "outliers"),
+    # sum |W| / n exactly halfway between two floats: the double estimate
+    # cannot decide gamma, the exact sum in the final block does
+    (1, 64, torch.bfloat16, "midpoint"),
+    (4, 64, torch.float32, "midpoint"),
+    (64, 4096, torch.bfloat16, "midpoint"),
 ])
 def test_quant_weights(N, K, dtype, kind):
     if kind == "normal":
@@ -63,6 +68,16 @@ def test_quant_weights(N, K, dtype, kind):
         W = W.to(dtype)
     elif kind == "zeros":
         W = torch.zeros(N, K, dtype=dtype)
+    elif kind == "midpoint":
+        # n / 2 - 1 entries of 2, one of 1, one of -1 and one of -2^-24 n, the
+        # rest zero: sum |W| = n (1 + 2^-24)
+        n = N * K
+        W = torch.zeros(n, dtype=torch.float32)
+        W[: n // 2 - 1] = 2.0
+        W[n // 2 - 1] = 1.0
+        W[n // 2] = -1.0
+        W[n // 2 + 1] = -(2.0 ** -24) * n
+        W = W.reshape(N, K).to(dtype)
     elif kind == "outliers":
         # a few values outside the summing window of their block (tiny, a
         # subnormal, huge) among normal ones: only the threads that meet
