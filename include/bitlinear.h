@@ -132,8 +132,9 @@ bl_status bl_quant_weights_noalloc(const void *W, bl_dtype wdt, int64_t N, int64
                                    uint8_t *packed, float *gamma, bl_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
-/* Step 1 for several weight matrices in two launches (one reduction grid    */
-/* and one pack grid over all of them), e.g. the projections of a layer      */
+/* Step 1 for several weight matrices in three launches (one reduction     */
+/* grid, one finalize grid of a block per matrix and one pack grid over all  */
+/* of them), e.g. the projections of a layer                                 */
 /* that are re-quantized every call: their reduction latency chains overlap  */
 /* instead of running one after the other.  Same definition and the same    */
 /* bits as bl_quant_weights for each matrix.                                 */

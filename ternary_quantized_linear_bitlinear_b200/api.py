@@ -242,7 +242,7 @@ def bl_quant_weights_noalloc(W: torch.Tensor, packed=None, gamma=None, stream=No
 
 
 def bl_quant_weights_grouped(Ws, packed=None, gammas=None, workspace=None, stream=None):
-    """Several weight matrices (same dtype) in two launches -> ([packed], [gamma]),
+    """Several weight matrices (same dtype) in three launches -> ([packed], [gamma]),
     each as bl_quant_weights(W) would give it."""
     Ws = list(Ws)
     if not 1 <= len(Ws) <= 8:
