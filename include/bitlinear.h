@@ -132,12 +132,12 @@ bl_status bl_quant_weights_noalloc(const void *W, bl_dtype wdt, int64_t N, int64
                                    uint8_t *packed, float *gamma, bl_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
-/* Step 1 for several weight matrices in three launches (one reduction     */
+/* Step 1 for several weight matrices in three launches (one reduction      */
 /* grid, one finalize grid of a block per matrix and one pack grid over all  */
-/* of them), e.g. the projections of a layer                                 */
-/* that are re-quantized every call: their reduction latency chains overlap  */
-/* instead of running one after the other.  Same definition and the same    */
-/* bits as bl_quant_weights for each matrix.                                 */
+/* of them), e.g. the projections of a layer that are re-quantized every     */
+/* call: their reduction latency chains overlap instead of running one       */
+/* after the other.  Same definition and the same bits as bl_quant_weights   */
+/* for each matrix.                                                          */
 /*                                                                           */
 /* problems  HOST array of `count` (1 <= count <= BL_MAX_WQ_GROUP) matrices, */
 /*           read during the call only; each W of dtype wdt, each with its    */
