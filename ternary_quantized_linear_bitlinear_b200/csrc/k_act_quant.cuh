@@ -144,7 +144,7 @@ __global__ void __launch_bounds__(1024, 1) k_act_quant(const __grid_constant__ A
 
 // One warp per row: VPL 16-byte vectors per lane, the row in registers,
 // reductions by warp shuffles -- no block barrier at all.
-constexpr int AQW_WARPS = 8;
+constexpr int AQW_WARPS = 4;
 
 // Per-half unsigned max of two 16-bit lanes.
 __device__ __forceinline__ u32 vmax_u16x2(u32 a, u32 b) {
