@@ -69,10 +69,18 @@ __device__ __forceinline__ u32 pack4_s8_rne(float a, float b, float c, float d, 
     return __byte_perm(__byte_perm(ra, rb, 0x0040u), __byte_perm(rc, rd, 0x0040u), 0x5410u);
 }
 
+// |x| of a float's bits as a double: exponent rebiased, mantissa moved;
+// exact for normal x, in [2^-127, 2^-126) for zero and subnormal x (also the
+// weight absmean's terms).
+__device__ __forceinline__ double abs_as_double(u32 bits) {
+    const u32 a = bits & 0x7fffffffu;
+    return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
+}
+
 // SubLN's f = float(double(S) / K) for S = sum x^2 from a double estimate.
 // The square of a float is exact in double and cannot over- or underflow
-// there; sq_abs_double gives |x| for the estimate (exact for normal x, below
-// 2^-125 for zero and subnormal x, so no per-element test).  An estimate
+// there; abs_as_double gives |x| for the estimate (exact for normal x, below
+// 2^-126 for zero and subnormal x, so no per-element test).  An estimate
 // S_hat summed from those squares with at most K + 256 roundings of a
 // non-negative sum lies within beta * S_hat of their sum, beta = 2 (K + 256)
 // 2^-53, and their sum within K 2^-250 above S: S lies in
@@ -81,11 +89,6 @@ __device__ __forceinline__ u32 pack4_s8_rne(float a, float b, float c, float d, 
 // *f set.  False (the caller sums exactly) when they differ -- S / K within
 // about 10^-12 of a float rounding boundary -- or when amax_bits (max |x|
 // of the row as float bits) says the row holds inf / NaN.
-__device__ __forceinline__ double sq_abs_double(u32 bits) {
-    const u32 a = bits & 0x7fffffffu;
-    return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
-}
-
 __device__ __forceinline__ bool subln_mean_sq_from_estimate(double s_hat, int K, u32 amax_bits, float *f) {
     if (amax_bits >= 0x7f800000u) return false;
     const double beta = 2.0 * (double)(K + 256) * 0x1p-53;

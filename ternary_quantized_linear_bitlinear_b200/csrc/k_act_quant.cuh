@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid
                 const u32 b = aq_bits<BF16>(c[i], j);
                 amax = max(amax, b & 0x7fffffffu);
                 if (g4 != nullptr) {
-                    const double xd = sq_abs_double(b);
+                    const double xd = abs_as_double(b);
                     dsq = __fma_rn(xd, xd, dsq);
                 }
             }
@@ -442,7 +442,7 @@ __global__ void __launch_bounds__(AQW_WARPS * 32) k_act_quant_subln(const __grid
 // hide the latency of the arithmetic.
 //
 // r needs f = float(double(S) / K) for the exact S = sum x^2: pass 1 also
-// sums the squares in double as it loads the row (sq_abs_double), and
+// sums the squares in double as it loads the row (abs_as_double), and
 // subln_mean_sq_from_estimate decides f from that estimate for all but rows
 // within about 10^-12 of a float rounding boundary or with inf / NaN, which
 // sum the squares exactly by windows over the cached row, as
@@ -516,7 +516,7 @@ __global__ void __launch_bounds__(AQR_THREADS, 8) k_act_quant_subln_row(const __
                 const u32 b = aq_bits<BF16>(c[i], j);
                 amax = max(amax, b & 0x7fffffffu);
                 if (sub) {
-                    const double xd = sq_abs_double(b);
+                    const double xd = abs_as_double(b);
                     dsq = __fma_rn(xd, xd, dsq);
                 }
                 f[j] = __uint_as_float(b);

@@ -238,7 +238,7 @@ __device__ float dec_quant_row(const DecSlot &pr, int m, int K, int RS, uint8_t 
                 const u32 b = dec_x_bits<BF16>(c[i], j);
                 amax = max(amax, b & 0x7fffffffu);
                 if (g4 != nullptr) {
-                    const double xd = sq_abs_double(b);
+                    const double xd = abs_as_double(b);
                     dsq = __fma_rn(xd, xd, dsq);
                 }
             }

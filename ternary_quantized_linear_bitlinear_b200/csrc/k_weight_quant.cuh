@@ -87,13 +87,6 @@ __device__ __forceinline__ u32 vec_elem_bits(const uint4 &v, int j) {
     }
 }
 
-// |w| of a float's bits as a double: exponent rebiased, mantissa moved;
-// exact for normal w, in [2^-127, 2^-126) for zero and subnormal w.
-__device__ __forceinline__ double wq_abs_double(u32 bits) {
-    const u32 a = bits & 0x7fffffffu;
-    return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
-}
-
 // gamma = float(S / n) + 1e-5f (S already rounded to double) and the
 // smallest float t with float(t / gamma) > 0.5.
 __device__ __forceinline__ void wq_gamma_threshold_of(double S, long long n, float *g_out, u32 *t_out) {
@@ -192,8 +185,8 @@ __global__ void __launch_bounds__(WQ_THREADS, 2) k_absmean_partial(const __grid_
     auto add_vec = [&](const uint4 &v) {
 #pragma unroll
         for (int j = 0; j < EPV; j += 2) {
-            d0 = __dadd_rn(d0, wq_abs_double(vec_elem_bits<BF16>(v, j)));
-            d1 = __dadd_rn(d1, wq_abs_double(vec_elem_bits<BF16>(v, j + 1)));
+            d0 = __dadd_rn(d0, abs_as_double(vec_elem_bits<BF16>(v, j)));
+            d1 = __dadd_rn(d1, abs_as_double(vec_elem_bits<BF16>(v, j + 1)));
         }
     };
     uint4 a[4];
