@@ -427,3 +427,51 @@ def test_ffn_act_quant_constant_row():
     assert s.tolist() == [float(np.float32(127.0) / np.float32(1.5))] * 2
     xq2, s2 = oracle.ffn_act_quant(g, u, np.ones(256, np.float32), 1e-6)
     assert xq2[0].tolist() == [127] * 256 and xq2[1].tolist() == [-127] * 256
+
+
+# -- exact ties that the GPU parity cases build ---------------------------------
+
+def _midpoint_weights(n: int) -> np.ndarray:
+    # n/2 - 1 entries of 2, one of 1, one of -1, one of -2^-24 n, the rest 0:
+    # sum |W| = n (1 + 2^-24), so sum |W| / n lies exactly halfway between
+    # 1 and the next float 1 + 2^-23
+    w = np.zeros(n, dtype=np.float32)
+    w[: n // 2 - 1] = 2.0
+    w[n // 2 - 1] = 1.0
+    w[n // 2] = -1.0
+    w[n // 2 + 1] = -(2.0 ** -24) * n
+    return w
+
+
+@pytest.mark.parametrize("n", [64, 256, 64 * 4096])
+def test_gamma_at_an_exact_midpoint_ties_to_even(n):
+    """mean|W| exactly halfway between two floats rounds to the even one
+    (1.0), so gamma = 1 + 1e-5 in float: an oracle that summed |W| in float
+    or double with rounding (landing on either side) or rounded the mean
+    away from zero would give the odd neighbour's gamma."""
+    w = _midpoint_weights(n)
+    assert exact_abs_sum(w) == n * (1 + Fraction(1, 2 ** 24))
+    assert oracle.absmean_gamma(w) == np.float32(np.float32(1.0) + np.float32(1e-5))
+    assert oracle.absmean_gamma(w) != np.float32(np.float32(1.0 + 2.0 ** -23) + np.float32(1e-5))
+
+
+@pytest.mark.parametrize("K", [1024, 2048, 4096])
+def test_subln_at_an_exact_midpoint_ties_to_even(K):
+    """Row [8, 2^-9, 0, ...]: sum x^2 / K = (64 + 2^-18) / K, exactly halfway
+    between two floats for K a power of two; ms rounds to the even one
+    (64 / K), then r = sqrtf(ms + eps) and y follow (checked by Fractions)."""
+    x = np.zeros(K, dtype=np.float32)
+    x[0], x[1] = 8.0, 2.0 ** -9
+    g = np.ones(K, dtype=np.float32)
+    eps = np.float32(1e-6)
+    mid = (Fraction(64) + Fraction(1, 2 ** 18)) / K
+    assert f32_rne(mid) == 64.0 / K  # the tie goes to the even float
+    arg = f32_rne(Fraction(64, K) + Fraction(float(eps)))
+    r0 = np.float32(math.sqrt(arg))
+    cands = [np.nextafter(r0, np.float32(0)), r0, np.nextafter(r0, np.float32(np.inf))]
+    r = min(cands, key=lambda c: abs(Fraction(float(c)) ** 2 - Fraction(arg)))
+    y = oracle.rmsnorm(x, g, 1e-6)
+    assert float(y[0]) == f32_rne(Fraction(8) / Fraction(float(r)))
+    assert float(y[1]) == f32_rne(Fraction(1, 2 ** 9) / Fraction(float(r)))
+    xq, s = oracle.quant_act(x.reshape(1, K), g, 1e-6)
+    assert xq[0, 0] == 127 and s[0] == np.float32(np.float32(127.0) / y[0])
